@@ -1,0 +1,9 @@
+"""CPU oracle for the Sparse-BitLinear forward (test infrastructure only).
+
+Imported by the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU
+baseline leg; never by the library itself.
+"""
+from .sbl_oracle import *  # noqa: F401,F403
+from .sbl_oracle import (SUPPORTED_NM, acc_entries, dequant, int_contract, linear, nm_mask,  # noqa: F401
+                         pack_codes, pack_mask_bits, prepare_weights, quant_act, row_scale,
+                         ternarise, unpack_codes)

@@ -1,0 +1,201 @@
+"""CPU oracle for the Sparse-BitLinear forward — TEST INFRASTRUCTURE ONLY.
+
+Only the test-suite, the package smoke check and the benchmark's CPU-baseline
+leg may import this module.  The library never does: it shares no code,
+table or helper with the CUDA path and must not be used as a fallback.
+
+What it computes (the Sparse-BitLinear operator of "Sparse-BitNet Guide: 1.58-Bit
+LLMs Meet 2:4 Sparsity", section "Mathematical Formulation of Sparse-BitLinear",
+with the per-row scale of the halo-sparse-bitnet-3:4-500m card's "Recipe" and
+the 2-bit code table of its "What ships with this repo / Packed vs raw"):
+
+    mask      keep the N largest |W| of every M contiguous input-dim weights
+    scale_i   absmean of the kept |W| of row i
+    W_t       clip(round(W / scale), -1, 1) on kept positions, 0 elsewhere
+    packed    2 bits per weight, 00 = 0, 01 = +1, 10 = -1, 4 codes per byte
+    x_q       clip(round(x * 127 / max|x|), -128, 127) per token
+    acc       x_q . W_t^T in integers
+    y         acc * scale_i / s_t,  s_t = 127 / max|x_t|
+
+Readings taken where the pages are silent or disagree (each one is listed
+with its reason in the design notes):
+
+* ties in the Top-N go to the lower index; -0 and +0 tie;
+* scale: per row over the kept weights; sum of |w| formed exactly and
+  rounded once to double (``math.fsum``), divided by the kept count in double,
+  rounded to float, then clamped below at 1e-5 (the epsilon of the guide's
+  module listing);
+* round() is round-half-to-even (``torch.round`` semantics in the guide's
+  listing); W / scale is evaluated in double, which decides |W|/scale against
+  the 0.5 threshold exactly for float inputs;
+* the activation scale and x * s are float32 operations (the guide's module
+  computes in the activation's float type); x is bf16 widened exactly;
+* 2-bit codes are stored LSB-first: weight k sits in byte k // 4 at bits
+  2 (k % 4) .. 2 (k % 4) + 1; mask bits: bit k % 8 of byte k // 8;
+* dequantisation in double: y = acc * scale / s_t.
+
+Every function here is pinned by tests that do not call it to build their
+expected values (worked examples from the pages, closed forms, brute force).
+Parity pinned for all functions; none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+EPS_SCALE = np.float32(1e-5)   # clamp of the weight absmean (guide's module listing)
+EPS_ACT = np.float32(1e-5)     # clamp of the activation absmax (guide's module listing)
+SUPPORTED_NM = ((2, 4), (3, 4), (6, 8))
+
+
+def _check_nm(K: int, n: int, m: int) -> None:
+    if (n, m) not in SUPPORTED_NM:
+        raise ValueError(f"unsupported N:M pattern {n}:{m}")
+    if K % m or K % 4:
+        raise ValueError("K must be a multiple of M and of 4")
+
+
+def nm_mask(W: np.ndarray, n: int, m: int) -> np.ndarray:
+    """Boolean keep-mask [O, K]: Top-N |W| in each group of M input-dim weights.
+
+    Sparse-BitNet Guide, "Mathematical Formulation of Sparse-BitLinear", the
+    mask equation (Top-N indices of |W[i, Mk : Mk+M]|); Sparse-BitNet README,
+    "How It Works / N:M Structured Sparsity".  Equal magnitudes: the lower
+    index is kept first (a stable sort on -|w|).
+    """
+    W = np.asarray(W, dtype=np.float32)
+    O, K = W.shape
+    _check_nm(K, n, m)
+    if not np.all(np.isfinite(W)):
+        raise ValueError("non-finite weight")
+    a = np.abs(W.astype(np.float64)).reshape(O, K // m, m)
+    order = np.argsort(-a, axis=-1, kind="stable")
+    keep = np.zeros(a.shape, dtype=bool)
+    np.put_along_axis(keep, order[..., :n], True, axis=-1)
+    return keep.reshape(O, K)
+
+
+def row_scale(W: np.ndarray, mask: np.ndarray) -> np.ndarray:
+    """fp32 [O]: per-row absmean of the kept weights, clamped at 1e-5.
+
+    halo-sparse-bitnet-3:4-500m card, "Recipe" (per-row absmean scale); the
+    guide's gamma equation gives the absmean form.  The sum is exact up to one
+    final rounding to double (``math.fsum``).
+    """
+    W = np.asarray(W, dtype=np.float32)
+    O = W.shape[0]
+    out = np.empty(O, dtype=np.float32)
+    for i in range(O):
+        kept = np.abs(W[i][mask[i]]).astype(np.float64)
+        mean = math.fsum(kept.tolist()) / float(kept.size)
+        out[i] = max(np.float32(mean), EPS_SCALE)
+    return out
+
+
+def ternarise(W: np.ndarray, scale: np.ndarray, mask: np.ndarray) -> np.ndarray:
+    """int8 [O, K] in {-1, 0, +1}: mask * clip(round(W / scale), -1, 1).
+
+    Sparse-BitNet Guide, "Mathematical Formulation of Sparse-BitLinear", the
+    joint sparse-ternary equation; the README's "Sparse-BitNet" section
+    (mask first, then quantise what remains).
+    """
+    q = np.rint(np.asarray(W, np.float64) / np.asarray(scale, np.float64)[:, None])
+    q = np.clip(q, -1.0, 1.0) * mask
+    return q.astype(np.int8)
+
+
+def pack_codes(Wt: np.ndarray) -> np.ndarray:
+    """uint8 [O, K/4]: 2-bit codes 00 = 0, 01 = +1, 10 = -1, LSB-first.
+
+    halo-sparse-bitnet-3:4-500m card, "What ships with this repo" /
+    "Packed vs raw" (NAME.packed, 4 codes per byte).
+    """
+    Wt = np.asarray(Wt)
+    O, K = Wt.shape
+    code = np.zeros(Wt.shape, dtype=np.uint8)
+    code[Wt == 1] = 1
+    code[Wt == -1] = 2
+    c = code.reshape(O, K // 4, 4)
+    return (c[..., 0] | (c[..., 1] << 2) | (c[..., 2] << 4) | (c[..., 3] << 6)).astype(np.uint8)
+
+
+def pack_mask_bits(mask: np.ndarray) -> np.ndarray:
+    """uint8 [O, K/8]: bit k % 8 of byte k // 8 is set when weight k is kept."""
+    O, K = mask.shape
+    b = mask.reshape(O, K // 8, 8).astype(np.uint8)
+    out = np.zeros((O, K // 8), dtype=np.uint8)
+    for j in range(8):
+        out |= (b[..., j] << j).astype(np.uint8)
+    return out
+
+
+def prepare_weights(W: np.ndarray, n: int, m: int):
+    """Latent fp32 weights -> (packed uint8 [O,K/4], scale fp32 [O], mask bits uint8 [O,K/8], W_t int8 [O,K])."""
+    mask = nm_mask(W, n, m)
+    scale = row_scale(W, mask)
+    Wt = ternarise(W, scale, mask)
+    return pack_codes(Wt), scale, pack_mask_bits(mask), Wt
+
+
+def quant_act(x: np.ndarray):
+    """Per-token absmax int8: (x_q int8 [T,K], s_tok fp32 [T]), s_t = 127 / max(max|x_t|, 1e-5).
+
+    Sparse-BitNet Guide, "Mathematical Formulation of Sparse-BitLinear", the
+    activation equation (per-token beta = max |x_j|, clip to [-128, 127]);
+    BitNet-TinyDialogues card (W1.58A8, 8-bit per-token activations).
+    ``x`` holds bf16 values widened to fp32.
+    """
+    x = np.asarray(x, dtype=np.float32)
+    if not np.all(np.isfinite(x)):
+        raise ValueError("non-finite activation")
+    amax = np.max(np.abs(x), axis=1) if x.shape[1] else np.zeros(x.shape[0], np.float32)
+    s = (np.float32(127.0) / np.maximum(amax, EPS_ACT)).astype(np.float32)
+    q = np.rint((x * s[:, None]).astype(np.float32))
+    return np.clip(q, -128, 127).astype(np.int8), s
+
+
+def int_contract(xq: np.ndarray, Wt: np.ndarray) -> np.ndarray:
+    """int32 [T, O] = x_q . W_t^T (the guide's integer product before rescaling).
+
+    Evaluated as a float64 matrix product: every product and partial sum is an
+    integer of magnitude <= 128 * K < 2**53, so each is exact whatever the
+    summation order; the result is checked to be integral and to fit int32.
+    """
+    acc = np.asarray(xq, np.float64) @ np.asarray(Wt, np.float64).T
+    r = np.rint(acc)
+    if not np.array_equal(r, acc):
+        raise ArithmeticError("non-integral contraction")
+    if r.size and np.max(np.abs(r)) >= 2**31:
+        raise OverflowError("accumulator exceeds int32")
+    return r.astype(np.int32)
+
+
+def dequant(acc: np.ndarray, scale: np.ndarray, s_tok: np.ndarray) -> np.ndarray:
+    """float64 [T, O] = acc * scale_o / s_t (the guide's beta * gamma / 127 rescale)."""
+    return (np.asarray(acc, np.float64) * np.asarray(scale, np.float64)[None, :]
+            / np.asarray(s_tok, np.float64)[:, None])
+
+
+def linear(x: np.ndarray, Wt: np.ndarray, scale: np.ndarray):
+    """Full forward on prepared weights: (y float64 [T,O], acc int32 [T,O], x_q, s_tok)."""
+    xq, s = quant_act(x)
+    acc = int_contract(xq, Wt)
+    return dequant(acc, scale, s), acc, xq, s
+
+
+def unpack_codes(packed: np.ndarray, K: int) -> np.ndarray:
+    """Inverse of :func:`pack_codes` (code 11 is invalid and raises)."""
+    p = np.asarray(packed, dtype=np.uint8)
+    O = p.shape[0]
+    c = np.stack([(p >> (2 * j)) & 3 for j in range(4)], axis=-1).reshape(O, K)
+    if np.any(c == 3):
+        raise ValueError("invalid 2-bit code 11")
+    return np.where(c == 1, 1, np.where(c == 2, -1, 0)).astype(np.int8)
+
+
+def acc_entries(xq: np.ndarray, Wt: np.ndarray, idx_t, idx_o) -> np.ndarray:
+    """int64 acc[t, o] for the listed (t, o) pairs, one dot product each (sampled checks)."""
+    xq = np.asarray(xq, np.int64)
+    Wt = np.asarray(Wt, np.int64)
+    return np.array([int(np.dot(xq[t], Wt[o])) for t, o in zip(idx_t, idx_o)], dtype=np.int64)

@@ -1,0 +1,379 @@
+"""Pins of the CPU oracle to facts that do not come from the oracle itself.
+
+* worked examples: the 4-element block the Sparse-BitNet Guide prints in
+  "The Hardware Mechanics of 2:4 Sparsity", plus hand-derived tie, rounding and
+  degenerate cases (tests/golden/worked_examples.json, each with its source);
+* brute force on tiny shapes: the Top-N set found by enumerating every subset,
+  exact rational means (fractions.Fraction), the |w| > scale/2 threshold form
+  of clip(round(w/scale)), bit-string packing, explicit integer loops;
+* invariants that hold at any size (codes in {-1,0,1}, at most N nonzeros per
+  group, sign agreement, packed size O*K/4, argmax token element -> +-127);
+* the guide's own rescale form y = acc * beta * gamma / 127.
+
+Each plausible mistake (a reversed input index, scale over all weights, half away
+from zero, ties to the higher index, MSB-first packing, a dropped clamp, a sign
+flip) is planted in a copy of the oracle at the end of this file, and some pin
+below must reject it.
+"""
+import itertools
+import json
+import os
+import types
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+from sparse_linear_layers_b200 import synthetic
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "worked_examples.json")
+PATTERNS = [(2, 4), (3, 4), (6, 8)]
+
+
+def _cases():
+    with open(GOLDEN) as f:
+        return json.load(f)["cases"]
+
+
+# --------------------------------------------------------------------------
+# pins written as functions of an oracle-like namespace, so the planted
+# mistakes at the bottom can be run through the very same checks
+# --------------------------------------------------------------------------
+
+def pin_golden(o):
+    for c in _cases():
+        if "w" in c and "w_t" in c:
+            W = np.array([c["w"]], dtype=np.float32)
+            n, m = c["n"], c["m"]
+            mask = o.nm_mask(W, n, m)
+            assert sorted(np.nonzero(mask[0])[0].tolist()) == c["kept_indices"], c["name"]
+            scale = o.row_scale(W, mask)
+            assert abs(float(scale[0]) - c["scale"]) <= 1e-6 * c["scale"], c["name"]
+            Wt = o.ternarise(W, scale, mask)
+            assert Wt[0].tolist() == c["w_t"], c["name"]
+            assert o.pack_codes(Wt)[0].tolist() == c["packed"], c["name"]
+            # mask bits need K % 8 == 0: pad with a second group of zeros
+            W8 = np.concatenate([W, np.zeros((1, 4), np.float32)], axis=1)
+            mb = o.pack_mask_bits(o.nm_mask(W8, n, m))
+            assert int(mb[0, 0]) & 0xF == c["mask_byte_low_nibble"], c["name"]
+        if "x" in c and "x_q" in c:
+            x = np.array([c["x"]], dtype=np.float32)
+            xq, s = o.quant_act(x)
+            assert xq[0].tolist() == c["x_q"], c["name"]
+            if "s_tok" in c:
+                assert float(s[0]) == c["s_tok"], c["name"]
+        if "acc" in c:
+            W = np.array([c["w"]], dtype=np.float32)
+            mask = o.nm_mask(W, c["n"], c["m"])
+            scale = o.row_scale(W, mask)
+            Wt = o.ternarise(W, scale, mask)
+            y, acc, _, _ = o.linear(np.array([c["x"]], np.float32), Wt, scale)
+            assert int(acc[0, 0]) == c["acc"], c["name"]
+            if c["y"] == 0.0:
+                assert y[0, 0] == 0.0
+            else:
+                assert abs(y[0, 0] - c["y"]) <= 1e-6 * abs(c["y"]), c["name"]
+
+
+def _brute_mask_group(a, n):
+    """The unique N-subset S with |a_i| > |a_j| or (equal and i < j) for all i in S, j not in S."""
+    m = len(a)
+    found = []
+    for S in itertools.combinations(range(m), n):
+        ok = all((abs(a[i]) > abs(a[j])) or (abs(a[i]) == abs(a[j]) and i < j)
+                 for i in S for j in range(m) if j not in S)
+        if ok:
+            found.append(S)
+    assert len(found) == 1
+    return found[0]
+
+
+def _exact_scale(row, kept):
+    tot = sum((Fraction(float(abs(row[k]))) for k in kept), Fraction(0))
+    mean = float(tot) / float(len(kept))       # float(Fraction) rounds correctly to double
+    return max(np.float32(mean), np.float32(1e-5))
+
+
+def _brute_prepare(W, n, m):
+    O, K = W.shape
+    mask = np.zeros((O, K), bool)
+    for i in range(O):
+        for g in range(K // m):
+            for j in _brute_mask_group([float(v) for v in W[i, g * m:(g + 1) * m]], n):
+                mask[i, g * m + j] = True
+    scale = np.array([_exact_scale(W[i], np.nonzero(mask[i])[0]) for i in range(O)], np.float32)
+    Wt = np.zeros((O, K), np.int8)
+    for i in range(O):
+        half = np.float32(0.5) * scale[i]          # exact in float32
+        for k in range(K):
+            if mask[i, k] and abs(W[i, k]) > half:  # round(w/s) != 0  <=>  |w|/s > 1/2
+                Wt[i, k] = 1 if W[i, k] > 0 else -1
+    return mask, scale, Wt
+
+
+def _bitstring_pack(Wt):
+    O, K = Wt.shape
+    out = np.zeros((O, K // 4), np.uint8)
+    for i in range(O):
+        for b in range(K // 4):
+            bits = ""
+            for j in reversed(range(4)):           # most significant code first in the string
+                v = int(Wt[i, 4 * b + j])
+                bits += {0: "00", 1: "01", -1: "10"}[v]
+            out[i, b] = int(bits, 2)
+    return out
+
+
+def _loop_contract(xq, Wt):
+    T, K = xq.shape
+    O = Wt.shape[0]
+    acc = np.zeros((T, O), np.int64)
+    for t in range(T):
+        for o in range(O):
+            s = 0
+            for k in range(K):
+                s += int(xq[t, k]) * int(Wt[o, k])
+            acc[t, o] = s
+    return acc
+
+
+def pin_brute_force(o, shapes=((8, 16), (5, 24), (3, 64)), T=3, seeds=(0, 1, 2)):
+    for seed in seeds:
+        for (O, K) in shapes:
+            for (n, m) in PATTERNS:
+                if K % m:
+                    continue
+                W = synthetic.latent_weights(O, K, seed=seed, tag=f"bf{O}x{K}")
+                # plant exact ties and zeros so the tie rule is exercised
+                W[0, :m] = np.float32(0.25)
+                W[-1, m:2 * m] = 0.0
+                W[1 % O, :4] = [np.float32(0.5), np.float32(-0.5), np.float32(0.5), np.float32(0.125)]
+                mask_b, scale_b, Wt_b = _brute_prepare(W, n, m)
+                packed, scale, mbits, Wt = o.prepare_weights(W, n, m)
+                assert np.array_equal(o.nm_mask(W, n, m), mask_b)
+                assert np.array_equal(scale.view(np.uint32), scale_b.view(np.uint32))
+                assert np.array_equal(Wt, Wt_b)
+                assert np.array_equal(packed, _bitstring_pack(Wt_b))
+                _, xv = synthetic.activations(T, K, seed=seed, tag=f"bfx{K}")
+                xq, s = o.quant_act(xv)
+                acc_b = _loop_contract(xq, Wt_b)
+                y, acc, _, _ = o.linear(xv, Wt, scale)
+                assert np.array_equal(acc.astype(np.int64), acc_b)
+                # the guide's rescale: y = acc * beta * gamma / 127, beta = max|x_t|
+                beta = np.maximum(np.max(np.abs(xv.astype(np.float64)), axis=1), 1e-5)
+                y_page = acc_b * beta[:, None] * scale.astype(np.float64)[None, :] / 127.0
+                assert np.allclose(y, y_page, rtol=1e-6, atol=0.0)
+
+
+def pin_invariants(o, O=64, K=512, T=16):
+    for (n, m) in PATTERNS:
+        for seed in (0, 1):
+            W = synthetic.latent_weights(O, K, seed=seed, tag="inv")
+            packed, scale, mbits, Wt = o.prepare_weights(W, n, m)
+            assert packed.shape == (O, K // 4) and packed.dtype == np.uint8   # 2 bits per weight
+            assert set(np.unique(Wt).tolist()) <= {-1, 0, 1}
+            codes = np.stack([(packed >> (2 * j)) & 3 for j in range(4)], -1)
+            assert not np.any(codes == 3)
+            mask = np.unpackbits(mbits, axis=1, bitorder="little").astype(bool)
+            assert np.all(mask.reshape(O, K // m, m).sum(-1) == n)
+            assert np.all((Wt != 0).reshape(O, K // m, m).sum(-1) <= n)
+            assert np.all(mask[Wt != 0])
+            nz = Wt != 0
+            assert np.all(np.sign(W[nz]) == Wt[nz])
+            # kept weights dominate dropped ones inside every group
+            a = np.abs(W).reshape(O, K // m, m)
+            mk = mask.reshape(O, K // m, m)
+            kept_min = np.where(mk, a, np.inf).min(-1)
+            drop_max = np.where(~mk, a, -np.inf).max(-1)
+            assert np.all(kept_min >= drop_max)
+            # scale is the mean of the kept magnitudes (loose check against float64 mean)
+            mean = np.where(mask, np.abs(W.astype(np.float64)), 0).sum(1) / (K * n // m)
+            assert np.allclose(scale, mean, rtol=1e-6)
+            # round(w/s) != 0 exactly when |w| > s/2
+            assert np.array_equal(nz, mask & (np.abs(W) > np.float32(0.5) * scale[:, None]))
+    _, x = synthetic.activations(T, K, seed=3, tag="invx", outlier_p=0.01)
+    xq, s = o.quant_act(x)
+    assert xq.min() >= -127 and xq.max() <= 127
+    arg = np.argmax(np.abs(x), axis=1)
+    assert np.all(np.abs(xq[np.arange(T), arg]) == 127)
+    exact = x.astype(np.float64) * s.astype(np.float64)[:, None]
+    assert np.all(np.abs(xq - exact) <= 0.5 + 1e-6)
+    # monotone in x within each token
+    for t in range(T):
+        order = np.argsort(x[t], kind="stable")
+        assert np.all(np.diff(xq[t][order].astype(np.int32)) >= 0)
+
+
+def pin_closed_forms(o):
+    # every kept magnitude equal to c: scale == c exactly, W_t == sign(W) on kept positions
+    c = np.float32(0.0375)
+    K = 64
+    for (n, m) in PATTERNS:
+        W = np.full((2, K), c, np.float32)
+        W[1, ::2] = -c
+        mask = o.nm_mask(W, n, m)
+        scale = o.row_scale(W, mask)
+        assert np.all(scale == c)
+        Wt = o.ternarise(W, scale, mask)
+        assert np.array_equal(Wt, (np.sign(W) * mask).astype(np.int8))
+        # first N of each group kept (all tie)
+        assert np.array_equal(mask.reshape(2, K // m, m)[..., :n], np.ones((2, K // m, n), bool))
+    # zero token -> zero codes, zero output
+    x = np.zeros((1, K), np.float32)
+    xq, s = o.quant_act(x)
+    assert not xq.any() and s[0] == np.float32(127.0) / np.float32(1e-5)
+
+
+# --------------------------------------------------------------------------
+
+def test_golden_worked_examples():
+    pin_golden(oracle)
+
+
+def test_brute_force_tiny_shapes():
+    pin_brute_force(oracle)
+
+
+def test_invariants():
+    pin_invariants(oracle)
+
+
+def test_closed_forms():
+    pin_closed_forms(oracle)
+
+
+def test_unpack_roundtrip_and_bad_code():
+    W = synthetic.latent_weights(16, 128, seed=5)
+    packed, _, _, Wt = oracle.prepare_weights(W, 3, 4)
+    assert np.array_equal(oracle.unpack_codes(packed, 128), Wt)
+    bad = packed.copy()
+    bad[0, 0] = 0xFF
+    with pytest.raises(ValueError):
+        oracle.unpack_codes(bad, 128)
+
+
+def test_rejects_bad_input():
+    with pytest.raises(ValueError):
+        oracle.nm_mask(np.ones((2, 8), np.float32), 1, 4)
+    W = np.ones((2, 8), np.float32)
+    W[0, 3] = np.nan
+    with pytest.raises(ValueError):
+        oracle.nm_mask(W, 2, 4)
+    x = np.ones((1, 8), np.float32)
+    x[0, 0] = np.inf
+    with pytest.raises(ValueError):
+        oracle.quant_act(x)
+
+
+def test_acc_entries_matches_contract():
+    W = synthetic.latent_weights(32, 256, seed=1)
+    _, scale, _, Wt = oracle.prepare_weights(W, 2, 4)
+    _, x = synthetic.activations(4, 256, seed=1)
+    xq, _ = oracle.quant_act(x)
+    full = oracle.int_contract(xq, Wt)
+    t = np.array([0, 1, 3, 2])
+    o_ = np.array([0, 31, 7, 19])
+    assert np.array_equal(oracle.acc_entries(xq, Wt, t, o_), full[t, o_])
+
+
+# --------------------------------------------------------------------------
+# planted mistakes: each mutant must fail at least one pin
+# --------------------------------------------------------------------------
+
+def _mutant(**over):
+    ns = types.SimpleNamespace(**{k: getattr(oracle, k) for k in (
+        "nm_mask", "row_scale", "ternarise", "pack_codes", "pack_mask_bits", "quant_act",
+        "int_contract", "dequant")})
+    ns.__dict__.update(over)
+
+    def prepare_weights(W, n, m):
+        mask = ns.nm_mask(W, n, m)
+        scale = ns.row_scale(W, mask)
+        Wt = ns.ternarise(W, scale, mask)
+        return ns.pack_codes(Wt), scale, ns.pack_mask_bits(mask), Wt
+
+    def linear(x, Wt, scale):
+        xq, s = ns.quant_act(x)
+        acc = ns.int_contract(xq, Wt)
+        return ns.dequant(acc, scale, s), acc, xq, s
+
+    ns.prepare_weights = prepare_weights
+    ns.linear = linear
+    return ns
+
+
+def _ties_high(W, n, m):
+    O, K = W.shape
+    a = np.abs(W.astype(np.float64)).reshape(O, K // m, m)[..., ::-1]
+    order = np.argsort(-a, axis=-1, kind="stable")
+    keep = np.zeros(a.shape, bool)
+    np.put_along_axis(keep, order[..., :n], True, axis=-1)
+    return keep[..., ::-1].reshape(O, K)
+
+
+def _scale_all(W, mask):
+    return np.maximum(np.mean(np.abs(W.astype(np.float64)), axis=1).astype(np.float32), np.float32(1e-5))
+
+
+def _half_away(W, scale, mask):
+    r = np.asarray(W, np.float64) / np.asarray(scale, np.float64)[:, None]
+    q = np.sign(r) * np.floor(np.abs(r) + 0.5)
+    return (np.clip(q, -1, 1) * mask).astype(np.int8)
+
+
+def _msb_first(Wt):
+    O, K = Wt.shape
+    code = np.where(Wt == 1, 1, np.where(Wt == -1, 2, 0)).astype(np.uint8).reshape(O, K // 4, 4)
+    return (code[..., 3] | (code[..., 2] << 2) | (code[..., 1] << 4) | (code[..., 0] << 6)).astype(np.uint8)
+
+
+def _swapped_codes(Wt):
+    return oracle.pack_codes(-np.asarray(Wt))
+
+
+def _no_mask(W, scale, mask):
+    return oracle.ternarise(W, scale, np.ones_like(mask))
+
+
+def _k_reversed(xq, Wt):
+    return oracle.int_contract(xq, np.asarray(Wt)[:, ::-1])
+
+
+def _quant_no_round(x):
+    xq, s = oracle.quant_act(x)
+    x = np.asarray(x, np.float32)
+    q = np.trunc(x * s[:, None])
+    return np.clip(q, -128, 127).astype(np.int8), s
+
+
+def _dequant_inverted(acc, scale, s_tok):
+    return np.asarray(acc, np.float64) * np.asarray(scale, np.float64)[None, :] * np.asarray(s_tok, np.float64)[:, None] / 127.0 ** 2
+
+
+MUTANTS = {
+    "ties_to_higher_index": dict(nm_mask=_ties_high),
+    "scale_over_all_weights": dict(row_scale=_scale_all),
+    "round_half_away": dict(ternarise=_half_away),
+    "msb_first_packing": dict(pack_codes=_msb_first),
+    "swapped_code_table": dict(pack_codes=_swapped_codes),
+    "mask_not_applied": dict(ternarise=_no_mask),
+    "input_dim_reversed": dict(int_contract=_k_reversed),
+    "activation_truncated": dict(quant_act=_quant_no_round),
+    "rescale_inverted": dict(dequant=_dequant_inverted),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(name):
+    o = _mutant(**MUTANTS[name])
+    caught = []
+    for pin in (pin_golden, pin_closed_forms, pin_brute_force, pin_invariants):
+        try:
+            if pin is pin_brute_force:
+                pin(o, shapes=((8, 16), (4, 32)), T=2, seeds=(0,))
+            else:
+                pin(o)
+        except (AssertionError, ValueError, IndexError):
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught the planted mistake {name}"
