@@ -1,0 +1,433 @@
+"""Benchmark of the Sparse-BitLinear forward on B200.
+
+Workload (one "step"): the seven Qwen2.5-0.5B-shaped projections of one layer
+(q 896->896, k/v 896->128, o 896->896, gate/up 896->4864, down 4864->896) at
+3:4 sparsity, each taken from latent fp32 weights through the whole path:
+weight preparation (mask, scale, ternarise, pack), activation quantisation,
+the prefill contraction at T = 2048 tokens and the decode contraction at
+T = 1, with fp32 outputs.  Inputs are seeded synthetic draws (W ~ N(0, 0.02^2),
+x ~ N(0, 1) in bf16), resident in HBM; L2 is flushed (a 256 MiB write)
+between timed steps.  The metric is tokens per second: 2049 tokens per step
+per GPU (the 2048-token prefill batch plus one decode token).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs its own copy of the step on its own GPU (the
+forward has no cross-GPU exchange): weak scaling, timed as the max over ranks.
+``--impl reference`` times the CPU oracle on a bounded sample of the same step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_linear_layers_b200 import synthetic  # noqa: E402
+
+METRIC = "Sparse-BitLinear tokens/s; decode HBM GB/s and prefill int8 TOPS vs B200 peak"
+N, M = 3, 4
+T_PREFILL, T_DECODE = 2048, 1
+TOKENS_PER_STEP = T_PREFILL + T_DECODE
+WORKLOAD = "qwen2.5-0.5b layer projections (q,k,v,o,gate,up,down), 3:4, prep + T=2048 prefill + T=1 decode"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def _config(extra=None):
+    c = {"workload": WORKLOAD, "layers": [f"{nm} {k}->{o}" for nm, k, o in synthetic.QWEN05_LAYER],
+         "sparsity": f"{N}:{M}", "tokens_prefill": T_PREFILL, "tokens_decode": T_DECODE,
+         "output_dtype": "fp32", "l2": "flushed between timed steps (256 MiB write)", "seed": 0}
+    if extra:
+        c.update(extra)
+    return c
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling during the timed region (SM clock, throttle reasons)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- our arm
+
+class Layer:
+    def __init__(self, name, K, O, dev, seed=0):
+        import sparse_linear_layers_b200 as sbl
+        self.name, self.K, self.O = name, K, O
+        W = synthetic.latent_weights(O, K, seed=seed, tag=f"bench-{name}")
+        xb, _ = synthetic.activations(T_PREFILL, K, seed=seed, tag=f"bench-x-{name}")
+        x1, _ = synthetic.activations(T_DECODE, K, seed=seed, tag=f"bench-x1-{name}")
+        self.W_host = torch.from_numpy(W).pin_memory()
+        self.x_host = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).pin_memory()
+        self.x1_host = torch.from_numpy(x1.view(np.int16)).view(torch.bfloat16).pin_memory()
+        self.W = self.W_host.to(dev)
+        self.x = self.x_host.to(dev)
+        self.x1 = self.x1_host.to(dev)
+        self.w = sbl.PreparedWeights(torch.empty((O, K // 4), dtype=torch.uint8, device=dev),
+                                     torch.empty((O,), dtype=torch.float32, device=dev), N, M, K)
+        self.y = torch.empty((T_PREFILL, O), dtype=torch.float32, device=dev)
+        self.y1 = torch.empty((T_DECODE, O), dtype=torch.float32, device=dev)
+        self.ws = sbl.workspace_for(T_PREFILL, K, O, N, M, dev)
+        self.y_host = torch.empty((T_PREFILL, O), dtype=torch.float32).pin_memory()
+        self.y1_host = torch.empty((T_DECODE, O), dtype=torch.float32).pin_memory()
+
+    # algorithmic work
+    def prefill_ops(self):
+        return 2.0 * T_PREFILL * self.O * self.K
+
+    def prefill_bytes(self):
+        return self.O * self.K / 4 + 4 * self.O + 2 * T_PREFILL * self.K + 4 * T_PREFILL * self.O
+
+    def decode_bytes(self, T=T_DECODE):
+        return self.O * self.K / 4 + 4 * self.O + 2 * T * self.K + 4 * T * self.O
+
+
+def _step(sbl, layers, ev=None):
+    """One pass of the whole path over the seven projections; optional events around the prefill calls."""
+    for i, L in enumerate(layers):
+        sbl.sbl_prepare_weights(L.W, N, M, out=L.w)
+        if ev is not None:
+            ev[i][0].record()
+        sbl.sbl_linear(L.x, L.w, y=L.y, workspace=L.ws)
+        if ev is not None:
+            ev[i][1].record()
+        sbl.sbl_linear(L.x1, L.w, y=L.y1, workspace=L.ws)
+
+
+def _step_e2e(sbl, layers):
+    """Same step from pinned host buffers: H2D of W and x, D2H of y, inside the timed region."""
+    h2d = d2h = 0
+    for L in layers:
+        L.W.copy_(L.W_host, non_blocking=True)
+        L.x.copy_(L.x_host, non_blocking=True)
+        L.x1.copy_(L.x1_host, non_blocking=True)
+        h2d += L.W_host.numel() * 4 + L.x_host.numel() * 2 + L.x1_host.numel() * 2
+        sbl.sbl_prepare_weights(L.W, N, M, out=L.w)
+        sbl.sbl_linear(L.x, L.w, y=L.y, workspace=L.ws)
+        sbl.sbl_linear(L.x1, L.w, y=L.y1, workspace=L.ws)
+        L.y_host.copy_(L.y, non_blocking=True)
+        L.y1_host.copy_(L.y1, non_blocking=True)
+        d2h += L.y.numel() * 4 + L.y1.numel() * 4
+    return h2d, d2h
+
+
+def _decode_roofline(sbl, dev, hbm_peak, K=2048, O=7168, reps=64):
+    """T = 1 decode of a 2048 -> 7168 layer over a pool of distinct packed weights
+    larger than 3x L2, replayed from a CUDA graph: per-call GB/s on algorithmic bytes."""
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    per = O * K // 4
+    pool = max(8, int(3 * l2 // per) + 1)
+    W = torch.from_numpy(synthetic.latent_weights(O, K, seed=11, tag="decode-pool")).to(dev)
+    base = sbl.sbl_prepare_weights(W, 2, 4)
+    del W
+    packs = [base.packed.clone() for _ in range(pool)]
+    x1 = torch.from_numpy(synthetic.activations(1, K, seed=11, tag="decode-x")[0].view(np.int16)).view(
+        torch.bfloat16).to(dev)
+    y1 = torch.empty((1, O), dtype=torch.float32, device=dev)
+    ws = sbl.workspace_for(1, K, O, 2, 4, dev)
+    ws_list = [sbl.PreparedWeights(p, base.row_scale, 2, 4, K) for p in packs]
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        for w in ws_list[:4]:
+            sbl.sbl_linear(x1, w, y=y1, workspace=ws)
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for i in range(reps):
+            sbl.sbl_linear(x1, ws_list[i % pool], y=y1, workspace=ws)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    n_rep = 10
+    for _ in range(n_rep):
+        g.replay()
+    e1.record(s)
+    torch.cuda.synchronize()
+    per_call_s = e0.elapsed_time(e1) / 1e3 / (n_rep * reps)
+    # isolated single call (cold weights)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    iso = []
+    for i in range(20):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        sbl.sbl_linear(x1, ws_list[i % pool], y=y1, workspace=ws)
+        b.record()
+        torch.cuda.synchronize()
+        iso.append(a.elapsed_time(b) / 1e3)
+    byts = O * K / 4 + 4 * O + 2 * K + 4 * O
+    del g, packs, ws_list, flush
+    ach = byts / per_call_s / 1e9
+    return {"layer": f"{K}->{O} 2:4 T=1", "bytes_per_call": byts, "calls_in_graph": reps, "weight_pool": pool,
+            "us_per_call": per_call_s * 1e6, "achieved_gbs": ach, "peak_gbs": hbm_peak, "frac": ach / hbm_peak,
+            "isolated_call_us": statistics.median(iso) * 1e6}
+
+
+def run_ours(args, rank, world, dev):
+    import sparse_linear_layers_b200 as sbl
+    hbm_peak, bf16_peak, bf16_sus, peak_kind = _peaks()
+    int8_peak_tops = 2.0 * bf16_peak  # nominal dense int8 : bf16 ratio of B200 (4.5 : 2.25 POPS)
+    layers = [Layer(nm, K, O, dev) for nm, K, O in synthetic.QWEN05_LAYER]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    for _ in range(args.warmup):
+        _step(sbl, layers)
+    torch.cuda.synchronize()
+    status = sbl.sbl_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after warm-up")
+
+    K = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    pev = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in layers]
+           for _ in range(K)]
+    _barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for i in range(K):
+            flush.zero_()
+            starts[i].record()
+            _step(sbl, layers, pev[i])
+            ends[i].record()
+        torch.cuda.synchronize()
+    _barrier(world)
+    step_ms = [starts[i].elapsed_time(ends[i]) for i in range(K)]
+    total_s = sum(step_ms) / 1e3
+    total_s = _max_over_ranks(total_s, world, dev)
+    clocks = clk.summary()
+
+    # prefill contraction roofline (quantisation + tcgen05 GEMM, the dominant calls)
+    pre_s = sum(pev[i][j][0].elapsed_time(pev[i][j][1]) for i in range(K) for j in range(len(layers))) / 1e3
+    pre_s_per_step = pre_s / K
+    ops = sum(L.prefill_ops() for L in layers)
+    byts = sum(L.prefill_bytes() for L in layers)
+    t_tensor = ops / (int8_peak_tops * 1e12)
+    t_hbm = byts / (hbm_peak * 1e9)
+    if t_hbm >= t_tensor:
+        ach = byts / pre_s_per_step / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": ach / hbm_peak}
+    else:
+        ach = ops / pre_s_per_step / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": int8_peak_tops, "unit": "TOPS", "frac": ach / int8_peak_tops}
+    roof.update({"traffic": None, "kernel": "sbl_linear prefill calls (activation quant + tcgen05 int8 GEMM)",
+                 "algorithmic_bytes_per_step": byts, "algorithmic_ops_per_step": ops,
+                 "us_per_step": pre_s_per_step * 1e6, "peak_source": f"{peak_kind} (int8 = 2 x bf16 burst)"
+                 if roof["bound"] == "tensor" else f"{peak_kind} hbm_gbs",
+                 "tensor_tops": ops / pre_s_per_step / 1e12, "tensor_frac": ops / pre_s_per_step / 1e12 / int8_peak_tops})
+
+    # end to end through host buffers
+    for _ in range(2):
+        _step_e2e(sbl, layers)
+    torch.cuda.synchronize()
+    _barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(K):
+        h2d, d2h = _step_e2e(sbl, layers)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_s = _max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev)
+
+    decode = _decode_roofline(sbl, dev, hbm_peak) if rank == 0 else None
+    launches_per_step = len(layers) * (1 + 2 + 2)  # prep + (quant + GEMM) x 2 token counts
+    value = world * TOKENS_PER_STEP * K / total_s
+    out = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": total_s * 1e3 / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8", "data": "synthetic (seeded N(0,0.02^2) fp32 weights, N(0,1) bf16 activations)",
+        "config": _config({"parallelism": f"replicas x{world} (no collective on the data path)"}),
+        "roofline": roof,
+        "decode_roofline": decode,
+        "e2e": {"value": world * TOKENS_PER_STEP * K / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * K,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline_sample(budget_s=args.cpu_budget)
+    return out
+
+
+# --------------------------------------------------------------------------- oracle arm
+
+def cpu_baseline_sample(budget_s=20.0, sample_tokens=32):
+    """The CPU oracle on a bounded sample of the step: full weight preparation of
+    all seven projections plus ``sample_tokens`` of the 2048 prefill tokens and the
+    decode token; the step time is extrapolated to 2048 + 1 tokens."""
+    import oracle
+    threads = _cpu_threads()
+    t_prep = t_lin = 0.0
+    tok = 0
+    for nm, K, O in synthetic.QWEN05_LAYER:
+        W = synthetic.latent_weights(O, K, seed=0, tag=f"bench-{nm}")
+        _, xv = synthetic.activations(T_PREFILL, K, seed=0, tag=f"bench-x-{nm}")
+        _, x1 = synthetic.activations(T_DECODE, K, seed=0, tag=f"bench-x1-{nm}")
+        a = time.perf_counter()
+        _, scale, _, Wt = oracle.prepare_weights(W, N, M)
+        b = time.perf_counter()
+        oracle.linear(xv[:sample_tokens], Wt, scale)
+        oracle.linear(x1, Wt, scale)
+        c = time.perf_counter()
+        t_prep += b - a
+        t_lin += c - b
+    tok = sample_tokens + T_DECODE
+    step_s = t_prep + t_lin * TOKENS_PER_STEP / tok
+    return {"value": TOKENS_PER_STEP / step_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"weight prep of all 7 projections + {sample_tokens} of 2048 prefill tokens + the decode "
+                      f"token; step time extrapolated to 2049 tokens (measured prep {t_prep:.2f}s, "
+                      f"linear {t_lin:.2f}s)"}
+
+
+def _cpu_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = max((d.get("num_threads", 1) for d in info), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    vals = []
+    for _ in range(args.warmup):
+        cpu_baseline_sample(sample_tokens=8)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        r = cpu_baseline_sample(sample_tokens=8)
+        vals.append(r["value"])
+    wall = time.perf_counter() - t0
+    v = statistics.median(vals)
+    return {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * TOKENS_PER_STEP / v, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": _config({"parallelism": "CPU oracle, rank 0 only"}), "impl": "reference",
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": _cpu_threads(), "kind": "oracle",
+                             "sample": r["sample"]},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "wall_s": wall}
+
+
+# --------------------------------------------------------------------------- plumbing
+
+def _barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def _max_over_ranks(v, world, dev):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    try:
+        out = run_ours(args, rank, world, dev)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

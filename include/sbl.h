@@ -1,0 +1,175 @@
+/*
+ * sbl.h — C ABI of the Sparse-BitLinear forward on NVIDIA B200 (sm_100a).
+ *
+ * The operator (Sparse-BitNet Guide: 1.58-Bit LLMs Meet 2:4 Sparsity, section
+ * "Mathematical Formulation of Sparse-BitLinear"):
+ *
+ *     y = ( x_q . W_t^T ) * scale_o / s_t
+ *
+ * with W_t the N:M-masked ternary weights, x_q the per-token absmax int8
+ * activations, scale_o the per-row absmean of the kept weights
+ * (halo-sparse-bitnet-3:4-500m card, "Recipe") and s_t = 127 / max|x_t|.
+ *
+ * Conventions every entry point follows
+ *   - All pointers are DEVICE pointers unless stated, owned by the caller, and
+ *     16-byte aligned.  The library allocates no device memory: scratch space
+ *     is a caller-provided workspace (see sbl_linear_workspace_bytes).
+ *   - `stream` is a cudaStream_t passed as void*; NULL means the legacy
+ *     default stream.  Every call is asynchronous on `stream`; it returns once
+ *     the work is enqueued.
+ *   - Argument errors are detected on the host before anything is enqueued and
+ *     returned synchronously; a CUDA launch failure returns SBL_ERR_CUDA.
+ *   - Conditions only the device can see (non-finite inputs, a pipeline wait
+ *     that ran out) set bits in a per-device status word that
+ *     sbl_device_status() reads; kernels never trap.
+ *   - Shapes: row-major, int64 sizes; O, T >= 0 (zero sizes are no-ops);
+ *     K > 0 and K % 16 == 0.  (n, m) must be (2,4), (3,4) or (6,8).
+ *   - Nothing throws across this boundary.
+ */
+#ifndef SBL_H
+#define SBL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SBL_OK = 0,
+    SBL_ERR_INVALID_ARG = 1,   /* null/unaligned pointer, negative or bad size      */
+    SBL_ERR_UNSUPPORTED = 2,   /* N:M pattern or shape outside what the kernels do  */
+    SBL_ERR_NONFINITE = 3,     /* device saw NaN/Inf in W or x (sbl_device_status)  */
+    SBL_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed                 */
+    SBL_ERR_TIMEOUT = 5,       /* a bounded device-side wait ran out                */
+    SBL_ERR_WORKSPACE = 6      /* workspace missing, too small or unaligned         */
+} sbl_status;
+
+/* Output element types of sbl_linear. */
+enum { SBL_F32 = 0, SBL_BF16 = 1 };
+
+/* Contraction paths of sbl_linear_path. */
+enum { SBL_PATH_AUTO = 0, SBL_PATH_DECODE = 1, SBL_PATH_PREFILL = 2 };
+
+/*
+ * sbl_prepare_weights — N:M mask, per-row scale, ternarise and 2-bit pack.
+ *
+ * Follows the Sparse-BitNet Guide, "Mathematical Formulation of
+ * Sparse-BitLinear" (mask equation: Top-N |W| of every M contiguous input-dim
+ * weights; joint sparse-ternary equation W_t = mask * clip(round(W/scale),-1,1)),
+ * the Sparse-BitNet README, "How It Works / Sparse-BitNet" (mask first, then
+ * quantise what remains), and the halo-sparse-bitnet-3:4-500m card
+ * ("Recipe": per-row absmean; "Packed vs raw": 2 bits per weight,
+ * 00 = 0, 01 = +1, 10 = -1, four codes per byte).
+ *
+ *   W          fp32 [O, K] latent weights (input).
+ *   O, K, n, m shape and N:M pattern; K % 16 == 0, K % m == 0.
+ *   packed     uint8 [O, K/4] (output).  Weight k of a row is byte k/4,
+ *              bits 2(k%4)..2(k%4)+1 (least significant code first).
+ *   row_scale  fp32 [O] (output): mean of |W| over the kept weights of the
+ *              row — the exact sum rounded once to double, divided by the
+ *              kept count in double, rounded to float — clamped below at 1e-5.
+ *   mask_bits  uint8 [O, K/8] (output, may be NULL): bit k%8 of byte k/8 is
+ *              set when weight k is kept.  Ties in |W| keep the lower index.
+ *   round(W/scale) is round-half-to-even; a weight is nonzero exactly when it
+ *   is kept and |W| > scale/2.
+ *   Non-finite W sets SBL_ERR_NONFINITE in the device status word; the
+ *   outputs of such a row are unspecified.
+ */
+sbl_status sbl_prepare_weights(const float* W, int64_t O, int64_t K, int n, int m,
+                               uint8_t* packed, float* row_scale, uint8_t* mask_bits,
+                               void* stream);
+
+/*
+ * sbl_quant_act — per-token absmax int8 activation quantisation.
+ *
+ * Follows the activation equation of the Sparse-BitNet Guide, "Mathematical
+ * Formulation of Sparse-BitLinear" (beta = max_j |x_j| per token,
+ * clip(round(x * 127 / beta), -128, 127)) and the BitNet-TinyDialogues card
+ * (W1.58A8: 8-bit per-token activations).
+ *
+ *   x_bf16  bf16 bit patterns [T, K] (input).
+ *   x_q     int8 [T, K] (output), natural column order.
+ *   s_tok   fp32 [T] (output): s_t = 127 / max(max_k |x_tk|, 1e-5) in IEEE
+ *           float division; x_q = clamp(round_half_even(x * s_t), -128, 127)
+ *           with the product rounded to float.
+ *   Non-finite x sets SBL_ERR_NONFINITE in the device status word.
+ */
+sbl_status sbl_quant_act(const uint16_t* x_bf16, int64_t T, int64_t K,
+                         int8_t* x_q, float* s_tok, void* stream);
+
+/*
+ * sbl_linear_workspace_bytes — bytes of device workspace sbl_linear needs for
+ * these sizes (the quantised activations and their scales, in the kernels'
+ * internal layout).  Never 0 for T > 0.
+ */
+size_t sbl_linear_workspace_bytes(int64_t T, int64_t K, int64_t O, int n, int m);
+
+/*
+ * sbl_linear — y = dequant(int8(x) . W_t^T) on prepared weights.
+ *
+ * Follows the linear-evaluation equation of the Sparse-BitNet Guide,
+ * "Mathematical Formulation of Sparse-BitLinear": the integer product of the
+ * int8 activations and the ternary weights, rescaled by beta * gamma / 127,
+ * here scale_o / s_t with int32 accumulation.
+ *
+ *   x_bf16     bf16 bit patterns [T, K] (input).
+ *   packed     uint8 [O, K/4] and row_scale fp32 [O] from sbl_prepare_weights.
+ *   n, m       the N:M pattern the weights were prepared with.
+ *   y          [T, O] (output), fp32 (y_dtype SBL_F32) or bf16 (SBL_BF16,
+ *              round to nearest even of the fp32 value).
+ *   acc_out    int32 [T, O] (output, may be NULL): the integer accumulators.
+ *   workspace  device scratch of at least sbl_linear_workspace_bytes(), 256-byte
+ *              aligned; its contents on entry do not matter and are
+ *              overwritten.  Calls that share a workspace must be ordered on
+ *              one stream.
+ *   Chooses the CUDA-core decode path for T <= sbl_decode_max_tokens() and the
+ *   tcgen05 tensor-core prefill path above it (the latter needs K % 64 == 0;
+ *   other K always take the decode path).
+ */
+sbl_status sbl_linear(const uint16_t* x_bf16, int64_t T, int64_t K,
+                      const uint8_t* packed, const float* row_scale, int64_t O, int n, int m,
+                      void* y, int y_dtype, int32_t* acc_out,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * sbl_linear_path — sbl_linear with the contraction path forced
+ * (SBL_PATH_DECODE or SBL_PATH_PREFILL; SBL_PATH_AUTO is sbl_linear).
+ * SBL_PATH_PREFILL with K % 64 != 0 returns SBL_ERR_UNSUPPORTED.
+ */
+sbl_status sbl_linear_path(const uint16_t* x_bf16, int64_t T, int64_t K,
+                           const uint8_t* packed, const float* row_scale, int64_t O, int n, int m,
+                           void* y, int y_dtype, int32_t* acc_out,
+                           void* workspace, size_t workspace_bytes, int path, void* stream);
+
+/* Largest T that sbl_linear sends to the decode path. */
+int64_t sbl_decode_max_tokens(void);
+
+/*
+ * sbl_device_status — synchronises `stream`, then returns and clears the
+ * current device's status word: SBL_OK, or the first of SBL_ERR_NONFINITE /
+ * SBL_ERR_TIMEOUT that any kernel raised since the last call.
+ */
+sbl_status sbl_device_status(void* stream);
+
+/*
+ * sbl_selftest_bounded_wait — launches one block that waits on a barrier that
+ * nothing ever completes, with the same bounded wait the pipelines use but a
+ * short limit of `max_polls` polls.  The kernel records SBL_ERR_TIMEOUT in the
+ * status word and returns; the call then reports sbl_device_status().
+ * Exists so that the timeout path is tested without hanging a GPU.
+ */
+sbl_status sbl_selftest_bounded_wait(uint32_t max_polls, void* stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* sbl_status_string(sbl_status s);
+
+/* Library version string (static storage). */
+const char* sbl_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SBL_H */

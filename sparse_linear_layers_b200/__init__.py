@@ -1,0 +1,27 @@
+"""Sparse-BitLinear forward for NVIDIA B200 (sm_100a).
+
+y = dequant(int8(x) . ternary_NM(W)^T) behind a C ABI (include/sbl.h) with
+hand-written CUDA kernels: fused weight preparation, per-token activation
+quantisation, a CUDA-core decode path and a tcgen05 tensor-core prefill path.
+
+The library entry points (sbl_prepare_weights, sbl_quant_act, sbl_linear, ...)
+load libsbl.so on first use and raise ImportError if it has not been built;
+there is no CPU fallback.  ``synthetic`` (seeded input generators) needs no
+GPU library.
+"""
+__version__ = "0.1.0"
+
+_API = ("PreparedWeights", "sbl_decode_max_tokens", "sbl_device_status", "sbl_linear",
+        "sbl_linear_workspace_bytes", "sbl_prepare_weights", "sbl_quant_act", "sbl_selftest_bounded_wait",
+        "workspace_for", "SblError")
+
+
+def __getattr__(name):
+    if name in _API:
+        from . import api
+        from ._lib import SblError
+        return SblError if name == "SblError" else getattr(api, name)
+    raise AttributeError(name)
+
+
+__all__ = list(_API)

@@ -1,0 +1,122 @@
+"""PyTorch-facing calls of the Sparse-BitLinear library.
+
+PyTorch provides device memory and streams; every call forwards raw pointers
+to the C ABI (include/sbl.h) and the CUDA kernels do all the arithmetic.
+The function names follow the C entry points.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import check, lib
+
+_PATHS = {"auto": _lib.SBL_PATH_AUTO, "decode": _lib.SBL_PATH_DECODE, "prefill": _lib.SBL_PATH_PREFILL}
+
+
+def _stream(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _need_cuda(t: torch.Tensor, name: str, dtype: torch.dtype) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+@dataclass
+class PreparedWeights:
+    """2-bit packed ternary weights of one layer plus its per-row scales."""
+    packed: torch.Tensor      # uint8 [O, K/4]
+    row_scale: torch.Tensor   # fp32 [O]
+    n: int
+    m: int
+    K: int
+    mask_bits: Optional[torch.Tensor] = None  # uint8 [O, K/8]
+
+    @property
+    def O(self) -> int:
+        return self.packed.shape[0]
+
+
+def sbl_prepare_weights(W: torch.Tensor, n: int, m: int, with_mask: bool = False,
+                        out: Optional[PreparedWeights] = None,
+                        stream: Optional[torch.cuda.Stream] = None) -> PreparedWeights:
+    """N:M mask, per-row absmean scale, ternarise and pack (one kernel)."""
+    _need_cuda(W, "W", torch.float32)
+    O, K = W.shape
+    if out is None:
+        packed = torch.empty((O, K // 4), dtype=torch.uint8, device=W.device)
+        scale = torch.empty((O,), dtype=torch.float32, device=W.device)
+        mask = torch.empty((O, K // 8), dtype=torch.uint8, device=W.device) if with_mask else None
+        out = PreparedWeights(packed, scale, n, m, K, mask)
+    mb = out.mask_bits.data_ptr() if out.mask_bits is not None else None
+    check(lib.sbl_prepare_weights(W.data_ptr(), O, K, n, m, out.packed.data_ptr(), out.row_scale.data_ptr(), mb,
+                                  _stream(stream)), "sbl_prepare_weights")
+    return out
+
+
+def sbl_quant_act(x: torch.Tensor, stream: Optional[torch.cuda.Stream] = None):
+    """Per-token absmax int8 quantisation: returns (x_q int8 [T,K], s_tok fp32 [T])."""
+    _need_cuda(x, "x", torch.bfloat16)
+    T, K = x.shape
+    xq = torch.empty((T, K), dtype=torch.int8, device=x.device)
+    s = torch.empty((T,), dtype=torch.float32, device=x.device)
+    check(lib.sbl_quant_act(x.data_ptr(), T, K, xq.data_ptr(), s.data_ptr(), _stream(stream)), "sbl_quant_act")
+    return xq, s
+
+
+def sbl_linear_workspace_bytes(T: int, K: int, O: int, n: int, m: int) -> int:
+    return int(lib.sbl_linear_workspace_bytes(T, K, O, n, m))
+
+
+def workspace_for(T: int, K: int, O: int, n: int, m: int, device) -> torch.Tensor:
+    """A workspace tensor of the size sbl_linear needs (256-byte aligned by the caching allocator)."""
+    return torch.empty((max(1, sbl_linear_workspace_bytes(T, K, O, n, m)),), dtype=torch.uint8, device=device)
+
+
+def sbl_linear(x: torch.Tensor, w: PreparedWeights, out_dtype: torch.dtype = torch.float32,
+               y: Optional[torch.Tensor] = None, acc_out: Optional[torch.Tensor] = None,
+               workspace: Optional[torch.Tensor] = None, path: str = "auto",
+               stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """y = dequant(int8(x) . W_t^T); ``acc_out`` (int32 [T,O]) receives the integer accumulators."""
+    _need_cuda(x, "x", torch.bfloat16)
+    T, K = x.shape
+    if K != w.K:
+        raise ValueError(f"x has K={K}, weights were prepared with K={w.K}")
+    O = w.O
+    if y is None:
+        y = torch.empty((T, O), dtype=out_dtype, device=x.device)
+    if y.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("y must be float32 or bfloat16")
+    _need_cuda(y, "y", y.dtype)
+    ydt = _lib.SBL_F32 if y.dtype == torch.float32 else _lib.SBL_BF16
+    if acc_out is not None:
+        _need_cuda(acc_out, "acc_out", torch.int32)
+    if workspace is None:
+        workspace = workspace_for(T, K, O, w.n, w.m, x.device)
+    check(lib.sbl_linear_path(x.data_ptr(), T, K, w.packed.data_ptr(), w.row_scale.data_ptr(), O, w.n, w.m,
+                              y.data_ptr(), ydt, acc_out.data_ptr() if acc_out is not None else None,
+                              workspace.data_ptr(), workspace.numel(), _PATHS[path], _stream(stream)),
+          "sbl_linear")
+    return y
+
+
+def sbl_decode_max_tokens() -> int:
+    return int(lib.sbl_decode_max_tokens())
+
+
+def sbl_device_status(stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Synchronise and return (and clear) the device status code (0 = ok)."""
+    return int(lib.sbl_device_status(_stream(stream)))
+
+
+def sbl_selftest_bounded_wait(max_polls: int = 1000, stream: Optional[torch.cuda.Stream] = None) -> int:
+    return int(lib.sbl_selftest_bounded_wait(max_polls, _stream(stream)))

@@ -1,0 +1,194 @@
+// Weight preparation: N:M magnitude mask, per-row absmean scale over the kept
+// weights, ternarisation and 2-bit packing, fused in one pass per row.
+//
+// Operator: Sparse-BitNet Guide: 1.58-Bit LLMs Meet 2:4 Sparsity, "Mathematical
+// Formulation of Sparse-BitLinear" (mask equation, joint sparse-ternary
+// equation); per-row absmean from the halo-sparse-bitnet-3:4-500m card,
+// "Recipe"; code table 00 = 0, 01 = +1, 10 = -1 from its "Packed vs raw".
+//
+// One warp per row.  Each lane owns 16-weight chunks (c = lane, lane+32, ...),
+// read as four 16-byte loads.  Pass 1 builds the keep-mask of every group and
+// adds the kept |w| into an exact fixed-point accumulator; pass 2 re-reads the
+// chunk (L1/L2 resident), ternarises against the row scale and writes one
+// 32-bit word of codes and 16 mask bits per chunk.
+//
+// Exact sum: a finite float |w| = m * 2^(p - 149) with a 24-bit integer m and
+// 0 <= p <= 253, so the row sum is an integer in units of 2^-149 below 2^300.
+// Each lane keeps it in ten 32-bit limbs held in 64-bit shared-memory words
+// (carries are resolved once, at the end), which makes the sum independent of
+// the order of additions; the total is rounded once to double.
+#include "sbl_common.cuh"
+
+namespace sbl {
+
+constexpr int kPrepWarps = 8;
+constexpr int kLimbs = 10;
+
+__device__ __forceinline__ void exact_add(unsigned long long* limb_col, uint32_t abs_bits) {
+    const uint32_t e = abs_bits >> 23;
+    const uint32_t m24 = (abs_bits & 0x7FFFFFu) | (e ? 0x800000u : 0u);
+    const uint32_t p = e ? e - 1u : 0u;
+    const uint32_t li = p >> 5;
+    const unsigned long long v = static_cast<unsigned long long>(m24) << (p & 31u);
+    limb_col[li * 32] += v & 0xFFFFFFFFull;
+    limb_col[(li + 1) * 32] += v >> 32;
+}
+
+// Round the 320-bit integer w[0..9] (32-bit limbs, units of 2^-149) to double.
+__device__ double limbs_to_double(const uint32_t (&w)[kLimbs]) {
+    int h = -1;
+#pragma unroll
+    for (int i = kLimbs - 1; i >= 0; --i)
+        if (h < 0 && w[i] != 0u) h = i;
+    const double two_m149 = 1.4012984643248170709e-45;  // 2^-149, exact
+    if (h < 0) return 0.0;
+    if (h <= 1) {
+        const unsigned long long x = (static_cast<unsigned long long>(w[1]) << 32) | w[0];
+        return __ull2double_rn(x) * two_m149;
+    }
+    const int lz = __clz(w[h]);
+    unsigned long long top;
+    uint32_t dropped;
+    if (lz == 0) {
+        top = (static_cast<unsigned long long>(w[h]) << 32) | w[h - 1];
+        dropped = w[h - 2];
+    } else {
+        top = (static_cast<unsigned long long>(w[h]) << (32 + lz)) |
+              (static_cast<unsigned long long>(w[h - 1]) << lz) | (w[h - 2] >> (32 - lz));
+        dropped = w[h - 2] & ((1u << (32 - lz)) - 1u);
+    }
+    for (int i = 0; i < h - 2; ++i) dropped |= w[i];
+    top |= (dropped != 0u) ? 1ull : 0ull;  // sticky bit: below the rounding position
+    const int e2 = 32 * h - 32 - lz - 149;  // weight of bit 0 of `top`
+    const double scale = __longlong_as_double(static_cast<long long>(1023 + e2) << 52);
+    return __ull2double_rn(top) * scale;
+}
+
+// keep[i] for the M weights of one group: rank by magnitude, ties to the lower index.
+template <int M>
+__device__ __forceinline__ uint32_t group_keep_bits(const uint32_t* a, int n) {
+    int rank[M];
+#pragma unroll
+    for (int j = 0; j < M; ++j) rank[j] = 0;
+#pragma unroll
+    for (int i = 0; i < M; ++i)
+#pragma unroll
+        for (int j = i + 1; j < M; ++j) {
+            if (a[i] >= a[j]) ++rank[j];
+            else ++rank[i];
+        }
+    uint32_t bits = 0;
+#pragma unroll
+    for (int j = 0; j < M; ++j) bits |= (rank[j] < n ? 1u : 0u) << j;
+    return bits;
+}
+
+template <int M>
+__device__ __forceinline__ uint32_t chunk_keep_bits(const uint32_t (&a)[16], int n) {
+    uint32_t bits = 0;
+#pragma unroll
+    for (int g = 0; g < 16 / M; ++g) bits |= group_keep_bits<M>(a + g * M, n) << (g * M);
+    return bits;
+}
+
+__device__ __forceinline__ void load_chunk(const float* p, uint32_t (&bits)[16]) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint4 v = ldg_nc(p + 4 * q);
+        bits[4 * q + 0] = v.x;
+        bits[4 * q + 1] = v.y;
+        bits[4 * q + 2] = v.z;
+        bits[4 * q + 3] = v.w;
+    }
+}
+
+template <int M>
+__global__ void __launch_bounds__(kPrepWarps * 32) prep_kernel(const float* __restrict__ W, long long O, long long K,
+                                                               int n, uint8_t* __restrict__ packed,
+                                                               float* __restrict__ row_scale,
+                                                               uint8_t* __restrict__ mask_bits, unsigned* status) {
+    __shared__ unsigned long long limbs[kPrepWarps][kLimbs][32];
+    __shared__ unsigned long long totals[kPrepWarps][kLimbs];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long row = static_cast<long long>(blockIdx.x) * kPrepWarps + warp;
+    if (row >= O) return;  // whole warps leave together; no block barrier below
+
+    const float* wr = W + row * K;
+    const int nchunks = static_cast<int>(K >> 4);
+    unsigned long long* my = &limbs[warp][0][lane];
+#pragma unroll
+    for (int l = 0; l < kLimbs; ++l) my[l * 32] = 0ull;
+
+    bool bad = false;
+    for (int c = lane; c < nchunks; c += 32) {
+        uint32_t a[16];
+        load_chunk(wr + 16 * c, a);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            a[i] &= 0x7FFFFFFFu;
+            bad |= a[i] >= 0x7F800000u;
+        }
+        const uint32_t keep = chunk_keep_bits<M>(a, n);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            if (keep & (1u << i)) exact_add(my, a[i]);
+    }
+    __syncwarp();
+    if (lane < kLimbs) {
+        unsigned long long s = 0;
+        for (int i = 0; i < 32; ++i) s += limbs[warp][lane][i];
+        totals[warp][lane] = s;
+    }
+    __syncwarp();
+
+    float scale = 0.f;
+    if (lane == 0) {
+        uint32_t w[kLimbs];
+        unsigned long long carry = 0;
+#pragma unroll
+        for (int i = 0; i < kLimbs; ++i) {
+            const unsigned long long t = totals[warp][i] + carry;
+            w[i] = static_cast<uint32_t>(t);
+            carry = t >> 32;
+        }
+        const double sum = limbs_to_double(w);
+        const double kept = static_cast<double>((K / M) * n);
+        scale = fmaxf(__double2float_rn(__ddiv_rn(sum, kept)), 1e-5f);
+        row_scale[row] = scale;
+    }
+    scale = __shfl_sync(0xFFFFFFFFu, scale, 0);
+    if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) raise_status(status, kStatusNonfinite);
+
+    const uint32_t half_bits = __float_as_uint(0.5f * scale);  // exact: scale >= 1e-5 is normal
+    uint32_t* prow = reinterpret_cast<uint32_t*>(packed + row * (K >> 2));
+    uint16_t* mrow = mask_bits ? reinterpret_cast<uint16_t*>(mask_bits + row * (K >> 3)) : nullptr;
+    for (int c = lane; c < nchunks; c += 32) {
+        uint32_t raw[16], a[16];
+        load_chunk(wr + 16 * c, raw);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) a[i] = raw[i] & 0x7FFFFFFFu;
+        const uint32_t keep = chunk_keep_bits<M>(a, n);
+        uint32_t codes = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            // round(w / scale) != 0  <=>  |w| / scale > 1/2  <=>  |w| > scale / 2 (exact compare)
+            const bool nz = ((keep >> i) & 1u) && (a[i] > half_bits);
+            const uint32_t code = nz ? ((raw[i] >> 31) ? 2u : 1u) : 0u;
+            codes |= code << (2 * i);
+        }
+        prow[c] = codes;
+        if (mrow) mrow[c] = static_cast<uint16_t>(keep);
+    }
+}
+
+cudaError_t launch_prep(const float* W, long long O, long long K, int n, int m, uint8_t* packed, float* row_scale,
+                        uint8_t* mask_bits, unsigned* status, cudaStream_t stream) {
+    const unsigned blocks = static_cast<unsigned>((O + kPrepWarps - 1) / kPrepWarps);
+    if (m == 4)
+        prep_kernel<4><<<blocks, kPrepWarps * 32, 0, stream>>>(W, O, K, n, packed, row_scale, mask_bits, status);
+    else
+        prep_kernel<8><<<blocks, kPrepWarps * 32, 0, stream>>>(W, O, K, n, packed, row_scale, mask_bits, status);
+    return cudaGetLastError();
+}
+
+}  // namespace sbl

@@ -1,0 +1,201 @@
+// C ABI of the Sparse-BitLinear library: argument validation, workspace
+// layout, path dispatch and the per-device status word.  All arithmetic runs
+// in the kernels of prep.cu, quant.cu, decode.cu and prefill.cu.
+#include <cstdint>
+#include <cstdio>
+#include <cuda_runtime.h>
+
+#include "sbl.h"
+#include "sbl_common.cuh"
+
+namespace sbl {
+cudaError_t launch_prep(const float* W, long long O, long long K, int n, int m, uint8_t* packed, float* row_scale,
+                        uint8_t* mask_bits, unsigned* status, cudaStream_t stream);
+cudaError_t launch_quant(const uint16_t* x, long long T, long long K, int8_t* xq, float* s_tok, bool interleaved,
+                         unsigned* status, cudaStream_t stream);
+cudaError_t launch_decode(const uint8_t* packed, const float* row_scale, long long O, long long K,
+                          const int8_t* xperm, const float* s_tok, long long T, void* y, int y_bf16,
+                          int32_t* acc_out, int num_sms, cudaStream_t stream);
+cudaError_t launch_prefill(const int8_t* xperm, const float* s_tok, long long T, long long K, const uint8_t* packed,
+                           const float* row_scale, long long O, void* y, int y_bf16, int32_t* acc_out,
+                           unsigned* status, int num_sms, cudaStream_t stream);
+
+// Status word: one per device, read and cleared by sbl_device_status().
+__device__ unsigned g_status_word;
+
+__global__ void bounded_wait_selftest(uint32_t max_polls, unsigned* status) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    for (uint32_t i = 0; i < max_polls; ++i)
+        if (mbar_try_wait(&bar, 0)) return;  // nothing ever arrives: phase 0 never completes
+    raise_status(status, kStatusTimeout);
+}
+}  // namespace sbl
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr long long kMaxK = 1ll << 24;            // keeps |acc| <= 127 * K below 2^31
+constexpr long long kDecodeMaxTokens = 16;
+
+struct DeviceInfo {
+    unsigned* status = nullptr;
+    int num_sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+
+sbl_status device_info(DeviceInfo** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SBL_ERR_CUDA;
+    DeviceInfo& d = g_dev[dev];
+    if (!d.status) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, sbl::g_status_word) != cudaSuccess) return SBL_ERR_CUDA;
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return SBL_ERR_CUDA;
+        d.num_sms = sms;
+        d.status = static_cast<unsigned*>(p);
+    }
+    *out = &d;
+    return SBL_OK;
+}
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+inline bool nm_ok(int n, int m) { return (n == 2 && m == 4) || (n == 3 && m == 4) || (n == 6 && m == 8); }
+
+inline size_t round256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
+inline sbl_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SBL_OK : SBL_ERR_CUDA; }
+
+sbl_status check_k(long long K) {
+    if (K <= 0 || K % 16 != 0) return SBL_ERR_INVALID_ARG;
+    if (K > kMaxK) return SBL_ERR_UNSUPPORTED;
+    return SBL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+sbl_status sbl_prepare_weights(const float* W, int64_t O, int64_t K, int n, int m, uint8_t* packed,
+                               float* row_scale, uint8_t* mask_bits, void* stream) {
+    if (O < 0) return SBL_ERR_INVALID_ARG;
+    if (sbl_status s = check_k(K)) return s;
+    if (!nm_ok(n, m)) return SBL_ERR_UNSUPPORTED;
+    if (O == 0) return SBL_OK;
+    if (!W || !packed || !row_scale) return SBL_ERR_INVALID_ARG;
+    if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(row_scale, 16)) return SBL_ERR_INVALID_ARG;
+    if (mask_bits && !aligned(mask_bits, 16)) return SBL_ERR_INVALID_ARG;
+    if (O > (1ll << 31) - 1) return SBL_ERR_UNSUPPORTED;
+    DeviceInfo* d;
+    if (sbl_status s = device_info(&d)) return s;
+    return from_cuda(sbl::launch_prep(W, O, K, n, m, packed, row_scale, mask_bits, d->status,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+sbl_status sbl_quant_act(const uint16_t* x_bf16, int64_t T, int64_t K, int8_t* x_q, float* s_tok, void* stream) {
+    if (T < 0) return SBL_ERR_INVALID_ARG;
+    if (sbl_status s = check_k(K)) return s;
+    if (T == 0) return SBL_OK;
+    if (!x_bf16 || !x_q || !s_tok) return SBL_ERR_INVALID_ARG;
+    if (!aligned(x_bf16, 16) || !aligned(x_q, 16) || !aligned(s_tok, 16)) return SBL_ERR_INVALID_ARG;
+    if (T > (1ll << 31) - 1) return SBL_ERR_UNSUPPORTED;
+    DeviceInfo* d;
+    if (sbl_status s = device_info(&d)) return s;
+    return from_cuda(sbl::launch_quant(x_bf16, T, K, x_q, s_tok, false, d->status, static_cast<cudaStream_t>(stream)));
+}
+
+size_t sbl_linear_workspace_bytes(int64_t T, int64_t K, int64_t O, int n, int m) {
+    (void)O;
+    (void)n;
+    (void)m;
+    if (T <= 0 || K <= 0) return 0;
+    return round256(static_cast<size_t>(T) * static_cast<size_t>(K)) + round256(static_cast<size_t>(T) * 4);
+}
+
+sbl_status sbl_linear_path(const uint16_t* x_bf16, int64_t T, int64_t K, const uint8_t* packed,
+                           const float* row_scale, int64_t O, int n, int m, void* y, int y_dtype, int32_t* acc_out,
+                           void* workspace, size_t workspace_bytes, int path, void* stream) {
+    if (T < 0 || O < 0) return SBL_ERR_INVALID_ARG;
+    if (sbl_status s = check_k(K)) return s;
+    if (!nm_ok(n, m)) return SBL_ERR_UNSUPPORTED;
+    if (y_dtype != SBL_F32 && y_dtype != SBL_BF16) return SBL_ERR_INVALID_ARG;
+    if (path != SBL_PATH_AUTO && path != SBL_PATH_DECODE && path != SBL_PATH_PREFILL) return SBL_ERR_INVALID_ARG;
+    if (path == SBL_PATH_PREFILL && K % 64 != 0) return SBL_ERR_UNSUPPORTED;
+    if (T == 0 || O == 0) return SBL_OK;
+    if (!x_bf16 || !packed || !row_scale || !y) return SBL_ERR_INVALID_ARG;
+    if (!aligned(x_bf16, 16) || !aligned(packed, 16) || !aligned(row_scale, 16) || !aligned(y, 16))
+        return SBL_ERR_INVALID_ARG;
+    if (acc_out && !aligned(acc_out, 16)) return SBL_ERR_INVALID_ARG;
+    if (T > (1ll << 31) - 1 || O > (1ll << 31) - 1) return SBL_ERR_UNSUPPORTED;
+    const size_t need = sbl_linear_workspace_bytes(T, K, O, n, m);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return SBL_ERR_WORKSPACE;
+
+    DeviceInfo* d;
+    if (sbl_status s = device_info(&d)) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int8_t* xq = static_cast<int8_t*>(workspace);
+    float* s_tok = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round256(static_cast<size_t>(T) * K));
+
+    bool prefill = path == SBL_PATH_PREFILL;
+    if (path == SBL_PATH_AUTO) prefill = (T > kDecodeMaxTokens) && (K % 64 == 0);
+
+    cudaError_t e = sbl::launch_quant(x_bf16, T, K, xq, s_tok, true, d->status, st);
+    if (e != cudaSuccess) return SBL_ERR_CUDA;
+    const int ybf = y_dtype == SBL_BF16 ? 1 : 0;
+    if (prefill)
+        e = sbl::launch_prefill(xq, s_tok, T, K, packed, row_scale, O, y, ybf, acc_out, d->status, d->num_sms, st);
+    else
+        e = sbl::launch_decode(packed, row_scale, O, K, xq, s_tok, T, y, ybf, acc_out, d->num_sms, st);
+    return from_cuda(e);
+}
+
+sbl_status sbl_linear(const uint16_t* x_bf16, int64_t T, int64_t K, const uint8_t* packed, const float* row_scale,
+                      int64_t O, int n, int m, void* y, int y_dtype, int32_t* acc_out, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+    return sbl_linear_path(x_bf16, T, K, packed, row_scale, O, n, m, y, y_dtype, acc_out, workspace,
+                           workspace_bytes, SBL_PATH_AUTO, stream);
+}
+
+int64_t sbl_decode_max_tokens(void) { return kDecodeMaxTokens; }
+
+sbl_status sbl_device_status(void* stream) {
+    DeviceInfo* d;
+    if (sbl_status s = device_info(&d)) return s;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SBL_ERR_CUDA;
+    unsigned word = 0;
+    if (cudaMemcpy(&word, d->status, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return SBL_ERR_CUDA;
+    const unsigned zero = 0;
+    if (cudaMemcpy(d->status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return SBL_ERR_CUDA;
+    if (word & sbl::kStatusTimeout) return SBL_ERR_TIMEOUT;
+    if (word & sbl::kStatusNonfinite) return SBL_ERR_NONFINITE;
+    return SBL_OK;
+}
+
+sbl_status sbl_selftest_bounded_wait(uint32_t max_polls, void* stream) {
+    DeviceInfo* d;
+    if (sbl_status s = device_info(&d)) return s;
+    sbl::bounded_wait_selftest<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(max_polls, d->status);
+    if (cudaGetLastError() != cudaSuccess) return SBL_ERR_CUDA;
+    return sbl_device_status(stream);
+}
+
+const char* sbl_status_string(sbl_status s) {
+    switch (s) {
+        case SBL_OK: return "ok";
+        case SBL_ERR_INVALID_ARG: return "invalid argument";
+        case SBL_ERR_UNSUPPORTED: return "unsupported pattern or shape";
+        case SBL_ERR_NONFINITE: return "non-finite input seen on the device";
+        case SBL_ERR_CUDA: return "CUDA error";
+        case SBL_ERR_TIMEOUT: return "bounded device wait ran out";
+        case SBL_ERR_WORKSPACE: return "workspace missing, too small or unaligned";
+    }
+    return "unknown status";
+}
+
+const char* sbl_version(void) { return "sbl 0.1.0 (sm_100a)"; }
+
+}  // extern "C"

@@ -8,3 +8,10 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+
+
+def pytest_sessionstart(session):
+    # The library is built in-tree (nvcc cross-compiles without a GPU); rebuild
+    # only when a source is newer than libsbl.so.
+    from sparse_linear_layers_b200.build import build_library
+    build_library()

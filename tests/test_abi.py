@@ -1,0 +1,96 @@
+"""The C ABI library loads, exports every entry point include/sbl.h declares, and
+rejects bad arguments on the host before touching a device (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sbl.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sbl_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for must in ("sbl_prepare_weights", "sbl_quant_act", "sbl_linear", "sbl_linear_workspace_bytes"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    from sparse_linear_layers_b200 import _lib
+    raw = ctypes.CDLL(_lib.LIB_PATH)
+    for name in _declared():
+        assert hasattr(raw, name), name
+    assert set(_declared()) == set(_lib.SIGNATURES), "binding signatures out of sync with sbl.h"
+
+
+def test_version_and_status_strings():
+    from sparse_linear_layers_b200._lib import lib, status_string
+    assert b"sm_100a" in lib.sbl_version()
+    for code in range(7):
+        assert status_string(code)
+    assert status_string(99) == "unknown status"
+
+
+def test_workspace_bytes():
+    from sparse_linear_layers_b200._lib import lib
+    assert lib.sbl_linear_workspace_bytes(0, 896, 896, 3, 4) == 0
+    # x_q (T*K rounded to 256) + s_tok (T*4 rounded to 256)
+    assert lib.sbl_linear_workspace_bytes(2048, 896, 896, 3, 4) == 2048 * 896 + 8192
+    assert lib.sbl_linear_workspace_bytes(3, 48, 16, 2, 4) == 256 + 256
+
+
+@pytest.mark.parametrize("args,code", [
+    # (O, K, n, m)
+    ((-1, 64, 2, 4), 1),     # negative O
+    ((8, 0, 2, 4), 1),       # K == 0
+    ((8, 40, 2, 4), 1),      # K % 16 != 0
+    ((8, 64, 1, 4), 2),      # unsupported N:M
+    ((8, 64, 4, 8), 2),
+    ((8, 1 << 25, 2, 4), 2), # K beyond the int32-accumulator bound
+])
+def test_prepare_rejects_on_host(args, code):
+    from sparse_linear_layers_b200._lib import lib
+    O, K, n, m = args
+    assert lib.sbl_prepare_weights(None, O, K, n, m, None, None, None, None) == code
+
+
+def test_zero_sizes_are_noops_without_a_device():
+    from sparse_linear_layers_b200._lib import lib
+    assert lib.sbl_prepare_weights(None, 0, 64, 2, 4, None, None, None, None) == 0
+    assert lib.sbl_quant_act(None, 0, 64, None, None, None) == 0
+    assert lib.sbl_linear(None, 0, 64, None, None, 16, 2, 4, None, 0, None, None, 0, None) == 0
+    assert lib.sbl_linear(None, 4, 64, None, None, 0, 2, 4, None, 0, None, None, 0, None) == 0
+
+
+def test_linear_rejects_on_host():
+    from sparse_linear_layers_b200._lib import lib
+    L = lib.sbl_linear_path
+    p = 4096  # a fake, 16-byte aligned address: never dereferenced, validation fails first
+    # bad output dtype
+    assert L(p, 4, 64, p, p, 16, 2, 4, p, 7, None, p, 1 << 20, 0, None) == 1
+    # bad path
+    assert L(p, 4, 64, p, p, 16, 2, 4, p, 0, None, p, 1 << 20, 9, None) == 1
+    # prefill needs K % 64 == 0
+    assert L(p, 4, 48, p, p, 16, 2, 4, p, 0, None, p, 1 << 20, 2, None) == 2
+    # unaligned y
+    assert L(p, 4, 64, p, p, 16, 2, 4, p + 4, 0, None, p, 1 << 20, 0, None) == 1
+    # workspace too small / unaligned
+    assert L(p, 4, 64, p, p, 16, 2, 4, p, 0, None, p, 16, 0, None) == 6
+    assert L(p, 4, 64, p, p, 16, 2, 4, p, 0, None, p + 16, 1 << 20, 0, None) == 6
+    assert L(p, 4, 64, p, p, 16, 2, 4, p, 0, None, None, 1 << 20, 0, None) == 6
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    import importlib
+    from sparse_linear_layers_b200 import _lib
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "absent.so"))
+    with pytest.raises(ImportError):
+        _lib._load()
+    importlib.reload(_lib)  # restore the real module state

@@ -1,0 +1,222 @@
+"""CUDA path against the CPU oracle, element by element, through the C ABI.
+
+Bit-exact: packed codes, mask bits, row scales (as fp32 bit patterns), x_q,
+s_tok and the int32 accumulators.  fp32 outputs within 1e-5 relative, bf16
+outputs within 2 ulp of the rounded oracle value.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity_util import (assert_bf16_close, assert_fp32_close, layer_inputs, oracle_layer, to_dev, x_dev)
+
+pytestmark = pytest.mark.gpu
+
+PATTERNS = [(2, 4), (3, 4), (6, 8)]
+
+
+@pytest.fixture(scope="module")
+def sbl():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import sparse_linear_layers_b200 as m
+    return m
+
+
+def _prep(sbl, W, n, m):
+    w = sbl.sbl_prepare_weights(to_dev(W), n, m, with_mask=True)
+    torch.cuda.synchronize()
+    return w
+
+
+# ------------------------------------------------------------------ weight prep
+
+@pytest.mark.parametrize("n,m", PATTERNS)
+@pytest.mark.parametrize("O,K", [(512, 256), (37, 48), (130, 320), (9, 16 * 8)])
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_prepare_bit_exact(sbl, n, m, O, K, seed):
+    if K % m:
+        pytest.skip("K not a multiple of M")
+    W, _, _ = layer_inputs(O, K, 1, seed=seed)
+    # plant ties, zero groups and a zero row
+    W[0, :m] = np.float32(0.03125)
+    W[1, : 2 * m] = 0.0
+    W[-1, :] = 0.0
+    w = _prep(sbl, W, n, m)
+    packed, scale, mbits, _ = oracle.prepare_weights(W, n, m)
+    assert np.array_equal(w.packed.cpu().numpy(), packed)
+    assert np.array_equal(w.row_scale.cpu().numpy().view(np.uint32), scale.view(np.uint32))
+    assert np.array_equal(w.mask_bits.cpu().numpy(), mbits)
+
+
+@pytest.mark.parametrize("n,m,O,K", [(3, 4, 4864, 896), (3, 4, 896, 4864), (2, 4, 7168, 2048),
+                                     (6, 8, 2048, 7168)])
+def test_prepare_bit_exact_full_layers(sbl, n, m, O, K):
+    W, _, _ = layer_inputs(O, K, 1, seed=0)
+    w = _prep(sbl, W, n, m)
+    packed, scale, mbits, _ = oracle.prepare_weights(W, n, m)
+    assert np.array_equal(w.row_scale.cpu().numpy().view(np.uint32), scale.view(np.uint32))
+    assert np.array_equal(w.packed.cpu().numpy(), packed)
+    assert np.array_equal(w.mask_bits.cpu().numpy(), mbits)
+
+
+def test_prepare_extreme_magnitudes(sbl):
+    # denormals, huge values and mixed exponents stress the exact row sum
+    rng = np.random.default_rng(7)
+    O, K = 64, 256
+    e = rng.integers(-149, 120, size=(O, K)).astype(np.float64)
+    W = (rng.choice([-1.0, 1.0], size=(O, K)) * rng.random((O, K)) * np.exp2(e)).astype(np.float32)
+    W[3] = np.float32(1e-45)
+    W[4] = np.float32(3.0e38)
+    for n, m in PATTERNS:
+        w = _prep(sbl, W, n, m)
+        packed, scale, mbits, _ = oracle.prepare_weights(W, n, m)
+        assert np.array_equal(w.row_scale.cpu().numpy().view(np.uint32), scale.view(np.uint32))
+        assert np.array_equal(w.packed.cpu().numpy(), packed)
+
+
+# ------------------------------------------------------------------ activation quant
+
+@pytest.mark.parametrize("T,K,p", [(16, 256, 0.0), (3, 48, 0.0), (257, 896, 0.01), (64, 4864, 0.01)])
+def test_quant_bit_exact(sbl, T, K, p):
+    _, xbits, xval = layer_inputs(8, K, T, seed=1, outlier_p=p)
+    xbits[0] = 0  # zero token
+    xval[0] = 0.0
+    xq, s = sbl.sbl_quant_act(x_dev(xbits))
+    rq, rs = oracle.quant_act(xval)
+    assert np.array_equal(xq.cpu().numpy(), rq)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+
+
+# ------------------------------------------------------------------ linear
+
+def _run_linear(sbl, w, xbits, T, O, path, out_dtype=torch.float32):
+    acc = torch.empty((T, O), dtype=torch.int32, device="cuda")
+    y = sbl.sbl_linear(x_dev(xbits), w, out_dtype=out_dtype, acc_out=acc, path=path)
+    assert sbl.sbl_device_status() == 0
+    return y, acc
+
+
+LINEAR_CASES = [
+    # (O, K, T, n, m): config-1 shape, ragged tiles and tails, K % 128 == 64, narrow/wide N tiles
+    (512, 256, 16, 2, 4),
+    (40, 64, 3, 3, 4),
+    (300, 320, 130, 6, 8),
+    (130, 192, 17, 2, 4),
+    (384, 896, 257, 3, 4),
+    (896, 128, 1, 3, 4),
+]
+
+
+@pytest.mark.parametrize("path", ["decode", "prefill"])
+@pytest.mark.parametrize("O,K,T,n,m", LINEAR_CASES)
+def test_linear_parity(sbl, path, O, K, T, n, m):
+    W, xbits, xval = layer_inputs(O, K, T, seed=2, outlier_p=0.01)
+    ref = oracle_layer(W, n, m, xval)
+    w = _prep(sbl, W, n, m)
+    y, acc = _run_linear(sbl, w, xbits, T, O, path)
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    assert_fp32_close(y.cpu().numpy(), ref["y"])
+    yb, _ = _run_linear(sbl, w, xbits, T, O, path, torch.bfloat16)
+    assert_bf16_close(yb.cpu().view(torch.int16).numpy(), ref["y"])
+
+
+@pytest.mark.parametrize("T", [1, 2, 5, 8, 9, 16])
+def test_decode_token_counts(sbl, T):
+    O, K, n, m = 200, 448, 3, 4
+    W, xbits, xval = layer_inputs(O, K, T, seed=0)
+    ref = oracle_layer(W, n, m, xval)
+    w = _prep(sbl, W, n, m)
+    y, acc = _run_linear(sbl, w, xbits, T, O, "decode")
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    assert_fp32_close(y.cpu().numpy(), ref["y"])
+
+
+def test_decode_k_not_multiple_of_64(sbl):
+    O, K, T, n, m = 77, 48, 4, 2, 4
+    W, xbits, xval = layer_inputs(O, K, T, seed=3)
+    ref = oracle_layer(W, n, m, xval)
+    w = _prep(sbl, W, n, m)
+    y, acc = _run_linear(sbl, w, xbits, T, O, "auto")
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    assert_fp32_close(y.cpu().numpy(), ref["y"])
+
+
+def test_zero_rows_and_tokens(sbl):
+    O, K, T, n, m = 256, 256, 40, 2, 4
+    W, xbits, xval = layer_inputs(O, K, T, seed=4)
+    W[5] = 0.0
+    xbits[7] = 0
+    xval[7] = 0.0
+    ref = oracle_layer(W, n, m, xval)
+    w = _prep(sbl, W, n, m)
+    for path in ("decode", "prefill"):
+        y, acc = _run_linear(sbl, w, xbits, T, O, path)
+        yn = y.cpu().numpy()
+        assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+        assert not yn[7].any() and not yn[:, 5].any()
+
+
+# ------------------------------------------------------------------ full-size layers
+
+@pytest.mark.parametrize("T", [1, 2048])
+def test_qwen_layer_full(sbl, T):
+    """Qwen2.5-0.5B-shaped projections at 3:4, fully compared."""
+    from sparse_linear_layers_b200.synthetic import QWEN05_LAYER
+    for name, K, O in QWEN05_LAYER:
+        W, xbits, xval = layer_inputs(O, K, T, seed=0, tag=name)
+        ref = oracle_layer(W, 3, 4, xval)
+        w = _prep(sbl, W, 3, 4)
+        y, acc = _run_linear(sbl, w, xbits, T, O, "auto")
+        assert np.array_equal(acc.cpu().numpy(), ref["acc"]), name
+        assert_fp32_close(y.cpu().numpy(), ref["y"], name)
+
+
+def test_ffn_prefill_32k_sampled(sbl):
+    """0.5B FFN shapes at T = 32768 (1% outliers x20), 3:4 and 2:4: sampled accumulators."""
+    from sparse_linear_layers_b200.synthetic import QWEN05_FFN
+    rng = np.random.default_rng(0)
+    T = 32768
+    for n, m in ((3, 4), (2, 4)):
+        for name, K, O in QWEN05_FFN:
+            W, xbits, xval = layer_inputs(O, K, T, seed=0, outlier_p=0.01, tag=name)
+            packed, scale, _, Wt = oracle.prepare_weights(W, n, m)
+            xq, s = oracle.quant_act(xval)
+            w = _prep(sbl, W, n, m)
+            assert np.array_equal(w.packed.cpu().numpy(), packed)
+            acc = torch.empty((T, O), dtype=torch.int32, device="cuda")
+            y = sbl.sbl_linear(x_dev(xbits), w, acc_out=acc)
+            assert sbl.sbl_device_status() == 0
+            ti = rng.integers(0, T, 4096)
+            oi = rng.integers(0, O, 4096)
+            ti[:2] = [0, T - 1]
+            oi[:2] = [0, O - 1]
+            ref_acc = oracle.acc_entries(xq, Wt, ti, oi)
+            got = acc.cpu().numpy()[ti, oi]
+            assert np.array_equal(got.astype(np.int64), ref_acc)
+            ref_y = ref_acc * scale.astype(np.float64)[oi] / s.astype(np.float64)[ti]
+            assert_fp32_close(y.cpu().numpy()[ti, oi], ref_y)
+
+
+# ------------------------------------------------------------------ device status paths
+
+def test_nonfinite_inputs_raise_status(sbl):
+    W, xbits, _ = layer_inputs(64, 128, 4, seed=5)
+    W[3, 7] = np.nan
+    sbl.sbl_prepare_weights(to_dev(W), 2, 4)
+    assert sbl.sbl_device_status() == 3
+    xbits[1, 2] = 0x7F80  # +inf
+    sbl.sbl_quant_act(x_dev(xbits))
+    assert sbl.sbl_device_status() == 3
+    assert sbl.sbl_device_status() == 0  # cleared
+
+
+def test_bounded_wait_times_out_cleanly(sbl):
+    assert sbl.sbl_selftest_bounded_wait(200) == 5
+    # the context stays usable
+    W, xbits, xval = layer_inputs(64, 128, 4, seed=6)
+    ref = oracle_layer(W, 2, 4, xval)
+    w = _prep(sbl, W, 2, 4)
+    _, acc = _run_linear(sbl, w, xbits, 4, 64, "prefill")
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
