@@ -147,16 +147,50 @@ class Layer:
         return self.O * self.K / 4 + 4 * self.O + 2 * T * self.K + 4 * T * self.O
 
 
-def _step(sbl, layers, ev=None):
-    """One pass of the whole path over the seven projections; optional events around the prefill calls."""
-    for i, L in enumerate(layers):
+def _prep_phase(sbl, layers):
+    for L in layers:
         sbl.sbl_prepare_weights(L.W, N, M, out=L.w)
-        if ev is not None:
-            ev[i][0].record()
+
+
+def _prefill_phase(sbl, layers):
+    for L in layers:
         sbl.sbl_linear(L.x, L.w, y=L.y, workspace=L.ws)
-        if ev is not None:
-            ev[i][1].record()
+
+
+def _decode_phase(sbl, layers):
+    for L in layers:
         sbl.sbl_linear(L.x1, L.w, y=L.y1, workspace=L.ws)
+
+
+PHASES = (("prep", _prep_phase), ("prefill", _prefill_phase), ("decode", _decode_phase))
+
+
+class StepGraphs:
+    """The step captured as three CUDA graphs (weight prep, T=2048 prefill,
+    T=1 decode) so that the timed region is free of host launch latency;
+    events between the graph launches give each phase's device time."""
+
+    def __init__(self, sbl, layers, stream):
+        self.stream = stream
+        self.graphs = []
+        with torch.cuda.stream(stream):
+            for _, fn in PHASES:       # one eager pass: sets kernel attributes before capture
+                fn(sbl, layers)
+        stream.synchronize()
+        for _, fn in PHASES:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                fn(sbl, layers)
+            self.graphs.append(g)
+
+    def replay(self, ev=None):
+        with torch.cuda.stream(self.stream):
+            if ev is not None:
+                ev[0].record(self.stream)
+            for i, g in enumerate(self.graphs):
+                g.replay()
+                if ev is not None:
+                    ev[i + 1].record(self.stream)
 
 
 def _step_e2e(sbl, layers):
@@ -200,15 +234,16 @@ def _decode_roofline(sbl, dev, hbm_peak, K=2048, O=7168, reps=64):
     with torch.cuda.graph(g, stream=s):
         for i in range(reps):
             sbl.sbl_linear(x1, ws_list[i % pool], y=y1, workspace=ws)
-    for _ in range(3):
-        g.replay()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(s)
     n_rep = 10
-    for _ in range(n_rep):
-        g.replay()
-    e1.record(s)
+    with torch.cuda.stream(s):
+        for _ in range(3):
+            g.replay()
+        e0.record(s)
+        for _ in range(n_rep):
+            g.replay()
+        e1.record(s)
     torch.cuda.synchronize()
     per_call_s = e0.elapsed_time(e1) / 1e3 / (n_rep * reps)
     # isolated single call (cold weights)
@@ -237,36 +272,38 @@ def run_ours(args, rank, world, dev):
     layers = [Layer(nm, K, O, dev) for nm, K, O in synthetic.QWEN05_LAYER]
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
-    for _ in range(args.warmup):
-        _step(sbl, layers)
+    stream = torch.cuda.Stream()
+    graphs = StepGraphs(sbl, layers, stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            flush.zero_()
+            graphs.replay()
     torch.cuda.synchronize()
     status = sbl.sbl_device_status()
     if status != 0:
         raise RuntimeError(f"device status {status} after warm-up")
 
     K = args.steps
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    pev = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in layers]
-           for _ in range(K)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(PHASES) + 1)] for _ in range(K)]
     _barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
-        for i in range(K):
-            flush.zero_()
-            starts[i].record()
-            _step(sbl, layers, pev[i])
-            ends[i].record()
+        time.sleep(0.3)  # let nvidia-smi start sampling before the timed region
+        with torch.cuda.stream(stream):
+            for i in range(K):
+                flush.zero_()
+                graphs.replay(ev[i])
         torch.cuda.synchronize()
     _barrier(world)
-    step_ms = [starts[i].elapsed_time(ends[i]) for i in range(K)]
+    step_ms = [ev[i][0].elapsed_time(ev[i][-1]) for i in range(K)]
+    phase_ms = {name: sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)) / K
+                for j, (name, _) in enumerate(PHASES)}
     total_s = sum(step_ms) / 1e3
     total_s = _max_over_ranks(total_s, world, dev)
     clocks = clk.summary()
 
-    # prefill contraction roofline (quantisation + tcgen05 GEMM, the dominant calls)
-    pre_s = sum(pev[i][j][0].elapsed_time(pev[i][j][1]) for i in range(K) for j in range(len(layers))) / 1e3
-    pre_s_per_step = pre_s / K
+    # prefill contraction roofline (quantisation + tcgen05 GEMM, the dominant phase)
+    pre_s_per_step = phase_ms["prefill"] / 1e3
     ops = sum(L.prefill_ops() for L in layers)
     byts = sum(L.prefill_bytes() for L in layers)
     t_tensor = ops / (int8_peak_tops * 1e12)
@@ -282,22 +319,27 @@ def run_ours(args, rank, world, dev):
                  "us_per_step": pre_s_per_step * 1e6, "peak_source": f"{peak_kind} (int8 = 2 x bf16 burst)"
                  if roof["bound"] == "tensor" else f"{peak_kind} hbm_gbs",
                  "tensor_tops": ops / pre_s_per_step / 1e12, "tensor_frac": ops / pre_s_per_step / 1e12 / int8_peak_tops})
+    prep_bytes = sum(L.O * L.K * 4 + L.O * L.K / 4 + 4 * L.O for L in layers)
+    phases = {name: {"us_per_step": 1e3 * v} for name, v in phase_ms.items()}
+    phases["prep"]["gbs"] = prep_bytes / (phase_ms["prep"] / 1e3) / 1e9
+    phases["decode"]["gbs"] = sum(L.decode_bytes() for L in layers) / (phase_ms["decode"] / 1e3) / 1e9
 
     # end to end through host buffers
     for _ in range(2):
         _step_e2e(sbl, layers)
     torch.cuda.synchronize()
     _barrier(world)
+    K_e2e = min(K, 50)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for _ in range(K):
+    for _ in range(K_e2e):
         h2d, d2h = _step_e2e(sbl, layers)
     e1.record()
     torch.cuda.synchronize()
     e2e_s = _max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev)
 
     decode = _decode_roofline(sbl, dev, hbm_peak) if rank == 0 else None
-    launches_per_step = len(layers) * (1 + 2 + 2)  # prep + (quant + GEMM) x 2 token counts
+    launches_per_step = len(layers) * (1 + 2 + 1)  # prep + (quant + tcgen05 GEMM) + fused decode
     value = world * TOKENS_PER_STEP * K / total_s
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
@@ -306,7 +348,8 @@ def run_ours(args, rank, world, dev):
         "config": _config({"parallelism": f"replicas x{world} (no collective on the data path)"}),
         "roofline": roof,
         "decode_roofline": decode,
-        "e2e": {"value": world * TOKENS_PER_STEP * K / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        "phases": phases,
+        "e2e": {"value": world * TOKENS_PER_STEP * K_e2e / e2e_s, "steps": K_e2e, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * K,
         "clocks": clocks,
@@ -396,8 +439,8 @@ def _max_over_ranks(v, world, dev):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

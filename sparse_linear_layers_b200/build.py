@@ -37,11 +37,12 @@ def _stale() -> bool:
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build_library(force: bool = False, verbose: bool = False, extra=()) -> str:
+def build_library(force: bool = False, verbose: bool = False, extra=(), lib_path: str = LIB,
+                  build_dir: str = "_build") -> str:
     """Compile every kernel into ``libsbl.so`` next to this file; returns its path."""
-    if not force and not _stale():
-        return LIB
-    out_dir = os.path.join(ROOT, "_build")
+    if not force and lib_path == LIB and not _stale():
+        return lib_path
+    out_dir = os.path.join(ROOT, build_dir)
     os.makedirs(out_dir, exist_ok=True)
     nvcc = _nvcc()
     common = [*ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC,
@@ -54,13 +55,13 @@ def build_library(force: bool = False, verbose: bool = False, extra=()) -> str:
             print(" ".join(cmd))
         subprocess.run(cmd, check=True)
         objs.append(obj)
-    tmp = LIB + ".tmp"
+    tmp = lib_path + ".tmp"
     cmd = [nvcc, *ARCH, "-shared", "-o", tmp, *objs, "-cudart", "static"]
     if verbose:
         print(" ".join(cmd))
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib_path)
+    return lib_path
 
 
 if __name__ == "__main__":

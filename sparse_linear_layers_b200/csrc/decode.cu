@@ -7,116 +7,186 @@
 //
 // Layout: a row of packed weights is K/4 bytes = CPR chunks of CW 32-bit words
 // (16 CW weights; CW = 4 when K % 64 == 0 so rows are 16-byte aligned, else
-// CW = 1).  L lanes share a row (32/L rows per warp); lane li of a row takes
-// chunks li, li+L, ...  Each chunk is one streaming load.
-// Activations (already quantised, interleaved in 16-element blocks) sit in
-// shared memory as xs[t][word][chunk] 16-byte units, so the L lanes of a row
-// read consecutive units (no bank conflicts) and rows of one warp read the
-// same units (broadcast).
+// CW = 1).  L lanes share a row (32/L rows per warp, one row group per warp);
+// lane li takes chunks li, li + L, ... in batches of NB chunks whose loads are
+// all in flight together.
+//
+// The kernel is a programmatic dependent launch: at entry it lets the next
+// kernel on the stream start, and before waiting for its own predecessor it
+// only prefetches its weights into L2 (a non-binding prefetch, correct whatever
+// the predecessor writes), so consecutive layers stream weights while the
+// previous one finishes.  After the wait it quantises the activations itself
+// (per-token absmax over x, then int8 into shared memory, interleaved in
+// 16-element blocks in the order of expand_codes() and stored word-major: the
+// 16-byte unit of block 4c + w at position w * CPR + c, so the lanes of a row
+// read consecutive units).
 //
 // Arithmetic per 32-bit weight word (16 weights): for j = 0..3 the masks
 // w & (0x01010101 << 2j) and w & (0x02020202 << 2j) pick the +1 and -1 codes
-// of weights 4b + j (scaled by 4^j and 2*4^j); one unsigned-by-signed dp4a each
-// against the interleaved activation word j accumulates them.  The scales are
-// removed exactly (every partial is a multiple of its power of two) before the
-// L-lane shuffle reduction.
+// of weights 4b + j (scaled by 4^j and 2 * 4^j); one unsigned-by-signed dp4a
+// each against interleaved activation word j accumulates them.  The scales
+// are removed exactly (every partial is a multiple of its power of two)
+// before the L-lane shuffle reduction.
 #include "sbl_common.cuh"
 
 namespace sbl {
 
-constexpr int kDecodeThreads = 256;
+constexpr int kDecodeThreads = 512;
+constexpr int kDecodeWarps = kDecodeThreads / 32;
+constexpr int kDecodeBatch = 4;  // chunks per lane in flight
+
+template <int CW>
+__device__ __forceinline__ void load_chunk_words(const uint8_t* prow, int c, uint32_t (&w)[CW]) {
+    if constexpr (CW == 4) {
+        const uint4 v = ldg_stream(prow + 16 * c);
+        w[0] = v.x;
+        w[1 % CW] = v.y;
+        w[2 % CW] = v.z;
+        w[3 % CW] = v.w;
+    } else {
+        w[0] = __ldg(reinterpret_cast<const unsigned int*>(prow) + c);
+    }
+}
 
 template <int L, int TT, int CW>
 __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const uint8_t* __restrict__ packed,
                                                                 const float* __restrict__ row_scale, long long O,
-                                                                int K, const int8_t* __restrict__ xperm,
-                                                                const float* __restrict__ s_tok, long long T,
+                                                                int K, const uint16_t* __restrict__ x, long long T,
                                                                 long long t0, void* __restrict__ y, int y_bf16,
-                                                                int32_t* __restrict__ acc_out) {
-    extern __shared__ uint4 xs[];
+                                                                int32_t* __restrict__ acc_out, unsigned* status) {
+    extern __shared__ uint4 xs[];  // TT x K/16 units of quantised activations (decode layout)
+    __shared__ uint32_t red[kDecodeWarps][TT];
+    __shared__ float s_sh[TT];
+    asm volatile("griddepcontrol.launch_dependents;");
+    constexpr int RW = 32 / L;
+    constexpr int NB = kDecodeBatch;
     const int CPR = K / (16 * CW);
-    const int units = TT * CW * CPR;
-    for (int i = threadIdx.x; i < units; i += blockDim.x) {
-        const int t = i / (CW * CPR);
-        const int r = i - t * CW * CPR;
-        const int c = r / CW, w = r % CW;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (t0 + t < T) v = ldg_nc(xperm + (t0 + t) * K + 16 * (CW * c + w));
-        xs[(t * CW + w) * CPR + c] = v;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int sub = lane / L, li = lane % L;
+    const long long g = static_cast<long long>(blockIdx.x) * kDecodeWarps + warp;
+    const long long row = g * RW + sub;
+    const bool valid = row < O;
+    const uint8_t* prow = packed + (valid ? row : 0) * (K >> 2);
+
+    // Before the dependency wait: warm L2 with this lane's first batch of weights.
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        const int c = li + b * L;
+        if (valid && c < CPR) asm volatile("prefetch.global.L2 [%0];" ::"l"(prow + 4 * CW * c));
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    uint32_t wb[NB][CW];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        const int c = li + b * L;
+        if (valid && c < CPR) load_chunk_words<CW>(prow, c, wb[b]);
+        else
+#pragma unroll
+            for (int w = 0; w < CW; ++w) wb[b][w] = 0u;
+    }
+
+    // Quantise this pass's tokens: per-token absmax, then int8 into shared memory.
+    const int nvec = K >> 3;
+    const int nblk = K >> 4;
+#pragma unroll
+    for (int t = 0; t < TT; ++t) {
+        const long long tt = t0 + t < T ? t0 + t : T - 1;
+        const uint4* xr = reinterpret_cast<const uint4*>(x + tt * K);
+        uint32_t mx = 0;
+        for (int v = threadIdx.x; v < nvec; v += kDecodeThreads) mx = absmax8(ldg_nc(xr + v), mx);
+        mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+        if (lane == 0) red[warp][t] = mx;
+    }
+    __syncthreads();
+    if (threadIdx.x < TT) {
+        uint32_t mx = 0;
+#pragma unroll
+        for (int w = 0; w < kDecodeWarps; ++w) mx = max(mx, red[w][threadIdx.x]);
+        if (mx >= 0x7F80u && blockIdx.x == 0) raise_status(status, kStatusNonfinite);
+        s_sh[threadIdx.x] = __fdiv_rn(127.0f, fmaxf(__uint_as_float(mx << 16), 1e-5f));
+    }
+    __syncthreads();
+#pragma unroll
+    for (int t = 0; t < TT; ++t) {
+        const long long tt = t0 + t < T ? t0 + t : T - 1;
+        const uint4* xr = reinterpret_cast<const uint4*>(x + tt * K);
+        const float st = s_sh[t];
+        for (int b = threadIdx.x; b < nblk; b += kDecodeThreads) {
+            const int pos = CW == 4 ? (b & 3) * CPR + (b >> 2) : b;
+            xs[t * nblk + pos] = quant_block16<true>(ldg_nc(xr + 2 * b), ldg_nc(xr + 2 * b + 1), st);
+        }
     }
     __syncthreads();
 
-    constexpr int RW = 32 / L;
-    const int lane = threadIdx.x & 31;
-    const int sub = lane / L, li = lane % L;
-    const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-    const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
-    const long long ngroups = (O + RW - 1) / RW;
+    int alo[TT][4], ahi[TT][4];
+#pragma unroll
+    for (int t = 0; t < TT; ++t)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) alo[t][j] = ahi[t][j] = 0;
 
-    for (long long g = gw; g < ngroups; g += nw) {
-        const long long row = g * RW + sub;
-        const bool valid = row < O;
-        int alo[TT][4], ahi[TT][4];
+    for (int c0 = li; c0 < CPR; c0 += NB * L) {
 #pragma unroll
-        for (int t = 0; t < TT; ++t)
+        for (int b = 0; b < NB; ++b) {
+            const int c = c0 + b * L;
+            if (c >= CPR) break;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) alo[t][j] = ahi[t][j] = 0;
-        if (valid) {
-            const uint8_t* prow = packed + row * (K >> 2);
-#pragma unroll 2
-            for (int c = li; c < CPR; c += L) {
-                uint32_t ww[CW];
-                if constexpr (CW == 4) {
-                    const uint4 wv = ldg_stream(prow + 16 * c);
-                    ww[0] = wv.x; ww[1 % CW] = wv.y; ww[2 % CW] = wv.z; ww[3 % CW] = wv.w;
-                } else {
-                    ww[0] = __ldg(reinterpret_cast<const unsigned int*>(prow) + c);
+            for (int w = 0; w < CW; ++w) {
+                const uint32_t word = wb[b][w];
+                uint32_t mlo[4], mhi[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    mlo[j] = word & (0x01010101u << (2 * j));
+                    mhi[j] = word & (0x02020202u << (2 * j));
                 }
 #pragma unroll
-                for (int w = 0; w < CW; ++w) {
-                    uint32_t mlo[4], mhi[4];
+                for (int t = 0; t < TT; ++t) {
+                    const uint4 xv = xs[t * nblk + w * CPR + c];
+                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        mlo[j] = ww[w] & (0x01010101u << (2 * j));
-                        mhi[j] = ww[w] & (0x02020202u << (2 * j));
-                    }
-#pragma unroll
-                    for (int t = 0; t < TT; ++t) {
-                        const uint4 xv = xs[(t * CW + w) * CPR + c];
-                        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            alo[t][j] = dp4a_us(mlo[j], xw[j], alo[t][j]);
-                            ahi[t][j] = dp4a_us(mhi[j], xw[j], ahi[t][j]);
-                        }
+                        alo[t][j] = dp4a_us(mlo[j], xw[j], alo[t][j]);
+                        ahi[t][j] = dp4a_us(mhi[j], xw[j], ahi[t][j]);
                     }
                 }
             }
         }
-        int acc[TT];
+        const int cn = c0 + NB * L;
+        if (cn < CPR) {
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+                const int c = cn + b * L;
+                if (valid && c < CPR) load_chunk_words<CW>(prow, c, wb[b]);
+                else
+#pragma unroll
+                    for (int w = 0; w < CW; ++w) wb[b][w] = 0u;
+            }
+        }
+    }
+
+    int acc[TT];
+#pragma unroll
+    for (int t = 0; t < TT; ++t) {
+        int a = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) a += (alo[t][j] >> (2 * j)) - (ahi[t][j] >> (2 * j + 1));
+#pragma unroll
+        for (int off = L / 2; off >= 1; off >>= 1) a += __shfl_xor_sync(0xFFFFFFFFu, a, off);
+        acc[t] = a;
+    }
+    if (valid && li == 0) {
+        const float sc = row_scale[row];
 #pragma unroll
         for (int t = 0; t < TT; ++t) {
-            int a = 0;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) a += (alo[t][j] >> (2 * j)) - (ahi[t][j] >> (2 * j + 1));
-#pragma unroll
-            for (int off = L / 2; off >= 1; off >>= 1) a += __shfl_xor_sync(0xFFFFFFFFu, a, off);
-            acc[t] = a;
-        }
-        if (valid && li == 0) {
-            const float sc = row_scale[row];
-#pragma unroll
-            for (int t = 0; t < TT; ++t) {
-                const long long tt = t0 + t;
-                if (tt < T) {
-                    const float v = __fdiv_rn(__fmul_rn(static_cast<float>(acc[t]), sc), s_tok[tt]);
-                    if (y_bf16)
-                        reinterpret_cast<__nv_bfloat16_raw*>(y)[tt * O + row] =
-                            static_cast<__nv_bfloat16_raw>(__float2bfloat16_rn(v));
-                    else
-                        reinterpret_cast<float*>(y)[tt * O + row] = v;
-                    if (acc_out) acc_out[tt * O + row] = acc[t];
-                }
+            const long long tt = t0 + t;
+            if (tt < T) {
+                const float v = __fdiv_rn(__fmul_rn(static_cast<float>(acc[t]), sc), s_sh[t]);
+                if (y_bf16)
+                    reinterpret_cast<__nv_bfloat16_raw*>(y)[tt * O + row] =
+                        static_cast<__nv_bfloat16_raw>(__float2bfloat16_rn(v));
+                else
+                    reinterpret_cast<float*>(y)[tt * O + row] = v;
+                if (acc_out) acc_out[tt * O + row] = acc[t];
             }
         }
     }
@@ -142,54 +212,62 @@ static int choose_lanes(long long O, int cpr, int num_sms) {
 
 template <int L, int TT, int CW>
 static cudaError_t launch_decode_lt(const uint8_t* packed, const float* row_scale, long long O, int K,
-                                    const int8_t* xperm, const float* s_tok, long long T, long long t0, void* y,
-                                    int y_bf16, int32_t* acc_out, int num_sms, cudaStream_t stream) {
+                                    const uint16_t* x, long long T, long long t0, void* y, int y_bf16,
+                                    int32_t* acc_out, unsigned* status, cudaStream_t stream) {
+    constexpr int RW = 32 / L;
+    const long long groups = (O + RW - 1) / RW;
+    const long long blocks = (groups + kDecodeWarps - 1) / kDecodeWarps;
     const size_t smem = static_cast<size_t>(TT) * K;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(decode_kernel<L, TT, CW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return e;
     }
-    constexpr int RW = 32 / L;
-    const long long groups = (O + RW - 1) / RW;
-    const long long warps_per_block = kDecodeThreads / 32;
-    long long blocks = (groups + warps_per_block - 1) / warps_per_block;
-    const long long cap = static_cast<long long>(num_sms) * 4;
-    if (blocks > cap) blocks = cap;
-    if (blocks < 1) blocks = 1;
-    decode_kernel<L, TT, CW><<<static_cast<unsigned>(blocks), kDecodeThreads, smem, stream>>>(
-        packed, row_scale, O, K, xperm, s_tok, T, t0, y, y_bf16, acc_out);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+    cfg.blockDim = dim3(kDecodeThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_kernel<L, TT, CW>, packed, row_scale, O, K, x, T, t0, y, y_bf16, acc_out,
+                              status);
 }
 
 template <int TT, int CW>
 static cudaError_t launch_decode_t(int L, const uint8_t* packed, const float* row_scale, long long O, int K,
-                                   const int8_t* xperm, const float* s_tok, long long T, long long t0, void* y,
-                                   int y_bf16, int32_t* acc_out, int num_sms, cudaStream_t stream) {
+                                   const uint16_t* x, long long T, long long t0, void* y, int y_bf16,
+                                   int32_t* acc_out, unsigned* status, cudaStream_t stream) {
+#define SBL_DECODE_CASE(LV) \
+    case LV: return launch_decode_lt<LV, TT, CW>(packed, row_scale, O, K, x, T, t0, y, y_bf16, acc_out, status, stream);
     switch (L) {
-        case 32: return launch_decode_lt<32, TT, CW>(packed, row_scale, O, K, xperm, s_tok, T, t0, y, y_bf16, acc_out, num_sms, stream);
-        case 16: return launch_decode_lt<16, TT, CW>(packed, row_scale, O, K, xperm, s_tok, T, t0, y, y_bf16, acc_out, num_sms, stream);
-        case 8: return launch_decode_lt<8, TT, CW>(packed, row_scale, O, K, xperm, s_tok, T, t0, y, y_bf16, acc_out, num_sms, stream);
-        case 4: return launch_decode_lt<4, TT, CW>(packed, row_scale, O, K, xperm, s_tok, T, t0, y, y_bf16, acc_out, num_sms, stream);
-        case 2: return launch_decode_lt<2, TT, CW>(packed, row_scale, O, K, xperm, s_tok, T, t0, y, y_bf16, acc_out, num_sms, stream);
-        default: return launch_decode_lt<1, TT, CW>(packed, row_scale, O, K, xperm, s_tok, T, t0, y, y_bf16, acc_out, num_sms, stream);
+        SBL_DECODE_CASE(32)
+        SBL_DECODE_CASE(16)
+        SBL_DECODE_CASE(8)
+        SBL_DECODE_CASE(4)
+        SBL_DECODE_CASE(2)
+        default: return launch_decode_lt<1, TT, CW>(packed, row_scale, O, K, x, T, t0, y, y_bf16, acc_out, status, stream);
     }
+#undef SBL_DECODE_CASE
 }
 
 template <int TT>
 static cudaError_t launch_decode_cw(int L, bool wide, const uint8_t* packed, const float* row_scale, long long O,
-                                    int K, const int8_t* xperm, const float* s_tok, long long T, long long t0,
-                                    void* y, int y_bf16, int32_t* acc_out, int num_sms, cudaStream_t stream) {
+                                    int K, const uint16_t* x, long long T, long long t0, void* y, int y_bf16,
+                                    int32_t* acc_out, unsigned* status, cudaStream_t stream) {
     if (wide)
-        return launch_decode_t<TT, 4>(L, packed, row_scale, O, K, xperm, s_tok, T, t0, y, y_bf16, acc_out, num_sms, stream);
-    return launch_decode_t<TT, 1>(L, packed, row_scale, O, K, xperm, s_tok, T, t0, y, y_bf16, acc_out, num_sms, stream);
+        return launch_decode_t<TT, 4>(L, packed, row_scale, O, K, x, T, t0, y, y_bf16, acc_out, status, stream);
+    return launch_decode_t<TT, 1>(L, packed, row_scale, O, K, x, T, t0, y, y_bf16, acc_out, status, stream);
 }
 
 // Decode for any T: passes of up to 8 tokens (later passes re-read the
-// weights, mostly from L2).  Needs K % 16 == 0.
+// weights, mostly from L2).  Needs K % 16 == 0 and TT * K bytes of shared memory.
 cudaError_t launch_decode(const uint8_t* packed, const float* row_scale, long long O, long long K,
-                          const int8_t* xperm, const float* s_tok, long long T, void* y, int y_bf16,
-                          int32_t* acc_out, int num_sms, cudaStream_t stream) {
+                          const uint16_t* x, long long T, void* y, int y_bf16, int32_t* acc_out, unsigned* status,
+                          int num_sms, cudaStream_t stream) {
     const int Ki = static_cast<int>(K);
     const bool wide = (Ki % 64) == 0;
     const int cpr = wide ? Ki / 64 : Ki / 16;
@@ -197,10 +275,10 @@ cudaError_t launch_decode(const uint8_t* packed, const float* row_scale, long lo
     for (long long t0 = 0; t0 < T; t0 += 8) {
         const long long rem = T - t0;
         cudaError_t e;
-        if (rem > 4) e = launch_decode_cw<8>(L, wide, packed, row_scale, O, Ki, xperm, s_tok, T, t0, y, y_bf16, acc_out, num_sms, stream);
-        else if (rem > 2) e = launch_decode_cw<4>(L, wide, packed, row_scale, O, Ki, xperm, s_tok, T, t0, y, y_bf16, acc_out, num_sms, stream);
-        else if (rem == 2) e = launch_decode_cw<2>(L, wide, packed, row_scale, O, Ki, xperm, s_tok, T, t0, y, y_bf16, acc_out, num_sms, stream);
-        else e = launch_decode_cw<1>(L, wide, packed, row_scale, O, Ki, xperm, s_tok, T, t0, y, y_bf16, acc_out, num_sms, stream);
+        if (rem > 4) e = launch_decode_cw<8>(L, wide, packed, row_scale, O, Ki, x, T, t0, y, y_bf16, acc_out, status, stream);
+        else if (rem > 2) e = launch_decode_cw<4>(L, wide, packed, row_scale, O, Ki, x, T, t0, y, y_bf16, acc_out, status, stream);
+        else if (rem == 2) e = launch_decode_cw<2>(L, wide, packed, row_scale, O, Ki, x, T, t0, y, y_bf16, acc_out, status, stream);
+        else e = launch_decode_cw<1>(L, wide, packed, row_scale, O, Ki, x, T, t0, y, y_bf16, acc_out, status, stream);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

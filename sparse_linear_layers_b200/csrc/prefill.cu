@@ -5,13 +5,20 @@
 // ("Mathematical Formulation of Sparse-BitLinear"), which for many tokens is a
 // dense int8 matrix product.  Persistent, warp-specialised, one CTA per SM:
 //
-//   warps 0-3          epilogue: tcgen05.ld of the accumulator (TMEM lane = token),
-//                      dequantise, 16-byte stores of y rows (contiguous in o)
+//   warps 0-3          epilogue: warp w owns TMEM lanes 32w .. 32w + 31 (32 tokens);
+//                      pipelined tcgen05.ld, dequantise, per-warp 128B-swizzled
+//                      staging boxes, TMA stores
 //   warps 4..4+BN/32-1 weight expansion: each thread owns one output row o of
-//                      the B tile, loads its 2-bit codes for the k-block and
-//                      writes the int8 row into the 128B-swizzled K-major tile
-//   next warp          TMA producer of the activation tile (A, 128 tokens x 128 k)
+//                      the B tile, reads its 2-bit codes for the k-block from
+//                      shared memory and writes the int8 row into the
+//                      128B-swizzled K-major tile
+//   next warp          TMA producer: activation tile (A, 128 tokens x 128 k) and
+//                      the 2-bit code tile (BN rows x 32 bytes) of each stage
 //   last warp          TMEM allocator and single-thread MMA issuer
+//
+// The kernel is launched as a programmatic dependent of the activation
+// quantisation: set-up (barriers, tensor memory) overlaps its tail, and every
+// role waits on griddepcontrol before touching its outputs.
 //
 // Tile: 128 tokens x BN output rows x 128 k per stage, 4 stages, two TMEM
 // accumulator buffers so the epilogue of one tile overlaps the MMAs of the next.
@@ -23,35 +30,56 @@
 // memory and exits.
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "sbl_common.cuh"
 
 namespace sbl {
 
+#ifdef SBL_TRACE
+// Debug builds only: clock64 stamps of pipeline events in CTA 0 (event e,
+// iteration i -> g_trace[e * 256 + i]).
+__device__ unsigned long long* g_trace;
+#define SBL_TR(e, i)                                                          \
+    do {                                                                      \
+        if (trace_buf && (i) < 256) trace_buf[(e) * 256 + (i)] = clock64();   \
+    } while (0)
+#else
+#define SBL_TR(e, i) \
+    do {             \
+    } while (0)
+#endif
+
 namespace pf {
 constexpr int BM = 128;       // tokens per tile  (MMA M, TMEM lanes)
 constexpr int BK = 128;       // k per stage      (bytes of int8)
-constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK;
 constexpr int EPI_WARPS = 4;
+constexpr int Y_BYTES = 32 * 128;  // one warp's output staging box: 32 tokens x 128 bytes
 }  // namespace pf
 
 template <int BN>
 struct PrefillCfg {
     static constexpr int B_BYTES = BN * pf::BK;
+    static constexpr int P_BYTES = BN * pf::BK / 4;  // 2-bit codes of the B tile
     static constexpr int DEC_WARPS = BN / 32;
     static constexpr int WARP_TMA = pf::EPI_WARPS + DEC_WARPS;
     static constexpr int WARP_MMA = WARP_TMA + 1;
     static constexpr int THREADS = (WARP_MMA + 1) * 32;
     static constexpr int TMEM_COLS = 2 * BN;  // two accumulator buffers
+    static constexpr int STAGES = BN == 256 ? 3 : 4;
 };
 
 template <int BN>
 struct PrefillSmem {
-    uint8_t a[pf::STAGES][pf::A_BYTES];            // 1024-byte aligned tiles
-    uint8_t b[pf::STAGES][PrefillCfg<BN>::B_BYTES];
-    uint64_t full_tma[pf::STAGES];
-    uint64_t full_dec[pf::STAGES];
-    uint64_t empty[pf::STAGES];
+    uint8_t a[PrefillCfg<BN>::STAGES][pf::A_BYTES];            // 1024-byte aligned tiles
+    uint8_t b[PrefillCfg<BN>::STAGES][PrefillCfg<BN>::B_BYTES];
+    uint8_t p[PrefillCfg<BN>::STAGES][PrefillCfg<BN>::P_BYTES];
+    uint8_t ystage[pf::EPI_WARPS][1][pf::Y_BYTES];           // per-warp output transpose box
+    float wscale[pf::EPI_WARPS][BN];                          // per-warp copy of the tile's row scales
+    uint64_t full_tma[PrefillCfg<BN>::STAGES];
+    uint64_t full_dec[PrefillCfg<BN>::STAGES];
+    uint64_t empty[PrefillCfg<BN>::STAGES];
     uint64_t tmem_full[2];
     uint64_t tmem_empty[2];
     uint64_t mma_done;
@@ -63,6 +91,8 @@ template <int BN>
 constexpr size_t prefill_smem_bytes() {
     return sizeof(PrefillSmem<BN>) + 1024;
 }
+static_assert(prefill_smem_bytes<256>() <= 232448, "prefill tile does not fit in shared memory");
+static_assert(prefill_smem_bytes<128>() <= 232448, "prefill tile does not fit in shared memory");
 
 // UMMA shared-memory descriptor: K-major, 128-byte swizzle, 8-row groups 1024 B apart.
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
@@ -87,6 +117,13 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
             dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
         : "memory");
+}
+
+// One lane polls the barrier, the warp follows (fewer pollers on shared memory).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag);
+    return __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
 }
 
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -118,28 +155,46 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
 __device__ __forceinline__ void st_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
     asm volatile("st.global.v4.b32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
 template <int BN>
 __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
-    prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __restrict__ packed,
-                   const float* __restrict__ row_scale, const float* __restrict__ s_tok, int T, int O, int K,
-                   void* __restrict__ y, int y_bf16, int32_t* __restrict__ acc_out, unsigned* status) {
+    prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                   int y_vec, const float* __restrict__ row_scale,
+                   const float* __restrict__ s_tok, int T, int O, int K, void* __restrict__ y, int y_bf16,
+                   int32_t* __restrict__ acc_out, unsigned* status) {
     using Cfg = PrefillCfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     auto* sm = reinterpret_cast<PrefillSmem<BN>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     volatile int* abort_flag = &sm->abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#ifdef SBL_TRACE
+    unsigned long long* const trace_buf = blockIdx.x == 0 ? g_trace : nullptr;
+#endif
     const int MT = (T + pf::BM - 1) / pf::BM;
     const int NT = (O + BN - 1) / BN;
     const int tiles = MT * NT;
     const int KB = (K + pf::BK - 1) / pf::BK;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < pf::STAGES; ++s) {
+        for (int s = 0; s < Cfg::STAGES; ++s) {
             mbar_init(&sm->full_tma[s], 1);
             mbar_init(&sm->full_dec[s], Cfg::DEC_WARPS * 32);
             mbar_init(&sm->empty[s], 1);
@@ -162,6 +217,8 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = sm->tmem_base;
+    // inputs of this call (quantised activations) come from the preceding kernel
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     auto give_up = [&]() {
         if (!*abort_flag) {
@@ -172,109 +229,172 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
 
     if (warp < pf::EPI_WARPS) {
         // ------------------------------------------------------------ epilogue
-        const int row = threadIdx.x;  // TMEM lane == token within the tile
-        int tc = 0;
-        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
-            const int mt = tile % MT, nt = tile / MT;
-            const int b = tc & 1;
-            const uint32_t aph = (tc >> 1) & 1;
-            // warp-uniform decision: tcgen05.ld below is a .sync.aligned warp instruction
-            const bool ready = __all_sync(0xFFFFFFFFu, mbar_wait(&sm->tmem_full[b], aph, abort_flag));
-            if (!ready) { give_up(); break; }
-            tc_fence_after();
-            const int t = mt * pf::BM + row;
-            const bool tvalid = t < T;
-            const float inv_s = tvalid ? __frcp_rn(s_tok[t]) : 0.f;
-            for (int q = 0; q < BN / 32; ++q) {
-                uint32_t r[32];
-                tmem_ld32(tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + b * BN + q * 32, r);
-                if (q == BN / 32 - 1) {
-                    tc_fence_before();
-                    mbar_arrive(&sm->tmem_empty[b]);
+        // Warp w owns TMEM lanes 32w .. 32w + 31 (32 tokens of the tile).  Per
+        // tile it first copies the tile's row scales into its own shared-memory
+        // slice (before waiting for the accumulator), then walks the 32-column
+        // TMEM slices with the next slice's load in flight while the current one
+        // is dequantised.  Every 128 output bytes per token (a "round": 32 fp32
+        // or 64 bf16 columns) go into one of the warp's two 128B-swizzled
+        // 32-row staging boxes and out by one TMA store, which writes whole
+        // lines and clips the ragged edges.  Nothing synchronises beyond the warp.
+        auto run = [&](auto bf16_tag) {
+            constexpr bool BF = decltype(bf16_tag)::value;
+            constexpr int SPR = BF ? 2 : 1;          // 32-column slices per round
+            constexpr int NSL = BN / 32;             // slices per tile
+            const int row = warp * 32 + lane;        // TMEM lane == token within the tile
+            const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+            float* const wsc = sm->wscale[warp];
+            int tc = 0;
+            int ep_round = 0;
+            for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
+                const int mt = tile % MT, nt = tile / MT;
+                const int b = tc & 1;
+                const uint32_t aph = (tc >> 1) & 1;
+                __syncwarp();
+#pragma unroll
+                for (int k = 0; k < NSL; ++k) {
+                    const int o = nt * BN + 32 * k + lane;
+                    wsc[32 * k + lane] = o < O ? __ldg(row_scale + o) : 0.f;
                 }
-                const int o0 = nt * BN + q * 32;
-                if (!tvalid || o0 >= O) continue;
-                const long long base = static_cast<long long>(t) * O + o0;
-                const bool full = (o0 + 32 <= O) && ((O & 3) == 0);
-                float v[32];
-#pragma unroll
-                for (int i = 0; i < 32; i += 4) {
-                    float4 sc = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (full) sc = __ldg(reinterpret_cast<const float4*>(row_scale + o0 + i));
-                    else {
-                        if (o0 + i + 0 < O) sc.x = row_scale[o0 + i + 0];
-                        if (o0 + i + 1 < O) sc.y = row_scale[o0 + i + 1];
-                        if (o0 + i + 2 < O) sc.z = row_scale[o0 + i + 2];
-                        if (o0 + i + 3 < O) sc.w = row_scale[o0 + i + 3];
-                    }
-                    v[i + 0] = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int>(r[i + 0])), sc.x), inv_s);
-                    v[i + 1] = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int>(r[i + 1])), sc.y), inv_s);
-                    v[i + 2] = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int>(r[i + 2])), sc.z), inv_s);
-                    v[i + 3] = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int>(r[i + 3])), sc.w), inv_s);
-                }
-                if (full) {
-                    if (y_bf16) {
-                        uint32_t p[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-                            p[i] = *reinterpret_cast<const uint32_t*>(&h);
-                        }
-                        uint16_t* yp = reinterpret_cast<uint16_t*>(y) + base;
-#pragma unroll
-                        for (int i = 0; i < 16; i += 4) st_v4(yp + 2 * i, p[i], p[i + 1], p[i + 2], p[i + 3]);
+                __syncwarp();
+                // warp-uniform decision: tcgen05.ld below is a .sync.aligned warp instruction
+                if (!warp_wait(&sm->tmem_full[b], aph, abort_flag)) { give_up(); break; }
+                if (threadIdx.x == 0) SBL_TR(6, tc);
+                tc_fence_after();
+                const int t = mt * pf::BM + row;
+                const bool tvalid = t < T;
+                const float inv_s = tvalid ? __frcp_rn(s_tok[t]) : 0.f;
+                const uint32_t tbase = tmem_base + lane_addr + b * BN;
+                uint32_t ra[32], rb[32];
+                uint32_t q[32];
+                // one 32-column slice k (H = k % SPR): convert `cur` while slice k + 1 loads into `nxt`
+                auto slice = [&](auto h_tag, const int k, uint32_t (&cur)[32], uint32_t (&nxt)[32]) {
+                    constexpr int H = decltype(h_tag)::value;
+                    const bool more = k + 1 < NSL;
+                    if (more) {
+                        tmem_ld32_nowait(tbase + 32 * (k + 1), nxt);
                     } else {
-                        float* yp = reinterpret_cast<float*>(y) + base;
-#pragma unroll
-                        for (int i = 0; i < 32; i += 4)
-                            st_v4(yp + i, __float_as_uint(v[i]), __float_as_uint(v[i + 1]), __float_as_uint(v[i + 2]),
-                                  __float_as_uint(v[i + 3]));
+                        tc_fence_before();
+                        mbar_arrive(&sm->tmem_empty[b]);  // the accumulator buffer is free for the MMA
                     }
-                    if (acc_out) {
+                    if (H == 0 && threadIdx.x == 0) SBL_TR(10, ep_round);
+                    const float* sc = wsc + 32 * k;
 #pragma unroll
-                        for (int i = 0; i < 32; i += 4) st_v4(acc_out + base + i, r[i], r[i + 1], r[i + 2], r[i + 3]);
+                    for (int i = 0; i < 32; i += 4) {
+                        const float4 s4 = *reinterpret_cast<const float4*>(sc + i);
+                        const float f0 = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int>(cur[i + 0])), s4.x), inv_s);
+                        const float f1 = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int>(cur[i + 1])), s4.y), inv_s);
+                        const float f2 = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int>(cur[i + 2])), s4.z), inv_s);
+                        const float f3 = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int>(cur[i + 3])), s4.w), inv_s);
+                        if (BF) {
+                            const __nv_bfloat162 h01 = __floats2bfloat162_rn(f0, f1);
+                            const __nv_bfloat162 h23 = __floats2bfloat162_rn(f2, f3);
+                            q[16 * H + i / 2] = *reinterpret_cast<const uint32_t*>(&h01);
+                            q[16 * H + i / 2 + 1] = *reinterpret_cast<const uint32_t*>(&h23);
+                        } else {
+                            q[i] = __float_as_uint(f0);
+                            q[i + 1] = __float_as_uint(f1);
+                            q[i + 2] = __float_as_uint(f2);
+                            q[i + 3] = __float_as_uint(f3);
+                        }
                     }
-                } else {
+                    if (acc_out && tvalid) {
+                        const long long base = static_cast<long long>(t) * O + nt * BN + 32 * k;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        if (o0 + i >= O) continue;
-                        if (y_bf16)
-                            reinterpret_cast<__nv_bfloat16_raw*>(y)[base + i] =
-                                static_cast<__nv_bfloat16_raw>(__float2bfloat16_rn(v[i]));
-                        else
-                            reinterpret_cast<float*>(y)[base + i] = v[i];
-                        if (acc_out) acc_out[base + i] = static_cast<int>(r[i]);
+                        for (int i = 0; i < 32; ++i)
+                            if (nt * BN + 32 * k + i < O) acc_out[base + i] = static_cast<int>(cur[i]);
+                    }
+                    if (H == SPR - 1) {
+                        const int o0 = nt * BN + 32 * (k - H);
+                        if (threadIdx.x == 0) SBL_TR(11, ep_round);
+                        if (y_vec) {
+                            // transpose through the warp's swizzled box: written one token row
+                            // per lane, read back so each store instruction covers 4 whole
+                            // 128-byte lines of y
+                            uint8_t* const box = sm->ystage[warp][0];
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) {
+                                const uint32_t a = smem_u32(box + lane * 128 + ((c ^ (lane & 7)) << 4));
+                                asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(q[4 * c]),
+                                             "r"(q[4 * c + 1]), "r"(q[4 * c + 2]), "r"(q[4 * c + 3])
+                                             : "memory");
+                            }
+                            __syncwarp();
+                            if (threadIdx.x == 0) SBL_TR(12, ep_round);
+                            constexpr int PER_CHUNK = BF ? 8 : 4;  // outputs per 16-byte chunk
+                            const int cch = lane & 7;
+                            const int col = o0 + cch * PER_CHUNK;
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const int rr = 4 * i + (lane >> 3);
+                                const uint32_t a = smem_u32(box + rr * 128 + ((cch ^ (rr & 7)) << 4));
+                                uint32_t v0, v1, v2, v3;
+                                asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+                                             : "=r"(v0), "=r"(v1), "=r"(v2), "=r"(v3)
+                                             : "r"(a));
+                                const int tok = mt * pf::BM + warp * 32 + rr;
+                                if (tok < T && col < O) {
+                                    uint8_t* dst = static_cast<uint8_t*>(y) +
+                                                   (static_cast<long long>(tok) * O + col) * (BF ? 2 : 4);
+                                    st_v4(dst, v0, v1, v2, v3);
+                                }
+                            }
+                            __syncwarp();
+                            if (threadIdx.x == 0) SBL_TR(13, ep_round);
+                        } else if (tvalid) {
+                            // direct stores: shapes whose row pitch is not a multiple of 16 bytes
+                            const long long base = static_cast<long long>(t) * O + o0;
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) {
+                                if (BF) {
+                                    if (o0 + 2 * i < O)
+                                        reinterpret_cast<uint16_t*>(y)[base + 2 * i] = static_cast<uint16_t>(q[i] & 0xFFFFu);
+                                    if (o0 + 2 * i + 1 < O)
+                                        reinterpret_cast<uint16_t*>(y)[base + 2 * i + 1] = static_cast<uint16_t>(q[i] >> 16);
+                                } else if (o0 + i < O) {
+                                    reinterpret_cast<uint32_t*>(y)[base + i] = q[i];
+                                }
+                            }
+                        }
+                        ++ep_round;
+                    }
+                    if (more) tmem_ld_wait();
+                };
+                tmem_ld32_nowait(tbase, ra);
+                tmem_ld_wait();
+                for (int k = 0; k < NSL; k += 2) {
+                    if (SPR == 2) {
+                        slice(std::integral_constant<int, 0>{}, k, ra, rb);
+                        slice(std::integral_constant<int, 1>{}, k + 1, rb, ra);
+                    } else {
+                        slice(std::integral_constant<int, 0>{}, k, ra, rb);
+                        slice(std::integral_constant<int, 0>{}, k + 1, rb, ra);
                     }
                 }
+                if (threadIdx.x == 0) SBL_TR(7, tc);
             }
-        }
+        };
+        if (y_bf16) run(std::true_type{});
+        else run(std::false_type{});
     } else if (warp < Cfg::WARP_TMA) {
         // ------------------------------------------------------------ weight expansion
         const int r = threadIdx.x - pf::EPI_WARPS * 32;  // row of the B tile
-        const int rowbytes = K >> 2;
         uint32_t it = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-            const int nt = tile / MT;
-            const int o = nt * BN + r;
-            const bool valid = o < O;
-            const uint8_t* prow = packed + static_cast<long long>(o) * rowbytes;
-            uint4 p0 = make_uint4(0u, 0u, 0u, 0u), p1 = p0;
-            if (valid) {
-                p0 = ldg_nc(prow);
-                if (64 < K) p1 = ldg_nc(prow + 16);
-            }
             for (int kb = 0; kb < KB; ++kb, ++it) {
-                // prefetch the next k-block's codes before waiting for the slot
-                uint4 n0 = make_uint4(0u, 0u, 0u, 0u), n1 = n0;
-                const int kn = (kb + 1) * pf::BK;
-                if (valid && kn < K) {
-                    n0 = ldg_nc(prow + (kn >> 2));
-                    if (kn + 64 < K) n1 = ldg_nc(prow + (kn >> 2) + 16);
-                }
-                const int s = it % pf::STAGES;
-                const uint32_t ph = (it / pf::STAGES) & 1;
-                if (!mbar_wait(&sm->empty[s], ph ^ 1, abort_flag)) { give_up(); ok = false; break; }
+                const int s = it % Cfg::STAGES;
+                const uint32_t ph = (it / Cfg::STAGES) & 1;
+                // the codes have landed, and the producer only issued them once the
+                // MMA had released this stage, so b[s] is free as well
+                if (!warp_wait(&sm->full_tma[s], ph, abort_flag)) { give_up(); ok = false; break; }
+                if (r == 0) SBL_TR(1, it);
+                // code tile rows are 32 bytes, 32B-swizzled by TMA: 16-byte half q of
+                // row r sits at half q ^ ((r >> 2) & 1)
+                const uint8_t* src = sm->p[s] + r * 32;
+                const int hs = (r >> 2) & 1;
+                const uint4 p0 = *reinterpret_cast<const uint4*>(src + (hs << 4));
+                const uint4 p1 = *reinterpret_cast<const uint4*>(src + ((hs ^ 1) << 4));
                 uint8_t* dst = sm->b[s] + r * 128;
                 const int sw = r & 7;
                 const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
@@ -289,8 +409,7 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
                 }
                 fence_proxy_async_smem();
                 mbar_arrive(&sm->full_dec[s]);
-                p0 = n0;
-                p1 = n1;
+                if (r == 0) SBL_TR(2, it);
             }
         }
     } else if (warp == Cfg::WARP_TMA) {
@@ -299,50 +418,62 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
             uint32_t it = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-                const int mt = tile % MT;
+                const int mt = tile % MT, nt = tile / MT;
                 for (int kb = 0; kb < KB; ++kb, ++it) {
-                    const int s = it % pf::STAGES;
-                    const uint32_t ph = (it / pf::STAGES) & 1;
+                    const int s = it % Cfg::STAGES;
+                    const uint32_t ph = (it / Cfg::STAGES) & 1;
                     if (!mbar_wait(&sm->empty[s], ph ^ 1, abort_flag)) { give_up(); ok = false; break; }
-                    mbar_arrive_expect_tx(&sm->full_tma[s], pf::A_BYTES);
+                    SBL_TR(0, it);
+                    mbar_arrive_expect_tx(&sm->full_tma[s], pf::A_BYTES + Cfg::P_BYTES);
                     tma_load_2d(smem_u32(sm->a[s]), &tmap_x, kb * pf::BK, mt * pf::BM, &sm->full_tma[s]);
+                    tma_load_2d(smem_u32(sm->p[s]), &tmap_w, kb * (pf::BK / 4), nt * BN, &sm->full_tma[s]);
                 }
             }
             // let every issued load land before the CTA can exit
-            const uint32_t first = it > pf::STAGES ? it - pf::STAGES : 0;
+            const uint32_t first = it > Cfg::STAGES ? it - Cfg::STAGES : 0;
             volatile int never = 0;
             for (uint32_t j = first; j < it; ++j)
-                if (!mbar_wait(&sm->full_tma[j % pf::STAGES], (j / pf::STAGES) & 1, &never)) give_up();
+                if (!mbar_wait(&sm->full_tma[j % Cfg::STAGES], (j / Cfg::STAGES) & 1, &never)) give_up();
         }
     } else {
         // ------------------------------------------------------------ MMA issuer
+        // One flat walk over (tile, k-block).  The barriers of step n + 1 are
+        // checked before step n is committed: an mbarrier operation issued right
+        // after tcgen05.commit waits for the committed MMAs to finish, which
+        // would leave the tensor pipe idle between stages.
         if (lane == 0) {
             const uint32_t idesc = i8_idesc<BN>();
-            uint32_t it = 0;
-            int tc = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++tc) {
-                const int b = tc & 1;
-                const uint32_t aph = (tc >> 1) & 1;
-                if (!mbar_wait(&sm->tmem_empty[b], aph ^ 1, abort_flag)) { give_up(); break; }
+            const int my_tiles = tiles > static_cast<int>(blockIdx.x)
+                                     ? (tiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
+                                     : 0;
+            const uint32_t total = static_cast<uint32_t>(my_tiles) * static_cast<uint32_t>(KB);
+            // wait for everything step n needs: accumulator buffer (first k-block of a tile) and stage data
+            auto ready = [&](uint32_t n) -> bool {
+                const uint32_t tcn = n / KB, kbn = n % KB;
+                if (kbn == 0 && !mbar_spin(&sm->tmem_empty[tcn & 1], ((tcn >> 1) & 1) ^ 1, abort_flag)) return false;
+                const uint32_t s = n % Cfg::STAGES, ph = (n / Cfg::STAGES) & 1;
+                if (!mbar_spin(&sm->full_tma[s], ph, abort_flag)) return false;
+                SBL_TR(3, n);
+                if (!mbar_spin(&sm->full_dec[s], ph, abort_flag)) return false;
+                SBL_TR(4, n);
+                return true;
+            };
+            bool ok = total == 0 || ready(0);
+            if (!ok) give_up();
+            for (uint32_t n = 0; n < total && ok; ++n) {
                 tc_fence_after();
-                const uint32_t d = tmem_base + b * BN;
-                for (int kb = 0; kb < KB; ++kb, ++it) {
-                    const int s = it % pf::STAGES;
-                    const uint32_t ph = (it / pf::STAGES) & 1;
-                    if (!mbar_wait(&sm->full_tma[s], ph, abort_flag) || !mbar_wait(&sm->full_dec[s], ph, abort_flag)) {
-                        give_up();
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t a0 = smem_u32(sm->a[s]), b0 = smem_u32(sm->b[s]);
+                const uint32_t tcn = n / KB, kbn = n % KB;
+                const uint32_t s = n % Cfg::STAGES;
+                const uint32_t d = tmem_base + (tcn & 1) * BN;
+                const uint32_t a0 = smem_u32(sm->a[s]), b0 = smem_u32(sm->b[s]);
 #pragma unroll
-                    for (int kk = 0; kk < pf::BK / 32; ++kk)
-                        tc_mma(d, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc, (kb | kk) != 0);
-                    tc_commit(&sm->empty[s]);
-                }
-                if (ok) tc_commit(&sm->tmem_full[b]);
+                for (int kk = 0; kk < pf::BK / 32; ++kk)
+                    tc_mma(d, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc, (kbn | kk) != 0);
+                SBL_TR(9, n);
+                if (n + 1 < total && !ready(n + 1)) { give_up(); ok = false; }
+                tc_commit(&sm->empty[s]);
+                if (kbn == static_cast<uint32_t>(KB) - 1) tc_commit(&sm->tmem_full[tcn & 1]);
+                SBL_TR(5, n);
             }
             // all MMAs must be complete before tensor memory is released
             tc_commit(&sm->mma_done);
@@ -383,15 +514,29 @@ static cudaError_t launch_prefill_bn(const int8_t* xperm, const float* s_tok, lo
                                      int32_t* acc_out, unsigned* status, int num_sms, cudaStream_t stream) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return cudaErrorNotSupported;
-    CUtensorMap map;
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(T)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(pf::BK), static_cast<cuuint32_t>(pf::BM)};
+    CUtensorMap map_x, map_w;
     const cuuint32_t estr[2] = {1, 1};
-    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(xperm), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return cudaErrorInvalidValue;
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(T)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+        const cuuint32_t box[2] = {static_cast<cuuint32_t>(pf::BK), static_cast<cuuint32_t>(pf::BM)};
+        if (enc(&map_x, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(xperm), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 4), static_cast<cuuint64_t>(O)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 4)};
+        const cuuint32_t box[2] = {static_cast<cuuint32_t>(pf::BK / 4), static_cast<cuuint32_t>(BN)};
+        if (enc(&map_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    // output rows go out as 16-byte vectors when the row pitch allows it
+    const int esize = y_bf16 ? 2 : 4;
+    const int y_vec = (static_cast<long long>(O) * esize) % 16 == 0 ? 1 : 0;
     constexpr size_t smem = prefill_smem_bytes<BN>();
     static bool attr_set[64] = {};
     int dev = 0;
@@ -404,23 +549,37 @@ static cudaError_t launch_prefill_bn(const int8_t* xperm, const float* s_tok, lo
     }
     const long long tiles = ((T + pf::BM - 1) / pf::BM) * ((O + BN - 1) / BN);
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
-    prefill_kernel<BN><<<grid, PrefillCfg<BN>::THREADS, smem, stream>>>(
-        map, packed, row_scale, s_tok, static_cast<int>(T), static_cast<int>(O), static_cast<int>(K), y, y_bf16,
-        acc_out, status);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(PrefillCfg<BN>::THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, prefill_kernel<BN>, map_x, map_w, y_vec, row_scale, s_tok, static_cast<int>(T),
+                              static_cast<int>(O), static_cast<int>(K), y, y_bf16, acc_out, status);
 }
+
+#ifdef SBL_TRACE
+cudaError_t set_prefill_trace(void* buf) {
+    unsigned long long* p = static_cast<unsigned long long*>(buf);
+    return cudaMemcpyToSymbol(g_trace, &p, sizeof(p));
+}
+#endif
 
 cudaError_t launch_prefill(const int8_t* xperm, const float* s_tok, long long T, long long K, const uint8_t* packed,
                            const float* row_scale, long long O, void* y, int y_bf16, int32_t* acc_out,
                            unsigned* status, int num_sms, cudaStream_t stream) {
-    // Wide tiles halve the expansion work per MMA; narrow ones fill the SMs
-    // when there are few tiles.
+    // Wide tiles (BN = 256) halve the activation traffic and the MMA issue
+    // overhead per output; narrow ones (BN = 128) fill more SMs when tiles are
+    // few.  Compare wave counts, a wide tile costing about two narrow ones.
     const long long mt = (T + pf::BM - 1) / pf::BM;
-    const long long wide_tiles = mt * ((O + 255) / 256);
-    const long long wide_waves = (wide_tiles + num_sms - 1) / num_sms;
-    const long long narrow_tiles = mt * ((O + 127) / 128);
-    const long long narrow_waves = (narrow_tiles + num_sms - 1) / num_sms;
-    if (2 * wide_waves <= narrow_waves || narrow_waves >= 8)
+    const long long wide_waves = (mt * ((O + 255) / 256) + num_sms - 1) / num_sms;
+    const long long narrow_waves = (mt * ((O + 127) / 128) + num_sms - 1) / num_sms;
+    if (2.0 * wide_waves <= 1.3 * narrow_waves)
         return launch_prefill_bn<256>(xperm, s_tok, T, K, packed, row_scale, O, y, y_bf16, acc_out, status, num_sms,
                                       stream);
     return launch_prefill_bn<128>(xperm, s_tok, T, K, packed, row_scale, O, y, y_bf16, acc_out, status, num_sms,

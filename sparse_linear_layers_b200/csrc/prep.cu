@@ -6,11 +6,13 @@
 // equation); per-row absmean from the halo-sparse-bitnet-3:4-500m card,
 // "Recipe"; code table 00 = 0, 01 = +1, 10 = -1 from its "Packed vs raw".
 //
-// One warp per row.  Each lane owns 16-weight chunks (c = lane, lane+32, ...),
-// read as four 16-byte loads.  Pass 1 builds the keep-mask of every group and
-// adds the kept |w| into an exact fixed-point accumulator; pass 2 re-reads the
-// chunk (L1/L2 resident), ternarises against the row scale and writes one
-// 32-bit word of codes and 16 mask bits per chunk.
+// TPR threads share a row (256 / TPR rows per block); each thread owns up to
+// two 16-weight chunks, read once as 16-byte loads and kept in registers.
+// Pass 1 builds the keep-mask of every group and adds the kept |w| into an
+// exact fixed-point accumulator; after a block-wide reduction of the row sums
+// pass 2 ternarises the registers against the row scale and writes one 32-bit
+// word of codes and 16 mask bits per chunk.  Rows longer than 512 chunks
+// (K > 8192) use a warp-per-row variant that reads the row twice.
 //
 // Exact sum: a finite float |w| = m * 2^(p - 149) with a 24-bit integer m and
 // 0 <= p <= 253, so the row sum is an integer in units of 2^-149 below 2^300.
@@ -181,13 +183,150 @@ __global__ void __launch_bounds__(kPrepWarps * 32) prep_kernel(const float* __re
     }
 }
 
+constexpr int kPrepThreads = 256;
+
+// Round the limb totals of one row to the float scale (exact sum -> double -> mean -> float).
+__device__ __forceinline__ float scale_from_totals(const unsigned long long* tot, long long K, int n, int M) {
+    uint32_t w[kLimbs];
+    unsigned long long carry = 0;
+#pragma unroll
+    for (int i = 0; i < kLimbs; ++i) {
+        const unsigned long long t = tot[i] + carry;
+        w[i] = static_cast<uint32_t>(t);
+        carry = t >> 32;
+    }
+    const double sum = limbs_to_double(w);
+    const double kept = static_cast<double>((K / M) * n);
+    return fmaxf(__double2float_rn(__ddiv_rn(sum, kept)), 1e-5f);
+}
+
+template <int M, int TPR>
+__global__ void __launch_bounds__(kPrepThreads, 3) prep_kernel_rr(const float* __restrict__ W, long long O,
+                                                               long long K, int n, uint8_t* __restrict__ packed,
+                                                               float* __restrict__ row_scale,
+                                                               uint8_t* __restrict__ mask_bits, unsigned* status) {
+    constexpr int RPB = kPrepThreads / TPR;  // rows per block
+    constexpr int CPT = 2;                   // chunks per thread
+    __shared__ unsigned long long limbs[kLimbs][kPrepThreads];
+    __shared__ unsigned long long totals[RPB][kLimbs];
+    __shared__ float scales[RPB];
+    const int sub = threadIdx.x / TPR, tr = threadIdx.x % TPR;
+    const long long row = static_cast<long long>(blockIdx.x) * RPB + sub;
+    const bool valid = row < O;
+    const int nchunks = static_cast<int>(K >> 4);
+    const float* wr = W + (valid ? row : 0) * K;
+
+    uint32_t raw[CPT][16];
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+        const int c = tr + TPR * j;
+        if (valid && c < nchunks) load_chunk(wr + 16 * c, raw[j]);
+        else
+#pragma unroll
+            for (int i = 0; i < 16; ++i) raw[j][i] = 0u;
+    }
+    unsigned long long* my = &limbs[0][threadIdx.x];
+#pragma unroll
+    for (int l = 0; l < kLimbs; ++l) my[l * kPrepThreads] = 0ull;
+
+    bool bad = false;
+    uint32_t keep[CPT];
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+        uint32_t a[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            a[i] = raw[j][i] & 0x7FFFFFFFu;
+            bad |= a[i] >= 0x7F800000u;
+        }
+        keep[j] = chunk_keep_bits<M>(a, n);
+        const int c = tr + TPR * j;
+        if (!(valid && c < nchunks)) keep[j] = 0u;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            if (keep[j] & (1u << i)) {
+                const uint32_t e = a[i] >> 23;
+                const uint32_t m24 = (a[i] & 0x7FFFFFu) | (e ? 0x800000u : 0u);
+                const uint32_t p = e ? e - 1u : 0u;
+                const uint32_t li = p >> 5;
+                const unsigned long long v = static_cast<unsigned long long>(m24) << (p & 31u);
+                my[li * kPrepThreads] += v & 0xFFFFFFFFull;
+                my[(li + 1) * kPrepThreads] += v >> 32;
+            }
+    }
+    if (__syncthreads_or(bad ? 1 : 0) && threadIdx.x == 0) raise_status(status, kStatusNonfinite);
+    // row totals: warp butterfly per limb (integer adds, any order), then the row's warps
+    __shared__ unsigned long long wsum[kPrepThreads / 32][kLimbs];
+    {
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+        for (int l = 0; l < kLimbs; ++l) {
+            unsigned long long v = limbs[l][threadIdx.x];
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
+            if (lane == 0) wsum[warp][l] = v;
+        }
+    }
+    __syncthreads();
+    if (tr < kLimbs) {
+        unsigned long long s = 0;
+#pragma unroll
+        for (int w = 0; w < TPR / 32; ++w) s += wsum[sub * (TPR / 32) + w][tr];
+        totals[sub][tr] = s;
+    }
+    __syncthreads();
+    if (tr == 0) {
+        const float sc = scale_from_totals(totals[sub], K, n, M);
+        scales[sub] = sc;
+        if (valid) row_scale[row] = sc;
+    }
+    __syncthreads();
+    if (!valid) return;
+    const uint32_t half_bits = __float_as_uint(0.5f * scales[sub]);  // exact: scale >= 1e-5 is normal
+    uint32_t* prow = reinterpret_cast<uint32_t*>(packed + row * (K >> 2));
+    uint16_t* mrow = mask_bits ? reinterpret_cast<uint16_t*>(mask_bits + row * (K >> 3)) : nullptr;
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+        const int c = tr + TPR * j;
+        if (c >= nchunks) continue;
+        uint32_t codes = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            // round(w / scale) != 0  <=>  |w| / scale > 1/2  <=>  |w| > scale / 2 (exact compare)
+            const bool nz = ((keep[j] >> i) & 1u) && ((raw[j][i] & 0x7FFFFFFFu) > half_bits);
+            codes |= (nz ? ((raw[j][i] >> 31) ? 2u : 1u) : 0u) << (2 * i);
+        }
+        prow[c] = codes;
+        if (mrow) mrow[c] = static_cast<uint16_t>(keep[j]);
+    }
+}
+
+template <int M, int TPR>
+static void launch_prep_rr(const float* W, long long O, long long K, int n, uint8_t* packed, float* row_scale,
+                           uint8_t* mask_bits, unsigned* status, cudaStream_t stream) {
+    constexpr int RPB = kPrepThreads / TPR;
+    const unsigned blocks = static_cast<unsigned>((O + RPB - 1) / RPB);
+    prep_kernel_rr<M, TPR><<<blocks, kPrepThreads, 0, stream>>>(W, O, K, n, packed, row_scale, mask_bits, status);
+}
+
+template <int M>
+static void launch_prep_m(const float* W, long long O, long long K, int n, uint8_t* packed, float* row_scale,
+                          uint8_t* mask_bits, unsigned* status, cudaStream_t stream) {
+    const long long nchunks = K >> 4;
+    if (nchunks <= 64) launch_prep_rr<M, 32>(W, O, K, n, packed, row_scale, mask_bits, status, stream);
+    else if (nchunks <= 128) launch_prep_rr<M, 64>(W, O, K, n, packed, row_scale, mask_bits, status, stream);
+    else if (nchunks <= 256) launch_prep_rr<M, 128>(W, O, K, n, packed, row_scale, mask_bits, status, stream);
+    else if (nchunks <= 512) launch_prep_rr<M, 256>(W, O, K, n, packed, row_scale, mask_bits, status, stream);
+    else {
+        const unsigned blocks = static_cast<unsigned>((O + kPrepWarps - 1) / kPrepWarps);
+        prep_kernel<M><<<blocks, kPrepWarps * 32, 0, stream>>>(W, O, K, n, packed, row_scale, mask_bits, status);
+    }
+}
+
 cudaError_t launch_prep(const float* W, long long O, long long K, int n, int m, uint8_t* packed, float* row_scale,
                         uint8_t* mask_bits, unsigned* status, cudaStream_t stream) {
-    const unsigned blocks = static_cast<unsigned>((O + kPrepWarps - 1) / kPrepWarps);
-    if (m == 4)
-        prep_kernel<4><<<blocks, kPrepWarps * 32, 0, stream>>>(W, O, K, n, packed, row_scale, mask_bits, status);
-    else
-        prep_kernel<8><<<blocks, kPrepWarps * 32, 0, stream>>>(W, O, K, n, packed, row_scale, mask_bits, status);
+    if (m == 4) launch_prep_m<4>(W, O, K, n, packed, row_scale, mask_bits, status, stream);
+    else launch_prep_m<8>(W, O, K, n, packed, row_scale, mask_bits, status, stream);
     return cudaGetLastError();
 }
 

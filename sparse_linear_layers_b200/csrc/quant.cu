@@ -6,83 +6,130 @@
 // the guide's module listing.  Decisions are taken in float32: s = 127 / beta
 // is an IEEE division, x * s an IEEE product, round() is half-to-even.
 //
-// One warp per token.  Pass 1: max of |x| on the bf16 bit patterns (the
-// magnitude bits order like the values).  Pass 2: quantise 16-element blocks;
-// INTERLEAVED output stores each block as byte 4j + b <- element 4b + j (the
-// order in which the contraction kernels expand 2-bit weight codes).
+// TPT threads share a token; each holds up to BPT 16-element blocks in
+// registers, so x is read once.  The max of |x| is taken on the bf16 bit
+// patterns (magnitude bits order like the values).  Output layouts:
+//   NATURAL      x_q in column order (the public sbl_quant_act);
+//   INTERLEAVED  each 16-element block stored as byte 4j + b <- element 4b + j,
+//                the order in which the tensor-core kernel expands weight codes
+//                (read by TMA).
+// The kernel signals programmatic dependents at entry: the contraction kernel
+// that follows may start its own prologue while this one runs.
 #include "sbl_common.cuh"
 
 namespace sbl {
 
-constexpr int kQuantWarps = 8;
+enum QuantLayout { kNatural = 0, kInterleaved = 1 };
 
-__device__ __forceinline__ int quant1(uint32_t bf16_bits, float s) {
-    const float x = __uint_as_float(bf16_bits << 16);
-    const int q = __float2int_rn(__fmul_rn(x, s));
-    return max(-128, min(127, q));
+template <int LAYOUT>
+__device__ __forceinline__ void quant_block_store(const uint4& u0, const uint4& u1, float s, int8_t* out_row, int b,
+                                                  long long K) {
+    (void)K;
+    *reinterpret_cast<uint4*>(out_row + 16 * static_cast<long long>(b)) = quant_block16<LAYOUT != kNatural>(u0, u1, s);
 }
 
-template <bool INTERLEAVED>
-__global__ void __launch_bounds__(kQuantWarps * 32) quant_kernel(const uint16_t* __restrict__ x, long long T,
-                                                                 long long K, int8_t* __restrict__ xq,
-                                                                 float* __restrict__ s_tok, unsigned* status) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long t = static_cast<long long>(blockIdx.x) * kQuantWarps + warp;
-    if (t >= T) return;
-    const uint4* xr = reinterpret_cast<const uint4*>(x + t * K);
-    const int nvec = static_cast<int>(K >> 3);  // 8 bf16 per 16-byte vector
+// Register-resident variant: K / 16 <= TPT * BPT.
+template <int LAYOUT, int TPT, int BPT>
+__global__ void __launch_bounds__(256) quant_kernel(const uint16_t* __restrict__ x, long long T, long long K,
+                                                    int8_t* __restrict__ xq, float* __restrict__ s_tok,
+                                                    unsigned* status) {
+    asm volatile("griddepcontrol.launch_dependents;");
+    constexpr int TPC = 256 / TPT;
+    __shared__ uint32_t red[8];
+    const int sub = threadIdx.x / TPT, tr = threadIdx.x % TPT;
+    const long long t = static_cast<long long>(blockIdx.x) * TPC + sub;
+    const bool valid = t < T;
+    const int nblk = static_cast<int>(K >> 4);
+    const uint4* xr = reinterpret_cast<const uint4*>(x + (valid ? t : 0) * K);
 
+    uint4 v[BPT][2];
     uint32_t mx = 0;
-    for (int v = lane; v < nvec; v += 32) {
-        const uint4 u = ldg_nc(xr + v);
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            mx = max(mx, w[i] & 0x7FFFu);
-            mx = max(mx, (w[i] >> 16) & 0x7FFFu);
+    for (int j = 0; j < BPT; ++j) {
+        const int b = tr + TPT * j;
+        if (valid && b < nblk) {
+            v[j][0] = ldg_nc(xr + 2 * b);
+            v[j][1] = ldg_nc(xr + 2 * b + 1);
+        } else {
+            v[j][0] = v[j][1] = make_uint4(0u, 0u, 0u, 0u);
         }
     }
+#pragma unroll
+    for (int j = 0; j < BPT; ++j) mx = absmax8(v[j][1], absmax8(v[j][0], mx));
     mx = __reduce_max_sync(0xFFFFFFFFu, mx);
-    if (mx >= 0x7F80u && lane == 0) raise_status(status, kStatusNonfinite);
+    if constexpr (TPT > 32) {
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+        __syncthreads();
+        const int w0 = sub * (TPT / 32);
+#pragma unroll
+        for (int i = 0; i < TPT / 32; ++i) mx = max(mx, red[w0 + i]);
+    }
+    if (!valid) return;
+    if (mx >= 0x7F80u && tr == 0) raise_status(status, kStatusNonfinite);
     const float amax = __uint_as_float(mx << 16);
     const float s = __fdiv_rn(127.0f, fmaxf(amax, 1e-5f));
-    if (lane == 0) s_tok[t] = s;
-
+    if (tr == 0) s_tok[t] = s;
     int8_t* out = xq + t * K;
-    const int nblk = static_cast<int>(K >> 4);
-    for (int b = lane; b < nblk; b += 32) {
-        const uint4 u0 = ldg_nc(xr + 2 * b);
-        const uint4 u1 = ldg_nc(xr + 2 * b + 1);
-        const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-        int q[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            q[2 * i] = quant1(w[i] & 0xFFFFu, s);
-            q[2 * i + 1] = quant1(w[i] >> 16, s);
-        }
-        uint32_t o[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            uint32_t word = 0;
-#pragma unroll
-            for (int bb = 0; bb < 4; ++bb) {
-                const int src = INTERLEAVED ? (4 * bb + j) : (4 * j + bb);
-                word |= (static_cast<uint32_t>(q[src]) & 0xFFu) << (8 * bb);
-            }
-            o[j] = word;
-        }
-        *reinterpret_cast<uint4*>(out + 16 * b) = make_uint4(o[0], o[1], o[2], o[3]);
+    for (int j = 0; j < BPT; ++j) {
+        const int b = tr + TPT * j;
+        if (b < nblk) quant_block_store<LAYOUT>(v[j][0], v[j][1], s, out, b, K);
     }
 }
 
-cudaError_t launch_quant(const uint16_t* x, long long T, long long K, int8_t* xq, float* s_tok, bool interleaved,
-                         unsigned* status, cudaStream_t stream) {
-    const unsigned blocks = static_cast<unsigned>((T + kQuantWarps - 1) / kQuantWarps);
-    if (interleaved)
-        quant_kernel<true><<<blocks, kQuantWarps * 32, 0, stream>>>(x, T, K, xq, s_tok, status);
-    else
-        quant_kernel<false><<<blocks, kQuantWarps * 32, 0, stream>>>(x, T, K, xq, s_tok, status);
+// Any K: one warp per token, two passes over x (the second mostly from L1/L2).
+template <int LAYOUT>
+__global__ void __launch_bounds__(256) quant_kernel_loop(const uint16_t* __restrict__ x, long long T, long long K,
+                                                         int8_t* __restrict__ xq, float* __restrict__ s_tok,
+                                                         unsigned* status) {
+    asm volatile("griddepcontrol.launch_dependents;");
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long t = static_cast<long long>(blockIdx.x) * 8 + warp;
+    if (t >= T) return;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + t * K);
+    const int nvec = static_cast<int>(K >> 3);
+    uint32_t mx = 0;
+#pragma unroll 4
+    for (int v = lane; v < nvec; v += 32) mx = absmax8(ldg_nc(xr + v), mx);
+    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+    if (mx >= 0x7F80u && lane == 0) raise_status(status, kStatusNonfinite);
+    const float s = __fdiv_rn(127.0f, fmaxf(__uint_as_float(mx << 16), 1e-5f));
+    if (lane == 0) s_tok[t] = s;
+    const int nblk = static_cast<int>(K >> 4);
+#pragma unroll 2
+    for (int b = lane; b < nblk; b += 32)
+        quant_block_store<LAYOUT>(ldg_nc(xr + 2 * b), ldg_nc(xr + 2 * b + 1), s, xq + t * K, b, K);
+}
+
+template <int LAYOUT, int TPT, int BPT>
+static void launch_rr(const uint16_t* x, long long T, long long K, int8_t* xq, float* s_tok, unsigned* status,
+                      cudaStream_t stream) {
+    constexpr int TPC = 256 / TPT;
+    const unsigned blocks = static_cast<unsigned>((T + TPC - 1) / TPC);
+    quant_kernel<LAYOUT, TPT, BPT><<<blocks, 256, 0, stream>>>(x, T, K, xq, s_tok, status);
+}
+
+template <int LAYOUT>
+static cudaError_t launch_layout(const uint16_t* x, long long T, long long K, int8_t* xq, float* s_tok,
+                                 unsigned* status, cudaStream_t stream) {
+    const long long nblk = K >> 4;
+    if (nblk <= 32 * 4) launch_rr<LAYOUT, 32, 4>(x, T, K, xq, s_tok, status, stream);
+    else if (nblk <= 64 * 4) launch_rr<LAYOUT, 64, 4>(x, T, K, xq, s_tok, status, stream);
+    else if (nblk <= 128 * 4) launch_rr<LAYOUT, 128, 4>(x, T, K, xq, s_tok, status, stream);
+    else if (nblk <= 256 * 4) launch_rr<LAYOUT, 256, 4>(x, T, K, xq, s_tok, status, stream);
+    else {
+        const unsigned blocks = static_cast<unsigned>((T + 7) / 8);
+        quant_kernel_loop<LAYOUT><<<blocks, 256, 0, stream>>>(x, T, K, xq, s_tok, status);
+    }
     return cudaGetLastError();
+}
+
+cudaError_t launch_quant(const uint16_t* x, long long T, long long K, int8_t* xq, float* s_tok, int layout,
+                         unsigned* status, cudaStream_t stream) {
+    switch (layout) {
+        case kInterleaved: return launch_layout<kInterleaved>(x, T, K, xq, s_tok, status, stream);
+        default: return launch_layout<kNatural>(x, T, K, xq, s_tok, status, stream);
+    }
 }
 
 }  // namespace sbl

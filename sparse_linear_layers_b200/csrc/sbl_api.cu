@@ -11,14 +11,18 @@
 namespace sbl {
 cudaError_t launch_prep(const float* W, long long O, long long K, int n, int m, uint8_t* packed, float* row_scale,
                         uint8_t* mask_bits, unsigned* status, cudaStream_t stream);
-cudaError_t launch_quant(const uint16_t* x, long long T, long long K, int8_t* xq, float* s_tok, bool interleaved,
+cudaError_t launch_quant(const uint16_t* x, long long T, long long K, int8_t* xq, float* s_tok, int layout,
                          unsigned* status, cudaStream_t stream);
+constexpr int kLayoutNatural = 0, kLayoutInterleaved = 1;
 cudaError_t launch_decode(const uint8_t* packed, const float* row_scale, long long O, long long K,
-                          const int8_t* xperm, const float* s_tok, long long T, void* y, int y_bf16,
-                          int32_t* acc_out, int num_sms, cudaStream_t stream);
+                          const uint16_t* x, long long T, void* y, int y_bf16, int32_t* acc_out, unsigned* status,
+                          int num_sms, cudaStream_t stream);
 cudaError_t launch_prefill(const int8_t* xperm, const float* s_tok, long long T, long long K, const uint8_t* packed,
                            const float* row_scale, long long O, void* y, int y_bf16, int32_t* acc_out,
                            unsigned* status, int num_sms, cudaStream_t stream);
+#ifdef SBL_TRACE
+cudaError_t set_prefill_trace(void* buf);
+#endif
 
 // Status word: one per device, read and cleared by sbl_device_status().
 __device__ unsigned g_status_word;
@@ -39,6 +43,7 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr long long kMaxK = 1ll << 24;            // keeps |acc| <= 127 * K below 2^31
 constexpr long long kDecodeMaxTokens = 16;
+constexpr long long kDecodeMaxK = 24576;          // decode holds 8 tokens x K int8 in shared memory
 
 struct DeviceInfo {
     unsigned* status = nullptr;
@@ -105,7 +110,8 @@ sbl_status sbl_quant_act(const uint16_t* x_bf16, int64_t T, int64_t K, int8_t* x
     if (T > (1ll << 31) - 1) return SBL_ERR_UNSUPPORTED;
     DeviceInfo* d;
     if (sbl_status s = device_info(&d)) return s;
-    return from_cuda(sbl::launch_quant(x_bf16, T, K, x_q, s_tok, false, d->status, static_cast<cudaStream_t>(stream)));
+    return from_cuda(sbl::launch_quant(x_bf16, T, K, x_q, s_tok, sbl::kLayoutNatural, d->status,
+                                       static_cast<cudaStream_t>(stream)));
 }
 
 size_t sbl_linear_workspace_bytes(int64_t T, int64_t K, int64_t O, int n, int m) {
@@ -141,15 +147,19 @@ sbl_status sbl_linear_path(const uint16_t* x_bf16, int64_t T, int64_t K, const u
     float* s_tok = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round256(static_cast<size_t>(T) * K));
 
     bool prefill = path == SBL_PATH_PREFILL;
-    if (path == SBL_PATH_AUTO) prefill = (T > kDecodeMaxTokens) && (K % 64 == 0);
+    if (path == SBL_PATH_AUTO) prefill = ((T > kDecodeMaxTokens) || (K > kDecodeMaxK)) && (K % 64 == 0);
+    if (!prefill && K > kDecodeMaxK) return SBL_ERR_UNSUPPORTED;
 
-    cudaError_t e = sbl::launch_quant(x_bf16, T, K, xq, s_tok, true, d->status, st);
-    if (e != cudaSuccess) return SBL_ERR_CUDA;
     const int ybf = y_dtype == SBL_BF16 ? 1 : 0;
-    if (prefill)
+    cudaError_t e;
+    if (prefill) {
+        e = sbl::launch_quant(x_bf16, T, K, xq, s_tok, sbl::kLayoutInterleaved, d->status, st);
+        if (e != cudaSuccess) return SBL_ERR_CUDA;
         e = sbl::launch_prefill(xq, s_tok, T, K, packed, row_scale, O, y, ybf, acc_out, d->status, d->num_sms, st);
-    else
-        e = sbl::launch_decode(packed, row_scale, O, K, xq, s_tok, T, y, ybf, acc_out, d->num_sms, st);
+    } else {
+        // the decode kernel quantises the activations itself
+        e = sbl::launch_decode(packed, row_scale, O, K, x_bf16, T, y, ybf, acc_out, d->status, d->num_sms, st);
+    }
     return from_cuda(e);
 }
 
@@ -197,5 +207,10 @@ const char* sbl_status_string(sbl_status s) {
 }
 
 const char* sbl_version(void) { return "sbl 0.1.0 (sm_100a)"; }
+
+#ifdef SBL_TRACE
+// Debug builds only: device buffer of 16 x 256 uint64 for prefill event stamps (NULL disables).
+sbl_status sbl_debug_set_trace(void* buf) { return from_cuda(sbl::set_prefill_trace(buf)); }
+#endif
 
 }  // extern "C"

@@ -73,6 +73,32 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded spin on the non-blocking test: for single-thread roles (MMA issue,
+// TMA producer) whose reaction time after a phase completes matters.
+__device__ __forceinline__ bool mbar_spin(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_test_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_test_wait(bar, parity)) return true;
+        if ((i & 255u) == 0u) {
+            if (*abort_flag) return false;
+            if (global_ns() - t0 > kWaitLimitNs) return false;
+        }
+    }
+}
+
 __device__ __forceinline__ void fence_barrier_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
@@ -123,6 +149,51 @@ __device__ __forceinline__ void expand_codes(uint32_t w, uint32_t (&out)[4]) {
         const uint32_t lo = (j == 0 ? w : (w >> (2 * j))) & 0x01010101u; // 0x01 where the code is 01
         out[j] = neg | lo;
     }
+}
+
+// ---------------------------------------------------------------- activation quantisation
+// round_half_even(x * s) clamped to int8, x a bf16 bit pattern, s the token's 127 / max|x|.
+__device__ __forceinline__ int quant1(uint32_t bf16_bits, float s) {
+    const float x = __uint_as_float(bf16_bits << 16);
+    const int q = __float2int_rn(__fmul_rn(x, s));
+    return max(-128, min(127, q));
+}
+
+__device__ __forceinline__ uint32_t absmax8(const uint4& u, uint32_t mx) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        mx = max(mx, w[i] & 0x7FFFu);
+        mx = max(mx, (w[i] >> 16) & 0x7FFFu);
+    }
+    return mx;
+}
+
+
+// Quantise 16 consecutive activations (two 16-byte vectors of bf16) and return
+// them as four int8x4 words, either in column order or interleaved (byte
+// 4j + b <- element 4b + j, the order of expand_codes()).
+template <bool INTERLEAVED>
+__device__ __forceinline__ uint4 quant_block16(const uint4& u0, const uint4& u1, float s) {
+    const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+    int q[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        q[2 * i] = quant1(w[i] & 0xFFFFu, s);
+        q[2 * i + 1] = quant1(w[i] >> 16, s);
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) {
+            const int src = INTERLEAVED ? (4 * bb + j) : (4 * j + bb);
+            word |= (static_cast<uint32_t>(q[src]) & 0xFFu) << (8 * bb);
+        }
+        o[j] = word;
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 }  // namespace sbl
