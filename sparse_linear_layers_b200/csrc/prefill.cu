@@ -7,7 +7,7 @@
 //
 //   warps 0-3          epilogue: warp w owns TMEM lanes 32w .. 32w + 31 (32 tokens);
 //                      pipelined tcgen05.ld, dequantise, per-warp 128B-swizzled
-//                      staging boxes, TMA stores
+//                      double-buffered staging boxes, TMA bulk stores
 //   warps 4..4+BN/32-1 weight expansion: each thread owns one output row o of
 //                      the B tile, reads its 2-bit codes for the k-block from
 //                      shared memory and writes the int8 row into the
@@ -20,8 +20,12 @@
 // quantisation: set-up (barriers, tensor memory) overlaps its tail, and every
 // role waits on griddepcontrol before touching its outputs.
 //
-// Tile: 128 tokens x BN output rows x 128 k per stage, 4 stages, two TMEM
-// accumulator buffers so the epilogue of one tile overlaps the MMAs of the next.
+// Tile: 128 tokens x BN output rows x 128 k per stage (3 stages for BN = 256,
+// 4 for BN = 128), two TMEM accumulator buffers so the epilogue of one tile
+// overlaps the MMAs of the next.  Shared-memory bandwidth is the binding
+// resource: per k-block the MMA reads the activation and weight tiles, TMA
+// writes the activation and code tiles and the expansion writes the int8
+// weight tile (about 112 KB per 128 x 256 x 128 step at BN = 256).
 // The weights are expanded in the interleaved 16-element order of
 // expand_codes(); the activations were quantised into the same order.
 //
@@ -75,7 +79,7 @@ struct PrefillSmem {
     uint8_t a[PrefillCfg<BN>::STAGES][pf::A_BYTES];            // 1024-byte aligned tiles
     uint8_t b[PrefillCfg<BN>::STAGES][PrefillCfg<BN>::B_BYTES];
     uint8_t p[PrefillCfg<BN>::STAGES][PrefillCfg<BN>::P_BYTES];
-    uint8_t ystage[pf::EPI_WARPS][1][pf::Y_BYTES];           // per-warp output transpose box
+    uint8_t ystage[pf::EPI_WARPS][2][pf::Y_BYTES];           // per-warp output transpose box
     float wscale[pf::EPI_WARPS][BN];                          // per-warp copy of the tile's row scales
     uint64_t full_tma[PrefillCfg<BN>::STAGES];
     uint64_t full_dec[PrefillCfg<BN>::STAGES];
@@ -118,6 +122,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
         : "memory");
 }
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(src)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // One lane polls the barrier, the warp follows (fewer pollers on shared memory).
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
@@ -176,7 +191,7 @@ __device__ __forceinline__ void st_v4(void* p, uint32_t a, uint32_t b, uint32_t 
 template <int BN>
 __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                   int y_vec, const float* __restrict__ row_scale,
+                   const __grid_constant__ CUtensorMap tmap_y, int y_vec, const float* __restrict__ row_scale,
                    const float* __restrict__ s_tok, int T, int O, int K, void* __restrict__ y, int y_bf16,
                    int32_t* __restrict__ acc_out, unsigned* status) {
     using Cfg = PrefillCfg<BN>;
@@ -246,6 +261,7 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
             float* const wsc = sm->wscale[warp];
             int tc = 0;
             int ep_round = 0;
+            uint32_t nstore = 0;
             for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
                 const int mt = tile % MT, nt = tile / MT;
                 const int b = tc & 1;
@@ -308,10 +324,9 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
                         const int o0 = nt * BN + 32 * (k - H);
                         if (threadIdx.x == 0) SBL_TR(11, ep_round);
                         if (y_vec) {
-                            // transpose through the warp's swizzled box: written one token row
-                            // per lane, read back so each store instruction covers 4 whole
-                            // 128-byte lines of y
-                            uint8_t* const box = sm->ystage[warp][0];
+                            uint8_t* const box = sm->ystage[warp][nstore & 1];
+                            if (lane == 0) bulk_wait_read<1>();
+                            __syncwarp();
 #pragma unroll
                             for (int c = 0; c < 8; ++c) {
                                 const uint32_t a = smem_u32(box + lane * 128 + ((c ^ (lane & 7)) << 4));
@@ -319,28 +334,10 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
                                              "r"(q[4 * c + 1]), "r"(q[4 * c + 2]), "r"(q[4 * c + 3])
                                              : "memory");
                             }
+                            fence_proxy_async_smem();
                             __syncwarp();
-                            if (threadIdx.x == 0) SBL_TR(12, ep_round);
-                            constexpr int PER_CHUNK = BF ? 8 : 4;  // outputs per 16-byte chunk
-                            const int cch = lane & 7;
-                            const int col = o0 + cch * PER_CHUNK;
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                const int rr = 4 * i + (lane >> 3);
-                                const uint32_t a = smem_u32(box + rr * 128 + ((cch ^ (rr & 7)) << 4));
-                                uint32_t v0, v1, v2, v3;
-                                asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
-                                             : "=r"(v0), "=r"(v1), "=r"(v2), "=r"(v3)
-                                             : "r"(a));
-                                const int tok = mt * pf::BM + warp * 32 + rr;
-                                if (tok < T && col < O) {
-                                    uint8_t* dst = static_cast<uint8_t*>(y) +
-                                                   (static_cast<long long>(tok) * O + col) * (BF ? 2 : 4);
-                                    st_v4(dst, v0, v1, v2, v3);
-                                }
-                            }
-                            __syncwarp();
-                            if (threadIdx.x == 0) SBL_TR(13, ep_round);
+                            if (lane == 0) tma_store_2d(&tmap_y, smem_u32(box), o0, mt * pf::BM + warp * 32);
+                            ++nstore;
                         } else if (tvalid) {
                             // direct stores: shapes whose row pitch is not a multiple of 16 bytes
                             const long long base = static_cast<long long>(t) * O + o0;
@@ -373,6 +370,7 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
                 }
                 if (threadIdx.x == 0) SBL_TR(7, tc);
             }
+            if (lane == 0) bulk_wait_all();
         };
         if (y_bf16) run(std::true_type{});
         else run(std::false_type{});
@@ -387,7 +385,7 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
                 const uint32_t ph = (it / Cfg::STAGES) & 1;
                 // the codes have landed, and the producer only issued them once the
                 // MMA had released this stage, so b[s] is free as well
-                if (!warp_wait(&sm->full_tma[s], ph, abort_flag)) { give_up(); ok = false; break; }
+                if (!mbar_wait(&sm->full_tma[s], ph, abort_flag)) { give_up(); ok = false; break; }
                 if (r == 0) SBL_TR(1, it);
                 // code tile rows are 32 bytes, 32B-swizzled by TMA: 16-byte half q of
                 // row r sits at half q ^ ((r >> 2) & 1)
@@ -437,43 +435,34 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
         }
     } else {
         // ------------------------------------------------------------ MMA issuer
-        // One flat walk over (tile, k-block).  The barriers of step n + 1 are
-        // checked before step n is committed: an mbarrier operation issued right
-        // after tcgen05.commit waits for the committed MMAs to finish, which
-        // would leave the tensor pipe idle between stages.
+        // Per stage: wait for the activation and expanded weight tiles, four
+        // K = 32 MMAs, commit (releases the stage when the MMAs finish); per
+        // tile: wait for a free accumulator buffer, commit it to the epilogue.
         if (lane == 0) {
             const uint32_t idesc = i8_idesc<BN>();
-            const int my_tiles = tiles > static_cast<int>(blockIdx.x)
-                                     ? (tiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
-                                     : 0;
-            const uint32_t total = static_cast<uint32_t>(my_tiles) * static_cast<uint32_t>(KB);
-            // wait for everything step n needs: accumulator buffer (first k-block of a tile) and stage data
-            auto ready = [&](uint32_t n) -> bool {
-                const uint32_t tcn = n / KB, kbn = n % KB;
-                if (kbn == 0 && !mbar_spin(&sm->tmem_empty[tcn & 1], ((tcn >> 1) & 1) ^ 1, abort_flag)) return false;
-                const uint32_t s = n % Cfg::STAGES, ph = (n / Cfg::STAGES) & 1;
-                if (!mbar_spin(&sm->full_tma[s], ph, abort_flag)) return false;
-                SBL_TR(3, n);
-                if (!mbar_spin(&sm->full_dec[s], ph, abort_flag)) return false;
-                SBL_TR(4, n);
-                return true;
-            };
-            bool ok = total == 0 || ready(0);
-            if (!ok) give_up();
-            for (uint32_t n = 0; n < total && ok; ++n) {
+            uint32_t it = 0;
+            int tc = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++tc) {
+                const int b = tc & 1;
+                const uint32_t aph = (tc >> 1) & 1;
+                if (!mbar_wait(&sm->tmem_empty[b], aph ^ 1, abort_flag)) { give_up(); break; }
                 tc_fence_after();
-                const uint32_t tcn = n / KB, kbn = n % KB;
-                const uint32_t s = n % Cfg::STAGES;
-                const uint32_t d = tmem_base + (tcn & 1) * BN;
-                const uint32_t a0 = smem_u32(sm->a[s]), b0 = smem_u32(sm->b[s]);
+                const uint32_t d = tmem_base + b * BN;
+                for (int kb = 0; kb < KB; ++kb, ++it) {
+                    const int s = it % Cfg::STAGES;
+                    const uint32_t ph = (it / Cfg::STAGES) & 1;
+                    if (!mbar_wait(&sm->full_tma[s], ph, abort_flag) || !mbar_wait(&sm->full_dec[s], ph, abort_flag)) {
+                        give_up(); ok = false; break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(sm->a[s]), b0 = smem_u32(sm->b[s]);
 #pragma unroll
-                for (int kk = 0; kk < pf::BK / 32; ++kk)
-                    tc_mma(d, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc, (kbn | kk) != 0);
-                SBL_TR(9, n);
-                if (n + 1 < total && !ready(n + 1)) { give_up(); ok = false; }
-                tc_commit(&sm->empty[s]);
-                if (kbn == static_cast<uint32_t>(KB) - 1) tc_commit(&sm->tmem_full[tcn & 1]);
-                SBL_TR(5, n);
+                    for (int kk = 0; kk < pf::BK / 32; ++kk)
+                        tc_mma(d, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc, (kb | kk) != 0);
+                    tc_commit(&sm->empty[s]);
+                }
+                if (ok) tc_commit(&sm->tmem_full[b]);
             }
             // all MMAs must be complete before tensor memory is released
             tc_commit(&sm->mma_done);
@@ -536,7 +525,17 @@ static cudaError_t launch_prefill_bn(const int8_t* xperm, const float* s_tok, lo
     }
     // output rows go out as 16-byte vectors when the row pitch allows it
     const int esize = y_bf16 ? 2 : 4;
-    const int y_vec = (static_cast<long long>(O) * esize) % 16 == 0 ? 1 : 0;
+    int y_vec = (static_cast<long long>(O) * esize) % 16 == 0 ? 1 : 0;
+    CUtensorMap map_y = map_x;
+    if (y_vec) {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(O), static_cast<cuuint64_t>(T)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(O) * esize};
+        const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esize), 32u};
+        if (enc(&map_y, y_bf16 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, y, dims, strides,
+                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            y_vec = 0;
+    }
     constexpr size_t smem = prefill_smem_bytes<BN>();
     static bool attr_set[64] = {};
     int dev = 0;
@@ -559,7 +558,7 @@ static cudaError_t launch_prefill_bn(const int8_t* xperm, const float* s_tok, lo
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, prefill_kernel<BN>, map_x, map_w, y_vec, row_scale, s_tok, static_cast<int>(T),
+    return cudaLaunchKernelEx(&cfg, prefill_kernel<BN>, map_x, map_w, map_y, y_vec, row_scale, s_tok, static_cast<int>(T),
                               static_cast<int>(O), static_cast<int>(K), y, y_bf16, acc_out, status);
 }
 
