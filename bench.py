@@ -340,7 +340,7 @@ def run_ours(args, rank, world, dev):
 
     decode = _decode_roofline(sbl, dev, hbm_peak) if rank == 0 else None
     launches_per_step = len(layers) * (1 + 2 + 1)  # prep + (quant + tcgen05 GEMM) + fused decode
-    value = world * TOKENS_PER_STEP * K / total_s
+    value = _throughput(world, K, total_s)
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": total_s * 1e3 / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -426,6 +426,11 @@ def run_reference(args, rank, world):
 def _barrier(world):
     if world > 1:
         torch.distributed.barrier()
+
+
+def _throughput(world, steps, total_s):
+    """Whole-job tokens/s: every rank runs the step on its own GPU (weak scaling)."""
+    return world * TOKENS_PER_STEP * steps / total_s
 
 
 def _max_over_ranks(v, world, dev):

@@ -8,11 +8,12 @@
 //
 // TPR threads share a row (256 / TPR rows per block); each thread owns up to
 // two 16-weight chunks, read once as 16-byte loads and kept in registers.
-// Pass 1 builds the keep-mask of every group and adds the kept |w| into an
-// exact fixed-point accumulator; after a block-wide reduction of the row sums
-// pass 2 ternarises the registers against the row scale and writes one 32-bit
-// word of codes and 16 mask bits per chunk.  Rows longer than 512 chunks
-// (K > 8192) use a warp-per-row variant that reads the row twice.
+// Pass 1 builds the keep-mask of every group and adds the kept |w| exactly
+// into a register window anchored at the row's largest kept magnitude (see
+// kWindow); after a block-wide reduction of the row sums, pass 2 ternarises
+// the registers against the row scale and writes one 32-bit word of codes and
+// 16 mask bits per chunk.  Rows longer than 512 chunks (K > 8192) use a
+// warp-per-row variant that reads the row twice and sums in shared-memory limbs.
 //
 // Exact sum: a finite float |w| = m * 2^(p - 149) with a 24-bit integer m and
 // 0 <= p <= 253, so the row sum is an integer in units of 2^-149 below 2^300.
@@ -185,31 +186,61 @@ __global__ void __launch_bounds__(kPrepWarps * 32) prep_kernel(const float* __re
 
 constexpr int kPrepThreads = 256;
 
-// Round the limb totals of one row to the float scale (exact sum -> double -> mean -> float).
-__device__ __forceinline__ float scale_from_totals(const unsigned long long* tot, long long K, int n, int M) {
-    uint32_t w[kLimbs];
-    unsigned long long carry = 0;
-#pragma unroll
-    for (int i = 0; i < kLimbs; ++i) {
-        const unsigned long long t = tot[i] + carry;
-        w[i] = static_cast<uint32_t>(t);
-        carry = t >> 32;
+// Exact row sums in registers.  With p_max the largest exponent index among the
+// row's kept magnitudes (|w| = m * 2^(p - 149), m < 2^24), every kept value
+// with p >= base = p_max - 96 is added exactly into a 128-bit per-thread
+// accumulator in units of 2^(base - 149) (a value is below 2^120 there and a
+// thread adds at most 32 of them); smaller values only set a sticky flag.
+// Their total is below 2^24 * 2^base, at least 2^40 times smaller than the
+// rounding position of a double holding the sum (which is >= 2^(p_max + 23)),
+// so the 192-bit row total plus the sticky flag rounds to the same double as
+// the exact sum.
+constexpr int kWindow = 96;
+
+__device__ __forceinline__ void add128(unsigned long long& w0, unsigned long long& w1, unsigned long long a0,
+                                       unsigned long long a1) {
+    asm("add.cc.u64 %0, %0, %2;\n\taddc.u64 %1, %1, %3;" : "+l"(w0), "+l"(w1) : "l"(a0), "l"(a1));
+}
+
+__device__ __forceinline__ void add192(unsigned long long (&w)[3], const unsigned long long (&a)[3]) {
+    asm("add.cc.u64 %0, %0, %3;\n\taddc.cc.u64 %1, %1, %4;\n\taddc.u64 %2, %2, %5;"
+        : "+l"(w[0]), "+l"(w[1]), "+l"(w[2])
+        : "l"(a[0]), "l"(a[1]), "l"(a[2]));
+}
+
+// Round w[0..2] * 2^(base - 149) (+ a sticky remainder) to double.
+__device__ double window_to_double(const unsigned long long (&w)[3], bool sticky, int base) {
+    int h = 2;
+    while (h >= 0 && w[h] == 0ull) --h;
+    if (h < 0) return 0.0;  // sticky alone cannot happen: dropped values are nonzero only next to larger ones
+    const int lz = __clzll(w[h]);
+    unsigned long long top = w[h] << lz;
+    unsigned long long rest = 0;  // bits below `top`
+    if (h >= 1) {
+        if (lz) top |= w[h - 1] >> (64 - lz);
+        rest = w[h - 1] << lz;
+        if (lz == 0) rest = w[h - 1];
+        if (h == 2) rest |= w[0];
     }
-    const double sum = limbs_to_double(w);
-    const double kept = static_cast<double>((K / M) * n);
-    return fmaxf(__double2float_rn(__ddiv_rn(sum, kept)), 1e-5f);
+    if (rest || sticky) top |= 1ull;  // sticky bit: below the rounding position
+    const int e2 = 64 * h + (64 - lz) - 64 + base - 149;  // weight of bit 0 of `top`
+    const double scale = __longlong_as_double(static_cast<long long>(1023 + e2) << 52);
+    return __ull2double_rn(top) * scale;
 }
 
 template <int M, int TPR>
-__global__ void __launch_bounds__(kPrepThreads, 3) prep_kernel_rr(const float* __restrict__ W, long long O,
+__global__ void __launch_bounds__(kPrepThreads) prep_kernel_rr(const float* __restrict__ W, long long O,
                                                                long long K, int n, uint8_t* __restrict__ packed,
                                                                float* __restrict__ row_scale,
                                                                uint8_t* __restrict__ mask_bits, unsigned* status) {
     constexpr int RPB = kPrepThreads / TPR;  // rows per block
     constexpr int CPT = 2;                   // chunks per thread
-    __shared__ unsigned long long limbs[kLimbs][kPrepThreads];
-    __shared__ unsigned long long totals[RPB][kLimbs];
+    constexpr int WPR = TPR / 32;            // warps per row
+    __shared__ uint32_t wmax[kPrepThreads / 32];
+    __shared__ unsigned long long wsum[kPrepThreads / 32][3];
+    __shared__ uint32_t wsticky[kPrepThreads / 32];
     __shared__ float scales[RPB];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int sub = threadIdx.x / TPR, tr = threadIdx.x % TPR;
     const long long row = static_cast<long long>(blockIdx.x) * RPB + sub;
     const bool valid = row < O;
@@ -225,12 +256,11 @@ __global__ void __launch_bounds__(kPrepThreads, 3) prep_kernel_rr(const float* _
 #pragma unroll
             for (int i = 0; i < 16; ++i) raw[j][i] = 0u;
     }
-    unsigned long long* my = &limbs[0][threadIdx.x];
-#pragma unroll
-    for (int l = 0; l < kLimbs; ++l) my[l * kPrepThreads] = 0ull;
 
+    // keep-masks, non-finite check and the largest kept magnitude of the row
     bool bad = false;
     uint32_t keep[CPT];
+    uint32_t mx = 0;
 #pragma unroll
     for (int j = 0; j < CPT; ++j) {
         uint32_t a[16];
@@ -244,39 +274,68 @@ __global__ void __launch_bounds__(kPrepThreads, 3) prep_kernel_rr(const float* _
         if (!(valid && c < nchunks)) keep[j] = 0u;
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-            if (keep[j] & (1u << i)) {
-                const uint32_t e = a[i] >> 23;
-                const uint32_t m24 = (a[i] & 0x7FFFFFu) | (e ? 0x800000u : 0u);
-                const uint32_t p = e ? e - 1u : 0u;
-                const uint32_t li = p >> 5;
-                const unsigned long long v = static_cast<unsigned long long>(m24) << (p & 31u);
-                my[li * kPrepThreads] += v & 0xFFFFFFFFull;
-                my[(li + 1) * kPrepThreads] += v >> 32;
-            }
+            if (keep[j] & (1u << i)) mx = max(mx, a[i]);
     }
+    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+    if (lane == 0) wmax[warp] = mx;
     if (__syncthreads_or(bad ? 1 : 0) && threadIdx.x == 0) raise_status(status, kStatusNonfinite);
-    // row totals: warp butterfly per limb (integer adds, any order), then the row's warps
-    __shared__ unsigned long long wsum[kPrepThreads / 32][kLimbs];
-    {
-        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
-        for (int l = 0; l < kLimbs; ++l) {
-            unsigned long long v = limbs[l][threadIdx.x];
+    for (int w = 0; w < WPR; ++w) mx = max(mx, wmax[sub * WPR + w]);
+    const int emax = static_cast<int>(mx >> 23);
+    const int base = (emax ? emax - 1 : 0) - kWindow;
+
+    // exact accumulation of the kept magnitudes
+    unsigned long long w0 = 0, w1 = 0;
+    uint32_t sticky = 0;
 #pragma unroll
-            for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
-            if (lane == 0) wsum[warp][l] = v;
+    for (int j = 0; j < CPT; ++j)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if (!(keep[j] & (1u << i))) continue;
+            const uint32_t a = raw[j][i] & 0x7FFFFFFFu;
+            const uint32_t e = a >> 23;
+            const uint32_t m24 = (a & 0x7FFFFFu) | (e ? 0x800000u : 0u);
+            const int sh = (e ? static_cast<int>(e) - 1 : 0) - base;  // <= kWindow
+            if (sh < 0) {
+                sticky |= m24;
+            } else {
+                const int bit = sh & 63;
+                const unsigned long long v = static_cast<unsigned long long>(m24) << bit;
+                const unsigned long long hi = bit > 40 ? static_cast<unsigned long long>(m24) >> (64 - bit) : 0ull;
+                if (sh < 64) add128(w0, w1, v, hi);
+                else add128(w0, w1, 0ull, v);
+            }
         }
-    }
-    __syncthreads();
-    if (tr < kLimbs) {
-        unsigned long long s = 0;
+
+    // row total: warp butterfly on 192 bits, then the row's warps
+    unsigned long long t[3] = {w0, w1, 0ull};
 #pragma unroll
-        for (int w = 0; w < TPR / 32; ++w) s += wsum[sub * (TPR / 32) + w][tr];
-        totals[sub][tr] = s;
+    for (int off = 16; off >= 1; off >>= 1) {
+        const unsigned long long o[3] = {__shfl_xor_sync(0xFFFFFFFFu, t[0], off),
+                                         __shfl_xor_sync(0xFFFFFFFFu, t[1], off),
+                                         __shfl_xor_sync(0xFFFFFFFFu, t[2], off)};
+        add192(t, o);
+    }
+    sticky = __reduce_or_sync(0xFFFFFFFFu, sticky);
+    if (lane == 0) {
+        wsum[warp][0] = t[0];
+        wsum[warp][1] = t[1];
+        wsum[warp][2] = t[2];
+        wsticky[warp] = sticky;
     }
     __syncthreads();
     if (tr == 0) {
-        const float sc = scale_from_totals(totals[sub], K, n, M);
+        unsigned long long tot[3] = {0ull, 0ull, 0ull};
+        uint32_t st = 0;
+#pragma unroll
+        for (int w = 0; w < WPR; ++w) {
+            const unsigned long long o[3] = {wsum[sub * WPR + w][0], wsum[sub * WPR + w][1], wsum[sub * WPR + w][2]};
+            add192(tot, o);
+            st |= wsticky[sub * WPR + w];
+        }
+        const double sum = window_to_double(tot, st != 0, base);
+        const double kept = static_cast<double>((K / M) * n);
+        const float sc = fmaxf(__double2float_rn(__ddiv_rn(sum, kept)), 1e-5f);
         scales[sub] = sc;
         if (valid) row_scale[row] = sc;
     }
