@@ -143,6 +143,36 @@ sbl_status sbl_linear_path(const uint16_t* x_bf16, int64_t T, int64_t K,
                            void* y, int y_dtype, int32_t* acc_out,
                            void* workspace, size_t workspace_bytes, int path, void* stream);
 
+/*
+ * sbl_linear_noalloc — sbl_linear for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart for this entry point; it serves callers that
+ * cannot provide a workspace: a plugin whose host application owns the whole
+ * device-memory budget, a plain C caller with no allocator of its own, or a
+ * latency-critical path where an allocation could synchronise the device.
+ *
+ * Same arguments and results as sbl_linear, minus the workspace.  The scratch
+ * (quantised activations and per-token scales) lives in one array of
+ * SBL_NOALLOC_SCRATCH_BYTES of static device memory inside the library, which
+ * every GPU that loads the library holds until the process exits.  The call
+ * allocates nothing.
+ *   - Calls needing more scratch than the array holds, i.e.
+ *     sbl_linear_workspace_bytes(T, K, O, n, m) > SBL_NOALLOC_SCRATCH_BYTES
+ *     (T * K + 4 * T bytes, each rounded up to 256: T = 1024 fits at
+ *     K = 7168 but not at K = 8192), return SBL_ERR_WORKSPACE and enqueue
+ *     nothing.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls on a device share the one array: calls that may overlap on the
+ *     GPU (different streams without ordering between them) race on it and
+ *     give wrong results.  Order them on one stream.
+ */
+#define SBL_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+sbl_status sbl_linear_noalloc(const uint16_t* x_bf16, int64_t T, int64_t K,
+                              const uint8_t* packed, const float* row_scale, int64_t O, int n, int m,
+                              void* y, int y_dtype, int32_t* acc_out, void* stream);
+
 /* Largest T that sbl_linear sends to the decode path. */
 int64_t sbl_decode_max_tokens(void);
 
