@@ -6,14 +6,14 @@
 // equation); per-row absmean from the halo-sparse-bitnet-3:4-500m card,
 // "Recipe"; code table 00 = 0, 01 = +1, 10 = -1 from its "Packed vs raw".
 //
-// TPR threads share a row (256 / TPR rows per block); each thread owns up to
-// two 16-weight chunks, read once as 16-byte loads and kept in registers.
-// Pass 1 builds the keep-mask of every group and adds the kept |w| exactly
-// into a register window anchored at the row's largest kept magnitude (see
-// kWindow); after a block-wide reduction of the row sums, pass 2 ternarises
-// the registers against the row scale and writes one 32-bit word of codes and
-// 16 mask bits per chunk.  Rows longer than 512 chunks (K > 8192) use a
-// warp-per-row variant that reads the row twice and sums in shared-memory limbs.
+// One to eight warps share a row; each thread owns up to two 16-weight chunks,
+// read once as 16-byte loads and kept in registers.  Pass 1 applies the N:M
+// mask to the registers and finds the row's largest and smallest kept
+// magnitudes, pass 2 adds the kept |w| exactly (see kWin), pass 3 ternarises
+// the registers against the row scale and writes one 32-bit word of codes
+// (and optionally 16 mask bits) per chunk.  Rows longer than 512 chunks
+// (K > 8192) use a warp-per-row variant that reads the row twice and sums in
+// shared-memory limbs.
 //
 // Exact sum: a finite float |w| = m * 2^(p - 149) with a 24-bit integer m and
 // 0 <= p <= 253, so the row sum is an integer in units of 2^-149 below 2^300.
@@ -184,61 +184,66 @@ __global__ void __launch_bounds__(kPrepWarps * 32) prep_kernel(const float* __re
     }
 }
 
-constexpr int kPrepThreads = 256;
+// ---------------------------------------------------------------------------
+// Register-resident variant: each thread owns two 16-weight chunks of a row,
+// WPR warps share a row and a block holds 8 / WPR rows.
+//
+// Exact row sum.  A finite float is |w| = m * 2^(e - 150) with e its biased
+// exponent field (normal values; m < 2^24).  With e_max that of the row's
+// largest magnitude and e_b = e_max - kWin, every kept value with e >= e_b is
+// an integer below 2^(24 + kWin) in units of 2^(e_b - 150); a thread adds at
+// most 32 of them, so the sum stays below 2^53 and accumulates in a double
+// without rounding (one fused multiply-add by the power of two 2^(150 - e_b)
+// per weight).  Thread sums are then added as 64-bit integers.  When
+// e_b <= 0 every value of the row, subnormals included, is such an integer.
+// A row in which a kept nonzero magnitude lies below 2^(e_b - 127) is summed
+// instead with exact 320-bit shared-memory limbs; which rows do is known from
+// the row minimum before any summing.
+constexpr int kWin = 24;
+constexpr int kChunksPerThread = 2;
 
-// Exact row sums in registers.  With p_max the largest exponent index among the
-// row's kept magnitudes (|w| = m * 2^(p - 149), m < 2^24), every kept value
-// with p >= base = p_max - 96 is added exactly into a 128-bit per-thread
-// accumulator in units of 2^(base - 149) (a value is below 2^120 there and a
-// thread adds at most 32 of them); smaller values only set a sticky flag.
-// Their total is below 2^24 * 2^base, at least 2^40 times smaller than the
-// rounding position of a double holding the sum (which is >= 2^(p_max + 23)),
-// so the 192-bit row total plus the sticky flag rounds to the same double as
-// the exact sum.
-constexpr int kWindow = 96;
+// Bit 31 is set exactly when a >= b (both below 2^31).
+__device__ __forceinline__ uint32_t ge_bit(uint32_t a, uint32_t b) { return b - a - 1u; }
 
-__device__ __forceinline__ void add128(unsigned long long& w0, unsigned long long& w1, unsigned long long a0,
-                                       unsigned long long a1) {
-    asm("add.cc.u64 %0, %0, %2;\n\taddc.u64 %1, %1, %3;" : "+l"(w0), "+l"(w1) : "l"(a0), "l"(a1));
-}
-
-__device__ __forceinline__ void add192(unsigned long long (&w)[3], const unsigned long long (&a)[3]) {
-    asm("add.cc.u64 %0, %0, %3;\n\taddc.cc.u64 %1, %1, %4;\n\taddc.u64 %2, %2, %5;"
-        : "+l"(w[0]), "+l"(w[1]), "+l"(w[2])
-        : "l"(a[0]), "l"(a[1]), "l"(a[2]));
-}
-
-// Round w[0..2] * 2^(base - 149) (+ a sticky remainder) to double.
-__device__ double window_to_double(const unsigned long long (&w)[3], bool sticky, int base) {
-    int h = 2;
-    while (h >= 0 && w[h] == 0ull) --h;
-    if (h < 0) return 0.0;  // sticky alone cannot happen: dropped values are nonzero only next to larger ones
-    const int lz = __clzll(w[h]);
-    unsigned long long top = w[h] << lz;
-    unsigned long long rest = 0;  // bits below `top`
-    if (h >= 1) {
-        if (lz) top |= w[h - 1] >> (64 - lz);
-        rest = w[h - 1] << lz;
-        if (lz == 0) rest = w[h - 1];
-        if (h == 2) rest |= w[0];
+// Drop flags (bit 31) of one group of four magnitudes, ties going to the lower
+// index: a weight is dropped when it loses to at least N of the other three
+// (N = 3: to all three; N = 2: to two or more).
+template <int N>
+__device__ __forceinline__ void drop4(const uint32_t* a, uint32_t (&d)[4]) {
+    const uint32_t g01 = ge_bit(a[0], a[1]), g02 = ge_bit(a[0], a[2]), g03 = ge_bit(a[0], a[3]);
+    const uint32_t g12 = ge_bit(a[1], a[2]), g13 = ge_bit(a[1], a[3]), g23 = ge_bit(a[2], a[3]);
+    // losses: 0 loses to k when !g0k; 1 loses to 0 when g01, to k > 1 when !g1k; ...
+    if constexpr (N == 3) {
+        d[0] = ~g01 & ~g02 & ~g03;
+        d[1] = g01 & ~g12 & ~g13;
+        d[2] = g02 & g12 & ~g23;
+        d[3] = g03 & g13 & g23;
+    } else {
+        d[0] = (~g01 & ~g02) | (~g01 & ~g03) | (~g02 & ~g03);
+        d[1] = (g01 & ~g12) | (g01 & ~g13) | (~g12 & ~g13);
+        d[2] = (g02 & g12) | (g02 & ~g23) | (g12 & ~g23);
+        d[3] = (g03 & g13) | (g03 & g23) | (g13 & g23);
     }
-    if (rest || sticky) top |= 1ull;  // sticky bit: below the rounding position
-    const int e2 = 64 * h + (64 - lz) - 64 + base - 149;  // weight of bit 0 of `top`
-    const double scale = __longlong_as_double(static_cast<long long>(1023 + e2) << 52);
-    return __ull2double_rn(top) * scale;
 }
 
-template <int M, int TPR>
-__global__ void __launch_bounds__(kPrepThreads) prep_kernel_rr(const float* __restrict__ W, long long O,
-                                                               long long K, int n, uint8_t* __restrict__ packed,
-                                                               float* __restrict__ row_scale,
-                                                               uint8_t* __restrict__ mask_bits, unsigned* status) {
-    constexpr int RPB = kPrepThreads / TPR;  // rows per block
-    constexpr int CPT = 2;                   // chunks per thread
-    constexpr int WPR = TPR / 32;            // warps per row
-    __shared__ uint32_t wmax[kPrepThreads / 32];
-    __shared__ unsigned long long wsum[kPrepThreads / 32][3];
-    __shared__ uint32_t wsticky[kPrepThreads / 32];
+template <int WPR>
+__device__ __forceinline__ void row_sync() {
+    if constexpr (WPR == 1) __syncwarp();
+    else __syncthreads();
+}
+
+template <int M, int N, int WPR, bool WITH_MASK>
+__global__ void __launch_bounds__((8 / WPR) * WPR * 32) prep_kernel_rr(const float* __restrict__ W, long long O,
+                                                                      long long K, uint8_t* __restrict__ packed,
+                                                                      float* __restrict__ row_scale,
+                                                                      uint8_t* __restrict__ mask_bits,
+                                                                      unsigned* status) {
+    constexpr int RPB = 8 / WPR;  // rows per block
+    constexpr int TPR = WPR * 32;
+    constexpr int CPT = kChunksPerThread;
+    __shared__ uint32_t wmax[RPB * WPR], wmin[RPB * WPR];
+    __shared__ unsigned long long wsum[RPB * WPR];
+    __shared__ unsigned long long limbs[RPB][kLimbs];
     __shared__ float scales[RPB];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int sub = threadIdx.x / TPR, tr = threadIdx.x % TPR;
@@ -247,145 +252,212 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel_rr(const float* __re
     const int nchunks = static_cast<int>(K >> 4);
     const float* wr = W + (valid ? row : 0) * K;
 
-    uint32_t raw[CPT][16];
+    // kr: the weight's bits when it is kept, 0 when it is dropped
+    uint32_t kr[CPT][16];
 #pragma unroll
     for (int j = 0; j < CPT; ++j) {
         const int c = tr + TPR * j;
-        if (valid && c < nchunks) load_chunk(wr + 16 * c, raw[j]);
+        if (valid && c < nchunks) load_chunk(wr + 16 * c, kr[j]);
         else
 #pragma unroll
-            for (int i = 0; i < 16; ++i) raw[j][i] = 0u;
+            for (int i = 0; i < 16; ++i) kr[j][i] = 0u;
     }
 
-    // keep-masks, non-finite check and the largest kept magnitude of the row
-    bool bad = false;
-    uint32_t keep[CPT];
-    uint32_t mx = 0;
+    // pass 1: N:M mask, row maximum of |w|, row minimum of the kept nonzero |w|
+    uint32_t mx = 0, mn2 = 0xFFFFFFFFu, kbits = 0;
 #pragma unroll
     for (int j = 0; j < CPT; ++j) {
-        uint32_t a[16];
+        if constexpr (M == 4) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            a[i] = raw[j][i] & 0x7FFFFFFFu;
-            bad |= a[i] >= 0x7F800000u;
+            for (int g = 0; g < 4; ++g) {
+                uint32_t a[4], d[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    a[q] = kr[j][4 * g + q] & 0x7FFFFFFFu;
+                    mx = max(mx, a[q]);
+                }
+                drop4<N>(a, d);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    kr[j][4 * g + q] &= ~static_cast<uint32_t>(static_cast<int>(d[q]) >> 31);
+                    if constexpr (WITH_MASK) kbits |= ((~d[q]) >> 31) << (16 * j + 4 * g + q);
+                }
+            }
+        } else {
+            uint32_t a[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                a[i] = kr[j][i] & 0x7FFFFFFFu;
+                mx = max(mx, a[i]);
+            }
+            const uint32_t keep = group_keep_bits<8>(a, N) | (group_keep_bits<8>(a + 8, N) << 8);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) kr[j][i] = ((keep >> i) & 1u) ? kr[j][i] : 0u;
+            if constexpr (WITH_MASK) kbits |= keep << (16 * j);
         }
-        keep[j] = chunk_keep_bits<M>(a, n);
-        const int c = tr + TPR * j;
-        if (!(valid && c < nchunks)) keep[j] = 0u;
+        // 2|w| - 1 over the kept weights: zeros wrap to the largest value
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-            if (keep[j] & (1u << i)) mx = max(mx, a[i]);
+        for (int i = 0; i < 16; ++i) mn2 = min(mn2, (kr[j][i] << 1) - 1u);
     }
     mx = __reduce_max_sync(0xFFFFFFFFu, mx);
-    if (lane == 0) wmax[warp] = mx;
-    if (__syncthreads_or(bad ? 1 : 0) && threadIdx.x == 0) raise_status(status, kStatusNonfinite);
-#pragma unroll
-    for (int w = 0; w < WPR; ++w) mx = max(mx, wmax[sub * WPR + w]);
-    const int emax = static_cast<int>(mx >> 23);
-    const int base = (emax ? emax - 1 : 0) - kWindow;
-
-    // exact accumulation of the kept magnitudes
-    unsigned long long w0 = 0, w1 = 0;
-    uint32_t sticky = 0;
-#pragma unroll
-    for (int j = 0; j < CPT; ++j)
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            if (!(keep[j] & (1u << i))) continue;
-            const uint32_t a = raw[j][i] & 0x7FFFFFFFu;
-            const uint32_t e = a >> 23;
-            const uint32_t m24 = (a & 0x7FFFFFu) | (e ? 0x800000u : 0u);
-            const int sh = (e ? static_cast<int>(e) - 1 : 0) - base;  // <= kWindow
-            if (sh < 0) {
-                sticky |= m24;
-            } else {
-                const int bit = sh & 63;
-                const unsigned long long v = static_cast<unsigned long long>(m24) << bit;
-                const unsigned long long hi = bit > 40 ? static_cast<unsigned long long>(m24) >> (64 - bit) : 0ull;
-                if (sh < 64) add128(w0, w1, v, hi);
-                else add128(w0, w1, 0ull, v);
-            }
+    mn2 = __reduce_min_sync(0xFFFFFFFFu, mn2);
+    if constexpr (WPR > 1) {
+        if (lane == 0) {
+            wmax[warp] = mx;
+            wmin[warp] = mn2;
         }
-
-    // row total: warp butterfly on 192 bits, then the row's warps
-    unsigned long long t[3] = {w0, w1, 0ull};
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-        const unsigned long long o[3] = {__shfl_xor_sync(0xFFFFFFFFu, t[0], off),
-                                         __shfl_xor_sync(0xFFFFFFFFu, t[1], off),
-                                         __shfl_xor_sync(0xFFFFFFFFu, t[2], off)};
-        add192(t, o);
-    }
-    sticky = __reduce_or_sync(0xFFFFFFFFu, sticky);
-    if (lane == 0) {
-        wsum[warp][0] = t[0];
-        wsum[warp][1] = t[1];
-        wsum[warp][2] = t[2];
-        wsticky[warp] = sticky;
-    }
-    __syncthreads();
-    if (tr == 0) {
-        unsigned long long tot[3] = {0ull, 0ull, 0ull};
-        uint32_t st = 0;
+        __syncthreads();
 #pragma unroll
         for (int w = 0; w < WPR; ++w) {
-            const unsigned long long o[3] = {wsum[sub * WPR + w][0], wsum[sub * WPR + w][1], wsum[sub * WPR + w][2]};
-            add192(tot, o);
-            st |= wsticky[sub * WPR + w];
+            mx = max(mx, wmax[sub * WPR + w]);
+            mn2 = min(mn2, wmin[sub * WPR + w]);
         }
-        const double sum = window_to_double(tot, st != 0, base);
-        const double kept = static_cast<double>((K / M) * n);
-        const float sc = fmaxf(__double2float_rn(__ddiv_rn(sum, kept)), 1e-5f);
-        scales[sub] = sc;
-        if (valid) row_scale[row] = sc;
     }
-    __syncthreads();
+    if (mx >= 0x7F800000u && tr == 0 && valid) raise_status(status, kStatusNonfinite);
+    const int emax = static_cast<int>(mx >> 23);
+    const int eb = emax - kWin;
+    // a kept nonzero magnitude below 2^(eb - 127) leaves the window
+    const bool exact_path = eb >= 1 && mn2 < (static_cast<uint32_t>(eb) << 24) - 1u;
+
+    // pass 2: the sum of the kept |w|
+    double sum;
+    bool any_exact;
+    if constexpr (WPR == 1) any_exact = exact_path;  // warp-uniform
+    else any_exact = __syncthreads_or(exact_path);
+    if (!exact_path) {
+        const double up = __longlong_as_double(static_cast<long long>(1023 + 150 - eb) << 52);  // 2^(150 - eb)
+        double acc = 0.0;
+#pragma unroll
+        for (int j = 0; j < CPT; ++j)
+#pragma unroll
+            for (int i = 0; i < 16; ++i) acc = fma(static_cast<double>(fabsf(__uint_as_float(kr[j][i]))), up, acc);
+        unsigned long long t = __double2ull_rn(acc);  // an integer below 2^53
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) t += __shfl_xor_sync(0xFFFFFFFFu, t, off);
+        if constexpr (WPR > 1) {
+            if (lane == 0) wsum[warp] = t;
+        } else {
+            // units of 2^(eb - 150); the row total is below 2^61
+            sum = __ull2double_rn(t) * __longlong_as_double(static_cast<long long>(1023 + eb - 150) << 52);
+        }
+    }
+    if (any_exact) {
+        // exact 320-bit limbs (units of 2^-149), integer adds in any order
+        if (tr < kLimbs) limbs[sub][tr] = 0ull;
+        row_sync<WPR>();
+        if (exact_path) {
+#pragma unroll
+            for (int j = 0; j < CPT; ++j)
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const uint32_t a = kr[j][i] & 0x7FFFFFFFu;
+                    if (a == 0u) continue;
+                    const uint32_t e = a >> 23;
+                    const uint32_t m24 = (a & 0x7FFFFFu) | (e ? 0x800000u : 0u);
+                    const uint32_t p = e ? e - 1u : 0u;
+                    const unsigned long long v = static_cast<unsigned long long>(m24) << (p & 31u);
+                    atomicAdd(&limbs[sub][p >> 5], v & 0xFFFFFFFFull);
+                    atomicAdd(&limbs[sub][(p >> 5) + 1], v >> 32);
+                }
+        }
+        row_sync<WPR>();
+        if (exact_path && (WPR == 1 || tr == 0)) {
+            uint32_t w32[kLimbs];
+            unsigned long long carry = 0;
+#pragma unroll
+            for (int i = 0; i < kLimbs; ++i) {
+                const unsigned long long v = limbs[sub][i] + carry;
+                w32[i] = static_cast<uint32_t>(v);
+                carry = v >> 32;
+            }
+            sum = limbs_to_double(w32);
+        }
+    } else if constexpr (WPR > 1) {
+        __syncthreads();
+    }
+    float sc;
+    const double kept = static_cast<double>((K / M) * N);
+    if constexpr (WPR > 1) {
+        if (tr == 0) {
+            if (!exact_path) {
+                unsigned long long tot = 0;
+#pragma unroll
+                for (int w = 0; w < WPR; ++w) tot += wsum[sub * WPR + w];
+                sum = __ull2double_rn(tot) * __longlong_as_double(static_cast<long long>(1023 + eb - 150) << 52);
+            }
+            sc = fmaxf(__double2float_rn(__ddiv_rn(sum, kept)), 1e-5f);
+            scales[sub] = sc;
+            if (valid) row_scale[row] = sc;
+        }
+        __syncthreads();
+        sc = scales[sub];
+    } else {
+        sc = fmaxf(__double2float_rn(__ddiv_rn(sum, kept)), 1e-5f);
+        if (lane == 0 && valid) row_scale[row] = sc;
+    }
     if (!valid) return;
-    const uint32_t half_bits = __float_as_uint(0.5f * scales[sub]);  // exact: scale >= 1e-5 is normal
+
+    // pass 3: ternarise and pack.  round(w / scale) != 0 exactly when
+    // |w| > scale / 2, an exact compare (scale >= 1e-5 is normal, so halving
+    // it is exact); the code is 01 for +1 and 10 for -1.
+    const uint32_t half_bits = __float_as_uint(0.5f * sc);
     uint32_t* prow = reinterpret_cast<uint32_t*>(packed + row * (K >> 2));
-    uint16_t* mrow = mask_bits ? reinterpret_cast<uint16_t*>(mask_bits + row * (K >> 3)) : nullptr;
+    uint16_t* mrow = WITH_MASK ? reinterpret_cast<uint16_t*>(mask_bits + row * (K >> 3)) : nullptr;
 #pragma unroll
     for (int j = 0; j < CPT; ++j) {
         const int c = tr + TPR * j;
         if (c >= nchunks) continue;
-        uint32_t codes = 0;
+        uint32_t nzw = 0, sgw = 0;  // nonzero flags at bits 2i, signs at bits 2i + 1
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-            // round(w / scale) != 0  <=>  |w| / scale > 1/2  <=>  |w| > scale / 2 (exact compare)
-            const bool nz = ((keep[j] >> i) & 1u) && ((raw[j][i] & 0x7FFFFFFFu) > half_bits);
-            codes |= (nz ? ((raw[j][i] >> 31) ? 2u : 1u) : 0u) << (2 * i);
+            const uint32_t t = half_bits - (kr[j][i] & 0x7FFFFFFFu);  // bit 31: |w| > scale / 2
+            nzw |= (t >> (31 - 2 * i)) & (1u << (2 * i));
+            sgw |= (kr[j][i] >> (30 - 2 * i)) & (2u << (2 * i));
         }
-        prow[c] = codes;
-        if (mrow) mrow[c] = static_cast<uint16_t>(keep[j]);
+        prow[c] = (nzw & ~(sgw >> 1)) | ((nzw << 1) & sgw);
+        if constexpr (WITH_MASK) mrow[c] = static_cast<uint16_t>(kbits >> (16 * j));
     }
 }
 
-template <int M, int TPR>
-static void launch_prep_rr(const float* W, long long O, long long K, int n, uint8_t* packed, float* row_scale,
+template <int M, int N, int WPR>
+static void launch_prep_rr(const float* W, long long O, long long K, uint8_t* packed, float* row_scale,
                            uint8_t* mask_bits, unsigned* status, cudaStream_t stream) {
-    constexpr int RPB = kPrepThreads / TPR;
+    constexpr int RPB = 8 / WPR;
     const unsigned blocks = static_cast<unsigned>((O + RPB - 1) / RPB);
-    prep_kernel_rr<M, TPR><<<blocks, kPrepThreads, 0, stream>>>(W, O, K, n, packed, row_scale, mask_bits, status);
+    if (mask_bits)
+        prep_kernel_rr<M, N, WPR, true><<<blocks, RPB * WPR * 32, 0, stream>>>(W, O, K, packed, row_scale, mask_bits,
+                                                                              status);
+    else
+        prep_kernel_rr<M, N, WPR, false><<<blocks, RPB * WPR * 32, 0, stream>>>(W, O, K, packed, row_scale, nullptr,
+                                                                               status);
 }
 
-template <int M>
-static void launch_prep_m(const float* W, long long O, long long K, int n, uint8_t* packed, float* row_scale,
-                          uint8_t* mask_bits, unsigned* status, cudaStream_t stream) {
-    const long long nchunks = K >> 4;
-    if (nchunks <= 64) launch_prep_rr<M, 32>(W, O, K, n, packed, row_scale, mask_bits, status, stream);
-    else if (nchunks <= 128) launch_prep_rr<M, 64>(W, O, K, n, packed, row_scale, mask_bits, status, stream);
-    else if (nchunks <= 256) launch_prep_rr<M, 128>(W, O, K, n, packed, row_scale, mask_bits, status, stream);
-    else if (nchunks <= 512) launch_prep_rr<M, 256>(W, O, K, n, packed, row_scale, mask_bits, status, stream);
-    else {
-        const unsigned blocks = static_cast<unsigned>((O + kPrepWarps - 1) / kPrepWarps);
-        prep_kernel<M><<<blocks, kPrepWarps * 32, 0, stream>>>(W, O, K, n, packed, row_scale, mask_bits, status);
+template <int M, int N>
+static void launch_prep_mn(const float* W, long long O, long long K, uint8_t* packed, float* row_scale,
+                           uint8_t* mask_bits, unsigned* status, cudaStream_t stream) {
+    // warps per row: the fewest that give every 16-weight chunk a slot
+    const long long wpr = ((K >> 4) + 32 * kChunksPerThread - 1) / (32 * kChunksPerThread);
+    switch (wpr) {
+        case 1: launch_prep_rr<M, N, 1>(W, O, K, packed, row_scale, mask_bits, status, stream); break;
+        case 2: launch_prep_rr<M, N, 2>(W, O, K, packed, row_scale, mask_bits, status, stream); break;
+        case 3: launch_prep_rr<M, N, 3>(W, O, K, packed, row_scale, mask_bits, status, stream); break;
+        case 4: launch_prep_rr<M, N, 4>(W, O, K, packed, row_scale, mask_bits, status, stream); break;
+        case 5: launch_prep_rr<M, N, 5>(W, O, K, packed, row_scale, mask_bits, status, stream); break;
+        case 6: launch_prep_rr<M, N, 6>(W, O, K, packed, row_scale, mask_bits, status, stream); break;
+        case 7: launch_prep_rr<M, N, 7>(W, O, K, packed, row_scale, mask_bits, status, stream); break;
+        case 8: launch_prep_rr<M, N, 8>(W, O, K, packed, row_scale, mask_bits, status, stream); break;
+        default: {
+            const unsigned blocks = static_cast<unsigned>((O + kPrepWarps - 1) / kPrepWarps);
+            prep_kernel<M><<<blocks, kPrepWarps * 32, 0, stream>>>(W, O, K, N, packed, row_scale, mask_bits, status);
+        }
     }
 }
 
 cudaError_t launch_prep(const float* W, long long O, long long K, int n, int m, uint8_t* packed, float* row_scale,
                         uint8_t* mask_bits, unsigned* status, cudaStream_t stream) {
-    if (m == 4) launch_prep_m<4>(W, O, K, n, packed, row_scale, mask_bits, status, stream);
-    else launch_prep_m<8>(W, O, K, n, packed, row_scale, mask_bits, status, stream);
+    if (m == 4 && n == 2) launch_prep_mn<4, 2>(W, O, K, packed, row_scale, mask_bits, status, stream);
+    else if (m == 4) launch_prep_mn<4, 3>(W, O, K, packed, row_scale, mask_bits, status, stream);
+    else launch_prep_mn<8, 6>(W, O, K, packed, row_scale, mask_bits, status, stream);
     return cudaGetLastError();
 }
 

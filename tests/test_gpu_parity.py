@@ -76,6 +76,32 @@ def test_prepare_extreme_magnitudes(sbl):
         assert np.array_equal(w.packed.cpu().numpy(), packed)
 
 
+def test_prepare_window_boundaries(sbl):
+    # Kept magnitudes placed at chosen binade distances d below each row's
+    # largest one (d = 0 ... 200, both sides of 35/36 and 71/72, subnormals),
+    # and a row whose exact sum is a double rounding tie broken only by a value
+    # 100 binades down: the row scale must still be the exactly rounded mean.
+    rng = np.random.default_rng(11)
+    O, K = 96, 64
+    dists = [0, 1, 23, 24, 34, 35, 36, 37, 47, 48, 70, 71, 72, 73, 100, 200]
+    W = np.zeros((O, K), dtype=np.float32)
+    for r in range(O - 1):
+        p_max = int(rng.integers(0, 254))
+        W[r, 0] = np.float32(np.ldexp(float(rng.integers(1 << 23, 1 << 24)), p_max - 149))
+        for g in range(1, K // 4):
+            p = p_max - int(rng.choice(dists))
+            if p >= 0:
+                mant = int(rng.integers(1 << 23, 1 << 24)) if p > 0 else int(rng.integers(1, 1 << 23))
+                W[r, 4 * g] = np.float32(np.ldexp(float(mant), p - 149)) * np.float32(rng.choice([-1, 1]))
+    W[O - 1, 0], W[O - 1, 4], W[O - 1, 8] = 1.0, np.float32(2.0 ** -53), np.float32(2.0 ** -100)
+    for n, m in PATTERNS:
+        w = _prep(sbl, W, n, m)
+        packed, scale, mbits, _ = oracle.prepare_weights(W, n, m)
+        assert np.array_equal(w.row_scale.cpu().numpy().view(np.uint32), scale.view(np.uint32))
+        assert np.array_equal(w.packed.cpu().numpy(), packed)
+        assert np.array_equal(w.mask_bits.cpu().numpy(), mbits)
+
+
 # ------------------------------------------------------------------ activation quant
 
 @pytest.mark.parametrize("T,K,p", [(16, 256, 0.0), (3, 48, 0.0), (257, 896, 0.01), (64, 4864, 0.01)])
