@@ -49,8 +49,11 @@ typedef enum {
 /* Output element types of sbl_linear. */
 enum { SBL_F32 = 0, SBL_BF16 = 1 };
 
-/* Contraction paths of sbl_linear_path. */
-enum { SBL_PATH_AUTO = 0, SBL_PATH_DECODE = 1, SBL_PATH_PREFILL = 2 };
+/* Contraction paths of sbl_linear_path.  SBL_PATH_PREFILL lets the library
+ * pick the tensor-core kernel; the last two force one of them (tests, tuning):
+ * one CTA per 128-token tile, or a pair of CTAs on two SMs per 256-token tile. */
+enum { SBL_PATH_AUTO = 0, SBL_PATH_DECODE = 1, SBL_PATH_PREFILL = 2,
+       SBL_PATH_PREFILL_1CTA = 3, SBL_PATH_PREFILL_PAIR = 4 };
 
 /*
  * sbl_prepare_weights — N:M mask, per-row scale, ternarise and 2-bit pack.
@@ -135,8 +138,9 @@ sbl_status sbl_linear(const uint16_t* x_bf16, int64_t T, int64_t K,
 
 /*
  * sbl_linear_path — sbl_linear with the contraction path forced
- * (SBL_PATH_DECODE or SBL_PATH_PREFILL; SBL_PATH_AUTO is sbl_linear).
- * SBL_PATH_PREFILL with K % 64 != 0 returns SBL_ERR_UNSUPPORTED.
+ * (SBL_PATH_DECODE, or one of the SBL_PATH_PREFILL* tensor-core paths;
+ * SBL_PATH_AUTO is sbl_linear).  Every path gives the same results.
+ * A prefill path with K % 64 != 0 returns SBL_ERR_UNSUPPORTED.
  */
 sbl_status sbl_linear_path(const uint16_t* x_bf16, int64_t T, int64_t K,
                            const uint8_t* packed, const float* row_scale, int64_t O, int n, int m,

@@ -26,6 +26,8 @@ SBL_BF16 = 1
 SBL_PATH_AUTO = 0
 SBL_PATH_DECODE = 1
 SBL_PATH_PREFILL = 2
+SBL_PATH_PREFILL_1CTA = 3
+SBL_PATH_PREFILL_PAIR = 4
 
 # name -> (restype, argtypes); mirrors include/sbl.h
 _vp, _i64, _int, _sz, _u32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint32

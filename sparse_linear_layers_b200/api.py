@@ -14,7 +14,8 @@ import torch
 from . import _lib
 from ._lib import check, lib
 
-_PATHS = {"auto": _lib.SBL_PATH_AUTO, "decode": _lib.SBL_PATH_DECODE, "prefill": _lib.SBL_PATH_PREFILL}
+_PATHS = {"auto": _lib.SBL_PATH_AUTO, "decode": _lib.SBL_PATH_DECODE, "prefill": _lib.SBL_PATH_PREFILL,
+          "prefill_1cta": _lib.SBL_PATH_PREFILL_1CTA, "prefill_pair": _lib.SBL_PATH_PREFILL_PAIR}
 
 
 def _stream(stream: Optional[torch.cuda.Stream]) -> int:

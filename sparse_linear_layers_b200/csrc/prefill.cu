@@ -37,6 +37,7 @@
 #include <type_traits>
 
 #include "sbl_common.cuh"
+#include "tc_util.cuh"
 
 namespace sbl {
 
@@ -97,96 +98,6 @@ constexpr size_t prefill_smem_bytes() {
 }
 static_assert(prefill_smem_bytes<256>() <= 232448, "prefill tile does not fit in shared memory");
 static_assert(prefill_smem_bytes<128>() <= 232448, "prefill tile does not fit in shared memory");
-
-// UMMA shared-memory descriptor: K-major, 128-byte swizzle, 8-row groups 1024 B apart.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-    uint64_t d = static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-    d |= static_cast<uint64_t>(1u) << 16;            // leading byte offset (unused for this layout)
-    d |= static_cast<uint64_t>(1024u >> 4) << 32;    // stride byte offset
-    d |= static_cast<uint64_t>(1u) << 46;            // descriptor version
-    d |= static_cast<uint64_t>(2u) << 61;            // SWIZZLE_128B
-    return d;
-}
-
-// Instruction descriptor: s8 x s8 -> s32, both K-major, M = 128, N = BN.
-template <int BN>
-__device__ __forceinline__ uint32_t i8_idesc() {
-    return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
-           (static_cast<uint32_t>(pf::BM >> 4) << 24);
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-            dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-        : "memory");
-}
-
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(x), "r"(y), "r"(src)
-                 : "memory");
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory"); }
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-
-// One lane polls the barrier, the warp follows (fewer pollers on shared memory).
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-    bool ok = true;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag);
-    return __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
-}
-
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
-        : "memory");
-}
-
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
-__device__ __forceinline__ void st_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    asm volatile("st.global.v4.b32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
-}
 
 template <int BN>
 __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
@@ -439,7 +350,7 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
         // K = 32 MMAs, commit (releases the stage when the MMAs finish); per
         // tile: wait for a free accumulator buffer, commit it to the epilogue.
         if (lane == 0) {
-            const uint32_t idesc = i8_idesc<BN>();
+            const uint32_t idesc = i8_idesc<pf::BM, BN>();
             uint32_t it = 0;
             int tc = 0;
             bool ok = true;
@@ -479,22 +390,6 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(Cfg::TMEM_COLS)
                      : "memory");
     }
-}
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn get_encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
 }
 
 template <int BN>
@@ -569,16 +464,35 @@ cudaError_t set_prefill_trace(void* buf) {
 }
 #endif
 
+int prefill_pair_clusters(cudaStream_t stream);
+cudaError_t launch_prefill_pair(const int8_t* xperm, const float* s_tok, long long T, long long K,
+                                const uint8_t* packed, const float* row_scale, long long O, void* y, int y_bf16,
+                                int32_t* acc_out, unsigned* status, cudaStream_t stream);
+
 cudaError_t launch_prefill(const int8_t* xperm, const float* s_tok, long long T, long long K, const uint8_t* packed,
                            const float* row_scale, long long O, void* y, int y_bf16, int32_t* acc_out,
-                           unsigned* status, int num_sms, cudaStream_t stream) {
-    // Wide tiles (BN = 256) halve the activation traffic and the MMA issue
-    // overhead per output; narrow ones (BN = 128) fill more SMs when tiles are
-    // few.  Compare wave counts, a wide tile costing about two narrow ones.
+                           unsigned* status, int num_sms, int variant, cudaStream_t stream) {
+    // Cost model in units of one 128 x 256 tile on one SM: waves of tiles
+    // times the time of one tile.  A narrow 128 x 128 tile costs about 0.65
+    // of a wide one (BN = 256 halves the activation traffic and MMA issue
+    // overhead per output); a CTA pair finishes its 256 x 256 tile in about
+    // kPairCost of a wide one-CTA tile (half the expansion and shared-memory
+    // traffic per SM).
+    constexpr double kNarrowCost = 0.65, kPairCost = 0.65;
     const long long mt = (T + pf::BM - 1) / pf::BM;
-    const long long wide_waves = (mt * ((O + 255) / 256) + num_sms - 1) / num_sms;
-    const long long narrow_waves = (mt * ((O + 127) / 128) + num_sms - 1) / num_sms;
-    if (2.0 * wide_waves <= 1.3 * narrow_waves)
+    const double wide = static_cast<double>((mt * ((O + 255) / 256) + num_sms - 1) / num_sms);
+    const double narrow = kNarrowCost * static_cast<double>((mt * ((O + 127) / 128) + num_sms - 1) / num_sms);
+    bool pair = variant == 2;
+    if (variant == 0) {
+        const int clusters = prefill_pair_clusters(stream);
+        if (clusters > 0) {
+            const long long pt = ((T + 255) / 256) * ((O + 255) / 256);
+            pair = kPairCost * static_cast<double>((pt + clusters - 1) / clusters) < (wide < narrow ? wide : narrow);
+        }
+    }
+    if (pair)
+        return launch_prefill_pair(xperm, s_tok, T, K, packed, row_scale, O, y, y_bf16, acc_out, status, stream);
+    if (wide <= narrow)
         return launch_prefill_bn<256>(xperm, s_tok, T, K, packed, row_scale, O, y, y_bf16, acc_out, status, num_sms,
                                       stream);
     return launch_prefill_bn<128>(xperm, s_tok, T, K, packed, row_scale, O, y, y_bf16, acc_out, status, num_sms,

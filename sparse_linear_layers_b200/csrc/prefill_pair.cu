@@ -1,0 +1,468 @@
+// Prefill path on CTA pairs: acc[t, o] = sum_k x_q[t, k] * W_t[o, k] with
+// 2-SM tcgen05 MMAs (cta_group::2, kind::i8), then y = acc * scale_o / s_t.
+//
+// The contraction of the Sparse-BitNet Guide's linear-evaluation equation
+// ("Mathematical Formulation of Sparse-BitLinear"), for many tokens a dense
+// int8 matrix product.  A cluster of two CTAs (on two SMs) computes one
+// 256-token x 256-output tile per step of its persistent loop:
+//
+//   CTA rank r holds tokens 128r .. 128r + 127 of the tile (its half of A),
+//   output rows 128r .. 128r + 127 (its half of B: 2-bit codes loaded by TMA
+//   and expanded to int8 in its own shared memory) and, in its own tensor
+//   memory, the accumulators of its 128 tokens for all 256 outputs.  The
+//   even CTA issues the MMAs (M = 256, N = 256, K = 32), which read both
+//   CTAs' shared memory.
+//
+// Against one CTA computing a 128 x 256 tile, each SM now expands and stores
+// half as many weight bytes and its shared memory delivers half of B per MMA
+// instead of all of it; per 128-deep k-block an SM moves about 72 KB of
+// shared-memory traffic (activation tile written by TMA and read by the MMA,
+// code tile written and read, int8 weight half written and read) for the
+// same 128 x 256 x 128 multiply-adds that cost about 112 KB on one CTA.
+//
+// Warp roles in each CTA (320 threads):
+//   warps 0-3  epilogue: warp w owns TMEM lanes 32w .. 32w + 31 (32 tokens);
+//              pipelined tcgen05.ld, dequantise, 128B-swizzled staging
+//              boxes, TMA bulk stores
+//   warps 4-7  weight expansion: one thread per output row of the CTA's half
+//   warp 8     TMA producer (activation half-tile, code half-tile)
+//   warp 9     TMEM allocation (both CTAs) and, in the even CTA, MMA issue
+//
+// Barriers: the activation loads of both CTAs complete on the even CTA's
+// full_a; each CTA's code tile completes on its own full_c; the expansion
+// threads of both CTAs arrive on the even CTA's full_dec; MMA completion is
+// committed to empty / tmem_full / mma_done in both CTAs at once; the
+// epilogue threads of both CTAs arrive on the even CTA's tmem_empty.  Every
+// wait is bounded; a CTA that gives up records a timeout and winds down.
+#include <cuda.h>
+
+#include <type_traits>
+
+#include "sbl_common.cuh"
+#include "tc_util.cuh"
+
+namespace sbl {
+
+namespace pp {
+constexpr int BM = 128;                     // tokens per CTA (pair: 256)
+constexpr int BN = 256;                     // outputs per pair tile
+constexpr int BNH = BN / 2;                 // output rows held by one CTA
+constexpr int BK = 128;                     // k per stage (bytes of int8)
+constexpr int A_BYTES = BM * BK;
+constexpr int B_BYTES = BNH * BK;
+constexpr int P_BYTES = BNH * BK / 4;       // 2-bit codes of the CTA's half of B
+constexpr int STAGES = 5;
+constexpr int EPI_WARPS = 4;
+constexpr int DEC_WARPS = BNH / 32;
+constexpr int WARP_TMA = EPI_WARPS + DEC_WARPS;
+constexpr int WARP_MMA = WARP_TMA + 1;
+constexpr int THREADS = (WARP_MMA + 1) * 32;
+constexpr int TMEM_COLS = 2 * BN;           // two accumulator buffers
+constexpr int Y_BYTES = 32 * 128;           // one warp's staging box: 32 tokens x 128 bytes
+}  // namespace pp
+
+struct PairSmem {
+    uint8_t a[pp::STAGES][pp::A_BYTES];     // 1024-byte aligned tiles
+    uint8_t b[pp::STAGES][pp::B_BYTES];
+    uint8_t p[pp::STAGES][pp::P_BYTES];
+    uint8_t ystage[pp::EPI_WARPS][2][pp::Y_BYTES];
+    float wscale[pp::EPI_WARPS][pp::BN];
+    uint64_t full_a[pp::STAGES];            // used in the even CTA
+    uint64_t full_c[pp::STAGES];
+    uint64_t full_dec[pp::STAGES];          // used in the even CTA
+    uint64_t empty[pp::STAGES];
+    uint64_t tmem_full[2];
+    uint64_t tmem_empty[2];                 // used in the even CTA
+    uint64_t mma_done;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+constexpr size_t pair_smem_bytes() { return sizeof(PairSmem) + 1024; }
+static_assert(pair_smem_bytes() <= 232448, "pair prefill tile does not fit in shared memory");
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
+    prefill_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                        const __grid_constant__ CUtensorMap tmap_y, int y_vec, const float* __restrict__ row_scale,
+                        const float* __restrict__ s_tok, int T, int O, int K, void* __restrict__ y, int y_bf16,
+                        int32_t* __restrict__ acc_out, unsigned* status) {
+    extern __shared__ uint8_t smem_raw[];
+    auto* sm = reinterpret_cast<PairSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    volatile int* abort_flag = &sm->abort_flag;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int MT = (T + 2 * pp::BM - 1) / (2 * pp::BM);
+    const int NT = (O + pp::BN - 1) / pp::BN;
+    const int tiles = MT * NT;
+    const int KB = (K + pp::BK - 1) / pp::BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < pp::STAGES; ++s) {
+            mbar_init(&sm->full_a[s], 1);
+            mbar_init(&sm->full_c[s], 1);
+            mbar_init(&sm->full_dec[s], 2 * pp::DEC_WARPS);  // one arrival per expansion warp
+            mbar_init(&sm->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm->tmem_full[b], 1);
+            mbar_init(&sm->tmem_empty[b], 2 * pp::EPI_WARPS);  // one arrival per epilogue warp
+        }
+        mbar_init(&sm->mma_done, 1);
+        sm->abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == pp::WARP_MMA) {
+        // the same warp of both CTAs, the same destination offset
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm->tmem_base)),
+                     "r"(pp::TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    cluster_sync();  // barriers of both CTAs initialised, tensor memory allocated
+    tc_fence_after();
+    const uint32_t tmem_base = sm->tmem_base;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    auto give_up = [&]() {
+        if (!*abort_flag) {
+            *abort_flag = 1;
+            raise_status(status, kStatusTimeout);
+        }
+    };
+    // arrive on the even CTA's copy of a barrier
+    auto arrive_leader = [&](uint64_t* bar) {
+        if (leader) mbar_arrive(bar);
+        else mbar_arrive_cluster(map_to_cta(smem_u32(bar), 0));
+    };
+
+    if (warp < pp::EPI_WARPS) {
+        // ------------------------------------------------------------ epilogue
+        // As in the one-CTA kernel: per tile the warp copies the 256 row scales
+        // into its shared-memory slice, waits for the accumulator, then walks
+        // the 32-column TMEM slices with the next one in flight, dequantises
+        // and stores 128 output bytes per token per round through a staging box.
+        // The buffer is handed back to the even CTA's MMA issuer once read.
+        auto run = [&](auto bf16_tag) {
+            constexpr bool BF = decltype(bf16_tag)::value;
+            constexpr int SPR = BF ? 2 : 1;          // 32-column slices per round
+            constexpr int NSL = pp::BN / 32;         // slices per tile
+            const int row = warp * 32 + lane;        // TMEM lane == token within the CTA's half
+            const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+            float* const wsc = sm->wscale[warp];
+            int tc = 0;
+            uint32_t nstore = 0;
+            for (int tile = pair; tile < tiles; tile += npairs, ++tc) {
+                const int mt = tile % MT, nt = tile / MT;
+                const int b = tc & 1;
+                const uint32_t aph = (tc >> 1) & 1;
+                __syncwarp();
+#pragma unroll
+                for (int k = 0; k < NSL; ++k) {
+                    const int o = nt * pp::BN + 32 * k + lane;
+                    wsc[32 * k + lane] = o < O ? __ldg(row_scale + o) : 0.f;
+                }
+                __syncwarp();
+                if (!warp_wait(&sm->tmem_full[b], aph, abort_flag)) { give_up(); break; }
+                tc_fence_after();
+                const int trow0 = mt * 2 * pp::BM + static_cast<int>(rank) * pp::BM;
+                const int t = trow0 + row;
+                const bool tvalid = t < T;
+                const float inv_s = tvalid ? __frcp_rn(s_tok[t]) : 0.f;
+                const uint32_t tbase = tmem_base + lane_addr + b * pp::BN;
+                uint32_t ra[32], rb[32];
+                uint32_t q[32];
+                auto slice = [&](auto h_tag, const int k, uint32_t (&cur)[32], uint32_t (&nxt)[32]) {
+                    constexpr int H = decltype(h_tag)::value;
+                    const bool more = k + 1 < NSL;
+                    if (more) {
+                        tmem_ld32_nowait(tbase + 32 * (k + 1), nxt);
+                    } else {
+                        // the warp is done with the buffer (its loads completed above)
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) arrive_leader(&sm->tmem_empty[b]);
+                    }
+                    const float* sc = wsc + 32 * k;
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4) {
+                        const float4 s4 = *reinterpret_cast<const float4*>(sc + i);
+                        const float f0 = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int>(cur[i + 0])), s4.x), inv_s);
+                        const float f1 = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int>(cur[i + 1])), s4.y), inv_s);
+                        const float f2 = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int>(cur[i + 2])), s4.z), inv_s);
+                        const float f3 = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int>(cur[i + 3])), s4.w), inv_s);
+                        if (BF) {
+                            const __nv_bfloat162 h01 = __floats2bfloat162_rn(f0, f1);
+                            const __nv_bfloat162 h23 = __floats2bfloat162_rn(f2, f3);
+                            q[16 * H + i / 2] = *reinterpret_cast<const uint32_t*>(&h01);
+                            q[16 * H + i / 2 + 1] = *reinterpret_cast<const uint32_t*>(&h23);
+                        } else {
+                            q[i] = __float_as_uint(f0);
+                            q[i + 1] = __float_as_uint(f1);
+                            q[i + 2] = __float_as_uint(f2);
+                            q[i + 3] = __float_as_uint(f3);
+                        }
+                    }
+                    if (acc_out && tvalid) {
+                        const long long base = static_cast<long long>(t) * O + nt * pp::BN + 32 * k;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (nt * pp::BN + 32 * k + i < O) acc_out[base + i] = static_cast<int>(cur[i]);
+                    }
+                    if (H == SPR - 1) {
+                        const int o0 = nt * pp::BN + 32 * (k - H);
+                        if (y_vec) {
+                            uint8_t* const box = sm->ystage[warp][nstore & 1];
+                            if (lane == 0) bulk_wait_read<1>();
+                            __syncwarp();
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) {
+                                const uint32_t a = smem_u32(box + lane * 128 + ((c ^ (lane & 7)) << 4));
+                                asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(q[4 * c]),
+                                             "r"(q[4 * c + 1]), "r"(q[4 * c + 2]), "r"(q[4 * c + 3])
+                                             : "memory");
+                            }
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                            if (lane == 0) tma_store_2d(&tmap_y, smem_u32(box), o0, trow0 + warp * 32);
+                            ++nstore;
+                        } else if (tvalid) {
+                            // direct stores: shapes whose row pitch is not a multiple of 16 bytes
+                            const long long base = static_cast<long long>(t) * O + o0;
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) {
+                                if (BF) {
+                                    if (o0 + 2 * i < O)
+                                        reinterpret_cast<uint16_t*>(y)[base + 2 * i] = static_cast<uint16_t>(q[i] & 0xFFFFu);
+                                    if (o0 + 2 * i + 1 < O)
+                                        reinterpret_cast<uint16_t*>(y)[base + 2 * i + 1] = static_cast<uint16_t>(q[i] >> 16);
+                                } else if (o0 + i < O) {
+                                    reinterpret_cast<uint32_t*>(y)[base + i] = q[i];
+                                }
+                            }
+                        }
+                    }
+                    if (more) tmem_ld_wait();
+                };
+                tmem_ld32_nowait(tbase, ra);
+                tmem_ld_wait();
+                for (int k = 0; k < NSL; k += 2) {
+                    if (SPR == 2) {
+                        slice(std::integral_constant<int, 0>{}, k, ra, rb);
+                        slice(std::integral_constant<int, 1>{}, k + 1, rb, ra);
+                    } else {
+                        slice(std::integral_constant<int, 0>{}, k, ra, rb);
+                        slice(std::integral_constant<int, 0>{}, k + 1, rb, ra);
+                    }
+                }
+            }
+            if (lane == 0) bulk_wait_all();
+        };
+        if (y_bf16) run(std::true_type{});
+        else run(std::false_type{});
+    } else if (warp < pp::WARP_TMA) {
+        // ------------------------------------------------------------ weight expansion
+        // Thread r expands output row r of this CTA's half of B for each k-block
+        // and reports to the even CTA, whose MMAs read this shared memory.
+        const int r = threadIdx.x - pp::EPI_WARPS * 32;
+        uint32_t it = 0;
+        bool ok = true;
+        for (int tile = pair; tile < tiles && ok; tile += npairs) {
+            for (int kb = 0; kb < KB; ++kb, ++it) {
+                const int s = it % pp::STAGES;
+                const uint32_t ph = (it / pp::STAGES) & 1;
+                // the codes have landed; the producer loaded them only after the
+                // pair's MMAs released this stage, so b[s] is free as well
+                if (!mbar_wait(&sm->full_c[s], ph, abort_flag)) { give_up(); ok = false; break; }
+                // code rows are 32 bytes, 32B-swizzled by TMA: 16-byte half q of
+                // row r sits at half q ^ ((r >> 2) & 1)
+                const uint8_t* src = sm->p[s] + r * 32;
+                const int hs = (r >> 2) & 1;
+                const uint4 p0 = *reinterpret_cast<const uint4*>(src + (hs << 4));
+                const uint4 p1 = *reinterpret_cast<const uint4*>(src + ((hs ^ 1) << 4));
+                uint8_t* dst = sm->b[s] + r * 128;
+                const int sw = r & 7;
+                const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t e[4];
+                    expand_codes(words[c], e);
+                    const uint32_t a = smem_u32(dst + ((c ^ sw) << 4));
+                    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(e[0]), "r"(e[1]), "r"(e[2]),
+                                 "r"(e[3])
+                                 : "memory");
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if ((r & 31) == 0) arrive_leader(&sm->full_dec[s]);
+            }
+        }
+    } else if (warp == pp::WARP_TMA) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = pair; tile < tiles && ok; tile += npairs) {
+                const int mt = tile % MT, nt = tile / MT;
+                const int trow = mt * 2 * pp::BM + static_cast<int>(rank) * pp::BM;
+                const int orow = nt * pp::BN + static_cast<int>(rank) * pp::BNH;
+                for (int kb = 0; kb < KB; ++kb, ++it) {
+                    const int s = it % pp::STAGES;
+                    const uint32_t ph = (it / pp::STAGES) & 1;
+                    if (!mbar_wait(&sm->empty[s], ph ^ 1, abort_flag)) { give_up(); ok = false; break; }
+                    // the even CTA expects the activation bytes of both CTAs
+                    if (leader) mbar_arrive_expect_tx(&sm->full_a[s], 2 * pp::A_BYTES);
+                    mbar_arrive_expect_tx(&sm->full_c[s], pp::P_BYTES);
+                    tma_load_2d_pair(smem_u32(sm->a[s]), &tmap_x, kb * pp::BK, trow,
+                                     map_to_cta(smem_u32(&sm->full_a[s]), 0));
+                    tma_load_2d(smem_u32(sm->p[s]), &tmap_w, kb * (pp::BK / 4), orow, &sm->full_c[s]);
+                }
+            }
+            // let the issued loads land before the CTA can exit: its own code
+            // tiles here, and (in the even CTA) the activation tiles of both
+            const uint32_t first = it > pp::STAGES ? it - pp::STAGES : 0;
+            volatile int never = 0;
+            for (uint32_t j = first; j < it; ++j) {
+                const int s = j % pp::STAGES;
+                const uint32_t ph = (j / pp::STAGES) & 1;
+                if (!mbar_wait(&sm->full_c[s], ph, &never)) give_up();
+                if (leader && !mbar_wait(&sm->full_a[s], ph, &never)) give_up();
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ MMA issuer (even CTA)
+        if (lane == 0) {
+            if (leader) {
+                const uint32_t idesc = i8_idesc<2 * pp::BM, pp::BN>();
+                uint32_t it = 0;
+                int tc = 0;
+                bool ok = true;
+                for (int tile = pair; tile < tiles && ok; tile += npairs, ++tc) {
+                    const int b = tc & 1;
+                    const uint32_t aph = (tc >> 1) & 1;
+                    if (!mbar_wait(&sm->tmem_empty[b], aph ^ 1, abort_flag)) { give_up(); break; }
+                    tc_fence_after();
+                    const uint32_t d = tmem_base + b * pp::BN;
+                    for (int kb = 0; kb < KB; ++kb, ++it) {
+                        const int s = it % pp::STAGES;
+                        const uint32_t ph = (it / pp::STAGES) & 1;
+                        if (!mbar_wait(&sm->full_a[s], ph, abort_flag) ||
+                            !mbar_wait(&sm->full_dec[s], ph, abort_flag)) {
+                            give_up(); ok = false; break;
+                        }
+                        tc_fence_after();
+                        const uint32_t a0 = smem_u32(sm->a[s]), b0 = smem_u32(sm->b[s]);
+#pragma unroll
+                        for (int kk = 0; kk < pp::BK / 32; ++kk)
+                            tc_mma_pair(d, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc, (kb | kk) != 0);
+                        tc_commit_pair_both(&sm->empty[s]);
+                    }
+                    if (ok) tc_commit_pair_both(&sm->tmem_full[b]);
+                }
+                // every MMA must be complete before either CTA frees tensor memory
+                tc_commit_pair_both(&sm->mma_done);
+            }
+            volatile int never = 0;
+            if (!mbar_wait(&sm->mma_done, 0, &never)) give_up();
+        }
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    cluster_sync();  // neither CTA leaves while the other may still touch its shared memory
+    if (warp == pp::WARP_MMA) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(pp::TMEM_COLS)
+                     : "memory");
+    }
+}
+
+// Clusters of this kernel that fit on the device at once (one CTA per SM, two
+// SMs per cluster), cached per device; 0 when the query fails.
+int prefill_pair_clusters(cudaStream_t stream) {
+    static int cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (cached[dev] == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2);
+        cfg.blockDim = dim3(pp::THREADS);
+        cfg.dynamicSmemBytes = pair_smem_bytes();
+        cfg.stream = stream;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, prefill_pair_kernel, &cfg) != cudaSuccess || n <= 0) return 0;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+cudaError_t launch_prefill_pair(const int8_t* xperm, const float* s_tok, long long T, long long K,
+                                const uint8_t* packed, const float* row_scale, long long O, void* y, int y_bf16,
+                                int32_t* acc_out, unsigned* status, cudaStream_t stream) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(prefill_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(pair_smem_bytes()));
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+    const int max_clusters = prefill_pair_clusters(stream);
+    if (max_clusters <= 0) return cudaErrorNotSupported;
+
+    CUtensorMap map_x, map_w;
+    const cuuint32_t estr[2] = {1, 1};
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(T)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+        const cuuint32_t box[2] = {static_cast<cuuint32_t>(pp::BK), static_cast<cuuint32_t>(pp::BM)};
+        if (enc(&map_x, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(xperm), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 4), static_cast<cuuint64_t>(O)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 4)};
+        const cuuint32_t box[2] = {static_cast<cuuint32_t>(pp::BK / 4), static_cast<cuuint32_t>(pp::BNH)};
+        if (enc(&map_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    const int esize = y_bf16 ? 2 : 4;
+    int y_vec = (static_cast<long long>(O) * esize) % 16 == 0 ? 1 : 0;
+    CUtensorMap map_y = map_x;
+    if (y_vec) {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(O), static_cast<cuuint64_t>(T)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(O) * esize};
+        const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esize), 32u};
+        if (enc(&map_y, y_bf16 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, y, dims, strides,
+                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            y_vec = 0;
+    }
+    const long long tiles = ((T + 2 * pp::BM - 1) / (2 * pp::BM)) * ((O + pp::BN - 1) / pp::BN);
+    const int clusters = static_cast<int>(tiles < max_clusters ? tiles : max_clusters);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * clusters);
+    cfg.blockDim = dim3(pp::THREADS);
+    cfg.dynamicSmemBytes = pair_smem_bytes();
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, prefill_pair_kernel, map_x, map_w, map_y, y_vec, row_scale, s_tok,
+                              static_cast<int>(T), static_cast<int>(O), static_cast<int>(K), y, y_bf16, acc_out,
+                              status);
+}
+
+}  // namespace sbl

@@ -1,6 +1,6 @@
 // C ABI of the Sparse-BitLinear library: argument validation, workspace
 // layout, path dispatch and the per-device status word.  All arithmetic runs
-// in the kernels of prep.cu, quant.cu, decode.cu and prefill.cu.
+// in the kernels of prep.cu, quant.cu, decode.cu, prefill.cu and prefill_pair.cu.
 #include <cstdint>
 #include <cstdio>
 #include <cuda_runtime.h>
@@ -19,7 +19,8 @@ cudaError_t launch_decode(const uint8_t* packed, const float* row_scale, long lo
                           int num_sms, cudaStream_t stream);
 cudaError_t launch_prefill(const int8_t* xperm, const float* s_tok, long long T, long long K, const uint8_t* packed,
                            const float* row_scale, long long O, void* y, int y_bf16, int32_t* acc_out,
-                           unsigned* status, int num_sms, cudaStream_t stream);
+                           unsigned* status, int num_sms, int variant, cudaStream_t stream);
+constexpr int kPrefillAuto = 0, kPrefillOneCta = 1, kPrefillPair = 2;
 #ifdef SBL_TRACE
 cudaError_t set_prefill_trace(void* buf);
 #endif
@@ -129,8 +130,9 @@ sbl_status sbl_linear_path(const uint16_t* x_bf16, int64_t T, int64_t K, const u
     if (sbl_status s = check_k(K)) return s;
     if (!nm_ok(n, m)) return SBL_ERR_UNSUPPORTED;
     if (y_dtype != SBL_F32 && y_dtype != SBL_BF16) return SBL_ERR_INVALID_ARG;
-    if (path != SBL_PATH_AUTO && path != SBL_PATH_DECODE && path != SBL_PATH_PREFILL) return SBL_ERR_INVALID_ARG;
-    if (path == SBL_PATH_PREFILL && K % 64 != 0) return SBL_ERR_UNSUPPORTED;
+    if (path < SBL_PATH_AUTO || path > SBL_PATH_PREFILL_PAIR) return SBL_ERR_INVALID_ARG;
+    const bool forced_prefill = path >= SBL_PATH_PREFILL;
+    if (forced_prefill && K % 64 != 0) return SBL_ERR_UNSUPPORTED;
     if (T == 0 || O == 0) return SBL_OK;
     if (!x_bf16 || !packed || !row_scale || !y) return SBL_ERR_INVALID_ARG;
     if (!aligned(x_bf16, 16) || !aligned(packed, 16) || !aligned(row_scale, 16) || !aligned(y, 16))
@@ -146,7 +148,7 @@ sbl_status sbl_linear_path(const uint16_t* x_bf16, int64_t T, int64_t K, const u
     int8_t* xq = static_cast<int8_t*>(workspace);
     float* s_tok = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round256(static_cast<size_t>(T) * K));
 
-    bool prefill = path == SBL_PATH_PREFILL;
+    bool prefill = forced_prefill;
     if (path == SBL_PATH_AUTO) prefill = ((T > kDecodeMaxTokens) || (K > kDecodeMaxK)) && (K % 64 == 0);
     if (!prefill && K > kDecodeMaxK) return SBL_ERR_UNSUPPORTED;
 
@@ -155,7 +157,11 @@ sbl_status sbl_linear_path(const uint16_t* x_bf16, int64_t T, int64_t K, const u
     if (prefill) {
         e = sbl::launch_quant(x_bf16, T, K, xq, s_tok, sbl::kLayoutInterleaved, d->status, st);
         if (e != cudaSuccess) return SBL_ERR_CUDA;
-        e = sbl::launch_prefill(xq, s_tok, T, K, packed, row_scale, O, y, ybf, acc_out, d->status, d->num_sms, st);
+        const int variant = path == SBL_PATH_PREFILL_1CTA ? sbl::kPrefillOneCta
+                            : path == SBL_PATH_PREFILL_PAIR ? sbl::kPrefillPair
+                                                            : sbl::kPrefillAuto;
+        e = sbl::launch_prefill(xq, s_tok, T, K, packed, row_scale, O, y, ybf, acc_out, d->status, d->num_sms, variant,
+                                st);
     } else {
         // the decode kernel quantises the activations itself
         e = sbl::launch_decode(packed, row_scale, O, K, x_bf16, T, y, ybf, acc_out, d->status, d->num_sms, st);

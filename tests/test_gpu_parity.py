@@ -135,7 +135,7 @@ LINEAR_CASES = [
 ]
 
 
-@pytest.mark.parametrize("path", ["decode", "prefill"])
+@pytest.mark.parametrize("path", ["decode", "prefill", "prefill_1cta", "prefill_pair"])
 @pytest.mark.parametrize("O,K,T,n,m", LINEAR_CASES)
 def test_linear_parity(sbl, path, O, K, T, n, m):
     W, xbits, xval = layer_inputs(O, K, T, seed=2, outlier_p=0.01)
@@ -177,11 +177,34 @@ def test_zero_rows_and_tokens(sbl):
     xval[7] = 0.0
     ref = oracle_layer(W, n, m, xval)
     w = _prep(sbl, W, n, m)
-    for path in ("decode", "prefill"):
+    for path in ("decode", "prefill_1cta", "prefill_pair"):
         y, acc = _run_linear(sbl, w, xbits, T, O, path)
         yn = y.cpu().numpy()
         assert np.array_equal(acc.cpu().numpy(), ref["acc"])
         assert not yn[7].any() and not yn[:, 5].any()
+
+
+PAIR_CASES = [
+    # (O, K, T, n, m): full 256 x 256 pair tiles, a ragged half tile of outputs
+    # (896 = 3.5 x 256) and of tokens, an odd CTA with no tokens at all, N:M patterns
+    (4864, 896, 2048, 3, 4),
+    (896, 4864, 300, 2, 4),
+    (1000, 640, 513, 6, 8),
+    (256, 128, 128, 2, 4),
+]
+
+
+@pytest.mark.parametrize("O,K,T,n,m", PAIR_CASES)
+def test_pair_prefill_full(sbl, O, K, T, n, m):
+    """The CTA-pair tensor-core kernel, fully compared (fp32 and bf16 outputs)."""
+    W, xbits, xval = layer_inputs(O, K, T, seed=6, outlier_p=0.01)
+    ref = oracle_layer(W, n, m, xval)
+    w = _prep(sbl, W, n, m)
+    y, acc = _run_linear(sbl, w, xbits, T, O, "prefill_pair")
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    assert_fp32_close(y.cpu().numpy(), ref["y"])
+    yb, _ = _run_linear(sbl, w, xbits, T, O, "prefill_pair", torch.bfloat16)
+    assert_bf16_close(yb.cpu().view(torch.int16).numpy(), ref["y"])
 
 
 # ------------------------------------------------------------------ full-size layers
