@@ -53,7 +53,7 @@ PREFILL_TRAFFIC = {"sources_sha256": "f09882ef5c859ccbe08bcc41bff11ea06fc0c0cb89
 def _kernel_sources_digest():
     import hashlib
     h = hashlib.sha256()
-    for f in ("sbl_common.cuh", "quant.cu", "prefill.cu"):
+    for f in ("sbl_common.cuh", "tc_util.cuh", "quant.cu", "prefill.cu", "prefill_pair.cu"):
         with open(os.path.join(ROOT, "sparse_linear_layers_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
@@ -282,6 +282,50 @@ def _decode_roofline(sbl, dev, hbm_peak, K=2048, O=7168, reps=64):
             "isolated_call_us": statistics.median(iso) * 1e6}
 
 
+def _prefill_roofline(sbl, dev, int8_peak_tops, hbm_peak, K=896, O=4864, T=32768, reps=10):
+    """One prefill sbl_linear call (activation quantisation + tcgen05 GEMM) on the
+    0.5B FFN gate shape at T = 32768 (3:4, 1% outliers x20), bf16 and fp32
+    outputs; graph-replayed with L2 flushed before each call (every operand is
+    larger than L2 except the 1 MB of codes)."""
+    W = torch.from_numpy(synthetic.latent_weights(O, K, seed=12, tag="prefill-roof")).to(dev)
+    w = sbl.sbl_prepare_weights(W, 3, 4)
+    del W
+    xb, _ = synthetic.activations(T, K, seed=12, tag="prefill-roof", outlier_p=0.01)
+    x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)
+    ws = sbl.workspace_for(T, K, O, 3, 4, dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    ops = 2.0 * T * O * K
+    out = {"layer": f"{K}->{O} 3:4 T={T}", "ops_per_call": ops, "peak_tops": int8_peak_tops,
+           "peak_source": "int8 = 2 x measured bf16 burst (nominal dense ratio)"}
+    for name, dt, esz in (("bf16_out", torch.bfloat16, 2), ("fp32_out", torch.float32, 4)):
+        y = torch.empty((T, O), dtype=dt, device=dev)
+        s = torch.cuda.Stream()
+        with torch.cuda.stream(s):
+            sbl.sbl_linear(x, w, y=y, workspace=ws)
+        s.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            sbl.sbl_linear(x, w, y=y, workspace=ws)
+        ts = []
+        with torch.cuda.stream(s):
+            for i in range(reps + 3):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(s)
+                g.replay()
+                b.record(s)
+                b.synchronize()
+                if i >= 3:
+                    ts.append(a.elapsed_time(b) / 1e3)
+        t = statistics.median(ts)
+        byts = T * K * 2 + T * K * 2 + O * K / 4 + T * O * esz  # x read, x_q write + read, codes, y
+        out[name] = {"us_per_call": t * 1e6, "tops": ops / t / 1e12, "tensor_frac": ops / t / 1e12 / int8_peak_tops,
+                     "algorithmic_bytes": byts, "hbm_gbs": byts / t / 1e9, "hbm_frac": byts / t / 1e9 / hbm_peak}
+        del g, y
+    del w, x, ws, flush
+    return out
+
+
 def run_ours(args, rank, world, dev):
     import sparse_linear_layers_b200 as sbl
     hbm_peak, bf16_peak, bf16_sus, peak_kind = _peaks()
@@ -360,6 +404,7 @@ def run_ours(args, rank, world, dev):
     e2e_s = _max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev)
 
     decode = _decode_roofline(sbl, dev, hbm_peak) if rank == 0 else None
+    prefill_big = _prefill_roofline(sbl, dev, int8_peak_tops, hbm_peak) if rank == 0 else None
     launches_per_step = len(layers) * (1 + 2 + 1)  # prep + (quant + tcgen05 GEMM) + fused decode
     value = _throughput(world, K, total_s)
     out = {
@@ -369,6 +414,7 @@ def run_ours(args, rank, world, dev):
         "config": _config({"parallelism": f"replicas x{world} (no collective on the data path)"}),
         "roofline": roof,
         "decode_roofline": decode,
+        "prefill_roofline": prefill_big,
         "phases": phases,
         "e2e": {"value": world * TOKENS_PER_STEP * K_e2e / e2e_s, "steps": K_e2e, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},

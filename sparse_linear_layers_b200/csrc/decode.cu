@@ -34,6 +34,10 @@ namespace sbl {
 constexpr int kDecodeThreads = 512;
 constexpr int kDecodeWarps = kDecodeThreads / 32;
 constexpr int kDecodeBatch = 4;  // chunks per lane in flight
+// Two blocks of one-token passes share an SM, so the next call's blocks can
+// start (and prefetch their weights) while this one drains.
+template <int TT>
+constexpr int decode_min_blocks() { return TT == 1 ? 2 : 1; }
 
 template <int CW>
 __device__ __forceinline__ void load_chunk_words(const uint8_t* prow, int c, uint32_t (&w)[CW]) {
@@ -49,7 +53,7 @@ __device__ __forceinline__ void load_chunk_words(const uint8_t* prow, int c, uin
 }
 
 template <int L, int TT, int CW>
-__global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const uint8_t* __restrict__ packed,
+__global__ void __launch_bounds__(kDecodeThreads, decode_min_blocks<TT>()) decode_kernel(const uint8_t* __restrict__ packed,
                                                                 const float* __restrict__ row_scale, long long O,
                                                                 int K, const uint16_t* __restrict__ x, long long T,
                                                                 long long t0, void* __restrict__ y, int y_bf16,
@@ -59,7 +63,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const uint8_t* _
     __shared__ float s_sh[TT];
     asm volatile("griddepcontrol.launch_dependents;");
     constexpr int RW = 32 / L;
-    constexpr int NB = kDecodeBatch;
+    constexpr int NB = TT >= 8 ? kDecodeBatch / 2 : kDecodeBatch;  // eight tokens: accumulators take the registers
     const int CPR = K / (16 * CW);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int sub = lane / L, li = lane % L;
@@ -89,35 +93,74 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const uint8_t* _
     // Quantise this pass's tokens: per-token absmax, then int8 into shared memory.
     const int nvec = K >> 3;
     const int nblk = K >> 4;
-#pragma unroll
-    for (int t = 0; t < TT; ++t) {
-        const long long tt = t0 + t < T ? t0 + t : T - 1;
+    if (TT == 1 && nblk <= kDecodeThreads) {
+        // one token, K <= 8192: each thread keeps its 16-element block in
+        // registers between the absmax and the quantisation
+        constexpr int XB = 1;
+        const long long tt = t0 < T ? t0 : T - 1;
         const uint4* xr = reinterpret_cast<const uint4*>(x + tt * K);
-        uint32_t mx = 0;
-        for (int v = threadIdx.x; v < nvec; v += kDecodeThreads) mx = absmax8(ldg_nc(xr + v), mx);
-        mx = __reduce_max_sync(0xFFFFFFFFu, mx);
-        if (lane == 0) red[warp][t] = mx;
-    }
-    __syncthreads();
-    if (threadIdx.x < TT) {
+        uint4 xa[XB][2];
         uint32_t mx = 0;
 #pragma unroll
-        for (int w = 0; w < kDecodeWarps; ++w) mx = max(mx, red[w][threadIdx.x]);
-        if (mx >= 0x7F80u && blockIdx.x == 0) raise_status(status, kStatusNonfinite);
-        s_sh[threadIdx.x] = __fdiv_rn(127.0f, fmaxf(__uint_as_float(mx << 16), 1e-5f));
-    }
-    __syncthreads();
-#pragma unroll
-    for (int t = 0; t < TT; ++t) {
-        const long long tt = t0 + t < T ? t0 + t : T - 1;
-        const uint4* xr = reinterpret_cast<const uint4*>(x + tt * K);
-        const float st = s_sh[t];
-        for (int b = threadIdx.x; b < nblk; b += kDecodeThreads) {
-            const int pos = CW == 4 ? (b & 3) * CPR + (b >> 2) : b;
-            xs[t * nblk + pos] = quant_block16<true>(ldg_nc(xr + 2 * b), ldg_nc(xr + 2 * b + 1), st);
+        for (int i = 0; i < XB; ++i) {
+            const int b = threadIdx.x + i * kDecodeThreads;
+            if (b < nblk) {
+                xa[i][0] = ldg_nc(xr + 2 * b);
+                xa[i][1] = ldg_nc(xr + 2 * b + 1);
+                mx = absmax8(xa[i][1], absmax8(xa[i][0], mx));
+            }
         }
+        mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+        if (lane == 0) red[warp][0] = mx;
+        __syncthreads();
+        mx = 0;
+#pragma unroll
+        for (int w = 0; w < kDecodeWarps; ++w) mx = max(mx, red[w][0]);
+        const float st = __fdiv_rn(127.0f, fmaxf(__uint_as_float(mx << 16), 1e-5f));
+        if (threadIdx.x == 0) {
+            if (mx >= 0x7F80u && blockIdx.x == 0) raise_status(status, kStatusNonfinite);
+            s_sh[0] = st;
+        }
+#pragma unroll
+        for (int i = 0; i < XB; ++i) {
+            const int b = threadIdx.x + i * kDecodeThreads;
+            if (b < nblk) {
+                const int pos = CW == 4 ? (b & 3) * CPR + (b >> 2) : b;
+                xs[pos] = quant_block16<true>(xa[i][0], xa[i][1], st);
+            }
+        }
+        __syncthreads();
+    } else {
+#pragma unroll
+        for (int t = 0; t < TT; ++t) {
+            const long long tt = t0 + t < T ? t0 + t : T - 1;
+            const uint4* xr = reinterpret_cast<const uint4*>(x + tt * K);
+            uint32_t mx = 0;
+            for (int v = threadIdx.x; v < nvec; v += kDecodeThreads) mx = absmax8(ldg_nc(xr + v), mx);
+            mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+            if (lane == 0) red[warp][t] = mx;
+        }
+        __syncthreads();
+        if (threadIdx.x < TT) {
+            uint32_t mx = 0;
+#pragma unroll
+            for (int w = 0; w < kDecodeWarps; ++w) mx = max(mx, red[w][threadIdx.x]);
+            if (mx >= 0x7F80u && blockIdx.x == 0) raise_status(status, kStatusNonfinite);
+            s_sh[threadIdx.x] = __fdiv_rn(127.0f, fmaxf(__uint_as_float(mx << 16), 1e-5f));
+        }
+        __syncthreads();
+#pragma unroll
+        for (int t = 0; t < TT; ++t) {
+            const long long tt = t0 + t < T ? t0 + t : T - 1;
+            const uint4* xr = reinterpret_cast<const uint4*>(x + tt * K);
+            const float st = s_sh[t];
+            for (int b = threadIdx.x; b < nblk; b += kDecodeThreads) {
+                const int pos = CW == 4 ? (b & 3) * CPR + (b >> 2) : b;
+                xs[t * nblk + pos] = quant_block16<true>(ldg_nc(xr + 2 * b), ldg_nc(xr + 2 * b + 1), st);
+            }
+        }
+        __syncthreads();
     }
-    __syncthreads();
 
     int alo[TT][4], ahi[TT][4];
 #pragma unroll
@@ -192,16 +235,20 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const uint8_t* _
     }
 }
 
-// Lanes per row: best chunk utilisation, weighted by how well the warp count
-// fills the GPU (small layers prefer wide rows, large ones exact fits).
+// Lanes per row.  The call should fit in one block of kDecodeWarps warps per
+// SM, which leaves room on each SM for the next call's block, with every load
+// in flight at once: among the lane counts whose warps fit, take the best
+// chunk utilisation per batch of loads (ties: more lanes per row).
 static int choose_lanes(long long O, int cpr, int num_sms) {
-    int best = 32;
+    const long long cap = static_cast<long long>(num_sms) * kDecodeWarps;
+    int best = 1;
     double best_score = -1.0;
     for (int L = 32; L >= 1; L >>= 1) {
-        const double eff = static_cast<double>(cpr) / (static_cast<double>((cpr + L - 1) / L) * L);
-        const double warps = static_cast<double>((O + (32 / L) - 1) / (32 / L));
-        const double fill = warps / (num_sms * 16.0);
-        const double score = eff * (fill < 1.0 ? fill : 1.0);
+        const long long warps = (O + (32 / L) - 1) / (32 / L);
+        if (warps > cap) continue;
+        const int per_lane = (cpr + L - 1) / L;
+        const double eff = static_cast<double>(cpr) / (static_cast<double>(per_lane) * L);
+        const double score = eff / ((per_lane + kDecodeBatch - 1) / kDecodeBatch);
         if (score > best_score + 1e-9) {
             best_score = score;
             best = L;
