@@ -380,6 +380,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
     }
 }
 
+// Opt the kernel in to its dynamic shared memory (once per device).
+static cudaError_t pair_set_smem_attr() {
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64 && attr_set[dev]) return cudaSuccess;
+    e = cudaFuncSetAttribute(prefill_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(pair_smem_bytes()));
+    if (e == cudaSuccess && dev >= 0 && dev < 64) attr_set[dev] = true;
+    return e;
+}
+
 // Clusters of this kernel that fit on the device at once (one CTA per SM, two
 // SMs per cluster), cached per device; 0 when the query fails.
 int prefill_pair_clusters(cudaStream_t stream) {
@@ -387,6 +400,7 @@ int prefill_pair_clusters(cudaStream_t stream) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
     if (cached[dev] == 0) {
+        if (pair_set_smem_attr() != cudaSuccess) return 0;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2);
         cfg.blockDim = dim3(pp::THREADS);
@@ -404,15 +418,7 @@ cudaError_t launch_prefill_pair(const int8_t* xperm, const float* s_tok, long lo
                                 int32_t* acc_out, unsigned* status, cudaStream_t stream) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return cudaErrorNotSupported;
-    static bool attr_set[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(pair_smem_bytes()));
-        if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr_set[dev] = true;
-    }
+    if (cudaError_t e = pair_set_smem_attr()) return e;
     const int max_clusters = prefill_pair_clusters(stream);
     if (max_clusters <= 0) return cudaErrorNotSupported;
 
