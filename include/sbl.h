@@ -50,10 +50,11 @@ typedef enum {
 enum { SBL_F32 = 0, SBL_BF16 = 1 };
 
 /* Contraction paths of sbl_linear_path.  SBL_PATH_PREFILL lets the library
- * pick the tensor-core kernel; the last two force one of them (tests, tuning):
- * one CTA per 128-token tile, or a pair of CTAs on two SMs per 256-token tile. */
+ * pick the tensor-core kernel; the others force one of them (tests, tuning):
+ * one CTA per 128-token tile, a pair of CTAs on two SMs per 256-token tile,
+ * or (2:4 weights only) the structured-sparse MMA on compressed weights. */
 enum { SBL_PATH_AUTO = 0, SBL_PATH_DECODE = 1, SBL_PATH_PREFILL = 2,
-       SBL_PATH_PREFILL_1CTA = 3, SBL_PATH_PREFILL_PAIR = 4 };
+       SBL_PATH_PREFILL_1CTA = 3, SBL_PATH_PREFILL_PAIR = 4, SBL_PATH_PREFILL_SPARSE = 5 };
 
 /*
  * sbl_prepare_weights — N:M mask, per-row scale, ternarise and 2-bit pack.
@@ -104,8 +105,13 @@ sbl_status sbl_quant_act(const uint16_t* x_bf16, int64_t T, int64_t K,
 
 /*
  * sbl_linear_workspace_bytes — bytes of device workspace sbl_linear needs for
- * these sizes (the quantised activations and their scales, in the kernels'
- * internal layout).  Never 0 for T > 0.
+ * these sizes: the quantised activations and their scales, in the kernels'
+ * internal layout (T*K + 4*T bytes, each rounded up to 256), plus, for 2:4
+ * weights (K % 64 == 0) at sizes that take a prefill path, the weights'
+ * compressed form for the sparse tensor cores (O*K/2 + O*32*ceil(K/256)
+ * bytes, each rounded up to 256).  Never 0 for T > 0.  A smaller workspace
+ * that still holds the first part is accepted; sbl_linear then stays on the
+ * dense paths.
  */
 size_t sbl_linear_workspace_bytes(int64_t T, int64_t K, int64_t O, int n, int m);
 
@@ -141,6 +147,13 @@ sbl_status sbl_linear(const uint16_t* x_bf16, int64_t T, int64_t K,
  * (SBL_PATH_DECODE, or one of the SBL_PATH_PREFILL* tensor-core paths;
  * SBL_PATH_AUTO is sbl_linear).  Every path gives the same results.
  * A prefill path with K % 64 != 0 returns SBL_ERR_UNSUPPORTED.
+ * SBL_PATH_PREFILL_SPARSE (the Sparse-BitNet Guide, "The Hardware Mechanics
+ * of 2:4 Sparsity": two kept values and their 2-bit positions per group of
+ * four feed the structured-sparse MMA) needs (n, m) = (2, 4), else
+ * SBL_ERR_UNSUPPORTED, and a workspace that also holds the compressed weights,
+ * else SBL_ERR_WORKSPACE.  Packed codes with more than two nonzeros in a group
+ * of four are not 2:4 weights: the call then sets SBL_ERR_INVALID_ARG in the
+ * device status word and its results are unspecified.
  */
 sbl_status sbl_linear_path(const uint16_t* x_bf16, int64_t T, int64_t K,
                            const uint8_t* packed, const float* row_scale, int64_t O, int n, int m,
@@ -160,11 +173,11 @@ sbl_status sbl_linear_path(const uint16_t* x_bf16, int64_t T, int64_t K,
  * SBL_NOALLOC_SCRATCH_BYTES of static device memory inside the library, which
  * every GPU that loads the library holds until the process exits.  The call
  * allocates nothing.
- *   - Calls needing more scratch than the array holds, i.e.
- *     sbl_linear_workspace_bytes(T, K, O, n, m) > SBL_NOALLOC_SCRATCH_BYTES
- *     (T * K + 4 * T bytes, each rounded up to 256: T = 1024 fits at
- *     K = 7168 but not at K = 8192), return SBL_ERR_WORKSPACE and enqueue
- *     nothing.
+ *   - Calls whose quantised activations and scales (T * K + 4 * T bytes, each
+ *     rounded up to 256: T = 1024 fits at K = 7168 but not at K = 8192) do
+ *     not fit in the array return SBL_ERR_WORKSPACE and enqueue nothing.  2:4
+ *     calls use the sparse tensor cores only when the compressed weights fit
+ *     in the rest of the array.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress); make that first call before any stream capture.
  *   - All calls on a device share the one array: calls that may overlap on the
@@ -182,8 +195,9 @@ int64_t sbl_decode_max_tokens(void);
 
 /*
  * sbl_device_status — synchronises `stream`, then returns and clears the
- * current device's status word: SBL_OK, or the first of SBL_ERR_NONFINITE /
- * SBL_ERR_TIMEOUT that any kernel raised since the last call.
+ * current device's status word: SBL_OK, or the first of SBL_ERR_TIMEOUT /
+ * SBL_ERR_NONFINITE / SBL_ERR_INVALID_ARG (weights given as 2:4 that are not)
+ * that any kernel raised since the last call.
  */
 sbl_status sbl_device_status(void* stream);
 

@@ -28,6 +28,7 @@ SBL_PATH_DECODE = 1
 SBL_PATH_PREFILL = 2
 SBL_PATH_PREFILL_1CTA = 3
 SBL_PATH_PREFILL_PAIR = 4
+SBL_PATH_PREFILL_SPARSE = 5
 
 # name -> (restype, argtypes); mirrors include/sbl.h
 _vp, _i64, _int, _sz, _u32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint32

@@ -15,7 +15,8 @@ from . import _lib
 from ._lib import check, lib
 
 _PATHS = {"auto": _lib.SBL_PATH_AUTO, "decode": _lib.SBL_PATH_DECODE, "prefill": _lib.SBL_PATH_PREFILL,
-          "prefill_1cta": _lib.SBL_PATH_PREFILL_1CTA, "prefill_pair": _lib.SBL_PATH_PREFILL_PAIR}
+          "prefill_1cta": _lib.SBL_PATH_PREFILL_1CTA, "prefill_pair": _lib.SBL_PATH_PREFILL_PAIR,
+          "prefill_sparse": _lib.SBL_PATH_PREFILL_SPARSE}
 
 
 def _stream(stream: Optional[torch.cuda.Stream]) -> int:

@@ -42,7 +42,10 @@ extern "C" sbl_status sbl_linear_noalloc(const uint16_t* x_bf16, int64_t T, int6
                                          const float* row_scale, int64_t O, int n, int m, void* y, int y_dtype,
                                          int32_t* acc_out, void* stream) {
     if (T < 0 || K <= 0) return SBL_ERR_INVALID_ARG;
-    const size_t need = sbl_linear_workspace_bytes(T, K, O, n, m);
+    // quantised activations and token scales must fit; sbl_linear takes the
+    // 2:4 sparse path only when the compressed weights fit as well
+    const size_t need = ((static_cast<size_t>(T) * static_cast<size_t>(K) + 255) & ~static_cast<size_t>(255)) +
+                        ((static_cast<size_t>(T) * 4 + 255) & ~static_cast<size_t>(255));
     if (need > static_cast<size_t>(SBL_NOALLOC_SCRATCH_BYTES)) return SBL_ERR_WORKSPACE;
     void* scratch = nullptr;
     if (sbl_status s = scratch_address(&scratch)) return s;

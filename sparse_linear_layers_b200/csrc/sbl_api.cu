@@ -1,6 +1,6 @@
 // C ABI of the Sparse-BitLinear library: argument validation, workspace
 // layout, path dispatch and the per-device status word.  All arithmetic runs
-// in the kernels of prep.cu, quant.cu, decode.cu, prefill.cu and prefill_pair.cu.
+// in the kernels of prep.cu, quant.cu, decode.cu, prefill.cu, prefill_pair.cu and prefill_sp.cu.
 #include <cstdint>
 #include <cstdio>
 #include <cuda_runtime.h>
@@ -21,6 +21,10 @@ cudaError_t launch_prefill(const int8_t* xperm, const float* s_tok, long long T,
                            const float* row_scale, long long O, void* y, int y_bf16, int32_t* acc_out,
                            unsigned* status, int num_sms, int variant, cudaStream_t stream);
 constexpr int kPrefillAuto = 0, kPrefillOneCta = 1, kPrefillPair = 2;
+size_t sp_scratch_bytes(long long O, long long K);
+cudaError_t launch_prefill_sp(const int8_t* xq, const float* s_tok, long long T, long long K, const uint8_t* packed,
+                              const float* row_scale, long long O, void* y, int y_bf16, int32_t* acc_out,
+                              uint8_t* scratch, unsigned* status, int num_sms, cudaStream_t stream);
 #ifdef SBL_TRACE
 cudaError_t set_prefill_trace(void* buf);
 #endif
@@ -115,12 +119,29 @@ sbl_status sbl_quant_act(const uint16_t* x_bf16, int64_t T, int64_t K, int8_t* x
                                        static_cast<cudaStream_t>(stream)));
 }
 
-size_t sbl_linear_workspace_bytes(int64_t T, int64_t K, int64_t O, int n, int m) {
-    (void)O;
-    (void)n;
-    (void)m;
-    if (T <= 0 || K <= 0) return 0;
+// Quantised activations and their scales: what every path needs.
+static size_t base_workspace_bytes(int64_t T, int64_t K) {
     return round256(static_cast<size_t>(T) * static_cast<size_t>(K)) + round256(static_cast<size_t>(T) * 4);
+}
+
+// 2:4 weights on the sparse tensor cores also need their compressed form.
+static bool sparse_eligible(int64_t K, int n, int m) { return n == 2 && m == 4 && K % 64 == 0; }
+
+size_t sbl_linear_workspace_bytes(int64_t T, int64_t K, int64_t O, int n, int m) {
+    if (T <= 0 || K <= 0) return 0;
+    size_t b = base_workspace_bytes(T, K);
+    const bool prefill_sized = T > kDecodeMaxTokens || K > kDecodeMaxK;
+    if (O > 0 && sparse_eligible(K, n, m) && prefill_sized) b += sbl::sp_scratch_bytes(O, K);
+    return b;
+}
+
+// Whether the automatic choice sends a 2:4 prefill to the sparse tensor cores.
+static bool sparse_preferred(int64_t T, int64_t K, int64_t O, int num_sms) {
+    (void)T;
+    (void)K;
+    (void)O;
+    (void)num_sms;
+    return false;
 }
 
 sbl_status sbl_linear_path(const uint16_t* x_bf16, int64_t T, int64_t K, const uint8_t* packed,
@@ -130,7 +151,8 @@ sbl_status sbl_linear_path(const uint16_t* x_bf16, int64_t T, int64_t K, const u
     if (sbl_status s = check_k(K)) return s;
     if (!nm_ok(n, m)) return SBL_ERR_UNSUPPORTED;
     if (y_dtype != SBL_F32 && y_dtype != SBL_BF16) return SBL_ERR_INVALID_ARG;
-    if (path < SBL_PATH_AUTO || path > SBL_PATH_PREFILL_PAIR) return SBL_ERR_INVALID_ARG;
+    if (path < SBL_PATH_AUTO || path > SBL_PATH_PREFILL_SPARSE) return SBL_ERR_INVALID_ARG;
+    if (path == SBL_PATH_PREFILL_SPARSE && !sparse_eligible(K, n, m)) return SBL_ERR_UNSUPPORTED;
     const bool forced_prefill = path >= SBL_PATH_PREFILL;
     if (forced_prefill && K % 64 != 0) return SBL_ERR_UNSUPPORTED;
     if (T == 0 || O == 0) return SBL_OK;
@@ -139,8 +161,12 @@ sbl_status sbl_linear_path(const uint16_t* x_bf16, int64_t T, int64_t K, const u
         return SBL_ERR_INVALID_ARG;
     if (acc_out && !aligned(acc_out, 16)) return SBL_ERR_INVALID_ARG;
     if (T > (1ll << 31) - 1 || O > (1ll << 31) - 1) return SBL_ERR_UNSUPPORTED;
-    const size_t need = sbl_linear_workspace_bytes(T, K, O, n, m);
+    const size_t need = base_workspace_bytes(T, K);
     if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return SBL_ERR_WORKSPACE;
+    // the sparse path runs only in a workspace that also holds the compressed weights
+    const size_t sparse_need = sparse_eligible(K, n, m) ? need + sbl::sp_scratch_bytes(O, K) : 0;
+    const bool sparse_fits = sparse_need != 0 && workspace_bytes >= sparse_need;
+    if (path == SBL_PATH_PREFILL_SPARSE && !sparse_fits) return SBL_ERR_WORKSPACE;
 
     DeviceInfo* d;
     if (sbl_status s = device_info(&d)) return s;
@@ -154,7 +180,15 @@ sbl_status sbl_linear_path(const uint16_t* x_bf16, int64_t T, int64_t K, const u
 
     const int ybf = y_dtype == SBL_BF16 ? 1 : 0;
     cudaError_t e;
-    if (prefill) {
+    const bool sparse = prefill && sparse_fits && (path == SBL_PATH_PREFILL_SPARSE ||
+                                                   (path <= SBL_PATH_PREFILL && sparse_preferred(T, K, O, d->num_sms)));
+    if (sparse) {
+        uint8_t* scratch = static_cast<uint8_t*>(workspace) + need;
+        e = sbl::launch_quant(x_bf16, T, K, xq, s_tok, sbl::kLayoutNatural, d->status, st);
+        if (e != cudaSuccess) return SBL_ERR_CUDA;
+        e = sbl::launch_prefill_sp(xq, s_tok, T, K, packed, row_scale, O, y, ybf, acc_out, scratch, d->status,
+                                   d->num_sms, st);
+    } else if (prefill) {
         e = sbl::launch_quant(x_bf16, T, K, xq, s_tok, sbl::kLayoutInterleaved, d->status, st);
         if (e != cudaSuccess) return SBL_ERR_CUDA;
         const int variant = path == SBL_PATH_PREFILL_1CTA ? sbl::kPrefillOneCta
@@ -188,6 +222,7 @@ sbl_status sbl_device_status(void* stream) {
     if (cudaMemcpy(d->status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return SBL_ERR_CUDA;
     if (word & sbl::kStatusTimeout) return SBL_ERR_TIMEOUT;
     if (word & sbl::kStatusNonfinite) return SBL_ERR_NONFINITE;
+    if (word & sbl::kStatusInvalid) return SBL_ERR_INVALID_ARG;
     return SBL_OK;
 }
 

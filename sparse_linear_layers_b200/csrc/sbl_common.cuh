@@ -10,6 +10,7 @@ namespace sbl {
 // Bits of the per-device status word (see sbl_device_status in sbl.h).
 constexpr unsigned kStatusNonfinite = 1u;
 constexpr unsigned kStatusTimeout = 2u;
+constexpr unsigned kStatusInvalid = 4u;  // input data the kernel cannot represent (not 2:4 where 2:4 is required)
 
 // Upper bound of any pipeline wait: a healthy wait is microseconds; after this
 // the kernel records a timeout and winds down instead of spinning forever.

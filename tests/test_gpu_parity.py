@@ -207,6 +207,68 @@ def test_pair_prefill_full(sbl, O, K, T, n, m):
     assert_bf16_close(yb.cpu().view(torch.int16).numpy(), ref["y"])
 
 
+SPARSE_CASES = [
+    # (O, K, T): 2:4 weights on the structured-sparse MMA.  A full 128 x 160 tile
+    # and K multiple of 256; ragged output rows and token tiles; K % 256 = 64,
+    # 128, 192 (a partial last k-block); the FFN gate and down shapes.
+    (256, 256, 160),
+    (300, 320, 130),
+    (1000, 640, 513),
+    (130, 448, 17),
+    (4864, 896, 2048),
+    (896, 4864, 300),
+]
+
+
+@pytest.mark.parametrize("O,K,T", SPARSE_CASES)
+def test_sparse_prefill_full(sbl, O, K, T):
+    """2:4 weights through the sparse tensor cores, fully compared (fp32 and bf16 outputs)."""
+    W, xbits, xval = layer_inputs(O, K, T, seed=8, outlier_p=0.01)
+    W[0, :8] = 0.0        # all-zero groups
+    W[1, 1::4] = 0.0      # groups with a single kept nonzero at every position
+    W[1, 2::4] = 0.0
+    W[2, ::4] = 0.0
+    W[2, 1::4] = 0.0
+    ref = oracle_layer(W, 2, 4, xval)
+    w = _prep(sbl, W, 2, 4)
+    y, acc = _run_linear(sbl, w, xbits, T, O, "prefill_sparse")
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    assert_fp32_close(y.cpu().numpy(), ref["y"])
+    yb, _ = _run_linear(sbl, w, xbits, T, O, "prefill_sparse", torch.bfloat16)
+    assert_bf16_close(yb.cpu().view(torch.int16).numpy(), ref["y"])
+
+
+def test_sparse_prefill_rejections(sbl):
+    from sparse_linear_layers_b200._lib import SBL_ERR_UNSUPPORTED, SBL_ERR_WORKSPACE, SblError
+    O, K, T = 128, 256, 64
+    W, xbits, _ = layer_inputs(O, K, T, seed=9)
+    w34 = _prep(sbl, W, 3, 4)
+    with pytest.raises(SblError) as e:
+        sbl.sbl_linear(x_dev(xbits), w34, path="prefill_sparse")
+    assert e.value.code == SBL_ERR_UNSUPPORTED
+    w24 = _prep(sbl, W, 2, 4)
+    small = torch.empty((T * K + 4 * T + 512,), dtype=torch.uint8, device="cuda")  # no room for compressed weights
+    with pytest.raises(SblError) as e:
+        sbl.sbl_linear(x_dev(xbits), w24, workspace=small, path="prefill_sparse")
+    assert e.value.code == SBL_ERR_WORKSPACE
+    # the automatic choice falls back to a dense path in that workspace
+    y = sbl.sbl_linear(x_dev(xbits), w24, workspace=small)
+    assert sbl.sbl_device_status() == 0
+    assert torch.isfinite(y).all()
+
+
+def test_sparse_prefill_flags_non_24_codes(sbl):
+    from sparse_linear_layers_b200._lib import SBL_ERR_INVALID_ARG
+    O, K, T = 128, 256, 64
+    W, xbits, _ = layer_inputs(O, K, T, seed=10)
+    w = _prep(sbl, W, 2, 4)
+    packed = w.packed.clone()
+    packed[5, 3] = 0b01010101  # four +1 codes in one group of four
+    bad = sbl.PreparedWeights(packed, w.row_scale, 2, 4, K)
+    sbl.sbl_linear(x_dev(xbits), bad, path="prefill_sparse")
+    assert sbl.sbl_device_status() == SBL_ERR_INVALID_ARG
+
+
 # ------------------------------------------------------------------ full-size layers
 
 @pytest.mark.parametrize("T", [1, 2048])
