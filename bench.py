@@ -282,23 +282,19 @@ def _decode_roofline(sbl, dev, hbm_peak, K=2048, O=7168, reps=64):
             "isolated_call_us": statistics.median(iso) * 1e6}
 
 
-def _prefill_roofline(sbl, dev, int8_peak_tops, hbm_peak, K=896, O=4864, T=32768, reps=10):
-    """One prefill sbl_linear call (activation quantisation + tcgen05 GEMM) on the
-    0.5B FFN gate shape at T = 32768 (3:4, 1% outliers x20), bf16 and fp32
-    outputs; graph-replayed with L2 flushed before each call (every operand is
-    larger than L2 except the 1 MB of codes)."""
-    W = torch.from_numpy(synthetic.latent_weights(O, K, seed=12, tag="prefill-roof")).to(dev)
-    w = sbl.sbl_prepare_weights(W, 3, 4)
+def _prefill_case(sbl, dev, int8_peak_tops, hbm_peak, K, O, n, m, dtypes, T=32768, reps=10, tag="prefill-roof"):
+    """One prefill sbl_linear call (activation quantisation + GEMM) at T tokens,
+    graph-replayed with L2 flushed before each call; x carries 1% outliers x20."""
+    W = torch.from_numpy(synthetic.latent_weights(O, K, seed=12, tag=tag)).to(dev)
+    w = sbl.sbl_prepare_weights(W, n, m)
     del W
-    xb, _ = synthetic.activations(T, K, seed=12, tag="prefill-roof", outlier_p=0.01)
+    xb, _ = synthetic.activations(T, K, seed=12, tag=tag, outlier_p=0.01)
     x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)
-    ws = sbl.workspace_for(T, K, O, 3, 4, dev)
+    ws = sbl.workspace_for(T, K, O, n, m, dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     ops = 2.0 * T * O * K
-    torch.cuda.nvtx.range_push("prefill_roofline")  # lets a profiler select these launches
-    out = {"layer": f"{K}->{O} 3:4 T={T}", "ops_per_call": ops, "peak_tops": int8_peak_tops,
-           "peak_source": "int8 = 2 x measured bf16 burst (nominal dense ratio)"}
-    for name, dt, esz in (("bf16_out", torch.bfloat16, 2), ("fp32_out", torch.float32, 4)):
+    out = {"layer": f"{K}->{O} {n}:{m} T={T}", "ops_per_call": ops}
+    for name, dt, esz in dtypes:
         y = torch.empty((T, O), dtype=dt, device=dev)
         s = torch.cuda.Stream()
         with torch.cuda.stream(s):
@@ -319,12 +315,27 @@ def _prefill_roofline(sbl, dev, int8_peak_tops, hbm_peak, K=896, O=4864, T=32768
                 if i >= 3:
                     ts.append(a.elapsed_time(b) / 1e3)
         t = statistics.median(ts)
-        byts = T * K * 2 + T * K * 2 + O * K / 4 + T * O * esz  # x read, x_q write + read, codes, y
+        byts = T * K * 2 + T * K * 2 + O * K / 4 + T * O * esz  # x read, x_q written + read, codes, y
         out[name] = {"us_per_call": t * 1e6, "tops": ops / t / 1e12, "tensor_frac": ops / t / 1e12 / int8_peak_tops,
                      "algorithmic_bytes": byts, "hbm_gbs": byts / t / 1e9, "hbm_frac": byts / t / 1e9 / hbm_peak}
         del g, y
-    torch.cuda.nvtx.range_pop()
     del w, x, ws, flush
+    return out
+
+
+def _prefill_roofline(sbl, dev, int8_peak_tops, hbm_peak):
+    """The 0.5B FFN shapes at T = 32768, 3:4 against 2:4 (2:4 with K >= 2048 runs on
+    the structured-sparse tensor cores; tensor_frac counts the dense-equivalent
+    2*T*O*K ops).  The gate at 3:4 also with fp32 output."""
+    torch.cuda.nvtx.range_push("prefill_roofline")  # lets a profiler select these launches
+    bf16 = ("bf16_out", torch.bfloat16, 2)
+    out = {"peak_tops": int8_peak_tops, "peak_source": "int8 = 2 x measured bf16 burst (nominal dense ratio)",
+           "gate_3:4": _prefill_case(sbl, dev, int8_peak_tops, hbm_peak, 896, 4864, 3, 4,
+                                     (bf16, ("fp32_out", torch.float32, 4))),
+           "gate_2:4": _prefill_case(sbl, dev, int8_peak_tops, hbm_peak, 896, 4864, 2, 4, (bf16,)),
+           "down_3:4": _prefill_case(sbl, dev, int8_peak_tops, hbm_peak, 4864, 896, 3, 4, (bf16,)),
+           "down_2:4": _prefill_case(sbl, dev, int8_peak_tops, hbm_peak, 4864, 896, 2, 4, (bf16,))}
+    torch.cuda.nvtx.range_pop()
     return out
 
 

@@ -114,6 +114,12 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
 #ifdef SBL_TRACE
     unsigned long long* const trace_buf = blockIdx.x == 0 ? g_trace : nullptr;
 #endif
+    if (threadIdx.x == 0) SBL_TR(14, 0);  // kernel entry
+    if (threadIdx.x == 32) {
+        prefetch_tmap(&tmap_x);
+        prefetch_tmap(&tmap_w);
+        prefetch_tmap(&tmap_y);
+    }
     const int MT = (T + pf::BM - 1) / pf::BM;
     const int NT = (O + BN - 1) / BN;
     const int tiles = MT * NT;
@@ -145,6 +151,7 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
     const uint32_t tmem_base = sm->tmem_base;
     // inputs of this call (quantised activations) come from the preceding kernel
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (threadIdx.x == 0) SBL_TR(15, 0);  // inputs visible
 
     auto give_up = [&]() {
         if (!*abort_flag) {
@@ -174,7 +181,7 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
             int ep_round = 0;
             uint32_t nstore = 0;
             for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
-                const int mt = tile % MT, nt = tile / MT;
+                const int nt = tile % NT, mt = tile / NT;  // output tiles fastest: a token tile is read once
                 const int b = tc & 1;
                 const uint32_t aph = (tc >> 1) & 1;
                 __syncwarp();
@@ -327,7 +334,7 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
             uint32_t it = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-                const int mt = tile % MT, nt = tile / MT;
+                const int nt = tile % NT, mt = tile / NT;  // output tiles fastest: a token tile is read once
                 for (int kb = 0; kb < KB; ++kb, ++it) {
                     const int s = it % Cfg::STAGES;
                     const uint32_t ph = (it / Cfg::STAGES) & 1;
@@ -385,6 +392,7 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
 
     tc_fence_before();
     __syncthreads();
+    if (threadIdx.x == 0) SBL_TR(13, 0);  // every role done
     if (warp == Cfg::WARP_MMA) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(Cfg::TMEM_COLS)

@@ -99,6 +99,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
     const int tiles = MT * NT;
     const int KB = (K + pp::BK - 1) / pp::BK;
 
+    if (threadIdx.x == 32) {
+        prefetch_tmap(&tmap_x);
+        prefetch_tmap(&tmap_w);
+        prefetch_tmap(&tmap_y);
+    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < pp::STAGES; ++s) {
             mbar_init(&sm->full_a[s], 1);
@@ -156,7 +161,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
             int tc = 0;
             uint32_t nstore = 0;
             for (int tile = pair; tile < tiles; tile += npairs, ++tc) {
-                const int mt = tile % MT, nt = tile / MT;
+                const int nt = tile % NT, mt = tile / NT;  // output tiles fastest: a token tile is read once
                 const int b = tc & 1;
                 const uint32_t aph = (tc >> 1) & 1;
                 __syncwarp();
@@ -306,7 +311,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
             uint32_t it = 0;
             bool ok = true;
             for (int tile = pair; tile < tiles && ok; tile += npairs) {
-                const int mt = tile % MT, nt = tile / MT;
+                const int nt = tile % NT, mt = tile / NT;  // output tiles fastest: a token tile is read once
                 const int trow = mt * 2 * pp::BM + static_cast<int>(rank) * pp::BM;
                 const int orow = nt * pp::BN + static_cast<int>(rank) * pp::BNH;
                 for (int kb = 0; kb < KB; ++kb, ++it) {

@@ -184,6 +184,11 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
     const int tiles = MT * NT;
     const int KB = (K + sp::BK - 1) / sp::BK;
 
+    if (threadIdx.x == 32) {
+        prefetch_tmap(&tmap_a);
+        prefetch_tmap(&tmap_x);
+        prefetch_tmap(&tmap_y);
+    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < sp::STAGES; ++s) {
             mbar_init(&sm->full_tma[s], 1);

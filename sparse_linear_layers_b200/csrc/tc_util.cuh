@@ -24,6 +24,12 @@ __device__ __forceinline__ uint32_t i8_idesc() {
            (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Bring a tensor map (a __grid_constant__ kernel parameter) into the descriptor
+// cache before its first TMA use.
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
