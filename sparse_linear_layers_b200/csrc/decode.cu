@@ -21,12 +21,15 @@
 // 16-byte unit of block 4c + w at position w * CPR + c, so the lanes of a row
 // read consecutive units).
 //
-// Arithmetic per 32-bit weight word (16 weights): for j = 0..3 the masks
-// w & (0x01010101 << 2j) and w & (0x02020202 << 2j) pick the +1 and -1 codes
-// of weights 4b + j (scaled by 4^j and 2 * 4^j); one unsigned-by-signed dp4a
-// each against interleaved activation word j accumulates them.  The scales
-// are removed exactly (every partial is a multiple of its power of two)
-// before the L-lane shuffle reduction.
+// Arithmetic per 32-bit weight word (16 weights).  Up to three tokens: for
+// j = 0..3 the masks w & (0x01010101 << 2j) and w & (0x02020202 << 2j) pick
+// the +1 and -1 codes of weights 4b + j (scaled by 4^j and 2 * 4^j); one
+// unsigned-by-signed dp4a each against interleaved activation word j
+// accumulates them, and the scales are removed exactly (every partial is a
+// multiple of its power of two) before the L-lane shuffle reduction.  Four
+// tokens or more: the word is expanded once into four int8x4 words of
+// {-1, 0, +1} and each token takes four signed dp4a, which costs less once
+// the expansion is shared by enough tokens.
 #include "sbl_common.cuh"
 
 namespace sbl {
@@ -63,7 +66,7 @@ __global__ void __launch_bounds__(kDecodeThreads, decode_min_blocks<TT>()) decod
     __shared__ float s_sh[TT];
     asm volatile("griddepcontrol.launch_dependents;");
     constexpr int RW = 32 / L;
-    constexpr int NB = TT >= 8 ? kDecodeBatch / 2 : kDecodeBatch;  // eight tokens: accumulators take the registers
+    constexpr int NB = kDecodeBatch;
     const int CPR = K / (16 * CW);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int sub = lane / L, li = lane % L;
@@ -162,9 +165,17 @@ __global__ void __launch_bounds__(kDecodeThreads, decode_min_blocks<TT>()) decod
         __syncthreads();
     }
 
-    int alo[TT][4], ahi[TT][4];
+    // Four or more tokens: expand each code word once into int8 {-1, 0, +1}
+    // (expand_codes, word j = weights 4b + j) and take one signed dp4a per
+    // activation word and token.  Fewer tokens: split the +1 and -1 codes with
+    // masks (no expansion) and remove their power-of-two scales afterwards.
+    constexpr bool EXPAND = TT >= 4;
+    int acc[TT];
+    int alo[EXPAND ? 1 : TT][4], ahi[EXPAND ? 1 : TT][4];
 #pragma unroll
-    for (int t = 0; t < TT; ++t)
+    for (int t = 0; t < TT; ++t) acc[t] = 0;
+#pragma unroll
+    for (int t = 0; t < (EXPAND ? 1 : TT); ++t)
 #pragma unroll
         for (int j = 0; j < 4; ++j) alo[t][j] = ahi[t][j] = 0;
 
@@ -176,20 +187,33 @@ __global__ void __launch_bounds__(kDecodeThreads, decode_min_blocks<TT>()) decod
 #pragma unroll
             for (int w = 0; w < CW; ++w) {
                 const uint32_t word = wb[b][w];
-                uint32_t mlo[4], mhi[4];
+                if constexpr (EXPAND) {
+                    uint32_t e[4];
+                    expand_codes(word, e);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    mlo[j] = word & (0x01010101u << (2 * j));
-                    mhi[j] = word & (0x02020202u << (2 * j));
-                }
-#pragma unroll
-                for (int t = 0; t < TT; ++t) {
-                    const uint4 xv = xs[t * nblk + w * CPR + c];
-                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                    for (int t = 0; t < TT; ++t) {
+                        const uint4 xv = xs[t * nblk + w * CPR + c];
+                        acc[t] = __dp4a(static_cast<int>(e[0]), static_cast<int>(xv.x), acc[t]);
+                        acc[t] = __dp4a(static_cast<int>(e[1]), static_cast<int>(xv.y), acc[t]);
+                        acc[t] = __dp4a(static_cast<int>(e[2]), static_cast<int>(xv.z), acc[t]);
+                        acc[t] = __dp4a(static_cast<int>(e[3]), static_cast<int>(xv.w), acc[t]);
+                    }
+                } else {
+                    uint32_t mlo[4], mhi[4];
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        alo[t][j] = dp4a_us(mlo[j], xw[j], alo[t][j]);
-                        ahi[t][j] = dp4a_us(mhi[j], xw[j], ahi[t][j]);
+                        mlo[j] = word & (0x01010101u << (2 * j));
+                        mhi[j] = word & (0x02020202u << (2 * j));
+                    }
+#pragma unroll
+                    for (int t = 0; t < TT; ++t) {
+                        const uint4 xv = xs[t * nblk + w * CPR + c];
+                        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            alo[EXPAND ? 0 : t][j] = dp4a_us(mlo[j], xw[j], alo[EXPAND ? 0 : t][j]);
+                            ahi[EXPAND ? 0 : t][j] = dp4a_us(mhi[j], xw[j], ahi[EXPAND ? 0 : t][j]);
+                        }
                     }
                 }
             }
@@ -207,12 +231,13 @@ __global__ void __launch_bounds__(kDecodeThreads, decode_min_blocks<TT>()) decod
         }
     }
 
-    int acc[TT];
 #pragma unroll
     for (int t = 0; t < TT; ++t) {
-        int a = 0;
+        int a = acc[t];
+        if constexpr (!EXPAND) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) a += (alo[t][j] >> (2 * j)) - (ahi[t][j] >> (2 * j + 1));
+            for (int j = 0; j < 4; ++j) a += (alo[t][j] >> (2 * j)) - (ahi[t][j] >> (2 * j + 1));
+        }
 #pragma unroll
         for (int off = L / 2; off >= 1; off >>= 1) a += __shfl_xor_sync(0xFFFFFFFFu, a, off);
         acc[t] = a;
