@@ -56,7 +56,13 @@ __global__ void __launch_bounds__(256) quant_kernel(const uint16_t* __restrict__
     }
 #pragma unroll
     for (int j = 0; j < BPT; ++j) mx = absmax8(v[j][1], absmax8(v[j][0], mx));
-    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+    if constexpr (TPT >= 32) {
+        mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+    } else {
+        // TPT lanes of the warp per token: reduce within each group
+#pragma unroll
+        for (int off = TPT / 2; off >= 1; off >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+    }
     if constexpr (TPT > 32) {
         if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
         __syncthreads();
@@ -109,17 +115,39 @@ static void launch_rr(const uint16_t* x, long long T, long long K, int8_t* xq, f
     quant_kernel<LAYOUT, TPT, BPT><<<blocks, 256, 0, stream>>>(x, T, K, xq, s_tok, status);
 }
 
+static int device_sms() {
+    static int cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cached[dev] && cudaDeviceGetAttribute(&cached[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        cached[dev] = 148;
+    return cached[dev];
+}
+
 template <int LAYOUT>
 static cudaError_t launch_layout(const uint16_t* x, long long T, long long K, int8_t* xq, float* s_tok,
                                  unsigned* status, cudaStream_t stream) {
     const long long nblk = K >> 4;
-    if (nblk <= 32 * 4) launch_rr<LAYOUT, 32, 4>(x, T, K, xq, s_tok, status, stream);
-    else if (nblk <= 64 * 4) launch_rr<LAYOUT, 64, 4>(x, T, K, xq, s_tok, status, stream);
-    else if (nblk <= 128 * 4) launch_rr<LAYOUT, 128, 4>(x, T, K, xq, s_tok, status, stream);
-    else if (nblk <= 256 * 4) launch_rr<LAYOUT, 256, 4>(x, T, K, xq, s_tok, status, stream);
-    else {
+    // Threads per token: the fewest whose registers hold the row (so each thread
+    // has up to four 16-element blocks, eight 16-byte loads, in flight), more
+    // while the grid would be under two blocks per SM.
+    int tpt = 16;
+    while (tpt < 256 && tpt * 4 < nblk) tpt *= 2;
+    const long long min_blocks = 2LL * device_sms();
+    while (tpt < 256 && (T * tpt + 255) / 256 < min_blocks) tpt *= 2;
+    if (nblk > 256 * 4) {
         const unsigned blocks = static_cast<unsigned>((T + 7) / 8);
         quant_kernel_loop<LAYOUT><<<blocks, 256, 0, stream>>>(x, T, K, xq, s_tok, status);
+    } else if (tpt == 16) {
+        launch_rr<LAYOUT, 16, 4>(x, T, K, xq, s_tok, status, stream);
+    } else if (tpt == 32) {
+        launch_rr<LAYOUT, 32, 4>(x, T, K, xq, s_tok, status, stream);
+    } else if (tpt == 64) {
+        launch_rr<LAYOUT, 64, 4>(x, T, K, xq, s_tok, status, stream);
+    } else if (tpt == 128) {
+        launch_rr<LAYOUT, 128, 4>(x, T, K, xq, s_tok, status, stream);
+    } else {
+        launch_rr<LAYOUT, 256, 4>(x, T, K, xq, s_tok, status, stream);
     }
     return cudaGetLastError();
 }
