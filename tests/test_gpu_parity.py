@@ -331,3 +331,56 @@ def test_bounded_wait_times_out_cleanly(sbl):
     w = _prep(sbl, W, 2, 4)
     _, acc = _run_linear(sbl, w, xbits, 4, 64, "prefill")
     assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+
+
+# ------------------------------------------------------------------ streams and graphs
+
+def test_concurrent_streams_in_a_graph(sbl):
+    """Independent projections on separate streams, each with its own workspace,
+    captured into one CUDA graph and replayed twice: every output matches the oracle."""
+    shapes = [(512, 256, 300, 3, 4), (128, 256, 300, 3, 4), (640, 256, 1, 2, 4), (1024, 256, 40, 6, 8)]
+    cases = []
+    for i, (O, K, T, n, m) in enumerate(shapes):
+        W, xbits, xval = layer_inputs(O, K, T, seed=20 + i)
+        ref = oracle_layer(W, n, m, xval)
+        w = _prep(sbl, W, n, m)
+        x = x_dev(xbits)
+        y = torch.empty((T, O), dtype=torch.float32, device="cuda")
+        acc = torch.empty((T, O), dtype=torch.int32, device="cuda")
+        ws = sbl.workspace_for(T, K, O, n, m, torch.device("cuda"))
+        cases.append((w, x, y, acc, ws, ref))
+    main = torch.cuda.Stream()
+    side = [torch.cuda.Stream() for _ in cases]
+
+    def launch():
+        fork = torch.cuda.Event()
+        fork.record(main)
+        joins = []
+        for (w, x, y, acc, ws, _), st in zip(cases, side):
+            st.wait_event(fork)
+            with torch.cuda.stream(st):
+                sbl.sbl_linear(x, w, y=y, acc_out=acc, workspace=ws)
+            ev = torch.cuda.Event()
+            ev.record(st)
+            joins.append(ev)
+        for ev in joins:
+            main.wait_event(ev)
+
+    with torch.cuda.stream(main):
+        launch()  # eager pass before capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=main):
+        launch()
+    for _ in range(2):
+        for _, _, y, acc, _, _ in cases:
+            y.zero_()
+            acc.zero_()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(main):
+            g.replay()
+        torch.cuda.synchronize()
+        assert sbl.sbl_device_status() == 0
+        for _, _, y, acc, _, ref in cases:
+            assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+            assert_fp32_close(y.cpu().numpy(), ref["y"])
