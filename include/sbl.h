@@ -190,6 +190,16 @@ sbl_status sbl_linear_noalloc(const uint16_t* x_bf16, int64_t T, int64_t K,
                               const uint8_t* packed, const float* row_scale, int64_t O, int n, int m,
                               void* y, int y_dtype, int32_t* acc_out, void* stream);
 
+/*
+ * sbl_linear_plan — the contraction path sbl_linear takes for these sizes on
+ * the current device with a workspace of `workspace_bytes`: SBL_PATH_DECODE,
+ * SBL_PATH_PREFILL_1CTA, SBL_PATH_PREFILL_PAIR or SBL_PATH_PREFILL_SPARSE.
+ * Enqueues nothing.  Invalid sizes or patterns return the negated status
+ * (e.g. -SBL_ERR_UNSUPPORTED); a workspace too small for any path returns
+ * -SBL_ERR_WORKSPACE.
+ */
+int sbl_linear_plan(int64_t T, int64_t K, int64_t O, int n, int m, size_t workspace_bytes);
+
 /* Largest T that sbl_linear sends to the decode path. */
 int64_t sbl_decode_max_tokens(void);
 

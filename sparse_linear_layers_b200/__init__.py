@@ -11,7 +11,7 @@ GPU library.
 """
 __version__ = "0.1.0"
 
-_API = ("PreparedWeights", "sbl_decode_max_tokens", "sbl_device_status", "sbl_linear",
+_API = ("PreparedWeights", "sbl_decode_max_tokens", "sbl_device_status", "sbl_linear", "sbl_linear_plan",
         "sbl_linear_workspace_bytes", "sbl_prepare_weights", "sbl_quant_act", "sbl_selftest_bounded_wait",
         "workspace_for", "SblError")
 

@@ -111,6 +111,20 @@ def sbl_linear(x: torch.Tensor, w: PreparedWeights, out_dtype: torch.dtype = tor
     return y
 
 
+_PATH_NAMES = {v: k for k, v in _PATHS.items()}
+
+
+def sbl_linear_plan(T: int, K: int, O: int, n: int, m: int, workspace_bytes: Optional[int] = None) -> str:
+    """Name of the path sbl_linear takes for these sizes ("decode", "prefill_1cta",
+    "prefill_pair" or "prefill_sparse"); the default workspace is workspace_for's."""
+    if workspace_bytes is None:
+        workspace_bytes = max(1, sbl_linear_workspace_bytes(T, K, O, n, m))
+    r = int(lib.sbl_linear_plan(T, K, O, n, m, workspace_bytes))
+    if r < 0:
+        raise _lib.SblError(-r, "sbl_linear_plan")
+    return _PATH_NAMES[r]
+
+
 def sbl_decode_max_tokens() -> int:
     return int(lib.sbl_decode_max_tokens())
 

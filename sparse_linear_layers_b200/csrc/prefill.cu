@@ -477,30 +477,45 @@ cudaError_t launch_prefill_pair(const int8_t* xperm, const float* s_tok, long lo
                                 const uint8_t* packed, const float* row_scale, long long O, void* y, int y_bf16,
                                 int32_t* acc_out, unsigned* status, cudaStream_t stream);
 
-cudaError_t launch_prefill(const int8_t* xperm, const float* s_tok, long long T, long long K, const uint8_t* packed,
-                           const float* row_scale, long long O, void* y, int y_bf16, int32_t* acc_out,
-                           unsigned* status, int num_sms, int variant, cudaStream_t stream) {
-    // Cost model in units of one 128 x 256 tile on one SM: waves of tiles
-    // times the time of one tile.  A narrow 128 x 128 tile costs about 0.65
-    // of a wide one (BN = 256 halves the activation traffic and MMA issue
-    // overhead per output); a CTA pair finishes its 256 x 256 tile in about
-    // kPairCost of a wide one-CTA tile (half the expansion and shared-memory
-    // traffic per SM).
+// The dense tensor-core kernel the automatic choice takes: 0 one CTA with
+// 128-output tiles, 1 one CTA with 256-output tiles, 2 CTA pairs.
+// Cost model in units of one 128 x 256 tile on one SM: waves of tiles times
+// the time of one tile.  A narrow 128 x 128 tile costs about 0.65 of a wide
+// one (BN = 256 halves the activation traffic and MMA issue overhead per
+// output); a CTA pair finishes its 256 x 256 tile in about kPairCost of a wide
+// one-CTA tile (half the expansion and shared-memory traffic per SM).
+int choose_dense_prefill(long long T, long long O, int num_sms, cudaStream_t stream) {
     constexpr double kNarrowCost = 0.65, kPairCost = 0.65;
     const long long mt = (T + pf::BM - 1) / pf::BM;
     const double wide = static_cast<double>((mt * ((O + 255) / 256) + num_sms - 1) / num_sms);
     const double narrow = kNarrowCost * static_cast<double>((mt * ((O + 127) / 128) + num_sms - 1) / num_sms);
-    bool pair = variant == 2;
-    if (variant == 0) {
-        const int clusters = prefill_pair_clusters(stream);
-        if (clusters > 0) {
-            const long long pt = ((T + 255) / 256) * ((O + 255) / 256);
-            pair = kPairCost * static_cast<double>((pt + clusters - 1) / clusters) < (wide < narrow ? wide : narrow);
+    const int clusters = prefill_pair_clusters(stream);
+    if (clusters > 0) {
+        const long long pt = ((T + 255) / 256) * ((O + 255) / 256);
+        if (kPairCost * static_cast<double>((pt + clusters - 1) / clusters) < (wide < narrow ? wide : narrow)) return 2;
+    }
+    return wide <= narrow ? 1 : 0;
+}
+
+cudaError_t launch_prefill(const int8_t* xperm, const float* s_tok, long long T, long long K, const uint8_t* packed,
+                           const float* row_scale, long long O, void* y, int y_bf16, int32_t* acc_out,
+                           unsigned* status, int num_sms, int variant, cudaStream_t stream) {
+    // variant 0: the automatic choice; 1: one CTA (BN by wave count); 2: CTA pairs
+    int kind;
+    if (variant == 2) {
+        kind = 2;
+    } else {
+        kind = choose_dense_prefill(T, O, num_sms, stream);
+        if (variant == 1 && kind == 2) {
+            const long long mt = (T + pf::BM - 1) / pf::BM;
+            const double wide = static_cast<double>((mt * ((O + 255) / 256) + num_sms - 1) / num_sms);
+            const double narrow = 0.65 * static_cast<double>((mt * ((O + 127) / 128) + num_sms - 1) / num_sms);
+            kind = wide <= narrow ? 1 : 0;
         }
     }
-    if (pair)
+    if (kind == 2)
         return launch_prefill_pair(xperm, s_tok, T, K, packed, row_scale, O, y, y_bf16, acc_out, status, stream);
-    if (wide <= narrow)
+    if (kind == 1)
         return launch_prefill_bn<256>(xperm, s_tok, T, K, packed, row_scale, O, y, y_bf16, acc_out, status, num_sms,
                                       stream);
     return launch_prefill_bn<128>(xperm, s_tok, T, K, packed, row_scale, O, y, y_bf16, acc_out, status, num_sms,

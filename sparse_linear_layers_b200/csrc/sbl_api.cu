@@ -21,6 +21,7 @@ cudaError_t launch_prefill(const int8_t* xperm, const float* s_tok, long long T,
                            const float* row_scale, long long O, void* y, int y_bf16, int32_t* acc_out,
                            unsigned* status, int num_sms, int variant, cudaStream_t stream);
 constexpr int kPrefillAuto = 0, kPrefillOneCta = 1, kPrefillPair = 2;
+int choose_dense_prefill(long long T, long long O, int num_sms, cudaStream_t stream);
 size_t sp_scratch_bytes(long long O, long long K);
 cudaError_t launch_prefill_sp(const int8_t* xq, const float* s_tok, long long T, long long K, const uint8_t* packed,
                               const float* row_scale, long long O, void* y, int y_bf16, int32_t* acc_out,
@@ -213,6 +214,22 @@ sbl_status sbl_linear(const uint16_t* x_bf16, int64_t T, int64_t K, const uint8_
 }
 
 int64_t sbl_decode_max_tokens(void) { return kDecodeMaxTokens; }
+
+int sbl_linear_plan(int64_t T, int64_t K, int64_t O, int n, int m, size_t workspace_bytes) {
+    if (T <= 0 || O <= 0) return -static_cast<int>(SBL_ERR_INVALID_ARG);
+    if (sbl_status s = check_k(K)) return -static_cast<int>(s);
+    if (!nm_ok(n, m)) return -static_cast<int>(SBL_ERR_UNSUPPORTED);
+    const bool prefill = ((T > kDecodeMaxTokens) || (K > kDecodeMaxK)) && (K % 64 == 0);
+    if (!prefill) return K > kDecodeMaxK ? -static_cast<int>(SBL_ERR_UNSUPPORTED) : SBL_PATH_DECODE;
+    const size_t need = base_workspace_bytes(T, K);
+    if (workspace_bytes < need) return -static_cast<int>(SBL_ERR_WORKSPACE);
+    DeviceInfo* d;
+    if (sbl_status s = device_info(&d)) return -static_cast<int>(s);
+    if (sparse_eligible(K, n, m) && workspace_bytes >= need + sbl::sp_scratch_bytes(O, K) &&
+        sparse_preferred(T, K, O, d->num_sms))
+        return SBL_PATH_PREFILL_SPARSE;
+    return sbl::choose_dense_prefill(T, O, d->num_sms, nullptr) == 2 ? SBL_PATH_PREFILL_PAIR : SBL_PATH_PREFILL_1CTA;
+}
 
 sbl_status sbl_device_status(void* stream) {
     DeviceInfo* d;

@@ -384,3 +384,18 @@ def test_concurrent_streams_in_a_graph(sbl):
         for _, _, y, acc, _, ref in cases:
             assert np.array_equal(acc.cpu().numpy(), ref["acc"])
             assert_fp32_close(y.cpu().numpy(), ref["y"])
+
+
+def test_linear_plan(sbl):
+    from sparse_linear_layers_b200._lib import SBL_ERR_UNSUPPORTED, SblError
+    assert sbl.sbl_linear_plan(1, 2048, 7168, 2, 4) == "decode"
+    assert sbl.sbl_linear_plan(16, 896, 896, 3, 4) == "decode"
+    assert sbl.sbl_linear_plan(2048, 896, 896, 3, 4) == "prefill_1cta"
+    assert sbl.sbl_linear_plan(32768, 896, 4864, 3, 4) == "prefill_pair"
+    assert sbl.sbl_linear_plan(32768, 2048, 7168, 2, 4) == "prefill_sparse"
+    # 2:4 without room for the compressed weights stays dense
+    base = 32768 * 2048 + 32768 * 4 + 1024
+    assert sbl.sbl_linear_plan(32768, 2048, 7168, 2, 4, workspace_bytes=base) == "prefill_pair"
+    with pytest.raises(SblError) as e:
+        sbl.sbl_linear_plan(64, 256, 128, 1, 4)
+    assert e.value.code == SBL_ERR_UNSUPPORTED
