@@ -98,7 +98,8 @@ sbl_status sbl_prepare_weights(const float* W, int64_t O, int64_t K, int n, int 
  *   s_tok   fp32 [T] (output): s_t = 127 / max(max_k |x_tk|, 1e-5) in IEEE
  *           float division; x_q = clamp(round_half_even(x * s_t), -128, 127)
  *           with the product rounded to float.
- *   Non-finite x sets SBL_ERR_NONFINITE in the device status word.
+ *   Non-finite x sets SBL_ERR_NONFINITE in the device status word; x_q and
+ *   s_tok of that token are then unspecified.
  */
 sbl_status sbl_quant_act(const uint16_t* x_bf16, int64_t T, int64_t K,
                          int8_t* x_q, float* s_tok, void* stream);

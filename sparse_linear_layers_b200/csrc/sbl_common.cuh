@@ -153,11 +153,31 @@ __device__ __forceinline__ void expand_codes(uint32_t w, uint32_t (&out)[4]) {
 }
 
 // ---------------------------------------------------------------- activation quantisation
-// round_half_even(x * s) clamped to int8, x a bf16 bit pattern, s the token's 127 / max|x|.
-__device__ __forceinline__ int quant1(uint32_t bf16_bits, float s) {
-    const float x = __uint_as_float(bf16_bits << 16);
-    const int q = __float2int_rn(__fmul_rn(x, s));
-    return max(-128, min(127, q));
+// round_half_even(x * s) for an activation x (as float) and its token's
+// s = 127 / max|x|, returned as the bit pattern of x * s + 1.5 * 2^23.  The
+// product is rounded to float first, as in the definition; adding 1.5 * 2^23
+// then rounds it to an integer (IEEE round to nearest even) that lands in the
+// low mantissa bits, so the low byte is the int8 two's-complement code.  For
+// finite x, |x * s| <= 127 (s is the correctly rounded 127 / max|x| and
+// |x| <= max|x|), so the clamp to [-128, 127] never acts and is not applied.
+__device__ __forceinline__ uint32_t quant_code_bits(float x, float s) {
+    return __float_as_uint(__fadd_rn(__fmul_rn(x, s), 12582912.0f));
+}
+
+// Low bytes of four code words into one int8x4 word (a in byte 0).
+__device__ __forceinline__ uint32_t pack_codes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    return prmt(prmt(a, b, 0x0040u), prmt(c, d, 0x0040u), 0x5410u);
+}
+
+// Codes of the 16 activations held as eight bf16 pairs (element 2i in the low
+// half of word i, 2i + 1 in the high half).
+__device__ __forceinline__ void quant_codes16(const uint4& u0, const uint4& u1, float s, uint32_t (&q)[16]) {
+    const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        q[2 * i] = quant_code_bits(__uint_as_float(w[i] << 16), s);
+        q[2 * i + 1] = quant_code_bits(__uint_as_float(w[i] & 0xFFFF0000u), s);
+    }
 }
 
 __device__ __forceinline__ uint32_t absmax8(const uint4& u, uint32_t mx) {
@@ -176,23 +196,15 @@ __device__ __forceinline__ uint32_t absmax8(const uint4& u, uint32_t mx) {
 // 4j + b <- element 4b + j, the order of expand_codes()).
 template <bool INTERLEAVED>
 __device__ __forceinline__ uint4 quant_block16(const uint4& u0, const uint4& u1, float s) {
-    const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-    int q[16];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        q[2 * i] = quant1(w[i] & 0xFFFFu, s);
-        q[2 * i + 1] = quant1(w[i] >> 16, s);
-    }
+    uint32_t q[16];
+    quant_codes16(u0, u1, s, q);
     uint32_t o[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int bb = 0; bb < 4; ++bb) {
-            const int src = INTERLEAVED ? (4 * bb + j) : (4 * j + bb);
-            word |= (static_cast<uint32_t>(q[src]) & 0xFFu) << (8 * bb);
-        }
-        o[j] = word;
+        if (INTERLEAVED)
+            o[j] = pack_codes(q[j], q[4 + j], q[8 + j], q[12 + j]);
+        else
+            o[j] = pack_codes(q[4 * j], q[4 * j + 1], q[4 * j + 2], q[4 * j + 3]);
     }
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
