@@ -1,6 +1,6 @@
 // C ABI of the Sparse-BitLinear library: argument validation, workspace
 // layout, path dispatch and the per-device status word.  All arithmetic runs
-// in the kernels of prep.cu, quant.cu, decode.cu, prefill.cu, prefill_pair.cu and prefill_sp.cu.
+// in the kernels of prep.cu, quant.cu, decode.cu, decode_mma.cu, prefill.cu, prefill_pair.cu and prefill_sp.cu.
 #include <cstdint>
 #include <cstdio>
 #include <cuda_runtime.h>
@@ -17,6 +17,10 @@ constexpr int kLayoutNatural = 0, kLayoutInterleaved = 1;
 cudaError_t launch_decode(const uint8_t* packed, const float* row_scale, long long O, long long K,
                           const uint16_t* x, long long T, void* y, int y_bf16, int32_t* acc_out, unsigned* status,
                           int num_sms, cudaStream_t stream);
+bool decode_mma_supported(long long K);
+cudaError_t launch_decode_mma(const uint8_t* packed, const float* row_scale, long long O, long long K,
+                              const uint16_t* x, long long T, void* y, int y_bf16, int32_t* acc_out, unsigned* status,
+                              int num_sms, cudaStream_t stream);
 cudaError_t launch_prefill(const int8_t* xperm, const float* s_tok, long long T, long long K, const uint8_t* packed,
                            const float* row_scale, long long O, void* y, int y_bf16, int32_t* acc_out,
                            unsigned* status, int num_sms, int variant, cudaStream_t stream);
@@ -50,6 +54,7 @@ constexpr int kMaxDevices = 64;
 constexpr long long kMaxK = 1ll << 24;            // keeps |acc| <= 127 * K below 2^31
 constexpr long long kDecodeMaxTokens = 16;
 constexpr long long kDecodeMaxK = 24576;          // decode holds 8 tokens x K int8 in shared memory
+constexpr long long kDecodeMmaMinTokens = 3;      // from here on the decode runs on the warp-level MMA
 
 struct DeviceInfo {
     unsigned* status = nullptr;
@@ -200,8 +205,11 @@ sbl_status sbl_linear_path(const uint16_t* x_bf16, int64_t T, int64_t K, const u
         e = sbl::launch_prefill(xq, s_tok, T, K, packed, row_scale, O, y, ybf, acc_out, d->status, d->num_sms, variant,
                                 st);
     } else {
-        // the decode kernel quantises the activations itself
-        e = sbl::launch_decode(packed, row_scale, O, K, x_bf16, T, y, ybf, acc_out, d->status, d->num_sms, st);
+        // the decode kernels quantise the activations themselves
+        if (T >= kDecodeMmaMinTokens && sbl::decode_mma_supported(K))
+            e = sbl::launch_decode_mma(packed, row_scale, O, K, x_bf16, T, y, ybf, acc_out, d->status, d->num_sms, st);
+        else
+            e = sbl::launch_decode(packed, row_scale, O, K, x_bf16, T, y, ybf, acc_out, d->status, d->num_sms, st);
     }
     return from_cuda(e);
 }

@@ -159,6 +159,23 @@ def test_decode_token_counts(sbl, T):
     assert_fp32_close(y.cpu().numpy(), ref["y"])
 
 
+@pytest.mark.parametrize("O,K,T", [(7168, 2048, 8), (896, 4864, 16), (4864, 896, 3), (48, 24576, 16),
+                                   (136, 2048, 12), (24, 320, 7)])
+def test_decode_mma_shapes(sbl, O, K, T):
+    """Warp-MMA decode: every code-word width (K % 256, % 128, % 64), split-K
+    row tiles, one and two n8 token tiles, passes limited by shared memory,
+    activations re-read past four blocks per thread, ragged row tiles."""
+    n, m = 2, 4
+    W, xbits, xval = layer_inputs(O, K, T, seed=5, outlier_p=0.01)
+    ref = oracle_layer(W, n, m, xval)
+    w = _prep(sbl, W, n, m)
+    y, acc = _run_linear(sbl, w, xbits, T, O, "decode")
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    assert_fp32_close(y.cpu().numpy(), ref["y"])
+    yb, _ = _run_linear(sbl, w, xbits, T, O, "decode", torch.bfloat16)
+    assert_bf16_close(yb.cpu().view(torch.int16).numpy(), ref["y"])
+
+
 def test_decode_k_not_multiple_of_64(sbl):
     O, K, T, n, m = 77, 48, 4, 2, 4
     W, xbits, xval = layer_inputs(O, K, T, seed=3)
