@@ -49,9 +49,19 @@ __device__ unsigned long long* g_trace;
     do {                                                                      \
         if (trace_buf && (i) < 256) trace_buf[(e) * 256 + (i)] = clock64();   \
     } while (0)
+// per-CTA stamps of event e: global timer at g_trace[e * 256 + b] and clock64
+// at g_trace[(e + 20) * 256 + b] for CTA b (the buffer holds 40 x 256 words)
+#define SBL_TRB(e)                                                                          \
+    do {                                                                                    \
+        if (g_trace && blockIdx.x < 256) g_trace[(e) * 256 + blockIdx.x] = global_ns();     \
+        if (g_trace && blockIdx.x < 256) g_trace[((e) + 20) * 256 + blockIdx.x] = clock64(); \
+    } while (0)
 #else
 #define SBL_TR(e, i) \
     do {             \
+    } while (0)
+#define SBL_TRB(e) \
+    do {           \
     } while (0)
 #endif
 
@@ -104,7 +114,7 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                    const __grid_constant__ CUtensorMap tmap_y, int y_vec, const float* __restrict__ row_scale,
                    const float* __restrict__ s_tok, int T, int O, int K, void* __restrict__ y, int y_bf16,
-                   int32_t* __restrict__ acc_out, unsigned* status) {
+                   int32_t* __restrict__ acc_out, int ksplit, int32_t* __restrict__ part, unsigned* status) {
     using Cfg = PrefillCfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     auto* sm = reinterpret_cast<PrefillSmem<BN>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -114,7 +124,9 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
 #ifdef SBL_TRACE
     unsigned long long* const trace_buf = blockIdx.x == 0 ? g_trace : nullptr;
 #endif
+    asm volatile("griddepcontrol.launch_dependents;");
     if (threadIdx.x == 0) SBL_TR(14, 0);  // kernel entry
+    if (threadIdx.x == 0) SBL_TRB(12);
     if (threadIdx.x == 32) {
         prefetch_tmap(&tmap_x);
         prefetch_tmap(&tmap_w);
@@ -124,6 +136,13 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
     const int NT = (O + BN - 1) / BN;
     const int tiles = MT * NT;
     const int KB = (K + pf::BK - 1) / pf::BK;
+    // work items: (tile, k-slice), the slices of a tile on consecutive items
+    const int items = tiles * ksplit;
+    auto kslice = [&](int wi, int& kb0, int& kb1) {
+        const int ks = wi % ksplit;
+        kb0 = static_cast<int>(static_cast<long long>(KB) * ks / ksplit);
+        kb1 = static_cast<int>(static_cast<long long>(KB) * (ks + 1) / ksplit);
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < Cfg::STAGES; ++s) {
@@ -160,7 +179,44 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
         }
     };
 
-    if (warp < pf::EPI_WARPS) {
+    if (BN == 128 && warp < pf::EPI_WARPS && ksplit > 1) {
+        // ------------------------------------------------------------ split-K epilogue
+        // Each work item adds its int32 partial tile into the tile's slot of
+        // `part` with reductions performed at L2 (no round trip), column-major
+        // by token (element (t, c) of a tile at c * 128 + t, so a warp's 32
+        // tokens touch 128 contiguous bytes per column).  The slots are zeroed
+        // by the quantisation kernel before and dequantised by
+        // split_dequant_kernel after this kernel.
+        constexpr int NSL = BN / 32;
+        constexpr size_t kSlot = static_cast<size_t>(pf::BM) * BN;
+        const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+        int tc = 0;
+        for (int wi = blockIdx.x; wi < items; wi += gridDim.x, ++tc) {
+            const int tile = wi / ksplit;
+            const int mt = tile / NT;
+            const int b = tc & 1;
+            const uint32_t aph = (tc >> 1) & 1;
+            if (!warp_wait(&sm->tmem_full[b], aph, abort_flag)) { give_up(); break; }
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + lane_addr + b * BN;
+            if (mt * pf::BM + warp * 32 < T) {
+                int32_t* slot = part + static_cast<size_t>(tile) * kSlot + warp * 32 + lane;
+#pragma unroll 1
+                for (int k = 0; k < NSL; ++k) {
+                    uint32_t cur[32];
+                    tmem_ld32_nowait(tbase + 32 * k, cur);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        asm volatile("red.relaxed.gpu.global.add.s32 [%0], %1;" ::"l"(slot + (32 * k + i) * pf::BM),
+                                     "r"(cur[i])
+                                     : "memory");
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&sm->tmem_empty[b]);  // the accumulator buffer is free for the MMA
+        }
+    } else if (warp < pf::EPI_WARPS) {
         // ------------------------------------------------------------ epilogue
         // Warp w owns TMEM lanes 32w .. 32w + 31 (32 tokens of the tile).  Per
         // tile it first copies the tile's row scales into its own shared-memory
@@ -297,8 +353,10 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
         const int r = threadIdx.x - pf::EPI_WARPS * 32;  // row of the B tile
         uint32_t it = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-            for (int kb = 0; kb < KB; ++kb, ++it) {
+        for (int wi = blockIdx.x; wi < items && ok; wi += gridDim.x) {
+            int kb0, kb1;
+            kslice(wi, kb0, kb1);
+            for (int kb = kb0; kb < kb1; ++kb, ++it) {
                 const int s = it % Cfg::STAGES;
                 const uint32_t ph = (it / Cfg::STAGES) & 1;
                 // the codes have landed, and the producer only issued them once the
@@ -333,9 +391,12 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
         if (lane == 0) {
             uint32_t it = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+            for (int wi = blockIdx.x; wi < items && ok; wi += gridDim.x) {
+                const int tile = wi / ksplit;
                 const int nt = tile % NT, mt = tile / NT;  // output tiles fastest: a token tile is read once
-                for (int kb = 0; kb < KB; ++kb, ++it) {
+                int kb0, kb1;
+                kslice(wi, kb0, kb1);
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % Cfg::STAGES;
                     const uint32_t ph = (it / Cfg::STAGES) & 1;
                     if (!mbar_wait(&sm->empty[s], ph ^ 1, abort_flag)) { give_up(); ok = false; break; }
@@ -361,13 +422,15 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
             uint32_t it = 0;
             int tc = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++tc) {
+            for (int wi = blockIdx.x; wi < items && ok; wi += gridDim.x, ++tc) {
                 const int b = tc & 1;
                 const uint32_t aph = (tc >> 1) & 1;
                 if (!mbar_wait(&sm->tmem_empty[b], aph ^ 1, abort_flag)) { give_up(); break; }
                 tc_fence_after();
                 const uint32_t d = tmem_base + b * BN;
-                for (int kb = 0; kb < KB; ++kb, ++it) {
+                int kb0, kb1;
+                kslice(wi, kb0, kb1);
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % Cfg::STAGES;
                     const uint32_t ph = (it / Cfg::STAGES) & 1;
                     if (!mbar_wait(&sm->full_tma[s], ph, abort_flag) || !mbar_wait(&sm->full_dec[s], ph, abort_flag)) {
@@ -377,7 +440,7 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
                     const uint32_t a0 = smem_u32(sm->a[s]), b0 = smem_u32(sm->b[s]);
 #pragma unroll
                     for (int kk = 0; kk < pf::BK / 32; ++kk)
-                        tc_mma(d, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc, (kb | kk) != 0);
+                        tc_mma(d, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc, (kb != kb0) || (kk != 0));
                     tc_commit(&sm->empty[s]);
                 }
                 if (ok) tc_commit(&sm->tmem_full[b]);
@@ -393,6 +456,7 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
     tc_fence_before();
     __syncthreads();
     if (threadIdx.x == 0) SBL_TR(13, 0);  // every role done
+    if (threadIdx.x == 0) SBL_TRB(16);
     if (warp == Cfg::WARP_MMA) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(Cfg::TMEM_COLS)
@@ -403,7 +467,8 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
 template <int BN>
 static cudaError_t launch_prefill_bn(const int8_t* xperm, const float* s_tok, long long T, long long K,
                                      const uint8_t* packed, const float* row_scale, long long O, void* y, int y_bf16,
-                                     int32_t* acc_out, unsigned* status, int num_sms, cudaStream_t stream) {
+                                     int32_t* acc_out, int ksplit, int32_t* part, unsigned* status,
+                                     int num_sms, cudaStream_t stream) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return cudaErrorNotSupported;
     CUtensorMap map_x, map_w;
@@ -449,8 +514,8 @@ static cudaError_t launch_prefill_bn(const int8_t* xperm, const float* s_tok, lo
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
-    const long long tiles = ((T + pf::BM - 1) / pf::BM) * ((O + BN - 1) / BN);
-    const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
+    const long long items = ((T + pf::BM - 1) / pf::BM) * ((O + BN - 1) / BN) * ksplit;
+    const int grid = static_cast<int>(items < num_sms ? items : num_sms);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(PrefillCfg<BN>::THREADS);
@@ -462,7 +527,7 @@ static cudaError_t launch_prefill_bn(const int8_t* xperm, const float* s_tok, lo
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, prefill_kernel<BN>, map_x, map_w, map_y, y_vec, row_scale, s_tok, static_cast<int>(T),
-                              static_cast<int>(O), static_cast<int>(K), y, y_bf16, acc_out, status);
+                              static_cast<int>(O), static_cast<int>(K), y, y_bf16, acc_out, ksplit, part, status);
 }
 
 #ifdef SBL_TRACE
@@ -497,10 +562,100 @@ int choose_dense_prefill(long long T, long long O, int num_sms, cudaStream_t str
     return wide <= narrow ? 1 : 0;
 }
 
+// Dequantisation of split-K accumulators: y[t, o] = acc[t, o] * row_scale[o] *
+// (1 / s_tok[t]), the float steps of the one-CTA epilogue.  A block of 8 warps
+// takes 32 tokens x 32 outputs: it reads the column-major slots with lanes
+// along tokens, transposes through shared memory and writes output rows with
+// lanes along outputs.  A programmatic dependent of the contraction kernel.
+__global__ void __launch_bounds__(256) split_dequant_kernel(const int32_t* __restrict__ part,
+                                                            const float* __restrict__ row_scale,
+                                                            const float* __restrict__ s_tok, int T, int O,
+                                                            void* __restrict__ y, int y_bf16,
+                                                            int32_t* __restrict__ acc_out) {
+    __shared__ int box[32][33];
+    asm volatile("griddepcontrol.launch_dependents;");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int lane = threadIdx.x & 31, wy = threadIdx.x >> 5;
+    const int o0 = blockIdx.x * 32, t0 = blockIdx.y * 32;
+    const int NT = (O + 127) / 128;
+    const int t = t0 + lane;
+#pragma unroll
+    for (int j = wy; j < 32; j += 8) {
+        const int o = o0 + j;
+        int v = 0;
+        if (t < T && o < O) {
+            const size_t tile = static_cast<size_t>(t / pf::BM) * NT + o / 128;
+            v = __ldcg(part + tile * (pf::BM * 128) + (o % 128) * pf::BM + (t % pf::BM));
+        }
+        box[j][lane] = v;
+    }
+    __syncthreads();
+    const int o = o0 + lane;
+    if (o >= O) return;
+    const float sc = __ldg(row_scale + o);
+#pragma unroll
+    for (int r = wy; r < 32; r += 8) {
+        const int tt = t0 + r;
+        if (tt >= T) break;
+        const int a = box[lane][r];
+        const float f = __fmul_rn(__fmul_rn(static_cast<float>(a), sc), __frcp_rn(s_tok[tt]));
+        const size_t idx = static_cast<size_t>(tt) * O + o;
+        if (y_bf16)
+            reinterpret_cast<__nv_bfloat16_raw*>(y)[idx] = static_cast<__nv_bfloat16_raw>(__float2bfloat16_rn(f));
+        else
+            reinterpret_cast<float*>(y)[idx] = f;
+        if (acc_out) acc_out[idx] = a;
+    }
+}
+
+// Split-K plan of the one-CTA kernel with 128-output tiles: when its tiles
+// fill at most half of the SMs, each tile's k-blocks are divided among up to
+// num_sms / tiles CTAs (at most 16, at least two k-blocks each).  Measured on
+// B200, a split costs about as much as 8 to 10 k-blocks of one CTA (L2
+// reductions and the dequantisation kernel), so it is taken only when it
+// removes at least 12 k-blocks from each CTA's run.  Returns the number of
+// slices (1: no split).
+int prefill_ksplit(long long T, long long K, long long O, int num_sms) {
+    const long long tiles = ((T + pf::BM - 1) / pf::BM) * ((O + 127) / 128);
+    const long long kb = (K + pf::BK - 1) / pf::BK;
+    if (tiles * 2 > num_sms || kb < 4) return 1;
+    long long ks = num_sms / tiles;
+    if (ks > kb / 2) ks = kb / 2;
+    if (ks > 16) ks = 16;
+    if (ks < 2 || kb - (kb + ks - 1) / ks < 12) return 1;
+    return static_cast<int>(ks);
+}
+
+// Workspace of a split: one int32 accumulator tile (128 tokens x 128 outputs)
+// per tile, zero when the contraction kernel starts.
+size_t prefill_split_part_bytes(long long T, long long O, int ksplit) {
+    const size_t tiles = static_cast<size_t>((T + pf::BM - 1) / pf::BM) * ((O + 127) / 128);
+    return ksplit > 1 ? tiles * pf::BM * 128 * 4 : 0;
+}
+
 cudaError_t launch_prefill(const int8_t* xperm, const float* s_tok, long long T, long long K, const uint8_t* packed,
                            const float* row_scale, long long O, void* y, int y_bf16, int32_t* acc_out,
-                           unsigned* status, int num_sms, int variant, cudaStream_t stream) {
-    // variant 0: the automatic choice; 1: one CTA (BN by wave count); 2: CTA pairs
+                           unsigned* status, int num_sms, int variant, int ksplit, int32_t* part,
+                           cudaStream_t stream) {
+    // variant 0: the automatic choice; 1: one CTA (BN by wave count); 2: CTA pairs.
+    // ksplit > 1 (not with CTA pairs): the one-CTA kernel with 128-output tiles,
+    // split along k into `part` (zero on entry), then split_dequant_kernel.
+    if (ksplit > 1 && variant != 2) {
+        cudaError_t e = launch_prefill_bn<128>(xperm, s_tok, T, K, packed, row_scale, O, y, y_bf16, acc_out, ksplit,
+                                               part, status, num_sms, stream);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>((O + 31) / 32), static_cast<unsigned>((T + 31) / 32));
+        cfg.blockDim = dim3(256);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, split_dequant_kernel, static_cast<const int32_t*>(part), row_scale, s_tok,
+                                  static_cast<int>(T), static_cast<int>(O), y, y_bf16, acc_out);
+    }
     int kind;
     if (variant == 2) {
         kind = 2;
@@ -516,10 +671,10 @@ cudaError_t launch_prefill(const int8_t* xperm, const float* s_tok, long long T,
     if (kind == 2)
         return launch_prefill_pair(xperm, s_tok, T, K, packed, row_scale, O, y, y_bf16, acc_out, status, stream);
     if (kind == 1)
-        return launch_prefill_bn<256>(xperm, s_tok, T, K, packed, row_scale, O, y, y_bf16, acc_out, status, num_sms,
-                                      stream);
-    return launch_prefill_bn<128>(xperm, s_tok, T, K, packed, row_scale, O, y, y_bf16, acc_out, status, num_sms,
-                                  stream);
+        return launch_prefill_bn<256>(xperm, s_tok, T, K, packed, row_scale, O, y, y_bf16, acc_out, 1, nullptr,
+                                      status, num_sms, stream);
+    return launch_prefill_bn<128>(xperm, s_tok, T, K, packed, row_scale, O, y, y_bf16, acc_out, 1, nullptr, status,
+                                  num_sms, stream);
 }
 
 }  // namespace sbl

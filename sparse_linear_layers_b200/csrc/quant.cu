@@ -28,12 +28,20 @@ __device__ __forceinline__ void quant_block_store(const uint4& u0, const uint4& 
     *reinterpret_cast<uint4*>(out_row + 16 * static_cast<long long>(b)) = quant_block16<LAYOUT != kNatural>(u0, u1, s);
 }
 
+// Zero `n16` 16-byte words at p, spread over the whole grid.
+__device__ __forceinline__ void zero_fill(uint4* p, long long n16) {
+    const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n16; i += stride)
+        p[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
 // Register-resident variant: K / 16 <= TPT * BPT.
 template <int LAYOUT, int TPT, int BPT>
 __global__ void __launch_bounds__(256) quant_kernel(const uint16_t* __restrict__ x, long long T, long long K,
                                                     int8_t* __restrict__ xq, float* __restrict__ s_tok,
-                                                    unsigned* status) {
+                                                    uint4* __restrict__ zero_words, long long nzero, unsigned* status) {
     asm volatile("griddepcontrol.launch_dependents;");
+    zero_fill(zero_words, nzero);
     constexpr int TPC = 256 / TPT;
     __shared__ uint32_t red[8];
     const int sub = threadIdx.x / TPT, tr = threadIdx.x % TPT;
@@ -87,8 +95,9 @@ __global__ void __launch_bounds__(256) quant_kernel(const uint16_t* __restrict__
 template <int LAYOUT>
 __global__ void __launch_bounds__(256) quant_kernel_loop(const uint16_t* __restrict__ x, long long T, long long K,
                                                          int8_t* __restrict__ xq, float* __restrict__ s_tok,
-                                                         unsigned* status) {
+                                                         uint4* __restrict__ zero_words, long long nzero, unsigned* status) {
     asm volatile("griddepcontrol.launch_dependents;");
+    zero_fill(zero_words, nzero);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long t = static_cast<long long>(blockIdx.x) * 8 + warp;
     if (t >= T) return;
@@ -108,11 +117,11 @@ __global__ void __launch_bounds__(256) quant_kernel_loop(const uint16_t* __restr
 }
 
 template <int LAYOUT, int TPT, int BPT>
-static void launch_rr(const uint16_t* x, long long T, long long K, int8_t* xq, float* s_tok, unsigned* status,
-                      cudaStream_t stream) {
+static void launch_rr(const uint16_t* x, long long T, long long K, int8_t* xq, float* s_tok, uint4* zero_words,
+                      long long nzero, unsigned* status, cudaStream_t stream) {
     constexpr int TPC = 256 / TPT;
     const unsigned blocks = static_cast<unsigned>((T + TPC - 1) / TPC);
-    quant_kernel<LAYOUT, TPT, BPT><<<blocks, 256, 0, stream>>>(x, T, K, xq, s_tok, status);
+    quant_kernel<LAYOUT, TPT, BPT><<<blocks, 256, 0, stream>>>(x, T, K, xq, s_tok, zero_words, nzero, status);
 }
 
 static int device_sms() {
@@ -126,7 +135,7 @@ static int device_sms() {
 
 template <int LAYOUT>
 static cudaError_t launch_layout(const uint16_t* x, long long T, long long K, int8_t* xq, float* s_tok,
-                                 unsigned* status, cudaStream_t stream) {
+                                 uint4* zero_words, long long nzero, unsigned* status, cudaStream_t stream) {
     const long long nblk = K >> 4;
     // Threads per token: the fewest whose registers hold the row (so each thread
     // has up to four 16-element blocks, eight 16-byte loads, in flight), more
@@ -137,26 +146,30 @@ static cudaError_t launch_layout(const uint16_t* x, long long T, long long K, in
     while (tpt < 256 && (T * tpt + 255) / 256 < min_blocks) tpt *= 2;
     if (nblk > 256 * 4) {
         const unsigned blocks = static_cast<unsigned>((T + 7) / 8);
-        quant_kernel_loop<LAYOUT><<<blocks, 256, 0, stream>>>(x, T, K, xq, s_tok, status);
+        quant_kernel_loop<LAYOUT><<<blocks, 256, 0, stream>>>(x, T, K, xq, s_tok, zero_words, nzero, status);
     } else if (tpt == 16) {
-        launch_rr<LAYOUT, 16, 4>(x, T, K, xq, s_tok, status, stream);
+        launch_rr<LAYOUT, 16, 4>(x, T, K, xq, s_tok, zero_words, nzero, status, stream);
     } else if (tpt == 32) {
-        launch_rr<LAYOUT, 32, 4>(x, T, K, xq, s_tok, status, stream);
+        launch_rr<LAYOUT, 32, 4>(x, T, K, xq, s_tok, zero_words, nzero, status, stream);
     } else if (tpt == 64) {
-        launch_rr<LAYOUT, 64, 4>(x, T, K, xq, s_tok, status, stream);
+        launch_rr<LAYOUT, 64, 4>(x, T, K, xq, s_tok, zero_words, nzero, status, stream);
     } else if (tpt == 128) {
-        launch_rr<LAYOUT, 128, 4>(x, T, K, xq, s_tok, status, stream);
+        launch_rr<LAYOUT, 128, 4>(x, T, K, xq, s_tok, zero_words, nzero, status, stream);
     } else {
-        launch_rr<LAYOUT, 256, 4>(x, T, K, xq, s_tok, status, stream);
+        launch_rr<LAYOUT, 256, 4>(x, T, K, xq, s_tok, zero_words, nzero, status, stream);
     }
     return cudaGetLastError();
 }
 
+// zero16[0 .. nzero16) (16-byte words) are set to zero as well: the split-K
+// accumulators of the contraction that follows.
 cudaError_t launch_quant(const uint16_t* x, long long T, long long K, int8_t* xq, float* s_tok, int layout,
-                         unsigned* status, cudaStream_t stream) {
+                         unsigned* status, cudaStream_t stream, void* zero16, long long nzero16) {
+    uint4* zero_words = static_cast<uint4*>(zero16);
+    const long long nzero = nzero16;
     switch (layout) {
-        case kInterleaved: return launch_layout<kInterleaved>(x, T, K, xq, s_tok, status, stream);
-        default: return launch_layout<kNatural>(x, T, K, xq, s_tok, status, stream);
+        case kInterleaved: return launch_layout<kInterleaved>(x, T, K, xq, s_tok, zero_words, nzero, status, stream);
+        default: return launch_layout<kNatural>(x, T, K, xq, s_tok, zero_words, nzero, status, stream);
     }
 }
 

@@ -12,7 +12,7 @@ namespace sbl {
 cudaError_t launch_prep(const float* W, long long O, long long K, int n, int m, uint8_t* packed, float* row_scale,
                         uint8_t* mask_bits, unsigned* status, cudaStream_t stream);
 cudaError_t launch_quant(const uint16_t* x, long long T, long long K, int8_t* xq, float* s_tok, int layout,
-                         unsigned* status, cudaStream_t stream);
+                         unsigned* status, cudaStream_t stream, void* zero16 = nullptr, long long nzero16 = 0);
 constexpr int kLayoutNatural = 0, kLayoutInterleaved = 1;
 cudaError_t launch_decode(const uint8_t* packed, const float* row_scale, long long O, long long K,
                           const uint16_t* x, long long T, void* y, int y_bf16, int32_t* acc_out, unsigned* status,
@@ -23,8 +23,11 @@ cudaError_t launch_decode_mma(const uint8_t* packed, const float* row_scale, lon
                               int num_sms, cudaStream_t stream);
 cudaError_t launch_prefill(const int8_t* xperm, const float* s_tok, long long T, long long K, const uint8_t* packed,
                            const float* row_scale, long long O, void* y, int y_bf16, int32_t* acc_out,
-                           unsigned* status, int num_sms, int variant, cudaStream_t stream);
+                           unsigned* status, int num_sms, int variant, int ksplit, int32_t* part,
+                           cudaStream_t stream);
 constexpr int kPrefillAuto = 0, kPrefillOneCta = 1, kPrefillPair = 2;
+int prefill_ksplit(long long T, long long K, long long O, int num_sms);
+size_t prefill_split_part_bytes(long long T, long long O, int ksplit);
 int choose_dense_prefill(long long T, long long O, int num_sms, cudaStream_t stream);
 size_t sp_scratch_bytes(long long O, long long K);
 cudaError_t launch_prefill_sp(const int8_t* xq, const float* s_tok, long long T, long long K, const uint8_t* packed,
@@ -133,11 +136,28 @@ static size_t base_workspace_bytes(int64_t T, int64_t K) {
 // 2:4 weights on the sparse tensor cores also need their compressed form.
 static bool sparse_eligible(int64_t K, int n, int m) { return n == 2 && m == 4 && K % 64 == 0; }
 
+// Split-K area of the one-CTA prefill (one int32 accumulator tile per output
+// tile); 0 when the sizes take no split.
+static size_t split_bytes(int64_t T, int64_t K, int64_t O, int num_sms, int* ksplit = nullptr) {
+    const int ks = sbl::prefill_ksplit(T, K, O, num_sms);
+    if (ksplit) *ksplit = ks;
+    if (ks <= 1) return 0;
+    return sbl::prefill_split_part_bytes(T, O, ks);
+}
+
 size_t sbl_linear_workspace_bytes(int64_t T, int64_t K, int64_t O, int n, int m) {
     if (T <= 0 || K <= 0) return 0;
     size_t b = base_workspace_bytes(T, K);
     const bool prefill_sized = T > kDecodeMaxTokens || K > kDecodeMaxK;
-    if (O > 0 && sparse_eligible(K, n, m) && prefill_sized) b += sbl::sp_scratch_bytes(O, K);
+    if (O > 0 && prefill_sized && K % 64 == 0) {
+        size_t extra = sparse_eligible(K, n, m) ? sbl::sp_scratch_bytes(O, K) : 0;
+        DeviceInfo* d;
+        if (device_info(&d) == SBL_OK) {
+            const size_t sb = split_bytes(T, K, O, d->num_sms);
+            if (sb > extra) extra = sb;
+        }
+        b += extra;
+    }
     return b;
 }
 
@@ -197,13 +217,28 @@ sbl_status sbl_linear_path(const uint16_t* x_bf16, int64_t T, int64_t K, const u
         e = sbl::launch_prefill_sp(xq, s_tok, T, K, packed, row_scale, O, y, ybf, acc_out, scratch, d->status,
                                    d->num_sms, st);
     } else if (prefill) {
-        e = sbl::launch_quant(x_bf16, T, K, xq, s_tok, sbl::kLayoutInterleaved, d->status, st);
+        // a split along k when the one-CTA tiles would leave most SMs idle and
+        // the workspace holds the accumulator tiles, which the quantisation
+        // kernel zeroes
+        int ksplit = 1;
+        int32_t* part = nullptr;
+        long long nzero16 = 0;
+        if (path != SBL_PATH_PREFILL_PAIR) {
+            int ks = 1;
+            const size_t sb = split_bytes(T, K, O, d->num_sms, &ks);
+            if (ks > 1 && workspace_bytes >= need + sb) {
+                ksplit = ks;
+                part = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + need);
+                nzero16 = static_cast<long long>(sb / 16);
+            }
+        }
+        e = sbl::launch_quant(x_bf16, T, K, xq, s_tok, sbl::kLayoutInterleaved, d->status, st, part, nzero16);
         if (e != cudaSuccess) return SBL_ERR_CUDA;
         const int variant = path == SBL_PATH_PREFILL_1CTA ? sbl::kPrefillOneCta
                             : path == SBL_PATH_PREFILL_PAIR ? sbl::kPrefillPair
                                                             : sbl::kPrefillAuto;
         e = sbl::launch_prefill(xq, s_tok, T, K, packed, row_scale, O, y, ybf, acc_out, d->status, d->num_sms, variant,
-                                st);
+                                ksplit, part, st);
     } else {
         // the decode kernels quantise the activations themselves
         if (T >= kDecodeMmaMinTokens && sbl::decode_mma_supported(K))
@@ -236,6 +271,9 @@ int sbl_linear_plan(int64_t T, int64_t K, int64_t O, int n, int m, size_t worksp
     if (sparse_eligible(K, n, m) && workspace_bytes >= need + sbl::sp_scratch_bytes(O, K) &&
         sparse_preferred(T, K, O, d->num_sms))
         return SBL_PATH_PREFILL_SPARSE;
+    int ks = 1;
+    const size_t sb = split_bytes(T, K, O, d->num_sms, &ks);
+    if (ks > 1 && workspace_bytes >= need + sb) return SBL_PATH_PREFILL_1CTA;
     return sbl::choose_dense_prefill(T, O, d->num_sms, nullptr) == 2 ? SBL_PATH_PREFILL_PAIR : SBL_PATH_PREFILL_1CTA;
 }
 

@@ -176,6 +176,29 @@ def test_decode_mma_shapes(sbl, O, K, T):
     assert_bf16_close(yb.cpu().view(torch.int16).numpy(), ref["y"])
 
 
+@pytest.mark.parametrize("O,K,T,n,m", [(2048, 7168, 64, 2, 4), (896, 4864, 64, 3, 4), (300, 4096, 40, 6, 8),
+                                       (512, 2048, 200, 2, 4)])
+def test_prefill_split_k(sbl, O, K, T, n, m):
+    """One-CTA prefill split along k (few tiles, long K): the automatic path
+    takes it, a second call on the same workspace agrees (the accumulators
+    are zeroed every call), and ragged token and row counts are covered."""
+    assert sbl.sbl_linear_plan(T, K, O, n, m) == "prefill_1cta"
+    W, xbits, xval = layer_inputs(O, K, T, seed=6, outlier_p=0.01)
+    ref = oracle_layer(W, n, m, xval)
+    w = _prep(sbl, W, n, m)
+    ws = sbl.workspace_for(T, K, O, n, m, "cuda")
+    assert ws.numel() > T * K + 4 * T + 512  # the split area is part of the default workspace
+    for out_dtype in (torch.float32, torch.bfloat16, torch.float32):
+        acc = torch.empty((T, O), dtype=torch.int32, device="cuda")
+        y = sbl.sbl_linear(x_dev(xbits), w, out_dtype=out_dtype, acc_out=acc, workspace=ws)
+        assert sbl.sbl_device_status() == 0
+        assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+        if out_dtype == torch.float32:
+            assert_fp32_close(y.cpu().numpy(), ref["y"])
+        else:
+            assert_bf16_close(y.cpu().view(torch.int16).numpy(), ref["y"])
+
+
 def test_decode_k_not_multiple_of_64(sbl):
     O, K, T, n, m = 77, 48, 4, 2, 4
     W, xbits, xval = layer_inputs(O, K, T, seed=3)
