@@ -47,7 +47,7 @@ WORKLOAD = "qwen2.5-0.5b layer projections (q,k,v,o,gate,up,down), 3:4, prep + T
 # capture of this step's eager pass (dram__bytes_read.sum + dram__bytes_write.sum).
 # Only valid for the kernel sources the counters were taken on; reported as null
 # once those change.
-PREFILL_TRAFFIC = {"sources_sha256": "7d7f8e9947500fc795448fa6caac0af1ab904c700de671be638a97456a760f5b", "bytes_per_call": 9612398}
+PREFILL_TRAFFIC = {"sources_sha256": "8c37b854e885afcdb1149611a5095429e4dbce19a7194b55bf9af2ecf46baf75", "bytes_per_call": 9617993}
 
 
 def _kernel_sources_digest():
@@ -284,8 +284,8 @@ class E2E:
         self.main.wait_stream(self.back)
 
 
-def _decode_roofline(sbl, dev, hbm_peak, K=2048, O=7168, reps=64):
-    """T = 1 decode of a 2048 -> 7168 layer over a pool of distinct packed weights
+def _decode_roofline(sbl, dev, hbm_peak, K=2048, O=7168, T=1, reps=64):
+    """T-token decode of a 2048 -> 7168 layer over a pool of distinct packed weights
     larger than 3x L2, replayed from a CUDA graph: per-call GB/s on algorithmic bytes."""
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     per = O * K // 4
@@ -294,10 +294,10 @@ def _decode_roofline(sbl, dev, hbm_peak, K=2048, O=7168, reps=64):
     base = sbl.sbl_prepare_weights(W, 2, 4)
     del W
     packs = [base.packed.clone() for _ in range(pool)]
-    x1 = torch.from_numpy(synthetic.activations(1, K, seed=11, tag="decode-x")[0].view(np.int16)).view(
+    x1 = torch.from_numpy(synthetic.activations(T, K, seed=11, tag="decode-x")[0].view(np.int16)).view(
         torch.bfloat16).to(dev)
-    y1 = torch.empty((1, O), dtype=torch.float32, device=dev)
-    ws = sbl.workspace_for(1, K, O, 2, 4, dev)
+    y1 = torch.empty((T, O), dtype=torch.float32, device=dev)
+    ws = sbl.workspace_for(T, K, O, 2, 4, dev)
     ws_list = [sbl.PreparedWeights(p, base.row_scale, 2, 4, K) for p in packs]
     s = torch.cuda.Stream()
     with torch.cuda.stream(s):
@@ -335,10 +335,10 @@ def _decode_roofline(sbl, dev, hbm_peak, K=2048, O=7168, reps=64):
         b.record()
         torch.cuda.synchronize()
         iso.append(a.elapsed_time(b) / 1e3)
-    byts = O * K / 4 + 4 * O + 2 * K + 4 * O
+    byts = O * K / 4 + 4 * O + T * (2 * K + 4 * O)
     del g, packs, ws_list, flush
     ach = byts / per_call_s / 1e9
-    return {"layer": f"{K}->{O} 2:4 T=1", "bytes_per_call": byts, "calls_in_graph": reps, "weight_pool": pool,
+    return {"layer": f"{K}->{O} 2:4 T={T}", "bytes_per_call": byts, "calls_in_graph": reps, "weight_pool": pool,
             "us_per_call": per_call_s * 1e6, "achieved_gbs": ach, "peak_gbs": hbm_peak, "frac": ach / hbm_peak,
             "isolated_call_us": statistics.median(iso) * 1e6}
 
@@ -354,7 +354,11 @@ def _prefill_case(sbl, dev, int8_peak_tops, hbm_peak, K, O, n, m, dtypes, T=3276
     ws = sbl.workspace_for(T, K, O, n, m, dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     ops = 2.0 * T * O * K
-    out = {"layer": f"{K}->{O} {n}:{m} T={T}", "ops_per_call": ops}
+    path = sbl.sbl_linear_plan(T, K, O, n, m, ws.numel())
+    # the sparse tensor cores run at twice the dense rate: their utilisation is
+    # dense-equivalent TOPS over twice the dense peak
+    path_peak = int8_peak_tops * (2.0 if path == "prefill_sparse" else 1.0)
+    out = {"layer": f"{K}->{O} {n}:{m} T={T}", "ops_per_call": ops, "path": path}
     for name, dt, esz in dtypes:
         y = torch.empty((T, O), dtype=dt, device=dev)
         s = torch.cuda.Stream()
@@ -378,6 +382,7 @@ def _prefill_case(sbl, dev, int8_peak_tops, hbm_peak, K, O, n, m, dtypes, T=3276
         t = statistics.median(ts)
         byts = T * K * 2 + T * K * 2 + O * K / 4 + T * O * esz  # x read, x_q written + read, codes, y
         out[name] = {"us_per_call": t * 1e6, "tops": ops / t / 1e12, "tensor_frac": ops / t / 1e12 / int8_peak_tops,
+                     "tensor_frac_of_path_peak": ops / t / 1e12 / path_peak,
                      "algorithmic_bytes": byts, "hbm_gbs": byts / t / 1e9, "hbm_frac": byts / t / 1e9 / hbm_peak}
         del g, y
     del w, x, ws, flush
@@ -396,7 +401,99 @@ def _prefill_roofline(sbl, dev, int8_peak_tops, hbm_peak):
            "gate_2:4": _prefill_case(sbl, dev, int8_peak_tops, hbm_peak, 896, 4864, 2, 4, (bf16,)),
            "down_3:4": _prefill_case(sbl, dev, int8_peak_tops, hbm_peak, 4864, 896, 3, 4, (bf16,)),
            "down_2:4": _prefill_case(sbl, dev, int8_peak_tops, hbm_peak, 4864, 896, 2, 4, (bf16,))}
+    # the pages claim 2x for 2:4 on the sparse tensor cores: time(3:4) / time(2:4) per shape, bf16 output
+    out["time_ratio_3to4_over_2to4"] = {
+        shape: out[f"{shape}_3:4"]["bf16_out"]["us_per_call"] / out[f"{shape}_2:4"]["bf16_out"]["us_per_call"]
+        for shape in ("gate", "down")}
     torch.cuda.nvtx.range_pop()
+    return out
+
+
+def _pool_call_us(sbl, x, w, y, ws, reps=5):
+    """Per-call device time of sbl_linear in steady state: a CUDA graph of
+    back-to-back calls that cycle through copies of the weights and
+    activations whose total exceeds 3x L2, so every call reads cold inputs.
+    Median over ``reps`` replays of the graph, divided by its call count."""
+    l2 = torch.cuda.get_device_properties(x.device).L2_cache_size
+    per = w.packed.numel() + x.numel() * 2
+    pool = max(2, min(64, -(-3 * l2 // per), (4 << 30) // per))
+    calls = max(pool, 16)
+    ws_ = [sbl.PreparedWeights(w.packed.clone(), w.row_scale, w.n, w.m, w.K) for _ in range(pool)]
+    xs = [x.clone() for _ in range(pool)]
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        for i in range(2):
+            sbl.sbl_linear(xs[i], ws_[i], y=y, workspace=ws)
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for i in range(calls):
+            sbl.sbl_linear(xs[i % pool], ws_[i % pool], y=y, workspace=ws)
+    ts = []
+    with torch.cuda.stream(s):
+        g.replay()
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(s)
+            g.replay()
+            b.record(s)
+            b.synchronize()
+            ts.append(a.elapsed_time(b) * 1e3 / calls)
+    del g, ws_, xs
+    return statistics.median(ts)
+
+
+def _configs_sweep(sbl, dev):
+    """Tokens/s of the other workload configurations (fp32 output, seeded
+    synthetic inputs, steady-state per-call times from _pool_call_us).  A
+    stack's time is the sum of its projections' calls; projections of equal
+    shape are timed once and counted for each."""
+    cache, weights, acts = {}, {}, {}
+
+    def call_us(K, O, n, m, T, tag):
+        key = (K, O, n, m, T)
+        if key in cache:
+            return cache[key]
+        if (K, O, n, m) not in weights:
+            W = torch.from_numpy(synthetic.latent_weights(O, K, seed=13, tag=f"cfg-{tag}")).to(dev)
+            weights[(K, O, n, m)] = sbl.sbl_prepare_weights(W, n, m)
+            del W
+        if (T, K) not in acts:
+            xb, _ = synthetic.activations(T, K, seed=13, tag=f"cfg-x-{tag}", outlier_p=0.01 if T >= 4096 else 0.0)
+            acts[(T, K)] = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)
+        w, x = weights[(K, O, n, m)], acts[(T, K)]
+        y = torch.empty((T, O), dtype=torch.float32, device=dev)
+        ws = sbl.workspace_for(T, K, O, n, m, dev)
+        us = _pool_call_us(sbl, x, w, y, ws)
+        cache[key] = (us, sbl.sbl_linear_plan(T, K, O, n, m, ws.numel()))
+        del y, ws
+        return cache[key]
+
+    out = {}
+    us, path = call_us(256, 512, 2, 4, 16, "c1")
+    out["config1_256->512_2:4_T16"] = {"us_per_call": us, "tokens_per_s": 16 / (us * 1e-6), "path": path}
+    for n, m in ((3, 4), (2, 4)):
+        g_us, g_path = call_us(896, 4864, n, m, 32768, "c3-gate")
+        d_us, d_path = call_us(4864, 896, n, m, 32768, "c3-down")
+        t = 2 * g_us + d_us
+        out[f"config3_ffn_{n}:{m}_T32768"] = {"us_per_stack": t, "tokens_per_s": 32768 / (t * 1e-6),
+                                               "paths": {"gate/up": g_path, "down": d_path}}
+    qo_us, qo_path = call_us(2048, 2048, 2, 4, 4096, "c4-qo")
+    gu_us, gu_path = call_us(2048, 7168, 2, 4, 4096, "c4-gu")
+    dn_us, dn_path = call_us(7168, 2048, 2, 4, 4096, "c4-down")
+    t = 2 * qo_us + 2 * gu_us + dn_us
+    out["config4_h2048_2:4_T4096"] = {"us_per_stack": t, "tokens_per_s": 4096 / (t * 1e-6),
+                                      "paths": {"q/o": qo_path, "gate/up": gu_path, "down": dn_path}}
+    sweep = {}
+    for T in (1, 8, 64, 512, 4096):
+        for K, O in ((2048, 7168), (7168, 2048)):
+            for n, m in ((2, 4), (3, 4), (6, 8)):
+                us, path = call_us(K, O, n, m, T, f"c5-{K}-{O}")
+                sweep.setdefault(f"{K}->{O}_{n}:{m}", {})[f"T{T}"] = {
+                    "us_per_call": us, "tokens_per_s": T / (us * 1e-6), "path": path}
+    out["config5_sweep"] = sweep
+    weights.clear()
+    acts.clear()
     return out
 
 
@@ -481,7 +578,10 @@ def run_ours(args, rank, world, dev):
     e2e_s = _max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev)
 
     decode = _decode_roofline(sbl, dev, hbm_peak) if rank == 0 else None
+    if decode is not None:
+        decode["T8"] = _decode_roofline(sbl, dev, hbm_peak, T=8)
     prefill_big = _prefill_roofline(sbl, dev, int8_peak_tops, hbm_peak) if rank == 0 else None
+    configs = _configs_sweep(sbl, dev) if rank == 0 and not args.no_configs else None
     launches_per_step = len(layers) * (1 + 2 + 1)  # prep + (quant + tcgen05 GEMM) + fused decode
     value = _throughput(world, K, total_s)
     out = {
@@ -493,6 +593,7 @@ def run_ours(args, rank, world, dev):
         "roofline": roof,
         "decode_roofline": decode,
         "prefill_roofline": prefill_big,
+        "configs": configs,
         "phases": phases,
         "e2e": {"value": world * TOKENS_PER_STEP * K_e2e / e2e_s, "steps": K_e2e, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
@@ -594,6 +695,7 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration sweep (profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
