@@ -17,12 +17,10 @@
 // share a row tile and their int32 partial tiles are summed in shared memory.
 //
 // Expansion: code word w (weights 0..15 of a 16-weight block) becomes four
-// int8x4 words by one byte permute each, the selector nibbles being the codes
-// themselves: e0 = weights 0,2,4,6; e1 = 1,3,5,7; e2 = 8,10,12,14;
-// e3 = 9,11,13,15.  The MMA sums over k in any order as long as the A and B
-// fragments of one thread agree, so the activations of each 16-element block
-// are stored in that same order (even elements of the first eight, odd ones,
-// even of the last eight, odd ones).  In shared memory token n's blocks sit at
+// int8x4 words with expand_pairs() (one byte permute each: weights 0,2,4,6;
+// 1,3,5,7; 8,10,12,14; 9,11,13,15).  The MMA sums over k in any order as long
+// as the A and B fragments of one thread agree, so the activations of each
+// 16-element block are stored in that same order (quant_block16_pairs).  In shared memory token n's blocks sit at
 // n * S, S = K bytes padded to 64 mod 128 so that the two tokens of a
 // quarter-warp read disjoint banks, and within a chunk the block of thread t's
 // i-th word sits at 4 i + t, so the four threads of a group read 64
@@ -40,22 +38,12 @@ constexpr int kDmWarps = kDmThreads / 32;
 constexpr int kDmBatch = 4;                       // chunks of one warp loaded together
 constexpr int kDmMinBlocks = 1;                   // blocks per SM the register budget allows
 constexpr int kDmMaxTokens = 16;                  // tokens of one pass (two n8 tiles)
-constexpr uint32_t kTernaryBytes = 0x00FF0100u;   // byte c = int8 value of 2-bit code c (0, +1, -1)
 
 // Shared-memory stride of one token's activations (K % 64 == 0).
 __host__ __device__ inline int dm_stride(int K) { return (K % 128 == 64) ? K : K + 64; }
 
 __host__ __device__ inline size_t dm_smem_bytes(int K, int TP, int NT) {
     return static_cast<size_t>(TP) * dm_stride(K) + static_cast<size_t>(kDmWarps) * 32 * 4 * NT * 4;
-}
-
-__device__ __forceinline__ void expand_pairs(uint32_t w, uint32_t (&e)[4]) {
-    const uint32_t lo = w & 0x33333333u;           // codes of the even weights, one per nibble
-    const uint32_t hi = (w >> 2) & 0x33333333u;    // codes of the odd weights
-    e[0] = prmt(kTernaryBytes, 0u, lo);
-    e[1] = prmt(kTernaryBytes, 0u, hi);
-    e[2] = prmt(kTernaryBytes, 0u, lo >> 16);
-    e[3] = prmt(kTernaryBytes, 0u, hi >> 16);
 }
 
 __device__ __forceinline__ void mma_s8_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -65,14 +53,6 @@ __device__ __forceinline__ void mma_s8_16832(int (&d)[4], uint32_t a0, uint32_t 
         "{%0,%1,%2,%3};"
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// Quantise 16 consecutive activations into the expansion order above.
-__device__ __forceinline__ uint4 quant_block16_pairs(const uint4& u0, const uint4& u1, float s) {
-    uint32_t q[16];
-    quant_codes16(u0, u1, s, q);
-    return make_uint4(pack_codes(q[0], q[2], q[4], q[6]), pack_codes(q[1], q[3], q[5], q[7]),
-                      pack_codes(q[8], q[10], q[12], q[14]), pack_codes(q[9], q[11], q[13], q[15]));
 }
 
 template <int CW>

@@ -26,8 +26,8 @@
 // resource: per k-block the MMA reads the activation and weight tiles, TMA
 // writes the activation and code tiles and the expansion writes the int8
 // weight tile (about 112 KB per 128 x 256 x 128 step at BN = 256).
-// The weights are expanded in the interleaved 16-element order of
-// expand_codes(); the activations were quantised into the same order.
+// The weights are expanded in the 16-element pairing order of
+// expand_pairs(); the activations were quantised into the same order.
 //
 // Every wait is bounded (mbar_wait); a CTA that gives up raises the timeout
 // status, lets in-flight TMA loads and MMAs finish (bounded), frees its tensor
@@ -375,7 +375,7 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     uint32_t e[4];
-                    expand_codes(words[c], e);
+                    expand_pairs(words[c], e);
                     const uint32_t a = smem_u32(dst + ((c ^ sw) << 4));
                     asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(e[0]), "r"(e[1]), "r"(e[2]),
                                  "r"(e[3])

@@ -294,7 +294,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     uint32_t e[4];
-                    expand_codes(words[c], e);
+                    expand_pairs(words[c], e);
                     const uint32_t a = smem_u32(dst + ((c ^ sw) << 4));
                     asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(e[0]), "r"(e[1]), "r"(e[2]),
                                  "r"(e[3])

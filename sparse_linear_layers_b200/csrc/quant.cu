@@ -10,22 +10,24 @@
 // registers, so x is read once.  The max of |x| is taken on the bf16 bit
 // patterns (magnitude bits order like the values).  Output layouts:
 //   NATURAL      x_q in column order (the public sbl_quant_act);
-//   INTERLEAVED  each 16-element block stored as byte 4j + b <- element 4b + j,
-//                the order in which the tensor-core kernel expands weight codes
-//                (read by TMA).
+//   PAIRS        each 16-element block stored as its even elements 0..6, odd
+//                elements 1..7, even 8..14, odd 9..15: the order in which the
+//                tensor-core kernels expand weight codes (expand_pairs; read
+//                by TMA).
 // The kernel signals programmatic dependents at entry: the contraction kernel
 // that follows may start its own prologue while this one runs.
 #include "sbl_common.cuh"
 
 namespace sbl {
 
-enum QuantLayout { kNatural = 0, kInterleaved = 1 };
+enum QuantLayout { kNatural = 0, kPairs = 1 };
 
 template <int LAYOUT>
 __device__ __forceinline__ void quant_block_store(const uint4& u0, const uint4& u1, float s, int8_t* out_row, int b,
                                                   long long K) {
     (void)K;
-    *reinterpret_cast<uint4*>(out_row + 16 * static_cast<long long>(b)) = quant_block16<LAYOUT != kNatural>(u0, u1, s);
+    *reinterpret_cast<uint4*>(out_row + 16 * static_cast<long long>(b)) =
+        LAYOUT == kNatural ? quant_block16<false>(u0, u1, s) : quant_block16_pairs(u0, u1, s);
 }
 
 // Zero `n16` 16-byte words at p, spread over the whole grid.
@@ -168,7 +170,7 @@ cudaError_t launch_quant(const uint16_t* x, long long T, long long K, int8_t* xq
     uint4* zero_words = static_cast<uint4*>(zero16);
     const long long nzero = nzero16;
     switch (layout) {
-        case kInterleaved: return launch_layout<kInterleaved>(x, T, K, xq, s_tok, zero_words, nzero, status, stream);
+        case kPairs: return launch_layout<kPairs>(x, T, K, xq, s_tok, zero_words, nzero, status, stream);
         default: return launch_layout<kNatural>(x, T, K, xq, s_tok, zero_words, nzero, status, stream);
     }
 }

@@ -13,7 +13,7 @@ cudaError_t launch_prep(const float* W, long long O, long long K, int n, int m, 
                         uint8_t* mask_bits, unsigned* status, cudaStream_t stream);
 cudaError_t launch_quant(const uint16_t* x, long long T, long long K, int8_t* xq, float* s_tok, int layout,
                          unsigned* status, cudaStream_t stream, void* zero16 = nullptr, long long nzero16 = 0);
-constexpr int kLayoutNatural = 0, kLayoutInterleaved = 1;
+constexpr int kLayoutNatural = 0, kLayoutPairs = 1;
 cudaError_t launch_decode(const uint8_t* packed, const float* row_scale, long long O, long long K,
                           const uint16_t* x, long long T, void* y, int y_bf16, int32_t* acc_out, unsigned* status,
                           int num_sms, cudaStream_t stream);
@@ -232,7 +232,7 @@ sbl_status sbl_linear_path(const uint16_t* x_bf16, int64_t T, int64_t K, const u
                 nzero16 = static_cast<long long>(sb / 16);
             }
         }
-        e = sbl::launch_quant(x_bf16, T, K, xq, s_tok, sbl::kLayoutInterleaved, d->status, st, part, nzero16);
+        e = sbl::launch_quant(x_bf16, T, K, xq, s_tok, sbl::kLayoutPairs, d->status, st, part, nzero16);
         if (e != cudaSuccess) return SBL_ERR_CUDA;
         const int variant = path == SBL_PATH_PREFILL_1CTA ? sbl::kPrefillOneCta
                             : path == SBL_PATH_PREFILL_PAIR ? sbl::kPrefillPair

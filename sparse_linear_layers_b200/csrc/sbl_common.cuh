@@ -152,6 +152,23 @@ __device__ __forceinline__ void expand_codes(uint32_t w, uint32_t (&out)[4]) {
     }
 }
 
+// Expand one 32-bit code word into four int8x4 words, pairing order: word 0
+// holds weights 0, 2, 4, 6, word 1 weights 1, 3, 5, 7, word 2 weights 8, 10,
+// 12, 14 and word 3 weights 9, 11, 13, 15 (byte b = the b-th of each list).
+// Each is one byte permute whose selector nibbles are the 2-bit codes
+// themselves, from a table whose bytes 0, 1, 2 are the values 0, +1, -1 of
+// codes 00, 01, 10.  Activations are stored in the same order
+// (quant_block16_pairs) so dot products need no further shuffling.
+constexpr uint32_t kTernaryBytes = 0x00FF0100u;
+__device__ __forceinline__ void expand_pairs(uint32_t w, uint32_t (&e)[4]) {
+    const uint32_t lo = w & 0x33333333u;           // codes of the even weights, one per nibble
+    const uint32_t hi = (w >> 2) & 0x33333333u;    // codes of the odd weights
+    e[0] = prmt(kTernaryBytes, 0u, lo);
+    e[1] = prmt(kTernaryBytes, 0u, hi);
+    e[2] = prmt(kTernaryBytes, 0u, lo >> 16);
+    e[3] = prmt(kTernaryBytes, 0u, hi >> 16);
+}
+
 // ---------------------------------------------------------------- activation quantisation
 // round_half_even(x * s) for an activation x (as float) and its token's
 // s = 127 / max|x|, returned as the bit pattern of x * s + 1.5 * 2^23.  The
@@ -207,6 +224,14 @@ __device__ __forceinline__ uint4 quant_block16(const uint4& u0, const uint4& u1,
             o[j] = pack_codes(q[4 * j], q[4 * j + 1], q[4 * j + 2], q[4 * j + 3]);
     }
     return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// Quantise 16 consecutive activations into the pairing order of expand_pairs().
+__device__ __forceinline__ uint4 quant_block16_pairs(const uint4& u0, const uint4& u1, float s) {
+    uint32_t q[16];
+    quant_codes16(u0, u1, s, q);
+    return make_uint4(pack_codes(q[0], q[2], q[4], q[6]), pack_codes(q[1], q[3], q[5], q[7]),
+                      pack_codes(q[8], q[10], q[12], q[14]), pack_codes(q[9], q[11], q[13], q[15]));
 }
 
 }  // namespace sbl
