@@ -5,5 +5,5 @@ baseline leg; never by the library itself.
 """
 from .sbl_oracle import *  # noqa: F401,F403
 from .sbl_oracle import (SUPPORTED_NM, acc_entries, dequant, int_contract, linear, nm_mask,  # noqa: F401
-                         pack_codes, pack_mask_bits, prepare_weights, quant_act, row_scale,
-                         ternarise, unpack_codes)
+                         pack_codes, pack_mask_bits, prepare_weights, quant_act, rms_sumsq, rmsnorm,
+                         rmsnorm_quant_act, row_scale, ternarise, unpack_codes)

@@ -14,6 +14,8 @@ the 2-bit code table of its "What ships with this repo / Packed vs raw"):
     W_t       clip(round(W / scale), -1, 1) on kept positions, 0 elsewhere
     packed    2 bits per weight, 00 = 0, 01 = +1, 10 = -1, 4 codes per byte
     x_q       clip(round(x * 127 / max|x|), -128, 127) per token
+    (RMSNorm) x <- x / sqrt(mean(x^2) + eps) * g before x_q, as the guide's
+              module does (optional, the fused RMSNorm entry points)
     acc       x_q . W_t^T in integers
     y         acc * scale_i / s_t,  s_t = 127 / max|x_t|
 
@@ -32,7 +34,14 @@ with its reason in the design notes):
   computes in the activation's float type); x is bf16 widened exactly;
 * 2-bit codes are stored LSB-first: weight k sits in byte k // 4 at bits
   2 (k % 4) .. 2 (k % 4) + 1; mask bits: bit k % 8 of byte k // 8;
-* dequantisation in double: y = acc * scale / s_t.
+* dequantisation in double: y = acc * scale / s_t;
+* RMSNorm (the guide's module normalises x with torch's RMSNorm before the
+  absmax; the pages give no arithmetic order): float32 throughout, every step
+  an IEEE-rounded operation; the sum of squares in a fixed order (lane l of
+  32 sums, in increasing k, the squares of the 16-element blocks b with
+  b % 32 == l; the 32 lane sums are combined by an xor butterfly at offsets
+  16, 8, 4, 2, 1); mean = sum / K; inv = 1 / sqrt(mean + eps);
+  x_norm = (x * inv) * g.
 
 Every function here is pinned by tests that do not call it to build their
 expected values (worked examples from the pages, closed forms, brute force).
@@ -155,6 +164,63 @@ def quant_act(x: np.ndarray):
     return np.clip(q, -128, 127).astype(np.int8), s
 
 
+RMS_LANES = 32
+RMS_BLOCK = 16
+
+
+def rms_sumsq(x: np.ndarray) -> np.ndarray:
+    """float32 [T]: the sum of x_k^2 over each token in the fixed float32 order.
+
+    Lane l (0..31) adds, in increasing k, the squares of the elements of the
+    16-element blocks b with b % 32 == l, one float32 rounding per addition
+    (a bf16 value's square is exact in float32 unless it underflows, where it
+    is rounded like any float32 product); the 32 lane sums are then combined
+    by an xor butterfly at offsets 16, 8, 4, 2, 1 (lane 0's value is taken).
+    """
+    x = np.asarray(x, dtype=np.float32)
+    T, K = x.shape
+    if K % RMS_BLOCK:
+        raise ValueError("K must be a multiple of 16")
+    part = np.zeros((T, RMS_LANES), np.float32)
+    for k in range(K):
+        lane = (k // RMS_BLOCK) % RMS_LANES
+        v = x[:, k]
+        part[:, lane] = (part[:, lane] + (v * v).astype(np.float32)).astype(np.float32)
+    idx = np.arange(RMS_LANES)
+    for off in (16, 8, 4, 2, 1):
+        part = (part + part[:, idx ^ off]).astype(np.float32)
+    return part[:, 0].copy()
+
+
+def rmsnorm(x: np.ndarray, g: np.ndarray, eps: float) -> np.ndarray:
+    """float32 [T, K]: x * (1 / sqrt(sum_k x_k^2 / K + eps)) * g.
+
+    Sparse-BitNet Guide, "Mathematical Formulation of Sparse-BitLinear" (x is
+    normalised by RMSNorm before the absmax) and its SparseBitLinear module
+    listing (torch RMSNorm over the input features, elementwise weight g,
+    default eps = float32 machine epsilon).  Every step is one IEEE float32
+    operation: the sum of squares of :func:`rms_sumsq`, a division by K, an
+    addition of eps, a square root, a division of 1 by it, and two products.
+    """
+    x = np.asarray(x, dtype=np.float32)
+    g = np.asarray(g, dtype=np.float32)
+    if not (np.all(np.isfinite(x)) and np.all(np.isfinite(g))):
+        raise ValueError("non-finite input")
+    T, K = x.shape
+    if g.shape != (K,):
+        raise ValueError("g must have K entries")
+    ms = (rms_sumsq(x) / np.float32(K)).astype(np.float32)
+    den = np.sqrt((ms + np.float32(eps)).astype(np.float32)).astype(np.float32)
+    inv = (np.float32(1.0) / den).astype(np.float32)
+    return ((x * inv[:, None]).astype(np.float32) * g[None, :]).astype(np.float32)
+
+
+def rmsnorm_quant_act(x: np.ndarray, g: np.ndarray, eps: float):
+    """(x_q int8 [T,K], s_tok fp32 [T]) of the RMS-normalised activations: the
+    guide module's normalise-then-absmax-quantise front end."""
+    return quant_act(rmsnorm(x, g, eps))
+
+
 def int_contract(xq: np.ndarray, Wt: np.ndarray) -> np.ndarray:
     """int32 [T, O] = x_q . W_t^T (the guide's integer product before rescaling).
 
@@ -177,9 +243,11 @@ def dequant(acc: np.ndarray, scale: np.ndarray, s_tok: np.ndarray) -> np.ndarray
             / np.asarray(s_tok, np.float64)[:, None])
 
 
-def linear(x: np.ndarray, Wt: np.ndarray, scale: np.ndarray):
-    """Full forward on prepared weights: (y float64 [T,O], acc int32 [T,O], x_q, s_tok)."""
-    xq, s = quant_act(x)
+def linear(x: np.ndarray, Wt: np.ndarray, scale: np.ndarray, g=None, eps=None):
+    """Full forward on prepared weights: (y float64 [T,O], acc int32 [T,O], x_q, s_tok).
+
+    With ``g`` (and ``eps``) the activations are RMS-normalised first."""
+    xq, s = quant_act(x) if g is None else rmsnorm_quant_act(x, g, eps)
     acc = int_contract(xq, Wt)
     return dequant(acc, scale, s), acc, xq, s
 

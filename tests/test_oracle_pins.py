@@ -8,7 +8,10 @@
   of clip(round(w/scale)), bit-string packing, explicit integer loops;
 * invariants that hold at any size (codes in {-1,0,1}, at most N nonzeros per
   group, sign agreement, packed size O*K/4, argmax token element -> +-127);
-* the guide's own rescale form y = acc * beta * gamma / 127.
+* the guide's own rescale form y = acc * beta * gamma / 127;
+* RMSNorm front end: torch's rms_norm in float64 (the library routine the
+  guide's module calls), hand-derived float32 sums that fix the summation
+  order, constant rows, and invariance under x -> 4x.
 
 Each plausible mistake (a reversed input index, scale over all weights, half away
 from zero, ties to the higher index, MSB-first packing, a dropped clamp, a sign
@@ -374,6 +377,162 @@ def test_planted_mistake_is_caught(name):
                 pin(o, shapes=((8, 16), (4, 32)), T=2, seeds=(0,))
             else:
                 pin(o)
+        except (AssertionError, ValueError, IndexError):
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught the planted mistake {name}"
+
+
+# --------------------------------------------------------------------------
+# RMSNorm front end (the guide's module normalises x before the absmax)
+# --------------------------------------------------------------------------
+
+def pin_rms_library(o):
+    """torch's own rms_norm in float64 (the guide's module uses torch RMSNorm):
+    the float32 oracle agrees within a few float32 roundings; eps = 0.5 and a
+    random weight make the placement of eps and of g visible."""
+    import torch
+    rng = np.random.default_rng(7)
+    for K in (64, 256):
+        x = synthetic.activations(5, K, seed=3)[1]
+        g = rng.uniform(0.5, 1.5, K).astype(np.float32)
+        for eps in (0.5, 2.0 ** -23):
+            ref = torch.nn.functional.rms_norm(torch.from_numpy(x.astype(np.float64)), (K,),
+                                               weight=torch.from_numpy(g.astype(np.float64)), eps=eps).numpy()
+            got = o.rmsnorm(x, g, eps).astype(np.float64)
+            assert np.all(np.abs(got - ref) <= 2e-5 * np.abs(ref) + 1e-30)
+
+
+def pin_rms_order(o):
+    """The float32 order of the sum of squares, from hand-derived values.
+
+    K = 16, x = [4096, 1 x 15]: one lane adds 2^24 then fifteen 1s; each sum
+    2^24 + 1 is a tie between 2^24 and 2^24 + 2 and rounds to even, 2^24.
+    K = 512, x_0 = 4096 and the first element of blocks 1..31 = 1: lane l holds
+    block l; the butterfly at 16, 8, 4, 2, 1 gives lane 0 2^24 (2^24 + 1 ties
+    to even), then 2^24 + 2, + 4, + 8, + 16: 16777246 (the exact sum is
+    16777247, a sequential sum 16777216).
+    K = 512, x_0 = 4096, first elements of blocks 16 and 24 = 1: offset 16
+    first adds one 1 to 2^24 (a tie: 2^24), and the other reaches lane 0 alone
+    at offset 8 (2^24 again): 16777216; the butterfly taken from offset 1 up
+    would pair the two 1s first and give 16777218."""
+    x = np.zeros((1, 16), np.float32)
+    x[0, 0] = 4096.0
+    x[0, 1:] = 1.0
+    assert float(o.rms_sumsq(x)[0]) == 16777216.0
+    x = np.zeros((1, 512), np.float32)
+    x[0, 0] = 4096.0
+    x[0, 16::16] = 1.0
+    assert float(o.rms_sumsq(x)[0]) == 16777246.0
+    x = np.zeros((1, 512), np.float32)
+    x[0, 0] = 4096.0
+    x[0, 16 * 16] = 1.0
+    x[0, 24 * 16] = 1.0
+    assert float(o.rms_sumsq(x)[0]) == 16777216.0
+
+
+def pin_rms_closed_forms(o):
+    """Constant rows normalise to +-1 (fl(1/3) * 3 rounds to 1 in float32), so
+    every code is +-127 with s = 127; with eps = 0 the front end is invariant
+    under x -> 4x (powers of two scale every step exactly); the largest |x g|
+    of a token maps to +-127."""
+    K = 32
+    x = np.full((2, K), 3.0, np.float32)
+    x[1, 1::2] = -3.0
+    xq, s = o.rmsnorm_quant_act(x, np.ones(K, np.float32), 0.0)
+    assert xq[0].tolist() == [127] * K and s[0] == np.float32(127.0)
+    assert xq[1].tolist() == [127, -127] * (K // 2)
+    xb, xv = synthetic.activations(6, 128, seed=4)
+    g = np.random.default_rng(2).uniform(0.25, 2.0, 128).astype(np.float32)
+    q1, s1 = o.rmsnorm_quant_act(xv, g, 0.0)
+    q4, s4 = o.rmsnorm_quant_act(xv * np.float32(4.0), g, 0.0)
+    assert np.array_equal(q1, q4) and np.array_equal(s1, s4)
+    q, _ = o.rmsnorm_quant_act(xv, g, 2.0 ** -23)
+    am = np.argmax(np.abs(xv.astype(np.float64) * g), axis=1)
+    assert np.all(np.abs(q[np.arange(6), am]) == 127)
+
+
+def test_rms_pins():
+    for pin in (pin_rms_library, pin_rms_order, pin_rms_closed_forms):
+        pin(oracle)
+
+
+def _rms_ns(**over):
+    ns = types.SimpleNamespace(rms_sumsq=oracle.rms_sumsq, quant_act=oracle.quant_act)
+    ns.__dict__.update(over)
+
+    def rmsnorm(x, g, eps):
+        x = np.asarray(x, np.float32)
+        K = x.shape[1]
+        ms = (ns.rms_sumsq(x) / np.float32(K)).astype(np.float32)
+        inv = (np.float32(1.0) / np.sqrt((ms + np.float32(eps)).astype(np.float32))).astype(np.float32)
+        return ((x * inv[:, None]).astype(np.float32) * np.asarray(g, np.float32)[None, :]).astype(np.float32)
+
+    if "rmsnorm" not in over:
+        ns.rmsnorm = rmsnorm
+    ns.rmsnorm_quant_act = lambda x, g, eps: ns.quant_act(ns.rmsnorm(x, g, eps))
+    return ns
+
+
+def _rms_seq(x):
+    x = np.asarray(x, np.float32)
+    acc = np.zeros(x.shape[0], np.float32)
+    for k in range(x.shape[1]):
+        acc = (acc + (x[:, k] * x[:, k]).astype(np.float32)).astype(np.float32)
+    return acc
+
+
+def _rms_butterfly_up(x):
+    x = np.asarray(x, np.float32)
+    part = np.zeros((x.shape[0], 32), np.float32)
+    for k in range(x.shape[1]):
+        lane = (k // 16) % 32
+        part[:, lane] = (part[:, lane] + (x[:, k] * x[:, k]).astype(np.float32)).astype(np.float32)
+    idx = np.arange(32)
+    for off in (1, 2, 4, 8, 16):
+        part = (part + part[:, idx ^ off]).astype(np.float32)
+    return part[:, 0].copy()
+
+
+def _rms_no_sqrt(x, g, eps):
+    x = np.asarray(x, np.float32)
+    ms = (oracle.rms_sumsq(x) / np.float32(x.shape[1])).astype(np.float32)
+    return (x / (ms + np.float32(eps))[:, None] * np.asarray(g, np.float32)[None, :]).astype(np.float32)
+
+
+def _rms_eps_outside(x, g, eps):
+    x = np.asarray(x, np.float32)
+    ms = (oracle.rms_sumsq(x) / np.float32(x.shape[1])).astype(np.float32)
+    return (x / (np.sqrt(ms) + np.float32(eps))[:, None] * np.asarray(g, np.float32)[None, :]).astype(np.float32)
+
+
+def _rms_no_weight(x, g, eps):
+    return oracle.rmsnorm(x, np.ones_like(np.asarray(g, np.float32)), eps)
+
+
+def _rms_mean_k_minus_1(x, g, eps):
+    x = np.asarray(x, np.float32)
+    ms = (oracle.rms_sumsq(x) / np.float32(x.shape[1] - 1)).astype(np.float32)
+    inv = (np.float32(1.0) / np.sqrt((ms + np.float32(eps)).astype(np.float32))).astype(np.float32)
+    return ((x * inv[:, None]).astype(np.float32) * np.asarray(g, np.float32)[None, :]).astype(np.float32)
+
+
+RMS_MUTANTS = {
+    "rms_sequential_sum": dict(rms_sumsq=_rms_seq),
+    "rms_butterfly_from_offset_1": dict(rms_sumsq=_rms_butterfly_up),
+    "rms_no_sqrt": dict(rmsnorm=_rms_no_sqrt),
+    "rms_eps_outside_sqrt": dict(rmsnorm=_rms_eps_outside),
+    "rms_weight_dropped": dict(rmsnorm=_rms_no_weight),
+    "rms_mean_over_k_minus_1": dict(rmsnorm=_rms_mean_k_minus_1),
+}
+
+
+@pytest.mark.parametrize("name", sorted(RMS_MUTANTS))
+def test_planted_rms_mistake_is_caught(name):
+    o = _rms_ns(**RMS_MUTANTS[name])
+    caught = []
+    for pin in (pin_rms_library, pin_rms_order, pin_rms_closed_forms):
+        try:
+            pin(o)
         except (AssertionError, ValueError, IndexError):
             caught.append(pin.__name__)
     assert caught, f"no pin caught the planted mistake {name}"
