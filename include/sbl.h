@@ -105,6 +105,33 @@ sbl_status sbl_quant_act(const uint16_t* x_bf16, int64_t T, int64_t K,
                          int8_t* x_q, float* s_tok, void* stream);
 
 /*
+ * sbl_rmsnorm_quant_act — RMSNorm, then per-token absmax int8 quantisation.
+ *
+ * The activation step of the Sparse-BitNet Guide, "Mathematical Formulation of
+ * Sparse-BitLinear" (activations are normalised by RMSNorm before the absmax),
+ * in the form of the guide's SparseBitLinear module listing (torch RMSNorm
+ * over the K input features with an elementwise weight):
+ *   x_norm = (x * (1 / sqrt(sum_k x_k^2 / K + eps))) * g
+ * in float32, every step IEEE-rounded (the pages give no order; the sum of
+ * squares is formed in a fixed one: lane l of 32 adds, in increasing k, the
+ * squares of the 16-element blocks b with b % 32 == l, and the lane sums are
+ * combined by an xor butterfly at offsets 16, 8, 4, 2, 1), then x_q and s_tok
+ * exactly as sbl_quant_act computes them from x_norm.
+ *
+ *   x_bf16  bf16 bit patterns [T, K] (input), K % 16 == 0 like every entry
+ *           point (else SBL_ERR_INVALID_ARG).
+ *   g       fp32 [K] (input): the RMSNorm weight, 16-byte aligned.
+ *   eps     finite, >= 0 (torch's default for float32 is 2^-23); else
+ *           SBL_ERR_INVALID_ARG.
+ *   x_q     int8 [T, K] (output), natural column order.
+ *   s_tok   fp32 [T] (output): 127 / max(max_k |x_norm|, 1e-5).
+ *   Non-finite x or a non-finite normalised value sets SBL_ERR_NONFINITE in
+ *   the device status word; that token's outputs are then unspecified.
+ */
+sbl_status sbl_rmsnorm_quant_act(const uint16_t* x_bf16, const float* g, float eps, int64_t T, int64_t K,
+                                 int8_t* x_q, float* s_tok, void* stream);
+
+/*
  * sbl_linear_workspace_bytes — bytes of device workspace sbl_linear needs for
  * these sizes: the quantised activations and their scales, in the kernels'
  * internal layout (T*K + 4*T bytes, each rounded up to 256), plus, for 2:4
@@ -134,9 +161,10 @@ size_t sbl_linear_workspace_bytes(int64_t T, int64_t K, int64_t O, int n, int m)
  *              aligned; its contents on entry do not matter and are
  *              overwritten.  Calls that share a workspace must be ordered on
  *              one stream.
- *   Chooses the CUDA-core decode path for T <= sbl_decode_max_tokens() and the
- *   tcgen05 tensor-core prefill path above it (the latter needs K % 64 == 0;
- *   other K always take the decode path).
+ *   Chooses the decode path for T <= sbl_decode_max_tokens() (CUDA-core dp4a
+ *   for one or two tokens, the warp-level int8 MMA for more when K % 64 == 0)
+ *   and the tcgen05 tensor-core prefill path above it (the latter needs
+ *   K % 64 == 0; other K always take the decode path).
  */
 sbl_status sbl_linear(const uint16_t* x_bf16, int64_t T, int64_t K,
                       const uint8_t* packed, const float* row_scale, int64_t O, int n, int m,
@@ -160,6 +188,22 @@ sbl_status sbl_linear_path(const uint16_t* x_bf16, int64_t T, int64_t K,
                            const uint8_t* packed, const float* row_scale, int64_t O, int n, int m,
                            void* y, int y_dtype, int32_t* acc_out,
                            void* workspace, size_t workspace_bytes, int path, void* stream);
+
+/*
+ * sbl_linear_rmsnorm — the whole forward of the Sparse-BitNet Guide's
+ * SparseBitLinear module on prepared weights: RMSNorm of x (as in
+ * sbl_rmsnorm_quant_act, weight g, epsilon eps), per-token absmax int8, the
+ * integer product with the ternary weights and the rescale, y as sbl_linear
+ * returns it.  Arguments and `path` as sbl_linear_path, plus g (fp32 [K],
+ * 16-byte aligned, not NULL) and eps (finite, >= 0).  Needs K % 64 == 0 at
+ * the sizes that take the decode path (there the activations are normalised
+ * and quantised by one kernel and contracted on the warp-level MMA), else
+ * SBL_ERR_UNSUPPORTED.  The workspace is sized by sbl_linear_workspace_bytes().
+ */
+sbl_status sbl_linear_rmsnorm(const uint16_t* x_bf16, const float* g, float eps, int64_t T, int64_t K,
+                              const uint8_t* packed, const float* row_scale, int64_t O, int n, int m,
+                              void* y, int y_dtype, int32_t* acc_out,
+                              void* workspace, size_t workspace_bytes, int path, void* stream);
 
 /*
  * sbl_linear_noalloc — sbl_linear for callers that cannot allocate device memory.

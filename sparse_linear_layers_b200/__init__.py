@@ -2,7 +2,8 @@
 
 y = dequant(int8(x) . ternary_NM(W)^T) behind a C ABI (include/sbl.h) with
 hand-written CUDA kernels: fused weight preparation, per-token activation
-quantisation, a CUDA-core decode path and a tcgen05 tensor-core prefill path.
+quantisation (optionally after RMSNorm, as the guide's module does), decode
+paths on CUDA cores and the warp-level MMA, and tcgen05 tensor-core prefill.
 
 The library entry points (sbl_prepare_weights, sbl_quant_act, sbl_linear, ...)
 load libsbl.so on first use and raise ImportError if it has not been built;
@@ -12,8 +13,8 @@ GPU library.
 __version__ = "0.1.0"
 
 _API = ("PreparedWeights", "sbl_decode_max_tokens", "sbl_device_status", "sbl_linear", "sbl_linear_plan",
-        "sbl_linear_workspace_bytes", "sbl_prepare_weights", "sbl_quant_act", "sbl_selftest_bounded_wait",
-        "workspace_for", "SblError")
+        "sbl_linear_rmsnorm", "sbl_linear_workspace_bytes", "sbl_prepare_weights", "sbl_quant_act",
+        "sbl_rmsnorm_quant_act", "sbl_selftest_bounded_wait", "workspace_for", "RMSNORM_EPS_F32", "SblError")
 
 
 def __getattr__(name):

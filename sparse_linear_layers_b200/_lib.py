@@ -32,12 +32,16 @@ SBL_PATH_PREFILL_SPARSE = 5
 
 # name -> (restype, argtypes); mirrors include/sbl.h
 _vp, _i64, _int, _sz, _u32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint32
+_f32 = ctypes.c_float
 SIGNATURES = {
     "sbl_prepare_weights": (_int, [_vp, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp]),
     "sbl_quant_act": (_int, [_vp, _i64, _i64, _vp, _vp, _vp]),
+    "sbl_rmsnorm_quant_act": (_int, [_vp, _vp, _f32, _i64, _i64, _vp, _vp, _vp]),
     "sbl_linear_workspace_bytes": (_sz, [_i64, _i64, _i64, _int, _int]),
     "sbl_linear": (_int, [_vp, _i64, _i64, _vp, _vp, _i64, _int, _int, _vp, _int, _vp, _vp, _sz, _vp]),
     "sbl_linear_path": (_int, [_vp, _i64, _i64, _vp, _vp, _i64, _int, _int, _vp, _int, _vp, _vp, _sz, _int, _vp]),
+    "sbl_linear_rmsnorm": (_int, [_vp, _vp, _f32, _i64, _i64, _vp, _vp, _i64, _int, _int, _vp, _int, _vp, _vp, _sz,
+                                  _int, _vp]),
     "sbl_linear_noalloc": (_int, [_vp, _i64, _i64, _vp, _vp, _i64, _int, _int, _vp, _int, _vp, _vp]),
     "sbl_linear_plan": (_int, [_i64, _i64, _i64, _int, _int, _sz]),
     "sbl_decode_max_tokens": (_i64, []),

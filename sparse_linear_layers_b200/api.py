@@ -75,6 +75,22 @@ def sbl_quant_act(x: torch.Tensor, stream: Optional[torch.cuda.Stream] = None):
     return xq, s
 
 
+RMSNORM_EPS_F32 = 2.0 ** -23  # torch's default RMSNorm epsilon for float32 (machine epsilon)
+
+
+def sbl_rmsnorm_quant_act(x: torch.Tensor, g: torch.Tensor, eps: float = RMSNORM_EPS_F32,
+                          stream: Optional[torch.cuda.Stream] = None):
+    """RMSNorm (weight g, fp32 [K]) then per-token absmax int8: (x_q int8 [T,K], s_tok fp32 [T])."""
+    _need_cuda(x, "x", torch.bfloat16)
+    _need_cuda(g, "g", torch.float32)
+    T, K = x.shape
+    xq = torch.empty((T, K), dtype=torch.int8, device=x.device)
+    s = torch.empty((T,), dtype=torch.float32, device=x.device)
+    check(lib.sbl_rmsnorm_quant_act(x.data_ptr(), g.data_ptr(), float(eps), T, K, xq.data_ptr(), s.data_ptr(),
+                                    _stream(stream)), "sbl_rmsnorm_quant_act")
+    return xq, s
+
+
 def sbl_linear_workspace_bytes(T: int, K: int, O: int, n: int, m: int) -> int:
     return int(lib.sbl_linear_workspace_bytes(T, K, O, n, m))
 
@@ -108,6 +124,34 @@ def sbl_linear(x: torch.Tensor, w: PreparedWeights, out_dtype: torch.dtype = tor
                               y.data_ptr(), ydt, acc_out.data_ptr() if acc_out is not None else None,
                               workspace.data_ptr(), workspace.numel(), _PATHS[path], _stream(stream)),
           "sbl_linear")
+    return y
+
+
+def sbl_linear_rmsnorm(x: torch.Tensor, w: PreparedWeights, g: torch.Tensor, eps: float = RMSNORM_EPS_F32,
+                       out_dtype: torch.dtype = torch.float32, y: Optional[torch.Tensor] = None,
+                       acc_out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                       path: str = "auto", stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """The guide module's forward: y = dequant(int8(RMSNorm(x; g, eps)) . W_t^T)."""
+    _need_cuda(x, "x", torch.bfloat16)
+    _need_cuda(g, "g", torch.float32)
+    T, K = x.shape
+    if K != w.K or g.numel() != K:
+        raise ValueError(f"x has K={K}; weights were prepared with K={w.K}; g has {g.numel()} entries")
+    O = w.O
+    if y is None:
+        y = torch.empty((T, O), dtype=out_dtype, device=x.device)
+    if y.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("y must be float32 or bfloat16")
+    _need_cuda(y, "y", y.dtype)
+    ydt = _lib.SBL_F32 if y.dtype == torch.float32 else _lib.SBL_BF16
+    if acc_out is not None:
+        _need_cuda(acc_out, "acc_out", torch.int32)
+    if workspace is None:
+        workspace = workspace_for(T, K, O, w.n, w.m, x.device)
+    check(lib.sbl_linear_rmsnorm(x.data_ptr(), g.data_ptr(), float(eps), T, K, w.packed.data_ptr(),
+                                 w.row_scale.data_ptr(), O, w.n, w.m, y.data_ptr(), ydt,
+                                 acc_out.data_ptr() if acc_out is not None else None, workspace.data_ptr(),
+                                 workspace.numel(), _PATHS[path], _stream(stream)), "sbl_linear_rmsnorm")
     return y
 
 

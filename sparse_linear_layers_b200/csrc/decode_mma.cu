@@ -77,10 +77,14 @@ __device__ __forceinline__ void load_words(const uint8_t* p, bool ok, uint32_t (
     }
 }
 
-template <int NT, int CW>
+// PREQ: the activations arrive already quantised (x_q int8 [T, K] with each
+// 16-element block in the pairing order, and s_tok [T], from the RMSNorm
+// front end) and are only copied into shared memory.
+template <int NT, int CW, bool PREQ>
 __global__ void __launch_bounds__(kDmThreads, kDmMinBlocks)
     decode_mma_kernel(const uint8_t* __restrict__ packed, const float* __restrict__ row_scale, int O, int K,
-                      const uint16_t* __restrict__ x, int t0, int TP, int KS, void* __restrict__ y, int y_bf16,
+                      const uint16_t* __restrict__ x, const int8_t* __restrict__ xq_in,
+                      const float* __restrict__ stok_in, int t0, int TP, int KS, void* __restrict__ y, int y_bf16,
                       int32_t* __restrict__ acc_out, unsigned* status) {
     extern __shared__ __align__(16) uint8_t dm_smem[];
     __shared__ uint32_t red_max[kDmWarps];
@@ -119,61 +123,71 @@ __global__ void __launch_bounds__(kDmThreads, kDmMinBlocks)
     const float sc0 = (v0 && ks == 0) ? row_scale[r0] : 0.0f;
     const float sc1 = (v1 && ks == 0) ? row_scale[r1] : 0.0f;
 
-    // Quantise the pass's TP tokens: 16 / TP warps per token, each thread
-    // keeping up to four 16-element blocks in registers between the absmax and
-    // the quantisation (blocks beyond that are read again, four at a time).
     const int nblk = K >> 4;
-    const int wpt = kDmWarps / TP;
-    const int qt = warp / wpt;
-    const bool qw = qt < TP;
-    const int qj = (warp - qt * wpt) * 32 + lane;
-    const int nthr = wpt * 32;
-    const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t0 + (qw ? qt : 0)) * K);
-    constexpr int XB = 4;
-    uint4 xa[XB][2];
-    uint32_t mx = 0;
-    if (qw) {
-#pragma unroll
-        for (int i = 0; i < XB; ++i) {
-            const int b = qj + i * nthr;
-            if (b < nblk) {
-                xa[i][0] = ldg_nc(xr + 2 * b);
-                xa[i][1] = ldg_nc(xr + 2 * b + 1);
-                mx = absmax8(xa[i][1], absmax8(xa[i][0], mx));
+    auto pos = [](int blk) {  // shared-memory slot of 16-element block blk of a token
+        const int c = blk / (4 * CW), l = blk % (4 * CW);
+        return c * 4 * CW + (l % CW) * 4 + l / CW;
+    };
+    if constexpr (PREQ) {
+        for (int u = threadIdx.x; u < TP * nblk; u += kDmThreads) {
+            const int tok = u / nblk, blk = u - tok * nblk;
+            reinterpret_cast<uint4*>(dm_smem + static_cast<size_t>(tok) * S)[pos(blk)] =
+                __ldg(reinterpret_cast<const uint4*>(xq_in + static_cast<size_t>(t0 + tok) * K) + blk);
+        }
+        if (threadIdx.x < TP) s_sh[threadIdx.x] = stok_in[t0 + threadIdx.x];
+        __syncthreads();
+    } else {
+        // Quantise the pass's TP tokens: 16 / TP warps per token, each thread
+        // keeping up to four 16-element blocks in registers between the absmax and
+        // the quantisation (blocks beyond that are read again, four at a time).
+        const int wpt = kDmWarps / TP;
+        const int qt = warp / wpt;
+        const bool qw = qt < TP;
+        const int qj = (warp - qt * wpt) * 32 + lane;
+        const int nthr = wpt * 32;
+        const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t0 + (qw ? qt : 0)) * K);
+        constexpr int XB = 4;
+        uint4 xa[XB][2];
+        uint32_t mx = 0;
+        if (qw) {
+    #pragma unroll
+            for (int i = 0; i < XB; ++i) {
+                const int b = qj + i * nthr;
+                if (b < nblk) {
+                    xa[i][0] = ldg_nc(xr + 2 * b);
+                    xa[i][1] = ldg_nc(xr + 2 * b + 1);
+                    mx = absmax8(xa[i][1], absmax8(xa[i][0], mx));
+                }
             }
+    #pragma unroll 4
+            for (int b = qj + XB * nthr; b < nblk; b += nthr) mx = absmax8(ldg_nc(xr + 2 * b + 1), absmax8(ldg_nc(xr + 2 * b), mx));
         }
-#pragma unroll 4
-        for (int b = qj + XB * nthr; b < nblk; b += nthr) mx = absmax8(ldg_nc(xr + 2 * b + 1), absmax8(ldg_nc(xr + 2 * b), mx));
-    }
-    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
-    if (lane == 0) red_max[warp] = mx;
-    __syncthreads();
-    if (threadIdx.x < TP) {
-        uint32_t m = 0;
-#pragma unroll
-        for (int w = 0; w < kDmWarps; ++w)
-            if (w / wpt == static_cast<int>(threadIdx.x)) m = max(m, red_max[w]);
-        if (m >= 0x7F80u && blockIdx.x == 0) raise_status(status, kStatusNonfinite);
-        s_sh[threadIdx.x] = __fdiv_rn(127.0f, fmaxf(__uint_as_float(m << 16), 1e-5f));
-    }
-    __syncthreads();
-    if (qw) {
-        const float st = s_sh[qt];
-        uint4* xt = reinterpret_cast<uint4*>(dm_smem + static_cast<size_t>(qt) * S);
-        auto pos = [](int blk) {
-            const int c = blk / (4 * CW), l = blk % (4 * CW);
-            return c * 4 * CW + (l % CW) * 4 + l / CW;
-        };
-#pragma unroll
-        for (int i = 0; i < XB; ++i) {
-            const int b = qj + i * nthr;
-            if (b < nblk) xt[pos(b)] = quant_block16_pairs(xa[i][0], xa[i][1], st);
+        mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+        if (lane == 0) red_max[warp] = mx;
+        __syncthreads();
+        if (threadIdx.x < TP) {
+            uint32_t m = 0;
+    #pragma unroll
+            for (int w = 0; w < kDmWarps; ++w)
+                if (w / wpt == static_cast<int>(threadIdx.x)) m = max(m, red_max[w]);
+            if (m >= 0x7F80u && blockIdx.x == 0) raise_status(status, kStatusNonfinite);
+            s_sh[threadIdx.x] = __fdiv_rn(127.0f, fmaxf(__uint_as_float(m << 16), 1e-5f));
         }
-#pragma unroll 4
-        for (int b = qj + XB * nthr; b < nblk; b += nthr)
-            xt[pos(b)] = quant_block16_pairs(ldg_nc(xr + 2 * b), ldg_nc(xr + 2 * b + 1), st);
+        __syncthreads();
+        if (qw) {
+            const float st = s_sh[qt];
+            uint4* xt = reinterpret_cast<uint4*>(dm_smem + static_cast<size_t>(qt) * S);
+    #pragma unroll
+            for (int i = 0; i < XB; ++i) {
+                const int b = qj + i * nthr;
+                if (b < nblk) xt[pos(b)] = quant_block16_pairs(xa[i][0], xa[i][1], st);
+            }
+    #pragma unroll 4
+            for (int b = qj + XB * nthr; b < nblk; b += nthr)
+                xt[pos(b)] = quant_block16_pairs(ldg_nc(xr + 2 * b), ldg_nc(xr + 2 * b + 1), st);
+        }
+        __syncthreads();
     }
-    __syncthreads();
 
     int acc[NT][4];
 #pragma unroll
@@ -275,8 +289,9 @@ static int choose_ks(int R, int C, int nb, int num_sms) {
     return ks;
 }
 
-template <int NT, int CW>
-static cudaError_t launch_dm(const uint8_t* packed, const float* row_scale, int O, int K, const uint16_t* x, int t0,
+template <int NT, int CW, bool PREQ>
+static cudaError_t launch_dm(const uint8_t* packed, const float* row_scale, int O, int K, const uint16_t* x,
+                             const int8_t* xq_in, const float* stok_in, int t0,
                              int TP, int KS, void* y, int y_bf16, int32_t* acc_out, unsigned* status,
                              cudaStream_t stream) {
     const int R = (O + 15) / 16;
@@ -284,7 +299,7 @@ static cudaError_t launch_dm(const uint8_t* packed, const float* row_scale, int 
     const int blocks = (R + tiles_per_block - 1) / tiles_per_block;
     const size_t smem = dm_smem_bytes(K, TP, NT);
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<NT, CW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<NT, CW, PREQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return e;
     }
@@ -298,26 +313,33 @@ static cudaError_t launch_dm(const uint8_t* packed, const float* row_scale, int 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_mma_kernel<NT, CW>, packed, row_scale, O, K, x, t0, TP, KS, y, y_bf16,
+    return cudaLaunchKernelEx(&cfg, decode_mma_kernel<NT, CW, PREQ>, packed, row_scale, O, K, x, xq_in, stok_in, t0, TP, KS, y, y_bf16,
                               acc_out, status);
 }
 
-template <int NT>
+template <int NT, bool PREQ>
 static cudaError_t launch_dm_cw(int CW, const uint8_t* packed, const float* row_scale, int O, int K,
-                                const uint16_t* x, int t0, int TP, int KS, void* y, int y_bf16, int32_t* acc_out,
-                                unsigned* status, cudaStream_t stream) {
-    if (CW == 4) return launch_dm<NT, 4>(packed, row_scale, O, K, x, t0, TP, KS, y, y_bf16, acc_out, status, stream);
-    if (CW == 2) return launch_dm<NT, 2>(packed, row_scale, O, K, x, t0, TP, KS, y, y_bf16, acc_out, status, stream);
-    return launch_dm<NT, 1>(packed, row_scale, O, K, x, t0, TP, KS, y, y_bf16, acc_out, status, stream);
+                                const uint16_t* x, const int8_t* xq_in, const float* stok_in, int t0, int TP, int KS,
+                                void* y, int y_bf16, int32_t* acc_out, unsigned* status, cudaStream_t stream) {
+    if (CW == 4)
+        return launch_dm<NT, 4, PREQ>(packed, row_scale, O, K, x, xq_in, stok_in, t0, TP, KS, y, y_bf16, acc_out,
+                                      status, stream);
+    if (CW == 2)
+        return launch_dm<NT, 2, PREQ>(packed, row_scale, O, K, x, xq_in, stok_in, t0, TP, KS, y, y_bf16, acc_out,
+                                      status, stream);
+    return launch_dm<NT, 1, PREQ>(packed, row_scale, O, K, x, xq_in, stok_in, t0, TP, KS, y, y_bf16, acc_out, status,
+                                  stream);
 }
 
 bool decode_mma_supported(long long K) { return K % 64 == 0 && K > 0 && dm_smem_bytes(static_cast<int>(K), 1, 2) <= 200 * 1024; }
 
 // Passes of up to 16 tokens (as many as fit 200 KB of shared memory); later
-// passes read the weights again, mostly from L2.  Needs K % 64 == 0.
+// passes read the weights again, mostly from L2.  Needs K % 64 == 0.  With
+// xq_in (and stok_in) the activations come already quantised (pairing order)
+// and x is not read.
 cudaError_t launch_decode_mma(const uint8_t* packed, const float* row_scale, long long O, long long K,
                               const uint16_t* x, long long T, void* y, int y_bf16, int32_t* acc_out, unsigned* status,
-                              int num_sms, cudaStream_t stream) {
+                              int num_sms, cudaStream_t stream, const int8_t* xq_in, const float* stok_in) {
     const int Ki = static_cast<int>(K), Oi = static_cast<int>(O);
     const int CW = (Ki % 256 == 0) ? 4 : (Ki % 128 == 0) ? 2 : 1;
     const int C = Ki / (64 * CW);
@@ -327,9 +349,17 @@ cudaError_t launch_decode_mma(const uint8_t* packed, const float* row_scale, lon
     while (cap > 1 && dm_smem_bytes(Ki, cap, cap > 8 ? 2 : 1) > 200 * 1024) --cap;
     for (long long t0 = 0; t0 < T; t0 += cap) {
         const int TP = static_cast<int>(T - t0 < cap ? T - t0 : cap);
-        cudaError_t e = TP > 8 ? launch_dm_cw<2>(CW, packed, row_scale, Oi, Ki, x, static_cast<int>(t0), TP, KS, y,
+        const int t0i = static_cast<int>(t0);
+        cudaError_t e;
+        if (xq_in)
+            e = TP > 8 ? launch_dm_cw<2, true>(CW, packed, row_scale, Oi, Ki, x, xq_in, stok_in, t0i, TP, KS, y, y_bf16,
+                                               acc_out, status, stream)
+                       : launch_dm_cw<1, true>(CW, packed, row_scale, Oi, Ki, x, xq_in, stok_in, t0i, TP, KS, y, y_bf16,
+                                               acc_out, status, stream);
+        else
+            e = TP > 8 ? launch_dm_cw<2, false>(CW, packed, row_scale, Oi, Ki, x, nullptr, nullptr, t0i, TP, KS, y,
                                                 y_bf16, acc_out, status, stream)
-                               : launch_dm_cw<1>(CW, packed, row_scale, Oi, Ki, x, static_cast<int>(t0), TP, KS, y,
+                       : launch_dm_cw<1, false>(CW, packed, row_scale, Oi, Ki, x, nullptr, nullptr, t0i, TP, KS, y,
                                                 y_bf16, acc_out, status, stream);
         if (e != cudaSuccess) return e;
     }

@@ -175,4 +175,134 @@ cudaError_t launch_quant(const uint16_t* x, long long T, long long K, int8_t* xq
     }
 }
 
+// ---------------------------------------------------------------- RMSNorm front end
+// The guide's SparseBitLinear module normalises x with RMSNorm before the
+// per-token absmax ("Mathematical Formulation of Sparse-BitLinear", activation
+// step, and the module listing): x_norm = x * (1 / sqrt(mean(x^2) + eps)) * g,
+// every step an IEEE float32 operation, then the absmax quantisation above.
+// One warp per token; lane l owns the 16-element blocks b with b % 32 == l.
+// The sum of squares follows a fixed order: each lane adds its squares in
+// increasing k, then an xor butterfly at offsets 16, 8, 4, 2, 1 combines the
+// lanes (every lane ends with the same total).  A lane keeps up to RB blocks
+// in registers across the three passes (sum of squares, absmax of the
+// normalised values, quantisation); blocks beyond that are read again.
+template <int LAYOUT>
+__global__ void __launch_bounds__(256) rmsnorm_quant_kernel(const uint16_t* __restrict__ x,
+                                                            const float* __restrict__ g, float eps, long long T,
+                                                            long long K, int8_t* __restrict__ xq,
+                                                            float* __restrict__ s_tok, uint4* __restrict__ zero_words,
+                                                            long long nzero, unsigned* status) {
+    asm volatile("griddepcontrol.launch_dependents;");
+    zero_fill(zero_words, nzero);
+    constexpr int RB = 4;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long t = static_cast<long long>(blockIdx.x) * 8 + warp;
+    if (t >= T) return;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + t * K);
+    const int nblk = static_cast<int>(K >> 4);
+    uint4 v[RB][2];
+    // pass 1: sum of squares in the lane's k order; non-finite inputs flagged
+    float ss = 0.f;
+    uint32_t bad = 0;
+    auto add_sq = [&](const uint4& a, const uint4& b) {
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xFFFF0000u);
+            ss = __fadd_rn(ss, __fmul_rn(lo, lo));
+            ss = __fadd_rn(ss, __fmul_rn(hi, hi));
+            bad |= ((w[i] & 0x7F80u) == 0x7F80u) | ((w[i] & 0x7F800000u) == 0x7F800000u);
+        }
+    };
+#pragma unroll
+    for (int j = 0; j < RB; ++j) {
+        const int b = lane + 32 * j;
+        if (b < nblk) {
+            v[j][0] = ldg_nc(xr + 2 * b);
+            v[j][1] = ldg_nc(xr + 2 * b + 1);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < RB; ++j)
+        if (lane + 32 * j < nblk) add_sq(v[j][0], v[j][1]);
+    for (int b = lane + 32 * RB; b < nblk; b += 32) add_sq(ldg_nc(xr + 2 * b), ldg_nc(xr + 2 * b + 1));
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xFFFFFFFFu, ss, off));
+    const float ms = __fdiv_rn(ss, static_cast<float>(K));
+    const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+
+    // normalised values of one block: (x * inv) * g
+    auto norm16 = [&](const uint4& a, const uint4& b, int blk, float (&n)[16]) {
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        const float4* g4 = reinterpret_cast<const float4*>(g + 16 * blk);
+        float gv[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float4 q = __ldg(g4 + i);
+            gv[4 * i] = q.x;
+            gv[4 * i + 1] = q.y;
+            gv[4 * i + 2] = q.z;
+            gv[4 * i + 3] = q.w;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            n[2 * i] = __fmul_rn(__fmul_rn(__uint_as_float(w[i] << 16), inv), gv[2 * i]);
+            n[2 * i + 1] = __fmul_rn(__fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), inv), gv[2 * i + 1]);
+        }
+    };
+    // pass 2: absmax of the normalised values (bit patterns of |n| order like the values)
+    uint32_t mx = 0;
+    auto max16 = [&](const uint4& a, const uint4& b, int blk) {
+        float n[16];
+        norm16(a, b, blk, n);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) mx = max(mx, __float_as_uint(n[i]) & 0x7FFFFFFFu);
+    };
+#pragma unroll
+    for (int j = 0; j < RB; ++j)
+        if (lane + 32 * j < nblk) max16(v[j][0], v[j][1], lane + 32 * j);
+    for (int b = lane + 32 * RB; b < nblk; b += 32) max16(ldg_nc(xr + 2 * b), ldg_nc(xr + 2 * b + 1), b);
+    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+    bad = __reduce_or_sync(0xFFFFFFFFu, bad);
+    if (lane == 0 && (bad || mx >= 0x7F800000u)) raise_status(status, kStatusNonfinite);
+    const float s = __fdiv_rn(127.0f, fmaxf(__uint_as_float(mx), 1e-5f));
+    if (lane == 0) s_tok[t] = s;
+
+    // pass 3: quantise and store in the requested layout
+    int8_t* out = xq + t * K;
+    auto store16 = [&](const uint4& a, const uint4& b, int blk) {
+        float n[16];
+        norm16(a, b, blk, n);
+        uint32_t q[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) q[i] = quant_code_bits(n[i], s);
+        uint4 o;
+        if (LAYOUT == kNatural)
+            o = make_uint4(pack_codes(q[0], q[1], q[2], q[3]), pack_codes(q[4], q[5], q[6], q[7]),
+                           pack_codes(q[8], q[9], q[10], q[11]), pack_codes(q[12], q[13], q[14], q[15]));
+        else
+            o = make_uint4(pack_codes(q[0], q[2], q[4], q[6]), pack_codes(q[1], q[3], q[5], q[7]),
+                           pack_codes(q[8], q[10], q[12], q[14]), pack_codes(q[9], q[11], q[13], q[15]));
+        *reinterpret_cast<uint4*>(out + 16 * static_cast<long long>(blk)) = o;
+    };
+#pragma unroll
+    for (int j = 0; j < RB; ++j)
+        if (lane + 32 * j < nblk) store16(v[j][0], v[j][1], lane + 32 * j);
+    for (int b = lane + 32 * RB; b < nblk; b += 32) store16(ldg_nc(xr + 2 * b), ldg_nc(xr + 2 * b + 1), b);
+}
+
+// RMSNorm then per-token absmax int8 (layout as launch_quant); g fp32 [K]
+// must be 16-byte aligned.
+cudaError_t launch_rmsnorm_quant(const uint16_t* x, const float* g, float eps, long long T, long long K, int8_t* xq,
+                                 float* s_tok, int layout, unsigned* status, cudaStream_t stream, void* zero16,
+                                 long long nzero16) {
+    const unsigned blocks = static_cast<unsigned>((T + 7) / 8);
+    uint4* zw = static_cast<uint4*>(zero16);
+    if (layout == kPairs)
+        rmsnorm_quant_kernel<kPairs><<<blocks, 256, 0, stream>>>(x, g, eps, T, K, xq, s_tok, zw, nzero16, status);
+    else
+        rmsnorm_quant_kernel<kNatural><<<blocks, 256, 0, stream>>>(x, g, eps, T, K, xq, s_tok, zw, nzero16, status);
+    return cudaGetLastError();
+}
+
 }  // namespace sbl

@@ -20,7 +20,11 @@ cudaError_t launch_decode(const uint8_t* packed, const float* row_scale, long lo
 bool decode_mma_supported(long long K);
 cudaError_t launch_decode_mma(const uint8_t* packed, const float* row_scale, long long O, long long K,
                               const uint16_t* x, long long T, void* y, int y_bf16, int32_t* acc_out, unsigned* status,
-                              int num_sms, cudaStream_t stream);
+                              int num_sms, cudaStream_t stream, const int8_t* xq_in = nullptr,
+                              const float* stok_in = nullptr);
+cudaError_t launch_rmsnorm_quant(const uint16_t* x, const float* g, float eps, long long T, long long K, int8_t* xq,
+                                 float* s_tok, int layout, unsigned* status, cudaStream_t stream, void* zero16,
+                                 long long nzero16);
 cudaError_t launch_prefill(const int8_t* xperm, const float* s_tok, long long T, long long K, const uint8_t* packed,
                            const float* row_scale, long long O, void* y, int y_bf16, int32_t* acc_out,
                            unsigned* status, int num_sms, int variant, int ksplit, int32_t* part,
@@ -128,6 +132,22 @@ sbl_status sbl_quant_act(const uint16_t* x_bf16, int64_t T, int64_t K, int8_t* x
                                        static_cast<cudaStream_t>(stream)));
 }
 
+sbl_status sbl_rmsnorm_quant_act(const uint16_t* x_bf16, const float* g, float eps, int64_t T, int64_t K,
+                                 int8_t* x_q, float* s_tok, void* stream) {
+    if (T < 0) return SBL_ERR_INVALID_ARG;
+    if (sbl_status s = check_k(K)) return s;
+    if (!(eps >= 0.0f) || !(eps < 3.0e38f)) return SBL_ERR_INVALID_ARG;
+    if (T == 0) return SBL_OK;
+    if (!x_bf16 || !g || !x_q || !s_tok) return SBL_ERR_INVALID_ARG;
+    if (!aligned(x_bf16, 16) || !aligned(g, 16) || !aligned(x_q, 16) || !aligned(s_tok, 16))
+        return SBL_ERR_INVALID_ARG;
+    if (T > (1ll << 31) - 1) return SBL_ERR_UNSUPPORTED;
+    DeviceInfo* d;
+    if (sbl_status s = device_info(&d)) return s;
+    return from_cuda(sbl::launch_rmsnorm_quant(x_bf16, g, eps, T, K, x_q, s_tok, sbl::kLayoutNatural, d->status,
+                                               static_cast<cudaStream_t>(stream), nullptr, 0));
+}
+
 // Quantised activations and their scales: what every path needs.
 static size_t base_workspace_bytes(int64_t T, int64_t K) {
     return round256(static_cast<size_t>(T) * static_cast<size_t>(K)) + round256(static_cast<size_t>(T) * 4);
@@ -172,11 +192,19 @@ static bool sparse_preferred(int64_t T, int64_t K, int64_t O, int num_sms) {
     return T >= 16384 && K >= 2048;
 }
 
-sbl_status sbl_linear_path(const uint16_t* x_bf16, int64_t T, int64_t K, const uint8_t* packed,
-                           const float* row_scale, int64_t O, int n, int m, void* y, int y_dtype, int32_t* acc_out,
-                           void* workspace, size_t workspace_bytes, int path, void* stream) {
+// The forward behind sbl_linear_path and sbl_linear_rmsnorm: with g the
+// activations are RMS-normalised by the front-end kernel before quantisation,
+// and the decode sizes take the warp-MMA kernel on the quantised activations.
+static sbl_status linear_impl(const uint16_t* x_bf16, const float* g, float eps, int64_t T, int64_t K,
+                              const uint8_t* packed, const float* row_scale, int64_t O, int n, int m, void* y,
+                              int y_dtype, int32_t* acc_out, void* workspace, size_t workspace_bytes, int path,
+                              void* stream) {
     if (T < 0 || O < 0) return SBL_ERR_INVALID_ARG;
     if (sbl_status s = check_k(K)) return s;
+    if (g) {
+        if (!(eps >= 0.0f) || !(eps < 3.0e38f)) return SBL_ERR_INVALID_ARG;
+        if (T > 0 && O > 0 && !aligned(g, 16)) return SBL_ERR_INVALID_ARG;
+    }
     if (!nm_ok(n, m)) return SBL_ERR_UNSUPPORTED;
     if (y_dtype != SBL_F32 && y_dtype != SBL_BF16) return SBL_ERR_INVALID_ARG;
     if (path < SBL_PATH_AUTO || path > SBL_PATH_PREFILL_SPARSE) return SBL_ERR_INVALID_ARG;
@@ -195,16 +223,21 @@ sbl_status sbl_linear_path(const uint16_t* x_bf16, int64_t T, int64_t K, const u
     const size_t sparse_need = sparse_eligible(K, n, m) ? need + sbl::sp_scratch_bytes(O, K) : 0;
     const bool sparse_fits = sparse_need != 0 && workspace_bytes >= sparse_need;
     if (path == SBL_PATH_PREFILL_SPARSE && !sparse_fits) return SBL_ERR_WORKSPACE;
+    bool prefill = forced_prefill;
+    if (path == SBL_PATH_AUTO) prefill = ((T > kDecodeMaxTokens) || (K > kDecodeMaxK)) && (K % 64 == 0);
+    if (!prefill && K > kDecodeMaxK) return SBL_ERR_UNSUPPORTED;
+    if (g && !prefill && !sbl::decode_mma_supported(K)) return SBL_ERR_UNSUPPORTED;
 
     DeviceInfo* d;
     if (sbl_status s = device_info(&d)) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     int8_t* xq = static_cast<int8_t*>(workspace);
     float* s_tok = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round256(static_cast<size_t>(T) * K));
-
-    bool prefill = forced_prefill;
-    if (path == SBL_PATH_AUTO) prefill = ((T > kDecodeMaxTokens) || (K > kDecodeMaxK)) && (K % 64 == 0);
-    if (!prefill && K > kDecodeMaxK) return SBL_ERR_UNSUPPORTED;
+    // the activation front end: absmax quantisation, RMSNorm first when g is given
+    auto front = [&](int layout, void* zero16, long long nzero16) {
+        return g ? sbl::launch_rmsnorm_quant(x_bf16, g, eps, T, K, xq, s_tok, layout, d->status, st, zero16, nzero16)
+                 : sbl::launch_quant(x_bf16, T, K, xq, s_tok, layout, d->status, st, zero16, nzero16);
+    };
 
     const int ybf = y_dtype == SBL_BF16 ? 1 : 0;
     cudaError_t e;
@@ -212,7 +245,7 @@ sbl_status sbl_linear_path(const uint16_t* x_bf16, int64_t T, int64_t K, const u
                                                    (path <= SBL_PATH_PREFILL && sparse_preferred(T, K, O, d->num_sms)));
     if (sparse) {
         uint8_t* scratch = static_cast<uint8_t*>(workspace) + need;
-        e = sbl::launch_quant(x_bf16, T, K, xq, s_tok, sbl::kLayoutNatural, d->status, st);
+        e = front(sbl::kLayoutNatural, nullptr, 0);
         if (e != cudaSuccess) return SBL_ERR_CUDA;
         e = sbl::launch_prefill_sp(xq, s_tok, T, K, packed, row_scale, O, y, ybf, acc_out, scratch, d->status,
                                    d->num_sms, st);
@@ -232,13 +265,19 @@ sbl_status sbl_linear_path(const uint16_t* x_bf16, int64_t T, int64_t K, const u
                 nzero16 = static_cast<long long>(sb / 16);
             }
         }
-        e = sbl::launch_quant(x_bf16, T, K, xq, s_tok, sbl::kLayoutPairs, d->status, st, part, nzero16);
+        e = front(sbl::kLayoutPairs, part, nzero16);
         if (e != cudaSuccess) return SBL_ERR_CUDA;
         const int variant = path == SBL_PATH_PREFILL_1CTA ? sbl::kPrefillOneCta
                             : path == SBL_PATH_PREFILL_PAIR ? sbl::kPrefillPair
                                                             : sbl::kPrefillAuto;
         e = sbl::launch_prefill(xq, s_tok, T, K, packed, row_scale, O, y, ybf, acc_out, d->status, d->num_sms, variant,
                                 ksplit, part, st);
+    } else if (g) {
+        // RMSNorm front end, then the warp-MMA decode on the quantised activations
+        e = front(sbl::kLayoutPairs, nullptr, 0);
+        if (e != cudaSuccess) return SBL_ERR_CUDA;
+        e = sbl::launch_decode_mma(packed, row_scale, O, K, x_bf16, T, y, ybf, acc_out, d->status, d->num_sms, st, xq,
+                                   s_tok);
     } else {
         // the decode kernels quantise the activations themselves
         if (T >= kDecodeMmaMinTokens && sbl::decode_mma_supported(K))
@@ -247,6 +286,22 @@ sbl_status sbl_linear_path(const uint16_t* x_bf16, int64_t T, int64_t K, const u
             e = sbl::launch_decode(packed, row_scale, O, K, x_bf16, T, y, ybf, acc_out, d->status, d->num_sms, st);
     }
     return from_cuda(e);
+}
+
+sbl_status sbl_linear_path(const uint16_t* x_bf16, int64_t T, int64_t K, const uint8_t* packed,
+                           const float* row_scale, int64_t O, int n, int m, void* y, int y_dtype, int32_t* acc_out,
+                           void* workspace, size_t workspace_bytes, int path, void* stream) {
+    return linear_impl(x_bf16, nullptr, 0.0f, T, K, packed, row_scale, O, n, m, y, y_dtype, acc_out, workspace,
+                       workspace_bytes, path, stream);
+}
+
+sbl_status sbl_linear_rmsnorm(const uint16_t* x_bf16, const float* g, float eps, int64_t T, int64_t K,
+                              const uint8_t* packed, const float* row_scale, int64_t O, int n, int m, void* y,
+                              int y_dtype, int32_t* acc_out, void* workspace, size_t workspace_bytes, int path,
+                              void* stream) {
+    if (!g) return SBL_ERR_INVALID_ARG;
+    return linear_impl(x_bf16, g, eps, T, K, packed, row_scale, O, n, m, y, y_dtype, acc_out, workspace,
+                       workspace_bytes, path, stream);
 }
 
 sbl_status sbl_linear(const uint16_t* x_bf16, int64_t T, int64_t K, const uint8_t* packed, const float* row_scale,

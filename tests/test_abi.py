@@ -87,6 +87,23 @@ def test_linear_rejects_on_host():
     assert L(p, 4, 64, p, p, 16, 2, 4, p, 0, None, None, 1 << 20, 0, None) == 6
 
 
+def test_rmsnorm_rejects_on_host():
+    from sparse_linear_layers_b200._lib import lib
+    p = 4096
+    R = lib.sbl_rmsnorm_quant_act
+    assert R(None, None, 1e-6, 0, 64, None, None, None) == 0          # T == 0: nothing to do
+    assert R(p, p, 1e-6, 4, 40, p, p, None) == 1                       # K % 16 != 0
+    assert R(p, p, -1.0, 4, 64, p, p, None) == 1                       # negative eps
+    assert R(p, p, float("nan"), 4, 64, p, p, None) == 1               # NaN eps
+    assert R(p, p + 4, 1e-6, 4, 64, p, p, None) == 1                   # unaligned g
+    L = lib.sbl_linear_rmsnorm
+    assert L(p, None, 1e-6, 4, 64, p, p, 16, 2, 4, p, 0, None, p, 1 << 20, 0, None) == 1   # g is required
+    assert L(p, p, -1.0, 4, 64, p, p, 16, 2, 4, p, 0, None, p, 1 << 20, 0, None) == 1     # negative eps
+    assert L(p, p, 1e-6, 4, 40, p, p, 16, 2, 4, p, 0, None, p, 1 << 20, 0, None) == 1     # K % 16 != 0
+    assert L(p, p, 1e-6, 4, 48, p, p, 16, 2, 4, p, 0, None, p, 1 << 20, 1, None) == 2     # decode needs K % 64
+    assert L(p, p, 1e-6, 4, 64, p, p, 16, 2, 4, p, 0, None, p, 16, 0, None) == 6          # workspace too small
+
+
 def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     import importlib
     from sparse_linear_layers_b200 import _lib
