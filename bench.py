@@ -409,6 +409,64 @@ def _prefill_roofline(sbl, dev, int8_peak_tops, hbm_peak):
     return out
 
 
+def _flushed_graph_us(fn, dev, reps=10):
+    """Median device time of ``fn`` captured in a CUDA graph, L2 flushed (256 MiB
+    write) before every timed replay, three untimed replays first."""
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        fn()
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        fn()
+    ts = []
+    with torch.cuda.stream(s):
+        for i in range(reps + 3):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(s)
+            g.replay()
+            b.record(s)
+            b.synchronize()
+            if i >= 3:
+                ts.append(a.elapsed_time(b) * 1e3)
+    del g, flush
+    return statistics.median(ts)
+
+
+def _rmsnorm_front(sbl, dev, hbm_peak, T=32768):
+    """The guide module's front end (RMSNorm, then per-token absmax int8) against
+    the plain quantisation at the 0.5B FFN input widths, and the whole module
+    forward against sbl_linear on the FFN gate (896 -> 4864, 3:4, bf16 output)."""
+    out = {"tokens": T, "eps": sbl.RMSNORM_EPS_F32}
+    for K in (896, 4864):
+        xb, _ = synthetic.activations(T, K, seed=14, tag="rms", outlier_p=0.01)
+        x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)
+        gw = torch.from_numpy(np.random.default_rng(14).uniform(0.5, 1.5, K).astype(np.float32)).to(dev)
+        byts = T * K * 2 + T * K + 4 * T + 4 * K
+        q_us = _flushed_graph_us(lambda: sbl.sbl_quant_act(x), dev)
+        r_us = _flushed_graph_us(lambda: sbl.sbl_rmsnorm_quant_act(x, gw), dev)
+        out[f"K{K}"] = {"algorithmic_bytes": byts, "quant_us": q_us, "rmsnorm_quant_us": r_us,
+                        "rmsnorm_quant_gbs": byts / r_us / 1e3, "rmsnorm_quant_hbm_frac": byts / r_us / 1e3 / hbm_peak,
+                        "quant_gbs": byts / q_us / 1e3}
+        del x
+    K, O = 896, 4864
+    W = torch.from_numpy(synthetic.latent_weights(O, K, seed=14, tag="rms-gate")).to(dev)
+    w = sbl.sbl_prepare_weights(W, 3, 4)
+    del W
+    xb, _ = synthetic.activations(T, K, seed=14, tag="rms-gate", outlier_p=0.01)
+    x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)
+    gw = torch.ones(K, dtype=torch.float32, device=dev)
+    y = torch.empty((T, O), dtype=torch.bfloat16, device=dev)
+    ws = sbl.workspace_for(T, K, O, 3, 4, dev)
+    lin = _flushed_graph_us(lambda: sbl.sbl_linear(x, w, y=y, workspace=ws), dev)
+    mod = _flushed_graph_us(lambda: sbl.sbl_linear_rmsnorm(x, w, gw, y=y, workspace=ws), dev)
+    out["gate_896->4864_3:4_bf16"] = {"sbl_linear_us": lin, "sbl_linear_rmsnorm_us": mod, "ratio": mod / lin}
+    del x, y, ws, w
+    return out
+
+
 def _pool_call_us(sbl, x, w, y, ws, reps=5):
     """Per-call device time of sbl_linear in steady state: a CUDA graph of
     back-to-back calls that cycle through copies of the weights and
@@ -582,6 +640,7 @@ def run_ours(args, rank, world, dev):
         decode["T8"] = _decode_roofline(sbl, dev, hbm_peak, T=8)
     prefill_big = _prefill_roofline(sbl, dev, int8_peak_tops, hbm_peak) if rank == 0 else None
     configs = _configs_sweep(sbl, dev) if rank == 0 and not args.no_configs else None
+    rms_front = _rmsnorm_front(sbl, dev, hbm_peak) if rank == 0 and not args.no_configs else None
     launches_per_step = len(layers) * (1 + 2 + 1)  # prep + (quant + tcgen05 GEMM) + fused decode
     value = _throughput(world, K, total_s)
     out = {
@@ -594,6 +653,7 @@ def run_ours(args, rank, world, dev):
         "decode_roofline": decode,
         "prefill_roofline": prefill_big,
         "configs": configs,
+        "rmsnorm_front": rms_front,
         "phases": phases,
         "e2e": {"value": world * TOKENS_PER_STEP * K_e2e / e2e_s, "steps": K_e2e, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},

@@ -186,7 +186,41 @@ cudaError_t launch_quant(const uint16_t* x, long long T, long long K, int8_t* xq
 // lanes (every lane ends with the same total).  A lane keeps up to RB blocks
 // in registers across the three passes (sum of squares, absmax of the
 // normalised values, quantisation); blocks beyond that are read again.
-template <int LAYOUT>
+// Non-finite input shows as a non-finite sum of squares (a square that
+// overflows float32 does too) or normalised value, and sets the status bit.
+// Pairs of floats in one 64-bit register, for the sm_100 paired float
+// instructions (each half rounded exactly like the scalar IEEE operation).
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2split(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+// Three-input max / min that propagate NaN.
+__device__ __forceinline__ float max3n(float a, float b, float c) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+__device__ __forceinline__ float min3n(float a, float b, float c) {
+    float r;
+    asm("min.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+template <int LAYOUT, int RB>
 __global__ void __launch_bounds__(256) rmsnorm_quant_kernel(const uint16_t* __restrict__ x,
                                                             const float* __restrict__ g, float eps, long long T,
                                                             long long K, int8_t* __restrict__ xq,
@@ -194,24 +228,23 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_kernel(const uint16_t* __re
                                                             long long nzero, unsigned* status) {
     asm volatile("griddepcontrol.launch_dependents;");
     zero_fill(zero_words, nzero);
-    constexpr int RB = 4;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long t = static_cast<long long>(blockIdx.x) * 8 + warp;
     if (t >= T) return;
     const uint4* xr = reinterpret_cast<const uint4*>(x + t * K);
     const int nblk = static_cast<int>(K >> 4);
     uint4 v[RB][2];
-    // pass 1: sum of squares in the lane's k order; non-finite inputs flagged
+    // pass 1: sum of squares in the lane's k order
     float ss = 0.f;
-    uint32_t bad = 0;
     auto add_sq = [&](const uint4& a, const uint4& b) {
         const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xFFFF0000u);
-            ss = __fadd_rn(ss, __fmul_rn(lo, lo));
-            ss = __fadd_rn(ss, __fmul_rn(hi, hi));
-            bad |= ((w[i] & 0x7F80u) == 0x7F80u) | ((w[i] & 0x7F800000u) == 0x7F800000u);
+            const uint64_t p = f2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+            float lo, hi;
+            f2split(mul2(p, p), lo, hi);  // squares of elements 2i and 2i + 1
+            ss = __fadd_rn(ss, lo);
+            ss = __fadd_rn(ss, hi);
         }
     };
 #pragma unroll
@@ -231,64 +264,83 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_kernel(const uint16_t* __re
     const float ms = __fdiv_rn(ss, static_cast<float>(K));
     const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
 
-    // normalised values of one block: (x * inv) * g
-    auto norm16 = [&](const uint4& a, const uint4& b, int blk, float (&n)[16]) {
-        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-        const float4* g4 = reinterpret_cast<const float4*>(g + 16 * blk);
-        float gv[16];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float4 q = __ldg(g4 + i);
-            gv[4 * i] = q.x;
-            gv[4 * i + 1] = q.y;
-            gv[4 * i + 2] = q.z;
-            gv[4 * i + 3] = q.w;
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            n[2 * i] = __fmul_rn(__fmul_rn(__uint_as_float(w[i] << 16), inv), gv[2 * i]);
-            n[2 * i + 1] = __fmul_rn(__fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), inv), gv[2 * i + 1]);
-        }
+    // Passes 2 and 3 take a coalesced mapping (any works: the absmax and the
+    // elementwise quantisation do not depend on order): lane l handles the
+    // four elements 4l + 128i .. 4l + 128i + 3, re-reading x (now in L1) with
+    // 8-byte loads and g with 16-byte loads, every warp access contiguous.
+    const uint64_t inv2 = f2(inv, inv);
+    const uint2* xr2 = reinterpret_cast<const uint2*>(x + t * K);
+    const float4* g4 = reinterpret_cast<const float4*>(g);
+    const int nstripe = static_cast<int>((K + 127) >> 7);
+    // (x * inv) * g of four elements, as two pairs
+    auto norm4 = [&](int k4, uint64_t& n01, uint64_t& n23) {
+        const uint2 w = __ldg(xr2 + k4);
+        const float4 q = __ldg(g4 + k4);
+        n01 = mul2(mul2(f2(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u)), inv2), f2(q.x, q.y));
+        n23 = mul2(mul2(f2(__uint_as_float(w.y << 16), __uint_as_float(w.y & 0xFFFF0000u)), inv2), f2(q.z, q.w));
     };
-    // pass 2: absmax of the normalised values (bit patterns of |n| order like the values)
-    uint32_t mx = 0;
-    auto max16 = [&](const uint4& a, const uint4& b, int blk) {
-        float n[16];
-        norm16(a, b, blk, n);
+    // pass 2: largest and smallest normalised value (NaN propagates)
+    float hi_v = 0.f, lo_v = 0.f;
+    for (int i = 0; i < nstripe; ++i) {
+        const int k4 = lane + 32 * i;  // index of the 4-element group
+        if (4 * k4 < K) {
+            uint64_t n01, n23;
+            norm4(k4, n01, n23);
+            float e0, e1, e2, e3;
+            f2split(n01, e0, e1);
+            f2split(n23, e2, e3);
+            hi_v = max3n(hi_v, e0, e1);
+            lo_v = min3n(lo_v, e0, e1);
+            hi_v = max3n(hi_v, e2, e3);
+            lo_v = min3n(lo_v, e2, e3);
+        }
+    }
+    float amax = max3n(hi_v, -lo_v, 0.f);  // max |x_norm| of this lane (NaN if any value was NaN)
 #pragma unroll
-        for (int i = 0; i < 16; ++i) mx = max(mx, __float_as_uint(n[i]) & 0x7FFFFFFFu);
-    };
-#pragma unroll
-    for (int j = 0; j < RB; ++j)
-        if (lane + 32 * j < nblk) max16(v[j][0], v[j][1], lane + 32 * j);
-    for (int b = lane + 32 * RB; b < nblk; b += 32) max16(ldg_nc(xr + 2 * b), ldg_nc(xr + 2 * b + 1), b);
-    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
-    bad = __reduce_or_sync(0xFFFFFFFFu, bad);
-    if (lane == 0 && (bad || mx >= 0x7F800000u)) raise_status(status, kStatusNonfinite);
-    const float s = __fdiv_rn(127.0f, fmaxf(__uint_as_float(mx), 1e-5f));
+    for (int off = 16; off >= 1; off >>= 1) amax = max3n(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off), 0.f);
+    if (lane == 0 && !(fabsf(ss) <= 3.4028235e38f && amax <= 3.4028235e38f)) raise_status(status, kStatusNonfinite);
+    const float s = __fdiv_rn(127.0f, fmaxf(amax, 1e-5f));
     if (lane == 0) s_tok[t] = s;
 
-    // pass 3: quantise and store in the requested layout
-    int8_t* out = xq + t * K;
-    auto store16 = [&](const uint4& a, const uint4& b, int blk) {
-        float n[16];
-        norm16(a, b, blk, n);
-        uint32_t q[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) q[i] = quant_code_bits(n[i], s);
-        uint4 o;
-        if (LAYOUT == kNatural)
-            o = make_uint4(pack_codes(q[0], q[1], q[2], q[3]), pack_codes(q[4], q[5], q[6], q[7]),
-                           pack_codes(q[8], q[9], q[10], q[11]), pack_codes(q[12], q[13], q[14], q[15]));
-        else
-            o = make_uint4(pack_codes(q[0], q[2], q[4], q[6]), pack_codes(q[1], q[3], q[5], q[7]),
-                           pack_codes(q[8], q[10], q[12], q[14]), pack_codes(q[9], q[11], q[13], q[15]));
-        *reinterpret_cast<uint4*>(out + 16 * static_cast<long long>(blk)) = o;
-    };
-#pragma unroll
-    for (int j = 0; j < RB; ++j)
-        if (lane + 32 * j < nblk) store16(v[j][0], v[j][1], lane + 32 * j);
-    for (int b = lane + 32 * RB; b < nblk; b += 32) store16(ldg_nc(xr + 2 * b), ldg_nc(xr + 2 * b + 1), b);
+    // pass 3: quantise (quant_code_bits two at a time) and store.  In the
+    // pairing layout a 16-element block's word q holds the even (q = 0, 2) or
+    // odd (q = 1, 3) elements of lanes q & ~1 and q | 1, so neighbouring lanes
+    // swap codes once and each stores the word at its own position.
+    const uint64_t s2 = f2(s, s), magic2 = f2(12582912.0f, 12582912.0f);
+    uint32_t* out = reinterpret_cast<uint32_t*>(xq + t * K);
+    for (int i = 0; i < nstripe; ++i) {
+        const int k4 = lane + 32 * i;
+        const bool ok = 4 * k4 < K;  // whole 16-element blocks: lanes l and l ^ 1 agree
+        uint32_t p = 0;
+        if (ok) {
+            uint64_t n01, n23;
+            norm4(k4, n01, n23);
+            float c0, c1, c2, c3;
+            f2split(add2(mul2(n01, s2), magic2), c0, c1);
+            f2split(add2(mul2(n23, s2), magic2), c2, c3);
+            p = pack_codes(__float_as_uint(c0), __float_as_uint(c1), __float_as_uint(c2), __float_as_uint(c3));
+        }
+        if (LAYOUT == kNatural) {
+            if (ok) out[k4] = p;
+        } else {
+            const uint32_t pp = __shfl_xor_sync(0xFFFFFFFFu, p, 1);
+            const uint32_t word = (lane & 1) ? prmt(pp, p, 0x7531u) : prmt(p, pp, 0x6420u);
+            if (ok) out[k4] = word;
+        }
+    }
+}
+
+template <int LAYOUT>
+static void launch_rms_rb(const uint16_t* x, const float* g, float eps, long long T, long long K, int8_t* xq,
+                          float* s_tok, uint4* zw, long long nzero, unsigned* status, cudaStream_t stream) {
+    const unsigned blocks = static_cast<unsigned>((T + 7) / 8);
+    const long long per_lane = ((K >> 4) + 31) / 32;  // blocks per lane
+    if (per_lane <= 1)
+        rmsnorm_quant_kernel<LAYOUT, 1><<<blocks, 256, 0, stream>>>(x, g, eps, T, K, xq, s_tok, zw, nzero, status);
+    else if (per_lane <= 2)
+        rmsnorm_quant_kernel<LAYOUT, 2><<<blocks, 256, 0, stream>>>(x, g, eps, T, K, xq, s_tok, zw, nzero, status);
+    else
+        rmsnorm_quant_kernel<LAYOUT, 4><<<blocks, 256, 0, stream>>>(x, g, eps, T, K, xq, s_tok, zw, nzero, status);
 }
 
 // RMSNorm then per-token absmax int8 (layout as launch_quant); g fp32 [K]
@@ -296,12 +348,11 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_kernel(const uint16_t* __re
 cudaError_t launch_rmsnorm_quant(const uint16_t* x, const float* g, float eps, long long T, long long K, int8_t* xq,
                                  float* s_tok, int layout, unsigned* status, cudaStream_t stream, void* zero16,
                                  long long nzero16) {
-    const unsigned blocks = static_cast<unsigned>((T + 7) / 8);
     uint4* zw = static_cast<uint4*>(zero16);
     if (layout == kPairs)
-        rmsnorm_quant_kernel<kPairs><<<blocks, 256, 0, stream>>>(x, g, eps, T, K, xq, s_tok, zw, nzero16, status);
+        launch_rms_rb<kPairs>(x, g, eps, T, K, xq, s_tok, zw, nzero16, status, stream);
     else
-        rmsnorm_quant_kernel<kNatural><<<blocks, 256, 0, stream>>>(x, g, eps, T, K, xq, s_tok, zw, nzero16, status);
+        launch_rms_rb<kNatural>(x, g, eps, T, K, xq, s_tok, zw, nzero16, status, stream);
     return cudaGetLastError();
 }
 

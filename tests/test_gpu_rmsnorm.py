@@ -86,3 +86,18 @@ def test_linear_rmsnorm_decode_needs_k_multiple_of_64(sbl):
     w = sbl.sbl_prepare_weights(to_dev(W), 2, 4)
     with pytest.raises(sbl.SblError):
         sbl.sbl_linear_rmsnorm(x_dev(xbits), w, to_dev(np.ones(48, np.float32)))
+
+
+def test_rmsnorm_nonfinite_sets_status(sbl):
+    K = 64
+    _, xbits, _ = layer_inputs(8, K, 3, seed=6)
+    xbits = xbits.copy()
+    xbits[1, 5] = 0x7F80  # +inf
+    sbl.sbl_rmsnorm_quant_act(x_dev(xbits), to_dev(np.ones(K, np.float32)))
+    assert sbl.sbl_device_status() == 3
+    zeros = np.zeros((2, K), np.uint16)  # an all-zero token with eps = 0 divides by zero
+    sbl.sbl_rmsnorm_quant_act(x_dev(zeros), to_dev(np.ones(K, np.float32)), 0.0)
+    assert sbl.sbl_device_status() == 3
+    xq, s = sbl.sbl_rmsnorm_quant_act(x_dev(zeros), to_dev(np.ones(K, np.float32)), 1e-6)
+    assert sbl.sbl_device_status() == 0
+    assert not xq.cpu().numpy().any()
