@@ -221,6 +221,26 @@ def rmsnorm_quant_act(x: np.ndarray, g: np.ndarray, eps: float):
     return quant_act(rmsnorm(x, g, eps))
 
 
+def mask_monitor(old_bits: np.ndarray, new_bits: np.ndarray, K: int, n: int, m: int):
+    """Mask change rate and verification between two mask bitmaps uint8 [O, K/8]
+    (bit k % 8 of byte k // 8 set when weight k is kept).
+
+    Returns (changed, bad_groups, row_changed): the number of positions whose
+    kept state differs, the number of M-groups of ``new_bits`` that do not keep
+    exactly N weights, and the changed count per row (int64 [O]).
+    The Sparse-BitNet README ("Features": dynamic mask monitoring; the CLI's
+    mask-monitor interval: the mask change rate every N steps) and the
+    halo-sparse-bitnet-3:4-500m card ("Recipe": mask-verify every 500 steps);
+    the rate is changed / (O * K).
+    """
+    _check_nm(K, n, m)
+    old = np.unpackbits(np.asarray(old_bits, np.uint8), axis=1, bitorder="little")[:, :K].astype(bool)
+    new = np.unpackbits(np.asarray(new_bits, np.uint8), axis=1, bitorder="little")[:, :K].astype(bool)
+    row_changed = np.count_nonzero(old != new, axis=1).astype(np.int64)
+    kept = new.reshape(new.shape[0], K // m, m).sum(axis=2)
+    return int(row_changed.sum()), int(np.count_nonzero(kept != n)), row_changed
+
+
 def int_contract(xq: np.ndarray, Wt: np.ndarray) -> np.ndarray:
     """int32 [T, O] = x_q . W_t^T (the guide's integer product before rescaling).
 

@@ -536,3 +536,78 @@ def test_planted_rms_mistake_is_caught(name):
         except (AssertionError, ValueError, IndexError):
             caught.append(pin.__name__)
     assert caught, f"no pin caught the planted mistake {name}"
+
+
+# --------------------------------------------------------------------------
+# mask monitor (change rate between two masks, mask verification)
+# --------------------------------------------------------------------------
+
+def _brute_monitor(old_bits, new_bits, K, n, m):
+    """Bit by bit with Python integers: byte k // 8, bit k % 8."""
+    O = old_bits.shape[0]
+    changed, bad, rows = 0, 0, []
+    for i in range(O):
+        r = 0
+        for k in range(K):
+            a = (int(old_bits[i, k // 8]) >> (k % 8)) & 1
+            b = (int(new_bits[i, k // 8]) >> (k % 8)) & 1
+            r += a != b
+        rows.append(r)
+        changed += r
+        for grp in range(K // m):
+            kept = sum((int(new_bits[i, k // 8]) >> (k % 8)) & 1 for k in range(grp * m, grp * m + m))
+            bad += kept != n
+    return changed, bad, rows
+
+
+def pin_mask_monitor(o):
+    rng = np.random.default_rng(11)
+    for (O, K, n, m) in ((3, 16, 2, 4), (5, 64, 3, 4), (2, 48, 6, 8), (4, 32, 2, 4)):
+        a = rng.integers(0, 256, (O, K // 8), dtype=np.uint8)
+        b = rng.integers(0, 256, (O, K // 8), dtype=np.uint8)
+        ch, bad, rows = o.mask_monitor(a, b, K, n, m)
+        bch, bbad, brows = _brute_monitor(a, b, K, n, m)
+        assert (ch, bad, list(rows)) == (bch, bbad, brows)
+        assert o.mask_monitor(a, a, K, n, m)[0] == 0
+        assert o.mask_monitor(a, ~a, K, n, m)[0] == O * K
+        assert o.mask_monitor(b, a, K, n, m)[0] == ch
+    # masks made by the weight preparation keep exactly N per group; one flipped
+    # bit is one changed position and one bad group
+    for n, m in PATTERNS:
+        W = synthetic.latent_weights(6, 64, seed=5)
+        _, _, mb, _ = oracle.prepare_weights(W, n, m)
+        assert o.mask_monitor(mb, mb, 64, n, m)[:2] == (0, 0)
+        mb2 = mb.copy()
+        mb2[2, 3] ^= 0x10  # weight 28 of row 2
+        ch, bad, rows = o.mask_monitor(mb, mb2, 64, n, m)
+        assert (ch, bad) == (1, 1) and rows.tolist() == [0, 0, 1, 0, 0, 0]
+
+
+def test_mask_monitor_pins():
+    pin_mask_monitor(oracle)
+
+
+def _mm_changed_bytes(old_bits, new_bits, K, n, m):
+    _, bad, _ = oracle.mask_monitor(old_bits, new_bits, K, n, m)
+    rows = np.count_nonzero(np.asarray(old_bits) != np.asarray(new_bits), axis=1).astype(np.int64)
+    return int(rows.sum()), bad, rows
+
+
+def _mm_verify_old(old_bits, new_bits, K, n, m):
+    return oracle.mask_monitor(new_bits, old_bits, K, n, m)[0], oracle.mask_monitor(new_bits, old_bits, K, n, m)[1], \
+        oracle.mask_monitor(old_bits, new_bits, K, n, m)[2]
+
+
+def _mm_kept_at_most(old_bits, new_bits, K, n, m):
+    ch, _, rows = oracle.mask_monitor(old_bits, new_bits, K, n, m)
+    new = np.unpackbits(np.asarray(new_bits, np.uint8), axis=1, bitorder="little")[:, :K].astype(bool)
+    kept = new.reshape(new.shape[0], K // m, m).sum(axis=2)
+    return ch, int(np.count_nonzero(kept > n)), rows
+
+
+@pytest.mark.parametrize("name,fn", [("changed_bytes_not_bits", _mm_changed_bytes), ("verifies_old_mask", _mm_verify_old),
+                                     ("counts_only_excess", _mm_kept_at_most)])
+def test_planted_mask_monitor_mistake_is_caught(name, fn):
+    o = types.SimpleNamespace(mask_monitor=fn)
+    with pytest.raises(AssertionError):
+        pin_mask_monitor(o)
