@@ -467,6 +467,28 @@ def _rmsnorm_front(sbl, dev, hbm_peak, T=32768):
     return out
 
 
+def _mask_monitor_bench(sbl, dev, hbm_peak):
+    """Mask change count and verification between two bitmaps: a large pair
+    (32768 x 8192 weights, 2 x 32 MiB, HBM-bound) and one 2048 -> 7168
+    projection (2 x 1.8 MB, latency-bound), graph-replayed with L2 flushed."""
+    out = {}
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(15)
+    for name, (O, K) in (("32768x8192", (32768, 8192)), ("7168x2048", (7168, 2048))):
+        a = torch.randint(0, 256, (O, K // 8), dtype=torch.uint8, device=dev, generator=gen)
+        b = torch.randint(0, 256, (O, K // 8), dtype=torch.uint8, device=dev, generator=gen)
+        totals = torch.empty(2, dtype=torch.int64, device=dev)
+        from sparse_linear_layers_b200 import _lib
+        fn = lambda: _lib.check(_lib.lib.sbl_mask_monitor(a.data_ptr(), b.data_ptr(), O, K, 2, 4, totals.data_ptr(),
+                                                          None, torch.cuda.current_stream().cuda_stream),
+                                "sbl_mask_monitor")
+        us = _flushed_graph_us(fn, dev)
+        byts = 2 * O * K // 8
+        out[name] = {"bytes": byts, "us_per_call": us, "gbs": byts / us / 1e3, "hbm_frac": byts / us / 1e3 / hbm_peak}
+        del a, b
+    return out
+
+
 def _pool_call_us(sbl, x, w, y, ws, reps=5):
     """Per-call device time of sbl_linear in steady state: a CUDA graph of
     back-to-back calls that cycle through copies of the weights and
@@ -641,6 +663,7 @@ def run_ours(args, rank, world, dev):
     prefill_big = _prefill_roofline(sbl, dev, int8_peak_tops, hbm_peak) if rank == 0 else None
     configs = _configs_sweep(sbl, dev) if rank == 0 and not args.no_configs else None
     rms_front = _rmsnorm_front(sbl, dev, hbm_peak) if rank == 0 and not args.no_configs else None
+    mask_mon = _mask_monitor_bench(sbl, dev, hbm_peak) if rank == 0 and not args.no_configs else None
     launches_per_step = len(layers) * (1 + 2 + 1)  # prep + (quant + tcgen05 GEMM) + fused decode
     value = _throughput(world, K, total_s)
     out = {
@@ -654,6 +677,7 @@ def run_ours(args, rank, world, dev):
         "prefill_roofline": prefill_big,
         "configs": configs,
         "rmsnorm_front": rms_front,
+        "mask_monitor": mask_mon,
         "phases": phases,
         "e2e": {"value": world * TOKENS_PER_STEP * K_e2e / e2e_s, "steps": K_e2e, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},

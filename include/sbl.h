@@ -132,6 +132,27 @@ sbl_status sbl_rmsnorm_quant_act(const uint16_t* x_bf16, const float* g, float e
                                  int8_t* x_q, float* s_tok, void* stream);
 
 /*
+ * sbl_mask_monitor — mask change rate and mask verification.
+ *
+ * The Sparse-BitNet README ("Features": dynamic mask monitoring during
+ * training; its CLI monitors the mask change rate every N steps) and the
+ * halo-sparse-bitnet-3:4-500m card ("Recipe": mask-verify every 500 steps).
+ * Compares two mask bitmaps as sbl_prepare_weights writes them (uint8
+ * [O, K/8], bit k % 8 of byte k / 8 set when weight k is kept, 16-byte
+ * aligned):
+ *   totals       uint64 [2] on the device (output, 8-byte aligned):
+ *                totals[0] = positions whose kept state differs between
+ *                old_bits and new_bits (the change rate is totals[0] / (O*K));
+ *                totals[1] = M-groups of new_bits that do not keep exactly N.
+ *   row_changed  uint32 [O] on the device (output, may be NULL): the changed
+ *                positions of each row.
+ * (n, m) as for sbl_prepare_weights.  Asynchronous on `stream`; totals are
+ * overwritten (not accumulated).
+ */
+sbl_status sbl_mask_monitor(const uint8_t* old_bits, const uint8_t* new_bits, int64_t O, int64_t K, int n, int m,
+                            uint64_t* totals, uint32_t* row_changed, void* stream);
+
+/*
  * sbl_linear_workspace_bytes — bytes of device workspace sbl_linear needs for
  * these sizes: the quantised activations and their scales, in the kernels'
  * internal layout (T*K + 4*T bytes, each rounded up to 256), plus, for 2:4

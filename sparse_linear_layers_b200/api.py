@@ -155,6 +155,23 @@ def sbl_linear_rmsnorm(x: torch.Tensor, w: PreparedWeights, g: torch.Tensor, eps
     return y
 
 
+def sbl_mask_monitor(old_bits: torch.Tensor, new_bits: torch.Tensor, K: int, n: int, m: int, per_row: bool = False,
+                     stream: Optional[torch.cuda.Stream] = None):
+    """Mask change and verification on the device: (totals int64 [2] = [changed
+    positions, groups not keeping exactly N], row_changed int32 [O] or None).
+    Nothing is copied to the host."""
+    _need_cuda(old_bits, "old_bits", torch.uint8)
+    _need_cuda(new_bits, "new_bits", torch.uint8)
+    O = old_bits.shape[0]
+    if old_bits.shape != (O, K // 8) or new_bits.shape != (O, K // 8):
+        raise ValueError("mask bitmaps must both be uint8 [O, K/8]")
+    totals = torch.empty(2, dtype=torch.int64, device=old_bits.device)
+    rows = torch.empty(O, dtype=torch.int32, device=old_bits.device) if per_row else None
+    check(lib.sbl_mask_monitor(old_bits.data_ptr(), new_bits.data_ptr(), O, K, n, m, totals.data_ptr(),
+                               rows.data_ptr() if rows is not None else None, _stream(stream)), "sbl_mask_monitor")
+    return totals, rows
+
+
 _PATH_NAMES = {v: k for k, v in _PATHS.items()}
 
 

@@ -25,6 +25,8 @@ cudaError_t launch_decode_mma(const uint8_t* packed, const float* row_scale, lon
 cudaError_t launch_rmsnorm_quant(const uint16_t* x, const float* g, float eps, long long T, long long K, int8_t* xq,
                                  float* s_tok, int layout, unsigned* status, cudaStream_t stream, void* zero16,
                                  long long nzero16);
+cudaError_t launch_mask_monitor(const uint8_t* old_bits, const uint8_t* new_bits, long long O, long long K, int n,
+                                int m, unsigned long long* totals, uint32_t* row_changed, cudaStream_t stream);
 cudaError_t launch_prefill(const int8_t* xperm, const float* s_tok, long long T, long long K, const uint8_t* packed,
                            const float* row_scale, long long O, void* y, int y_bf16, int32_t* acc_out,
                            unsigned* status, int num_sms, int variant, int ksplit, int32_t* part,
@@ -146,6 +148,23 @@ sbl_status sbl_rmsnorm_quant_act(const uint16_t* x_bf16, const float* g, float e
     if (sbl_status s = device_info(&d)) return s;
     return from_cuda(sbl::launch_rmsnorm_quant(x_bf16, g, eps, T, K, x_q, s_tok, sbl::kLayoutNatural, d->status,
                                                static_cast<cudaStream_t>(stream), nullptr, 0));
+}
+
+sbl_status sbl_mask_monitor(const uint8_t* old_bits, const uint8_t* new_bits, int64_t O, int64_t K, int n, int m,
+                            uint64_t* totals, uint32_t* row_changed, void* stream) {
+    if (O < 0) return SBL_ERR_INVALID_ARG;
+    if (sbl_status s = check_k(K)) return s;
+    if (!nm_ok(n, m)) return SBL_ERR_UNSUPPORTED;
+    if (!totals || !aligned(totals, 8)) return SBL_ERR_INVALID_ARG;
+    if (O > 0 && (!old_bits || !new_bits || !aligned(old_bits, 16) || !aligned(new_bits, 16))) return SBL_ERR_INVALID_ARG;
+    if (row_changed && !aligned(row_changed, 4)) return SBL_ERR_INVALID_ARG;
+    if (O > (1ll << 31) - 1) return SBL_ERR_UNSUPPORTED;
+    DeviceInfo* d;
+    if (sbl_status s = device_info(&d)) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (O == 0) return from_cuda(cudaMemsetAsync(totals, 0, 2 * sizeof(uint64_t), st));
+    return from_cuda(sbl::launch_mask_monitor(old_bits, new_bits, O, K, n, m,
+                                              reinterpret_cast<unsigned long long*>(totals), row_changed, st));
 }
 
 // Quantised activations and their scales: what every path needs.

@@ -104,6 +104,18 @@ def test_rmsnorm_rejects_on_host():
     assert L(p, p, 1e-6, 4, 64, p, p, 16, 2, 4, p, 0, None, p, 16, 0, None) == 6          # workspace too small
 
 
+def test_mask_monitor_rejects_on_host():
+    from sparse_linear_layers_b200._lib import lib
+    p = 4096
+    M = lib.sbl_mask_monitor
+    assert M(p, p, 8, 40, 2, 4, p, None, None) == 1          # K % 16 != 0
+    assert M(p, p, 8, 64, 4, 8, p, None, None) == 2          # unsupported pattern
+    assert M(p, p, 8, 64, 2, 4, None, None, None) == 1       # totals required
+    assert M(p + 8, p, 8, 64, 2, 4, p, None, None) == 1      # unaligned bitmap
+    assert M(p, p, 8, 64, 2, 4, p, p + 2, None) == 1         # unaligned row counts
+    assert M(p, p, -1, 64, 2, 4, p, None, None) == 1         # negative O
+
+
 def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     import importlib
     from sparse_linear_layers_b200 import _lib
