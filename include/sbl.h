@@ -23,7 +23,7 @@
  *     that ran out) set bits in a per-device status word that
  *     sbl_device_status() reads; kernels never trap.
  *   - Shapes: row-major, int64 sizes; O, T >= 0 (zero sizes are no-ops);
- *     K > 0 and K % 16 == 0.  (n, m) must be (2,4), (3,4) or (6,8).
+ *     K > 0 and K % 16 == 0.  (n, m) must be (2,4), (3,4), (6,8) or (4,8).
  *   - Nothing throws across this boundary.
  */
 #ifndef SBL_H

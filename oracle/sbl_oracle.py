@@ -55,7 +55,7 @@ import numpy as np
 
 EPS_SCALE = np.float32(1e-5)   # clamp of the weight absmean (guide's module listing)
 EPS_ACT = np.float32(1e-5)     # clamp of the activation absmax (guide's module listing)
-SUPPORTED_NM = ((2, 4), (3, 4), (6, 8))
+SUPPORTED_NM = ((2, 4), (3, 4), (6, 8), (4, 8))
 
 
 def _check_nm(K: int, n: int, m: int) -> None:

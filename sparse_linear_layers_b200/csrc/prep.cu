@@ -457,6 +457,7 @@ cudaError_t launch_prep(const float* W, long long O, long long K, int n, int m, 
                         uint8_t* mask_bits, unsigned* status, cudaStream_t stream) {
     if (m == 4 && n == 2) launch_prep_mn<4, 2>(W, O, K, packed, row_scale, mask_bits, status, stream);
     else if (m == 4) launch_prep_mn<4, 3>(W, O, K, packed, row_scale, mask_bits, status, stream);
+    else if (n == 4) launch_prep_mn<8, 4>(W, O, K, packed, row_scale, mask_bits, status, stream);
     else launch_prep_mn<8, 6>(W, O, K, packed, row_scale, mask_bits, status, stream);
     return cudaGetLastError();
 }

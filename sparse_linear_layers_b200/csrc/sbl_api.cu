@@ -89,7 +89,11 @@ sbl_status device_info(DeviceInfo** out) {
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
-inline bool nm_ok(int n, int m) { return (n == 2 && m == 4) || (n == 3 && m == 4) || (n == 6 && m == 8); }
+// 2:4, 3:4 and 6:8 (the patterns of the guide and the halo card) and 4:8 (the
+// guide's "Architectural Comparison" table)
+inline bool nm_ok(int n, int m) {
+    return (n == 2 && m == 4) || (n == 3 && m == 4) || (n == 6 && m == 8) || (n == 4 && m == 8);
+}
 
 inline size_t round256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
 

@@ -52,7 +52,7 @@ def test_workspace_bytes():
     ((8, 0, 2, 4), 1),       # K == 0
     ((8, 40, 2, 4), 1),      # K % 16 != 0
     ((8, 64, 1, 4), 2),      # unsupported N:M
-    ((8, 64, 4, 8), 2),
+    ((8, 64, 5, 8), 2),
     ((8, 1 << 25, 2, 4), 2), # K beyond the int32-accumulator bound
 ])
 def test_prepare_rejects_on_host(args, code):
@@ -109,7 +109,7 @@ def test_mask_monitor_rejects_on_host():
     p = 4096
     M = lib.sbl_mask_monitor
     assert M(p, p, 8, 40, 2, 4, p, None, None) == 1          # K % 16 != 0
-    assert M(p, p, 8, 64, 4, 8, p, None, None) == 2          # unsupported pattern
+    assert M(p, p, 8, 64, 5, 8, p, None, None) == 2          # unsupported pattern
     assert M(p, p, 8, 64, 2, 4, None, None, None) == 1       # totals required
     assert M(p + 8, p, 8, 64, 2, 4, p, None, None) == 1      # unaligned bitmap
     assert M(p, p, 8, 64, 2, 4, p, p + 2, None) == 1         # unaligned row counts

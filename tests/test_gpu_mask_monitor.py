@@ -21,7 +21,7 @@ def sbl():
 
 # K = 1024 (16-byte words), 96 (4-byte words), 48 (2-byte words); ragged row counts
 @pytest.mark.parametrize("O,K", [(333, 1024), (70, 96), (9, 48), (4864, 896), (1, 16)])
-@pytest.mark.parametrize("n,m", [(2, 4), (3, 4), (6, 8)])
+@pytest.mark.parametrize("n,m", [(2, 4), (3, 4), (6, 8), (4, 8)])
 def test_mask_monitor_random_bitmaps(sbl, O, K, n, m):
     rng = np.random.default_rng(O * 7 + K + n)
     a = rng.integers(0, 256, (O, K // 8), dtype=np.uint8)

@@ -13,7 +13,7 @@ from parity_util import (assert_bf16_close, assert_fp32_close, layer_inputs, ora
 
 pytestmark = pytest.mark.gpu
 
-PATTERNS = [(2, 4), (3, 4), (6, 8)]
+PATTERNS = [(2, 4), (3, 4), (6, 8), (4, 8)]
 
 
 @pytest.fixture(scope="module")
@@ -51,7 +51,7 @@ def test_prepare_bit_exact(sbl, n, m, O, K, seed):
 
 
 @pytest.mark.parametrize("n,m,O,K", [(3, 4, 4864, 896), (3, 4, 896, 4864), (2, 4, 7168, 2048),
-                                     (6, 8, 2048, 7168)])
+                                     (6, 8, 2048, 7168), (4, 8, 7168, 2048), (4, 8, 2048, 16384)])
 def test_prepare_bit_exact_full_layers(sbl, n, m, O, K):
     W, _, _ = layer_inputs(O, K, 1, seed=0)
     w = _prep(sbl, W, n, m)
@@ -132,6 +132,8 @@ LINEAR_CASES = [
     (130, 192, 17, 2, 4),
     (384, 896, 257, 3, 4),
     (896, 128, 1, 3, 4),
+    (256, 512, 33, 4, 8),
+    (640, 1024, 5, 4, 8),
 ]
 
 

@@ -31,7 +31,7 @@ import oracle
 from sparse_linear_layers_b200 import synthetic
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "worked_examples.json")
-PATTERNS = [(2, 4), (3, 4), (6, 8)]
+PATTERNS = [(2, 4), (3, 4), (6, 8), (4, 8)]
 
 
 def _cases():
