@@ -47,7 +47,7 @@ WORKLOAD = "qwen2.5-0.5b layer projections (q,k,v,o,gate,up,down), 3:4, prep + T
 # capture of this step's eager pass (dram__bytes_read.sum + dram__bytes_write.sum).
 # Only valid for the kernel sources the counters were taken on; reported as null
 # once those change.
-PREFILL_TRAFFIC = {"sources_sha256": "8c37b854e885afcdb1149611a5095429e4dbce19a7194b55bf9af2ecf46baf75", "bytes_per_call": 9617993}
+PREFILL_TRAFFIC = {"sources_sha256": "3de882157c1acbdd3fcad541e3734d9aac47022a5a87bba8ae24b637919ca1fa", "bytes_per_call": 9617920}
 
 
 def _kernel_sources_digest():
@@ -780,6 +780,9 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration sweep (profiling runs)")
+    ap.add_argument("--only", choices=("rmsnorm_front", "mask_monitor"),
+                    help="run only this auxiliary measurement on one GPU and print its JSON (profiling runs)")
+    ap.add_argument("--tokens", type=int, default=32768, help="tokens of the --only rmsnorm_front measurement")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -795,6 +798,13 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if args.only:
+        import sparse_linear_layers_b200 as sbl
+        hbm_peak = _peaks()[0]
+        res = (_rmsnorm_front(sbl, dev, hbm_peak, T=args.tokens) if args.only == "rmsnorm_front"
+               else _mask_monitor_bench(sbl, dev, hbm_peak))
+        print(json.dumps({"only": args.only, "result": res}), flush=True)
+        return
     if world > 1:
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
