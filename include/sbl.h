@@ -86,6 +86,20 @@ sbl_status sbl_prepare_weights(const float* W, int64_t O, int64_t K, int n, int 
                                void* stream);
 
 /*
+ * sbl_prepare_weights_ex — sbl_prepare_weights with convention flags.
+ *
+ *   flags  0, or SBL_PREP_SCALE_BF16: the row scale is stored as the halo
+ *          card's "Packed vs raw" format keeps it, one bf16 row_scale per row:
+ *          the fp32 scale above (after the 1e-5 clamp) is rounded to nearest
+ *          even bf16, and that value ternarises the row and is written to
+ *          row_scale (as fp32, exactly).  Other bits: SBL_ERR_INVALID_ARG.
+ */
+#define SBL_PREP_SCALE_BF16 1
+sbl_status sbl_prepare_weights_ex(const float* W, int64_t O, int64_t K, int n, int m,
+                                  uint8_t* packed, float* row_scale, uint8_t* mask_bits,
+                                  int flags, void* stream);
+
+/*
  * sbl_quant_act — per-token absmax int8 activation quantisation.
  *
  * Follows the activation equation of the Sparse-BitNet Guide, "Mathematical

@@ -6,4 +6,4 @@ baseline leg; never by the library itself.
 from .sbl_oracle import *  # noqa: F401,F403
 from .sbl_oracle import (SUPPORTED_NM, acc_entries, dequant, int_contract, linear, mask_monitor, nm_mask,  # noqa: F401
                          pack_codes, pack_mask_bits, prepare_weights, quant_act, rms_sumsq, rmsnorm,
-                         rmsnorm_quant_act, row_scale, ternarise, unpack_codes)
+                         rmsnorm_quant_act, round_to_bf16, row_scale, ternarise, unpack_codes)

@@ -139,10 +139,26 @@ def pack_mask_bits(mask: np.ndarray) -> np.ndarray:
     return out
 
 
-def prepare_weights(W: np.ndarray, n: int, m: int):
-    """Latent fp32 weights -> (packed uint8 [O,K/4], scale fp32 [O], mask bits uint8 [O,K/8], W_t int8 [O,K])."""
+def round_to_bf16(v: np.ndarray) -> np.ndarray:
+    """float32 values rounded to the nearest bf16 (ties to even), as float32.
+
+    The halo-sparse-bitnet-3:4-500m card, "What ships with this repo / Packed vs
+    raw": row_scale is stored as bf16.  bf16 keeps the top 16 bits of a float32;
+    round to nearest even on the dropped 16 (finite inputs)."""
+    b = np.asarray(v, np.float32).view(np.uint32).astype(np.uint64)
+    r = (b + 0x7FFF + ((b >> 16) & 1)) & 0xFFFF0000
+    return r.astype(np.uint32).view(np.float32)
+
+
+def prepare_weights(W: np.ndarray, n: int, m: int, scale_bf16: bool = False):
+    """Latent fp32 weights -> (packed uint8 [O,K/4], scale fp32 [O], mask bits uint8 [O,K/8], W_t int8 [O,K]).
+
+    With ``scale_bf16`` the row scale is rounded to bf16 (:func:`round_to_bf16`)
+    before it ternarises the row; the returned scale is that bf16 value."""
     mask = nm_mask(W, n, m)
     scale = row_scale(W, mask)
+    if scale_bf16:
+        scale = round_to_bf16(scale)
     Wt = ternarise(W, scale, mask)
     return pack_codes(Wt), scale, pack_mask_bits(mask), Wt
 

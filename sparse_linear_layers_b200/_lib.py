@@ -20,6 +20,8 @@ SBL_ERR_CUDA = 4
 SBL_ERR_TIMEOUT = 5
 SBL_ERR_WORKSPACE = 6
 
+SBL_PREP_SCALE_BF16 = 1
+
 SBL_F32 = 0
 SBL_BF16 = 1
 
@@ -35,6 +37,7 @@ _vp, _i64, _int, _sz, _u32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctyp
 _f32 = ctypes.c_float
 SIGNATURES = {
     "sbl_prepare_weights": (_int, [_vp, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp]),
+    "sbl_prepare_weights_ex": (_int, [_vp, _i64, _i64, _int, _int, _vp, _vp, _vp, _int, _vp]),
     "sbl_quant_act": (_int, [_vp, _i64, _i64, _vp, _vp, _vp]),
     "sbl_rmsnorm_quant_act": (_int, [_vp, _vp, _f32, _i64, _i64, _vp, _vp, _vp]),
     "sbl_linear_workspace_bytes": (_sz, [_i64, _i64, _i64, _int, _int]),

@@ -49,9 +49,10 @@ class PreparedWeights:
 
 
 def sbl_prepare_weights(W: torch.Tensor, n: int, m: int, with_mask: bool = False,
-                        out: Optional[PreparedWeights] = None,
+                        out: Optional[PreparedWeights] = None, scale_bf16: bool = False,
                         stream: Optional[torch.cuda.Stream] = None) -> PreparedWeights:
-    """N:M mask, per-row absmean scale, ternarise and pack (one kernel)."""
+    """N:M mask, per-row absmean scale, ternarise and pack (one kernel).  With
+    ``scale_bf16`` the scale is rounded to bf16 (the halo card's storage) first."""
     _need_cuda(W, "W", torch.float32)
     O, K = W.shape
     if out is None:
@@ -60,8 +61,9 @@ def sbl_prepare_weights(W: torch.Tensor, n: int, m: int, with_mask: bool = False
         mask = torch.empty((O, K // 8), dtype=torch.uint8, device=W.device) if with_mask else None
         out = PreparedWeights(packed, scale, n, m, K, mask)
     mb = out.mask_bits.data_ptr() if out.mask_bits is not None else None
-    check(lib.sbl_prepare_weights(W.data_ptr(), O, K, n, m, out.packed.data_ptr(), out.row_scale.data_ptr(), mb,
-                                  _stream(stream)), "sbl_prepare_weights")
+    check(lib.sbl_prepare_weights_ex(W.data_ptr(), O, K, n, m, out.packed.data_ptr(), out.row_scale.data_ptr(), mb,
+                                     _lib.SBL_PREP_SCALE_BF16 if scale_bf16 else 0, _stream(stream)),
+          "sbl_prepare_weights")
     return out
 
 

@@ -105,11 +105,18 @@ __device__ __forceinline__ void load_chunk(const float* p, uint32_t (&bits)[16])
     }
 }
 
+// The scale as the halo card stores it ("Packed vs raw": one bf16 row_scale per
+// row): round to nearest even bf16 when asked, before it ternarises the row.
+__device__ __forceinline__ float scale_storage(float sc, int scale_bf16) {
+    return scale_bf16 ? __bfloat162float(__float2bfloat16_rn(sc)) : sc;
+}
+
 template <int M>
 __global__ void __launch_bounds__(kPrepWarps * 32) prep_kernel(const float* __restrict__ W, long long O, long long K,
                                                                int n, uint8_t* __restrict__ packed,
                                                                float* __restrict__ row_scale,
-                                                               uint8_t* __restrict__ mask_bits, unsigned* status) {
+                                                               uint8_t* __restrict__ mask_bits, int scale_bf16,
+                                                               unsigned* status) {
     __shared__ unsigned long long limbs[kPrepWarps][kLimbs][32];
     __shared__ unsigned long long totals[kPrepWarps][kLimbs];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -156,7 +163,7 @@ __global__ void __launch_bounds__(kPrepWarps * 32) prep_kernel(const float* __re
         }
         const double sum = limbs_to_double(w);
         const double kept = static_cast<double>((K / M) * n);
-        scale = fmaxf(__double2float_rn(__ddiv_rn(sum, kept)), 1e-5f);
+        scale = scale_storage(fmaxf(__double2float_rn(__ddiv_rn(sum, kept)), 1e-5f), scale_bf16);
         row_scale[row] = scale;
     }
     scale = __shfl_sync(0xFFFFFFFFu, scale, 0);
@@ -237,7 +244,7 @@ __global__ void __launch_bounds__((8 / WPR) * WPR * 32) prep_kernel_rr(const flo
                                                                       long long K, uint8_t* __restrict__ packed,
                                                                       float* __restrict__ row_scale,
                                                                       uint8_t* __restrict__ mask_bits,
-                                                                      unsigned* status) {
+                                                                      int scale_bf16, unsigned* status) {
     constexpr int RPB = 8 / WPR;  // rows per block
     constexpr int TPR = WPR * 32;
     constexpr int CPT = kChunksPerThread;
@@ -385,14 +392,14 @@ __global__ void __launch_bounds__((8 / WPR) * WPR * 32) prep_kernel_rr(const flo
                 for (int w = 0; w < WPR; ++w) tot += wsum[sub * WPR + w];
                 sum = __ull2double_rn(tot) * __longlong_as_double(static_cast<long long>(1023 + eb - 150) << 52);
             }
-            sc = fmaxf(__double2float_rn(__ddiv_rn(sum, kept)), 1e-5f);
+            sc = scale_storage(fmaxf(__double2float_rn(__ddiv_rn(sum, kept)), 1e-5f), scale_bf16);
             scales[sub] = sc;
             if (valid) row_scale[row] = sc;
         }
         __syncthreads();
         sc = scales[sub];
     } else {
-        sc = fmaxf(__double2float_rn(__ddiv_rn(sum, kept)), 1e-5f);
+        sc = scale_storage(fmaxf(__double2float_rn(__ddiv_rn(sum, kept)), 1e-5f), scale_bf16);
         if (lane == 0 && valid) row_scale[row] = sc;
     }
     if (!valid) return;
@@ -421,44 +428,45 @@ __global__ void __launch_bounds__((8 / WPR) * WPR * 32) prep_kernel_rr(const flo
 
 template <int M, int N, int WPR>
 static void launch_prep_rr(const float* W, long long O, long long K, uint8_t* packed, float* row_scale,
-                           uint8_t* mask_bits, unsigned* status, cudaStream_t stream) {
+                           uint8_t* mask_bits, int scale_bf16, unsigned* status, cudaStream_t stream) {
     constexpr int RPB = 8 / WPR;
     const unsigned blocks = static_cast<unsigned>((O + RPB - 1) / RPB);
     if (mask_bits)
         prep_kernel_rr<M, N, WPR, true><<<blocks, RPB * WPR * 32, 0, stream>>>(W, O, K, packed, row_scale, mask_bits,
-                                                                              status);
+                                                                              scale_bf16, status);
     else
         prep_kernel_rr<M, N, WPR, false><<<blocks, RPB * WPR * 32, 0, stream>>>(W, O, K, packed, row_scale, nullptr,
-                                                                               status);
+                                                                               scale_bf16, status);
 }
 
 template <int M, int N>
 static void launch_prep_mn(const float* W, long long O, long long K, uint8_t* packed, float* row_scale,
-                           uint8_t* mask_bits, unsigned* status, cudaStream_t stream) {
+                           uint8_t* mask_bits, int scale_bf16, unsigned* status, cudaStream_t stream) {
     // warps per row: the fewest that give every 16-weight chunk a slot
     const long long wpr = ((K >> 4) + 32 * kChunksPerThread - 1) / (32 * kChunksPerThread);
     switch (wpr) {
-        case 1: launch_prep_rr<M, N, 1>(W, O, K, packed, row_scale, mask_bits, status, stream); break;
-        case 2: launch_prep_rr<M, N, 2>(W, O, K, packed, row_scale, mask_bits, status, stream); break;
-        case 3: launch_prep_rr<M, N, 3>(W, O, K, packed, row_scale, mask_bits, status, stream); break;
-        case 4: launch_prep_rr<M, N, 4>(W, O, K, packed, row_scale, mask_bits, status, stream); break;
-        case 5: launch_prep_rr<M, N, 5>(W, O, K, packed, row_scale, mask_bits, status, stream); break;
-        case 6: launch_prep_rr<M, N, 6>(W, O, K, packed, row_scale, mask_bits, status, stream); break;
-        case 7: launch_prep_rr<M, N, 7>(W, O, K, packed, row_scale, mask_bits, status, stream); break;
-        case 8: launch_prep_rr<M, N, 8>(W, O, K, packed, row_scale, mask_bits, status, stream); break;
+        case 1: launch_prep_rr<M, N, 1>(W, O, K, packed, row_scale, mask_bits, scale_bf16, status, stream); break;
+        case 2: launch_prep_rr<M, N, 2>(W, O, K, packed, row_scale, mask_bits, scale_bf16, status, stream); break;
+        case 3: launch_prep_rr<M, N, 3>(W, O, K, packed, row_scale, mask_bits, scale_bf16, status, stream); break;
+        case 4: launch_prep_rr<M, N, 4>(W, O, K, packed, row_scale, mask_bits, scale_bf16, status, stream); break;
+        case 5: launch_prep_rr<M, N, 5>(W, O, K, packed, row_scale, mask_bits, scale_bf16, status, stream); break;
+        case 6: launch_prep_rr<M, N, 6>(W, O, K, packed, row_scale, mask_bits, scale_bf16, status, stream); break;
+        case 7: launch_prep_rr<M, N, 7>(W, O, K, packed, row_scale, mask_bits, scale_bf16, status, stream); break;
+        case 8: launch_prep_rr<M, N, 8>(W, O, K, packed, row_scale, mask_bits, scale_bf16, status, stream); break;
         default: {
             const unsigned blocks = static_cast<unsigned>((O + kPrepWarps - 1) / kPrepWarps);
-            prep_kernel<M><<<blocks, kPrepWarps * 32, 0, stream>>>(W, O, K, N, packed, row_scale, mask_bits, status);
+            prep_kernel<M><<<blocks, kPrepWarps * 32, 0, stream>>>(W, O, K, N, packed, row_scale, mask_bits,
+                                                                   scale_bf16, status);
         }
     }
 }
 
 cudaError_t launch_prep(const float* W, long long O, long long K, int n, int m, uint8_t* packed, float* row_scale,
-                        uint8_t* mask_bits, unsigned* status, cudaStream_t stream) {
-    if (m == 4 && n == 2) launch_prep_mn<4, 2>(W, O, K, packed, row_scale, mask_bits, status, stream);
-    else if (m == 4) launch_prep_mn<4, 3>(W, O, K, packed, row_scale, mask_bits, status, stream);
-    else if (n == 4) launch_prep_mn<8, 4>(W, O, K, packed, row_scale, mask_bits, status, stream);
-    else launch_prep_mn<8, 6>(W, O, K, packed, row_scale, mask_bits, status, stream);
+                        uint8_t* mask_bits, int scale_bf16, unsigned* status, cudaStream_t stream) {
+    if (m == 4 && n == 2) launch_prep_mn<4, 2>(W, O, K, packed, row_scale, mask_bits, scale_bf16, status, stream);
+    else if (m == 4) launch_prep_mn<4, 3>(W, O, K, packed, row_scale, mask_bits, scale_bf16, status, stream);
+    else if (n == 4) launch_prep_mn<8, 4>(W, O, K, packed, row_scale, mask_bits, scale_bf16, status, stream);
+    else launch_prep_mn<8, 6>(W, O, K, packed, row_scale, mask_bits, scale_bf16, status, stream);
     return cudaGetLastError();
 }
 

@@ -10,7 +10,7 @@
 
 namespace sbl {
 cudaError_t launch_prep(const float* W, long long O, long long K, int n, int m, uint8_t* packed, float* row_scale,
-                        uint8_t* mask_bits, unsigned* status, cudaStream_t stream);
+                        uint8_t* mask_bits, int scale_bf16, unsigned* status, cudaStream_t stream);
 cudaError_t launch_quant(const uint16_t* x, long long T, long long K, int8_t* xq, float* s_tok, int layout,
                          unsigned* status, cudaStream_t stream, void* zero16 = nullptr, long long nzero16 = 0);
 constexpr int kLayoutNatural = 0, kLayoutPairs = 1;
@@ -111,7 +111,13 @@ extern "C" {
 
 sbl_status sbl_prepare_weights(const float* W, int64_t O, int64_t K, int n, int m, uint8_t* packed,
                                float* row_scale, uint8_t* mask_bits, void* stream) {
+    return sbl_prepare_weights_ex(W, O, K, n, m, packed, row_scale, mask_bits, 0, stream);
+}
+
+sbl_status sbl_prepare_weights_ex(const float* W, int64_t O, int64_t K, int n, int m, uint8_t* packed,
+                                  float* row_scale, uint8_t* mask_bits, int flags, void* stream) {
     if (O < 0) return SBL_ERR_INVALID_ARG;
+    if (flags & ~SBL_PREP_SCALE_BF16) return SBL_ERR_INVALID_ARG;
     if (sbl_status s = check_k(K)) return s;
     if (!nm_ok(n, m)) return SBL_ERR_UNSUPPORTED;
     if (O == 0) return SBL_OK;
@@ -121,7 +127,8 @@ sbl_status sbl_prepare_weights(const float* W, int64_t O, int64_t K, int n, int 
     if (O > (1ll << 31) - 1) return SBL_ERR_UNSUPPORTED;
     DeviceInfo* d;
     if (sbl_status s = device_info(&d)) return s;
-    return from_cuda(sbl::launch_prep(W, O, K, n, m, packed, row_scale, mask_bits, d->status,
+    return from_cuda(sbl::launch_prep(W, O, K, n, m, packed, row_scale, mask_bits,
+                                      (flags & SBL_PREP_SCALE_BF16) ? 1 : 0, d->status,
                                       static_cast<cudaStream_t>(stream)));
 }
 

@@ -61,6 +61,13 @@ def test_prepare_rejects_on_host(args, code):
     assert lib.sbl_prepare_weights(None, O, K, n, m, None, None, None, None) == code
 
 
+def test_prepare_ex_rejects_unknown_flags():
+    from sparse_linear_layers_b200._lib import lib
+    p = 4096
+    assert lib.sbl_prepare_weights_ex(p, 8, 64, 2, 4, p, p, None, 2, None) == 1
+    assert lib.sbl_prepare_weights_ex(p, 8, 64, 2, 4, p, p, None, -1, None) == 1
+
+
 def test_zero_sizes_are_noops_without_a_device():
     from sparse_linear_layers_b200._lib import lib
     assert lib.sbl_prepare_weights(None, 0, 64, 2, 4, None, None, None, None) == 0

@@ -441,3 +441,21 @@ def test_linear_plan(sbl):
     with pytest.raises(SblError) as e:
         sbl.sbl_linear_plan(64, 256, 128, 1, 4)
     assert e.value.code == SBL_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("n,m", PATTERNS)
+@pytest.mark.parametrize("O,K", [(300, 896), (64, 16384)])
+def test_prepare_scale_bf16(sbl, n, m, O, K):
+    """bf16 scale storage: the rounded scale ternarises the row; both prep
+    kernels (rows held in registers, and the long-row kernel) bit-exact."""
+    W, xbits, xval = layer_inputs(O, K, 5, seed=7)
+    packed, scale, mbits, Wt = oracle.prepare_weights(W, n, m, scale_bf16=True)
+    w = sbl.sbl_prepare_weights(to_dev(W), n, m, with_mask=True, scale_bf16=True)
+    assert sbl.sbl_device_status() == 0
+    assert np.array_equal(w.packed.cpu().numpy(), packed)
+    assert np.array_equal(w.row_scale.cpu().numpy().view(np.uint32), scale.view(np.uint32))
+    assert np.array_equal(w.mask_bits.cpu().numpy(), mbits)
+    y_ref, acc_ref, _, _ = oracle.linear(xval, Wt, scale)
+    y, acc = _run_linear(sbl, w, xbits, 5, O, "auto")
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    assert_fp32_close(y.cpu().numpy(), y_ref)

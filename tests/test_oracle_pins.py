@@ -611,3 +611,39 @@ def test_planted_mask_monitor_mistake_is_caught(name, fn):
     o = types.SimpleNamespace(mask_monitor=fn)
     with pytest.raises(AssertionError):
         pin_mask_monitor(o)
+
+
+# --------------------------------------------------------------------------
+# bf16 scale storage (the halo card keeps one bf16 row_scale per row)
+# --------------------------------------------------------------------------
+
+def pin_scale_bf16(o):
+    """The rounding agrees with torch's float32 -> bfloat16 conversion (a library
+    routine, round to nearest even) on random values and on exact ties; the
+    weights are ternarised with the rounded scale (|w| > s/2 on kept weights)."""
+    import torch
+    v = np.random.default_rng(12).uniform(1e-6, 1.0, 4096).astype(np.float32)
+    ties = (np.array([0x3F808000, 0x3F818000, 0x3F80FFFF, 0x3F807FFF], np.uint32)).view(np.float32)
+    for a in (v, ties):
+        ref = torch.from_numpy(a).to(torch.bfloat16).float().numpy()
+        assert np.array_equal(o.round_to_bf16(a).view(np.uint32), ref.view(np.uint32))
+    for n, m in PATTERNS:
+        W = synthetic.latent_weights(16, 64, seed=9)
+        _, s32, _, _ = o.prepare_weights(W, n, m)
+        _, s16, mb, Wt = o.prepare_weights(W, n, m, scale_bf16=True)
+        assert np.array_equal(s16.view(np.uint32), torch.from_numpy(s32).to(torch.bfloat16).float().numpy().view(np.uint32))
+        keep = np.unpackbits(mb, axis=1, bitorder="little")[:, :64].astype(bool)
+        expect = np.where(keep & (np.abs(W) > np.float32(0.5) * s16[:, None]), np.sign(W), 0).astype(np.int8)
+        assert np.array_equal(Wt, expect)
+
+
+def test_scale_bf16_pins():
+    pin_scale_bf16(oracle)
+
+
+def test_planted_scale_bf16_truncation_is_caught():
+    def trunc(v):
+        return (np.asarray(v, np.float32).view(np.uint32) & np.uint32(0xFFFF0000)).view(np.float32)
+    o = types.SimpleNamespace(round_to_bf16=trunc, prepare_weights=oracle.prepare_weights)
+    with pytest.raises(AssertionError):
+        pin_scale_bf16(o)
