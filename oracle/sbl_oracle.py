@@ -150,13 +150,27 @@ def round_to_bf16(v: np.ndarray) -> np.ndarray:
     return r.astype(np.uint32).view(np.float32)
 
 
-def prepare_weights(W: np.ndarray, n: int, m: int, scale_bf16: bool = False):
+def global_scale(W: np.ndarray) -> np.float32:
+    """One scale for the whole matrix: mean of |W| over all O*K weights, masked
+    ones included, clamped below at 1e-5 — the gamma of the Sparse-BitNet
+    Guide's module listing (``torch.mean(torch.abs(weight)).clamp(min=1e-5)``).
+    The sum is exact up to one final rounding to double (``math.fsum``)."""
+    a = np.abs(np.asarray(W, dtype=np.float32)).astype(np.float64).ravel()
+    mean = math.fsum(a.tolist()) / float(a.size)
+    return max(np.float32(mean), EPS_SCALE)
+
+
+def prepare_weights(W: np.ndarray, n: int, m: int, scale_bf16: bool = False, scale_global: bool = False):
     """Latent fp32 weights -> (packed uint8 [O,K/4], scale fp32 [O], mask bits uint8 [O,K/8], W_t int8 [O,K]).
 
     With ``scale_bf16`` the row scale is rounded to bf16 (:func:`round_to_bf16`)
-    before it ternarises the row; the returned scale is that bf16 value."""
+    before it ternarises the row; the returned scale is that bf16 value.  With
+    ``scale_global`` every row takes :func:`global_scale` instead."""
     mask = nm_mask(W, n, m)
-    scale = row_scale(W, mask)
+    if scale_global:
+        scale = np.full(np.asarray(W).shape[0], global_scale(W), dtype=np.float32)
+    else:
+        scale = row_scale(W, mask)
     if scale_bf16:
         scale = round_to_bf16(scale)
     Wt = ternarise(W, scale, mask)

@@ -19,6 +19,7 @@ flip) is planted in a copy of the oracle at the end of this file, and some pin
 below must reject it.
 """
 import itertools
+import math
 import json
 import os
 import types
@@ -647,3 +648,63 @@ def test_planted_scale_bf16_truncation_is_caught():
     o = types.SimpleNamespace(round_to_bf16=trunc, prepare_weights=oracle.prepare_weights)
     with pytest.raises(AssertionError):
         pin_scale_bf16(o)
+
+
+# --------------------------------------------------------------------------
+# global scale (the guide's module listing: one mean |W| over the whole matrix)
+# --------------------------------------------------------------------------
+
+def pin_global_scale(o):
+    """Exact rational mean (fractions) on small matrices, including values whose
+    float sum would lose low bits; torch's float64 mean of |W| agrees within
+    rounding; the weights are ternarised with that single scale."""
+    import torch
+    rng = np.random.default_rng(21)
+    for O, K in ((3, 16), (8, 64), (5, 48)):
+        W = (rng.standard_normal((O, K)) * 0.02).astype(np.float32)
+        W[0, 0] = np.float32(3.0e7)       # a huge and a tiny weight in one sum
+        W[1, 3] = np.float32(1.0e-30)
+        exact = sum((Fraction(float(abs(v))) for v in W.ravel()), Fraction(0))
+        want = max(np.float32(float(exact) / float(O * K)), np.float32(1e-5))
+        assert o.global_scale(W) == want
+        ref = float(torch.from_numpy(np.abs(W).astype(np.float64)).mean())
+        assert abs(float(o.global_scale(W)) - ref) <= 1e-6 * ref
+        for n, m in PATTERNS:
+            _, s, mb, Wt = o.prepare_weights(W, n, m, scale_global=True)
+            assert np.all(s == want)
+            keep = np.unpackbits(mb, axis=1, bitorder="little")[:, :K].astype(bool)
+            expect = np.where(keep & (np.abs(W) > np.float32(0.5) * want), np.sign(W), 0).astype(np.int8)
+            assert np.array_equal(Wt, expect)
+    tiny = np.full((2, 16), 1e-9, np.float32)
+    assert o.global_scale(tiny) == np.float32(1e-5)  # the clamp
+
+
+def test_global_scale_pins():
+    pin_global_scale(oracle)
+
+
+@pytest.mark.parametrize("name", ["kept_only", "divided_by_kept_count", "float32_sum"])
+def test_planted_global_scale_mistake_is_caught(name):
+    def kept_only(W):
+        mask = oracle.nm_mask(W, 2, 4)
+        a = np.abs(W[mask]).astype(np.float64)
+        return max(np.float32(math.fsum(a.tolist()) / a.size), np.float32(1e-5))
+
+    def divided_by_kept_count(W):
+        tot = math.fsum(np.abs(W).astype(np.float64).ravel().tolist())
+        return max(np.float32(tot / (W.size // 2)), np.float32(1e-5))
+
+    def float32_sum(W):
+        return max(np.float32(np.sum(np.abs(W), dtype=np.float32) / np.float32(W.size)), np.float32(1e-5))
+
+    fn = {"kept_only": kept_only, "divided_by_kept_count": divided_by_kept_count, "float32_sum": float32_sum}[name]
+
+    def prep(W, n, m, scale_global=False):
+        mask = oracle.nm_mask(W, n, m)
+        scale = np.full(W.shape[0], fn(W), np.float32)
+        Wt = oracle.ternarise(W, scale, mask)
+        return oracle.pack_codes(Wt), scale, oracle.pack_mask_bits(mask), Wt
+
+    o = types.SimpleNamespace(global_scale=fn, prepare_weights=prep)
+    with pytest.raises(AssertionError):
+        pin_global_scale(o)
