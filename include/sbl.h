@@ -92,9 +92,19 @@ sbl_status sbl_prepare_weights(const float* W, int64_t O, int64_t K, int n, int 
  *          card's "Packed vs raw" format keeps it, one bf16 row_scale per row:
  *          the fp32 scale above (after the 1e-5 clamp) is rounded to nearest
  *          even bf16, and that value ternarises the row and is written to
- *          row_scale (as fp32, exactly).  Other bits: SBL_ERR_INVALID_ARG.
+ *          row_scale (as fp32, exactly).
+ *          SBL_PREP_SCALE_GLOBAL: one scale for the whole matrix, as the
+ *          Sparse-BitNet Guide's module listing computes gamma: the mean of |W|
+ *          over all O*K weights (masked ones included) — the exact sum rounded
+ *          once to double, divided by O*K in double, rounded to float, clamped
+ *          below at 1e-5 (then rounded to bf16 with SBL_PREP_SCALE_BF16) — used
+ *          for every row and written to every row_scale entry.  Needs
+ *          O*K < 2^32 (else SBL_ERR_UNSUPPORTED); calls with this flag on one
+ *          device must be ordered, as they share a small static scratch.
+ *          Other bits: SBL_ERR_INVALID_ARG.
  */
 #define SBL_PREP_SCALE_BF16 1
+#define SBL_PREP_SCALE_GLOBAL 2
 sbl_status sbl_prepare_weights_ex(const float* W, int64_t O, int64_t K, int n, int m,
                                   uint8_t* packed, float* row_scale, uint8_t* mask_bits,
                                   int flags, void* stream);

@@ -21,6 +21,7 @@ SBL_ERR_TIMEOUT = 5
 SBL_ERR_WORKSPACE = 6
 
 SBL_PREP_SCALE_BF16 = 1
+SBL_PREP_SCALE_GLOBAL = 2
 
 SBL_F32 = 0
 SBL_BF16 = 1

@@ -50,9 +50,12 @@ class PreparedWeights:
 
 def sbl_prepare_weights(W: torch.Tensor, n: int, m: int, with_mask: bool = False,
                         out: Optional[PreparedWeights] = None, scale_bf16: bool = False,
+                        scale_global: bool = False,
                         stream: Optional[torch.cuda.Stream] = None) -> PreparedWeights:
     """N:M mask, per-row absmean scale, ternarise and pack (one kernel).  With
-    ``scale_bf16`` the scale is rounded to bf16 (the halo card's storage) first."""
+    ``scale_bf16`` the scale is rounded to bf16 (the halo card's storage) first;
+    with ``scale_global`` one scale, the mean of |W| over the whole matrix (the
+    guide's module listing), serves every row."""
     _need_cuda(W, "W", torch.float32)
     O, K = W.shape
     if out is None:
@@ -62,7 +65,8 @@ def sbl_prepare_weights(W: torch.Tensor, n: int, m: int, with_mask: bool = False
         out = PreparedWeights(packed, scale, n, m, K, mask)
     mb = out.mask_bits.data_ptr() if out.mask_bits is not None else None
     check(lib.sbl_prepare_weights_ex(W.data_ptr(), O, K, n, m, out.packed.data_ptr(), out.row_scale.data_ptr(), mb,
-                                     _lib.SBL_PREP_SCALE_BF16 if scale_bf16 else 0, _stream(stream)),
+                                     (_lib.SBL_PREP_SCALE_BF16 if scale_bf16 else 0) |
+                                     (_lib.SBL_PREP_SCALE_GLOBAL if scale_global else 0), _stream(stream)),
           "sbl_prepare_weights")
     return out
 

@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(kPrepWarps * 32) prep_kernel(const float* __re
                                                                int n, uint8_t* __restrict__ packed,
                                                                float* __restrict__ row_scale,
                                                                uint8_t* __restrict__ mask_bits, int scale_bf16,
-                                                               unsigned* status) {
+                                                               const float* __restrict__ ext_scale, unsigned* status) {
     __shared__ unsigned long long limbs[kPrepWarps][kLimbs][32];
     __shared__ unsigned long long totals[kPrepWarps][kLimbs];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(kPrepWarps * 32) prep_kernel(const float* __re
         }
         const double sum = limbs_to_double(w);
         const double kept = static_cast<double>((K / M) * n);
-        scale = scale_storage(fmaxf(__double2float_rn(__ddiv_rn(sum, kept)), 1e-5f), scale_bf16);
+        scale = ext_scale ? *ext_scale : scale_storage(fmaxf(__double2float_rn(__ddiv_rn(sum, kept)), 1e-5f), scale_bf16);
         row_scale[row] = scale;
     }
     scale = __shfl_sync(0xFFFFFFFFu, scale, 0);
@@ -244,7 +244,8 @@ __global__ void __launch_bounds__((8 / WPR) * WPR * 32) prep_kernel_rr(const flo
                                                                       long long K, uint8_t* __restrict__ packed,
                                                                       float* __restrict__ row_scale,
                                                                       uint8_t* __restrict__ mask_bits,
-                                                                      int scale_bf16, unsigned* status) {
+                                                                      int scale_bf16, const float* __restrict__ ext_scale,
+                                                                      unsigned* status) {
     constexpr int RPB = 8 / WPR;  // rows per block
     constexpr int TPR = WPR * 32;
     constexpr int CPT = kChunksPerThread;
@@ -392,14 +393,14 @@ __global__ void __launch_bounds__((8 / WPR) * WPR * 32) prep_kernel_rr(const flo
                 for (int w = 0; w < WPR; ++w) tot += wsum[sub * WPR + w];
                 sum = __ull2double_rn(tot) * __longlong_as_double(static_cast<long long>(1023 + eb - 150) << 52);
             }
-            sc = scale_storage(fmaxf(__double2float_rn(__ddiv_rn(sum, kept)), 1e-5f), scale_bf16);
+            sc = ext_scale ? *ext_scale : scale_storage(fmaxf(__double2float_rn(__ddiv_rn(sum, kept)), 1e-5f), scale_bf16);
             scales[sub] = sc;
             if (valid) row_scale[row] = sc;
         }
         __syncthreads();
         sc = scales[sub];
     } else {
-        sc = scale_storage(fmaxf(__double2float_rn(__ddiv_rn(sum, kept)), 1e-5f), scale_bf16);
+        sc = ext_scale ? *ext_scale : scale_storage(fmaxf(__double2float_rn(__ddiv_rn(sum, kept)), 1e-5f), scale_bf16);
         if (lane == 0 && valid) row_scale[row] = sc;
     }
     if (!valid) return;
@@ -428,45 +429,122 @@ __global__ void __launch_bounds__((8 / WPR) * WPR * 32) prep_kernel_rr(const flo
 
 template <int M, int N, int WPR>
 static void launch_prep_rr(const float* W, long long O, long long K, uint8_t* packed, float* row_scale,
-                           uint8_t* mask_bits, int scale_bf16, unsigned* status, cudaStream_t stream) {
+                           uint8_t* mask_bits, int scale_bf16, const float* ext_scale, unsigned* status,
+                           cudaStream_t stream) {
     constexpr int RPB = 8 / WPR;
     const unsigned blocks = static_cast<unsigned>((O + RPB - 1) / RPB);
     if (mask_bits)
         prep_kernel_rr<M, N, WPR, true><<<blocks, RPB * WPR * 32, 0, stream>>>(W, O, K, packed, row_scale, mask_bits,
-                                                                              scale_bf16, status);
+                                                                              scale_bf16, ext_scale, status);
     else
         prep_kernel_rr<M, N, WPR, false><<<blocks, RPB * WPR * 32, 0, stream>>>(W, O, K, packed, row_scale, nullptr,
-                                                                               scale_bf16, status);
+                                                                               scale_bf16, ext_scale, status);
 }
 
 template <int M, int N>
 static void launch_prep_mn(const float* W, long long O, long long K, uint8_t* packed, float* row_scale,
-                           uint8_t* mask_bits, int scale_bf16, unsigned* status, cudaStream_t stream) {
+                           uint8_t* mask_bits, int scale_bf16, const float* ext_scale, unsigned* status,
+                           cudaStream_t stream) {
     // warps per row: the fewest that give every 16-weight chunk a slot
     const long long wpr = ((K >> 4) + 32 * kChunksPerThread - 1) / (32 * kChunksPerThread);
     switch (wpr) {
-        case 1: launch_prep_rr<M, N, 1>(W, O, K, packed, row_scale, mask_bits, scale_bf16, status, stream); break;
-        case 2: launch_prep_rr<M, N, 2>(W, O, K, packed, row_scale, mask_bits, scale_bf16, status, stream); break;
-        case 3: launch_prep_rr<M, N, 3>(W, O, K, packed, row_scale, mask_bits, scale_bf16, status, stream); break;
-        case 4: launch_prep_rr<M, N, 4>(W, O, K, packed, row_scale, mask_bits, scale_bf16, status, stream); break;
-        case 5: launch_prep_rr<M, N, 5>(W, O, K, packed, row_scale, mask_bits, scale_bf16, status, stream); break;
-        case 6: launch_prep_rr<M, N, 6>(W, O, K, packed, row_scale, mask_bits, scale_bf16, status, stream); break;
-        case 7: launch_prep_rr<M, N, 7>(W, O, K, packed, row_scale, mask_bits, scale_bf16, status, stream); break;
-        case 8: launch_prep_rr<M, N, 8>(W, O, K, packed, row_scale, mask_bits, scale_bf16, status, stream); break;
+        case 1: launch_prep_rr<M, N, 1>(W, O, K, packed, row_scale, mask_bits, scale_bf16, ext_scale, status, stream); break;
+        case 2: launch_prep_rr<M, N, 2>(W, O, K, packed, row_scale, mask_bits, scale_bf16, ext_scale, status, stream); break;
+        case 3: launch_prep_rr<M, N, 3>(W, O, K, packed, row_scale, mask_bits, scale_bf16, ext_scale, status, stream); break;
+        case 4: launch_prep_rr<M, N, 4>(W, O, K, packed, row_scale, mask_bits, scale_bf16, ext_scale, status, stream); break;
+        case 5: launch_prep_rr<M, N, 5>(W, O, K, packed, row_scale, mask_bits, scale_bf16, ext_scale, status, stream); break;
+        case 6: launch_prep_rr<M, N, 6>(W, O, K, packed, row_scale, mask_bits, scale_bf16, ext_scale, status, stream); break;
+        case 7: launch_prep_rr<M, N, 7>(W, O, K, packed, row_scale, mask_bits, scale_bf16, ext_scale, status, stream); break;
+        case 8: launch_prep_rr<M, N, 8>(W, O, K, packed, row_scale, mask_bits, scale_bf16, ext_scale, status, stream); break;
         default: {
             const unsigned blocks = static_cast<unsigned>((O + kPrepWarps - 1) / kPrepWarps);
             prep_kernel<M><<<blocks, kPrepWarps * 32, 0, stream>>>(W, O, K, N, packed, row_scale, mask_bits,
-                                                                   scale_bf16, status);
+                                                                   scale_bf16, ext_scale, status);
         }
     }
 }
 
+// ---------------------------------------------------------------- global scale
+// The guide's module listing takes one scale for the whole matrix, the mean of
+// |W| over every weight (masked ones included).  The sum is formed exactly with
+// the limb columns above: every warp adds its share into per-lane columns in
+// shared memory, sums its lanes and adds the ten column totals to global
+// columns (64-bit atomics; a column stays below 2^64 while O * K < 2^32).  A
+// single thread then resolves the carries, rounds once to double, divides by
+// O * K in double and rounds to float, clamps at 1e-5 and, if asked, rounds to
+// bf16.  The ternarisation kernels then read that scale instead of their own.
+__global__ void __launch_bounds__(kPrepWarps * 32) abs_sum_kernel(const float* __restrict__ W, long long total,
+                                                                  unsigned long long* __restrict__ cols,
+                                                                  unsigned* status) {
+    __shared__ unsigned long long limbs[kPrepWarps][kLimbs][32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    unsigned long long* my = &limbs[warp][0][lane];
+#pragma unroll
+    for (int l = 0; l < kLimbs; ++l) my[l * 32] = 0ull;
+    bool bad = false;
+    const long long nvec = total >> 2;  // K % 16 == 0, so whole float4 vectors
+    const uint4* w4 = reinterpret_cast<const uint4*>(W);
+    for (long long v = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; v < nvec;
+         v += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const uint4 q = ldg_nc(w4 + v);
+        const uint32_t a[4] = {q.x & 0x7FFFFFFFu, q.y & 0x7FFFFFFFu, q.z & 0x7FFFFFFFu, q.w & 0x7FFFFFFFu};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            bad |= a[i] >= 0x7F800000u;
+            if (a[i] < 0x7F800000u) exact_add(my, a[i]);
+        }
+    }
+    if (bad) raise_status(status, kStatusNonfinite);
+    __syncwarp();
+    if (lane < kLimbs) {
+        unsigned long long s = 0;
+        for (int i = 0; i < 32; ++i) s += limbs[warp][lane][i];
+        if (s) atomicAdd(cols + lane, s);
+    }
+}
+
+__global__ void gamma_finalize_kernel(const unsigned long long* __restrict__ cols, long long total, int scale_bf16,
+                                      float* __restrict__ gamma) {
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    uint32_t w[kLimbs];
+    unsigned long long carry = 0;
+#pragma unroll
+    for (int i = 0; i < kLimbs; ++i) {
+        const unsigned long long lo = cols[i] & 0xFFFFFFFFull, hi = cols[i] >> 32;
+        const unsigned long long t = lo + carry;
+        w[i] = static_cast<uint32_t>(t);
+        carry = (t >> 32) + hi;
+    }
+    const double sum = limbs_to_double(w);
+    *gamma = scale_storage(fmaxf(__double2float_rn(__ddiv_rn(sum, static_cast<double>(total))), 1e-5f), scale_bf16);
+}
+
+// Per-device scratch of the global-scale path: ten columns and the scale.  Calls
+// that use it on one device must be ordered (one stream, or synchronised).
+__device__ unsigned long long g_gamma_cols[kLimbs];
+__device__ float g_gamma;
+
 cudaError_t launch_prep(const float* W, long long O, long long K, int n, int m, uint8_t* packed, float* row_scale,
-                        uint8_t* mask_bits, int scale_bf16, unsigned* status, cudaStream_t stream) {
-    if (m == 4 && n == 2) launch_prep_mn<4, 2>(W, O, K, packed, row_scale, mask_bits, scale_bf16, status, stream);
-    else if (m == 4) launch_prep_mn<4, 3>(W, O, K, packed, row_scale, mask_bits, scale_bf16, status, stream);
-    else if (n == 4) launch_prep_mn<8, 4>(W, O, K, packed, row_scale, mask_bits, scale_bf16, status, stream);
-    else launch_prep_mn<8, 6>(W, O, K, packed, row_scale, mask_bits, scale_bf16, status, stream);
+                        uint8_t* mask_bits, int scale_bf16, int scale_global, unsigned* status, cudaStream_t stream) {
+    const float* ext = nullptr;
+    if (scale_global) {
+        unsigned long long* cols = nullptr;
+        float* gamma = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&cols), g_gamma_cols);
+        if (e == cudaSuccess) e = cudaGetSymbolAddress(reinterpret_cast<void**>(&gamma), g_gamma);
+        if (e == cudaSuccess) e = cudaMemsetAsync(cols, 0, sizeof(unsigned long long) * kLimbs, stream);
+        if (e != cudaSuccess) return e;
+        const long long total = O * K;
+        long long blocks = (total / 4 + kPrepWarps * 32 - 1) / (kPrepWarps * 32);
+        if (blocks > 4096) blocks = 4096;
+        abs_sum_kernel<<<static_cast<unsigned>(blocks), kPrepWarps * 32, 0, stream>>>(W, total, cols, status);
+        gamma_finalize_kernel<<<1, 32, 0, stream>>>(cols, total, scale_bf16, gamma);
+        ext = gamma;
+    }
+    if (m == 4 && n == 2) launch_prep_mn<4, 2>(W, O, K, packed, row_scale, mask_bits, scale_bf16, ext, status, stream);
+    else if (m == 4) launch_prep_mn<4, 3>(W, O, K, packed, row_scale, mask_bits, scale_bf16, ext, status, stream);
+    else if (n == 4) launch_prep_mn<8, 4>(W, O, K, packed, row_scale, mask_bits, scale_bf16, ext, status, stream);
+    else launch_prep_mn<8, 6>(W, O, K, packed, row_scale, mask_bits, scale_bf16, ext, status, stream);
     return cudaGetLastError();
 }
 

@@ -10,7 +10,8 @@
 
 namespace sbl {
 cudaError_t launch_prep(const float* W, long long O, long long K, int n, int m, uint8_t* packed, float* row_scale,
-                        uint8_t* mask_bits, int scale_bf16, unsigned* status, cudaStream_t stream);
+                        uint8_t* mask_bits, int scale_bf16, int scale_global, unsigned* status,
+                        cudaStream_t stream);
 cudaError_t launch_quant(const uint16_t* x, long long T, long long K, int8_t* xq, float* s_tok, int layout,
                          unsigned* status, cudaStream_t stream, void* zero16 = nullptr, long long nzero16 = 0);
 constexpr int kLayoutNatural = 0, kLayoutPairs = 1;
@@ -117,7 +118,8 @@ sbl_status sbl_prepare_weights(const float* W, int64_t O, int64_t K, int n, int 
 sbl_status sbl_prepare_weights_ex(const float* W, int64_t O, int64_t K, int n, int m, uint8_t* packed,
                                   float* row_scale, uint8_t* mask_bits, int flags, void* stream) {
     if (O < 0) return SBL_ERR_INVALID_ARG;
-    if (flags & ~SBL_PREP_SCALE_BF16) return SBL_ERR_INVALID_ARG;
+    if (flags & ~(SBL_PREP_SCALE_BF16 | SBL_PREP_SCALE_GLOBAL)) return SBL_ERR_INVALID_ARG;
+    if ((flags & SBL_PREP_SCALE_GLOBAL) && O * K >= (1ll << 32)) return SBL_ERR_UNSUPPORTED;
     if (sbl_status s = check_k(K)) return s;
     if (!nm_ok(n, m)) return SBL_ERR_UNSUPPORTED;
     if (O == 0) return SBL_OK;
@@ -128,7 +130,8 @@ sbl_status sbl_prepare_weights_ex(const float* W, int64_t O, int64_t K, int n, i
     DeviceInfo* d;
     if (sbl_status s = device_info(&d)) return s;
     return from_cuda(sbl::launch_prep(W, O, K, n, m, packed, row_scale, mask_bits,
-                                      (flags & SBL_PREP_SCALE_BF16) ? 1 : 0, d->status,
+                                      (flags & SBL_PREP_SCALE_BF16) ? 1 : 0, (flags & SBL_PREP_SCALE_GLOBAL) ? 1 : 0,
+                                      d->status,
                                       static_cast<cudaStream_t>(stream)));
 }
 

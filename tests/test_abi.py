@@ -64,8 +64,9 @@ def test_prepare_rejects_on_host(args, code):
 def test_prepare_ex_rejects_unknown_flags():
     from sparse_linear_layers_b200._lib import lib
     p = 4096
-    assert lib.sbl_prepare_weights_ex(p, 8, 64, 2, 4, p, p, None, 2, None) == 1
+    assert lib.sbl_prepare_weights_ex(p, 8, 64, 2, 4, p, p, None, 4, None) == 1
     assert lib.sbl_prepare_weights_ex(p, 8, 64, 2, 4, p, p, None, -1, None) == 1
+    assert lib.sbl_prepare_weights_ex(p, 1 << 20, 4096, 2, 4, p, p, None, 2, None) == 2  # global scale: O*K >= 2^32
 
 
 def test_zero_sizes_are_noops_without_a_device():

@@ -459,3 +459,25 @@ def test_prepare_scale_bf16(sbl, n, m, O, K):
     y, acc = _run_linear(sbl, w, xbits, 5, O, "auto")
     assert np.array_equal(acc.cpu().numpy(), acc_ref)
     assert_fp32_close(y.cpu().numpy(), y_ref)
+
+
+@pytest.mark.parametrize("n,m", PATTERNS)
+@pytest.mark.parametrize("O,K", [(300, 896), (64, 16384)])
+@pytest.mark.parametrize("bf16", [False, True])
+def test_prepare_scale_global(sbl, n, m, O, K, bf16):
+    """The guide listing's single scale: the exact mean of |W| over the matrix
+    (a huge and a tiny weight included), bit-exact, in both prep kernels."""
+    W, xbits, xval = layer_inputs(O, K, 3, seed=9)
+    W = W.copy()
+    W[0, 5] = np.float32(2.5e6)
+    W[O - 1, K - 1] = np.float32(3.0e-33)
+    packed, scale, mbits, Wt = oracle.prepare_weights(W, n, m, scale_bf16=bf16, scale_global=True)
+    w = sbl.sbl_prepare_weights(to_dev(W), n, m, with_mask=True, scale_bf16=bf16, scale_global=True)
+    assert sbl.sbl_device_status() == 0
+    assert np.array_equal(w.row_scale.cpu().numpy().view(np.uint32), scale.view(np.uint32))
+    assert np.array_equal(w.packed.cpu().numpy(), packed)
+    assert np.array_equal(w.mask_bits.cpu().numpy(), mbits)
+    y_ref, acc_ref, _, _ = oracle.linear(xval, Wt, scale)
+    y, acc = _run_linear(sbl, w, xbits, 3, O, "auto")
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    assert_fp32_close(y.cpu().numpy(), y_ref)
