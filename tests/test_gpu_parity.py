@@ -481,3 +481,20 @@ def test_prepare_scale_global(sbl, n, m, O, K, bf16):
     y, acc = _run_linear(sbl, w, xbits, 3, O, "auto")
     assert np.array_equal(acc.cpu().numpy(), acc_ref)
     assert_fp32_close(y.cpu().numpy(), y_ref)
+
+
+@pytest.mark.parametrize("path", ["prefill", "prefill_1cta", "prefill_pair"])
+def test_prefill_large_t_full(sbl, path):
+    """T = 16500 on the dense paths (ragged last token tile), every output
+    element compared, and a second call reusing the workspace."""
+    O, K, T, n, m = 256, 256, 16500, 3, 4
+    W, xbits, xval = layer_inputs(O, K, T, seed=10, outlier_p=0.01)
+    ref = oracle_layer(W, n, m, xval)
+    w = _prep(sbl, W, n, m)
+    ws = sbl.workspace_for(T, K, O, n, m, "cuda")
+    for _ in range(2):
+        acc = torch.empty((T, O), dtype=torch.int32, device="cuda")
+        y = sbl.sbl_linear(x_dev(xbits), w, acc_out=acc, workspace=ws, path=path)
+        assert sbl.sbl_device_status() == 0
+        assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+        assert_fp32_close(y.cpu().numpy(), ref["y"])
