@@ -182,9 +182,12 @@ sbl_status sbl_mask_monitor(const uint8_t* old_bits, const uint8_t* new_bits, in
  * internal layout (T*K + 4*T bytes, each rounded up to 256), plus, for 2:4
  * weights (K % 64 == 0) at sizes that take a prefill path, the weights'
  * compressed form for the sparse tensor cores (O*K/2 + O*32*ceil(K/256)
- * bytes, each rounded up to 256).  Never 0 for T > 0.  A smaller workspace
- * that still holds the first part is accepted; sbl_linear then stays on the
- * dense paths.
+ * bytes, each rounded up to 256) or, when the one-CTA tensor-core kernel is
+ * split along k (few output tiles facing a long K, small T), its int32
+ * accumulator tiles (64 KiB per 128 x 128 output tile), whichever is larger.
+ * Depends on the current device's SM count.  Never 0 for T > 0.  A smaller
+ * workspace that still holds the first part is accepted; sbl_linear then
+ * stays on the dense, unsplit paths.
  */
 size_t sbl_linear_workspace_bytes(int64_t T, int64_t K, int64_t O, int n, int m);
 

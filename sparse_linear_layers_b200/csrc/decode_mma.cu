@@ -3,8 +3,9 @@
 // Same result as the CUDA-core decode kernel (decode.cu): the integer product
 // of the Sparse-BitNet Guide's linear-evaluation equation ("Mathematical
 // Formulation of Sparse-BitLinear") over 2-bit weights read once from HBM,
-// with the activations quantised per token inside the kernel and the dequant
-// epilogue fused.  With several tokens the CUDA-core form spends four dp4a per
+// with the activations quantised per token inside the kernel (or, after the
+// RMSNorm front end, copied in already quantised) and the dequant epilogue
+// fused.  With several tokens the CUDA-core form spends four dp4a per
 // 16 weights and token plus a shared-memory load per token; here the ternary
 // codes are expanded once into int8 registers that are the A fragments of
 // mma.sync m16n8k32 (16 output rows x 32 weights), and the activations of up

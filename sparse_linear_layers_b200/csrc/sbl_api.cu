@@ -1,6 +1,7 @@
 // C ABI of the Sparse-BitLinear library: argument validation, workspace
 // layout, path dispatch and the per-device status word.  All arithmetic runs
-// in the kernels of prep.cu, quant.cu, decode.cu, decode_mma.cu, prefill.cu, prefill_pair.cu and prefill_sp.cu.
+// in the kernels of prep.cu, quant.cu, decode.cu, decode_mma.cu, prefill.cu, prefill_pair.cu, prefill_sp.cu and
+// mask_monitor.cu.
 #include <cstdint>
 #include <cstdio>
 #include <cuda_runtime.h>
