@@ -498,3 +498,52 @@ def test_prefill_large_t_full(sbl, path):
         assert sbl.sbl_device_status() == 0
         assert np.array_equal(acc.cpu().numpy(), ref["acc"])
         assert_fp32_close(y.cpu().numpy(), ref["y"])
+
+
+def test_graph_replay_of_split_rmsnorm_and_monitor(sbl):
+    """A CUDA graph holding a split-K prefill (its accumulators zeroed inside
+    the graph by the quantisation kernel), an RMSNorm-fronted decode and a mask
+    monitor (a memset node), replayed three times: every replay matches."""
+    O, K, T, n, m = 512, 4096, 40, 2, 4
+    W, xbits, xval = layer_inputs(O, K, T, seed=12)
+    W2 = W + np.float32(0.003)
+    ref = oracle_layer(W, n, m, xval)
+    g = np.random.default_rng(4).uniform(0.5, 1.5, K).astype(np.float32)
+    _, scale, mb1, Wt = oracle.prepare_weights(W, n, m)
+    _, _, mb2, _ = oracle.prepare_weights(W2, n, m)
+    y_rms, acc_rms, _, _ = oracle.linear(xval[:8], Wt, scale, g=g, eps=2.0 ** -23)
+    changed, bad, _ = oracle.mask_monitor(mb1, mb2, K, n, m)
+    w = sbl.sbl_prepare_weights(to_dev(W), n, m, with_mask=True)
+    w2 = sbl.sbl_prepare_weights(to_dev(W2), n, m, with_mask=True)
+    assert sbl.sbl_linear_plan(T, K, O, n, m) == "prefill_1cta"
+    x, x8, gd = x_dev(xbits), x_dev(xbits[:8]), to_dev(g)
+    ws = sbl.workspace_for(T, K, O, n, m, "cuda")
+    ws8 = sbl.workspace_for(8, K, O, n, m, "cuda")
+    acc = torch.empty((T, O), dtype=torch.int32, device="cuda")
+    y = torch.empty((T, O), dtype=torch.float32, device="cuda")
+    acc8 = torch.empty((8, O), dtype=torch.int32, device="cuda")
+    y8 = torch.empty((8, O), dtype=torch.float32, device="cuda")
+    out = {}
+    s = torch.cuda.Stream()
+
+    def step():
+        sbl.sbl_linear(x, w, y=y, acc_out=acc, workspace=ws)
+        sbl.sbl_linear_rmsnorm(x8, w, gd, y=y8, acc_out=acc8, workspace=ws8)
+        out["tot"], _ = sbl.sbl_mask_monitor(w.mask_bits, w2.mask_bits, K, n, m)
+
+    with torch.cuda.stream(s):
+        step()
+    s.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        step()
+    for _ in range(3):
+        acc.zero_(), acc8.zero_(), y.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert sbl.sbl_device_status() == 0
+        assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+        assert_fp32_close(y.cpu().numpy(), ref["y"])
+        assert np.array_equal(acc8.cpu().numpy(), acc_rms)
+        assert_fp32_close(y8.cpu().numpy(), y_rms)
+        assert out["tot"].cpu().tolist() == [changed, bad]
