@@ -64,6 +64,10 @@ def test_noalloc_matches_linear_on_two_calls_in_a_row(abi):
     # contents in the shared scratch array and must not depend on them
     _run_both(abi, O=768, K=896, T=1000, n=3, m=4, seed=0)
     _run_both(abi, O=512, K=2048, T=384, n=2, m=4, seed=1)
+    # long K, few tiles: both entry points split the one-CTA prefill along k;
+    # the accumulators in the shared scratch hold the previous call's sums
+    _run_both(abi, O=2048, K=7168, T=64, n=2, m=4, seed=2)
+    _run_both(abi, O=2048, K=7168, T=64, n=2, m=4, seed=3)
 
 
 def test_noalloc_rejects_calls_beyond_its_scratch(abi):
