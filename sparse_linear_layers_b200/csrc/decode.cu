@@ -92,6 +92,8 @@ __global__ void __launch_bounds__(kDecodeThreads, decode_min_blocks<TT>()) decod
 #pragma unroll
             for (int w = 0; w < CW; ++w) wb[b][w] = 0u;
     }
+    // the row scale is needed only by the epilogue: load it now, off the critical path
+    const float sc = (valid && li == 0) ? row_scale[row] : 0.0f;
 
     // Quantise this pass's tokens: per-token absmax, then int8 into shared memory.
     const int nvec = K >> 3;
@@ -243,7 +245,6 @@ __global__ void __launch_bounds__(kDecodeThreads, decode_min_blocks<TT>()) decod
         acc[t] = a;
     }
     if (valid && li == 0) {
-        const float sc = row_scale[row];
 #pragma unroll
         for (int t = 0; t < TT; ++t) {
             const long long tt = t0 + t;
