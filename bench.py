@@ -713,7 +713,10 @@ def cpu_baseline_sample(budget_s=20.0, sample_tokens=32):
         t_lin += c - b
     tok = sample_tokens + T_DECODE
     step_s = t_prep + t_lin * TOKENS_PER_STEP / tok
+    # dense-equivalent integer ops of the sampled contractions (2 * T * O * K per projection)
+    lin_ops = 2.0 * tok * sum(O * K for _, K, O in synthetic.QWEN05_LAYER)
     return {"value": TOKENS_PER_STEP / step_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "contraction_gops": lin_ops / t_lin / 1e9 if t_lin > 0 else None,
             "sample": f"weight prep of all 7 projections + {sample_tokens} of 2048 prefill tokens + the decode "
                       f"token; step time extrapolated to 2049 tokens (measured prep {t_prep:.2f}s, "
                       f"linear {t_lin:.2f}s)"}
@@ -746,7 +749,7 @@ def run_reference(args, rank, world):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": _config({"parallelism": "CPU oracle, rank 0 only"}), "impl": "reference",
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": _cpu_threads(), "kind": "oracle",
-                             "sample": r["sample"]},
+                             "sample": r["sample"], "contraction_gops": r.get("contraction_gops")},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "wall_s": wall}
 
