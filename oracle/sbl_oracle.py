@@ -18,6 +18,8 @@ the 2-bit code table of its "What ships with this repo / Packed vs raw"):
               module does (optional, the fused RMSNorm entry points)
     acc       x_q . W_t^T in integers
     y         acc * scale_i / s_t,  s_t = 127 / max|x_t|
+    (backward) straight-through gradients dX = dY . (scale * W_t),
+              dW = dY^T . (x_q / s_t) (the training path)
 
 Readings taken where the pages are silent or disagree (each one is listed
 with its reason in the design notes):
@@ -42,6 +44,10 @@ with its reason in the design notes):
   b % 32 == l; the 32 lane sums are combined by an xor butterfly at offsets
   16, 8, 4, 2, 1); mean = sum / K; inv = 1 / sqrt(mean + eps);
   x_norm = (x * inv) * g.
+* training (straight-through) backward: every quantiser acts as the identity,
+  so dX = dY . (scale * W_t) and dW = dY^T . (x_q / s_t) over all positions,
+  masked ones included; optionally (the guide's module) dW taken at the
+  ternary matrix, i.e. scaled once more by scale_o.
 
 Every function here is pinned by tests that do not call it to build their
 expected values (worked examples from the pages, closed forms, brute force).
@@ -317,3 +323,36 @@ def acc_entries(xq: np.ndarray, Wt: np.ndarray, idx_t, idx_o) -> np.ndarray:
     xq = np.asarray(xq, np.int64)
     Wt = np.asarray(Wt, np.int64)
     return np.array([int(np.dot(xq[t], Wt[o])) for t, o in zip(idx_t, idx_o)], dtype=np.int64)
+
+
+def ste_backward(dY: np.ndarray, xq: np.ndarray, s_tok: np.ndarray, Wt: np.ndarray, scale: np.ndarray,
+                 dw_ternary: bool = False):
+    """Straight-through gradients of the forward y = (x_q . W_t^T) * scale_o / s_t:
+    (dX float64 [T, K], dW float64 [O, K]) for the loss gradient dY [T, O].
+
+    Reading (the guide's "Training Stability & The Straight-Through Estimator":
+    the backward bypasses the N:M mask and the ternary rounding and reaches the
+    latent weights; the Sparse-BitNet README, "How It Works / BitLinear": the
+    gradient passes the quantiser by straight-through estimation): in the
+    backward every quantiser is the identity, so the forward reads as
+    y = x_hat . W_hat^T with x_hat[t,k] = x_q[t,k] / s_t (the activations the
+    forward used) and W_hat[o,k] = scale_o * W_t[o,k] (the weights it used):
+
+        dX[t,k] = sum_o dY[t,o] * scale_o * W_t[o,k]
+        dW[o,k] = sum_t dY[t,o] * x_q[t,k] / s_t     (every position, masked ones too)
+
+    dX is the gradient at the quantiser's input (after the RMSNorm, when the
+    fused front end ran).  With ``dw_ternary`` the weight gradient is the one the
+    guide's module returns: taken at the ternary matrix of its equation
+    y = (x~ . W~^T) * beta * gamma / 127, i.e. dW[o,k] scaled once more by scale_o.
+    Products and sums in float64 (numpy matrix products).
+    """
+    dY = np.asarray(dY, np.float64)
+    xhat = np.asarray(xq, np.float64) / np.asarray(s_tok, np.float64)[:, None]
+    sc = np.asarray(scale, np.float64)
+    Wt = np.asarray(Wt, np.float64)
+    dX = (dY * sc[None, :]) @ Wt
+    dW = dY.T @ xhat
+    if dw_ternary:
+        dW = dW * sc[:, None]
+    return dX, dW

@@ -70,6 +70,11 @@ def activations(T: int, K: int, seed: int = 0, tag: str = "x", outlier_p: float 
     return bits, bf16_bits_to_f32(bits)
 
 
+def output_grads(T: int, O: int, seed: int = 0, tag: str = "dY") -> np.ndarray:
+    """fp32 [T, O] loss gradients at the layer output, i.i.d. N(0, 1)."""
+    return _rng(seed, tag).standard_normal((T, O), dtype=np.float32)
+
+
 # Layer shapes (K -> O) of the workloads.  Qwen2.5-0.5B skeleton: d_model 896,
 # d_ffn 4864, 14 heads / 2 KV heads of width 64 (halo card, "Recipe").  The
 # hidden-2048 / FFN-7168 stack follows the tritter-500m card's shapes.

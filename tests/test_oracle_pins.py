@@ -708,3 +708,93 @@ def test_planted_global_scale_mistake_is_caught(name):
     o = types.SimpleNamespace(global_scale=fn, prepare_weights=prep)
     with pytest.raises(AssertionError):
         pin_global_scale(o)
+
+
+# --------------------------------------------------------------------------
+# training path: straight-through backward
+# --------------------------------------------------------------------------
+
+def _ste_inputs(O, K, T, n, m, seed):
+    W = synthetic.latent_weights(O, K, seed=seed)
+    _, x = synthetic.activations(T, K, seed=seed)
+    dY = synthetic.output_grads(T, O, seed=seed)
+    _, scale, mb, Wt = oracle.prepare_weights(W, n, m)
+    xq, s = oracle.quant_act(x)
+    keep = np.unpackbits(mb, axis=1, bitorder="little")[:, :K].astype(bool)
+    return W, x, dY, Wt, scale, xq, s, keep
+
+
+def pin_ste_backward(o):
+    """torch autograd (float64) through the straight-through surrogate of the
+    forward — x_hat = x + (x_q/s - x).detach(), W_hat = W + (scale*W_t - W).detach(),
+    and for the guide's module form W~ = W + (W_t - W).detach() with the scale
+    applied after the product — whose value is checked to equal the forward's y;
+    one-hot loss gradients place single rows; the gradient reaches masked weights."""
+    import torch
+    f64 = torch.float64
+    for (O, K, T, n, m, seed) in ((8, 32, 5, 2, 4, 0), (16, 64, 3, 3, 4, 1), (12, 48, 7, 6, 8, 2),
+                                  (32, 32, 4, 4, 8, 3)):
+        W, x, dY, Wt, scale, xq, s, keep = _ste_inputs(O, K, T, n, m, seed)
+        y_fwd = oracle.linear(x, Wt, scale)[0]
+        xl = torch.tensor(x, dtype=f64, requires_grad=True)
+        Wl = torch.tensor(W, dtype=f64, requires_grad=True)
+        x_hat = xl + (torch.tensor(xq, dtype=f64) / torch.tensor(s, dtype=f64)[:, None] - xl).detach()
+        W_hat = Wl + (torch.tensor(Wt, dtype=f64) * torch.tensor(scale, dtype=f64)[:, None] - Wl).detach()
+        y = x_hat @ W_hat.T
+        np.testing.assert_allclose(y.detach().numpy(), y_fwd, rtol=1e-12, atol=1e-15)
+        (y * torch.tensor(dY, dtype=f64)).sum().backward()
+        dX, dW = o.ste_backward(dY, xq, s, Wt, scale)
+        assert dX.shape == (T, K) and dW.shape == (O, K)
+        np.testing.assert_allclose(dX, xl.grad.numpy(), rtol=1e-12, atol=1e-12 * np.abs(dX).max())
+        np.testing.assert_allclose(dW, Wl.grad.numpy(), rtol=1e-12, atol=1e-12 * np.abs(dW).max())
+        assert np.count_nonzero(dW[~keep]) == np.count_nonzero(~keep)  # masked weights get gradient
+
+        W2 = torch.tensor(W, dtype=f64, requires_grad=True)
+        W_tern = W2 + (torch.tensor(Wt, dtype=f64) - W2).detach()
+        y2 = (x_hat.detach() @ W_tern.T) * torch.tensor(scale, dtype=f64)[None, :]
+        np.testing.assert_allclose(y2.detach().numpy(), y_fwd, rtol=1e-12, atol=1e-15)
+        (y2 * torch.tensor(dY, dtype=f64)).sum().backward()
+        dX2, dW2 = o.ste_backward(dY, xq, s, Wt, scale, dw_ternary=True)
+        np.testing.assert_allclose(dW2, W2.grad.numpy(), rtol=1e-12, atol=1e-12 * np.abs(dW2).max())
+        np.testing.assert_array_equal(dX2, dX)
+
+        t, i = T // 2, O - 1                               # one-hot loss gradient
+        e = np.zeros((T, O), np.float32)
+        e[t, i] = 1.0
+        dXe, dWe = o.ste_backward(e, xq, s, Wt, scale)
+        assert np.array_equal(np.nonzero(np.any(dXe != 0, axis=1))[0], [t])
+        np.testing.assert_array_equal(dXe[t], scale[i].astype(np.float64) * Wt[i])
+        assert np.array_equal(np.nonzero(np.any(dWe != 0, axis=1))[0], [i])
+        np.testing.assert_allclose(dWe[i], xq[t].astype(np.float64) / float(s[t]), rtol=1e-15, atol=0)
+    dX, dW = o.ste_backward(np.zeros((0, 4), np.float32), np.zeros((0, 16), np.int8), np.zeros(0, np.float32),
+                            np.ones((4, 16), np.int8), np.ones(4, np.float32))
+    assert dX.shape == (0, 16) and dW.shape == (4, 16) and not np.any(dW)
+
+
+def test_ste_backward_pins():
+    pin_ste_backward(oracle)
+
+
+@pytest.mark.parametrize("name", ["dw_masked", "dx_no_scale", "dw_no_token_scale", "dw_transposed",
+                                  "ternary_flag_ignored", "dx_latent_weights"])
+def test_planted_ste_backward_mistake_is_caught(name):
+    def bwd(dY, xq, s_tok, Wt, scale, dw_ternary=False):
+        dY = np.asarray(dY, np.float64)
+        sc = np.asarray(scale, np.float64)
+        xhat = np.asarray(xq, np.float64) / np.asarray(s_tok, np.float64)[:, None]
+        if name == "dw_no_token_scale":
+            xhat = np.asarray(xq, np.float64)
+        dX = (dY * (1.0 if name == "dx_no_scale" else sc[None, :])) @ np.asarray(Wt, np.float64)
+        if name == "dx_latent_weights":   # the dense latent-scale product, not the ternary one
+            dX = dY @ (np.sign(np.asarray(Wt, np.float64)) * sc[:, None] + 1e-3)
+        dW = dY.T @ xhat
+        if name == "dw_masked":
+            dW = dW * (np.asarray(Wt) != 0)
+        if name == "dw_transposed":
+            dW = (xhat.T @ dY) if dW.shape[0] == dW.shape[1] else dW.T
+        if dw_ternary and name != "ternary_flag_ignored":
+            dW = dW * sc[:, None]
+        return dX, dW
+
+    with pytest.raises(AssertionError):
+        pin_ste_backward(types.SimpleNamespace(ste_backward=bwd))
