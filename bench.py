@@ -489,6 +489,44 @@ def _mask_monitor_bench(sbl, dev, hbm_peak):
     return out
 
 
+# fp32 FMA peak of the CUDA cores: SMs x 128 fp32 lanes x 2 flops x clocks.max.sm (1965 MHz)
+FP32_LANES_PER_SM = 128
+SM_MAX_MHZ = 1965.0
+
+
+def _ste_backward_bench(sbl, dev, T=4096):
+    """The training path's straight-through gradients (dX = dY . W_hat,
+    dW = dY^T . x_hat) of the hidden-2048 stack's projections at T tokens,
+    each kernel graph-replayed with L2 flushed; flops 2 * T * O * K per
+    gradient against the fp32 FMA peak of the CUDA cores."""
+    props = torch.cuda.get_device_properties(dev)
+    peak = props.multi_processor_count * FP32_LANES_PER_SM * 2 * SM_MAX_MHZ * 1e6 / 1e12
+    out = {"tokens": T, "fp32_peak_tflops": peak,
+           "peak_source": f"{props.multi_processor_count} SMs x {FP32_LANES_PER_SM} fp32 lanes x 2 x {SM_MAX_MHZ} MHz"}
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(17)
+    from sparse_linear_layers_b200 import _lib
+    for name, K, O in (("q 2048->2048", 2048, 2048), ("gate 2048->7168", 2048, 7168), ("down 7168->2048", 7168, 2048)):
+        W = torch.randn((O, K), device=dev, generator=gen) * 0.02
+        w = sbl.sbl_prepare_weights(W, 2, 4)
+        x = torch.randn((T, K), device=dev, generator=gen).to(torch.bfloat16)
+        xq, st = sbl.sbl_quant_act(x)
+        dY = torch.randn((T, O), device=dev, generator=gen)
+        dX = torch.empty((T, K), device=dev)
+        dW = torch.empty((O, K), device=dev)
+        res = {}
+        for g, (px, pw) in (("dX", (dX.data_ptr(), None)), ("dW", (None, dW.data_ptr()))):
+            fn = lambda px=px, pw=pw: _lib.check(_lib.lib.sbl_linear_backward(
+                dY.data_ptr(), T, O, xq.data_ptr(), st.data_ptr(), K, w.packed.data_ptr(), w.row_scale.data_ptr(),
+                px, pw, 0, torch.cuda.current_stream().cuda_stream), "sbl_linear_backward")
+            us = _flushed_graph_us(fn, dev)
+            tf = 2.0 * T * O * K / us / 1e6
+            res[g] = {"us": us, "tflops": tf, "frac": tf / peak}
+        out[name] = res
+        del W, w, x, xq, dY, dX, dW
+    return out
+
+
 def _pool_call_us(sbl, x, w, y, ws, reps=5):
     """Per-call device time of sbl_linear in steady state: a CUDA graph of
     back-to-back calls that cycle through copies of the weights and
@@ -783,7 +821,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration sweep (profiling runs)")
-    ap.add_argument("--only", choices=("rmsnorm_front", "mask_monitor"),
+    ap.add_argument("--only", choices=("rmsnorm_front", "mask_monitor", "ste_backward"),
                     help="run only this auxiliary measurement on one GPU and print its JSON (profiling runs)")
     ap.add_argument("--tokens", type=int, default=32768, help="tokens of the --only rmsnorm_front measurement")
     args = ap.parse_args()
@@ -804,8 +842,12 @@ def main():
     if args.only:
         import sparse_linear_layers_b200 as sbl
         hbm_peak = _peaks()[0]
-        res = (_rmsnorm_front(sbl, dev, hbm_peak, T=args.tokens) if args.only == "rmsnorm_front"
-               else _mask_monitor_bench(sbl, dev, hbm_peak))
+        if args.only == "rmsnorm_front":
+            res = _rmsnorm_front(sbl, dev, hbm_peak, T=args.tokens)
+        elif args.only == "mask_monitor":
+            res = _mask_monitor_bench(sbl, dev, hbm_peak)
+        else:
+            res = _ste_backward_bench(sbl, dev)
         print(json.dumps({"only": args.only, "result": res}), flush=True)
         return
     if world > 1:

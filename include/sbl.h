@@ -176,6 +176,44 @@ sbl_status sbl_rmsnorm_quant_act(const uint16_t* x_bf16, const float* g, float e
 sbl_status sbl_mask_monitor(const uint8_t* old_bits, const uint8_t* new_bits, int64_t O, int64_t K, int n, int m,
                             uint64_t* totals, uint32_t* row_changed, void* stream);
 
+/* Flags of sbl_linear_backward. */
+enum { SBL_BWD_DW_TERNARY = 1 };
+
+/*
+ * sbl_linear_backward — straight-through (STE) gradients of sbl_linear, the
+ * training path.
+ *
+ * The Sparse-BitNet Guide, "Training Stability & The Straight-Through
+ * Estimator": the backward passes the N:M mask and the ternary rounding
+ * unchanged to the latent weights (masked positions included, so a pruned
+ * weight can re-enter the mask); the Sparse-BitNet README, "How It Works /
+ * BitLinear": gradients pass the quantiser by straight-through estimation.
+ * With the activation quantiser passed through too, the forward reads
+ * y = x_hat . W_hat^T, x_hat[t,k] = x_q[t,k] / s_t, W_hat[o,k] = scale_o * W_t[o,k]:
+ *
+ *   dY         fp32 [T, O]: gradient of the loss with respect to y.
+ *   x_q, s_tok the forward's int8 [T, K] activations in natural column order
+ *              and fp32 [T] scales (sbl_quant_act / sbl_rmsnorm_quant_act).
+ *   packed, row_scale  the prepared weights (sbl_prepare_weights), [O, K/4], [O].
+ *   dX         fp32 [T, K] (output, may be NULL):
+ *              dX[t,k] = sum_o dY[t,o] * scale_o * W_t[o,k] — the gradient at
+ *              the quantiser's input (after the RMSNorm, for the fused front end).
+ *   dW         fp32 [O, K] (output, may be NULL):
+ *              dW[o,k] = sum_t dY[t,o] * x_q[t,k] / s_t; with
+ *              SBL_BWD_DW_TERNARY each row is multiplied by scale_o once more
+ *              (the gradient at the ternary matrix of the guide's equation
+ *              y = (x~ . W~^T) * beta * gamma / 127, as its module returns it).
+ * fp32 arithmetic with fused multiply-adds in an unspecified order: each
+ * output is within (n + 2) * 2^-24 * sum |terms| of the exact value, n the
+ * reduction length (O for dX, T for dW).  Empty reductions write zeros
+ * (dW for T == 0, dX for O == 0).  Only the pointers the requested outputs
+ * read must be valid.  At least one of dX, dW must be non-NULL.
+ * K % 16 == 0; any T, O >= 0.  Asynchronous on `stream`; no workspace.
+ */
+sbl_status sbl_linear_backward(const float* dY, int64_t T, int64_t O, const int8_t* x_q, const float* s_tok,
+                               int64_t K, const uint8_t* packed, const float* row_scale, float* dX, float* dW,
+                               int flags, void* stream);
+
 /*
  * sbl_linear_workspace_bytes — bytes of device workspace sbl_linear needs for
  * these sizes: the quantised activations and their scales, in the kernels'

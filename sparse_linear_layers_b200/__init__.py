@@ -3,7 +3,8 @@
 y = dequant(int8(x) . ternary_NM(W)^T) behind a C ABI (include/sbl.h) with
 hand-written CUDA kernels: fused weight preparation, per-token activation
 quantisation (optionally after RMSNorm, as the guide's module does), decode
-paths on CUDA cores and the warp-level MMA, and tcgen05 tensor-core prefill.
+paths on CUDA cores and the warp-level MMA, tcgen05 tensor-core prefill, a
+mask monitor and the straight-through backward of the training path.
 
 The library entry points (sbl_prepare_weights, sbl_quant_act, sbl_linear, ...)
 load libsbl.so on first use and raise ImportError if it has not been built;
@@ -12,7 +13,7 @@ GPU library.
 """
 __version__ = "0.1.0"
 
-_API = ("PreparedWeights", "sbl_decode_max_tokens", "sbl_device_status", "sbl_linear", "sbl_linear_plan",
+_API = ("PreparedWeights", "sbl_decode_max_tokens", "sbl_device_status", "sbl_linear", "sbl_linear_backward", "sbl_linear_plan",
         "sbl_linear_rmsnorm", "sbl_linear_workspace_bytes", "sbl_mask_monitor", "sbl_prepare_weights", "sbl_quant_act",
         "sbl_rmsnorm_quant_act", "sbl_selftest_bounded_wait", "workspace_for", "RMSNORM_EPS_F32", "SblError")
 

@@ -23,6 +23,8 @@ SBL_ERR_WORKSPACE = 6
 SBL_PREP_SCALE_BF16 = 1
 SBL_PREP_SCALE_GLOBAL = 2
 
+SBL_BWD_DW_TERNARY = 1
+
 SBL_F32 = 0
 SBL_BF16 = 1
 
@@ -49,6 +51,7 @@ SIGNATURES = {
     "sbl_linear_noalloc": (_int, [_vp, _i64, _i64, _vp, _vp, _i64, _int, _int, _vp, _int, _vp, _vp]),
     "sbl_linear_plan": (_int, [_i64, _i64, _i64, _int, _int, _sz]),
     "sbl_mask_monitor": (_int, [_vp, _vp, _i64, _i64, _int, _int, _vp, _vp, _vp]),
+    "sbl_linear_backward": (_int, [_vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _int, _vp]),
     "sbl_decode_max_tokens": (_i64, []),
     "sbl_device_status": (_int, [_vp]),
     "sbl_selftest_bounded_wait": (_int, [_u32, _vp]),

@@ -178,6 +178,40 @@ def sbl_mask_monitor(old_bits: torch.Tensor, new_bits: torch.Tensor, K: int, n: 
     return totals, rows
 
 
+def sbl_linear_backward(dY: torch.Tensor, x_q: torch.Tensor, s_tok: torch.Tensor, w: PreparedWeights,
+                        need_dx: bool = True, need_dw: bool = True, dw_ternary: bool = False,
+                        dX: Optional[torch.Tensor] = None, dW: Optional[torch.Tensor] = None,
+                        stream: Optional[torch.cuda.Stream] = None):
+    """Straight-through gradients of sbl_linear: (dX fp32 [T,K] or None, dW fp32 [O,K] or None).
+
+    dX = dY . (scale * W_t) and dW = dY^T . (x_q / s_t) over every weight position
+    (``dw_ternary``: dW rows scaled by scale_o once more, the guide module's form).
+    ``x_q``/``s_tok`` are the forward's quantised activations in natural order
+    (sbl_quant_act or sbl_rmsnorm_quant_act)."""
+    _need_cuda(dY, "dY", torch.float32)
+    _need_cuda(x_q, "x_q", torch.int8)
+    _need_cuda(s_tok, "s_tok", torch.float32)
+    T, O = dY.shape
+    K = w.K
+    if O != w.O or x_q.shape != (T, K) or s_tok.shape != (T,):
+        raise ValueError(f"dY {tuple(dY.shape)}, x_q {tuple(x_q.shape)} and s_tok {tuple(s_tok.shape)} do not match "
+                         f"weights with O={w.O}, K={K}")
+    if not (need_dx or need_dw):
+        raise ValueError("ask for dX, dW or both")
+    if need_dx:
+        dX = torch.empty((T, K), dtype=torch.float32, device=dY.device) if dX is None else dX
+        _need_cuda(dX, "dX", torch.float32)
+    if need_dw:
+        dW = torch.empty((O, K), dtype=torch.float32, device=dY.device) if dW is None else dW
+        _need_cuda(dW, "dW", torch.float32)
+    check(lib.sbl_linear_backward(dY.data_ptr(), T, O, x_q.data_ptr(), s_tok.data_ptr(), K, w.packed.data_ptr(),
+                                  w.row_scale.data_ptr(), dX.data_ptr() if need_dx else None,
+                                  dW.data_ptr() if need_dw else None,
+                                  _lib.SBL_BWD_DW_TERNARY if dw_ternary else 0, _stream(stream)),
+          "sbl_linear_backward")
+    return (dX if need_dx else None), (dW if need_dw else None)
+
+
 _PATH_NAMES = {v: k for k, v in _PATHS.items()}
 
 

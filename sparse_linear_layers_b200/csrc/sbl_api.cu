@@ -1,7 +1,7 @@
 // C ABI of the Sparse-BitLinear library: argument validation, workspace
 // layout, path dispatch and the per-device status word.  All arithmetic runs
-// in the kernels of prep.cu, quant.cu, decode.cu, decode_mma.cu, prefill.cu, prefill_pair.cu, prefill_sp.cu and
-// mask_monitor.cu.
+// in the kernels of prep.cu, quant.cu, decode.cu, decode_mma.cu, prefill.cu, prefill_pair.cu, prefill_sp.cu,
+// mask_monitor.cu and backward.cu.
 #include <cstdint>
 #include <cstdio>
 #include <cuda_runtime.h>
@@ -29,6 +29,10 @@ cudaError_t launch_rmsnorm_quant(const uint16_t* x, const float* g, float eps, l
                                  long long nzero16);
 cudaError_t launch_mask_monitor(const uint8_t* old_bits, const uint8_t* new_bits, long long O, long long K, int n,
                                 int m, unsigned long long* totals, uint32_t* row_changed, cudaStream_t stream);
+long long ste_backward_tiles(long long rows, long long K);
+cudaError_t launch_ste_backward(const float* dY, long long T, long long O, long long K, const uint8_t* packed,
+                                const float* row_scale, const int8_t* xq, const float* s_tok, float* dX, float* dW,
+                                int dw_ternary, cudaStream_t stream);
 cudaError_t launch_prefill(const int8_t* xperm, const float* s_tok, long long T, long long K, const uint8_t* packed,
                            const float* row_scale, long long O, void* y, int y_bf16, int32_t* acc_out,
                            unsigned* status, int num_sms, int variant, int ksplit, int32_t* part,
@@ -180,6 +184,30 @@ sbl_status sbl_mask_monitor(const uint8_t* old_bits, const uint8_t* new_bits, in
     if (O == 0) return from_cuda(cudaMemsetAsync(totals, 0, 2 * sizeof(uint64_t), st));
     return from_cuda(sbl::launch_mask_monitor(old_bits, new_bits, O, K, n, m,
                                               reinterpret_cast<unsigned long long*>(totals), row_changed, st));
+}
+
+sbl_status sbl_linear_backward(const float* dY, int64_t T, int64_t O, const int8_t* x_q, const float* s_tok,
+                               int64_t K, const uint8_t* packed, const float* row_scale, float* dX, float* dW,
+                               int flags, void* stream) {
+    if (T < 0 || O < 0) return SBL_ERR_INVALID_ARG;
+    if (flags & ~SBL_BWD_DW_TERNARY) return SBL_ERR_INVALID_ARG;
+    if (sbl_status s = check_k(K)) return s;
+    if (!dX && !dW) return SBL_ERR_INVALID_ARG;
+    const bool any_dx = dX && T > 0, any_dw = dW && O > 0;  // outputs with elements
+    const bool ternary = (flags & SBL_BWD_DW_TERNARY) != 0;
+    // what the requested outputs read: every pointer non-null and 16-byte aligned
+    auto ok = [](const void* p) { return p != nullptr && aligned(p, 16); };
+    if (any_dx && !(ok(dX) && (O == 0 || (ok(dY) && ok(packed) && ok(row_scale))))) return SBL_ERR_INVALID_ARG;
+    if (any_dw && !(ok(dW) && (T == 0 || (ok(dY) && ok(x_q) && ok(s_tok))) && (!ternary || ok(row_scale))))
+        return SBL_ERR_INVALID_ARG;
+    if (sbl::ste_backward_tiles(T, K) > (1ll << 31) - 1 || sbl::ste_backward_tiles(O, K) > (1ll << 31) - 1)
+        return SBL_ERR_UNSUPPORTED;
+    if (!any_dx && !any_dw) return SBL_OK;
+    DeviceInfo* d;
+    if (sbl_status s = device_info(&d)) return s;
+    return from_cuda(sbl::launch_ste_backward(dY, T, O, K, packed, row_scale, x_q, s_tok, any_dx ? dX : nullptr,
+                                              any_dw ? dW : nullptr, ternary ? 1 : 0,
+                                              static_cast<cudaStream_t>(stream)));
 }
 
 // Quantised activations and their scales: what every path needs.

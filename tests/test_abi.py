@@ -124,6 +124,38 @@ def test_mask_monitor_rejects_on_host():
     assert M(p, p, -1, 64, 2, 4, p, None, None) == 1         # negative O
 
 
+def _has_device():
+    import torch
+    return torch.cuda.is_available()
+
+
+def test_backward_rejects_on_host():
+    from sparse_linear_layers_b200._lib import lib
+    p = 4096
+    B = lib.sbl_linear_backward
+    # (dY, T, O, x_q, s_tok, K, packed, row_scale, dX, dW, flags, stream)
+    assert B(p, 4, 8, p, p, 40, p, p, p, p, 0, None) == 1          # K % 16 != 0
+    assert B(p, -1, 8, p, p, 64, p, p, p, p, 0, None) == 1         # negative T
+    assert B(p, 4, -1, p, p, 64, p, p, p, p, 0, None) == 1         # negative O
+    assert B(p, 4, 8, p, p, 64, p, p, None, None, 0, None) == 1    # no output asked for
+    assert B(p, 4, 8, p, p, 64, p, p, p, p, 2, None) == 1          # unknown flag
+    assert B(p, 4, 8, p, p, 64, None, p, p, None, 0, None) == 1    # dX needs the packed weights
+    assert B(p, 4, 8, None, p, 64, p, p, None, p, 0, None) == 1    # dW needs x_q
+    assert B(p, 4, 8, p, None, 64, p, p, None, p, 0, None) == 1    # dW needs s_tok
+    assert B(p, 4, 8, p, p, 64, p, None, None, p, 1, None) == 1    # the ternary form needs row_scale
+    assert B(p + 4, 4, 8, p, p, 64, p, p, p, None, 0, None) == 1   # unaligned dY
+    assert B(p, 4, 8, p, p, 64, p, p, p + 8, None, 0, None) == 1   # unaligned dX
+    assert B(p, 4, 8, p, p, 1 << 25, p, p, p, None, 0, None) == 2  # K above the library's limit
+    # both outputs and the ternary flag: every host check passes and the missing
+    # device is reported (only without a device: these pointers are not real)
+    if not _has_device():
+        assert B(p, 4, 8, p, p, 64, p, p, p, p, 1, None) == 4
+        assert B(p, 4, 8, p, p, 64, p, p, p + 16, p + 32, 0, None) == 4
+    # nothing to write: accepted before any device work
+    assert B(None, 0, 8, None, None, 64, None, None, p, None, 0, None) == 0
+    assert B(None, 4, 0, None, None, 64, None, None, None, p, 0, None) == 0
+
+
 def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     import importlib
     from sparse_linear_layers_b200 import _lib
