@@ -1,5 +1,5 @@
 /*
- * sbl.h — C ABI of the Sparse-BitLinear forward on NVIDIA B200 (sm_100a).
+ * sbl.h — C ABI of the Sparse-BitLinear layer on NVIDIA B200 (sm_100a).
  *
  * The operator (Sparse-BitNet Guide: 1.58-Bit LLMs Meet 2:4 Sparsity, section
  * "Mathematical Formulation of Sparse-BitLinear"):
@@ -9,6 +9,7 @@
  * with W_t the N:M-masked ternary weights, x_q the per-token absmax int8
  * activations, scale_o the per-row absmean of the kept weights
  * (halo-sparse-bitnet-3:4-500m card, "Recipe") and s_t = 127 / max|x_t|.
+ * sbl_linear_backward gives its straight-through gradients for training.
  *
  * Conventions every entry point follows
  *   - All pointers are DEVICE pointers unless stated, owned by the caller, and
