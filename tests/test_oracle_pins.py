@@ -798,3 +798,22 @@ def test_planted_ste_backward_mistake_is_caught(name):
 
     with pytest.raises(AssertionError):
         pin_ste_backward(types.SimpleNamespace(ste_backward=bwd))
+
+
+def test_ste_backward_worked_block():
+    """The guide's 4-element block carried through the backward by hand
+    (tests/golden/ste_backward_worked.json)."""
+    with open(os.path.join(os.path.dirname(__file__), "golden", "ste_backward_worked.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        W = np.array([c["w"]], np.float32)
+        mask = oracle.nm_mask(W, c["n"], c["m"])
+        scale = oracle.row_scale(W, mask)
+        Wt = oracle.ternarise(W, scale, mask)
+        xq, s = oracle.quant_act(np.array([c["x"]], np.float32))
+        dY = np.array([[c["dY"]]], np.float32)
+        dX, dW = oracle.ste_backward(dY, xq, s, Wt, scale)
+        _, dWt = oracle.ste_backward(dY, xq, s, Wt, scale, dw_ternary=True)
+        np.testing.assert_allclose(dX[0], c["dX"], rtol=1e-6, atol=0)
+        np.testing.assert_allclose(dW[0], c["dW"], rtol=1e-6, atol=0)
+        np.testing.assert_allclose(dWt[0], c["dW_ternary"], rtol=1e-6, atol=0)
