@@ -18,7 +18,13 @@ _API = ("PreparedWeights", "sbl_decode_max_tokens", "sbl_device_status", "sbl_li
         "sbl_rmsnorm_quant_act", "sbl_selftest_bounded_wait", "workspace_for", "RMSNORM_EPS_F32", "SblError")
 
 
+_TRAIN = ("SparseBitLinear", "SparseBitLinearFunction")
+
+
 def __getattr__(name):
+    if name in _TRAIN:
+        from . import train
+        return getattr(train, name)
     if name in _API:
         from . import api
         from ._lib import SblError
@@ -26,4 +32,4 @@ def __getattr__(name):
     raise AttributeError(name)
 
 
-__all__ = list(_API)
+__all__ = list(_API) + list(_TRAIN)

@@ -1,0 +1,85 @@
+"""Autograd form of the layer for training.
+
+The Sparse-BitNet Guide's module ("End-to-End Implementation: Building a
+Sparse-BitLinear Layer") keeps fp32 latent weights, rebuilds the N:M mask and
+the ternary weights from them on every forward, and trains them through the
+straight-through estimator ("Training Stability & The Straight-Through
+Estimator").  Here every step of that runs in the library's kernels:
+
+    forward   sbl_prepare_weights (mask, scale, ternarise, pack; every call,
+              so the mask follows the latent weights), sbl_quant_act (the
+              int8 activations kept for the backward) and sbl_linear;
+    backward  sbl_linear_backward (dX = dY . (scale * W_t) to the activations,
+              dW = dY^T . (x_q / s_t) to every latent weight).
+
+The guide's module normalises x with an RMSNorm first; that normalisation and
+its gradient belong to the caller here (x is the layer's input as quantised).
+Argument marshalling only: no arithmetic of the layer runs in PyTorch.
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import api
+
+
+class SparseBitLinearFunction(torch.autograd.Function):
+    """y = dequant(int8(x) . ternary_NM(W)^T) with straight-through gradients.
+
+    x: bf16 [T, K] (contiguous), weight: fp32 [O, K] latent weights; returns fp32 [T, O]."""
+
+    @staticmethod
+    def forward(ctx, x, weight, n, m, dw_ternary):
+        w = api.sbl_prepare_weights(weight.detach(), n, m)
+        xq, s = api.sbl_quant_act(x)
+        y = api.sbl_linear(x, w)
+        ctx.save_for_backward(xq, s, w.packed, w.row_scale)
+        ctx.layer = (n, m, weight.shape[1], x.dtype, bool(dw_ternary))
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        xq, s, packed, row_scale = ctx.saved_tensors
+        n, m, K, x_dtype, dw_ternary = ctx.layer
+        need_dx, need_dw = ctx.needs_input_grad[0], ctx.needs_input_grad[1]
+        if not (need_dx or need_dw):
+            return None, None, None, None, None
+        w = api.PreparedWeights(packed, row_scale, n, m, K)
+        dX, dW = api.sbl_linear_backward(dy.float().contiguous(), xq, s, w, need_dx=need_dx, need_dw=need_dw,
+                                         dw_ternary=dw_ternary)
+        return (dX.to(x_dtype) if need_dx else None), dW, None, None, None
+
+
+class SparseBitLinear(torch.nn.Module):
+    """The guide's Sparse-BitLinear layer without its RMSNorm: fp32 latent
+    weights [out_features, in_features], N:M-sparse ternary in the forward.
+
+    ``dw_ternary`` selects the guide module's weight gradient (taken at the
+    ternary matrix, i.e. scaled by the row scale) instead of the
+    straight-through gradient of the dequantised weight.  Inputs of any
+    leading shape with last dimension in_features are cast to bf16 (the
+    library's activation type); the output is fp32."""
+
+    def __init__(self, in_features: int, out_features: int, n: int = 2, m: int = 4, dw_ternary: bool = False,
+                 device=None):
+        super().__init__()
+        self.in_features, self.out_features = in_features, out_features
+        self.n, self.m, self.dw_ternary = n, m, dw_ternary
+        self.weight = torch.nn.Parameter(torch.empty((out_features, in_features), dtype=torch.float32,
+                                                     device=device))
+        self.reset_parameters()
+
+    def reset_parameters(self) -> None:
+        # the same initialisation as the guide's module (torch's Linear default)
+        torch.nn.init.kaiming_uniform_(self.weight, a=math.sqrt(5))
+
+    def forward(self, x: torch.Tensor) -> torch.Tensor:
+        lead = x.shape[:-1]
+        x2 = x.reshape(-1, self.in_features).to(torch.bfloat16).contiguous()
+        y = SparseBitLinearFunction.apply(x2, self.weight, self.n, self.m, self.dw_ternary)
+        return y.reshape(*lead, self.out_features)
+
+    def extra_repr(self) -> str:
+        return f"in_features={self.in_features}, out_features={self.out_features}, {self.n}:{self.m}"

@@ -163,3 +163,13 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     with pytest.raises(ImportError):
         _lib._load()
     importlib.reload(_lib)  # restore the real module state
+
+
+def test_training_layer_has_no_cpu_fallback():
+    """The autograd layer reaches the library for every step; CPU tensors are refused."""
+    import torch
+    import sparse_linear_layers_b200 as sbl
+    layer = sbl.SparseBitLinear(64, 128, 2, 4)
+    assert tuple(layer.weight.shape) == (128, 64) and layer.weight.dtype == torch.float32
+    with pytest.raises(ValueError, match="CUDA"):
+        layer(torch.zeros(3, 64))
