@@ -702,6 +702,7 @@ def run_ours(args, rank, world, dev):
     configs = _configs_sweep(sbl, dev) if rank == 0 and not args.no_configs else None
     rms_front = _rmsnorm_front(sbl, dev, hbm_peak) if rank == 0 and not args.no_configs else None
     mask_mon = _mask_monitor_bench(sbl, dev, hbm_peak) if rank == 0 and not args.no_configs else None
+    ste_bwd = _ste_backward_bench(sbl, dev) if rank == 0 and not args.no_configs else None
     launches_per_step = len(layers) * (1 + 2 + 1)  # prep + (quant + tcgen05 GEMM) + fused decode
     value = _throughput(world, K, total_s)
     out = {
@@ -716,6 +717,7 @@ def run_ours(args, rank, world, dev):
         "configs": configs,
         "rmsnorm_front": rms_front,
         "mask_monitor": mask_mon,
+        "ste_backward": ste_bwd,
         "phases": phases,
         "e2e": {"value": world * TOKENS_PER_STEP * K_e2e / e2e_s, "steps": K_e2e, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
