@@ -817,3 +817,50 @@ def test_ste_backward_worked_block():
         np.testing.assert_allclose(dX[0], c["dX"], rtol=1e-6, atol=0)
         np.testing.assert_allclose(dW[0], c["dW"], rtol=1e-6, atol=0)
         np.testing.assert_allclose(dWt[0], c["dW_ternary"], rtol=1e-6, atol=0)
+
+
+# --------------------------------------------------------------------------
+# property-based: adversarial weight values against the brute force
+# --------------------------------------------------------------------------
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+# exact ties, both zeros, tiny and huge magnitudes, and values on the 0.5 * scale threshold
+_POOL = (0.0, -0.0, 1e-30, -1e-30, 1e-7, 0.25, -0.25, 0.5, -0.5, 0.75, 1.0, -1.0, 1.5, 3.0e4, -3.0e4, 1e30)
+
+
+@st.composite
+def _weight_case(draw):
+    n, m = draw(st.sampled_from(PATTERNS))
+    O = draw(st.integers(1, 3))
+    K = 8 * draw(st.integers(1, 3))
+    elem = st.one_of(st.sampled_from(_POOL), st.floats(-2.0, 2.0, width=32, allow_subnormal=False))
+    vals = draw(st.lists(elem, min_size=O * K, max_size=O * K))
+    return np.array(vals, np.float32).reshape(O, K), n, m
+
+
+@settings(max_examples=150, deadline=None)
+@given(_weight_case())
+def test_prepare_matches_brute_force_on_adversarial_values(case):
+    W, n, m = case
+    packed, scale, mbits, Wt = oracle.prepare_weights(W, n, m)
+    mask_b, scale_b, Wt_b = _brute_prepare(W, n, m)
+    assert np.array_equal(np.unpackbits(mbits, axis=1, bitorder="little").astype(bool), mask_b)
+    assert np.array_equal(scale.view(np.uint32), scale_b.view(np.uint32))
+    assert np.array_equal(Wt, Wt_b)
+    assert np.array_equal(packed, _bitstring_pack(Wt_b))
+
+
+@settings(max_examples=150, deadline=None)
+@given(st.lists(st.one_of(st.sampled_from(_POOL), st.floats(-1e4, 1e4, width=32, allow_subnormal=False)),
+                min_size=16, max_size=48).filter(lambda v: len(v) % 16 == 0))
+def test_quant_invariants_on_adversarial_values(vals):
+    x = np.array([vals], np.float32)
+    xq, s = oracle.quant_act(x)
+    amax = float(np.max(np.abs(x)))
+    assert s[0] == np.float32(127.0) / max(np.float32(amax), np.float32(1e-5))
+    exact = x.astype(np.float64) * float(s[0])
+    assert np.all(np.abs(xq - exact) <= 0.5 + 2.0 ** -17 * np.abs(exact))
+    assert xq.min() >= -127 and xq.max() <= 127
+    if amax >= 1e-5:
+        assert abs(int(xq[0, np.argmax(np.abs(x[0]))])) == 127
