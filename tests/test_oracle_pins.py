@@ -864,3 +864,33 @@ def test_quant_invariants_on_adversarial_values(vals):
     assert xq.min() >= -127 and xq.max() <= 127
     if amax >= 1e-5:
         assert abs(int(xq[0, np.argmax(np.abs(x[0]))])) == 127
+
+
+@settings(max_examples=60, deadline=None)
+@given(st.sampled_from(PATTERNS), st.integers(1, 6), st.sampled_from([16, 32]), st.integers(0, 5),
+       st.integers(0, 2 ** 16), st.booleans())
+def test_ste_backward_matches_autograd_on_random_shapes(nm, O, K, T, seed, tern):
+    """Any shape, the empty token set included: float64 autograd through the
+    straight-through surrogate agrees with the oracle's gradients."""
+    import torch
+    n, m = nm
+    f64 = torch.float64
+    W = synthetic.latent_weights(O, K, seed=seed, tag="hyp")
+    _, x = synthetic.activations(T, K, seed=seed, tag="hyp")
+    dY = synthetic.output_grads(T, O, seed=seed, tag="hyp")
+    _, scale, _, Wt = oracle.prepare_weights(W, n, m)
+    xq, s = oracle.quant_act(x) if T else (np.zeros((0, K), np.int8), np.zeros(0, np.float32))
+    xl = torch.tensor(x, dtype=f64, requires_grad=True)
+    Wl = torch.tensor(W, dtype=f64, requires_grad=True)
+    x_hat = xl + (torch.tensor(xq, dtype=f64) / torch.tensor(s, dtype=f64)[:, None] - xl).detach()
+    wq = torch.tensor(Wt, dtype=f64)
+    sc = torch.tensor(scale, dtype=f64)
+    if tern:
+        y = (x_hat @ (Wl + (wq - Wl).detach()).T) * sc[None, :]
+    else:
+        y = x_hat @ (Wl + (wq * sc[:, None] - Wl).detach()).T
+    (y * torch.tensor(dY, dtype=f64)).sum().backward()
+    dX, dW = oracle.ste_backward(dY, xq, s, Wt, scale, dw_ternary=tern)
+    gx = xl.grad.numpy() if xl.grad is not None else np.zeros((T, K))
+    np.testing.assert_allclose(dX, gx, rtol=1e-12, atol=1e-12 * (np.abs(gx).max(initial=0.0) + 1e-300))
+    np.testing.assert_allclose(dW, Wl.grad.numpy(), rtol=1e-12, atol=1e-12 * (np.abs(dW).max(initial=0.0) + 1e-300))
