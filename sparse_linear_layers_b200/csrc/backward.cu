@@ -17,7 +17,8 @@
 // ternary codes decoded while staging, or int8 activations), accumulated in
 // fp32 with fused multiply-adds: the products with {-1, 0, 1} or an int8 are
 // exact up to the fma's single rounding, so every output is within
-// (n + 2) * 2^-24 * sum |terms| of the exact value for a reduction of length n.
+// (n + 2) * 2^-24 * sum |terms| of the exact value for a reduction of length n
+// ((n + 3) with the extra row-scale product of the ternary form).
 // One CTA computes a 128 x 128 output tile C[i, j] = sum_r A[r, i] * B[r, j]
 // on the CUDA cores (16 x 16 threads, 8 x 8 outputs each), staging 16-deep
 // slices of A and B in two shared-memory buffers: the next slice is loaded
