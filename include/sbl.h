@@ -206,9 +206,10 @@ enum { SBL_BWD_DW_TERNARY = 1 };
  *              y = (x~ . W~^T) * beta * gamma / 127, as its module returns it).
  * fp32 arithmetic with fused multiply-adds in an unspecified order: each
  * output is within (n + 2) * 2^-24 * sum |terms| of the exact value, n the
- * reduction length (O for dX, T for dW; n + 3 for SBL_BWD_DW_TERNARY).  Empty reductions write zeros
- * (dW for T == 0, dX for O == 0).  Only the pointers the requested outputs
- * read must be valid.  At least one of dX, dW must be non-NULL.
+ * reduction length (O for dX, T for dW; n + 3 for SBL_BWD_DW_TERNARY).
+ * Empty reductions write zeros (dW for T == 0, dX for O == 0).  Only the
+ * pointers the requested outputs read must be valid.  At least one of dX, dW
+ * must be non-NULL.
  * K % 16 == 0; any T, O >= 0.  Asynchronous on `stream`; no workspace.
  */
 sbl_status sbl_linear_backward(const float* dY, int64_t T, int64_t O, const int8_t* x_q, const float* s_tok,
