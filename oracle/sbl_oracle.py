@@ -38,12 +38,10 @@ with its reason in the design notes):
   2 (k % 4) .. 2 (k % 4) + 1; mask bits: bit k % 8 of byte k // 8;
 * dequantisation in double: y = acc * scale / s_t;
 * RMSNorm (the guide's module normalises x with torch's RMSNorm before the
-  absmax; the pages give no arithmetic order): float32 throughout, every step
-  an IEEE-rounded operation; the sum of squares in a fixed order (lane l of
-  32 sums, in increasing k, the squares of the 16-element blocks b with
-  b % 32 == l; the 32 lane sums are combined by an xor butterfly at offsets
-  16, 8, 4, 2, 1); mean = sum / K; inv = 1 / sqrt(mean + eps);
-  x_norm = (x * inv) * g.
+  absmax; the pages give no arithmetic order): the sum of squares is the
+  exact sum rounded once to float32, which no summation order changes; then
+  float32 steps, each an IEEE-rounded operation: mean = sum / K;
+  inv = 1 / sqrt(mean + eps); x_norm = (x * inv) * g.
 * training (straight-through) backward: every quantiser acts as the identity,
   so dX = dY . (scale * W_t) and dW = dY^T . (x_q / s_t) over all positions,
   masked ones included; optionally (the guide's module) dW taken at the
@@ -200,32 +198,66 @@ def quant_act(x: np.ndarray):
     return np.clip(q, -128, 127).astype(np.int8), s
 
 
-RMS_LANES = 32
-RMS_BLOCK = 16
+def round_exact_to_f32(num: int, exp2: int) -> np.float32:
+    """The float32 nearest to the exact value num * 2**exp2 (num >= 0 an
+    integer), ties to the even significand; values at or past the float32
+    overflow threshold give +inf.  A float32 keeps 24 significant bits down to
+    2**-126 and a fixed spacing of 2**-149 below it."""
+    if num < 0:
+        raise ValueError("num must be >= 0")
+    if num == 0:
+        return np.float32(0.0)
+    e = num.bit_length() - 1 + exp2           # the value lies in [2**e, 2**(e + 1))
+    q = max(e - 23, -149)                      # weight of the last bit float32 keeps there
+    drop = q - exp2
+    if drop <= 0:
+        m = num << -drop
+    else:
+        m = num >> drop
+        rest = num - (m << drop)
+        half = 1 << (drop - 1)
+        if rest > half or (rest == half and m & 1):
+            m += 1
+    if m.bit_length() - 1 + q >= 128:
+        return np.float32(np.inf)
+    return np.float32(math.ldexp(m, q))
 
 
 def rms_sumsq(x: np.ndarray) -> np.ndarray:
-    """float32 [T]: the sum of x_k^2 over each token in the fixed float32 order.
+    """float32 [T]: sum_k x_k^2 of every token, formed exactly and rounded once
+    to float32 (nearest, ties to even; +inf past the float32 range).
 
-    Lane l (0..31) adds, in increasing k, the squares of the elements of the
-    16-element blocks b with b % 32 == l, one float32 rounding per addition
-    (a bf16 value's square is exact in float32 unless it underflows, where it
-    is rounded like any float32 product); the 32 lane sums are then combined
-    by an xor butterfly at offsets 16, 8, 4, 2, 1 (lane 0's value is taken).
+    The sum of squares of torch's RMSNorm (the guide's SparseBitLinear module
+    listing), whose order the pages leave open; the exact sum is independent of
+    it.  ``x`` holds bf16 values (widened to float32): each is
+    x = M * 2**(E - 134), M its 8-bit significand (implicit bit included) and
+    E = max(biased exponent, 1), so x**2 = M**2 * 2**(2E - 268) is an integer
+    multiple of 2**-266 and the sum is an exact integer in that unit: the
+    squares are gathered per exponent (sums of M**2, exact) and the
+    per-exponent totals added as Python integers.
     """
     x = np.asarray(x, dtype=np.float32)
     T, K = x.shape
-    if K % RMS_BLOCK:
-        raise ValueError("K must be a multiple of 16")
-    part = np.zeros((T, RMS_LANES), np.float32)
-    for k in range(K):
-        lane = (k // RMS_BLOCK) % RMS_LANES
-        v = x[:, k]
-        part[:, lane] = (part[:, lane] + (v * v).astype(np.float32)).astype(np.float32)
-    idx = np.arange(RMS_LANES)
-    for off in (16, 8, 4, 2, 1):
-        part = (part + part[:, idx ^ off]).astype(np.float32)
-    return part[:, 0].copy()
+    u = x.view(np.uint32)
+    if np.any(u & 0xFFFF):
+        raise ValueError("x must hold bf16 values")
+    mag = (u >> 16) & 0x7FFF
+    if np.any(mag >= 0x7F80):
+        raise ValueError("non-finite input")
+    bexp = mag >> 7
+    M = np.where(bexp > 0, (mag & 0x7F) | 0x80, mag & 0x7F).astype(np.int64)
+    E = np.maximum(bexp, 1).astype(np.int64)            # 1 .. 254
+    # per-exponent sums of M**2: each below 2**16 * K < 2**53, so the float64
+    # accumulation of bincount is exact
+    idx = (np.arange(T, dtype=np.int64)[:, None] * 255 + E).ravel()
+    per_exp = np.bincount(idx, weights=(M * M).ravel().astype(np.float64), minlength=T * 255)
+    per_exp = per_exp.reshape(T, 255).astype(np.int64)
+    out = np.empty(T, np.float32)
+    for t in range(T):
+        nz = np.nonzero(per_exp[t])[0]
+        total = sum(int(per_exp[t, e]) << (2 * int(e) - 2) for e in nz)   # units of 2**-266
+        out[t] = round_exact_to_f32(total, -266)
+    return out
 
 
 def rmsnorm(x: np.ndarray, g: np.ndarray, eps: float) -> np.ndarray:
@@ -235,8 +267,10 @@ def rmsnorm(x: np.ndarray, g: np.ndarray, eps: float) -> np.ndarray:
     normalised by RMSNorm before the absmax) and its SparseBitLinear module
     listing (torch RMSNorm over the input features, elementwise weight g,
     default eps = float32 machine epsilon).  Every step is one IEEE float32
-    operation: the sum of squares of :func:`rms_sumsq`, a division by K, an
-    addition of eps, a square root, a division of 1 by it, and two products.
+    operation after the exact sum of squares of :func:`rms_sumsq`: a division
+    by K, an addition of eps, a square root, a division of 1 by it, and two
+    products.  A sum of squares past the float32 range is +inf, which makes
+    every normalised value 0 (the library flags such a token).
     """
     x = np.asarray(x, dtype=np.float32)
     g = np.asarray(g, dtype=np.float32)

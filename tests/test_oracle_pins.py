@@ -10,8 +10,11 @@
   group, sign agreement, packed size O*K/4, argmax token element -> +-127);
 * the guide's own rescale form y = acc * beta * gamma / 127;
 * RMSNorm front end: torch's rms_norm in float64 (the library routine the
-  guide's module calls), hand-derived float32 sums that fix the summation
-  order, constant rows, and invariance under x -> 4x.
+  guide's module calls); the sum of squares against exact rational sums
+  (fractions.Fraction) rounded by a nearest-float search, hand-derived sums at
+  float32 rounding boundaries (ties, a double-rounding trap, subnormal and
+  overflowing squares) and invariance under any reordering; constant rows,
+  and invariance under x -> 4x.
 
 Each plausible mistake (a reversed input index, scale over all weights, half away
 from zero, ties to the higher index, MSB-first packing, a dropped clamp, a sign
@@ -403,32 +406,74 @@ def pin_rms_library(o):
             assert np.all(np.abs(got - ref) <= 2e-5 * np.abs(ref) + 1e-30)
 
 
-def pin_rms_order(o):
-    """The float32 order of the sum of squares, from hand-derived values.
+def _bf16_row(vals, K=None):
+    x = np.zeros((1, K or len(vals)), np.float32)
+    x[0, :len(vals)] = np.asarray(vals, np.float64).astype(np.float32)
+    assert not np.any(x.view(np.uint32) & 0xFFFF), "test values must be bf16"
+    return x
 
-    K = 16, x = [4096, 1 x 15]: one lane adds 2^24 then fifteen 1s; each sum
-    2^24 + 1 is a tie between 2^24 and 2^24 + 2 and rounds to even, 2^24.
-    K = 512, x_0 = 4096 and the first element of blocks 1..31 = 1: lane l holds
-    block l; the butterfly at 16, 8, 4, 2, 1 gives lane 0 2^24 (2^24 + 1 ties
-    to even), then 2^24 + 2, + 4, + 8, + 16: 16777246 (the exact sum is
-    16777247, a sequential sum 16777216).
-    K = 512, x_0 = 4096, first elements of blocks 16 and 24 = 1: offset 16
-    first adds one 1 to 2^24 (a tie: 2^24), and the other reaches lane 0 alone
-    at offset 8 (2^24 again): 16777216; the butterfly taken from offset 1 up
-    would pair the two 1s first and give 16777218."""
-    x = np.zeros((1, 16), np.float32)
-    x[0, 0] = 4096.0
-    x[0, 1:] = 1.0
-    assert float(o.rms_sumsq(x)[0]) == 16777216.0
+
+def _nearest_f32(q: Fraction) -> np.float32:
+    """The float32 nearest to the rational q >= 0 (ties to the even bit
+    pattern; +inf from the overflow threshold (2 - 2^-24) * 2^127 on), by
+    comparing the distances of the candidates around the double nearest to q."""
+    if q >= Fraction(2 ** 128 - 2 ** 103):
+        return np.float32(np.inf)
+    c0 = np.float32(float(q))
+    cands = {c0, np.nextafter(c0, np.float32(0)), np.nextafter(c0, np.float32(np.inf))}
+    cands = [c for c in cands if np.isfinite(c)]
+    return min(cands, key=lambda c: (abs(Fraction(float(c)) - q), int(np.asarray(c).view(np.uint32)) & 1))
+
+
+def pin_rms_exact(o):
+    """The sum of squares is the exact sum rounded once to float32.
+
+    Hand-derived (float32 spacing is 2 between 2^24 and 2^25):
+      [4096, 1]: 2^24 + 1 is a tie between 2^24 and 2^24 + 2 -> even 2^24
+        (half away from zero would give 2^24 + 2);
+      [4096, 1 x 15]: 16777231, a tie -> even 16777232 (a float32 running
+        sum stays at 2^24: every + 1 ties back down);
+      K = 512, x_0 = 4096, the first element of blocks 1..31 = 1: 16777247,
+        a tie -> 16777248 (32 float32 lane sums combined by a butterfly give
+        16777246);
+      [4096, 1, 2^-30]: 2^24 + 1 + 2^-60 lies above the tie -> 16777218;
+        the exact sum rounded to double first is the tie itself, which then
+        rounds to 2^24 (double rounding);
+      [2^-75]: 2^-150 is half the smallest float32 -> ties to 0;
+        [2^-75, 2^-75]: 2^-149 exactly;
+      [2^64]: 2^128 overflows -> +inf; [1.5 * 2^63]: 1.125 * 2^127 exactly.
+    Brute force: random rows mixing bf16 subnormals, tiny, ordinary and large
+    magnitudes, against sum(Fraction(x)^2) rounded by a nearest-float search.
+    Any reordering of a row gives the same float."""
+    cases = [
+        ([4096.0, 1.0], 16777216.0),
+        ([4096.0] + [1.0] * 15, 16777232.0),
+        ([4096.0, 1.0, 2.0 ** -30], 16777218.0),
+        ([2.0 ** -75], 0.0),
+        ([2.0 ** -75, 2.0 ** -75], 2.0 ** -149),
+        ([2.0 ** 64], math.inf),
+        ([1.5 * 2.0 ** 63], 1.125 * 2.0 ** 127),
+    ]
+    for vals, want in cases:
+        assert float(o.rms_sumsq(_bf16_row(vals, K=16 * ((len(vals) + 15) // 16)))[0]) == want, vals
     x = np.zeros((1, 512), np.float32)
     x[0, 0] = 4096.0
     x[0, 16::16] = 1.0
-    assert float(o.rms_sumsq(x)[0]) == 16777246.0
-    x = np.zeros((1, 512), np.float32)
-    x[0, 0] = 4096.0
-    x[0, 16 * 16] = 1.0
-    x[0, 24 * 16] = 1.0
-    assert float(o.rms_sumsq(x)[0]) == 16777216.0
+    assert float(o.rms_sumsq(x)[0]) == 16777248.0
+    rng = np.random.default_rng(11)
+    pool = [0.0, 2.0 ** -133, 3 * 2.0 ** -133, 2.0 ** -126, 1e-30, 1e-12, 1e-4, 0.5, 1.0, 3.0, 1e4, 1e15, 3e18]
+    rows = []
+    for _ in range(40):
+        K = int(rng.choice([16, 32, 48]))
+        v = rng.choice(pool, K) * rng.choice([-1.0, 1.0], K) * (1 + rng.integers(0, 128, K) / 128.0)
+        v = synthetic.bf16_bits_to_f32(synthetic.f32_to_bf16_bits(v.astype(np.float32)))
+        rows.append(v)
+    for v in rows:
+        want = _nearest_f32(sum(Fraction(float(e)) ** 2 for e in v))
+        got = o.rms_sumsq(v[None, :])[0]
+        assert got.view(np.uint32) == want.view(np.uint32), (v, got, want)
+        perm = rng.permutation(v.size)
+        assert o.rms_sumsq(v[None, perm])[0].view(np.uint32) == got.view(np.uint32)
 
 
 def pin_rms_closed_forms(o):
@@ -453,7 +498,7 @@ def pin_rms_closed_forms(o):
 
 
 def test_rms_pins():
-    for pin in (pin_rms_library, pin_rms_order, pin_rms_closed_forms):
+    for pin in (pin_rms_library, pin_rms_exact, pin_rms_closed_forms):
         pin(oracle)
 
 
@@ -482,16 +527,51 @@ def _rms_seq(x):
     return acc
 
 
-def _rms_butterfly_up(x):
+def _rms_lane_butterfly(x):
+    """32 float32 lane sums of 16-element blocks, combined by an xor butterfly
+    (an order-dependent float32 sum)."""
     x = np.asarray(x, np.float32)
     part = np.zeros((x.shape[0], 32), np.float32)
     for k in range(x.shape[1]):
         lane = (k // 16) % 32
         part[:, lane] = (part[:, lane] + (x[:, k] * x[:, k]).astype(np.float32)).astype(np.float32)
     idx = np.arange(32)
-    for off in (1, 2, 4, 8, 16):
+    for off in (16, 8, 4, 2, 1):
         part = (part + part[:, idx ^ off]).astype(np.float32)
     return part[:, 0].copy()
+
+
+def _rms_fsum_then_f32(x):
+    """The exact sum rounded to double (fsum), then to float32: double rounding."""
+    x = np.asarray(x, np.float64)
+    return np.array([np.float32(math.fsum((r * r).tolist())) for r in x], np.float32)
+
+
+def _rms_ties_away(x):
+    """Exact sum, but ties rounded away from zero."""
+    x = np.asarray(x, np.float32)
+    out = np.empty(x.shape[0], np.float32)
+    for t, r in enumerate(x):
+        q = sum(Fraction(float(e)) ** 2 for e in r)
+        c = np.float32(float(q))
+        lo = c if Fraction(float(c)) <= q else np.nextafter(c, np.float32(0))
+        hi = np.nextafter(lo, np.float32(np.inf))
+        dlo, dhi = q - Fraction(float(lo)), Fraction(float(hi)) - q
+        out[t] = hi if dhi <= dlo else lo
+    return out
+
+
+def _rms_flush_subnormal_squares(x):
+    """Exact sum of the squares, but squares below 2^-126 dropped."""
+    x = np.asarray(x, np.float32)
+    sq = np.where(np.abs(x.astype(np.float64)) ** 2 < 2.0 ** -126, np.float32(0), x)
+    return oracle.rms_sumsq(sq.astype(np.float32))
+
+
+def _rms_saturate(x):
+    """Exact sum, but an overflowing sum saturated at the largest float32."""
+    s = oracle.rms_sumsq(x)
+    return np.where(np.isinf(s), np.finfo(np.float32).max, s).astype(np.float32)
 
 
 def _rms_no_sqrt(x, g, eps):
@@ -519,7 +599,11 @@ def _rms_mean_k_minus_1(x, g, eps):
 
 RMS_MUTANTS = {
     "rms_sequential_sum": dict(rms_sumsq=_rms_seq),
-    "rms_butterfly_from_offset_1": dict(rms_sumsq=_rms_butterfly_up),
+    "rms_lane_butterfly": dict(rms_sumsq=_rms_lane_butterfly),
+    "rms_fsum_then_float32": dict(rms_sumsq=_rms_fsum_then_f32),
+    "rms_ties_away": dict(rms_sumsq=_rms_ties_away),
+    "rms_flush_subnormal_squares": dict(rms_sumsq=_rms_flush_subnormal_squares),
+    "rms_saturate_overflow": dict(rms_sumsq=_rms_saturate),
     "rms_no_sqrt": dict(rmsnorm=_rms_no_sqrt),
     "rms_eps_outside_sqrt": dict(rmsnorm=_rms_eps_outside),
     "rms_weight_dropped": dict(rmsnorm=_rms_no_weight),
@@ -531,7 +615,7 @@ RMS_MUTANTS = {
 def test_planted_rms_mistake_is_caught(name):
     o = _rms_ns(**RMS_MUTANTS[name])
     caught = []
-    for pin in (pin_rms_library, pin_rms_order, pin_rms_closed_forms):
+    for pin in (pin_rms_library, pin_rms_exact, pin_rms_closed_forms):
         try:
             pin(o)
         except (AssertionError, ValueError, IndexError):
