@@ -24,13 +24,38 @@ def _stream(stream: Optional[torch.cuda.Stream]) -> int:
     return s.cuda_stream
 
 
-def _need_cuda(t: torch.Tensor, name: str, dtype: torch.dtype) -> None:
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor")
+def _need_cuda(t: torch.Tensor, name: str, dtype: torch.dtype, shape=None, device=None) -> None:
+    """Raise ValueError unless ``t`` is a contiguous CUDA tensor of ``dtype``
+    (and, when given, exactly ``shape`` and on ``device``): the kernels write
+    and read through raw pointers, so a tensor of the wrong size or on another
+    GPU must never reach them."""
     if t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the other operands on {device}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+
+
+def _need_2d(t: torch.Tensor, name: str):
+    if t.dim() != 2:
+        raise ValueError(f"{name} must be 2-D, got shape {tuple(t.shape)}")
+    return t.shape
+
+
+def _need_weights(w: "PreparedWeights", device) -> None:
+    _need_cuda(w.packed, "packed", torch.uint8, (w.O, w.K // 4), device)
+    _need_cuda(w.row_scale, "row_scale", torch.float32, (w.O,), device)
+
+
+def _need_workspace(ws: torch.Tensor, device) -> None:
+    if ws.dim() != 1:
+        raise ValueError("workspace must be a 1-D uint8 tensor")
+    _need_cuda(ws, "workspace", torch.uint8, None, device)
 
 
 @dataclass
@@ -56,13 +81,18 @@ def sbl_prepare_weights(W: torch.Tensor, n: int, m: int, with_mask: bool = False
     ``scale_bf16`` the scale is rounded to bf16 (the halo card's storage) first;
     with ``scale_global`` one scale, the mean of |W| over the whole matrix (the
     guide's module listing), serves every row."""
+    O, K = _need_2d(W, "W")
     _need_cuda(W, "W", torch.float32)
-    O, K = W.shape
     if out is None:
         packed = torch.empty((O, K // 4), dtype=torch.uint8, device=W.device)
         scale = torch.empty((O,), dtype=torch.float32, device=W.device)
         mask = torch.empty((O, K // 8), dtype=torch.uint8, device=W.device) if with_mask else None
         out = PreparedWeights(packed, scale, n, m, K, mask)
+    if out.K != K or out.O != O:
+        raise ValueError(f"out holds [{out.O}, {out.K}] weights, W is [{O}, {K}]")
+    _need_weights(out, W.device)
+    if out.mask_bits is not None:
+        _need_cuda(out.mask_bits, "mask_bits", torch.uint8, (O, K // 8), W.device)
     mb = out.mask_bits.data_ptr() if out.mask_bits is not None else None
     check(lib.sbl_prepare_weights_ex(W.data_ptr(), O, K, n, m, out.packed.data_ptr(), out.row_scale.data_ptr(), mb,
                                      (_lib.SBL_PREP_SCALE_BF16 if scale_bf16 else 0) |
@@ -73,8 +103,8 @@ def sbl_prepare_weights(W: torch.Tensor, n: int, m: int, with_mask: bool = False
 
 def sbl_quant_act(x: torch.Tensor, stream: Optional[torch.cuda.Stream] = None):
     """Per-token absmax int8 quantisation: returns (x_q int8 [T,K], s_tok fp32 [T])."""
+    T, K = _need_2d(x, "x")
     _need_cuda(x, "x", torch.bfloat16)
-    T, K = x.shape
     xq = torch.empty((T, K), dtype=torch.int8, device=x.device)
     s = torch.empty((T,), dtype=torch.float32, device=x.device)
     check(lib.sbl_quant_act(x.data_ptr(), T, K, xq.data_ptr(), s.data_ptr(), _stream(stream)), "sbl_quant_act")
@@ -87,9 +117,9 @@ RMSNORM_EPS_F32 = 2.0 ** -23  # torch's default RMSNorm epsilon for float32 (mac
 def sbl_rmsnorm_quant_act(x: torch.Tensor, g: torch.Tensor, eps: float = RMSNORM_EPS_F32,
                           stream: Optional[torch.cuda.Stream] = None):
     """RMSNorm (weight g, fp32 [K]) then per-token absmax int8: (x_q int8 [T,K], s_tok fp32 [T])."""
+    T, K = _need_2d(x, "x")
     _need_cuda(x, "x", torch.bfloat16)
-    _need_cuda(g, "g", torch.float32)
-    T, K = x.shape
+    _need_cuda(g, "g", torch.float32, (K,), x.device)
     xq = torch.empty((T, K), dtype=torch.int8, device=x.device)
     s = torch.empty((T,), dtype=torch.float32, device=x.device)
     check(lib.sbl_rmsnorm_quant_act(x.data_ptr(), g.data_ptr(), float(eps), T, K, xq.data_ptr(), s.data_ptr(),
@@ -111,21 +141,23 @@ def sbl_linear(x: torch.Tensor, w: PreparedWeights, out_dtype: torch.dtype = tor
                workspace: Optional[torch.Tensor] = None, path: str = "auto",
                stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
     """y = dequant(int8(x) . W_t^T); ``acc_out`` (int32 [T,O]) receives the integer accumulators."""
+    T, K = _need_2d(x, "x")
     _need_cuda(x, "x", torch.bfloat16)
-    T, K = x.shape
     if K != w.K:
         raise ValueError(f"x has K={K}, weights were prepared with K={w.K}")
+    _need_weights(w, x.device)
     O = w.O
     if y is None:
         y = torch.empty((T, O), dtype=out_dtype, device=x.device)
     if y.dtype not in (torch.float32, torch.bfloat16):
         raise ValueError("y must be float32 or bfloat16")
-    _need_cuda(y, "y", y.dtype)
+    _need_cuda(y, "y", y.dtype, (T, O), x.device)
     ydt = _lib.SBL_F32 if y.dtype == torch.float32 else _lib.SBL_BF16
     if acc_out is not None:
-        _need_cuda(acc_out, "acc_out", torch.int32)
+        _need_cuda(acc_out, "acc_out", torch.int32, (T, O), x.device)
     if workspace is None:
         workspace = workspace_for(T, K, O, w.n, w.m, x.device)
+    _need_workspace(workspace, x.device)
     check(lib.sbl_linear_path(x.data_ptr(), T, K, w.packed.data_ptr(), w.row_scale.data_ptr(), O, w.n, w.m,
                               y.data_ptr(), ydt, acc_out.data_ptr() if acc_out is not None else None,
                               workspace.data_ptr(), workspace.numel(), _PATHS[path], _stream(stream)),
@@ -138,22 +170,24 @@ def sbl_linear_rmsnorm(x: torch.Tensor, w: PreparedWeights, g: torch.Tensor, eps
                        acc_out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
                        path: str = "auto", stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
     """The guide module's forward: y = dequant(int8(RMSNorm(x; g, eps)) . W_t^T)."""
+    T, K = _need_2d(x, "x")
     _need_cuda(x, "x", torch.bfloat16)
-    _need_cuda(g, "g", torch.float32)
-    T, K = x.shape
     if K != w.K or g.numel() != K:
         raise ValueError(f"x has K={K}; weights were prepared with K={w.K}; g has {g.numel()} entries")
+    _need_cuda(g, "g", torch.float32, (K,), x.device)
+    _need_weights(w, x.device)
     O = w.O
     if y is None:
         y = torch.empty((T, O), dtype=out_dtype, device=x.device)
     if y.dtype not in (torch.float32, torch.bfloat16):
         raise ValueError("y must be float32 or bfloat16")
-    _need_cuda(y, "y", y.dtype)
+    _need_cuda(y, "y", y.dtype, (T, O), x.device)
     ydt = _lib.SBL_F32 if y.dtype == torch.float32 else _lib.SBL_BF16
     if acc_out is not None:
-        _need_cuda(acc_out, "acc_out", torch.int32)
+        _need_cuda(acc_out, "acc_out", torch.int32, (T, O), x.device)
     if workspace is None:
         workspace = workspace_for(T, K, O, w.n, w.m, x.device)
+    _need_workspace(workspace, x.device)
     check(lib.sbl_linear_rmsnorm(x.data_ptr(), g.data_ptr(), float(eps), T, K, w.packed.data_ptr(),
                                  w.row_scale.data_ptr(), O, w.n, w.m, y.data_ptr(), ydt,
                                  acc_out.data_ptr() if acc_out is not None else None, workspace.data_ptr(),
@@ -166,11 +200,9 @@ def sbl_mask_monitor(old_bits: torch.Tensor, new_bits: torch.Tensor, K: int, n: 
     """Mask change and verification on the device: (totals int64 [2] = [changed
     positions, groups not keeping exactly N], row_changed int32 [O] or None).
     Nothing is copied to the host."""
-    _need_cuda(old_bits, "old_bits", torch.uint8)
-    _need_cuda(new_bits, "new_bits", torch.uint8)
-    O = old_bits.shape[0]
-    if old_bits.shape != (O, K // 8) or new_bits.shape != (O, K // 8):
-        raise ValueError("mask bitmaps must both be uint8 [O, K/8]")
+    O = _need_2d(old_bits, "old_bits")[0]
+    _need_cuda(old_bits, "old_bits", torch.uint8, (O, K // 8))
+    _need_cuda(new_bits, "new_bits", torch.uint8, (O, K // 8), old_bits.device)
     totals = torch.empty(2, dtype=torch.int64, device=old_bits.device)
     rows = torch.empty(O, dtype=torch.int32, device=old_bits.device) if per_row else None
     check(lib.sbl_mask_monitor(old_bits.data_ptr(), new_bits.data_ptr(), O, K, n, m, totals.data_ptr(),
@@ -188,22 +220,24 @@ def sbl_linear_backward(dY: torch.Tensor, x_q: torch.Tensor, s_tok: torch.Tensor
     (``dw_ternary``: dW rows scaled by scale_o once more, the guide module's form).
     ``x_q``/``s_tok`` are the forward's quantised activations in natural order
     (sbl_quant_act or sbl_rmsnorm_quant_act)."""
-    _need_cuda(dY, "dY", torch.float32)
-    _need_cuda(x_q, "x_q", torch.int8)
-    _need_cuda(s_tok, "s_tok", torch.float32)
-    T, O = dY.shape
+    T, O = _need_2d(dY, "dY")
     K = w.K
     if O != w.O or x_q.shape != (T, K) or s_tok.shape != (T,):
         raise ValueError(f"dY {tuple(dY.shape)}, x_q {tuple(x_q.shape)} and s_tok {tuple(s_tok.shape)} do not match "
                          f"weights with O={w.O}, K={K}")
+    _need_cuda(dY, "dY", torch.float32)
+    dev = dY.device
+    _need_cuda(x_q, "x_q", torch.int8, (T, K), dev)
+    _need_cuda(s_tok, "s_tok", torch.float32, (T,), dev)
+    _need_weights(w, dev)
     if not (need_dx or need_dw):
         raise ValueError("ask for dX, dW or both")
     if need_dx:
-        dX = torch.empty((T, K), dtype=torch.float32, device=dY.device) if dX is None else dX
-        _need_cuda(dX, "dX", torch.float32)
+        dX = torch.empty((T, K), dtype=torch.float32, device=dev) if dX is None else dX
+        _need_cuda(dX, "dX", torch.float32, (T, K), dev)
     if need_dw:
-        dW = torch.empty((O, K), dtype=torch.float32, device=dY.device) if dW is None else dW
-        _need_cuda(dW, "dW", torch.float32)
+        dW = torch.empty((O, K), dtype=torch.float32, device=dev) if dW is None else dW
+        _need_cuda(dW, "dW", torch.float32, (O, K), dev)
     check(lib.sbl_linear_backward(dY.data_ptr(), T, O, x_q.data_ptr(), s_tok.data_ptr(), K, w.packed.data_ptr(),
                                   w.row_scale.data_ptr(), dX.data_ptr() if need_dx else None,
                                   dW.data_ptr() if need_dw else None,
