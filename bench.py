@@ -14,7 +14,7 @@ per GPU (the 2048-token prefill batch plus one decode token).
 
 Under torchrun each rank runs its own copy of the step on its own GPU (the
 forward has no cross-GPU exchange): weak scaling, timed as the max over ranks.
-``--impl reference`` times the CPU oracle on a bounded sample of the same step.
+``--impl reference`` times the CPU oracle on full steps of the same workload.
 """
 from __future__ import annotations
 
@@ -725,41 +725,60 @@ def run_ours(args, rank, world, dev):
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline_sample(budget_s=args.cpu_budget)
+        out["cpu_baseline"] = cpu_baseline_sample()
     return out
 
 
 # --------------------------------------------------------------------------- oracle arm
 
-def cpu_baseline_sample(budget_s=20.0, sample_tokens=32):
-    """The CPU oracle on a bounded sample of the step: full weight preparation of
-    all seven projections plus ``sample_tokens`` of the 2048 prefill tokens and the
-    decode token; the step time is extrapolated to 2048 + 1 tokens."""
-    import oracle
-    threads = _cpu_threads()
-    t_prep = t_lin = 0.0
-    tok = 0
+def _oracle_inputs():
+    """The step's inputs for the oracle: the same seeded draws as the GPU step."""
+    out = []
     for nm, K, O in synthetic.QWEN05_LAYER:
         W = synthetic.latent_weights(O, K, seed=0, tag=f"bench-{nm}")
         _, xv = synthetic.activations(T_PREFILL, K, seed=0, tag=f"bench-x-{nm}")
         _, x1 = synthetic.activations(T_DECODE, K, seed=0, tag=f"bench-x1-{nm}")
+        out.append((W, xv, x1))
+    return out
+
+
+def oracle_step(inputs):
+    """One full step of the CPU oracle, nothing sampled or extrapolated: the
+    weight preparation of all seven projections, the 2048-token prefill
+    forward and the one-token decode forward of each.  Returns
+    (seconds, prep seconds, contraction seconds)."""
+    import oracle
+    t_prep = t_lin = 0.0
+    for W, xv, x1 in inputs:
         a = time.perf_counter()
         _, scale, _, Wt = oracle.prepare_weights(W, N, M)
         b = time.perf_counter()
-        oracle.linear(xv[:sample_tokens], Wt, scale)
+        oracle.linear(xv, Wt, scale)
         oracle.linear(x1, Wt, scale)
         c = time.perf_counter()
         t_prep += b - a
         t_lin += c - b
-    tok = sample_tokens + T_DECODE
-    step_s = t_prep + t_lin * TOKENS_PER_STEP / tok
-    # dense-equivalent integer ops of the sampled contractions (2 * T * O * K per projection)
-    lin_ops = 2.0 * tok * sum(O * K for _, K, O in synthetic.QWEN05_LAYER)
-    return {"value": TOKENS_PER_STEP / step_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "contraction_gops": lin_ops / t_lin / 1e9 if t_lin > 0 else None,
-            "sample": f"weight prep of all 7 projections + {sample_tokens} of 2048 prefill tokens + the decode "
-                      f"token; step time extrapolated to 2049 tokens (measured prep {t_prep:.2f}s, "
-                      f"linear {t_lin:.2f}s)"}
+    return t_prep + t_lin, t_prep, t_lin
+
+
+def cpu_baseline_sample(budget_s=None, sample_tokens=None):
+    """The CPU oracle timed on full steps of the workload (2049 tokens, all seven
+    projections from latent weights): once on every host core the BLAS uses
+    and once on one thread, after one untimed step."""
+    import threadpoolctl
+    inputs = _oracle_inputs()
+    oracle_step(inputs)  # untimed: first-touch and library warm-up
+    all_s, prep_s, lin_s = oracle_step(inputs)
+    cores = _cpu_threads()
+    with threadpoolctl.threadpool_limits(limits=1):
+        one_s, _, _ = oracle_step(inputs)
+    ops = 2.0 * TOKENS_PER_STEP * sum(O * K for _, K, O in synthetic.QWEN05_LAYER)
+    return {"value": TOKENS_PER_STEP / all_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "single_thread": {"value": TOKENS_PER_STEP / one_s, "unit": "tokens/s", "cores": 1},
+            "contraction_gops": ops / lin_s / 1e9,
+            "sample": f"one full step (7 weight preparations + 2048 prefill tokens + 1 decode token), measured, "
+                      f"not extrapolated: {all_s:.2f} s on {cores} threads (prep {prep_s:.2f} s, contraction "
+                      f"{lin_s:.2f} s), {one_s:.2f} s on 1 thread; host {os.cpu_count()} logical CPUs"}
 
 
 def _cpu_threads():
@@ -773,25 +792,28 @@ def _cpu_threads():
 
 
 def run_reference(args, rank, world):
+    """The oracle arm: W untimed and K timed full oracle steps on the host's
+    cores (rank 0 only; the other ranks exit without work)."""
     if rank != 0:
         return None
-    vals = []
+    inputs = _oracle_inputs()
     for _ in range(args.warmup):
-        cpu_baseline_sample(sample_tokens=8)
-    t0 = time.perf_counter()
+        oracle_step(inputs)
+    times = []
     for _ in range(args.steps):
-        r = cpu_baseline_sample(sample_tokens=8)
-        vals.append(r["value"])
-    wall = time.perf_counter() - t0
-    v = statistics.median(vals)
+        times.append(oracle_step(inputs)[0])
+    total = sum(times)
+    v = TOKENS_PER_STEP * args.steps / total
+    cores = _cpu_threads()
     return {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": 1e3 * TOKENS_PER_STEP / v, "higher_is_better": True,
+            "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": _config({"parallelism": "CPU oracle, rank 0 only"}), "impl": "reference",
-            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": _cpu_threads(), "kind": "oracle",
-                             "sample": r["sample"], "contraction_gops": r.get("contraction_gops")},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{args.steps} full oracle steps (7 weight preparations + 2048 prefill "
+                                       f"tokens + 1 decode token each), measured on {cores} threads"},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-            "wall_s": wall}
+            "wall_s": total}
 
 
 # --------------------------------------------------------------------------- plumbing
@@ -820,7 +842,6 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration sweep (profiling runs)")
     ap.add_argument("--only", choices=("rmsnorm_front", "mask_monitor", "ste_backward"),
