@@ -179,16 +179,100 @@ cudaError_t launch_quant(const uint16_t* x, long long T, long long K, int8_t* xq
 // The guide's SparseBitLinear module normalises x with RMSNorm before the
 // per-token absmax ("Mathematical Formulation of Sparse-BitLinear", activation
 // step, and the module listing): x_norm = x * (1 / sqrt(mean(x^2) + eps)) * g,
-// every step an IEEE float32 operation, then the absmax quantisation above.
-// One warp per token; lane l owns the 16-element blocks b with b % 32 == l.
-// The sum of squares follows a fixed order: each lane adds its squares in
-// increasing k, then an xor butterfly at offsets 16, 8, 4, 2, 1 combines the
-// lanes (every lane ends with the same total).  Pass 1 loads up to RB of a
-// lane's blocks at once (the rest in a loop); the absmax of the normalised
-// values and the quantisation then read x again (from L1) in a coalesced
-// mapping, which their order-free arithmetic allows.
-// Non-finite input shows as a non-finite sum of squares (a square that
-// overflows float32 does too) or normalised value, and sets the status bit.
+// then the absmax quantisation above.  The sum of squares is the exact sum
+// rounded once to float32 (no summation order changes it); every later step
+// is one IEEE float32 operation.
+// One warp per token; for the sum, lane l owns the 16-element blocks b with
+// b % 32 == l (up to RB of them held in registers, the rest read again); the
+// absmax of the normalised values and the quantisation then read x again
+// (from L1) in a coalesced mapping, which their order-free arithmetic allows.
+// Non-finite input, a sum of squares past the float32 range and a non-finite
+// normalised value set the status bit.
+//
+// Exact sum of squares.  A finite bf16 value is x = M * 2^(E - 134), with
+// E = max(biased exponent, 1) and M its 8-bit significand (implicit bit
+// included; M < 128 for subnormals); x^2 = M^2 * 2^(2E - 268) exactly.  With
+// E_max the token's largest E, n the elements a lane adds and
+// w = floor((48 - ceil(log2 n)) / 2):
+//  * window path: every x with E >= E_max - w times 2^c, c = w + 134 - E_max,
+//    is an integer y < 2^(8 + w) (a power-of-two product, exact in float32);
+//    y^2 < 2^(16 + 2w) is exact in float32 and converts exactly to a 64-bit
+//    integer, and n of them stay below 2^64, so the lane's uint64 sum A is
+//    exact.  Values with E_max - 2w <= E < E_max - w take the factor 2^(c + w)
+//    into a second sum B under the same bound.  A * 2^(2w) + B is the lane's
+//    sum as a 128-bit integer in units of 2^(-2c - 2w); the warp adds the
+//    lanes' integers (below 2^114).
+//  * limb path, for a token with a nonzero value below E_max - 2w or whose
+//    factor 2^c or 2^(c + w) is not a float32 (all |x| below about 2^-80):
+//    every square M^2 * 2^(2E - 2) (units of 2^-266) is added, as two 32-bit
+//    halves, into eighteen 64-bit shared-memory columns of 32-bit limbs
+//    (576 bits); the carries are resolved once at the end.
+// The integer is rounded to 53 bits by round-to-odd (the last kept bit is set
+// when any dropped bit is nonzero) and that double rounded to the nearest
+// float32.  Rounding to odd with two or more extra bits, then to nearest,
+// equals one rounding to nearest of the exact value (Boldo and Melquiond,
+// "Emulation of FMA and correctly rounded sums: proved algorithms using
+// rounding to odd", IEEE Trans. Computers 57(4), 2008); the float32 overflow
+// threshold and subnormal spacing are representable at 53 bits, so both
+// carry over.
+constexpr int kSqLimbs = 18;
+
+__device__ __forceinline__ double pow2d(int k) {  // 2^k for -1022 <= k <= 1023
+    return __longlong_as_double(static_cast<long long>(1023 + k) << 52);
+}
+
+// The integer hi * 2^64 + lo, times 2^e0, rounded to 53 bits by round-to-odd.
+__device__ __forceinline__ double u128_round_odd(uint64_t hi, uint64_t lo, int e0) {
+    uint64_t m;
+    int sh;  // weight of bit 0 of m, in bits of the integer
+    if (hi == 0) {
+        if ((lo >> 53) == 0) {
+            m = lo;
+            sh = 0;
+        } else {
+            const int lz = __clzll(static_cast<long long>(lo));  // at most 10
+            const uint64_t top = lo << lz;
+            m = (top >> 11) | ((top & 0x7FFull) != 0 ? 1ull : 0ull);
+            sh = 11 - lz;
+        }
+    } else {
+        const int lz = __clzll(static_cast<long long>(hi));
+        const uint64_t top = lz ? (hi << lz) | (lo >> (64 - lz)) : hi;
+        const uint64_t rest = lz ? (lo << lz) : lo;
+        m = (top >> 11) | (((top & 0x7FFull) | rest) != 0 ? 1ull : 0ull);
+        sh = 75 - lz;
+    }
+    return __ull2double_rn(m) * pow2d(e0 + sh);  // m < 2^53: both exact
+}
+
+// Resolve the carries of the limb columns (32-bit limbs in 64-bit words,
+// units of 2^-266) and round the integer to 53 bits by round-to-odd.
+__device__ double limbs_round_odd(const unsigned long long* col) {
+    uint32_t w[kSqLimbs];
+    unsigned long long carry = 0;
+#pragma unroll
+    for (int i = 0; i < kSqLimbs; ++i) {
+        const unsigned long long t = col[i] + carry;
+        w[i] = static_cast<uint32_t>(t);
+        carry = t >> 32;
+    }
+    int h = 3;
+    for (int i = kSqLimbs - 1; i > 3; --i)
+        if (w[i] != 0u) {
+            h = i;
+            break;
+        }
+    uint32_t sticky = 0;
+    for (int i = 0; i < h - 3; ++i) sticky |= w[i];
+    const uint64_t hi = (static_cast<uint64_t>(w[h]) << 32) | w[h - 1];
+    const uint64_t lo = ((static_cast<uint64_t>(w[h - 2]) << 32) | w[h - 3]) | (sticky ? 1ull : 0ull);
+    return u128_round_odd(hi, lo, -266 + 32 * (h - 3));
+}
+
+__device__ __forceinline__ void add128(uint64_t& hi, uint64_t& lo, uint64_t bhi, uint64_t blo) {
+    asm("add.cc.u64 %0, %0, %2;\n\taddc.u64 %1, %1, %3;" : "+l"(lo), "+l"(hi) : "l"(blo), "l"(bhi));
+}
+
 // Pairs of floats in one 64-bit register, for the sm_100 paired float
 // instructions (each half rounded exactly like the scalar IEEE operation).
 __device__ __forceinline__ uint64_t f2(float lo, float hi) {
@@ -202,11 +286,6 @@ __device__ __forceinline__ void f2split(uint64_t v, float& lo, float& hi) {
 __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
     uint64_t r;
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
 // Three-input max / min that propagate NaN.
@@ -235,33 +314,118 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_kernel(const uint16_t* __re
     const uint4* xr = reinterpret_cast<const uint4*>(x + t * K);
     const int nblk = static_cast<int>(K >> 4);
     uint4 v[RB][2];
-    // pass 1: sum of squares in the lane's k order
-    float ss = 0.f;
-    auto add_sq = [&](const uint4& a, const uint4& b) {
-        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint64_t p = f2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
-            float lo, hi;
-            f2split(mul2(p, p), lo, hi);  // squares of elements 2i and 2i + 1
-            ss = __fadd_rn(ss, lo);
-            ss = __fadd_rn(ss, hi);
-        }
-    };
 #pragma unroll
     for (int j = 0; j < RB; ++j) {
         const int b = lane + 32 * j;
         if (b < nblk) {
             v[j][0] = ldg_nc(xr + 2 * b);
             v[j][1] = ldg_nc(xr + 2 * b + 1);
+        } else {
+            v[j][0] = v[j][1] = make_uint4(0u, 0u, 0u, 0u);
         }
     }
+    // Apply f to every 32-bit word (two bf16 values) of the lane's blocks.
+    auto each_word = [&](auto&& f) {
 #pragma unroll
-    for (int j = 0; j < RB; ++j)
-        if (lane + 32 * j < nblk) add_sq(v[j][0], v[j][1]);
-    for (int b = lane + 32 * RB; b < nblk; b += 32) add_sq(ldg_nc(xr + 2 * b), ldg_nc(xr + 2 * b + 1));
+        for (int j = 0; j < RB; ++j) {
+            f(v[j][0].x); f(v[j][0].y); f(v[j][0].z); f(v[j][0].w);
+            f(v[j][1].x); f(v[j][1].y); f(v[j][1].z); f(v[j][1].w);
+        }
+        for (int b = lane + 32 * RB; b < nblk; b += 32) {
+            const uint4 a0 = ldg_nc(xr + 2 * b), a1 = ldg_nc(xr + 2 * b + 1);
+            f(a0.x); f(a0.y); f(a0.z); f(a0.w);
+            f(a1.x); f(a1.y); f(a1.z); f(a1.w);
+        }
+    };
+    // pass 0: largest magnitude and smallest nonzero magnitude (bf16 bits;
+    // the halves of a word are handled as 16-bit lanes, a zero maps to 0xFFFF)
+    uint32_t mx2 = 0, mn2 = 0xFFFFFFFFu;
+    each_word([&](uint32_t w) {
+        const uint32_t m2 = w & 0x7FFF7FFFu;
+        mx2 = __vmaxu2(mx2, m2);
+        mn2 = __vminu2(mn2, (m2 + 0x7FFF7FFFu) ^ 0x80008000u);  // per half: mag - 1, or 0xFFFF for 0
+    });
+    const uint32_t mx = __reduce_max_sync(0xFFFFFFFFu, max(mx2 & 0xFFFFu, mx2 >> 16));
+    const uint32_t mn = __reduce_min_sync(0xFFFFFFFFu, min(mn2 & 0xFFFFu, mn2 >> 16)) + 1u;
+
+    // pass 1: the exact sum of squares, rounded once to float32
+    float ss;
+    if (mx >= 0x7F80u) {
+        ss = __int_as_float(0x7FC00000);  // Inf or NaN in x
+    } else if (mx == 0u) {
+        ss = 0.f;
+    } else {
+        const int e_max = max(static_cast<int>(mx >> 7), 1), e_min = max(static_cast<int>(mn >> 7), 1);
+        const int per_lane = 16 * ((nblk + 31) >> 5);
+        const int win = (48 - (32 - __clz(per_lane - 1))) >> 1;
+        const int c = win + 134 - e_max;
+        uint64_t hi = 0, lo = 0;
+        int e0 = 0;
+        const bool one_window = e_max - e_min <= win && c <= 127;
+        const bool two_windows = !one_window && e_max - e_min <= 2 * win && c + win <= 127;
+        if (one_window) {
+            const float fc = __uint_as_float(static_cast<uint32_t>(127 + c) << 23);  // 2^c
+            const uint64_t c2 = f2(fc, fc);
+            uint64_t acc = 0;
+            each_word([&](uint32_t w) {
+                uint64_t y = mul2(f2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)), c2);
+                float q0, q1;
+                f2split(mul2(y, y), q0, q1);
+                acc += __float2ull_rz(q0) + __float2ull_rz(q1);
+            });
+            lo = acc;
+            e0 = -2 * c;
+        } else if (two_windows) {
+            const float fa = __uint_as_float(static_cast<uint32_t>(127 + c) << 23);        // 2^c
+            const float fb = __uint_as_float(static_cast<uint32_t>(127 + c + win) << 23);  // 2^(c + w)
+            const uint32_t thr = static_cast<uint32_t>(e_max - win) << 7;  // E >= E_max - w (here E_max - w >= 2)
+            uint64_t acc_a = 0, acc_b = 0;
+            each_word([&](uint32_t w) {
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xFFFFFFFFu, ss, off));
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t bits = h ? (w & 0xFFFF0000u) : (w << 16);
+                    const bool big = ((bits >> 16) & 0x7FFFu) >= thr;
+                    const float y = __fmul_rn(__uint_as_float(bits), big ? fa : fb);
+                    const uint64_t q = __float2ull_rz(__fmul_rn(y, y));
+                    acc_a += big ? q : 0ull;
+                    acc_b += big ? 0ull : q;
+                }
+            });
+            hi = acc_a >> (64 - 2 * win);
+            lo = acc_a << (2 * win);
+            add128(hi, lo, 0ull, acc_b);
+            e0 = -2 * c - 2 * win;
+        }
+        if (one_window || two_windows) {
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1)
+                add128(hi, lo, __shfl_xor_sync(0xFFFFFFFFu, hi, off), __shfl_xor_sync(0xFFFFFFFFu, lo, off));
+            ss = __double2float_rn(u128_round_odd(hi, lo, e0));
+        } else {
+            __shared__ unsigned long long sq_limbs[8][kSqLimbs];
+            unsigned long long* col = sq_limbs[warp];
+            if (lane < kSqLimbs) col[lane] = 0ull;
+            __syncwarp();
+            each_word([&](uint32_t w) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t mag = (h ? (w >> 16) : w) & 0x7FFFu;
+                    if (mag != 0u) {
+                        const uint32_t e = mag >> 7;
+                        const uint32_t M = e ? ((mag & 0x7Fu) | 0x80u) : mag;
+                        const uint32_t p = 2u * max(e, 1u) - 2u;  // M^2 * 2^p in units of 2^-266
+                        const unsigned long long t = static_cast<unsigned long long>(M * M) << (p & 31u);
+                        atomicAdd(col + (p >> 5), t & 0xFFFFFFFFull);
+                        atomicAdd(col + (p >> 5) + 1, t >> 32);
+                    }
+                }
+            });
+            __syncwarp();
+            float s0 = 0.f;
+            if (lane == 0) s0 = __double2float_rn(limbs_round_odd(col));
+            ss = __shfl_sync(0xFFFFFFFFu, s0, 0);
+        }
+    }
     const float ms = __fdiv_rn(ss, static_cast<float>(K));
     const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
 
@@ -307,7 +471,10 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_kernel(const uint16_t* __re
     // pairing layout a 16-element block's word q holds the even (q = 0, 2) or
     // odd (q = 1, 3) elements of lanes q & ~1 and q | 1, so neighbouring lanes
     // swap codes once and each stores the word at its own position.
-    const uint64_t s2 = f2(s, s), magic2 = f2(12582912.0f, 12582912.0f);
+    // The product x_norm * s and the rounding add are scalar IEEE operations
+    // (quant_code_bits): a paired multiply followed by a paired add was
+    // observed to round like one fused multiply-add, which decides ties of
+    // x_norm * s (exactly k + 1/2 after rounding, not before) the wrong way.
     uint32_t* out = reinterpret_cast<uint32_t*>(xq + t * K);
     for (int i = 0; i < nstripe; ++i) {
         const int k4 = lane + 32 * i;
@@ -317,9 +484,10 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_kernel(const uint16_t* __re
             uint64_t n01, n23;
             norm4(k4, n01, n23);
             float c0, c1, c2, c3;
-            f2split(add2(mul2(n01, s2), magic2), c0, c1);
-            f2split(add2(mul2(n23, s2), magic2), c2, c3);
-            p = pack_codes(__float_as_uint(c0), __float_as_uint(c1), __float_as_uint(c2), __float_as_uint(c3));
+            f2split(n01, c0, c1);
+            f2split(n23, c2, c3);
+            p = pack_codes(quant_code_bits(c0, s), quant_code_bits(c1, s), quant_code_bits(c2, s),
+                           quant_code_bits(c3, s));
         }
         if (LAYOUT == kNatural) {
             if (ok) out[k4] = p;
@@ -335,13 +503,19 @@ template <int LAYOUT>
 static void launch_rms_rb(const uint16_t* x, const float* g, float eps, long long T, long long K, int8_t* xq,
                           float* s_tok, uint4* zw, long long nzero, unsigned* status, cudaStream_t stream) {
     const unsigned blocks = static_cast<unsigned>((T + 7) / 8);
-    const long long per_lane = ((K >> 4) + 31) / 32;  // blocks per lane
+    // blocks per lane; rows up to K = 8192 stay in registers for the sum of
+    // squares (read once from memory), longer ones read the rest again
+    const long long per_lane = ((K >> 4) + 31) / 32;
     if (per_lane <= 1)
         rmsnorm_quant_kernel<LAYOUT, 1><<<blocks, 256, 0, stream>>>(x, g, eps, T, K, xq, s_tok, zw, nzero, status);
     else if (per_lane <= 2)
         rmsnorm_quant_kernel<LAYOUT, 2><<<blocks, 256, 0, stream>>>(x, g, eps, T, K, xq, s_tok, zw, nzero, status);
-    else
+    else if (per_lane <= 4)
         rmsnorm_quant_kernel<LAYOUT, 4><<<blocks, 256, 0, stream>>>(x, g, eps, T, K, xq, s_tok, zw, nzero, status);
+    else if (per_lane <= 10)
+        rmsnorm_quant_kernel<LAYOUT, 10><<<blocks, 256, 0, stream>>>(x, g, eps, T, K, xq, s_tok, zw, nzero, status);
+    else
+        rmsnorm_quant_kernel<LAYOUT, 16><<<blocks, 256, 0, stream>>>(x, g, eps, T, K, xq, s_tok, zw, nzero, status);
 }
 
 // RMSNorm then per-token absmax int8 (layout as launch_quant); g fp32 [K]

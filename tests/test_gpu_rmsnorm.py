@@ -7,6 +7,7 @@ import torch
 
 import oracle
 from parity_util import assert_bf16_close, assert_fp32_close, layer_inputs, to_dev, x_dev
+from sparse_linear_layers_b200 import synthetic
 
 pytestmark = pytest.mark.gpu
 
@@ -37,6 +38,67 @@ def test_rmsnorm_quant_bit_exact(sbl, T, K, eps):
     assert sbl.sbl_device_status() == 0
     assert np.array_equal(xq.cpu().numpy(), xq_ref)
     assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+
+
+def _bf16(v):
+    return synthetic.bf16_bits_to_f32(synthetic.f32_to_bf16_bits(np.asarray(v, np.float32)))
+
+
+def _exact_sum_tokens(K):
+    """Tokens that reach every branch of the kernel's exact sum of squares:
+    ordinary draws (one integer window), a value 2^-25 or 2^-60 below the rest
+    (two windows / the limb columns), rows of tiny, subnormal or huge values,
+    a double-rounding trap and a tie at float32 rounding boundaries."""
+    rows = _bf16(synthetic.activations(12, K, seed=9)[1])
+    rows[1, K // 2] = 2.0 ** -25
+    rows[2, K // 3] = -(2.0 ** -60)
+    rows[3] = _bf16(rows[3] * np.float32(2.0 ** -110))  # squares below float32: sum 0
+    rows[4] = 0.0
+    rows[4, :3] = [4096.0, 1.0, 2.0 ** -30]          # 2^24 + 1 + 2^-60 -> 16777218
+    rows[5] = 0.0
+    rows[5, 0], rows[5, 1:16] = 4096.0, 1.0           # 16777231, a tie -> 16777232
+    rows[6] = _bf16(rows[6] * np.float32(2.0 ** -66))  # float32-subnormal sum
+    rows[6, ::5] = 3 * 2.0 ** -133                    # bf16 subnormals
+    rows[7, 0] = 1.5 * 2.0 ** 63                      # sum just below 2^127 * 1.2
+    rows[8, K - 1] = 2.0 ** -20
+    rows[9] = _bf16(rows[9] * np.float32(2.0 ** 50))
+    rows[10] = 3.0
+    rows[10, 1::2] = -3.0
+    rows[11] = 0.0
+    rows[11, K - 5] = -0.75
+    bits = synthetic.f32_to_bf16_bits(rows)
+    assert np.array_equal(synthetic.bf16_bits_to_f32(bits), rows)
+    return bits, rows
+
+
+@pytest.mark.parametrize("K", [16, 64, 512, 896, 2048, 4864, 7168, 16384])
+def test_rmsnorm_exact_sum_branches(sbl, K):
+    """x_q and s_tok bit-exact on tokens built to take each way the kernel forms
+    the exact sum of squares, at row lengths held in registers (K <= 8192)
+    and read again (K = 16384)."""
+    bits, rows = _exact_sum_tokens(K)
+    g = _g(K, seed=2)
+    xq_ref, s_ref = oracle.rmsnorm_quant_act(rows, g, EPS_TORCH)
+    xq, s = sbl.sbl_rmsnorm_quant_act(x_dev(bits), to_dev(g), EPS_TORCH)
+    assert sbl.sbl_device_status() == 0
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(xq.cpu().numpy(), xq_ref)
+
+
+def test_rmsnorm_overflowing_sum(sbl):
+    """A sum of squares past the float32 range is +inf: every normalised value
+    is 0 (as in the oracle) and the token is flagged."""
+    K = 64
+    rows = np.zeros((2, K), np.float32)
+    rows[:, 0] = rows[:, 1] = 1.5 * 2.0 ** 63
+    rows[1, 1] = 1.0
+    bits = synthetic.f32_to_bf16_bits(rows)
+    g = np.ones(K, np.float32)
+    xq_ref, s_ref = oracle.rmsnorm_quant_act(rows, g, 0.0)
+    xq, s = sbl.sbl_rmsnorm_quant_act(x_dev(bits), to_dev(g), 0.0)
+    assert sbl.sbl_device_status() == 3
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(xq.cpu().numpy(), xq_ref)
 
 
 def test_rmsnorm_constant_rows(sbl):
