@@ -57,3 +57,31 @@ def oracle_layer(W, n, m, xval):
     packed, scale, mbits, Wt = oracle.prepare_weights(W, n, m)
     y, acc, xq, s = oracle.linear(xval, Wt, scale)
     return dict(packed=packed, scale=scale, mbits=mbits, Wt=Wt, y=y, acc=acc, xq=xq, s=s)
+
+
+def oracle_acc(xq, Wt, chunk=4096):
+    """The oracle's int32 accumulators x_q . W_t^T, taken in token chunks so the
+    float64 operands of its (exact) matrix product stay a few hundred MB."""
+    T = xq.shape[0]
+    out = np.empty((T, Wt.shape[0]), np.int32)
+    for t0 in range(0, T, chunk):
+        out[t0:t0 + chunk] = oracle.int_contract(xq[t0:t0 + chunk], Wt)
+    return out
+
+
+def assert_layer_outputs(acc_gpu, y_gpu, yb_gpu_bits, xq, s, Wt, scale, what="", chunk=4096):
+    """Every accumulator bit-exact, every fp32 y within 1e-5 relative and every
+    bf16 y within 2 ulps of the oracle, chunk by chunk of tokens."""
+    T = xq.shape[0]
+    for t0 in range(0, T, chunk):
+        sl = slice(t0, t0 + chunk)
+        ref = oracle.int_contract(xq[sl], Wt)
+        got = acc_gpu[sl]
+        if not np.array_equal(got, ref):
+            bad = np.argwhere(got != ref)[0]
+            raise AssertionError(f"{what}: acc differs at token {t0 + bad[0]}, output {bad[1]}")
+        y_ref = oracle.dequant(ref, scale, s[sl])
+        if y_gpu is not None:
+            assert_fp32_close(y_gpu[sl], y_ref, f"{what} y (tokens {t0}..)")
+        if yb_gpu_bits is not None:
+            assert_bf16_close(yb_gpu_bits[sl], y_ref, f"{what} bf16 y (tokens {t0}..)")

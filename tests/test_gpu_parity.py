@@ -9,7 +9,8 @@ import pytest
 import torch
 
 import oracle
-from parity_util import (assert_bf16_close, assert_fp32_close, layer_inputs, oracle_layer, to_dev, x_dev)
+from parity_util import (assert_bf16_close, assert_fp32_close, assert_layer_outputs, layer_inputs, oracle_layer, to_dev,
+                         x_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -326,30 +327,29 @@ def test_qwen_layer_full(sbl, T):
         assert_fp32_close(y.cpu().numpy(), ref["y"], name)
 
 
-def test_ffn_prefill_32k_sampled(sbl):
-    """0.5B FFN shapes at T = 32768 (1% outliers x20), 3:4 and 2:4: sampled accumulators."""
+@pytest.mark.parametrize("n,m", [(3, 4), (2, 4)])
+def test_ffn_prefill_32k_full(sbl, n, m):
+    """0.5B FFN shapes (gate, up, down) at T = 32768 with 1% outliers x20, 3:4
+    and 2:4: every accumulator bit for bit, every fp32 and bf16 output within
+    tolerance (the oracle's exact float64 product, token chunk by chunk)."""
     from sparse_linear_layers_b200.synthetic import QWEN05_FFN
-    rng = np.random.default_rng(0)
     T = 32768
-    for n, m in ((3, 4), (2, 4)):
-        for name, K, O in QWEN05_FFN:
-            W, xbits, xval = layer_inputs(O, K, T, seed=0, outlier_p=0.01, tag=name)
-            packed, scale, _, Wt = oracle.prepare_weights(W, n, m)
-            xq, s = oracle.quant_act(xval)
-            w = _prep(sbl, W, n, m)
-            assert np.array_equal(w.packed.cpu().numpy(), packed)
-            acc = torch.empty((T, O), dtype=torch.int32, device="cuda")
-            y = sbl.sbl_linear(x_dev(xbits), w, acc_out=acc)
-            assert sbl.sbl_device_status() == 0
-            ti = rng.integers(0, T, 4096)
-            oi = rng.integers(0, O, 4096)
-            ti[:2] = [0, T - 1]
-            oi[:2] = [0, O - 1]
-            ref_acc = oracle.acc_entries(xq, Wt, ti, oi)
-            got = acc.cpu().numpy()[ti, oi]
-            assert np.array_equal(got.astype(np.int64), ref_acc)
-            ref_y = ref_acc * scale.astype(np.float64)[oi] / s.astype(np.float64)[ti]
-            assert_fp32_close(y.cpu().numpy()[ti, oi], ref_y)
+    for name, K, O in QWEN05_FFN:
+        W, xbits, xval = layer_inputs(O, K, T, seed=0, outlier_p=0.01, tag=name)
+        packed, scale, _, Wt = oracle.prepare_weights(W, n, m)
+        xq, s = oracle.quant_act(xval)
+        del xval
+        w = _prep(sbl, W, n, m)
+        assert np.array_equal(w.packed.cpu().numpy(), packed)
+        x = x_dev(xbits)
+        acc = torch.empty((T, O), dtype=torch.int32, device="cuda")
+        y = sbl.sbl_linear(x, w, acc_out=acc)
+        yb = sbl.sbl_linear(x, w, out_dtype=torch.bfloat16)
+        assert sbl.sbl_device_status() == 0
+        assert np.array_equal(s, sbl.sbl_quant_act(x)[1].cpu().numpy())
+        assert_layer_outputs(acc.cpu().numpy(), y.cpu().numpy(), yb.cpu().view(torch.int16).numpy(), xq, s, Wt, scale,
+                             what=f"{name} {n}:{m}")
+        del acc, y, yb, x
 
 
 # ------------------------------------------------------------------ device status paths
