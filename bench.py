@@ -497,12 +497,17 @@ SM_MAX_MHZ = 1965.0
 def _ste_backward_bench(sbl, dev, T=4096):
     """The training path's straight-through gradients (dX = dY . W_hat,
     dW = dY^T . x_hat) of the hidden-2048 stack's projections at T tokens,
-    each kernel graph-replayed with L2 flushed; flops 2 * T * O * K per
-    gradient against the fp32 FMA peak of the CUDA cores."""
+    each call graph-replayed with L2 flushed; flops 2 * T * O * K per
+    gradient.  Two paths: the tcgen05 tensor cores (sbl_linear_backward_ws:
+    operand passes + a bf16 GEMM over three bf16 parts of the fp32 factor, so
+    3 * 2 * T * O * K bf16 flops executed, against the measured bf16 peak) and
+    the CUDA cores (sbl_linear_backward, against the fp32 FMA peak)."""
     props = torch.cuda.get_device_properties(dev)
     peak = props.multi_processor_count * FP32_LANES_PER_SM * 2 * SM_MAX_MHZ * 1e6 / 1e12
+    bf16_peak = _peaks()[1]
     out = {"tokens": T, "fp32_peak_tflops": peak,
-           "peak_source": f"{props.multi_processor_count} SMs x {FP32_LANES_PER_SM} fp32 lanes x 2 x {SM_MAX_MHZ} MHz"}
+           "peak_source": f"{props.multi_processor_count} SMs x {FP32_LANES_PER_SM} fp32 lanes x 2 x {SM_MAX_MHZ} MHz",
+           "bf16_peak_tflops": bf16_peak}
     gen = torch.Generator(device=dev)
     gen.manual_seed(17)
     from sparse_linear_layers_b200 import _lib
@@ -514,16 +519,24 @@ def _ste_backward_bench(sbl, dev, T=4096):
         dY = torch.randn((T, O), device=dev, generator=gen)
         dX = torch.empty((T, K), device=dev)
         dW = torch.empty((O, K), device=dev)
+        ws = torch.empty((sbl.sbl_linear_backward_workspace_bytes(T, O, K),), dtype=torch.uint8, device=dev)
         res = {}
         for g, (px, pw) in (("dX", (dX.data_ptr(), None)), ("dW", (None, dW.data_ptr()))):
+            fn = lambda px=px, pw=pw: _lib.check(_lib.lib.sbl_linear_backward_ws(
+                dY.data_ptr(), T, O, xq.data_ptr(), st.data_ptr(), K, w.packed.data_ptr(), w.row_scale.data_ptr(),
+                px, pw, 0, ws.data_ptr(), ws.numel(), torch.cuda.current_stream().cuda_stream),
+                "sbl_linear_backward_ws")
+            us = _flushed_graph_us(fn, dev)
+            tf = 2.0 * T * O * K / us / 1e6
+            res[g] = {"us": us, "tflops": tf, "bf16_tflops_executed": 3 * tf, "frac_of_bf16_peak": 3 * tf / bf16_peak}
             fn = lambda px=px, pw=pw: _lib.check(_lib.lib.sbl_linear_backward(
                 dY.data_ptr(), T, O, xq.data_ptr(), st.data_ptr(), K, w.packed.data_ptr(), w.row_scale.data_ptr(),
                 px, pw, 0, torch.cuda.current_stream().cuda_stream), "sbl_linear_backward")
             us = _flushed_graph_us(fn, dev)
             tf = 2.0 * T * O * K / us / 1e6
-            res[g] = {"us": us, "tflops": tf, "frac": tf / peak}
+            res[g + "_cuda_cores"] = {"us": us, "tflops": tf, "frac": tf / peak}
         out[name] = res
-        del W, w, x, xq, dY, dX, dW
+        del W, w, x, xq, dY, dX, dW, ws
     return out
 
 

@@ -217,6 +217,35 @@ sbl_status sbl_linear_backward(const float* dY, int64_t T, int64_t O, const int8
                                int flags, void* stream);
 
 /*
+ * sbl_linear_backward_ws — the gradients of sbl_linear_backward on the tcgen05
+ * tensor cores, with a caller-provided workspace.
+ *
+ * Same operation, arguments, flags and results as sbl_linear_backward (the
+ * Sparse-BitNet Guide, "Training Stability & The Straight-Through
+ * Estimator"), plus:
+ *   workspace        device scratch of at least
+ *                    sbl_linear_backward_workspace_bytes(T, O, K, dX != NULL,
+ *                    dW != NULL) bytes, 256-byte aligned; contents on entry
+ *                    do not matter (else SBL_ERR_WORKSPACE).  Calls that share
+ *                    it must be ordered on one stream.
+ * How: the fp32 factor of each product (dY * scale_o for dX, dY / s_t for dW,
+ * each one IEEE rounding) is split exactly into three bf16 parts (hi, mid,
+ * lo: its 24 significand bits in three 8-bit pieces); the other factor
+ * (ternary W_t, or x_q with |x_q| <= 127) is exact in bf16; the workspace
+ * holds both operands in bf16, K-major, and a kind::f16 tensor-core GEMM with
+ * fp32 accumulation sums the 3n exact products.  Error: within
+ * (n + 2) * 2^-24 * sum |terms| of the exact value for the tensor cores' fp32
+ * accumulation as measured on B200 (n + 3 with SBL_BWD_DW_TERNARY); exact
+ * where every partial sum is a float.  T and O up to 2^21, else
+ * SBL_ERR_UNSUPPORTED.  Empty reductions (T == 0 or O == 0) write zeros and
+ * need no workspace.
+ */
+size_t sbl_linear_backward_workspace_bytes(int64_t T, int64_t O, int64_t K, int need_dx, int need_dw);
+sbl_status sbl_linear_backward_ws(const float* dY, int64_t T, int64_t O, const int8_t* x_q, const float* s_tok,
+                                  int64_t K, const uint8_t* packed, const float* row_scale, float* dX, float* dW,
+                                  int flags, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * sbl_linear_workspace_bytes — bytes of device workspace sbl_linear needs for
  * these sizes: the quantised activations and their scales, in the kernels'
  * internal layout (T*K + 4*T bytes, each rounded up to 256), plus, for 2:4

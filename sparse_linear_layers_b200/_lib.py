@@ -52,6 +52,8 @@ SIGNATURES = {
     "sbl_linear_plan": (_int, [_i64, _i64, _i64, _int, _int, _sz]),
     "sbl_mask_monitor": (_int, [_vp, _vp, _i64, _i64, _int, _int, _vp, _vp, _vp]),
     "sbl_linear_backward": (_int, [_vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _int, _vp]),
+    "sbl_linear_backward_workspace_bytes": (_sz, [_i64, _i64, _i64, _int, _int]),
+    "sbl_linear_backward_ws": (_int, [_vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _int, _vp, _sz, _vp]),
     "sbl_decode_max_tokens": (_i64, []),
     "sbl_device_status": (_int, [_vp]),
     "sbl_selftest_bounded_wait": (_int, [_u32, _vp]),

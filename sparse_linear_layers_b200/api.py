@@ -210,16 +210,24 @@ def sbl_mask_monitor(old_bits: torch.Tensor, new_bits: torch.Tensor, K: int, n: 
     return totals, rows
 
 
+def sbl_linear_backward_workspace_bytes(T: int, O: int, K: int, need_dx: bool = True, need_dw: bool = True) -> int:
+    return int(lib.sbl_linear_backward_workspace_bytes(T, O, K, int(need_dx), int(need_dw)))
+
+
 def sbl_linear_backward(dY: torch.Tensor, x_q: torch.Tensor, s_tok: torch.Tensor, w: PreparedWeights,
                         need_dx: bool = True, need_dw: bool = True, dw_ternary: bool = False,
                         dX: Optional[torch.Tensor] = None, dW: Optional[torch.Tensor] = None,
+                        tensor_cores: bool = True, workspace: Optional[torch.Tensor] = None,
                         stream: Optional[torch.cuda.Stream] = None):
     """Straight-through gradients of sbl_linear: (dX fp32 [T,K] or None, dW fp32 [O,K] or None).
 
     dX = dY . (scale * W_t) and dW = dY^T . (x_q / s_t) over every weight position
     (``dw_ternary``: dW rows scaled by scale_o once more, the guide module's form).
     ``x_q``/``s_tok`` are the forward's quantised activations in natural order
-    (sbl_quant_act or sbl_rmsnorm_quant_act)."""
+    (sbl_quant_act or sbl_rmsnorm_quant_act).  ``tensor_cores`` (default) runs
+    the tcgen05 path (sbl_linear_backward_ws; a workspace of
+    sbl_linear_backward_workspace_bytes() is allocated unless given), else the
+    CUDA-core kernels (sbl_linear_backward)."""
     T, O = _need_2d(dY, "dY")
     K = w.K
     if O != w.O or x_q.shape != (T, K) or s_tok.shape != (T,):
@@ -238,11 +246,21 @@ def sbl_linear_backward(dY: torch.Tensor, x_q: torch.Tensor, s_tok: torch.Tensor
     if need_dw:
         dW = torch.empty((O, K), dtype=torch.float32, device=dev) if dW is None else dW
         _need_cuda(dW, "dW", torch.float32, (O, K), dev)
-    check(lib.sbl_linear_backward(dY.data_ptr(), T, O, x_q.data_ptr(), s_tok.data_ptr(), K, w.packed.data_ptr(),
-                                  w.row_scale.data_ptr(), dX.data_ptr() if need_dx else None,
-                                  dW.data_ptr() if need_dw else None,
-                                  _lib.SBL_BWD_DW_TERNARY if dw_ternary else 0, _stream(stream)),
-          "sbl_linear_backward")
+    flags = _lib.SBL_BWD_DW_TERNARY if dw_ternary else 0
+    if tensor_cores:
+        if workspace is None:
+            workspace = torch.empty((max(1, sbl_linear_backward_workspace_bytes(T, O, K, need_dx, need_dw)),),
+                                    dtype=torch.uint8, device=dev)
+        _need_workspace(workspace, dev)
+        check(lib.sbl_linear_backward_ws(dY.data_ptr(), T, O, x_q.data_ptr(), s_tok.data_ptr(), K,
+                                         w.packed.data_ptr(), w.row_scale.data_ptr(), dX.data_ptr() if need_dx else None,
+                                         dW.data_ptr() if need_dw else None, flags, workspace.data_ptr(),
+                                         workspace.numel(), _stream(stream)), "sbl_linear_backward_ws")
+    else:
+        check(lib.sbl_linear_backward(dY.data_ptr(), T, O, x_q.data_ptr(), s_tok.data_ptr(), K, w.packed.data_ptr(),
+                                      w.row_scale.data_ptr(), dX.data_ptr() if need_dx else None,
+                                      dW.data_ptr() if need_dw else None, flags, _stream(stream)),
+              "sbl_linear_backward")
     return (dX if need_dx else None), (dW if need_dw else None)
 
 

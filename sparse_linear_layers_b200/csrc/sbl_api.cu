@@ -1,7 +1,7 @@
 // C ABI of the Sparse-BitLinear library: argument validation, workspace
 // layout, path dispatch and the per-device status word.  All arithmetic runs
 // in the kernels of prep.cu, quant.cu, decode.cu, decode_mma.cu, prefill.cu, prefill_pair.cu, prefill_sp.cu,
-// mask_monitor.cu and backward.cu.
+// mask_monitor.cu, backward.cu and backward_tc.cu.
 #include <cstdint>
 #include <cstdio>
 #include <cuda_runtime.h>
@@ -33,6 +33,10 @@ long long ste_backward_tiles(long long rows, long long K);
 cudaError_t launch_ste_backward(const float* dY, long long T, long long O, long long K, const uint8_t* packed,
                                 const float* row_scale, const int8_t* xq, const float* s_tok, float* dX, float* dW,
                                 int dw_ternary, cudaStream_t stream);
+size_t backward_tc_workspace_bytes(long long T, long long O, long long K, int need_dx, int need_dw);
+cudaError_t launch_backward_tc(const float* dY, long long T, long long O, const int8_t* xq, const float* s_tok,
+                               long long K, const uint8_t* packed, const float* row_scale, float* dX, float* dW,
+                               int dw_ternary, void* ws, unsigned* status, int num_sms, cudaStream_t stream);
 cudaError_t launch_prefill(const int8_t* xperm, const float* s_tok, long long T, long long K, const uint8_t* packed,
                            const float* row_scale, long long O, void* y, int y_bf16, int32_t* acc_out,
                            unsigned* status, int num_sms, int variant, int ksplit, int32_t* part,
@@ -208,6 +212,37 @@ sbl_status sbl_linear_backward(const float* dY, int64_t T, int64_t O, const int8
     return from_cuda(sbl::launch_ste_backward(dY, T, O, K, packed, row_scale, x_q, s_tok, any_dx ? dX : nullptr,
                                               any_dw ? dW : nullptr, ternary ? 1 : 0,
                                               static_cast<cudaStream_t>(stream)));
+}
+
+// Largest T and O of the tensor-core backward (grid extents of its operand passes).
+constexpr long long kBwdTcMaxRows = 1ll << 21;
+
+size_t sbl_linear_backward_workspace_bytes(int64_t T, int64_t O, int64_t K, int need_dx, int need_dw) {
+    if (T < 0 || O < 0 || K <= 0) return 0;
+    return sbl::backward_tc_workspace_bytes(T, O, K, need_dx ? 1 : 0, need_dw ? 1 : 0);
+}
+
+sbl_status sbl_linear_backward_ws(const float* dY, int64_t T, int64_t O, const int8_t* x_q, const float* s_tok,
+                                  int64_t K, const uint8_t* packed, const float* row_scale, float* dX, float* dW,
+                                  int flags, void* workspace, size_t workspace_bytes, void* stream) {
+    if (T < 0 || O < 0) return SBL_ERR_INVALID_ARG;
+    if (flags & ~SBL_BWD_DW_TERNARY) return SBL_ERR_INVALID_ARG;
+    if (sbl_status s = check_k(K)) return s;
+    if (!dX && !dW) return SBL_ERR_INVALID_ARG;
+    // empty reductions (all zeros) and empty outputs: the CUDA-core entry point
+    if (T == 0 || O == 0)
+        return sbl_linear_backward(dY, T, O, x_q, s_tok, K, packed, row_scale, dX, dW, flags, stream);
+    const bool ternary = (flags & SBL_BWD_DW_TERNARY) != 0;
+    auto ok = [](const void* p) { return p != nullptr && aligned(p, 16); };
+    if (dX && !(ok(dX) && ok(dY) && ok(packed) && ok(row_scale))) return SBL_ERR_INVALID_ARG;
+    if (dW && !(ok(dW) && ok(dY) && ok(x_q) && ok(s_tok) && (!ternary || ok(row_scale)))) return SBL_ERR_INVALID_ARG;
+    if (T > kBwdTcMaxRows || O > kBwdTcMaxRows) return SBL_ERR_UNSUPPORTED;
+    const size_t need = sbl::backward_tc_workspace_bytes(T, O, K, dX != nullptr, dW != nullptr);
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return SBL_ERR_WORKSPACE;
+    DeviceInfo* d;
+    if (sbl_status s = device_info(&d)) return s;
+    return from_cuda(sbl::launch_backward_tc(dY, T, O, x_q, s_tok, K, packed, row_scale, dX, dW, ternary ? 1 : 0,
+                                             workspace, d->status, d->num_sms, static_cast<cudaStream_t>(stream)));
 }
 
 // Quantised activations and their scales: what every path needs.

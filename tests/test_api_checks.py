@@ -94,8 +94,12 @@ def test_linear_rejects_bad_weights(rec):
 def test_backward_checks(rec):
     w, dY = _w(), torch.zeros((T, O))
     xq, s = torch.zeros((T, K), dtype=torch.int8), torch.ones(T)
-    api.sbl_linear_backward(dY, xq, s, w, dX=torch.empty((T, K)), dW=torch.empty((O, K)))
+    api.sbl_linear_backward(dY, xq, s, w, dX=torch.empty((T, K)), dW=torch.empty((O, K)), tensor_cores=False)
     assert rec.calls == ["sbl_linear_backward"]
+    rec.calls.clear()
+    api.sbl_linear_backward(dY, xq, s, w, dX=torch.empty((T, K)), dW=torch.empty((O, K)),
+                            workspace=torch.empty(64, dtype=torch.uint8))
+    assert rec.calls == ["sbl_linear_backward_ws"]
     rec.calls.clear()
     for kw in (dict(dW=torch.empty((O - 1, K))), dict(dW=torch.empty((O, K - 16))), dict(dX=torch.empty((T, K - 1))),
                dict(dX=torch.empty((T, K), device="meta")), dict(dW=torch.empty((O, K), dtype=torch.float64))):
@@ -105,6 +109,8 @@ def test_backward_checks(rec):
             api.sbl_linear_backward(dY, xq, s, w, **args)
     with pytest.raises(ValueError):
         api.sbl_linear_backward(dY, xq.to("meta"), s, w)
+    with pytest.raises(ValueError):
+        api.sbl_linear_backward(dY, xq, s, w, workspace=torch.empty(64, dtype=torch.uint8, device="meta"))
     assert rec.calls == []
 
 

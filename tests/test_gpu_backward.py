@@ -7,7 +7,9 @@ length (O for dX, T for dW).  On inputs whose every partial sum is a float
 (integer loss gradients, power-of-two scales) the result is exact, and there
 the comparison is bit for bit.  Shapes span several 128 x 128 tiles with
 ragged edges in every dimension; the hot-path sizes are checked on sampled
-entries; empty reductions write zeros."""
+entries; empty reductions write zeros.  Every test runs on both paths: the
+tcgen05 tensor cores (bf16 parts of the fp32 factor, fp32 accumulation in
+tensor memory) and the CUDA cores (fp32 fused multiply-adds)."""
 import functools
 
 import numpy as np
@@ -29,6 +31,13 @@ def sbl():
         pytest.skip("no CUDA device")
     import sparse_linear_layers_b200 as m
     return m
+
+
+@pytest.fixture(params=[True, False], ids=["tcgen05", "cuda_cores"])
+def bwd(request, sbl):
+    """sbl_linear_backward on the tensor cores (with a workspace) and on the
+    CUDA cores: both must meet the same bar."""
+    return functools.partial(sbl.sbl_linear_backward, tensor_cores=request.param)
 
 
 @functools.lru_cache(maxsize=2)
@@ -70,7 +79,7 @@ SHAPES = [(512, 256, 16, 2, 4), (896, 896, 300, 3, 4), (160, 80, 129, 6, 8), (36
 
 
 @pytest.mark.parametrize("O,K,T,n,m", SHAPES)
-def test_backward_random(sbl, O, K, T, n, m):
+def test_backward_random(sbl, bwd, O, K, T, n, m):
     w, xq_d, s_d, Wt, scale, xq, s = _layer(sbl, O, K, T, n, m, seed=O + T)
     dY = synthetic.output_grads(T, O, seed=O * 3 + T)
     dX_ref, dW_ref = oracle.ste_backward(dY, xq, s, Wt, scale)
@@ -79,15 +88,15 @@ def test_backward_random(sbl, O, K, T, n, m):
     absx = (a * scale.astype(np.float64)[None, :]) @ np.abs(Wt).astype(np.float64)
     absw = a.T @ (np.abs(xq).astype(np.float64) / s.astype(np.float64)[:, None])
     dY_d = to_dev(dY)
-    dX, dW = sbl.sbl_linear_backward(dY_d, xq_d, s_d, w)
+    dX, dW = bwd(dY_d, xq_d, s_d, w)
     _assert_within_bound(dX.cpu().numpy(), dX_ref, absx, O, "dX")
     _assert_within_bound(dW.cpu().numpy(), dW_ref, absw, T, "dW")
-    _, dWt = sbl.sbl_linear_backward(dY_d, xq_d, s_d, w, need_dx=False, dw_ternary=True)
+    _, dWt = bwd(dY_d, xq_d, s_d, w, need_dx=False, dw_ternary=True)
     _assert_within_bound(dWt.cpu().numpy(), dWt_ref, absw * scale.astype(np.float64)[:, None], T + 1, "dW ternary")
     # one output at a time gives the same bits
-    dX1, none = sbl.sbl_linear_backward(dY_d, xq_d, s_d, w, need_dw=False)
+    dX1, none = bwd(dY_d, xq_d, s_d, w, need_dw=False)
     assert none is None and torch.equal(dX1, dX)
-    none, dW1 = sbl.sbl_linear_backward(dY_d, xq_d, s_d, w, need_dx=False)
+    none, dW1 = bwd(dY_d, xq_d, s_d, w, need_dx=False)
     assert none is None and torch.equal(dW1, dW)
 
 
@@ -107,27 +116,27 @@ def _exact_inputs(sbl, O, K, T, n, m, seed):
 
 
 @pytest.mark.parametrize("O,K,T,n,m", [(896, 896, 300, 3, 4), (160, 80, 129, 2, 4), (36, 48, 7, 6, 8)])
-def test_backward_exact(sbl, O, K, T, n, m):
+def test_backward_exact(sbl, bwd, O, K, T, n, m):
     w, xq_d, s_d, dY_d, dY, Wt, scale, xq, s = _exact_inputs(sbl, O, K, T, n, m, seed=O + 1)
     dX_ref, dW_ref = oracle.ste_backward(dY, xq, s, Wt, scale)
     _, dWt_ref = oracle.ste_backward(dY, xq, s, Wt, scale, dw_ternary=True)
     for ref in (dX_ref, dW_ref, dWt_ref):
         assert np.array_equal(ref.astype(np.float32).astype(np.float64), ref)
-    dX, dW = sbl.sbl_linear_backward(dY_d, xq_d, s_d, w)
+    dX, dW = bwd(dY_d, xq_d, s_d, w)
     assert np.array_equal(dX.cpu().numpy(), dX_ref.astype(np.float32))
     assert np.array_equal(dW.cpu().numpy(), dW_ref.astype(np.float32))
-    _, dWt = sbl.sbl_linear_backward(dY_d, xq_d, s_d, w, need_dx=False, dw_ternary=True)
+    _, dWt = bwd(dY_d, xq_d, s_d, w, need_dx=False, dw_ternary=True)
     assert np.array_equal(dWt.cpu().numpy(), dWt_ref.astype(np.float32))
 
 
 # The hidden-2048 stack's down (7168 -> 2048) and gate (2048 -> 7168)
 # projections at 4096 tokens: the sizes the benchmark times.
 @pytest.mark.parametrize("K,O", [(7168, 2048), (2048, 7168)])
-def test_backward_full_size_sampled(sbl, K, O):
+def test_backward_full_size_sampled(sbl, bwd, K, O):
     T, n, m = 4096, 2, 4
     w, xq_d, s_d, Wt, scale, xq, s = _layer(sbl, O, K, T, n, m, seed=9)
     dY = synthetic.output_grads(T, O, seed=5)
-    dX, dW = sbl.sbl_linear_backward(to_dev(dY), xq_d, s_d, w)
+    dX, dW = bwd(to_dev(dY), xq_d, s_d, w)
     dX, dW = dX.cpu().numpy(), dW.cpu().numpy()
     rng = np.random.default_rng(6)
     dY64, Wt64, sc64 = dY.astype(np.float64), Wt.astype(np.float64), scale.astype(np.float64)
@@ -144,27 +153,27 @@ def test_backward_full_size_sampled(sbl, K, O):
     assert abs(dW[o, k] - (dY64[:, o] * xh[:, k]).sum()) <= (T + 3) * U * np.abs(dY64[:, o] * xh[:, k]).sum() + 1e-37
 
 
-def test_backward_full_size_exact(sbl):
+def test_backward_full_size_exact(sbl, bwd):
     O, K, T = 2048, 7168, 4096
     w, xq_d, s_d, dY_d, dY, Wt, scale, xq, s = _exact_inputs(sbl, O, K, T, 2, 4, seed=9)
-    dX, dW = sbl.sbl_linear_backward(dY_d, xq_d, s_d, w)
+    dX, dW = bwd(dY_d, xq_d, s_d, w)
     dX_ref, dW_ref = oracle.ste_backward(dY, xq, s, Wt, scale)
     assert np.array_equal(dX.cpu().numpy(), dX_ref.astype(np.float32))
     assert np.array_equal(dW.cpu().numpy(), dW_ref.astype(np.float32))
 
 
-def test_backward_empty_reductions(sbl):
+def test_backward_empty_reductions(sbl, bwd):
     from sparse_linear_layers_b200.api import PreparedWeights
     K, O, T = 64, 40, 5
     w, xq_d, s_d, *_ = _layer(sbl, O, K, T, 2, 4, seed=1)
     # T == 0: dW is a sum over no tokens
     dW = torch.full((O, K), float("nan"), device="cuda")
-    _, dW = sbl.sbl_linear_backward(torch.empty((0, O), device="cuda"), xq_d[:0], s_d[:0], w, need_dx=False, dW=dW)
+    _, dW = bwd(torch.empty((0, O), device="cuda"), xq_d[:0], s_d[:0], w, need_dx=False, dW=dW)
     assert torch.count_nonzero(dW).item() == 0
     # O == 0: dX is a sum over no output rows
     w0 = PreparedWeights(torch.empty((0, K // 4), dtype=torch.uint8, device="cuda"),
                          torch.empty((0,), device="cuda"), 2, 4, K)
     dX = torch.full((T, K), float("nan"), device="cuda")
-    dX, _ = sbl.sbl_linear_backward(torch.empty((T, 0), device="cuda"), xq_d, s_d, w0, need_dw=False, dX=dX)
+    dX, _ = bwd(torch.empty((T, 0), device="cuda"), xq_d, s_d, w0, need_dw=False, dX=dX)
     assert torch.count_nonzero(dX).item() == 0
     assert sbl.sbl_device_status() == 0
