@@ -82,3 +82,27 @@ def test_training_step_moves_the_mask(train):
         y = layer(x)
     _, scale, _, Wt = oracle.prepare_weights(W2, n, m)
     assert_fp32_close(y.cpu().numpy(), oracle.linear(xv, Wt, scale)[0])
+
+
+def test_forward_stops_on_nonfinite_input(train):
+    """The kernels flag NaN and Inf instead of propagating them, so the layer
+    reads the status word: a NaN activation or latent weight raises
+    FloatingPointError; with check_finite=False the forward runs on."""
+    K, O = 256, 128
+    layer, W = _layer(train, K, O, 2, 4, False, seed=5)
+    x = torch.randn((4, K), device="cuda")
+    layer(x)  # finite: no error
+    bad = x.clone()
+    bad[2, 7] = float("nan")
+    with pytest.raises(FloatingPointError):
+        layer(bad)
+    with torch.no_grad():
+        layer.weight[3, 5] = float("inf")
+    with pytest.raises(FloatingPointError):
+        layer(x)
+    layer.check_finite = False
+    layer(x)
+    torch.cuda.synchronize()
+    from sparse_linear_layers_b200 import api
+    assert api.sbl_device_status() == 3  # flagged, not raised
+    assert api.sbl_device_status() == 0

@@ -1,4 +1,5 @@
-"""sbl_linear_noalloc against sbl_linear, through the C ABI.
+"""sbl_linear_noalloc against the CPU oracle and against sbl_linear, through
+the C ABI.
 
 sbl_linear_noalloc is for callers that cannot allocate device memory (for
 example a plugin whose host application owns the device-memory budget): it
@@ -13,7 +14,8 @@ import numpy as np
 import pytest
 import torch
 
-from parity_util import FP32_RTOL, layer_inputs, to_dev, x_dev
+import oracle
+from parity_util import FP32_RTOL, assert_fp32_close, layer_inputs, to_dev, x_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -37,7 +39,7 @@ def _prepare(abi, W, n, m):
 
 
 def _run_both(abi, O, K, T, n, m, seed):
-    W, xbits, _ = layer_inputs(O, K, T, seed=seed, tag="noalloc", outlier_p=0.01)
+    W, xbits, xval = layer_inputs(O, K, T, seed=seed, tag="noalloc", outlier_p=0.01)
     packed, scale = _prepare(abi, W, n, m)
     x = x_dev(xbits)
     s = torch.cuda.current_stream().cuda_stream
@@ -54,6 +56,13 @@ def _run_both(abi, O, K, T, n, m, seed):
     assert abi.lib.sbl_linear_noalloc(x.data_ptr(), T, K, packed.data_ptr(), scale.data_ptr(), O, n, m,
                                       y.data_ptr(), abi.SBL_F32, acc.data_ptr(), s) == 0
     assert abi.lib.sbl_device_status(s) == 0
+    # against the oracle: accumulators bit-exact, y within 1e-5 relative
+    _, o_scale, _, Wt = oracle.prepare_weights(W, n, m)
+    assert np.array_equal(scale.cpu().numpy().view(np.uint32), o_scale.view(np.uint32))
+    y_o, acc_o, _, _ = oracle.linear(xval, Wt, o_scale)
+    assert np.array_equal(acc.cpu().numpy(), acc_o)
+    assert_fp32_close(y.cpu().numpy(), y_o)
+    # and against the entry point with a caller-provided workspace
     assert torch.equal(acc, acc_ref)
     yr = y_ref.cpu().numpy().astype(np.float64)
     assert np.all(np.abs(y.cpu().numpy() - yr) <= FP32_RTOL * np.abs(yr))
