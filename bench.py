@@ -133,79 +133,106 @@ class ClockSampler:
 # --------------------------------------------------------------------------- our arm
 
 class Layer:
+    """Weights and outputs of one projection."""
+
     def __init__(self, name, K, O, dev, seed=0):
         import sparse_linear_layers_b200 as sbl
         self.name, self.K, self.O = name, K, O
         W = synthetic.latent_weights(O, K, seed=seed, tag=f"bench-{name}")
-        xb, _ = synthetic.activations(T_PREFILL, K, seed=seed, tag=f"bench-x-{name}")
-        x1, _ = synthetic.activations(T_DECODE, K, seed=seed, tag=f"bench-x1-{name}")
         self.W_host = torch.from_numpy(W).pin_memory()
-        self.x_host = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).pin_memory()
-        self.x1_host = torch.from_numpy(x1.view(np.int16)).view(torch.bfloat16).pin_memory()
         self.W = self.W_host.to(dev)
-        self.x = self.x_host.to(dev)
-        self.x1 = self.x1_host.to(dev)
         self.w = sbl.PreparedWeights(torch.empty((O, K // 4), dtype=torch.uint8, device=dev),
                                      torch.empty((O,), dtype=torch.float32, device=dev), N, M, K)
         self.y = torch.empty((T_PREFILL, O), dtype=torch.float32, device=dev)
         self.y1 = torch.empty((T_DECODE, O), dtype=torch.float32, device=dev)
-        self.ws = sbl.workspace_for(T_PREFILL, K, O, N, M, dev)
         self.y_host = torch.empty((T_PREFILL, O), dtype=torch.float32).pin_memory()
         self.y1_host = torch.empty((T_DECODE, O), dtype=torch.float32).pin_memory()
 
-    # algorithmic work
     def prefill_ops(self):
         return 2.0 * T_PREFILL * self.O * self.K
 
+    def weight_bytes(self):
+        return self.O * self.K / 4 + 4 * self.O
+
+
+# One layer's projections in dependency order, grouped by the input they read:
+# q, k and v read the same normalised hidden state, o follows attention, gate
+# and up read the same normalised input, down follows.  Each group is one call
+# (sbl_linear_grouped for q|k|v and gate|up: x quantised once, and at decode
+# sizes one launch over the stacked weights).
+INPUT_GROUPS = (("attn", ("q", "k", "v")), ("attn_out", ("o",)), ("ffn", ("gate", "up")), ("ffn_out", ("down",)))
+PREP_BY_K = (("q", "k", "v", "o", "gate", "up"), ("down",))
+SCHEDULE = ("weight preparation: one sbl_prepare_weights_grouped launch for the six K = 896 projections, down "
+            "concurrently; prefill and decode on one stream: grouped {q,k,v} -> o -> grouped {gate,up} -> down "
+            "(projections that share an input are one sbl_linear_grouped call)")
+
+
+class InputGroup:
+    """The activations one group of projections reads, and the group's call."""
+
+    def __init__(self, name, members, dev, seed=0):
+        import sparse_linear_layers_b200 as sbl
+        self.name, self.members = name, members
+        self.K = K = members[0].K
+        xb, _ = synthetic.activations(T_PREFILL, K, seed=seed, tag=f"bench-x-{name}")
+        x1, _ = synthetic.activations(T_DECODE, K, seed=seed, tag=f"bench-x1-{name}")
+        self.x_host = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).pin_memory()
+        self.x1_host = torch.from_numpy(x1.view(np.int16)).view(torch.bfloat16).pin_memory()
+        self.x = self.x_host.to(dev)
+        self.x1 = self.x1_host.to(dev)
+        O = sum(L.O for L in members)
+        self.ws = sbl.workspace_for(T_PREFILL, K, O, N, M, dev)
+
+    def run(self, sbl, decode=False):
+        x = self.x1 if decode else self.x
+        if len(self.members) == 1:
+            L = self.members[0]
+            sbl.sbl_linear(x, L.w, y=L.y1 if decode else L.y, workspace=self.ws)
+        else:
+            sbl.sbl_linear_grouped(x, [L.w for L in self.members],
+                                   ys=[L.y1 if decode else L.y for L in self.members], workspace=self.ws)
+
+    # algorithmic bytes of one call: the shared activations once, every
+    # member's codes, scales and outputs
     def prefill_bytes(self):
-        return self.O * self.K / 4 + 4 * self.O + 2 * T_PREFILL * self.K + 4 * T_PREFILL * self.O
+        return 2 * T_PREFILL * self.K + sum(L.weight_bytes() + 4 * T_PREFILL * L.O for L in self.members)
 
-    def decode_bytes(self, T=T_DECODE):
-        return self.O * self.K / 4 + 4 * self.O + 2 * T * self.K + 4 * T * self.O
-
-
-# Dependency order of one layer's projections: q, k and v read the same
-# normalised input and run concurrently, o follows attention, gate and up read
-# the same input and run concurrently, down follows.  Weight preparations are
-# independent of one another.
-PREFILL_GROUPS = (("q", "k", "v"), ("o",), ("gate", "up"), ("down",))
-PREP_GROUPS = (("q", "k", "v", "o", "gate", "up", "down"),)
-SCHEDULE = "weight preps concurrent; prefill and decode: {q,k,v} concurrent, o, {gate,up} concurrent, down"
+    def decode_bytes(self):
+        return 2 * T_DECODE * self.K + sum(L.weight_bytes() + 4 * T_DECODE * L.O for L in self.members)
 
 
-def _run_groups(groups, layers, streams, fn):
-    """Run fn(layer) group by group: the members of a group on their own streams,
-    forked from and joined back to streams[0] (captured into the graph as such)."""
+def make_step(dev):
+    layers = [Layer(nm, K, O, dev) for nm, K, O in synthetic.QWEN05_LAYER]
     by_name = {L.name: L for L in layers}
-    main = streams[0]
-    for group in groups:
-        fork = torch.cuda.Event()
-        fork.record(main)
-        joins = []
-        for i, name in enumerate(group):
-            st = streams[i]
-            if i:
-                st.wait_event(fork)
-            with torch.cuda.stream(st):
-                fn(by_name[name])
-            if i:
-                ev = torch.cuda.Event()
-                ev.record(st)
-                joins.append(ev)
-        for ev in joins:
-            main.wait_event(ev)
+    groups = [InputGroup(g, [by_name[n] for n in names], dev) for g, names in INPUT_GROUPS]
+    return layers, groups
 
 
-def _prep_phase(sbl, layers, streams):
-    _run_groups(PREP_GROUPS, layers, streams, lambda L: sbl.sbl_prepare_weights(L.W, N, M, out=L.w))
+def _prep_phase(sbl, layers, groups, streams):
+    by_name = {L.name: L for L in layers}
+    main, side = streams[0], streams[1]
+    fork = torch.cuda.Event()
+    fork.record(main)
+    side.wait_event(fork)
+    for st, names in zip((main, side), PREP_BY_K):
+        with torch.cuda.stream(st):
+            Ls = [by_name[n] for n in names]
+            sbl.sbl_prepare_weights_grouped([L.W for L in Ls], N, M, outs=[L.w for L in Ls])
+    join = torch.cuda.Event()
+    join.record(side)
+    main.wait_event(join)
 
 
-def _prefill_phase(sbl, layers, streams):
-    _run_groups(PREFILL_GROUPS, layers, streams, lambda L: sbl.sbl_linear(L.x, L.w, y=L.y, workspace=L.ws))
+def _prefill_phase(sbl, layers, groups, streams):
+    with torch.cuda.stream(streams[0]):
+        for g in groups:
+            g.run(sbl)
 
 
-def _decode_phase(sbl, layers, streams):
-    _run_groups(PREFILL_GROUPS, layers, streams, lambda L: sbl.sbl_linear(L.x1, L.w, y=L.y1, workspace=L.ws))
+def _decode_phase(sbl, layers, groups, streams):
+    with torch.cuda.stream(streams[0]):
+        for g in groups:
+            g.run(sbl, decode=True)
 
 
 PHASES = (("prep", _prep_phase), ("prefill", _prefill_phase), ("decode", _decode_phase))
@@ -217,19 +244,19 @@ class StepGraphs:
     events between the graph launches give each phase's device time.  Inside a
     phase the projections follow the layer's dependency order (SCHEDULE)."""
 
-    def __init__(self, sbl, layers, stream):
+    def __init__(self, sbl, layers, groups, stream):
         self.stream = stream
         self.side = [torch.cuda.Stream() for _ in range(6)]
         streams = [stream] + self.side
         self.graphs = []
         with torch.cuda.stream(stream):
             for _, fn in PHASES:       # one eager pass: sets kernel attributes before capture
-                fn(sbl, layers, streams)
+                fn(sbl, layers, groups, streams)
         torch.cuda.synchronize()
         for _, fn in PHASES:
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
-                fn(sbl, layers, streams)
+                fn(sbl, layers, groups, streams)
             self.graphs.append(g)
 
     def replay(self, ev=None):
@@ -244,49 +271,72 @@ class StepGraphs:
 
 class E2E:
     """The step from pinned host buffers: H2D of W and x, D2H of y, inside the
-    timed region.  Host-to-device copies and the kernels run on one stream,
-    device-to-host copies on a second one, so the two copy directions overlap;
-    a layer's outputs are not overwritten by the next step before their copy
-    back has finished (per-layer events)."""
+    timed region.  Three streams: host-to-device copies, the kernels, and
+    device-to-host copies, so both directions of the host link and the
+    kernels overlap across groups and steps.  Events keep every buffer safe:
+    a group's inputs are not overwritten before the previous step's kernels
+    have read them, and its outputs not before they have been copied back."""
 
-    def __init__(self, layers):
+    def __init__(self, groups):
         self.main = torch.cuda.Stream()
+        self.h2d = torch.cuda.Stream()
         self.back = torch.cuda.Stream()
-        self.done = {L.name: None for L in layers}
+        self.consumed = {g.name: None for g in groups}
+        self.done = {g.name: None for g in groups}
 
-    def step(self, sbl, layers):
+    def begin(self):
+        """Order the copy streams after everything already on the main stream."""
+        ev = torch.cuda.Event()
+        ev.record(self.main)
+        self.h2d.wait_event(ev)
+        self.back.wait_event(ev)
+
+    def step(self, sbl, groups):
         h2d = d2h = 0
-        for L in layers:
+        for g in groups:
+            with torch.cuda.stream(self.h2d):
+                if self.consumed[g.name] is not None:
+                    self.h2d.wait_event(self.consumed[g.name])  # the previous step's kernels read these inputs
+                g.x.copy_(g.x_host, non_blocking=True)
+                g.x1.copy_(g.x1_host, non_blocking=True)
+                h2d += g.x_host.numel() * 2 + g.x1_host.numel() * 2
+                for L in g.members:
+                    L.W.copy_(L.W_host, non_blocking=True)
+                    h2d += L.W_host.numel() * 4
+                copied = torch.cuda.Event()
+                copied.record(self.h2d)
             with torch.cuda.stream(self.main):
-                L.W.copy_(L.W_host, non_blocking=True)
-                L.x.copy_(L.x_host, non_blocking=True)
-                L.x1.copy_(L.x1_host, non_blocking=True)
-                h2d += L.W_host.numel() * 4 + L.x_host.numel() * 2 + L.x1_host.numel() * 2
-                if self.done[L.name] is not None:
-                    self.main.wait_event(self.done[L.name])  # the previous step's y copied back
-                sbl.sbl_prepare_weights(L.W, N, M, out=L.w)
-                sbl.sbl_linear(L.x, L.w, y=L.y, workspace=L.ws)
-                sbl.sbl_linear(L.x1, L.w, y=L.y1, workspace=L.ws)
+                self.main.wait_event(copied)
+                if self.done[g.name] is not None:
+                    self.main.wait_event(self.done[g.name])  # the previous step's y copied back
+                sbl.sbl_prepare_weights_grouped([L.W for L in g.members], N, M, outs=[L.w for L in g.members])
+                g.run(sbl)
+                g.run(sbl, decode=True)
                 computed = torch.cuda.Event()
                 computed.record(self.main)
+                self.consumed[g.name] = computed
             self.back.wait_event(computed)
             with torch.cuda.stream(self.back):
-                L.y_host.copy_(L.y, non_blocking=True)
-                L.y1_host.copy_(L.y1, non_blocking=True)
-                d2h += L.y.numel() * 4 + L.y1.numel() * 4
+                for L in g.members:
+                    L.y_host.copy_(L.y, non_blocking=True)
+                    L.y1_host.copy_(L.y1, non_blocking=True)
+                    d2h += L.y.numel() * 4 + L.y1.numel() * 4
                 ev = torch.cuda.Event()
                 ev.record(self.back)
-                self.done[L.name] = ev
+                self.done[g.name] = ev
         return h2d, d2h
 
     def join(self):
-        """Make the main stream wait for every copy back (end of a timed region)."""
+        """Make the main stream wait for every copy (end of a timed region)."""
+        self.main.wait_stream(self.h2d)
         self.main.wait_stream(self.back)
 
 
-def _decode_roofline(sbl, dev, hbm_peak, K=2048, O=7168, T=1, reps=64):
+def _decode_roofline(sbl, dev, hbm_peak, K=2048, O=7168, T=1, reps=64, group=1):
     """T-token decode of a 2048 -> 7168 layer over a pool of distinct packed weights
-    larger than 3x L2, replayed from a CUDA graph: per-call GB/s on algorithmic bytes."""
+    larger than 3x L2, replayed from a CUDA graph: per-call GB/s on algorithmic bytes.
+    With group > 1 every call is one sbl_linear_grouped over `group` such layers
+    sharing x (each with its own output)."""
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     per = O * K // 4
     pool = max(8, int(3 * l2 // per) + 1)
@@ -299,15 +349,24 @@ def _decode_roofline(sbl, dev, hbm_peak, K=2048, O=7168, T=1, reps=64):
     y1 = torch.empty((T, O), dtype=torch.float32, device=dev)
     ws = sbl.workspace_for(T, K, O, 2, 4, dev)
     ws_list = [sbl.PreparedWeights(p, base.row_scale, 2, 4, K) for p in packs]
+    ys = [torch.empty((T, O), dtype=torch.float32, device=dev) for _ in range(group)]
+
+    def call(i):
+        if group == 1:
+            sbl.sbl_linear(x1, ws_list[i % pool], y=y1, workspace=ws)
+        else:
+            sbl.sbl_linear_grouped(x1, [ws_list[(i * group + j) % pool] for j in range(group)], ys=ys,
+                                   workspace=ws)
+
     s = torch.cuda.Stream()
     with torch.cuda.stream(s):
-        for w in ws_list[:4]:
-            sbl.sbl_linear(x1, w, y=y1, workspace=ws)
+        for i in range(4):
+            call(i)
     s.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=s):
         for i in range(reps):
-            sbl.sbl_linear(x1, ws_list[i % pool], y=y1, workspace=ws)
+            call(i)
     torch.cuda.synchronize()
     n_rep = 10
     batches = []
@@ -331,14 +390,15 @@ def _decode_roofline(sbl, dev, hbm_peak, K=2048, O=7168, T=1, reps=64):
         flush.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        sbl.sbl_linear(x1, ws_list[i % pool], y=y1, workspace=ws)
+        call(i)
         b.record()
         torch.cuda.synchronize()
         iso.append(a.elapsed_time(b) / 1e3)
-    byts = O * K / 4 + 4 * O + T * (2 * K + 4 * O)
+    byts = group * (O * K / 4 + 4 * O + T * 4 * O) + T * 2 * K
     del g, packs, ws_list, flush
     ach = byts / per_call_s / 1e9
-    return {"layer": f"{K}->{O} 2:4 T={T}", "bytes_per_call": byts, "calls_in_graph": reps, "weight_pool": pool,
+    return {"layer": f"{K}->{O} 2:4 T={T}" + (f", {group} layers per grouped call" if group > 1 else ""),
+            "bytes_per_call": byts, "calls_in_graph": reps, "weight_pool": pool,
             "us_per_call": per_call_s * 1e6, "achieved_gbs": ach, "peak_gbs": hbm_peak, "frac": ach / hbm_peak,
             "isolated_call_us": statistics.median(iso) * 1e6}
 
@@ -407,6 +467,29 @@ def _prefill_roofline(sbl, dev, int8_peak_tops, hbm_peak):
         for shape in ("gate", "down")}
     torch.cuda.nvtx.range_pop()
     return out
+
+
+def _int8_peak(dev, n=8192, reps=20):
+    """Dense int8 tensor throughput of the library GEMM (cuBLASLt through
+    torch._int_mm) on n x n x n, best of `reps` after warm-up: the measured
+    counterpart of the nominal int8 = 2 x bf16 peak."""
+    a = torch.randint(-128, 127, (n, n), dtype=torch.int8, device=dev)
+    b = torch.randint(-128, 127, (n, n), dtype=torch.int8, device=dev).t()
+    for _ in range(3):
+        torch._int_mm(a, b)
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        torch._int_mm(a, b)
+        e1.record()
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1) / 1e3)
+    best = min(ts)
+    return {"shape": f"{n}^3 int8 -> int32", "best_us": best * 1e6, "median_us": statistics.median(ts) * 1e6,
+            "tops_best": 2.0 * n ** 3 / best / 1e12, "tops_median": 2.0 * n ** 3 / statistics.median(ts) / 1e12,
+            "nominal_2x_bf16_measured": 2.0 * _peaks()[1]}
 
 
 def _flushed_graph_us(fn, dev, reps=10):
@@ -632,11 +715,11 @@ def run_ours(args, rank, world, dev):
     import sparse_linear_layers_b200 as sbl
     hbm_peak, bf16_peak, bf16_sus, peak_kind = _peaks()
     int8_peak_tops = 2.0 * bf16_peak  # nominal dense int8 : bf16 ratio of B200 (4.5 : 2.25 POPS)
-    layers = [Layer(nm, K, O, dev) for nm, K, O in synthetic.QWEN05_LAYER]
+    layers, groups = make_step(dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
     stream = torch.cuda.Stream()
-    graphs = StepGraphs(sbl, layers, stream)
+    graphs = StepGraphs(sbl, layers, groups, stream)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             flush.zero_()
@@ -668,7 +751,7 @@ def run_ours(args, rank, world, dev):
     # prefill contraction roofline (quantisation + tcgen05 GEMM, the dominant phase)
     pre_s_per_step = phase_ms["prefill"] / 1e3
     ops = sum(L.prefill_ops() for L in layers)
-    byts = sum(L.prefill_bytes() for L in layers)
+    byts = sum(g.prefill_bytes() for g in groups)
     t_tensor = ops / (int8_peak_tops * 1e12)
     t_hbm = byts / (hbm_peak * 1e9)
     if t_hbm >= t_tensor:
@@ -677,10 +760,11 @@ def run_ours(args, rank, world, dev):
     else:
         ach = ops / pre_s_per_step / 1e12
         roof = {"bound": "tensor", "achieved": ach, "peak": int8_peak_tops, "unit": "TOPS", "frac": ach / int8_peak_tops}
-    n_calls = len(layers)
+    n_calls = len(groups)
     traffic = PREFILL_TRAFFIC["bytes_per_call"] if _kernel_sources_digest() == PREFILL_TRAFFIC["sources_sha256"] else None
     roof.update({"traffic": traffic, "traffic_unit": "bytes per launch (DRAM read+write, ncu)",
-                 "kernel": "prefill sbl_linear call (activation quant + tcgen05 int8 GEMM), mean over the 7 projections",
+                 "kernel": "prefill call per input group (one activation quantisation + the tcgen05 int8 GEMM of "
+                           "each projection), mean over the 4 groups {q,k,v}, o, {gate,up}, down",
                  "launches_per_step": n_calls, "us_per_launch": pre_s_per_step * 1e6 / n_calls,
                  "algorithmic_bytes_per_launch": byts / n_calls, "algorithmic_ops_per_launch": ops / n_calls,
                  "peak_source": f"{peak_kind} (int8 = 2 x bf16 burst)" if roof["bound"] == "tensor"
@@ -689,20 +773,23 @@ def run_ours(args, rank, world, dev):
     prep_bytes = sum(L.O * L.K * 4 + L.O * L.K / 4 + 4 * L.O for L in layers)
     phases = {name: {"us_per_step": 1e3 * v} for name, v in phase_ms.items()}
     phases["prep"]["gbs"] = prep_bytes / (phase_ms["prep"] / 1e3) / 1e9
-    phases["decode"]["gbs"] = sum(L.decode_bytes() for L in layers) / (phase_ms["decode"] / 1e3) / 1e9
+    phases["decode"]["gbs"] = sum(g.decode_bytes() for g in groups) / (phase_ms["decode"] / 1e3) / 1e9
+    phases["decode"]["frac_of_hbm"] = phases["decode"]["gbs"] / hbm_peak
 
     # end to end through host buffers
-    e2e = E2E(layers)
+    e2e = E2E(groups)
+    e2e.begin()
     for _ in range(2):
-        e2e.step(sbl, layers)
+        e2e.step(sbl, groups)
     e2e.join()
     torch.cuda.synchronize()
     _barrier(world)
     K_e2e = min(K, 50)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(e2e.main)
+    e2e.begin()
     for _ in range(K_e2e):
-        h2d, d2h = e2e.step(sbl, layers)
+        h2d, d2h = e2e.step(sbl, groups)
     e2e.join()
     e1.record(e2e.main)
     torch.cuda.synchronize()
@@ -711,12 +798,15 @@ def run_ours(args, rank, world, dev):
     decode = _decode_roofline(sbl, dev, hbm_peak) if rank == 0 else None
     if decode is not None:
         decode["T8"] = _decode_roofline(sbl, dev, hbm_peak, T=8)
+        decode["grouped4"] = _decode_roofline(sbl, dev, hbm_peak, reps=16, group=4)
     prefill_big = _prefill_roofline(sbl, dev, int8_peak_tops, hbm_peak) if rank == 0 else None
     configs = _configs_sweep(sbl, dev) if rank == 0 and not args.no_configs else None
     rms_front = _rmsnorm_front(sbl, dev, hbm_peak) if rank == 0 and not args.no_configs else None
     mask_mon = _mask_monitor_bench(sbl, dev, hbm_peak) if rank == 0 and not args.no_configs else None
     ste_bwd = _ste_backward_bench(sbl, dev) if rank == 0 and not args.no_configs else None
-    launches_per_step = len(layers) * (1 + 2 + 1)  # prep + (quant + tcgen05 GEMM) + fused decode
+    # prep: one launch per K; prefill: per group one quantisation and one tcgen05 GEMM launch
+    # (a group's layers share it); decode: one launch per group (it quantises x itself)
+    launches_per_step = len(PREP_BY_K) + 2 * len(groups) + len(groups)
     value = _throughput(world, K, total_s)
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
@@ -745,13 +835,17 @@ def run_ours(args, rank, world, dev):
 # --------------------------------------------------------------------------- oracle arm
 
 def _oracle_inputs():
-    """The step's inputs for the oracle: the same seeded draws as the GPU step."""
+    """The step's inputs for the oracle: the same seeded draws as the GPU step
+    (one activation matrix per input group, shared by its projections)."""
     out = []
-    for nm, K, O in synthetic.QWEN05_LAYER:
-        W = synthetic.latent_weights(O, K, seed=0, tag=f"bench-{nm}")
-        _, xv = synthetic.activations(T_PREFILL, K, seed=0, tag=f"bench-x-{nm}")
-        _, x1 = synthetic.activations(T_DECODE, K, seed=0, tag=f"bench-x1-{nm}")
-        out.append((W, xv, x1))
+    K_of = {nm: K for nm, K, _ in synthetic.QWEN05_LAYER}
+    O_of = {nm: O for nm, _, O in synthetic.QWEN05_LAYER}
+    for g, names in INPUT_GROUPS:
+        K = K_of[names[0]]
+        _, xv = synthetic.activations(T_PREFILL, K, seed=0, tag=f"bench-x-{g}")
+        _, x1 = synthetic.activations(T_DECODE, K, seed=0, tag=f"bench-x1-{g}")
+        for nm in names:
+            out.append((synthetic.latent_weights(O_of[nm], K, seed=0, tag=f"bench-{nm}"), xv, x1))
     return out
 
 
@@ -857,7 +951,7 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration sweep (profiling runs)")
-    ap.add_argument("--only", choices=("rmsnorm_front", "mask_monitor", "ste_backward"),
+    ap.add_argument("--only", choices=("rmsnorm_front", "mask_monitor", "ste_backward", "int8_peak"),
                     help="run only this auxiliary measurement on one GPU and print its JSON (profiling runs)")
     ap.add_argument("--tokens", type=int, default=32768, help="tokens of the --only rmsnorm_front measurement")
     args = ap.parse_args()
@@ -882,6 +976,8 @@ def main():
             res = _rmsnorm_front(sbl, dev, hbm_peak, T=args.tokens)
         elif args.only == "mask_monitor":
             res = _mask_monitor_bench(sbl, dev, hbm_peak)
+        elif args.only == "int8_peak":
+            res = _int8_peak(dev)
         else:
             res = _ste_backward_bench(sbl, dev)
         print(json.dumps({"only": args.only, "result": res}), flush=True)

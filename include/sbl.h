@@ -47,6 +47,10 @@ typedef enum {
     SBL_ERR_WORKSPACE = 6      /* workspace missing, too small or unaligned         */
 } sbl_status;
 
+/* Most weight matrices one grouped call takes (sbl_prepare_weights_grouped,
+ * sbl_linear_grouped). */
+#define SBL_MAX_GROUP 8
+
 /* Output element types of sbl_linear. */
 enum { SBL_F32 = 0, SBL_BF16 = 1 };
 
@@ -109,6 +113,19 @@ sbl_status sbl_prepare_weights(const float* W, int64_t O, int64_t K, int n, int 
 sbl_status sbl_prepare_weights_ex(const float* W, int64_t O, int64_t K, int n, int m,
                                   uint8_t* packed, float* row_scale, uint8_t* mask_bits,
                                   int flags, void* stream);
+
+/*
+ * sbl_prepare_weights_grouped — sbl_prepare_weights for G weight matrices of
+ * the same K in one call (the projections of one layer), with the per-row
+ * scale and no flags.  W, O, packed, row_scale: HOST arrays of G entries
+ * (device pointers, row counts O[g] >= 0); mask_bits: NULL or a host array of
+ * G device pointers (entries may be NULL).  Each matrix's results are exactly
+ * sbl_prepare_weights'; rows up to K = 8192 are prepared by one launch over
+ * the stacked rows.  1 <= G <= SBL_MAX_GROUP, else SBL_ERR_INVALID_ARG.
+ */
+sbl_status sbl_prepare_weights_grouped(int G, const float* const* W, const int64_t* O, int64_t K, int n, int m,
+                                       uint8_t* const* packed, float* const* row_scale, uint8_t* const* mask_bits,
+                                       void* stream);
 
 /*
  * sbl_quant_act — per-token absmax int8 activation quantisation.
@@ -351,6 +368,38 @@ sbl_status sbl_linear_rmsnorm(const uint16_t* x_bf16, const float* g, float eps,
 sbl_status sbl_linear_noalloc(const uint16_t* x_bf16, int64_t T, int64_t K,
                               const uint8_t* packed, const float* row_scale, int64_t O, int n, int m,
                               void* y, int y_dtype, int32_t* acc_out, void* stream);
+
+/*
+ * sbl_linear_grouped — G layers that read the same activations (the q, k and v
+ * projections of an attention block; the gate and up projections of an FFN)
+ * in one call.
+ *
+ * Each result is exactly sbl_linear's for that layer (the Sparse-BitNet
+ * Guide, "Mathematical Formulation of Sparse-BitLinear", applied per weight
+ * matrix; the activations' int8 codes and scales depend on x alone, so one
+ * quantisation serves every layer).
+ *   packed, row_scale, O, y   HOST arrays of G entries: layer g's prepared
+ *                             weights (device pointers), its row count
+ *                             (O[g] >= 0; 0 skips it) and its [T, O[g]]
+ *                             output (device pointer); acc_out: NULL, or a
+ *                             host array of G device pointers (entries may
+ *                             be NULL).
+ *   x_bf16, T, K, n, m, y_dtype  as sbl_linear; one pattern for all layers.
+ *   workspace   for prefill sizes, sbl_linear_grouped_workspace_bytes(T, K)
+ *               bytes, 256-byte aligned (else SBL_ERR_WORKSPACE); decode
+ *               sizes use none (NULL allowed).
+ * One or two tokens: one launch streams all G weight matrices (one pass of
+ * their stacked rows).  Three to 16 tokens: the warp-level MMA decode per
+ * layer.  Prefill: x is quantised once, then one launch of the one-CTA
+ * tensor-core GEMM schedules the output tiles of up to four layers together
+ * (the CTA-pair and 2:4 sparse kernels and the split along k are not used).
+ * 1 <= G <= SBL_MAX_GROUP, else SBL_ERR_INVALID_ARG.
+ */
+size_t sbl_linear_grouped_workspace_bytes(int64_t T, int64_t K);
+sbl_status sbl_linear_grouped(const uint16_t* x_bf16, int64_t T, int64_t K, int G, const uint8_t* const* packed,
+                              const float* const* row_scale, const int64_t* O, int n, int m, void* const* y,
+                              int y_dtype, int32_t* const* acc_out, void* workspace, size_t workspace_bytes,
+                              void* stream);
 
 /*
  * sbl_linear_plan — the contraction path sbl_linear takes for these sizes on

@@ -25,6 +25,8 @@ SBL_PREP_SCALE_GLOBAL = 2
 
 SBL_BWD_DW_TERNARY = 1
 
+SBL_MAX_GROUP = 8
+
 SBL_F32 = 0
 SBL_BF16 = 1
 
@@ -41,6 +43,7 @@ _f32 = ctypes.c_float
 SIGNATURES = {
     "sbl_prepare_weights": (_int, [_vp, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp]),
     "sbl_prepare_weights_ex": (_int, [_vp, _i64, _i64, _int, _int, _vp, _vp, _vp, _int, _vp]),
+    "sbl_prepare_weights_grouped": (_int, [_int, _vp, _vp, _i64, _int, _int, _vp, _vp, _vp, _vp]),
     "sbl_quant_act": (_int, [_vp, _i64, _i64, _vp, _vp, _vp]),
     "sbl_rmsnorm_quant_act": (_int, [_vp, _vp, _f32, _i64, _i64, _vp, _vp, _vp]),
     "sbl_linear_workspace_bytes": (_sz, [_i64, _i64, _i64, _int, _int]),
@@ -48,6 +51,8 @@ SIGNATURES = {
     "sbl_linear_path": (_int, [_vp, _i64, _i64, _vp, _vp, _i64, _int, _int, _vp, _int, _vp, _vp, _sz, _int, _vp]),
     "sbl_linear_rmsnorm": (_int, [_vp, _vp, _f32, _i64, _i64, _vp, _vp, _i64, _int, _int, _vp, _int, _vp, _vp, _sz,
                                   _int, _vp]),
+    "sbl_linear_grouped_workspace_bytes": (_sz, [_i64, _i64]),
+    "sbl_linear_grouped": (_int, [_vp, _i64, _i64, _int, _vp, _vp, _vp, _int, _int, _vp, _int, _vp, _vp, _sz, _vp]),
     "sbl_linear_noalloc": (_int, [_vp, _i64, _i64, _vp, _vp, _i64, _int, _int, _vp, _int, _vp, _vp]),
     "sbl_linear_plan": (_int, [_i64, _i64, _i64, _int, _int, _sz]),
     "sbl_mask_monitor": (_int, [_vp, _vp, _i64, _i64, _int, _int, _vp, _vp, _vp]),

@@ -101,6 +101,42 @@ def sbl_prepare_weights(W: torch.Tensor, n: int, m: int, with_mask: bool = False
     return out
 
 
+def sbl_prepare_weights_grouped(Ws, n: int, m: int, outs=None, with_mask: bool = False,
+                                stream: Optional[torch.cuda.Stream] = None):
+    """sbl_prepare_weights for several latent matrices of the same K in one call
+    (per-row scales); returns the list of PreparedWeights."""
+    import ctypes
+    G = len(Ws)
+    if not 1 <= G <= _lib.SBL_MAX_GROUP:
+        raise ValueError(f"between 1 and {_lib.SBL_MAX_GROUP} matrices, got {G}")
+    K = _need_2d(Ws[0], "W[0]")[1]
+    dev = Ws[0].device
+    for g, W in enumerate(Ws):
+        if _need_2d(W, f"W[{g}]")[1] != K:
+            raise ValueError("every matrix must have the same K")
+        _need_cuda(W, f"W[{g}]", torch.float32, None, dev)
+    if outs is None:
+        outs = [PreparedWeights(torch.empty((W.shape[0], K // 4), dtype=torch.uint8, device=dev),
+                                torch.empty((W.shape[0],), dtype=torch.float32, device=dev), n, m, K,
+                                torch.empty((W.shape[0], K // 8), dtype=torch.uint8, device=dev) if with_mask else None)
+                for W in Ws]
+    if len(outs) != G:
+        raise ValueError("one output per matrix")
+    for W, o in zip(Ws, outs):
+        if o.K != K or o.O != W.shape[0]:
+            raise ValueError("outputs must match the matrices' shapes")
+        _need_weights(o, dev)
+        if o.mask_bits is not None:
+            _need_cuda(o.mask_bits, "mask_bits", torch.uint8, (o.O, K // 8), dev)
+    ptrs = lambda ts: (ctypes.c_void_p * G)(*[t.data_ptr() if t is not None else None for t in ts])
+    rows = (ctypes.c_int64 * G)(*[W.shape[0] for W in Ws])
+    masks = ptrs([o.mask_bits for o in outs]) if any(o.mask_bits is not None for o in outs) else None
+    check(lib.sbl_prepare_weights_grouped(G, ptrs(Ws), rows, K, n, m, ptrs([o.packed for o in outs]),
+                                          ptrs([o.row_scale for o in outs]), masks, _stream(stream)),
+          "sbl_prepare_weights_grouped")
+    return outs
+
+
 def sbl_quant_act(x: torch.Tensor, stream: Optional[torch.cuda.Stream] = None):
     """Per-token absmax int8 quantisation: returns (x_q int8 [T,K], s_tok fp32 [T])."""
     T, K = _need_2d(x, "x")
@@ -163,6 +199,47 @@ def sbl_linear(x: torch.Tensor, w: PreparedWeights, out_dtype: torch.dtype = tor
                               workspace.data_ptr(), workspace.numel(), _PATHS[path], _stream(stream)),
           "sbl_linear")
     return y
+
+
+def sbl_linear_grouped(x: torch.Tensor, ws, out_dtype: torch.dtype = torch.float32, ys=None, acc_outs=None,
+                       workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None):
+    """Several layers that read the same x (q/k/v, gate/up) in one call: x is
+    quantised once; returns the list of y [T, O_g].  Each result is exactly
+    sbl_linear's for that layer.  ``ws``: PreparedWeights with one N:M
+    pattern and one K; ``acc_outs``: None or a list (entries may be None)."""
+    import ctypes
+    T, K = _need_2d(x, "x")
+    _need_cuda(x, "x", torch.bfloat16)
+    G = len(ws)
+    if not 1 <= G <= _lib.SBL_MAX_GROUP:
+        raise ValueError(f"between 1 and {_lib.SBL_MAX_GROUP} layers, got {G}")
+    n, m = ws[0].n, ws[0].m
+    for w in ws:
+        if w.K != K or (w.n, w.m) != (n, m):
+            raise ValueError("every layer must have the activations' K and one N:M pattern")
+        _need_weights(w, x.device)
+    if ys is None:
+        ys = [torch.empty((T, w.O), dtype=out_dtype, device=x.device) for w in ws]
+    if len(ys) != G or (acc_outs is not None and len(acc_outs) != G):
+        raise ValueError("one output (and accumulator) per layer")
+    for g, (w, yg) in enumerate(zip(ws, ys)):
+        if yg.dtype not in (torch.float32, torch.bfloat16) or yg.dtype != ys[0].dtype:
+            raise ValueError("outputs must all be float32 or all bfloat16")
+        _need_cuda(yg, f"y[{g}]", yg.dtype, (T, w.O), x.device)
+        if acc_outs is not None and acc_outs[g] is not None:
+            _need_cuda(acc_outs[g], f"acc_out[{g}]", torch.int32, (T, w.O), x.device)
+    if workspace is None:
+        workspace = torch.empty((max(1, int(lib.sbl_linear_grouped_workspace_bytes(T, K))),), dtype=torch.uint8,
+                                device=x.device)
+    _need_workspace(workspace, x.device)
+    ptrs = lambda ts: (ctypes.c_void_p * G)(*[t.data_ptr() if t is not None else None for t in ts])
+    rows = (ctypes.c_int64 * G)(*[w.O for w in ws])
+    accs = ptrs(acc_outs) if acc_outs is not None else None
+    ydt = _lib.SBL_F32 if ys[0].dtype == torch.float32 else _lib.SBL_BF16
+    check(lib.sbl_linear_grouped(x.data_ptr(), T, K, G, ptrs([w.packed for w in ws]), ptrs([w.row_scale for w in ws]),
+                                 rows, n, m, ptrs(ys), ydt, accs, workspace.data_ptr(), workspace.numel(),
+                                 _stream(stream)), "sbl_linear_grouped")
+    return ys
 
 
 def sbl_linear_rmsnorm(x: torch.Tensor, w: PreparedWeights, g: torch.Tensor, eps: float = RMSNORM_EPS_F32,

@@ -36,11 +36,18 @@ namespace sbl {
 
 constexpr int kDecodeThreads = 512;
 constexpr int kDecodeWarps = kDecodeThreads / 32;
-constexpr int kDecodeBatch = 4;  // chunks per lane in flight
+constexpr int kDecodeBatch = 4;      // chunks per lane in flight
+constexpr int kDecodeBatchWide = 16; // the same for calls too large for one batch per lane (one block per SM)
+constexpr int kDecodeMaxGroup = 8;  // weight matrices per launch
 // Two blocks of one-token passes share an SM, so the next call's blocks can
 // start (and prefetch their weights) while this one drains.
-template <int TT>
-constexpr int decode_min_blocks() { return TT == 1 ? 2 : 1; }
+// Blocks of kDecodeThreads threads; the wide batches use blocks of 128 (about
+// 128 registers a thread, four blocks per SM), so a large call spreads its
+// warps over every SM.
+template <int NB>
+constexpr int decode_threads() { return NB > kDecodeBatch ? 128 : kDecodeThreads; }
+template <int TT, int NB>
+constexpr int decode_min_blocks() { return NB > kDecodeBatch ? 4 : (TT == 1 ? 2 : 1); }
 
 template <int CW>
 __device__ __forceinline__ void load_chunk_words(const uint8_t* prow, int c, uint32_t (&w)[CW]) {
@@ -55,24 +62,54 @@ __device__ __forceinline__ void load_chunk_words(const uint8_t* prow, int c, uin
     }
 }
 
-template <int L, int TT, int CW>
-__global__ void __launch_bounds__(kDecodeThreads, decode_min_blocks<TT>()) decode_kernel(const uint8_t* __restrict__ packed,
-                                                                const float* __restrict__ row_scale, long long O,
-                                                                int K, const uint16_t* __restrict__ x, long long T,
-                                                                long long t0, void* __restrict__ y, int y_bf16,
-                                                                int32_t* __restrict__ acc_out, unsigned* status) {
+// The weight matrices of one launch: G matrices that share the activations x,
+// their rows stacked (matrix g owns the rows row_end[g - 1] .. row_end[g] - 1
+// of the launch), each with its own codes, scales and outputs.  A single
+// layer is G = 1.
+struct DecodeGroup {
+    const uint8_t* packed[kDecodeMaxGroup];
+    const float* row_scale[kDecodeMaxGroup];
+    void* y[kDecodeMaxGroup];
+    int32_t* acc_out[kDecodeMaxGroup];
+    long long O[kDecodeMaxGroup];
+    long long row_end[kDecodeMaxGroup];
+    int G;
+};
+
+template <int L, int TT, int CW, int NB>
+__global__ void __launch_bounds__(decode_threads<NB>(), decode_min_blocks<TT, NB>()) decode_kernel(const DecodeGroup grp, int K,
+                                                                const uint16_t* __restrict__ x, long long T,
+                                                                long long t0, int y_bf16, unsigned* status) {
     extern __shared__ uint4 xs[];  // TT x K/16 units of quantised activations (decode layout)
-    __shared__ uint32_t red[kDecodeWarps][TT];
+    constexpr int NTH = decode_threads<NB>();
+    constexpr int NWP = NTH / 32;
+    __shared__ uint32_t red[NWP][TT];
     __shared__ float s_sh[TT];
     asm volatile("griddepcontrol.launch_dependents;");
     constexpr int RW = 32 / L;
-    constexpr int NB = kDecodeBatch;
     const int CPR = K / (16 * CW);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int sub = lane / L, li = lane % L;
-    const long long g = static_cast<long long>(blockIdx.x) * kDecodeWarps + warp;
-    const long long row = g * RW + sub;
-    const bool valid = row < O;
+    const long long gr = static_cast<long long>(blockIdx.x) * NWP + warp;
+    const long long grow = gr * RW + sub;  // row of the stacked matrices
+    const bool valid = grow < grp.row_end[grp.G - 1];
+    // the matrix this row belongs to (constant indices only: no local copy of the group)
+    const uint8_t* packed = grp.packed[0];
+    const float* row_scale = grp.row_scale[0];
+    void* y = grp.y[0];
+    int32_t* acc_out = grp.acc_out[0];
+    long long O = grp.O[0], row = grow;
+    if (grp.G > 1)
+#pragma unroll
+    for (int i = 1; i < kDecodeMaxGroup; ++i)
+        if (i < grp.G && grow >= grp.row_end[i - 1]) {
+            packed = grp.packed[i];
+            row_scale = grp.row_scale[i];
+            y = grp.y[i];
+            acc_out = grp.acc_out[i];
+            O = grp.O[i];
+            row = grow - grp.row_end[i - 1];
+        }
     const uint8_t* prow = packed + (valid ? row : 0) * (K >> 2);
 
     // Before the dependency wait: warm L2 with this lane's first batch of weights.
@@ -98,7 +135,7 @@ __global__ void __launch_bounds__(kDecodeThreads, decode_min_blocks<TT>()) decod
     // Quantise this pass's tokens: per-token absmax, then int8 into shared memory.
     const int nvec = K >> 3;
     const int nblk = K >> 4;
-    if (TT == 1 && nblk <= kDecodeThreads) {
+    if (TT == 1 && nblk <= NTH) {
         // one token, K <= 8192: each thread keeps its 16-element block in
         // registers between the absmax and the quantisation
         constexpr int XB = 1;
@@ -108,7 +145,7 @@ __global__ void __launch_bounds__(kDecodeThreads, decode_min_blocks<TT>()) decod
         uint32_t mx = 0;
 #pragma unroll
         for (int i = 0; i < XB; ++i) {
-            const int b = threadIdx.x + i * kDecodeThreads;
+            const int b = threadIdx.x + i * NTH;
             if (b < nblk) {
                 xa[i][0] = ldg_nc(xr + 2 * b);
                 xa[i][1] = ldg_nc(xr + 2 * b + 1);
@@ -120,7 +157,7 @@ __global__ void __launch_bounds__(kDecodeThreads, decode_min_blocks<TT>()) decod
         __syncthreads();
         mx = 0;
 #pragma unroll
-        for (int w = 0; w < kDecodeWarps; ++w) mx = max(mx, red[w][0]);
+        for (int w = 0; w < NWP; ++w) mx = max(mx, red[w][0]);
         const float st = __fdiv_rn(127.0f, fmaxf(__uint_as_float(mx << 16), 1e-5f));
         if (threadIdx.x == 0) {
             if (mx >= 0x7F80u && blockIdx.x == 0) raise_status(status, kStatusNonfinite);
@@ -128,7 +165,7 @@ __global__ void __launch_bounds__(kDecodeThreads, decode_min_blocks<TT>()) decod
         }
 #pragma unroll
         for (int i = 0; i < XB; ++i) {
-            const int b = threadIdx.x + i * kDecodeThreads;
+            const int b = threadIdx.x + i * NTH;
             if (b < nblk) {
                 const int pos = CW == 4 ? (b & 3) * CPR + (b >> 2) : b;
                 xs[pos] = quant_block16<true>(xa[i][0], xa[i][1], st);
@@ -141,7 +178,7 @@ __global__ void __launch_bounds__(kDecodeThreads, decode_min_blocks<TT>()) decod
             const long long tt = t0 + t < T ? t0 + t : T - 1;
             const uint4* xr = reinterpret_cast<const uint4*>(x + tt * K);
             uint32_t mx = 0;
-            for (int v = threadIdx.x; v < nvec; v += kDecodeThreads) mx = absmax8(ldg_nc(xr + v), mx);
+            for (int v = threadIdx.x; v < nvec; v += NTH) mx = absmax8(ldg_nc(xr + v), mx);
             mx = __reduce_max_sync(0xFFFFFFFFu, mx);
             if (lane == 0) red[warp][t] = mx;
         }
@@ -149,7 +186,7 @@ __global__ void __launch_bounds__(kDecodeThreads, decode_min_blocks<TT>()) decod
         if (threadIdx.x < TT) {
             uint32_t mx = 0;
 #pragma unroll
-            for (int w = 0; w < kDecodeWarps; ++w) mx = max(mx, red[w][threadIdx.x]);
+            for (int w = 0; w < NWP; ++w) mx = max(mx, red[w][threadIdx.x]);
             if (mx >= 0x7F80u && blockIdx.x == 0) raise_status(status, kStatusNonfinite);
             s_sh[threadIdx.x] = __fdiv_rn(127.0f, fmaxf(__uint_as_float(mx << 16), 1e-5f));
         }
@@ -159,7 +196,7 @@ __global__ void __launch_bounds__(kDecodeThreads, decode_min_blocks<TT>()) decod
             const long long tt = t0 + t < T ? t0 + t : T - 1;
             const uint4* xr = reinterpret_cast<const uint4*>(x + tt * K);
             const float st = s_sh[t];
-            for (int b = threadIdx.x; b < nblk; b += kDecodeThreads) {
+            for (int b = threadIdx.x; b < nblk; b += NTH) {
                 const int pos = CW == 4 ? (b & 3) * CPR + (b >> 2) : b;
                 xs[t * nblk + pos] = quant_block16<true>(ldg_nc(xr + 2 * b), ldg_nc(xr + 2 * b + 1), st);
             }
@@ -261,44 +298,67 @@ __global__ void __launch_bounds__(kDecodeThreads, decode_min_blocks<TT>()) decod
     }
 }
 
-// Lanes per row.  The call should fit in one block of kDecodeWarps warps per
-// SM, which leaves room on each SM for the next call's block, with every load
-// in flight at once: among the lane counts whose warps fit, take the best
-// chunk utilisation per batch of loads (ties: more lanes per row).
-static int choose_lanes(long long O, int cpr, int num_sms) {
-    const long long cap = static_cast<long long>(num_sms) * kDecodeWarps;
-    int best = 1;
-    double best_score = -1.0;
-    for (int L = 32; L >= 1; L >>= 1) {
-        const long long warps = (O + (32 / L) - 1) / (32 / L);
-        if (warps > cap) continue;
-        const int per_lane = (cpr + L - 1) / L;
-        const double eff = static_cast<double>(cpr) / (static_cast<double>(per_lane) * L);
-        const double score = eff / ((per_lane + kDecodeBatch - 1) / kDecodeBatch);
-        if (score > best_score + 1e-9) {
-            best_score = score;
-            best = L;
+// Lanes per row and chunks per lane in flight.  A call should fit in one block
+// of kDecodeWarps warps per SM, which leaves room on each SM for the next
+// call's block, with every load in flight at once: among the lane counts whose
+// warps fit, take the best chunk utilisation per batch of loads (ties: more
+// lanes per row).  A call too large for that (several batches per lane: big
+// layers, or several layers in one grouped launch) of one or two tokens takes
+// batches of kDecodeBatchWide chunks (more registers: 16 warps per SM in
+// blocks of four) when that needs fewer batches.
+struct DecodePlan {
+    int L;
+    int NB;
+};
+
+static DecodePlan choose_plan(long long O, int cpr, int num_sms, int tt, bool wide) {
+    auto best_for = [&](int nb, long long cap, int& batches) {
+        int best = 1;
+        double best_score = -1.0;
+        batches = 1 << 30;
+        for (int L = 32; L >= 1; L >>= 1) {
+            const long long warps = (O + (32 / L) - 1) / (32 / L);
+            if (warps > cap) continue;
+            const int per_lane = (cpr + L - 1) / L;
+            const double eff = static_cast<double>(cpr) / (static_cast<double>(per_lane) * L);
+            const int nbat = (per_lane + nb - 1) / nb;
+            const double score = eff / nbat;
+            if (score > best_score + 1e-9) {
+                best_score = score;
+                best = L;
+                batches = nbat;
+            }
         }
+        return best;
+    };
+    const long long cap = static_cast<long long>(num_sms) * kDecodeWarps;
+    int b1 = 0;
+    const int L1 = best_for(kDecodeBatch, cap, b1);
+    if (tt <= 2 && wide && b1 > 1) {
+        int b2 = 0;
+        const int L2 = best_for(kDecodeBatchWide, cap, b2);
+        if (b2 < b1) return {L2, kDecodeBatchWide};
     }
-    return best;
+    return {L1, kDecodeBatch};
 }
 
-template <int L, int TT, int CW>
-static cudaError_t launch_decode_lt(const uint8_t* packed, const float* row_scale, long long O, int K,
-                                    const uint16_t* x, long long T, long long t0, void* y, int y_bf16,
-                                    int32_t* acc_out, unsigned* status, cudaStream_t stream) {
+template <int L, int TT, int CW, int NB>
+static cudaError_t launch_decode_lt(const DecodeGroup& grp, int K, const uint16_t* x, long long T, long long t0,
+                                    int y_bf16, unsigned* status, cudaStream_t stream) {
     constexpr int RW = 32 / L;
-    const long long groups = (O + RW - 1) / RW;
-    const long long blocks = (groups + kDecodeWarps - 1) / kDecodeWarps;
+    const long long rows = grp.row_end[grp.G - 1];
+    const long long groups = (rows + RW - 1) / RW;
+    constexpr int NTH = decode_threads<NB>();
+    const long long blocks = (groups + NTH / 32 - 1) / (NTH / 32);
     const size_t smem = static_cast<size_t>(TT) * K;
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<L, TT, CW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<L, TT, CW, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return e;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(blocks));
-    cfg.blockDim = dim3(kDecodeThreads);
+    cfg.blockDim = dim3(NTH);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -306,55 +366,100 @@ static cudaError_t launch_decode_lt(const uint8_t* packed, const float* row_scal
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_kernel<L, TT, CW>, packed, row_scale, O, K, x, T, t0, y, y_bf16, acc_out,
-                              status);
+    return cudaLaunchKernelEx(&cfg, decode_kernel<L, TT, CW, NB>, grp, K, x, T, t0, y_bf16, status);
 }
 
-template <int TT, int CW>
-static cudaError_t launch_decode_t(int L, const uint8_t* packed, const float* row_scale, long long O, int K,
-                                   const uint16_t* x, long long T, long long t0, void* y, int y_bf16,
-                                   int32_t* acc_out, unsigned* status, cudaStream_t stream) {
+template <int TT, int CW, int NB>
+static cudaError_t launch_decode_t(int L, const DecodeGroup& grp, int K, const uint16_t* x, long long T,
+                                   long long t0, int y_bf16, unsigned* status, cudaStream_t stream) {
 #define SBL_DECODE_CASE(LV) \
-    case LV: return launch_decode_lt<LV, TT, CW>(packed, row_scale, O, K, x, T, t0, y, y_bf16, acc_out, status, stream);
+    case LV: return launch_decode_lt<LV, TT, CW, NB>(grp, K, x, T, t0, y_bf16, status, stream);
     switch (L) {
         SBL_DECODE_CASE(32)
         SBL_DECODE_CASE(16)
         SBL_DECODE_CASE(8)
         SBL_DECODE_CASE(4)
         SBL_DECODE_CASE(2)
-        default: return launch_decode_lt<1, TT, CW>(packed, row_scale, O, K, x, T, t0, y, y_bf16, acc_out, status, stream);
+        default: return launch_decode_lt<1, TT, CW, NB>(grp, K, x, T, t0, y_bf16, status, stream);
     }
 #undef SBL_DECODE_CASE
 }
 
 template <int TT>
-static cudaError_t launch_decode_cw(int L, bool wide, const uint8_t* packed, const float* row_scale, long long O,
-                                    int K, const uint16_t* x, long long T, long long t0, void* y, int y_bf16,
-                                    int32_t* acc_out, unsigned* status, cudaStream_t stream) {
-    if (wide)
-        return launch_decode_t<TT, 4>(L, packed, row_scale, O, K, x, T, t0, y, y_bf16, acc_out, status, stream);
-    return launch_decode_t<TT, 1>(L, packed, row_scale, O, K, x, T, t0, y, y_bf16, acc_out, status, stream);
+static cudaError_t launch_decode_cw(const DecodePlan& plan, bool wide, const DecodeGroup& grp, int K,
+                                    const uint16_t* x, long long T, long long t0, int y_bf16, unsigned* status,
+                                    cudaStream_t stream) {
+    if (wide) {
+        if constexpr (TT <= 2) {
+            if (plan.NB == kDecodeBatchWide)
+                return launch_decode_t<TT, 4, kDecodeBatchWide>(plan.L, grp, K, x, T, t0, y_bf16, status, stream);
+        }
+        return launch_decode_t<TT, 4, kDecodeBatch>(plan.L, grp, K, x, T, t0, y_bf16, status, stream);
+    }
+    return launch_decode_t<TT, 1, kDecodeBatch>(plan.L, grp, K, x, T, t0, y_bf16, status, stream);
 }
 
-// Decode for any T: passes of up to 8 tokens (later passes re-read the
-// weights, mostly from L2).  Needs K % 16 == 0 and TT * K bytes of shared memory.
-cudaError_t launch_decode(const uint8_t* packed, const float* row_scale, long long O, long long K,
-                          const uint16_t* x, long long T, void* y, int y_bf16, int32_t* acc_out, unsigned* status,
-                          int num_sms, cudaStream_t stream) {
+// Decode of G weight matrices that share x, for any T: passes of up to 8
+// tokens (later passes re-read the weights, mostly from L2).  Needs
+// K % 16 == 0, TT * K bytes of shared memory and 1 <= G <= kDecodeMaxGroup.
+static cudaError_t launch_decode_group(const DecodeGroup& grp, long long K, const uint16_t* x, long long T,
+                                       int y_bf16, int num_sms, cudaStream_t stream, unsigned* status) {
     const int Ki = static_cast<int>(K);
     const bool wide = (Ki % 64) == 0;
     const int cpr = wide ? Ki / 64 : Ki / 16;
-    const int L = choose_lanes(O, cpr, num_sms);
+    const long long rows = grp.row_end[grp.G - 1];
     for (long long t0 = 0; t0 < T; t0 += 8) {
         const long long rem = T - t0;
+        const int tt = rem > 4 ? 8 : rem > 2 ? 4 : static_cast<int>(rem);
+        const DecodePlan plan = choose_plan(rows, cpr, num_sms, tt, wide);
         cudaError_t e;
-        if (rem > 4) e = launch_decode_cw<8>(L, wide, packed, row_scale, O, Ki, x, T, t0, y, y_bf16, acc_out, status, stream);
-        else if (rem > 2) e = launch_decode_cw<4>(L, wide, packed, row_scale, O, Ki, x, T, t0, y, y_bf16, acc_out, status, stream);
-        else if (rem == 2) e = launch_decode_cw<2>(L, wide, packed, row_scale, O, Ki, x, T, t0, y, y_bf16, acc_out, status, stream);
-        else e = launch_decode_cw<1>(L, wide, packed, row_scale, O, Ki, x, T, t0, y, y_bf16, acc_out, status, stream);
+        if (tt == 8) e = launch_decode_cw<8>(plan, wide, grp, Ki, x, T, t0, y_bf16, status, stream);
+        else if (tt == 4) e = launch_decode_cw<4>(plan, wide, grp, Ki, x, T, t0, y_bf16, status, stream);
+        else if (tt == 2) e = launch_decode_cw<2>(plan, wide, grp, Ki, x, T, t0, y_bf16, status, stream);
+        else e = launch_decode_cw<1>(plan, wide, grp, Ki, x, T, t0, y_bf16, status, stream);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
+}
+
+cudaError_t launch_decode(const uint8_t* packed, const float* row_scale, long long O, long long K,
+                          const uint16_t* x, long long T, void* y, int y_bf16, int32_t* acc_out, unsigned* status,
+                          int num_sms, cudaStream_t stream) {
+    DecodeGroup grp = {};
+    grp.packed[0] = packed;
+    grp.row_scale[0] = row_scale;
+    grp.y[0] = y;
+    grp.acc_out[0] = acc_out;
+    grp.O[0] = O;
+    grp.row_end[0] = O;
+    grp.G = 1;
+    return launch_decode_group(grp, K, x, T, y_bf16, num_sms, stream, status);
+}
+
+int decode_max_group() { return kDecodeMaxGroup; }
+
+// G matrices (G <= decode_max_group()) that share x, in one launch per pass of
+// up to 8 tokens; matrix g has O[g] rows and its own packed, row_scale, y and
+// acc_out (which may be null).
+cudaError_t launch_decode_grouped(int G, const uint8_t* const* packed, const float* const* row_scale,
+                                  const long long* O, long long K, const uint16_t* x, long long T, void* const* y,
+                                  int y_bf16, int32_t* const* acc_out, unsigned* status, int num_sms,
+                                  cudaStream_t stream) {
+    if (G < 1 || G > kDecodeMaxGroup) return cudaErrorInvalidValue;
+    DecodeGroup grp = {};
+    long long end = 0;
+    for (int g = 0; g < G; ++g) {
+        grp.packed[g] = packed[g];
+        grp.row_scale[g] = row_scale[g];
+        grp.y[g] = y[g];
+        grp.acc_out[g] = acc_out ? acc_out[g] : nullptr;
+        grp.O[g] = O[g];
+        end += O[g];
+        grp.row_end[g] = end;
+    }
+    grp.G = G;
+    if (end == 0) return cudaSuccess;
+    return launch_decode_group(grp, K, x, T, y_bf16, num_sms, stream, status);
 }
 
 }  // namespace sbl

@@ -34,6 +34,7 @@
 // memory and exits.
 #include <cuda.h>
 
+#include <cstring>
 #include <type_traits>
 
 #include "sbl_common.cuh"
@@ -109,12 +110,59 @@ constexpr size_t prefill_smem_bytes() {
 static_assert(prefill_smem_bytes<256>() <= 232448, "prefill tile does not fit in shared memory");
 static_assert(prefill_smem_bytes<128>() <= 232448, "prefill tile does not fit in shared memory");
 
-template <int BN>
+// The weight matrices of one launch: G layers that read the same quantised
+// activations, each with its codes (tensor map), output (tensor map and
+// pointer), row scales and accumulators.  Their output tiles are numbered one
+// after the other: layer g owns the tiles nt_end[g - 1] .. nt_end[g] - 1 of
+// every token tile.  A single layer is G = 1.
+constexpr int kPrefillMaxGroup = 4;
+struct PrefillOut {
+    CUtensorMap tmap_w[kPrefillMaxGroup];
+    CUtensorMap tmap_y[kPrefillMaxGroup];
+    const float* row_scale[kPrefillMaxGroup];
+    void* y[kPrefillMaxGroup];
+    int32_t* acc_out[kPrefillMaxGroup];
+    int O[kPrefillMaxGroup];
+    int y_vec[kPrefillMaxGroup];
+    int nt_end[kPrefillMaxGroup];
+    int G;
+};
+
+// Layer of output tile nt (counted over all layers) and its tile within the layer.
+struct TileOwner {
+    const CUtensorMap* tmap_w;
+    const CUtensorMap* tmap_y;
+    const float* row_scale;
+    void* y;
+    int32_t* acc_out;
+    int O, y_vec, nt;
+};
+
+template <bool GROUPED>
+__device__ __forceinline__ TileOwner tile_owner(const PrefillOut& out, int nt) {
+    TileOwner r{&out.tmap_w[0], &out.tmap_y[0], out.row_scale[0], out.y[0], out.acc_out[0], out.O[0], out.y_vec[0], nt};
+    if (GROUPED && out.G > 1) {
+#pragma unroll
+        for (int i = 1; i < kPrefillMaxGroup; ++i)
+            if (i < out.G && nt >= out.nt_end[i - 1]) {  // constant indices only
+                r.tmap_w = &out.tmap_w[i];
+                r.tmap_y = &out.tmap_y[i];
+                r.row_scale = out.row_scale[i];
+                r.y = out.y[i];
+                r.acc_out = out.acc_out[i];
+                r.O = out.O[i];
+                r.y_vec = out.y_vec[i];
+                r.nt = nt - out.nt_end[i - 1];
+            }
+    }
+    return r;
+}
+
+template <int BN, bool GROUPED>
 __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
-    prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                   const __grid_constant__ CUtensorMap tmap_y, int y_vec, const float* __restrict__ row_scale,
-                   const float* __restrict__ s_tok, int T, int O, int K, void* __restrict__ y, int y_bf16,
-                   int32_t* __restrict__ acc_out, int ksplit, int32_t* __restrict__ part, unsigned* status) {
+    prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ PrefillOut out,
+                   const float* __restrict__ s_tok, int T, int K, int y_bf16, int ksplit,
+                   int32_t* __restrict__ part, unsigned* status) {
     using Cfg = PrefillCfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     auto* sm = reinterpret_cast<PrefillSmem<BN>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -129,11 +177,15 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
     if (threadIdx.x == 0) SBL_TRB(12);
     if (threadIdx.x == 32) {
         prefetch_tmap(&tmap_x);
-        prefetch_tmap(&tmap_w);
-        prefetch_tmap(&tmap_y);
+#pragma unroll
+        for (int i = 0; i < (GROUPED ? kPrefillMaxGroup : 1); ++i)
+            if (i < out.G) {
+                prefetch_tmap(&out.tmap_w[i]);
+                prefetch_tmap(&out.tmap_y[i]);
+            }
     }
     const int MT = (T + pf::BM - 1) / pf::BM;
-    const int NT = (O + BN - 1) / BN;
+    const int NT = GROUPED ? out.nt_end[out.G - 1] : out.nt_end[0];  // output tiles of all layers per token tile
     const int tiles = MT * NT;
     const int KB = (K + pf::BK - 1) / pf::BK;
     // work items: (tile, k-slice), the slices of a tile on consecutive items
@@ -237,7 +289,14 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
             int ep_round = 0;
             uint32_t nstore = 0;
             for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
-                const int nt = tile % NT, mt = tile / NT;  // output tiles fastest: a token tile is read once
+                const int mt = tile / NT;  // output tiles fastest: a token tile is read once
+                int g = 0, nt = tile % NT;
+                if (GROUPED) {
+                    while (g + 1 < out.G && nt >= out.nt_end[g]) ++g;
+                    if (g > 0) nt -= out.nt_end[g - 1];
+                }
+                const int O = out.O[g], y_vec = out.y_vec[g];
+                const float* const row_scale = out.row_scale[g];
                 const int b = tc & 1;
                 const uint32_t aph = (tc >> 1) & 1;
                 __syncwarp();
@@ -288,6 +347,7 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
                             q[i + 3] = __float_as_uint(f3);
                         }
                     }
+                    int32_t* const acc_out = out.acc_out[g];
                     if (acc_out && tvalid) {
                         const long long base = static_cast<long long>(t) * O + nt * BN + 32 * k;
 #pragma unroll
@@ -310,10 +370,11 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
                             }
                             fence_proxy_async_smem();
                             __syncwarp();
-                            if (lane == 0) tma_store_2d(&tmap_y, smem_u32(box), o0, mt * pf::BM + warp * 32);
+                            if (lane == 0) tma_store_2d(tile_owner<GROUPED>(out, tile % NT).tmap_y, smem_u32(box), o0, mt * pf::BM + warp * 32);
                             ++nstore;
                         } else if (tvalid) {
                             // direct stores: shapes whose row pitch is not a multiple of 16 bytes
+                            void* const y = out.y[g];
                             const long long base = static_cast<long long>(t) * O + o0;
 #pragma unroll
                             for (int i = 0; i < 32; ++i) {
@@ -393,7 +454,8 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
             bool ok = true;
             for (int wi = blockIdx.x; wi < items && ok; wi += gridDim.x) {
                 const int tile = wi / ksplit;
-                const int nt = tile % NT, mt = tile / NT;  // output tiles fastest: a token tile is read once
+                const int mt = tile / NT;  // output tiles fastest: a token tile is read once
+                const TileOwner own = tile_owner<GROUPED>(out, tile % NT);
                 int kb0, kb1;
                 kslice(wi, kb0, kb1);
                 for (int kb = kb0; kb < kb1; ++kb, ++it) {
@@ -403,7 +465,7 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
                     SBL_TR(0, it);
                     mbar_arrive_expect_tx(&sm->full_tma[s], pf::A_BYTES + Cfg::P_BYTES);
                     tma_load_2d(smem_u32(sm->a[s]), &tmap_x, kb * pf::BK, mt * pf::BM, &sm->full_tma[s]);
-                    tma_load_2d(smem_u32(sm->p[s]), &tmap_w, kb * (pf::BK / 4), nt * BN, &sm->full_tma[s]);
+                    tma_load_2d(smem_u32(sm->p[s]), own.tmap_w, kb * (pf::BK / 4), own.nt * BN, &sm->full_tma[s]);
                 }
             }
             // let every issued load land before the CTA can exit
@@ -464,14 +526,17 @@ __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
     }
 }
 
+// G layers (G <= kPrefillMaxGroup) that read the same quantised activations,
+// in one launch of the one-CTA kernel.
 template <int BN>
-static cudaError_t launch_prefill_bn(const int8_t* xperm, const float* s_tok, long long T, long long K,
-                                     const uint8_t* packed, const float* row_scale, long long O, void* y, int y_bf16,
-                                     int32_t* acc_out, int ksplit, int32_t* part, unsigned* status,
-                                     int num_sms, cudaStream_t stream) {
+static cudaError_t launch_prefill_bn(const int8_t* xperm, const float* s_tok, long long T, long long K, int G,
+                                     const uint8_t* const* packed, const float* const* row_scale, const long long* O,
+                                     void* const* y, int y_bf16, int32_t* const* acc_out, int ksplit, int32_t* part,
+                                     unsigned* status, int num_sms, cudaStream_t stream) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return cudaErrorNotSupported;
-    CUtensorMap map_x, map_w;
+    if (G < 1 || G > kPrefillMaxGroup) return cudaErrorInvalidValue;
+    CUtensorMap map_x;
     const cuuint32_t estr[2] = {1, 1};
     {
         const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(T)};
@@ -482,39 +547,54 @@ static cudaError_t launch_prefill_bn(const int8_t* xperm, const float* s_tok, lo
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
-    {
-        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 4), static_cast<cuuint64_t>(O)};
-        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 4)};
-        const cuuint32_t box[2] = {static_cast<cuuint32_t>(pf::BK / 4), static_cast<cuuint32_t>(BN)};
-        if (enc(&map_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
-    }
-    // output rows go out as 16-byte vectors when the row pitch allows it
-    const int esize = y_bf16 ? 2 : 4;
-    int y_vec = (static_cast<long long>(O) * esize) % 16 == 0 ? 1 : 0;
-    CUtensorMap map_y = map_x;
-    if (y_vec) {
-        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(O), static_cast<cuuint64_t>(T)};
-        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(O) * esize};
-        const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esize), 32u};
-        if (enc(&map_y, y_bf16 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, y, dims, strides,
-                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            y_vec = 0;
+    PrefillOut out;
+    memset(&out, 0, sizeof(out));
+    out.G = G;
+    int nt_end = 0;
+    for (int g = 0; g < G; ++g) {
+        {
+            const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 4), static_cast<cuuint64_t>(O[g])};
+            const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 4)};
+            const cuuint32_t box[2] = {static_cast<cuuint32_t>(pf::BK / 4), static_cast<cuuint32_t>(BN)};
+            if (enc(&out.tmap_w[g], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed[g]), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return cudaErrorInvalidValue;
+        }
+        // output rows go out as 16-byte vectors when the row pitch allows it
+        const int esize = y_bf16 ? 2 : 4;
+        out.y_vec[g] = (static_cast<long long>(O[g]) * esize) % 16 == 0 ? 1 : 0;
+        out.tmap_y[g] = map_x;
+        if (out.y_vec[g]) {
+            const cuuint64_t dims[2] = {static_cast<cuuint64_t>(O[g]), static_cast<cuuint64_t>(T)};
+            const cuuint64_t strides[1] = {static_cast<cuuint64_t>(O[g]) * esize};
+            const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esize), 32u};
+            if (enc(&out.tmap_y[g], y_bf16 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, y[g],
+                    dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                out.y_vec[g] = 0;
+        }
+        out.row_scale[g] = row_scale[g];
+        out.y[g] = y[g];
+        out.acc_out[g] = acc_out ? acc_out[g] : nullptr;
+        out.O[g] = static_cast<int>(O[g]);
+        nt_end += static_cast<int>((O[g] + BN - 1) / BN);
+        out.nt_end[g] = nt_end;
     }
     constexpr size_t smem = prefill_smem_bytes<BN>();
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(prefill_kernel<BN, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(prefill_kernel<BN, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(smem));
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
-    const long long items = ((T + pf::BM - 1) / pf::BM) * ((O + BN - 1) / BN) * ksplit;
+    const long long items = ((T + pf::BM - 1) / pf::BM) * nt_end * ksplit;
     const int grid = static_cast<int>(items < num_sms ? items : num_sms);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
@@ -526,8 +606,22 @@ static cudaError_t launch_prefill_bn(const int8_t* xperm, const float* s_tok, lo
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, prefill_kernel<BN>, map_x, map_w, map_y, y_vec, row_scale, s_tok, static_cast<int>(T),
-                              static_cast<int>(O), static_cast<int>(K), y, y_bf16, acc_out, ksplit, part, status);
+    if (G > 1)
+        return cudaLaunchKernelEx(&cfg, prefill_kernel<BN, true>, map_x, out, s_tok, static_cast<int>(T),
+                                  static_cast<int>(K), y_bf16, ksplit, part, status);
+    return cudaLaunchKernelEx(&cfg, prefill_kernel<BN, false>, map_x, out, s_tok, static_cast<int>(T),
+                              static_cast<int>(K), y_bf16, ksplit, part, status);
+}
+
+template <int BN>
+static cudaError_t launch_prefill_bn(const int8_t* xperm, const float* s_tok, long long T, long long K,
+                                     const uint8_t* packed, const float* row_scale, long long O, void* y, int y_bf16,
+                                     int32_t* acc_out, int ksplit, int32_t* part, unsigned* status,
+                                     int num_sms, cudaStream_t stream) {
+    void* yy[1] = {y};
+    int32_t* aa[1] = {acc_out};
+    return launch_prefill_bn<BN>(xperm, s_tok, T, K, 1, &packed, &row_scale, &O, yy, y_bf16, aa, ksplit, part,
+                                 status, num_sms, stream);
 }
 
 #ifdef SBL_TRACE
@@ -674,6 +768,31 @@ cudaError_t launch_prefill(const int8_t* xperm, const float* s_tok, long long T,
         return launch_prefill_bn<256>(xperm, s_tok, T, K, packed, row_scale, O, y, y_bf16, acc_out, 1, nullptr,
                                       status, num_sms, stream);
     return launch_prefill_bn<128>(xperm, s_tok, T, K, packed, row_scale, O, y, y_bf16, acc_out, 1, nullptr, status,
+                                  num_sms, stream);
+}
+
+// G layers (1 <= G <= prefill_max_group()) that read the same quantised
+// activations in one launch of the one-CTA kernel: their output tiles are
+// scheduled together, BN chosen by waves as for one layer (CTA pairs and the
+// split along k are not used).
+int prefill_max_group() { return kPrefillMaxGroup; }
+
+cudaError_t launch_prefill_grouped(const int8_t* xperm, const float* s_tok, long long T, long long K, int G,
+                                   const uint8_t* const* packed, const float* const* row_scale, const long long* O,
+                                   void* const* y, int y_bf16, int32_t* const* acc_out, unsigned* status,
+                                   int num_sms, cudaStream_t stream) {
+    const long long mt = (T + pf::BM - 1) / pf::BM;
+    long long t256 = 0, t128 = 0;
+    for (int g = 0; g < G; ++g) {
+        t256 += (O[g] + 255) / 256;
+        t128 += (O[g] + 127) / 128;
+    }
+    const double wide = static_cast<double>((mt * t256 + num_sms - 1) / num_sms);
+    const double narrow = 0.65 * static_cast<double>((mt * t128 + num_sms - 1) / num_sms);
+    if (wide <= narrow)
+        return launch_prefill_bn<256>(xperm, s_tok, T, K, G, packed, row_scale, O, y, y_bf16, acc_out, 1, nullptr,
+                                      status, num_sms, stream);
+    return launch_prefill_bn<128>(xperm, s_tok, T, K, G, packed, row_scale, O, y, y_bf16, acc_out, 1, nullptr, status,
                                   num_sms, stream);
 }
 

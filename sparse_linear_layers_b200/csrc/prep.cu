@@ -239,11 +239,20 @@ __device__ __forceinline__ void row_sync() {
     else __syncthreads();
 }
 
+// The matrices of one launch (equal K), their rows stacked: matrix g owns the
+// rows row_end[g - 1] .. row_end[g] - 1 of the launch.  A single matrix is G = 1.
+constexpr int kPrepMaxGroup = 8;
+struct PrepGroup {
+    const float* W[kPrepMaxGroup];
+    uint8_t* packed[kPrepMaxGroup];
+    float* row_scale[kPrepMaxGroup];
+    uint8_t* mask_bits[kPrepMaxGroup];
+    long long row_end[kPrepMaxGroup];
+    int G;
+};
+
 template <int M, int N, int WPR, bool WITH_MASK>
-__global__ void __launch_bounds__((8 / WPR) * WPR * 32) prep_kernel_rr(const float* __restrict__ W, long long O,
-                                                                      long long K, uint8_t* __restrict__ packed,
-                                                                      float* __restrict__ row_scale,
-                                                                      uint8_t* __restrict__ mask_bits,
+__global__ void __launch_bounds__((8 / WPR) * WPR * 32) prep_kernel_rr(const PrepGroup grp, long long K,
                                                                       int scale_bf16, const float* __restrict__ ext_scale,
                                                                       unsigned* status) {
     constexpr int RPB = 8 / WPR;  // rows per block
@@ -255,8 +264,24 @@ __global__ void __launch_bounds__((8 / WPR) * WPR * 32) prep_kernel_rr(const flo
     __shared__ float scales[RPB];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int sub = threadIdx.x / TPR, tr = threadIdx.x % TPR;
-    const long long row = static_cast<long long>(blockIdx.x) * RPB + sub;
-    const bool valid = row < O;
+    const long long grow = static_cast<long long>(blockIdx.x) * RPB + sub;  // row of the stacked matrices
+    const bool valid = grow < grp.row_end[grp.G - 1];
+    // the matrix of this row (constant indices only)
+    const float* W = grp.W[0];
+    uint8_t* packed = grp.packed[0];
+    float* row_scale = grp.row_scale[0];
+    uint8_t* mask_bits = grp.mask_bits[0];
+    long long row = grow;
+    if (grp.G > 1)
+#pragma unroll
+        for (int i = 1; i < kPrepMaxGroup; ++i)
+            if (i < grp.G && grow >= grp.row_end[i - 1]) {
+                W = grp.W[i];
+                packed = grp.packed[i];
+                row_scale = grp.row_scale[i];
+                mask_bits = grp.mask_bits[i];
+                row = grow - grp.row_end[i - 1];
+            }
     const int nchunks = static_cast<int>(K >> 4);
     const float* wr = W + (valid ? row : 0) * K;
 
@@ -410,7 +435,7 @@ __global__ void __launch_bounds__((8 / WPR) * WPR * 32) prep_kernel_rr(const flo
     // it is exact); the code is 01 for +1 and 10 for -1.
     const uint32_t half_bits = __float_as_uint(0.5f * sc);
     uint32_t* prow = reinterpret_cast<uint32_t*>(packed + row * (K >> 2));
-    uint16_t* mrow = WITH_MASK ? reinterpret_cast<uint16_t*>(mask_bits + row * (K >> 3)) : nullptr;
+    uint16_t* mrow = (WITH_MASK && mask_bits) ? reinterpret_cast<uint16_t*>(mask_bits + row * (K >> 3)) : nullptr;
 #pragma unroll
     for (int j = 0; j < CPT; ++j) {
         const int c = tr + TPR * j;
@@ -423,45 +448,65 @@ __global__ void __launch_bounds__((8 / WPR) * WPR * 32) prep_kernel_rr(const flo
             sgw |= (kr[j][i] >> (30 - 2 * i)) & (2u << (2 * i));
         }
         prow[c] = (nzw & ~(sgw >> 1)) | ((nzw << 1) & sgw);
-        if constexpr (WITH_MASK) mrow[c] = static_cast<uint16_t>(kbits >> (16 * j));
+        if constexpr (WITH_MASK)
+            if (mrow) mrow[c] = static_cast<uint16_t>(kbits >> (16 * j));
     }
 }
 
 template <int M, int N, int WPR>
-static void launch_prep_rr(const float* W, long long O, long long K, uint8_t* packed, float* row_scale,
-                           uint8_t* mask_bits, int scale_bf16, const float* ext_scale, unsigned* status,
-                           cudaStream_t stream) {
+static void launch_prep_rr(const PrepGroup& grp, long long K, bool with_mask, int scale_bf16, const float* ext_scale,
+                           unsigned* status, cudaStream_t stream) {
     constexpr int RPB = 8 / WPR;
-    const unsigned blocks = static_cast<unsigned>((O + RPB - 1) / RPB);
-    if (mask_bits)
-        prep_kernel_rr<M, N, WPR, true><<<blocks, RPB * WPR * 32, 0, stream>>>(W, O, K, packed, row_scale, mask_bits,
-                                                                              scale_bf16, ext_scale, status);
+    const unsigned blocks = static_cast<unsigned>((grp.row_end[grp.G - 1] + RPB - 1) / RPB);
+    if (with_mask)
+        prep_kernel_rr<M, N, WPR, true><<<blocks, RPB * WPR * 32, 0, stream>>>(grp, K, scale_bf16, ext_scale, status);
     else
-        prep_kernel_rr<M, N, WPR, false><<<blocks, RPB * WPR * 32, 0, stream>>>(W, O, K, packed, row_scale, nullptr,
-                                                                               scale_bf16, ext_scale, status);
+        prep_kernel_rr<M, N, WPR, false><<<blocks, RPB * WPR * 32, 0, stream>>>(grp, K, scale_bf16, ext_scale, status);
+}
+
+// Warps per row: the fewest that give every 16-weight chunk a slot (0: the
+// row is longer than eight warps hold, K > 8192).
+static int prep_wpr(long long K) {
+    const long long wpr = ((K >> 4) + 32 * kChunksPerThread - 1) / (32 * kChunksPerThread);
+    return wpr <= 8 ? static_cast<int>(wpr) : 0;
+}
+
+template <int M, int N>
+static void launch_prep_group(const PrepGroup& grp, long long K, bool with_mask, int scale_bf16,
+                              const float* ext_scale, unsigned* status, cudaStream_t stream) {
+    switch (prep_wpr(K)) {
+        case 1: launch_prep_rr<M, N, 1>(grp, K, with_mask, scale_bf16, ext_scale, status, stream); break;
+        case 2: launch_prep_rr<M, N, 2>(grp, K, with_mask, scale_bf16, ext_scale, status, stream); break;
+        case 3: launch_prep_rr<M, N, 3>(grp, K, with_mask, scale_bf16, ext_scale, status, stream); break;
+        case 4: launch_prep_rr<M, N, 4>(grp, K, with_mask, scale_bf16, ext_scale, status, stream); break;
+        case 5: launch_prep_rr<M, N, 5>(grp, K, with_mask, scale_bf16, ext_scale, status, stream); break;
+        case 6: launch_prep_rr<M, N, 6>(grp, K, with_mask, scale_bf16, ext_scale, status, stream); break;
+        case 7: launch_prep_rr<M, N, 7>(grp, K, with_mask, scale_bf16, ext_scale, status, stream); break;
+        case 8: launch_prep_rr<M, N, 8>(grp, K, with_mask, scale_bf16, ext_scale, status, stream); break;
+        default:  // rows longer than the register-resident kernel holds: one launch per matrix
+            for (int g = 0; g < grp.G; ++g) {
+                const long long O = grp.row_end[g] - (g ? grp.row_end[g - 1] : 0);
+                if (O == 0) continue;
+                const unsigned blocks = static_cast<unsigned>((O + kPrepWarps - 1) / kPrepWarps);
+                prep_kernel<M><<<blocks, kPrepWarps * 32, 0, stream>>>(grp.W[g], O, K, N, grp.packed[g],
+                                                                       grp.row_scale[g], grp.mask_bits[g],
+                                                                       scale_bf16, ext_scale, status);
+            }
+    }
 }
 
 template <int M, int N>
 static void launch_prep_mn(const float* W, long long O, long long K, uint8_t* packed, float* row_scale,
                            uint8_t* mask_bits, int scale_bf16, const float* ext_scale, unsigned* status,
                            cudaStream_t stream) {
-    // warps per row: the fewest that give every 16-weight chunk a slot
-    const long long wpr = ((K >> 4) + 32 * kChunksPerThread - 1) / (32 * kChunksPerThread);
-    switch (wpr) {
-        case 1: launch_prep_rr<M, N, 1>(W, O, K, packed, row_scale, mask_bits, scale_bf16, ext_scale, status, stream); break;
-        case 2: launch_prep_rr<M, N, 2>(W, O, K, packed, row_scale, mask_bits, scale_bf16, ext_scale, status, stream); break;
-        case 3: launch_prep_rr<M, N, 3>(W, O, K, packed, row_scale, mask_bits, scale_bf16, ext_scale, status, stream); break;
-        case 4: launch_prep_rr<M, N, 4>(W, O, K, packed, row_scale, mask_bits, scale_bf16, ext_scale, status, stream); break;
-        case 5: launch_prep_rr<M, N, 5>(W, O, K, packed, row_scale, mask_bits, scale_bf16, ext_scale, status, stream); break;
-        case 6: launch_prep_rr<M, N, 6>(W, O, K, packed, row_scale, mask_bits, scale_bf16, ext_scale, status, stream); break;
-        case 7: launch_prep_rr<M, N, 7>(W, O, K, packed, row_scale, mask_bits, scale_bf16, ext_scale, status, stream); break;
-        case 8: launch_prep_rr<M, N, 8>(W, O, K, packed, row_scale, mask_bits, scale_bf16, ext_scale, status, stream); break;
-        default: {
-            const unsigned blocks = static_cast<unsigned>((O + kPrepWarps - 1) / kPrepWarps);
-            prep_kernel<M><<<blocks, kPrepWarps * 32, 0, stream>>>(W, O, K, N, packed, row_scale, mask_bits,
-                                                                   scale_bf16, ext_scale, status);
-        }
-    }
+    PrepGroup grp = {};
+    grp.W[0] = W;
+    grp.packed[0] = packed;
+    grp.row_scale[0] = row_scale;
+    grp.mask_bits[0] = mask_bits;
+    grp.row_end[0] = O;
+    grp.G = 1;
+    launch_prep_group<M, N>(grp, K, mask_bits != nullptr, scale_bf16, ext_scale, status, stream);
 }
 
 // ---------------------------------------------------------------- global scale
@@ -545,6 +590,36 @@ cudaError_t launch_prep(const float* W, long long O, long long K, int n, int m, 
     else if (m == 4) launch_prep_mn<4, 3>(W, O, K, packed, row_scale, mask_bits, scale_bf16, ext, status, stream);
     else if (n == 4) launch_prep_mn<8, 4>(W, O, K, packed, row_scale, mask_bits, scale_bf16, ext, status, stream);
     else launch_prep_mn<8, 6>(W, O, K, packed, row_scale, mask_bits, scale_bf16, ext, status, stream);
+    return cudaGetLastError();
+}
+
+int prep_max_group() { return kPrepMaxGroup; }
+
+// G matrices of equal K, per-row scales (no flags), in one launch when their
+// rows fit the register-resident kernel (K <= 8192).  mask_bits may be null,
+// or hold null entries.
+cudaError_t launch_prep_grouped(int G, const float* const* W, const long long* O, long long K, int n, int m,
+                                uint8_t* const* packed, float* const* row_scale, uint8_t* const* mask_bits,
+                                unsigned* status, cudaStream_t stream) {
+    if (G < 1 || G > kPrepMaxGroup) return cudaErrorInvalidValue;
+    PrepGroup grp = {};
+    long long end = 0;
+    bool with_mask = false;
+    for (int g = 0; g < G; ++g) {
+        grp.W[g] = W[g];
+        grp.packed[g] = packed[g];
+        grp.row_scale[g] = row_scale[g];
+        grp.mask_bits[g] = mask_bits ? mask_bits[g] : nullptr;
+        with_mask |= grp.mask_bits[g] != nullptr;
+        end += O[g];
+        grp.row_end[g] = end;
+    }
+    grp.G = G;
+    if (end == 0) return cudaSuccess;
+    if (m == 4 && n == 2) launch_prep_group<4, 2>(grp, K, with_mask, 0, nullptr, status, stream);
+    else if (m == 4) launch_prep_group<4, 3>(grp, K, with_mask, 0, nullptr, status, stream);
+    else if (n == 4) launch_prep_group<8, 4>(grp, K, with_mask, 0, nullptr, status, stream);
+    else launch_prep_group<8, 6>(grp, K, with_mask, 0, nullptr, status, stream);
     return cudaGetLastError();
 }
 

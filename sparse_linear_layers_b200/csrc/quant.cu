@@ -14,8 +14,9 @@
 //                elements 1..7, even 8..14, odd 9..15: the order in which the
 //                tensor-core kernels expand weight codes (expand_pairs; read
 //                by TMA).
-// The kernel signals programmatic dependents at entry: the contraction kernel
-// that follows may start its own prologue while this one runs.
+// The kernel is itself a programmatic dependent (it waits for its predecessor
+// before reading x) and signals its own dependents at entry: the contraction
+// kernel that follows may start its prologue while this one runs.
 #include "sbl_common.cuh"
 
 namespace sbl {
@@ -43,6 +44,7 @@ __global__ void __launch_bounds__(256) quant_kernel(const uint16_t* __restrict__
                                                     int8_t* __restrict__ xq, float* __restrict__ s_tok,
                                                     uint4* __restrict__ zero_words, long long nzero, unsigned* status) {
     asm volatile("griddepcontrol.launch_dependents;");
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // the predecessor may write x or still read the slots
     zero_fill(zero_words, nzero);
     constexpr int TPC = 256 / TPT;
     __shared__ uint32_t red[8];
@@ -99,6 +101,7 @@ __global__ void __launch_bounds__(256) quant_kernel_loop(const uint16_t* __restr
                                                          int8_t* __restrict__ xq, float* __restrict__ s_tok,
                                                          uint4* __restrict__ zero_words, long long nzero, unsigned* status) {
     asm volatile("griddepcontrol.launch_dependents;");
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // the predecessor may write x or still read the slots
     zero_fill(zero_words, nzero);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long t = static_cast<long long>(blockIdx.x) * 8 + warp;
@@ -123,7 +126,8 @@ static void launch_rr(const uint16_t* x, long long T, long long K, int8_t* xq, f
                       long long nzero, unsigned* status, cudaStream_t stream) {
     constexpr int TPC = 256 / TPT;
     const unsigned blocks = static_cast<unsigned>((T + TPC - 1) / TPC);
-    quant_kernel<LAYOUT, TPT, BPT><<<blocks, 256, 0, stream>>>(x, T, K, xq, s_tok, zero_words, nzero, status);
+    pdl_launch(quant_kernel<LAYOUT, TPT, BPT>, dim3(blocks), dim3(256), 0, stream, x, T, K, xq, s_tok, zero_words, nzero,
+               status);
 }
 
 static int device_sms() {
@@ -148,7 +152,8 @@ static cudaError_t launch_layout(const uint16_t* x, long long T, long long K, in
     while (tpt < 256 && (T * tpt + 255) / 256 < min_blocks) tpt *= 2;
     if (nblk > 256 * 4) {
         const unsigned blocks = static_cast<unsigned>((T + 7) / 8);
-        quant_kernel_loop<LAYOUT><<<blocks, 256, 0, stream>>>(x, T, K, xq, s_tok, zero_words, nzero, status);
+        pdl_launch(quant_kernel_loop<LAYOUT>, dim3(blocks), dim3(256), 0, stream, x, T, K, xq, s_tok, zero_words,
+                   nzero, status);
     } else if (tpt == 16) {
         launch_rr<LAYOUT, 16, 4>(x, T, K, xq, s_tok, zero_words, nzero, status, stream);
     } else if (tpt == 32) {
@@ -307,6 +312,7 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_kernel(const uint16_t* __re
                                                             float* __restrict__ s_tok, uint4* __restrict__ zero_words,
                                                             long long nzero, unsigned* status) {
     asm volatile("griddepcontrol.launch_dependents;");
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // the predecessor may write x or still read the slots
     zero_fill(zero_words, nzero);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long t = static_cast<long long>(blockIdx.x) * 8 + warp;
@@ -507,15 +513,15 @@ static void launch_rms_rb(const uint16_t* x, const float* g, float eps, long lon
     // squares (read once from memory), longer ones read the rest again
     const long long per_lane = ((K >> 4) + 31) / 32;
     if (per_lane <= 1)
-        rmsnorm_quant_kernel<LAYOUT, 1><<<blocks, 256, 0, stream>>>(x, g, eps, T, K, xq, s_tok, zw, nzero, status);
+        pdl_launch(rmsnorm_quant_kernel<LAYOUT, 1>, dim3(blocks), dim3(256), 0, stream, x, g, eps, T, K, xq, s_tok, zw, nzero, status);
     else if (per_lane <= 2)
-        rmsnorm_quant_kernel<LAYOUT, 2><<<blocks, 256, 0, stream>>>(x, g, eps, T, K, xq, s_tok, zw, nzero, status);
+        pdl_launch(rmsnorm_quant_kernel<LAYOUT, 2>, dim3(blocks), dim3(256), 0, stream, x, g, eps, T, K, xq, s_tok, zw, nzero, status);
     else if (per_lane <= 4)
-        rmsnorm_quant_kernel<LAYOUT, 4><<<blocks, 256, 0, stream>>>(x, g, eps, T, K, xq, s_tok, zw, nzero, status);
+        pdl_launch(rmsnorm_quant_kernel<LAYOUT, 4>, dim3(blocks), dim3(256), 0, stream, x, g, eps, T, K, xq, s_tok, zw, nzero, status);
     else if (per_lane <= 10)
-        rmsnorm_quant_kernel<LAYOUT, 10><<<blocks, 256, 0, stream>>>(x, g, eps, T, K, xq, s_tok, zw, nzero, status);
+        pdl_launch(rmsnorm_quant_kernel<LAYOUT, 10>, dim3(blocks), dim3(256), 0, stream, x, g, eps, T, K, xq, s_tok, zw, nzero, status);
     else
-        rmsnorm_quant_kernel<LAYOUT, 16><<<blocks, 256, 0, stream>>>(x, g, eps, T, K, xq, s_tok, zw, nzero, status);
+        pdl_launch(rmsnorm_quant_kernel<LAYOUT, 16>, dim3(blocks), dim3(256), 0, stream, x, g, eps, T, K, xq, s_tok, zw, nzero, status);
 }
 
 // RMSNorm then per-token absmax int8 (layout as launch_quant); g fp32 [K]

@@ -13,6 +13,10 @@ namespace sbl {
 cudaError_t launch_prep(const float* W, long long O, long long K, int n, int m, uint8_t* packed, float* row_scale,
                         uint8_t* mask_bits, int scale_bf16, int scale_global, unsigned* status,
                         cudaStream_t stream);
+int prep_max_group();
+cudaError_t launch_prep_grouped(int G, const float* const* W, const long long* O, long long K, int n, int m,
+                                uint8_t* const* packed, float* const* row_scale, uint8_t* const* mask_bits,
+                                unsigned* status, cudaStream_t stream);
 cudaError_t launch_quant(const uint16_t* x, long long T, long long K, int8_t* xq, float* s_tok, int layout,
                          unsigned* status, cudaStream_t stream, void* zero16 = nullptr, long long nzero16 = 0);
 constexpr int kLayoutNatural = 0, kLayoutPairs = 1;
@@ -33,6 +37,16 @@ long long ste_backward_tiles(long long rows, long long K);
 cudaError_t launch_ste_backward(const float* dY, long long T, long long O, long long K, const uint8_t* packed,
                                 const float* row_scale, const int8_t* xq, const float* s_tok, float* dX, float* dW,
                                 int dw_ternary, cudaStream_t stream);
+int decode_max_group();
+int prefill_max_group();
+cudaError_t launch_prefill_grouped(const int8_t* xperm, const float* s_tok, long long T, long long K, int G,
+                                   const uint8_t* const* packed, const float* const* row_scale, const long long* O,
+                                   void* const* y, int y_bf16, int32_t* const* acc_out, unsigned* status,
+                                   int num_sms, cudaStream_t stream);
+cudaError_t launch_decode_grouped(int G, const uint8_t* const* packed, const float* const* row_scale,
+                                  const long long* O, long long K, const uint16_t* x, long long T, void* const* y,
+                                  int y_bf16, int32_t* const* acc_out, unsigned* status, int num_sms,
+                                  cudaStream_t stream);
 size_t backward_tc_workspace_bytes(long long T, long long O, long long K, int need_dx, int need_dw);
 cudaError_t launch_backward_tc(const float* dY, long long T, long long O, const int8_t* xq, const float* s_tok,
                                long long K, const uint8_t* packed, const float* row_scale, float* dX, float* dW,
@@ -142,6 +156,31 @@ sbl_status sbl_prepare_weights_ex(const float* W, int64_t O, int64_t K, int n, i
                                       (flags & SBL_PREP_SCALE_BF16) ? 1 : 0, (flags & SBL_PREP_SCALE_GLOBAL) ? 1 : 0,
                                       d->status,
                                       static_cast<cudaStream_t>(stream)));
+}
+
+sbl_status sbl_prepare_weights_grouped(int G, const float* const* W, const int64_t* O, int64_t K, int n, int m,
+                                       uint8_t* const* packed, float* const* row_scale, uint8_t* const* mask_bits,
+                                       void* stream) {
+    if (G < 1 || G > SBL_MAX_GROUP || G > sbl::prep_max_group() || !W || !O || !packed || !row_scale)
+        return SBL_ERR_INVALID_ARG;
+    if (sbl_status s = check_k(K)) return s;
+    if (!nm_ok(n, m)) return SBL_ERR_UNSUPPORTED;
+    long long rows = 0, Ol[SBL_MAX_GROUP];
+    for (int g = 0; g < G; ++g) {
+        if (O[g] < 0 || O[g] > (1ll << 31) - 1) return SBL_ERR_INVALID_ARG;
+        Ol[g] = O[g];
+        rows += O[g];
+        if (O[g] == 0) continue;
+        if (!W[g] || !packed[g] || !row_scale[g]) return SBL_ERR_INVALID_ARG;
+        if (!aligned(W[g], 16) || !aligned(packed[g], 16) || !aligned(row_scale[g], 16)) return SBL_ERR_INVALID_ARG;
+        if (mask_bits && mask_bits[g] && !aligned(mask_bits[g], 16)) return SBL_ERR_INVALID_ARG;
+    }
+    if (rows == 0) return SBL_OK;
+    if (rows > (1ll << 31) - 1) return SBL_ERR_UNSUPPORTED;
+    DeviceInfo* d;
+    if (sbl_status s = device_info(&d)) return s;
+    return from_cuda(sbl::launch_prep_grouped(G, W, Ol, K, n, m, packed, row_scale, mask_bits, d->status,
+                                              static_cast<cudaStream_t>(stream)));
 }
 
 sbl_status sbl_quant_act(const uint16_t* x_bf16, int64_t T, int64_t K, int8_t* x_q, float* s_tok, void* stream) {
@@ -406,6 +445,86 @@ sbl_status sbl_linear(const uint16_t* x_bf16, int64_t T, int64_t K, const uint8_
                       size_t workspace_bytes, void* stream) {
     return sbl_linear_path(x_bf16, T, K, packed, row_scale, O, n, m, y, y_dtype, acc_out, workspace,
                            workspace_bytes, SBL_PATH_AUTO, stream);
+}
+
+size_t sbl_linear_grouped_workspace_bytes(int64_t T, int64_t K) {
+    if (T <= 0 || K <= 0) return 0;
+    return base_workspace_bytes(T, K);
+}
+
+sbl_status sbl_linear_grouped(const uint16_t* x_bf16, int64_t T, int64_t K, int G, const uint8_t* const* packed,
+                              const float* const* row_scale, const int64_t* O, int n, int m, void* const* y,
+                              int y_dtype, int32_t* const* acc_out, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+    if (G < 1 || G > SBL_MAX_GROUP || G > sbl::decode_max_group() || !packed || !row_scale || !O || !y)
+        return SBL_ERR_INVALID_ARG;
+    if (T < 0) return SBL_ERR_INVALID_ARG;
+    if (sbl_status s = check_k(K)) return s;
+    if (!nm_ok(n, m)) return SBL_ERR_UNSUPPORTED;
+    if (y_dtype != SBL_F32 && y_dtype != SBL_BF16) return SBL_ERR_INVALID_ARG;
+    long long rows = 0;
+    for (int g = 0; g < G; ++g) {
+        if (O[g] < 0 || O[g] > (1ll << 31) - 1) return SBL_ERR_INVALID_ARG;
+        rows += O[g];
+        if (T > 0 && O[g] > 0) {
+            if (!packed[g] || !row_scale[g] || !y[g]) return SBL_ERR_INVALID_ARG;
+            if (!aligned(packed[g], 16) || !aligned(row_scale[g], 16) || !aligned(y[g], 16)) return SBL_ERR_INVALID_ARG;
+            if (acc_out && acc_out[g] && !aligned(acc_out[g], 16)) return SBL_ERR_INVALID_ARG;
+        }
+    }
+    if (T == 0 || rows == 0) return SBL_OK;
+    if (!x_bf16 || !aligned(x_bf16, 16)) return SBL_ERR_INVALID_ARG;
+    if (T > (1ll << 31) - 1) return SBL_ERR_UNSUPPORTED;
+    const bool prefill = ((T > kDecodeMaxTokens) || (K > kDecodeMaxK)) && (K % 64 == 0);
+    if (!prefill && K > kDecodeMaxK) return SBL_ERR_UNSUPPORTED;
+    const size_t need = base_workspace_bytes(T, K);
+    if (prefill && (!workspace || workspace_bytes < need || !aligned(workspace, 256))) return SBL_ERR_WORKSPACE;
+    DeviceInfo* d;
+    if (sbl_status s = device_info(&d)) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int ybf = y_dtype == SBL_BF16 ? 1 : 0;
+    cudaError_t e = cudaSuccess;
+    if (!prefill && !(T >= kDecodeMmaMinTokens && sbl::decode_mma_supported(K))) {
+        // one launch streams every matrix's weights; the kernel quantises x once per block
+        long long Ol[SBL_MAX_GROUP];
+        for (int g = 0; g < G; ++g) Ol[g] = O[g];
+        e = sbl::launch_decode_grouped(G, packed, row_scale, Ol, K, x_bf16, T, y, ybf, acc_out, d->status,
+                                       d->num_sms, st);
+    } else if (!prefill) {
+        // warp-level MMA decode, one launch per matrix
+        for (int g = 0; g < G && e == cudaSuccess; ++g)
+            if (O[g] > 0)
+                e = sbl::launch_decode_mma(packed[g], row_scale[g], O[g], K, x_bf16, T, y[g], ybf,
+                                           acc_out ? acc_out[g] : nullptr, d->status, d->num_sms, st);
+    } else {
+        // x quantised once (pairing order), then the dense tensor-core GEMM per matrix
+        int8_t* xq = static_cast<int8_t*>(workspace);
+        float* s_tok = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round256(static_cast<size_t>(T) * K));
+        e = sbl::launch_quant(x_bf16, T, K, xq, s_tok, sbl::kLayoutPairs, d->status, st);
+        // the non-empty layers, up to prefill_max_group() per launch of the one-CTA kernel
+        const uint8_t* gp[SBL_MAX_GROUP];
+        const float* gs[SBL_MAX_GROUP];
+        long long go[SBL_MAX_GROUP];
+        void* gy[SBL_MAX_GROUP];
+        int32_t* ga[SBL_MAX_GROUP];
+        int n_l = 0;
+        for (int g = 0; g < G; ++g)
+            if (O[g] > 0) {
+                gp[n_l] = packed[g];
+                gs[n_l] = row_scale[g];
+                go[n_l] = O[g];
+                gy[n_l] = y[g];
+                ga[n_l] = acc_out ? acc_out[g] : nullptr;
+                ++n_l;
+            }
+        const int per = sbl::prefill_max_group();
+        for (int g0 = 0; g0 < n_l && e == cudaSuccess; g0 += per) {
+            const int cnt = n_l - g0 < per ? n_l - g0 : per;
+            e = sbl::launch_prefill_grouped(xq, s_tok, T, K, cnt, gp + g0, gs + g0, go + g0, gy + g0, ybf, ga + g0,
+                                            d->status, d->num_sms, st);
+        }
+    }
+    return from_cuda(e);
 }
 
 int64_t sbl_decode_max_tokens(void) { return kDecodeMaxTokens; }

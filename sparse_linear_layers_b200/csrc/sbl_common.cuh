@@ -7,6 +7,25 @@
 
 namespace sbl {
 
+// Launch as a programmatic dependent of the previous kernel on the stream:
+// the kernel may start (and run its prologue) while its predecessor drains,
+// and must execute griddepcontrol.wait before reading anything the
+// predecessor writes.
+template <typename Kern, typename... Args>
+inline cudaError_t pdl_launch(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Bits of the per-device status word (see sbl_device_status in sbl.h).
 constexpr unsigned kStatusNonfinite = 1u;
 constexpr unsigned kStatusTimeout = 2u;

@@ -173,3 +173,63 @@ def test_training_layer_has_no_cpu_fallback():
     assert tuple(layer.weight.shape) == (128, 64) and layer.weight.dtype == torch.float32
     with pytest.raises(ValueError, match="CUDA"):
         layer(torch.zeros(3, 64))
+
+
+def test_grouped_rejects_on_host():
+    import ctypes as C
+    from sparse_linear_layers_b200 import _lib
+    lib = _lib.lib
+    src = open(HEADER).read()
+    assert int(re.search(r"#define SBL_MAX_GROUP (\d+)", src).group(1)) == _lib.SBL_MAX_GROUP
+    G = 3
+    p = 4096  # never dereferenced: host checks come first
+    ptrs = (C.c_void_p * G)(p, p, p)
+    rows = (C.c_int64 * G)(896, 128, 128)
+    args = lambda T, K, g, n=3, m=4, rows=rows, ws=None, wsb=0: lib.sbl_linear_grouped(
+        p, T, K, g, ptrs, ptrs, rows, n, m, ptrs, 0, None, ws, wsb, None)
+    assert args(2048, 896, 0) == 1                       # no layers
+    assert args(2048, 896, _lib.SBL_MAX_GROUP + 1) == 1  # too many
+    assert args(2048, 40, G) == 1                        # K % 16
+    assert args(2048, 896, G, n=1) == 2                  # pattern
+    assert args(0, 896, G) == 0                          # no tokens: nothing to do
+    assert args(2048, 896, G) == 6                       # prefill sizes need the workspace
+    assert args(2048, 896, G, ws=p, wsb=16) == 6
+    assert args(2048, 896, G, rows=(C.c_int64 * G)(0, 0, 0)) == 0
+    assert args(2048, 896, G, rows=(C.c_int64 * G)(-1, 0, 0)) == 1
+    assert lib.sbl_linear_grouped_workspace_bytes(2048, 896) == lib.sbl_linear_workspace_bytes(2048, 896, 896, 3, 4)
+
+
+def test_backward_ws_rejects_on_host():
+    from sparse_linear_layers_b200._lib import lib
+    p = 4096
+    B = lib.sbl_linear_backward_ws
+    assert B(p, 8, 16, p, p, 64, p, p, p, p, 4, p, 1 << 20, None) == 1      # unknown flag
+    assert B(p, 8, 16, p, p, 40, p, p, p, p, 0, p, 1 << 20, None) == 1      # K % 16
+    assert B(p, 8, 16, p, p, 64, p, p, None, None, 0, p, 1 << 20, None) == 1  # no output asked for
+    assert B(p, 8, 16, p, p, 64, p, p, p, p, 0, None, 0, None) == 6          # no workspace
+    assert B(p, 8, 16, p, p, 64, p, p, p, p, 0, p + 16, 1 << 20, None) == 6  # unaligned workspace
+    need = lib.sbl_linear_backward_workspace_bytes(8, 16, 64, 1, 1)
+    assert need > 0 and B(p, 8, 16, p, p, 64, p, p, p, p, 0, p, need - 1, None) == 6
+    assert B(p, 1 << 22, 16, p, p, 64, p, p, p, p, 0, p, 1 << 40, None) == 2  # T beyond the tensor-core path
+    # workspace: A' [M, 3 * 64] and B [64, 64] bf16 per gradient, the larger of the two
+    assert lib.sbl_linear_backward_workspace_bytes(8, 16, 64, 1, 0) == 3 * 8 * 64 * 2 + 64 * 64 * 2
+    assert lib.sbl_linear_backward_workspace_bytes(0, 16, 64, 1, 1) == 0
+
+
+def test_prepare_grouped_rejects_on_host():
+    import ctypes as C
+    from sparse_linear_layers_b200 import _lib
+    lib = _lib.lib
+    p = 4096
+    G = 2
+    ptrs = (C.c_void_p * G)(p, p)
+    P = lambda g, rows, K=64, n=2, m=4: lib.sbl_prepare_weights_grouped(g, ptrs, rows, K, n, m, ptrs, ptrs, None, None)
+    ok_rows = (C.c_int64 * G)(8, 8)
+    assert P(0, ok_rows) == 1                                  # no matrices
+    assert P(_lib.SBL_MAX_GROUP + 1, ok_rows) == 1
+    assert P(G, ok_rows, K=40) == 1                            # K % 16
+    assert P(G, ok_rows, n=5, m=8) == 2                        # pattern
+    assert P(G, (C.c_int64 * G)(-1, 8)) == 1                   # negative rows
+    assert P(G, (C.c_int64 * G)(0, 0)) == 0                    # nothing to do
+    bad = (C.c_void_p * G)(p + 4, p)                           # unaligned latent weights
+    assert lib.sbl_prepare_weights_grouped(G, bad, ok_rows, 64, 2, 4, ptrs, ptrs, None, None) == 1

@@ -978,3 +978,26 @@ def test_ste_backward_matches_autograd_on_random_shapes(nm, O, K, T, seed, tern)
     gx = xl.grad.numpy() if xl.grad is not None else np.zeros((T, K))
     np.testing.assert_allclose(dX, gx, rtol=1e-12, atol=1e-12 * (np.abs(gx).max(initial=0.0) + 1e-300))
     np.testing.assert_allclose(dW, Wl.grad.numpy(), rtol=1e-12, atol=1e-12 * (np.abs(dW).max(initial=0.0) + 1e-300))
+
+
+def test_ternarise_threshold_equals_float32_division_reading():
+    """round(W / scale) read as an IEEE float32 division then round-half-even
+    (the other plausible reading of the guide's W~ equation) and the oracle's
+    exact reading (nonzero iff |w| > scale / 2) give the same codes for every
+    float w and normal scale: scale / 2 is a float, the next float above it,
+    h + ulp(h), gives w / scale - 1/2 >= 2^-24 / m > 2^-25 (h = m * 2^e), half
+    the float spacing just above 1/2, so the float32 quotient is already above
+    1/2.  Checked on the floats around the threshold of 400k scales."""
+    rng = np.random.default_rng(21)
+    n = 400_000
+    s = (rng.uniform(1, 2, n) * 2.0 ** rng.integers(-16, 16, n)).astype(np.float32)
+    s = np.maximum(s, oracle.EPS_SCALE)
+    h = (s / np.float32(2)).astype(np.float32)
+    for k in range(-3, 4):
+        w = h.copy()
+        for _ in range(abs(k)):
+            w = np.nextafter(w, np.float32(np.inf if k > 0 else -np.inf))
+        w = w * np.where(rng.random(n) < 0.5, np.float32(-1), np.float32(1))
+        fp32_reading = np.clip(np.rint((w / s).astype(np.float32)), -1, 1).astype(np.int8)
+        exact = oracle.ternarise(w[:, None], s, np.ones((n, 1), bool))[:, 0]
+        assert np.array_equal(fp32_reading, exact), k
