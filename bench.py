@@ -42,12 +42,14 @@ TOKENS_PER_STEP = T_PREFILL + T_DECODE
 WORKLOAD = "qwen2.5-0.5b layer projections (q,k,v,o,gate,up,down), 3:4, prep + T=2048 prefill + T=1 decode"
 
 
-# DRAM bytes (read + write) per prefill sbl_linear call (activation quantisation
-# + tcgen05 GEMM), mean over the seven projections at T = 2048, from one ncu
-# capture of this step's eager pass (dram__bytes_read.sum + dram__bytes_write.sum).
+# DRAM bytes (read + write) per prefill call of one input group (activation
+# quantisation + tcgen05 GEMM), mean over the four groups at T = 2048, from one
+# ncu capture of the step's eager pass (`bench.py --only step_once`,
+# dram__bytes_read.sum + dram__bytes_write.sum; outputs still in L2 when a
+# launch ends are not counted).
 # Only valid for the kernel sources the counters were taken on; reported as null
 # once those change.
-PREFILL_TRAFFIC = {"sources_sha256": "fbb2959aca9e10dd06c4869e47e9c3a26f82fa43fcb209e616835998371a021e", "bytes_per_call": 9617920}
+PREFILL_TRAFFIC = {"sources_sha256": "787ba7c0ef4d67d49476a29d55caa97c662e7b6c374ec867172b7f4d59d81a4c", "bytes_per_call": 17011840}
 
 
 def _kernel_sources_digest():
@@ -467,6 +469,21 @@ def _prefill_roofline(sbl, dev, int8_peak_tops, hbm_peak):
         for shape in ("gate", "down")}
     torch.cuda.nvtx.range_pop()
     return out
+
+
+def _step_once(sbl, dev):
+    """One eager pass of the step's three phases, no graphs and nothing else:
+    a small process for profilers (launch order: prep, then per input group
+    one quantisation and one GEMM, then one decode launch per group)."""
+    layers, groups = make_step(dev)
+    streams = [torch.cuda.current_stream(), torch.cuda.Stream()]
+    for _, fn in PHASES:
+        fn(sbl, layers, groups, streams)
+    torch.cuda.synchronize()
+    status = sbl.sbl_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status}")
+    return {"phases": [name for name, _ in PHASES], "groups": [g.name for g in groups], "status": status}
 
 
 def _int8_peak(dev, n=8192, reps=20):
@@ -951,7 +968,7 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration sweep (profiling runs)")
-    ap.add_argument("--only", choices=("rmsnorm_front", "mask_monitor", "ste_backward", "int8_peak"),
+    ap.add_argument("--only", choices=("rmsnorm_front", "mask_monitor", "ste_backward", "int8_peak", "step_once"),
                     help="run only this auxiliary measurement on one GPU and print its JSON (profiling runs)")
     ap.add_argument("--tokens", type=int, default=32768, help="tokens of the --only rmsnorm_front measurement")
     args = ap.parse_args()
@@ -978,6 +995,8 @@ def main():
             res = _mask_monitor_bench(sbl, dev, hbm_peak)
         elif args.only == "int8_peak":
             res = _int8_peak(dev)
+        elif args.only == "step_once":
+            res = _step_once(sbl, dev)
         else:
             res = _ste_backward_bench(sbl, dev)
         print(json.dumps({"only": args.only, "result": res}), flush=True)
