@@ -390,9 +390,10 @@ sbl_status sbl_linear_noalloc(const uint16_t* x_bf16, int64_t T, int64_t K,
  *               sizes use none (NULL allowed).
  * One or two tokens: one launch streams all G weight matrices (one pass of
  * their stacked rows).  Three to 16 tokens: the warp-level MMA decode per
- * layer.  Prefill: x is quantised once, then one launch of the one-CTA
- * tensor-core GEMM schedules the output tiles of up to four layers together
- * (the CTA-pair and 2:4 sparse kernels and the split along k are not used).
+ * layer.  Prefill: x is quantised once, then one launch of the tensor-core
+ * GEMM schedules the output tiles of up to four layers together (CTA pairs or
+ * one CTA, as for one layer of their combined size; the 2:4 sparse kernel and
+ * the split along k are not used).
  * 1 <= G <= SBL_MAX_GROUP, else SBL_ERR_INVALID_ARG.
  */
 size_t sbl_linear_grouped_workspace_bytes(int64_t T, int64_t K);

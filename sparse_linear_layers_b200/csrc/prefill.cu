@@ -110,54 +110,6 @@ constexpr size_t prefill_smem_bytes() {
 static_assert(prefill_smem_bytes<256>() <= 232448, "prefill tile does not fit in shared memory");
 static_assert(prefill_smem_bytes<128>() <= 232448, "prefill tile does not fit in shared memory");
 
-// The weight matrices of one launch: G layers that read the same quantised
-// activations, each with its codes (tensor map), output (tensor map and
-// pointer), row scales and accumulators.  Their output tiles are numbered one
-// after the other: layer g owns the tiles nt_end[g - 1] .. nt_end[g] - 1 of
-// every token tile.  A single layer is G = 1.
-constexpr int kPrefillMaxGroup = 4;
-struct PrefillOut {
-    CUtensorMap tmap_w[kPrefillMaxGroup];
-    CUtensorMap tmap_y[kPrefillMaxGroup];
-    const float* row_scale[kPrefillMaxGroup];
-    void* y[kPrefillMaxGroup];
-    int32_t* acc_out[kPrefillMaxGroup];
-    int O[kPrefillMaxGroup];
-    int y_vec[kPrefillMaxGroup];
-    int nt_end[kPrefillMaxGroup];
-    int G;
-};
-
-// Layer of output tile nt (counted over all layers) and its tile within the layer.
-struct TileOwner {
-    const CUtensorMap* tmap_w;
-    const CUtensorMap* tmap_y;
-    const float* row_scale;
-    void* y;
-    int32_t* acc_out;
-    int O, y_vec, nt;
-};
-
-template <bool GROUPED>
-__device__ __forceinline__ TileOwner tile_owner(const PrefillOut& out, int nt) {
-    TileOwner r{&out.tmap_w[0], &out.tmap_y[0], out.row_scale[0], out.y[0], out.acc_out[0], out.O[0], out.y_vec[0], nt};
-    if (GROUPED && out.G > 1) {
-#pragma unroll
-        for (int i = 1; i < kPrefillMaxGroup; ++i)
-            if (i < out.G && nt >= out.nt_end[i - 1]) {  // constant indices only
-                r.tmap_w = &out.tmap_w[i];
-                r.tmap_y = &out.tmap_y[i];
-                r.row_scale = out.row_scale[i];
-                r.y = out.y[i];
-                r.acc_out = out.acc_out[i];
-                r.O = out.O[i];
-                r.y_vec = out.y_vec[i];
-                r.nt = nt - out.nt_end[i - 1];
-            }
-    }
-    return r;
-}
-
 template <int BN, bool GROUPED>
 __global__ void __launch_bounds__(PrefillCfg<BN>::THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ PrefillOut out,
@@ -632,6 +584,10 @@ cudaError_t set_prefill_trace(void* buf) {
 #endif
 
 int prefill_pair_clusters(cudaStream_t stream);
+cudaError_t launch_prefill_pair_group(const int8_t* xperm, const float* s_tok, long long T, long long K, int G,
+                                      const uint8_t* const* packed, const float* const* row_scale,
+                                      const long long* O, void* const* y, int y_bf16, int32_t* const* acc_out,
+                                      unsigned* status, cudaStream_t stream);
 cudaError_t launch_prefill_pair(const int8_t* xperm, const float* s_tok, long long T, long long K,
                                 const uint8_t* packed, const float* row_scale, long long O, void* y, int y_bf16,
                                 int32_t* acc_out, unsigned* status, cudaStream_t stream);
@@ -772,15 +728,17 @@ cudaError_t launch_prefill(const int8_t* xperm, const float* s_tok, long long T,
 }
 
 // G layers (1 <= G <= prefill_max_group()) that read the same quantised
-// activations in one launch of the one-CTA kernel: their output tiles are
-// scheduled together, BN chosen by waves as for one layer (CTA pairs and the
-// split along k are not used).
+// activations in one launch: their output tiles are scheduled together on
+// the kernel the cost model of choose_dense_prefill picks for the sum of
+// their tiles (CTA pairs, or one CTA with 256- or 128-output tiles; the split
+// along k is not used).
 int prefill_max_group() { return kPrefillMaxGroup; }
 
 cudaError_t launch_prefill_grouped(const int8_t* xperm, const float* s_tok, long long T, long long K, int G,
                                    const uint8_t* const* packed, const float* const* row_scale, const long long* O,
                                    void* const* y, int y_bf16, int32_t* const* acc_out, unsigned* status,
                                    int num_sms, cudaStream_t stream) {
+    constexpr double kNarrowCost = 0.65, kPairCost = 0.65;
     const long long mt = (T + pf::BM - 1) / pf::BM;
     long long t256 = 0, t128 = 0;
     for (int g = 0; g < G; ++g) {
@@ -788,7 +746,14 @@ cudaError_t launch_prefill_grouped(const int8_t* xperm, const float* s_tok, long
         t128 += (O[g] + 127) / 128;
     }
     const double wide = static_cast<double>((mt * t256 + num_sms - 1) / num_sms);
-    const double narrow = 0.65 * static_cast<double>((mt * t128 + num_sms - 1) / num_sms);
+    const double narrow = kNarrowCost * static_cast<double>((mt * t128 + num_sms - 1) / num_sms);
+    const int clusters = prefill_pair_clusters(stream);
+    if (clusters > 0) {
+        const long long pt = ((T + 255) / 256) * t256;
+        if (kPairCost * static_cast<double>((pt + clusters - 1) / clusters) < (wide < narrow ? wide : narrow))
+            return launch_prefill_pair_group(xperm, s_tok, T, K, G, packed, row_scale, O, y, y_bf16, acc_out, status,
+                                             stream);
+    }
     if (wide <= narrow)
         return launch_prefill_bn<256>(xperm, s_tok, T, K, G, packed, row_scale, O, y, y_bf16, acc_out, 1, nullptr,
                                       status, num_sms, stream);

@@ -36,6 +36,7 @@
 // wait is bounded; a CTA that gives up records a timeout and winds down.
 #include <cuda.h>
 
+#include <cstring>
 #include <type_traits>
 
 #include "sbl_common.cuh"
@@ -81,11 +82,10 @@ struct PairSmem {
 constexpr size_t pair_smem_bytes() { return sizeof(PairSmem) + 1024; }
 static_assert(pair_smem_bytes() <= 232448, "pair prefill tile does not fit in shared memory");
 
+template <bool GROUPED>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
-    prefill_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                        const __grid_constant__ CUtensorMap tmap_y, int y_vec, const float* __restrict__ row_scale,
-                        const float* __restrict__ s_tok, int T, int O, int K, void* __restrict__ y, int y_bf16,
-                        int32_t* __restrict__ acc_out, unsigned* status) {
+    prefill_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ PrefillOut out,
+                        const float* __restrict__ s_tok, int T, int K, int y_bf16, unsigned* status) {
     extern __shared__ uint8_t smem_raw[];
     auto* sm = reinterpret_cast<PairSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     volatile int* abort_flag = &sm->abort_flag;
@@ -95,14 +95,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
     const bool leader = rank == 0;
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
     const int MT = (T + 2 * pp::BM - 1) / (2 * pp::BM);
-    const int NT = (O + pp::BN - 1) / pp::BN;
+    const int NT = GROUPED ? out.nt_end[out.G - 1] : out.nt_end[0];  // output tiles of all layers
     const int tiles = MT * NT;
     const int KB = (K + pp::BK - 1) / pp::BK;
 
     if (threadIdx.x == 32) {
         prefetch_tmap(&tmap_x);
-        prefetch_tmap(&tmap_w);
-        prefetch_tmap(&tmap_y);
+#pragma unroll
+        for (int i = 0; i < (GROUPED ? kPrefillMaxGroup : 1); ++i)
+            if (i < out.G) {
+                prefetch_tmap(&out.tmap_w[i]);
+                prefetch_tmap(&out.tmap_y[i]);
+            }
     }
     if (threadIdx.x == 0) {
         for (int s = 0; s < pp::STAGES; ++s) {
@@ -161,7 +165,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
             int tc = 0;
             uint32_t nstore = 0;
             for (int tile = pair; tile < tiles; tile += npairs, ++tc) {
-                const int nt = tile % NT, mt = tile / NT;  // output tiles fastest: a token tile is read once
+                const int mt = tile / NT;  // output tiles fastest: a token tile is read once
+                int g = 0, nt = tile % NT;
+                if (GROUPED) {
+                    while (g + 1 < out.G && nt >= out.nt_end[g]) ++g;
+                    if (g > 0) nt -= out.nt_end[g - 1];
+                }
+                const int O = out.O[g], y_vec = out.y_vec[g];
+                const float* const row_scale = out.row_scale[g];
                 const int b = tc & 1;
                 const uint32_t aph = (tc >> 1) & 1;
                 __syncwarp();
@@ -211,6 +222,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
                             q[i + 3] = __float_as_uint(f3);
                         }
                     }
+                    int32_t* const acc_out = out.acc_out[g];
                     if (acc_out && tvalid) {
                         const long long base = static_cast<long long>(t) * O + nt * pp::BN + 32 * k;
 #pragma unroll
@@ -232,10 +244,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
                             }
                             fence_proxy_async_smem();
                             __syncwarp();
-                            if (lane == 0) tma_store_2d(&tmap_y, smem_u32(box), o0, trow0 + warp * 32);
+                            if (lane == 0)
+                                tma_store_2d(tile_owner<GROUPED>(out, tile % NT).tmap_y, smem_u32(box), o0, trow0 + warp * 32);
                             ++nstore;
                         } else if (tvalid) {
                             // direct stores: shapes whose row pitch is not a multiple of 16 bytes
+                            void* const y = out.y[g];
                             const long long base = static_cast<long long>(t) * O + o0;
 #pragma unroll
                             for (int i = 0; i < 32; ++i) {
@@ -311,9 +325,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
             uint32_t it = 0;
             bool ok = true;
             for (int tile = pair; tile < tiles && ok; tile += npairs) {
-                const int nt = tile % NT, mt = tile / NT;  // output tiles fastest: a token tile is read once
+                const int mt = tile / NT;  // output tiles fastest: a token tile is read once
+                const TileOwner own = tile_owner<GROUPED>(out, tile % NT);
                 const int trow = mt * 2 * pp::BM + static_cast<int>(rank) * pp::BM;
-                const int orow = nt * pp::BN + static_cast<int>(rank) * pp::BNH;
+                const int orow = own.nt * pp::BN + static_cast<int>(rank) * pp::BNH;
                 for (int kb = 0; kb < KB; ++kb, ++it) {
                     const int s = it % pp::STAGES;
                     const uint32_t ph = (it / pp::STAGES) & 1;
@@ -323,7 +338,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
                     mbar_arrive_expect_tx(&sm->full_c[s], pp::P_BYTES);
                     tma_load_2d_pair(smem_u32(sm->a[s]), &tmap_x, kb * pp::BK, trow,
                                      map_to_cta(smem_u32(&sm->full_a[s]), 0));
-                    tma_load_2d(smem_u32(sm->p[s]), &tmap_w, kb * (pp::BK / 4), orow, &sm->full_c[s]);
+                    tma_load_2d(smem_u32(sm->p[s]), own.tmap_w, kb * (pp::BK / 4), orow, &sm->full_c[s]);
                 }
             }
             // let the issued loads land before the CTA can exit: its own code
@@ -392,8 +407,11 @@ static cudaError_t pair_set_smem_attr() {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64 && attr_set[dev]) return cudaSuccess;
-    e = cudaFuncSetAttribute(prefill_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(prefill_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(pair_smem_bytes()));
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(prefill_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(pair_smem_bytes()));
     if (e == cudaSuccess && dev >= 0 && dev < 64) attr_set[dev] = true;
     return e;
 }
@@ -412,22 +430,26 @@ int prefill_pair_clusters(cudaStream_t stream) {
         cfg.dynamicSmemBytes = pair_smem_bytes();
         cfg.stream = stream;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, prefill_pair_kernel, &cfg) != cudaSuccess || n <= 0) return 0;
+        if (cudaOccupancyMaxActiveClusters(&n, prefill_pair_kernel<true>, &cfg) != cudaSuccess || n <= 0) return 0;
         cached[dev] = n;
     }
     return cached[dev];
 }
 
-cudaError_t launch_prefill_pair(const int8_t* xperm, const float* s_tok, long long T, long long K,
-                                const uint8_t* packed, const float* row_scale, long long O, void* y, int y_bf16,
-                                int32_t* acc_out, unsigned* status, cudaStream_t stream) {
+// G layers (1 <= G <= kPrefillMaxGroup) that read the same quantised
+// activations, in one launch of the CTA-pair kernel.
+cudaError_t launch_prefill_pair_group(const int8_t* xperm, const float* s_tok, long long T, long long K, int G,
+                                      const uint8_t* const* packed, const float* const* row_scale,
+                                      const long long* O, void* const* y, int y_bf16, int32_t* const* acc_out,
+                                      unsigned* status, cudaStream_t stream) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return cudaErrorNotSupported;
+    if (G < 1 || G > kPrefillMaxGroup) return cudaErrorInvalidValue;
     if (cudaError_t e = pair_set_smem_attr()) return e;
     const int max_clusters = prefill_pair_clusters(stream);
     if (max_clusters <= 0) return cudaErrorNotSupported;
 
-    CUtensorMap map_x, map_w;
+    CUtensorMap map_x;
     const cuuint32_t estr[2] = {1, 1};
     {
         const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(T)};
@@ -438,28 +460,40 @@ cudaError_t launch_prefill_pair(const int8_t* xperm, const float* s_tok, long lo
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
-    {
-        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 4), static_cast<cuuint64_t>(O)};
-        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 4)};
-        const cuuint32_t box[2] = {static_cast<cuuint32_t>(pp::BK / 4), static_cast<cuuint32_t>(pp::BNH)};
-        if (enc(&map_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
+    PrefillOut out;
+    memset(&out, 0, sizeof(out));
+    out.G = G;
+    int nt_end = 0;
+    for (int g = 0; g < G; ++g) {
+        {
+            const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 4), static_cast<cuuint64_t>(O[g])};
+            const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 4)};
+            const cuuint32_t box[2] = {static_cast<cuuint32_t>(pp::BK / 4), static_cast<cuuint32_t>(pp::BNH)};
+            if (enc(&out.tmap_w[g], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed[g]), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return cudaErrorInvalidValue;
+        }
+        const int esize = y_bf16 ? 2 : 4;
+        out.y_vec[g] = (static_cast<long long>(O[g]) * esize) % 16 == 0 ? 1 : 0;
+        out.tmap_y[g] = map_x;
+        if (out.y_vec[g]) {
+            const cuuint64_t dims[2] = {static_cast<cuuint64_t>(O[g]), static_cast<cuuint64_t>(T)};
+            const cuuint64_t strides[1] = {static_cast<cuuint64_t>(O[g]) * esize};
+            const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esize), 32u};
+            if (enc(&out.tmap_y[g], y_bf16 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, y[g],
+                    dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                out.y_vec[g] = 0;
+        }
+        out.row_scale[g] = row_scale[g];
+        out.y[g] = y[g];
+        out.acc_out[g] = acc_out ? acc_out[g] : nullptr;
+        out.O[g] = static_cast<int>(O[g]);
+        nt_end += static_cast<int>((O[g] + pp::BN - 1) / pp::BN);
+        out.nt_end[g] = nt_end;
     }
-    const int esize = y_bf16 ? 2 : 4;
-    int y_vec = (static_cast<long long>(O) * esize) % 16 == 0 ? 1 : 0;
-    CUtensorMap map_y = map_x;
-    if (y_vec) {
-        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(O), static_cast<cuuint64_t>(T)};
-        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(O) * esize};
-        const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esize), 32u};
-        if (enc(&map_y, y_bf16 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, y, dims, strides,
-                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            y_vec = 0;
-    }
-    const long long tiles = ((T + 2 * pp::BM - 1) / (2 * pp::BM)) * ((O + pp::BN - 1) / pp::BN);
+    const long long tiles = ((T + 2 * pp::BM - 1) / (2 * pp::BM)) * nt_end;
     const int clusters = static_cast<int>(tiles < max_clusters ? tiles : max_clusters);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * clusters);
@@ -471,9 +505,19 @@ cudaError_t launch_prefill_pair(const int8_t* xperm, const float* s_tok, long lo
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, prefill_pair_kernel, map_x, map_w, map_y, y_vec, row_scale, s_tok,
-                              static_cast<int>(T), static_cast<int>(O), static_cast<int>(K), y, y_bf16, acc_out,
-                              status);
+    if (G > 1)
+        return cudaLaunchKernelEx(&cfg, prefill_pair_kernel<true>, map_x, out, s_tok, static_cast<int>(T),
+                                  static_cast<int>(K), y_bf16, status);
+    return cudaLaunchKernelEx(&cfg, prefill_pair_kernel<false>, map_x, out, s_tok, static_cast<int>(T),
+                              static_cast<int>(K), y_bf16, status);
+}
+
+cudaError_t launch_prefill_pair(const int8_t* xperm, const float* s_tok, long long T, long long K,
+                                const uint8_t* packed, const float* row_scale, long long O, void* y, int y_bf16,
+                                int32_t* acc_out, unsigned* status, cudaStream_t stream) {
+    void* yy[1] = {y};
+    int32_t* aa[1] = {acc_out};
+    return launch_prefill_pair_group(xperm, s_tok, T, K, 1, &packed, &row_scale, &O, yy, y_bf16, aa, status, stream);
 }
 
 }  // namespace sbl

@@ -181,4 +181,53 @@ inline EncodeTiledFn get_encode_fn() {
     return fn;
 }
 
+// ---------------------------------------------------------------- grouped prefill
+// The weight matrices of one launch: G layers that read the same quantised
+// activations, each with its codes (tensor map), output (tensor map and
+// pointer), row scales and accumulators.  Their output tiles are numbered one
+// after the other: layer g owns the tiles nt_end[g - 1] .. nt_end[g] - 1 of
+// every token tile.  A single layer is G = 1.
+constexpr int kPrefillMaxGroup = 4;
+struct PrefillOut {
+    CUtensorMap tmap_w[kPrefillMaxGroup];
+    CUtensorMap tmap_y[kPrefillMaxGroup];
+    const float* row_scale[kPrefillMaxGroup];
+    void* y[kPrefillMaxGroup];
+    int32_t* acc_out[kPrefillMaxGroup];
+    int O[kPrefillMaxGroup];
+    int y_vec[kPrefillMaxGroup];
+    int nt_end[kPrefillMaxGroup];
+    int G;
+};
+
+// Layer of output tile nt (counted over all layers) and its tile within the layer.
+struct TileOwner {
+    const CUtensorMap* tmap_w;
+    const CUtensorMap* tmap_y;
+    const float* row_scale;
+    void* y;
+    int32_t* acc_out;
+    int O, y_vec, nt;
+};
+
+template <bool GROUPED>
+__device__ __forceinline__ TileOwner tile_owner(const PrefillOut& out, int nt) {
+    TileOwner r{&out.tmap_w[0], &out.tmap_y[0], out.row_scale[0], out.y[0], out.acc_out[0], out.O[0], out.y_vec[0], nt};
+    if (GROUPED && out.G > 1) {
+#pragma unroll
+        for (int i = 1; i < kPrefillMaxGroup; ++i)
+            if (i < out.G && nt >= out.nt_end[i - 1]) {  // constant indices only
+                r.tmap_w = &out.tmap_w[i];
+                r.tmap_y = &out.tmap_y[i];
+                r.row_scale = out.row_scale[i];
+                r.y = out.y[i];
+                r.acc_out = out.acc_out[i];
+                r.O = out.O[i];
+                r.y_vec = out.y_vec[i];
+                r.nt = nt - out.nt_end[i - 1];
+            }
+    }
+    return r;
+}
+
 }  // namespace sbl

@@ -4,8 +4,8 @@ relative, bf16 y within 2 ulps, and the same bits as separate sbl_linear
 calls.  Token counts reach every branch: one launch over the stacked rows
 (T <= 2, with wide load batches for large groups), the warp-level MMA per
 layer (3 <= T <= 16) and, for prefill, one quantisation and one launch of the
-tensor-core GEMM over up to four layers' output tiles (more layers: several
-launches); ragged, unaligned and empty layers, rows of one warp straddling
+tensor-core GEMM (one CTA or CTA pairs) over up to four layers' output tiles
+(more layers: several launches); ragged, unaligned and empty layers, rows of one warp straddling
 two layers, and K not a multiple of 64."""
 import numpy as np
 import pytest
@@ -38,7 +38,8 @@ def _layers(sbl, K, Os, n, m, seed):
 CASES = [
     # (K, Os, n, m, Ts)
     (896, (896, 128, 128), 3, 4, (1, 2, 5, 16, 300, 2048)),   # q, k, v of the 0.5B layer
-    (896, (4864, 4864), 3, 4, (1, 2, 40)),                     # gate, up
+    (896, (4864, 4864), 3, 4, (1, 2, 40, 2048)),               # gate, up (T = 2048: one CTA-pair launch)
+    (896, (4864, 130), 3, 4, (1000,)),                         # CTA pairs with a ragged, unaligned layer
     (256, (1, 31, 0, 130, 7, 64, 128, 3), 2, 4, (1, 2, 3, 40, 300)),  # eight ragged layers, one empty
     (48, (40, 24, 8), 6, 8, (1, 2, 7)),                        # K % 64 != 0: the dp4a decode only
     (2048, (2048, 7168), 2, 4, (1, 129)),
