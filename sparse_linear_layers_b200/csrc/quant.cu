@@ -188,7 +188,7 @@ cudaError_t launch_quant(const uint16_t* x, long long T, long long K, int8_t* xq
 // rounded once to float32 (no summation order changes it); every later step
 // is one IEEE float32 operation.
 // One warp per token; for the sum, lane l owns the 16-element blocks b with
-// b % 32 == l (up to RB of them held in registers, the rest read again); the
+// b % 32 == l (up to RB = 4 of them held in registers, the rest read again); the
 // absmax of the normalised values and the quantisation then read x again
 // (from L1) in a coalesced mapping, which their order-free arithmetic allows.
 // Non-finite input, a sum of squares past the float32 range and a non-finite
@@ -509,19 +509,17 @@ template <int LAYOUT>
 static void launch_rms_rb(const uint16_t* x, const float* g, float eps, long long T, long long K, int8_t* xq,
                           float* s_tok, uint4* zw, long long nzero, unsigned* status, cudaStream_t stream) {
     const unsigned blocks = static_cast<unsigned>((T + 7) / 8);
-    // blocks per lane; rows up to K = 8192 stay in registers for the sum of
-    // squares (read once from memory), longer ones read the rest again
+    // blocks per lane held in registers: up to four (rows up to K = 2048); the
+    // rest of a longer row is read again from L1/L2 in each pass.  Holding whole
+    // rows of K = 4864 (ten blocks, 128 registers) cut the resident warps from
+    // about 54% to 21% and ran slower (ncu), so four is the limit.
     const long long per_lane = ((K >> 4) + 31) / 32;
     if (per_lane <= 1)
         pdl_launch(rmsnorm_quant_kernel<LAYOUT, 1>, dim3(blocks), dim3(256), 0, stream, x, g, eps, T, K, xq, s_tok, zw, nzero, status);
     else if (per_lane <= 2)
         pdl_launch(rmsnorm_quant_kernel<LAYOUT, 2>, dim3(blocks), dim3(256), 0, stream, x, g, eps, T, K, xq, s_tok, zw, nzero, status);
-    else if (per_lane <= 4)
-        pdl_launch(rmsnorm_quant_kernel<LAYOUT, 4>, dim3(blocks), dim3(256), 0, stream, x, g, eps, T, K, xq, s_tok, zw, nzero, status);
-    else if (per_lane <= 10)
-        pdl_launch(rmsnorm_quant_kernel<LAYOUT, 10>, dim3(blocks), dim3(256), 0, stream, x, g, eps, T, K, xq, s_tok, zw, nzero, status);
     else
-        pdl_launch(rmsnorm_quant_kernel<LAYOUT, 16>, dim3(blocks), dim3(256), 0, stream, x, g, eps, T, K, xq, s_tok, zw, nzero, status);
+        pdl_launch(rmsnorm_quant_kernel<LAYOUT, 4>, dim3(blocks), dim3(256), 0, stream, x, g, eps, T, K, xq, s_tok, zw, nzero, status);
 }
 
 // RMSNorm then per-token absmax int8 (layout as launch_quant); g fp32 [K]
