@@ -76,17 +76,14 @@ struct DecodeGroup {
     int G;
 };
 
-// RT: the block has blockDim.x <= decode_threads<NB>() threads (a multiple of
-// 32, chosen at launch); otherwise exactly decode_threads<NB>().
-template <int L, int TT, int CW, int NB, bool RT>
+template <int L, int TT, int CW, int NB>
 __global__ void __launch_bounds__(decode_threads<NB>(), decode_min_blocks<TT, NB>()) decode_kernel(const DecodeGroup grp, int K,
                                                                 const uint16_t* __restrict__ x, long long T,
                                                                 long long t0, int y_bf16, unsigned* status) {
     extern __shared__ uint4 xs[];  // TT x K/16 units of quantised activations (decode layout)
-    constexpr int MAXW = decode_threads<NB>() / 32;
-    const int NTH = RT ? static_cast<int>(blockDim.x) : decode_threads<NB>();
-    const int NWP = NTH >> 5;
-    __shared__ uint32_t red[MAXW][TT];
+    constexpr int NTH = decode_threads<NB>();
+    constexpr int NWP = NTH / 32;
+    __shared__ uint32_t red[NWP][TT];
     __shared__ float s_sh[TT];
     asm volatile("griddepcontrol.launch_dependents;");
     constexpr int RW = 32 / L;
@@ -160,8 +157,7 @@ __global__ void __launch_bounds__(decode_threads<NB>(), decode_min_blocks<TT, NB
         __syncthreads();
         mx = 0;
 #pragma unroll
-        for (int w = 0; w < MAXW; ++w)
-            if (w < NWP) mx = max(mx, red[w][0]);
+        for (int w = 0; w < NWP; ++w) mx = max(mx, red[w][0]);
         const float st = __fdiv_rn(127.0f, fmaxf(__uint_as_float(mx << 16), 1e-5f));
         if (threadIdx.x == 0) {
             if (mx >= 0x7F80u && blockIdx.x == 0) raise_status(status, kStatusNonfinite);
@@ -190,8 +186,7 @@ __global__ void __launch_bounds__(decode_threads<NB>(), decode_min_blocks<TT, NB
         if (threadIdx.x < TT) {
             uint32_t mx = 0;
 #pragma unroll
-            for (int w = 0; w < MAXW; ++w)
-                if (w < NWP) mx = max(mx, red[w][threadIdx.x]);
+            for (int w = 0; w < NWP; ++w) mx = max(mx, red[w][threadIdx.x]);
             if (mx >= 0x7F80u && blockIdx.x == 0) raise_status(status, kStatusNonfinite);
             s_sh[threadIdx.x] = __fdiv_rn(127.0f, fmaxf(__uint_as_float(mx << 16), 1e-5f));
         }
@@ -347,18 +342,23 @@ static DecodePlan choose_plan(long long O, int cpr, int num_sms, int tt, bool wi
     return {L1, kDecodeBatch};
 }
 
-template <int L, int TT, int CW, int NB, bool RT>
-static cudaError_t launch_decode_k(const DecodeGroup& grp, int K, const uint16_t* x, long long T, long long t0,
-                                   int y_bf16, unsigned* status, long long blocks, int threads, cudaStream_t stream) {
+template <int L, int TT, int CW, int NB>
+static cudaError_t launch_decode_lt(const DecodeGroup& grp, int K, const uint16_t* x, long long T, long long t0,
+                                    int y_bf16, unsigned* status, cudaStream_t stream) {
+    constexpr int RW = 32 / L;
+    const long long rows = grp.row_end[grp.G - 1];
+    const long long groups = (rows + RW - 1) / RW;
+    constexpr int NTH = decode_threads<NB>();
+    const long long blocks = (groups + NTH / 32 - 1) / (NTH / 32);
     const size_t smem = static_cast<size_t>(TT) * K;
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<L, TT, CW, NB, RT>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<L, TT, CW, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
         if (e != cudaSuccess) return e;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(blocks));
-    cfg.blockDim = dim3(static_cast<unsigned>(threads));
+    cfg.blockDim = dim3(NTH);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -366,54 +366,21 @@ static cudaError_t launch_decode_k(const DecodeGroup& grp, int K, const uint16_t
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_kernel<L, TT, CW, NB, RT>, grp, K, x, T, t0, y_bf16, status);
-}
-
-template <int L, int TT, int CW, int NB>
-static cudaError_t launch_decode_lt(const DecodeGroup& grp, int K, const uint16_t* x, long long T, long long t0,
-                                    int y_bf16, unsigned* status, int num_sms, cudaStream_t stream) {
-    constexpr int RW = 32 / L;
-    constexpr int MAXW = decode_threads<NB>() / 32;
-    const long long rows = grp.row_end[grp.G - 1];
-    const long long groups = (rows + RW - 1) / RW;
-    const long long full_blocks = (groups + MAXW - 1) / MAXW;
-    // A one-token call whose full-size grid would cover most SMs (three
-    // quarters or more) or few of them (a quarter or less) takes blocks of as
-    // few warps as keep the grid within one block per SM (at least four, and
-    // enough threads to hold x one 16-element block each), so every SM gets
-    // the same share of row groups.  In between, full blocks leave the other
-    // SMs to the next call's blocks; in chains of dependent calls (graph
-    // replay) that measured faster for 896->4864 and 4864->896, and full
-    // blocks did for two tokens.
-    if constexpr (TT == 1 && NB == kDecodeBatch) {
-        const long long sms = num_sms > 0 ? num_sms : 1;
-        if (4 * full_blocks >= 3 * sms || 4 * full_blocks <= sms) {
-            long long nwp = (groups + sms - 1) / sms;
-            const long long need = ((K >> 4) + 31) / 32;  // warps to hold x one block per thread
-            if (nwp < need) nwp = need;
-            if (nwp < 4) nwp = 4;
-            if (nwp < MAXW)
-                return launch_decode_k<L, TT, CW, NB, true>(grp, K, x, T, t0, y_bf16, status,
-                                                            (groups + nwp - 1) / nwp, static_cast<int>(32 * nwp),
-                                                            stream);
-        }
-    }
-    return launch_decode_k<L, TT, CW, NB, false>(grp, K, x, T, t0, y_bf16, status, full_blocks,
-                                                 decode_threads<NB>(), stream);
+    return cudaLaunchKernelEx(&cfg, decode_kernel<L, TT, CW, NB>, grp, K, x, T, t0, y_bf16, status);
 }
 
 template <int TT, int CW, int NB>
 static cudaError_t launch_decode_t(int L, const DecodeGroup& grp, int K, const uint16_t* x, long long T,
-                                   long long t0, int y_bf16, unsigned* status, int num_sms, cudaStream_t stream) {
+                                   long long t0, int y_bf16, unsigned* status, cudaStream_t stream) {
 #define SBL_DECODE_CASE(LV) \
-    case LV: return launch_decode_lt<LV, TT, CW, NB>(grp, K, x, T, t0, y_bf16, status, num_sms, stream);
+    case LV: return launch_decode_lt<LV, TT, CW, NB>(grp, K, x, T, t0, y_bf16, status, stream);
     switch (L) {
         SBL_DECODE_CASE(32)
         SBL_DECODE_CASE(16)
         SBL_DECODE_CASE(8)
         SBL_DECODE_CASE(4)
         SBL_DECODE_CASE(2)
-        default: return launch_decode_lt<1, TT, CW, NB>(grp, K, x, T, t0, y_bf16, status, num_sms, stream);
+        default: return launch_decode_lt<1, TT, CW, NB>(grp, K, x, T, t0, y_bf16, status, stream);
     }
 #undef SBL_DECODE_CASE
 }
@@ -421,15 +388,15 @@ static cudaError_t launch_decode_t(int L, const DecodeGroup& grp, int K, const u
 template <int TT>
 static cudaError_t launch_decode_cw(const DecodePlan& plan, bool wide, const DecodeGroup& grp, int K,
                                     const uint16_t* x, long long T, long long t0, int y_bf16, unsigned* status,
-                                    int num_sms, cudaStream_t stream) {
+                                    cudaStream_t stream) {
     if (wide) {
         if constexpr (TT <= 2) {
             if (plan.NB == kDecodeBatchWide)
-                return launch_decode_t<TT, 4, kDecodeBatchWide>(plan.L, grp, K, x, T, t0, y_bf16, status, num_sms, stream);
+                return launch_decode_t<TT, 4, kDecodeBatchWide>(plan.L, grp, K, x, T, t0, y_bf16, status, stream);
         }
-        return launch_decode_t<TT, 4, kDecodeBatch>(plan.L, grp, K, x, T, t0, y_bf16, status, num_sms, stream);
+        return launch_decode_t<TT, 4, kDecodeBatch>(plan.L, grp, K, x, T, t0, y_bf16, status, stream);
     }
-    return launch_decode_t<TT, 1, kDecodeBatch>(plan.L, grp, K, x, T, t0, y_bf16, status, num_sms, stream);
+    return launch_decode_t<TT, 1, kDecodeBatch>(plan.L, grp, K, x, T, t0, y_bf16, status, stream);
 }
 
 // Decode of G weight matrices that share x, for any T: passes of up to 8
@@ -446,10 +413,10 @@ static cudaError_t launch_decode_group(const DecodeGroup& grp, long long K, cons
         const int tt = rem > 4 ? 8 : rem > 2 ? 4 : static_cast<int>(rem);
         const DecodePlan plan = choose_plan(rows, cpr, num_sms, tt, wide);
         cudaError_t e;
-        if (tt == 8) e = launch_decode_cw<8>(plan, wide, grp, Ki, x, T, t0, y_bf16, status, num_sms, stream);
-        else if (tt == 4) e = launch_decode_cw<4>(plan, wide, grp, Ki, x, T, t0, y_bf16, status, num_sms, stream);
-        else if (tt == 2) e = launch_decode_cw<2>(plan, wide, grp, Ki, x, T, t0, y_bf16, status, num_sms, stream);
-        else e = launch_decode_cw<1>(plan, wide, grp, Ki, x, T, t0, y_bf16, status, num_sms, stream);
+        if (tt == 8) e = launch_decode_cw<8>(plan, wide, grp, Ki, x, T, t0, y_bf16, status, stream);
+        else if (tt == 4) e = launch_decode_cw<4>(plan, wide, grp, Ki, x, T, t0, y_bf16, status, stream);
+        else if (tt == 2) e = launch_decode_cw<2>(plan, wide, grp, Ki, x, T, t0, y_bf16, status, stream);
+        else e = launch_decode_cw<1>(plan, wide, grp, Ki, x, T, t0, y_bf16, status, stream);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
