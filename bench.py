@@ -968,7 +968,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration sweep (profiling runs)")
-    ap.add_argument("--only", choices=("rmsnorm_front", "mask_monitor", "ste_backward", "int8_peak", "step_once"),
+    ap.add_argument("--only", choices=("rmsnorm_front", "mask_monitor", "ste_backward", "int8_peak", "step_once",
+                                       "decode_roofline"),
                     help="run only this auxiliary measurement on one GPU and print its JSON (profiling runs)")
     ap.add_argument("--tokens", type=int, default=32768, help="tokens of the --only rmsnorm_front measurement")
     args = ap.parse_args()
@@ -997,6 +998,8 @@ def main():
             res = _int8_peak(dev)
         elif args.only == "step_once":
             res = _step_once(sbl, dev)
+        elif args.only == "decode_roofline":
+            res = _decode_roofline(sbl, dev, hbm_peak)
         else:
             res = _ste_backward_bench(sbl, dev)
         print(json.dumps({"only": args.only, "result": res}), flush=True)

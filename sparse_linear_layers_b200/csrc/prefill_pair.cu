@@ -20,13 +20,15 @@
 // code tile written and read, int8 weight half written and read) for the
 // same 128 x 256 x 128 multiply-adds that cost about 112 KB on one CTA.
 //
-// Warp roles in each CTA (320 threads):
-//   warps 0-3  epilogue: warp w owns TMEM lanes 32w .. 32w + 31 (32 tokens);
-//              pipelined tcgen05.ld, dequantise, 128B-swizzled staging
-//              boxes, TMA bulk stores
-//   warps 4-7  weight expansion: one thread per output row of the CTA's half
-//   warp 8     TMA producer (activation half-tile, code half-tile)
-//   warp 9     TMEM allocation (both CTAs) and, in the even CTA, MMA issue
+// Warp roles in each CTA (448 threads):
+//   warps 0-7  epilogue: warp w owns TMEM lanes 32 (w % 4) .. + 31 (32 tokens)
+//              and accumulator columns 128 (w / 4) .. + 127; pipelined
+//              tcgen05.ld, dequantise, a 128B-swizzled staging box, TMA bulk
+//              stores (with four warps the fp32 epilogue of a 256 x 256 tile,
+//              128 KB per CTA, outlasted the tile's MMAs at K = 896)
+//   warps 8-11 weight expansion: one thread per output row of the CTA's half
+//   warp 12    TMA producer (activation half-tile, code half-tile)
+//   warp 13    TMEM allocation (both CTAs) and, in the even CTA, MMA issue
 //
 // Barriers: the activation loads of both CTAs complete on the even CTA's
 // full_a; each CTA's code tile completes on its own full_c; the expansion
@@ -53,7 +55,7 @@ constexpr int A_BYTES = BM * BK;
 constexpr int B_BYTES = BNH * BK;
 constexpr int P_BYTES = BNH * BK / 4;       // 2-bit codes of the CTA's half of B
 constexpr int STAGES = 5;
-constexpr int EPI_WARPS = 4;
+constexpr int EPI_WARPS = 8;              // two per TMEM lane quadrant, one per column half
 constexpr int DEC_WARPS = BNH / 32;
 constexpr int WARP_TMA = EPI_WARPS + DEC_WARPS;
 constexpr int WARP_MMA = WARP_TMA + 1;
@@ -66,8 +68,8 @@ struct PairSmem {
     uint8_t a[pp::STAGES][pp::A_BYTES];     // 1024-byte aligned tiles
     uint8_t b[pp::STAGES][pp::B_BYTES];
     uint8_t p[pp::STAGES][pp::P_BYTES];
-    uint8_t ystage[pp::EPI_WARPS][2][pp::Y_BYTES];
-    float wscale[pp::EPI_WARPS][pp::BN];
+    uint8_t ystage[pp::EPI_WARPS][pp::Y_BYTES];    // one staging box per epilogue warp
+    float wscale[pp::EPI_WARPS][pp::BN / 2];
     uint64_t full_a[pp::STAGES];            // used in the even CTA
     uint64_t full_c[pp::STAGES];
     uint64_t full_dec[pp::STAGES];          // used in the even CTA
@@ -150,20 +152,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
 
     if (warp < pp::EPI_WARPS) {
         // ------------------------------------------------------------ epilogue
-        // As in the one-CTA kernel: per tile the warp copies the 256 row scales
-        // into its shared-memory slice, waits for the accumulator, then walks
-        // the 32-column TMEM slices with the next one in flight, dequantises
-        // and stores 128 output bytes per token per round through a staging box.
-        // The buffer is handed back to the even CTA's MMA issuer once read.
+        // Warp w reads TMEM lanes 32 (w % 4) .. + 31 (32 tokens of the CTA's
+        // half) and the 128 accumulator columns of half w / 4.  Per tile it
+        // copies its 128 row scales into its shared-memory slice, waits for the
+        // accumulator, then walks its four 32-column TMEM slices with the next
+        // one in flight, dequantises and stores 128 output bytes per token per
+        // round through its staging box.  Once all eight warps of both CTAs have
+        // read the buffer it goes back to the even CTA's MMA issuer.
         auto run = [&](auto bf16_tag) {
             constexpr bool BF = decltype(bf16_tag)::value;
             constexpr int SPR = BF ? 2 : 1;          // 32-column slices per round
-            constexpr int NSL = pp::BN / 32;         // slices per tile
-            const int row = warp * 32 + lane;        // TMEM lane == token within the CTA's half
-            const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+            constexpr int NSL = pp::BN / 64;         // slices of this warp per tile
+            const int qd = warp & 3, half = warp >> 2;
+            const int row = qd * 32 + lane;          // TMEM lane == token within the CTA's half
+            const uint32_t lane_addr = static_cast<uint32_t>(qd * 32) << 16;
+            const int col0 = half * (pp::BN / 2);    // first accumulator column of this warp
             float* const wsc = sm->wscale[warp];
             int tc = 0;
-            uint32_t nstore = 0;
             for (int tile = pair; tile < tiles; tile += npairs, ++tc) {
                 const int mt = tile / NT;  // output tiles fastest: a token tile is read once
                 int g = 0, nt = tile % NT;
@@ -178,7 +183,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
                 __syncwarp();
 #pragma unroll
                 for (int k = 0; k < NSL; ++k) {
-                    const int o = nt * pp::BN + 32 * k + lane;
+                    const int o = nt * pp::BN + col0 + 32 * k + lane;
                     wsc[32 * k + lane] = o < O ? __ldg(row_scale + o) : 0.f;
                 }
                 __syncwarp();
@@ -188,9 +193,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
                 const int t = trow0 + row;
                 const bool tvalid = t < T;
                 const float inv_s = tvalid ? __frcp_rn(s_tok[t]) : 0.f;
-                const uint32_t tbase = tmem_base + lane_addr + b * pp::BN;
+                const uint32_t tbase = tmem_base + lane_addr + b * pp::BN + col0;
                 uint32_t ra[32], rb[32];
-                uint32_t q[32];
                 auto slice = [&](auto h_tag, const int k, uint32_t (&cur)[32], uint32_t (&nxt)[32]) {
                     constexpr int H = decltype(h_tag)::value;
                     const bool more = k + 1 < NSL;
@@ -203,66 +207,72 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
                         if (lane == 0) arrive_leader(&sm->tmem_empty[b]);
                     }
                     const float* sc = wsc + 32 * k;
+                    const int o0 = nt * pp::BN + col0 + 32 * (k - H);  // first output of the round
+                    uint8_t* const box = sm->ystage[warp];
+                    if (y_vec && H == 0) {
+                        if (lane == 0) bulk_wait_read<0>();  // the box's previous store has read it
+                        __syncwarp();
+                    }
+                    // 16 output bytes at a time: into the lane's row of the staging
+                    // box (128B-swizzled) or, for shapes whose row pitch is not a
+                    // multiple of 16 bytes, straight to y
+                    auto put = [&](const int c, uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
+                        if (y_vec) {
+                            const uint32_t a = smem_u32(box + lane * 128 + ((c ^ (lane & 7)) << 4));
+                            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(w0), "r"(w1), "r"(w2),
+                                         "r"(w3)
+                                         : "memory");
+                        } else if (tvalid) {
+                            void* const y = out.y[g];
+                            const long long base = static_cast<long long>(t) * O + o0;
+                            const uint32_t w[4] = {w0, w1, w2, w3};
 #pragma unroll
-                    for (int i = 0; i < 32; i += 4) {
-                        const float4 s4 = *reinterpret_cast<const float4*>(sc + i);
-                        const float f0 = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int>(cur[i + 0])), s4.x), inv_s);
-                        const float f1 = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int>(cur[i + 1])), s4.y), inv_s);
-                        const float f2 = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int>(cur[i + 2])), s4.z), inv_s);
-                        const float f3 = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int>(cur[i + 3])), s4.w), inv_s);
-                        if (BF) {
-                            const __nv_bfloat162 h01 = __floats2bfloat162_rn(f0, f1);
-                            const __nv_bfloat162 h23 = __floats2bfloat162_rn(f2, f3);
-                            q[16 * H + i / 2] = *reinterpret_cast<const uint32_t*>(&h01);
-                            q[16 * H + i / 2 + 1] = *reinterpret_cast<const uint32_t*>(&h23);
-                        } else {
-                            q[i] = __float_as_uint(f0);
-                            q[i + 1] = __float_as_uint(f1);
-                            q[i + 2] = __float_as_uint(f2);
-                            q[i + 3] = __float_as_uint(f3);
+                            for (int j = 0; j < 4; ++j) {
+                                if (BF) {
+                                    const int e = 8 * c + 2 * j;
+                                    if (o0 + e < O) reinterpret_cast<uint16_t*>(y)[base + e] = static_cast<uint16_t>(w[j] & 0xFFFFu);
+                                    if (o0 + e + 1 < O) reinterpret_cast<uint16_t*>(y)[base + e + 1] = static_cast<uint16_t>(w[j] >> 16);
+                                } else {
+                                    const int e = 4 * c + j;
+                                    if (o0 + e < O) reinterpret_cast<uint32_t*>(y)[base + e] = w[j];
+                                }
+                            }
+                        }
+                    };
+                    auto deq = [&](int i) {  // y of column i of the slice, before the output rounding
+                        return __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int>(cur[i])), sc[i]), inv_s);
+                    };
+                    if (BF) {
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {  // 8 columns per 16-byte chunk
+                            const int i = 8 * c;
+                            const __nv_bfloat162 h0 = __floats2bfloat162_rn(deq(i), deq(i + 1));
+                            const __nv_bfloat162 h1 = __floats2bfloat162_rn(deq(i + 2), deq(i + 3));
+                            const __nv_bfloat162 h2 = __floats2bfloat162_rn(deq(i + 4), deq(i + 5));
+                            const __nv_bfloat162 h3 = __floats2bfloat162_rn(deq(i + 6), deq(i + 7));
+                            put(4 * H + c, *reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1),
+                                *reinterpret_cast<const uint32_t*>(&h2), *reinterpret_cast<const uint32_t*>(&h3));
+                        }
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {  // 4 columns per 16-byte chunk
+                            const int i = 4 * c;
+                            put(c, __float_as_uint(deq(i)), __float_as_uint(deq(i + 1)), __float_as_uint(deq(i + 2)),
+                                __float_as_uint(deq(i + 3)));
                         }
                     }
                     int32_t* const acc_out = out.acc_out[g];
                     if (acc_out && tvalid) {
-                        const long long base = static_cast<long long>(t) * O + nt * pp::BN + 32 * k;
+                        const long long base = static_cast<long long>(t) * O + nt * pp::BN + col0 + 32 * k;
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
-                            if (nt * pp::BN + 32 * k + i < O) acc_out[base + i] = static_cast<int>(cur[i]);
+                            if (nt * pp::BN + col0 + 32 * k + i < O) acc_out[base + i] = static_cast<int>(cur[i]);
                     }
-                    if (H == SPR - 1) {
-                        const int o0 = nt * pp::BN + 32 * (k - H);
-                        if (y_vec) {
-                            uint8_t* const box = sm->ystage[warp][nstore & 1];
-                            if (lane == 0) bulk_wait_read<1>();
-                            __syncwarp();
-#pragma unroll
-                            for (int c = 0; c < 8; ++c) {
-                                const uint32_t a = smem_u32(box + lane * 128 + ((c ^ (lane & 7)) << 4));
-                                asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(q[4 * c]),
-                                             "r"(q[4 * c + 1]), "r"(q[4 * c + 2]), "r"(q[4 * c + 3])
-                                             : "memory");
-                            }
-                            fence_proxy_async_smem();
-                            __syncwarp();
-                            if (lane == 0)
-                                tma_store_2d(tile_owner<GROUPED>(out, tile % NT).tmap_y, smem_u32(box), o0, trow0 + warp * 32);
-                            ++nstore;
-                        } else if (tvalid) {
-                            // direct stores: shapes whose row pitch is not a multiple of 16 bytes
-                            void* const y = out.y[g];
-                            const long long base = static_cast<long long>(t) * O + o0;
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) {
-                                if (BF) {
-                                    if (o0 + 2 * i < O)
-                                        reinterpret_cast<uint16_t*>(y)[base + 2 * i] = static_cast<uint16_t>(q[i] & 0xFFFFu);
-                                    if (o0 + 2 * i + 1 < O)
-                                        reinterpret_cast<uint16_t*>(y)[base + 2 * i + 1] = static_cast<uint16_t>(q[i] >> 16);
-                                } else if (o0 + i < O) {
-                                    reinterpret_cast<uint32_t*>(y)[base + i] = q[i];
-                                }
-                            }
-                        }
+                    if (H == SPR - 1 && y_vec) {
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0)
+                            tma_store_2d(tile_owner<GROUPED>(out, tile % NT).tmap_y, smem_u32(box), o0, trow0 + qd * 32);
                     }
                     if (more) tmem_ld_wait();
                 };
