@@ -49,7 +49,7 @@ WORKLOAD = "qwen2.5-0.5b layer projections (q,k,v,o,gate,up,down), 3:4, prep + T
 # launch ends are not counted).
 # Only valid for the kernel sources the counters were taken on; reported as null
 # once those change.
-PREFILL_TRAFFIC = {"sources_sha256": "d1e0b78eabecd48e1203d7286ac19a8c70d069956a44d33ea50e64b968721ce7", "bytes_per_call": 16810176}
+PREFILL_TRAFFIC = {"sources_sha256": "7cb7760b82b9a491c8870f3eadc527cf5fe6ee26bab22a2512c73232c2691582", "bytes_per_call": 16878848}
 
 
 def _kernel_sources_digest():
@@ -969,7 +969,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration sweep (profiling runs)")
     ap.add_argument("--only", choices=("rmsnorm_front", "mask_monitor", "ste_backward", "int8_peak", "step_once",
-                                       "decode_roofline"),
+                                       "decode_roofline", "prefill_roofline"),
                     help="run only this auxiliary measurement on one GPU and print its JSON (profiling runs)")
     ap.add_argument("--tokens", type=int, default=32768, help="tokens of the --only rmsnorm_front measurement")
     args = ap.parse_args()
@@ -1000,6 +1000,8 @@ def main():
             res = _step_once(sbl, dev)
         elif args.only == "decode_roofline":
             res = _decode_roofline(sbl, dev, hbm_peak)
+        elif args.only == "prefill_roofline":
+            res = _prefill_roofline(sbl, dev, 2.0 * _peaks()[1], hbm_peak)
         else:
             res = _ste_backward_bench(sbl, dev)
         print(json.dumps({"only": args.only, "result": res}), flush=True)
