@@ -273,9 +273,10 @@ class StepGraphs:
 
 class E2E:
     """The step from pinned host buffers: H2D of W and x, D2H of y, inside the
-    timed region.  Three streams: host-to-device copies, the kernels, and
-    device-to-host copies, so both directions of the host link and the
-    kernels overlap across groups and steps.  Events keep every buffer safe:
+    timed region, every copy through the library's C ABI (sbl_copy_to_device,
+    sbl_copy_to_host) like every kernel.  Three streams: host-to-device
+    copies, the kernels, and device-to-host copies, so both directions of the
+    host link and the kernels overlap across groups and steps.  Events keep every buffer safe:
     a group's inputs are not overwritten before the previous step's kernels
     have read them, and its outputs not before they have been copied back."""
 
@@ -285,6 +286,20 @@ class E2E:
         self.back = torch.cuda.Stream()
         self.consumed = {g.name: None for g in groups}
         self.done = {g.name: None for g in groups}
+        # per group, the (destination, source, bytes) of every copy, checked once
+        # here so the timed loop only makes the C ABI calls
+        from sparse_linear_layers_b200 import api
+        pair = api._need_host_pair
+        self.ins, self.outs = {}, {}
+        for g in groups:
+            ins = [(g.x.data_ptr(), g.x_host.data_ptr(), pair(g.x_host, g.x, "x_host", "x")),
+                   (g.x1.data_ptr(), g.x1_host.data_ptr(), pair(g.x1_host, g.x1, "x1_host", "x1"))]
+            ins += [(L.W.data_ptr(), L.W_host.data_ptr(), pair(L.W_host, L.W, "W_host", "W")) for L in g.members]
+            outs = []
+            for L in g.members:
+                outs.append((L.y_host.data_ptr(), L.y.data_ptr(), pair(L.y_host, L.y, "y_host", "y")))
+                outs.append((L.y1_host.data_ptr(), L.y1.data_ptr(), pair(L.y1_host, L.y1, "y1_host", "y1")))
+            self.ins[g.name], self.outs[g.name] = ins, outs
 
     def begin(self):
         """Order the copy streams after everything already on the main stream."""
@@ -294,17 +309,16 @@ class E2E:
         self.back.wait_event(ev)
 
     def step(self, sbl, groups):
+        from sparse_linear_layers_b200._lib import check, lib
         h2d = d2h = 0
+        s_in, s_out = self.h2d.cuda_stream, self.back.cuda_stream
         for g in groups:
             with torch.cuda.stream(self.h2d):
                 if self.consumed[g.name] is not None:
                     self.h2d.wait_event(self.consumed[g.name])  # the previous step's kernels read these inputs
-                g.x.copy_(g.x_host, non_blocking=True)
-                g.x1.copy_(g.x1_host, non_blocking=True)
-                h2d += g.x_host.numel() * 2 + g.x1_host.numel() * 2
-                for L in g.members:
-                    L.W.copy_(L.W_host, non_blocking=True)
-                    h2d += L.W_host.numel() * 4
+                for dst, src, nb in self.ins[g.name]:
+                    check(lib.sbl_copy_to_device(dst, src, nb, s_in), "sbl_copy_to_device")
+                    h2d += nb
                 copied = torch.cuda.Event()
                 copied.record(self.h2d)
             with torch.cuda.stream(self.main):
@@ -319,10 +333,9 @@ class E2E:
                 self.consumed[g.name] = computed
             self.back.wait_event(computed)
             with torch.cuda.stream(self.back):
-                for L in g.members:
-                    L.y_host.copy_(L.y, non_blocking=True)
-                    L.y1_host.copy_(L.y1, non_blocking=True)
-                    d2h += L.y.numel() * 4 + L.y1.numel() * 4
+                for dst, src, nb in self.outs[g.name]:
+                    check(lib.sbl_copy_to_host(dst, src, nb, s_out), "sbl_copy_to_host")
+                    d2h += nb
                 ev = torch.cuda.Event()
                 ev.record(self.back)
                 self.done[g.name] = ev
@@ -840,7 +853,9 @@ def run_ours(args, rank, world, dev):
         "ste_backward": ste_bwd,
         "phases": phases,
         "e2e": {"value": world * TOKENS_PER_STEP * K_e2e / e2e_s, "steps": K_e2e, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+                "d2h_bytes_per_step": d2h,
+                "calls": "C ABI only: sbl_copy_to_device (W, x), sbl_prepare_weights_grouped, sbl_linear_grouped / "
+                         "sbl_linear, sbl_copy_to_host (y); pinned host buffers"},
         "gpu_launches": launches_per_step * K,
         "clocks": clocks,
     }

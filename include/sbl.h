@@ -306,6 +306,48 @@ sbl_status sbl_linear(const uint16_t* x_bf16, int64_t T, int64_t K,
                       void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * sbl_copy_to_device, sbl_copy_to_host — the host<->device transfers of a
+ * pass that starts and ends in host memory (x and the latent weights in, y
+ * out), enqueued on `stream` as one asynchronous copy each; they return
+ * before the copy has finished.
+ *
+ *   device_dst / device_src  device memory of the caller.
+ *   host_src / host_dst      host memory of the caller; page-locked memory
+ *                            (cudaHostAlloc, torch pin_memory) lets the copy
+ *                            overlap kernels and the other direction, pageable
+ *                            memory is staged by the runtime.
+ *   bytes                    0 is a no-op (the pointers are not read).
+ * Errors: SBL_ERR_INVALID_ARG for a NULL pointer with bytes > 0 (checked on
+ * the host before anything is enqueued); SBL_ERR_CUDA if the runtime rejects
+ * the copy.
+ */
+sbl_status sbl_copy_to_device(void* device_dst, const void* host_src, size_t bytes, void* stream);
+sbl_status sbl_copy_to_host(void* host_dst, const void* device_src, size_t bytes, void* stream);
+
+/*
+ * sbl_linear_hostio — sbl_linear on activations and outputs in host memory
+ * (the Sparse-BitNet Guide, "Mathematical Formulation of Sparse-BitLinear",
+ * as sbl_linear): copies x_host into x_dev, runs sbl_linear(x_dev, ..., y_dev,
+ * ...) and copies y_dev into y_host, all three enqueued on `stream` in that
+ * order; the call returns before they finish, so synchronise the stream
+ * before reading y_host.
+ *
+ *   x_host   bf16 bit patterns [T, K] in host memory (page-locked for overlap).
+ *   x_dev    device staging for x, T*K*2 bytes, 16-byte aligned.
+ *   y_dev    device staging for y, T*O*4 (SBL_F32) or T*O*2 (SBL_BF16) bytes,
+ *            16-byte aligned.
+ *   y_host   host memory for y, the same size.
+ *   Other arguments as sbl_linear (no acc_out).
+ * Errors: the argument checks of sbl_linear, and SBL_ERR_INVALID_ARG for a
+ * NULL host or staging pointer, all made on the host before anything is
+ * enqueued; SBL_ERR_CUDA if a copy or kernel launch fails.
+ */
+sbl_status sbl_linear_hostio(const uint16_t* x_host, int64_t T, int64_t K, uint16_t* x_dev,
+                             const uint8_t* packed, const float* row_scale, int64_t O, int n, int m,
+                             void* y_dev, void* y_host, int y_dtype,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * sbl_linear_path — sbl_linear with the contraction path forced
  * (SBL_PATH_DECODE, or one of the SBL_PATH_PREFILL* tensor-core paths;
  * SBL_PATH_AUTO is sbl_linear).  Every path gives the same results.

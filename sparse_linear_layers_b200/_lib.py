@@ -54,6 +54,9 @@ SIGNATURES = {
     "sbl_linear_grouped_workspace_bytes": (_sz, [_i64, _i64]),
     "sbl_linear_grouped": (_int, [_vp, _i64, _i64, _int, _vp, _vp, _vp, _int, _int, _vp, _int, _vp, _vp, _sz, _vp]),
     "sbl_linear_noalloc": (_int, [_vp, _i64, _i64, _vp, _vp, _i64, _int, _int, _vp, _int, _vp, _vp]),
+    "sbl_copy_to_device": (_int, [_vp, _vp, _sz, _vp]),
+    "sbl_copy_to_host": (_int, [_vp, _vp, _sz, _vp]),
+    "sbl_linear_hostio": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _int, _int, _vp, _vp, _int, _vp, _sz, _vp]),
     "sbl_linear_plan": (_int, [_i64, _i64, _i64, _int, _int, _sz]),
     "sbl_mask_monitor": (_int, [_vp, _vp, _i64, _i64, _int, _int, _vp, _vp, _vp]),
     "sbl_linear_backward": (_int, [_vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _int, _vp]),

@@ -201,6 +201,75 @@ def sbl_linear(x: torch.Tensor, w: PreparedWeights, out_dtype: torch.dtype = tor
     return y
 
 
+def _need_host_pair(host: torch.Tensor, dev: torch.Tensor, hname: str, dname: str) -> int:
+    """Byte count of a host <-> device copy between two contiguous tensors of
+    equal size in bytes, the host one in CPU memory, the other on a GPU."""
+    if host.is_cuda or not dev.is_cuda:
+        raise ValueError(f"{hname} must be a CPU tensor and {dname} a CUDA tensor")
+    if not host.is_contiguous() or not dev.is_contiguous():
+        raise ValueError(f"{hname} and {dname} must be contiguous")
+    nb = host.numel() * host.element_size()
+    if nb != dev.numel() * dev.element_size():
+        raise ValueError(f"{hname} and {dname} differ in size ({nb} and {dev.numel() * dev.element_size()} bytes)")
+    return nb
+
+
+def copy_to_device(dst: torch.Tensor, src: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Asynchronous copy of the host tensor ``src`` (pinned for overlap) into
+    the device tensor ``dst`` on the stream, through sbl_copy_to_device."""
+    nb = _need_host_pair(src, dst, "src", "dst")
+    check(lib.sbl_copy_to_device(dst.data_ptr(), src.data_ptr(), nb, _stream(stream)), "sbl_copy_to_device")
+    return dst
+
+
+def copy_to_host(dst: torch.Tensor, src: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Asynchronous copy of the device tensor ``src`` into the host tensor
+    ``dst`` (pinned for overlap) on the stream, through sbl_copy_to_host;
+    synchronise the stream before reading ``dst``."""
+    nb = _need_host_pair(dst, src, "dst", "src")
+    check(lib.sbl_copy_to_host(dst.data_ptr(), src.data_ptr(), nb, _stream(stream)), "sbl_copy_to_host")
+    return dst
+
+
+def sbl_linear_hostio(x_host: torch.Tensor, w: PreparedWeights, out_dtype: torch.dtype = torch.float32,
+                      y_host: Optional[torch.Tensor] = None, x_dev: Optional[torch.Tensor] = None,
+                      y_dev: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                      stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """sbl_linear with x and y in host memory (sbl_linear_hostio): copies
+    ``x_host`` (bf16 [T, K], pinned for overlap) in, contracts, copies y out
+    into ``y_host``, all enqueued on the stream; returns ``y_host``, valid once
+    the stream has been synchronised.  ``x_dev``/``y_dev`` are the device
+    staging buffers (allocated here when not given)."""
+    T, K = _need_2d(x_host, "x_host")
+    if x_host.dtype != torch.bfloat16 or x_host.is_cuda or not x_host.is_contiguous():
+        raise ValueError("x_host must be a contiguous bf16 CPU tensor")
+    if K != w.K:
+        raise ValueError(f"x has K={K}, weights were prepared with K={w.K}")
+    dev = w.packed.device
+    _need_weights(w, dev)
+    if out_dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("out_dtype must be float32 or bfloat16")
+    if y_host is None:
+        y_host = torch.empty((T, w.O), dtype=out_dtype, pin_memory=True)
+    if x_dev is None:
+        x_dev = torch.empty((T, K), dtype=torch.bfloat16, device=dev)
+    if y_dev is None:
+        y_dev = torch.empty((T, w.O), dtype=y_host.dtype, device=dev)
+    if y_host.dtype != y_dev.dtype or y_host.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("y_host and y_dev must both be float32 or both bfloat16")
+    _need_cuda(x_dev, "x_dev", torch.bfloat16, (T, K), dev)
+    _need_cuda(y_dev, "y_dev", y_host.dtype, (T, w.O), dev)
+    _need_host_pair(y_host, y_dev, "y_host", "y_dev")
+    if workspace is None:
+        workspace = workspace_for(T, K, w.O, w.n, w.m, dev)
+    _need_workspace(workspace, dev)
+    ydt = _lib.SBL_F32 if y_host.dtype == torch.float32 else _lib.SBL_BF16
+    check(lib.sbl_linear_hostio(x_host.data_ptr(), T, K, x_dev.data_ptr(), w.packed.data_ptr(), w.row_scale.data_ptr(),
+                                w.O, w.n, w.m, y_dev.data_ptr(), y_host.data_ptr(), ydt, workspace.data_ptr(),
+                                workspace.numel(), _stream(stream)), "sbl_linear_hostio")
+    return y_host
+
+
 def sbl_linear_grouped(x: torch.Tensor, ws, out_dtype: torch.dtype = torch.float32, ys=None, acc_outs=None,
                        workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None):
     """Several layers that read the same x (q/k/v, gate/up) in one call: x is

@@ -331,10 +331,12 @@ static bool sparse_preferred(int64_t T, int64_t K, int64_t O, int num_sms) {
 // The forward behind sbl_linear_path and sbl_linear_rmsnorm: with g the
 // activations are RMS-normalised by the front-end kernel before quantisation,
 // and the decode sizes take the warp-MMA kernel on the quantised activations.
+// check_only: run every host-side argument check and return before anything
+// is enqueued.
 static sbl_status linear_impl(const uint16_t* x_bf16, const float* g, float eps, int64_t T, int64_t K,
                               const uint8_t* packed, const float* row_scale, int64_t O, int n, int m, void* y,
                               int y_dtype, int32_t* acc_out, void* workspace, size_t workspace_bytes, int path,
-                              void* stream) {
+                              void* stream, bool check_only = false) {
     if (T < 0 || O < 0) return SBL_ERR_INVALID_ARG;
     if (sbl_status s = check_k(K)) return s;
     if (g) {
@@ -363,6 +365,7 @@ static sbl_status linear_impl(const uint16_t* x_bf16, const float* g, float eps,
     if (path == SBL_PATH_AUTO) prefill = ((T > kDecodeMaxTokens) || (K > kDecodeMaxK)) && (K % 64 == 0);
     if (!prefill && K > kDecodeMaxK) return SBL_ERR_UNSUPPORTED;
     if (g && !prefill && !sbl::decode_mma_supported(K)) return SBL_ERR_UNSUPPORTED;
+    if (check_only) return SBL_OK;
 
     DeviceInfo* d;
     if (sbl_status s = device_info(&d)) return s;
@@ -438,6 +441,38 @@ sbl_status sbl_linear_rmsnorm(const uint16_t* x_bf16, const float* g, float eps,
     if (!g) return SBL_ERR_INVALID_ARG;
     return linear_impl(x_bf16, g, eps, T, K, packed, row_scale, O, n, m, y, y_dtype, acc_out, workspace,
                        workspace_bytes, path, stream);
+}
+
+sbl_status sbl_copy_to_device(void* device_dst, const void* host_src, size_t bytes, void* stream) {
+    if (bytes == 0) return SBL_OK;
+    if (!device_dst || !host_src) return SBL_ERR_INVALID_ARG;
+    return from_cuda(cudaMemcpyAsync(device_dst, host_src, bytes, cudaMemcpyHostToDevice,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+sbl_status sbl_copy_to_host(void* host_dst, const void* device_src, size_t bytes, void* stream) {
+    if (bytes == 0) return SBL_OK;
+    if (!host_dst || !device_src) return SBL_ERR_INVALID_ARG;
+    return from_cuda(cudaMemcpyAsync(host_dst, device_src, bytes, cudaMemcpyDeviceToHost,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+sbl_status sbl_linear_hostio(const uint16_t* x_host, int64_t T, int64_t K, uint16_t* x_dev, const uint8_t* packed,
+                             const float* row_scale, int64_t O, int n, int m, void* y_dev, void* y_host, int y_dtype,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+    // every check first, so that an argument error enqueues nothing
+    if (sbl_status s = linear_impl(x_dev, nullptr, 0.0f, T, K, packed, row_scale, O, n, m, y_dev, y_dtype, nullptr,
+                                   workspace, workspace_bytes, SBL_PATH_AUTO, stream, true))
+        return s;
+    if (T == 0 || O == 0) return SBL_OK;
+    if (!x_host || !y_host) return SBL_ERR_INVALID_ARG;
+    const size_t x_bytes = static_cast<size_t>(T) * static_cast<size_t>(K) * 2;
+    const size_t y_bytes = static_cast<size_t>(T) * static_cast<size_t>(O) * (y_dtype == SBL_BF16 ? 2 : 4);
+    if (sbl_status s = sbl_copy_to_device(x_dev, x_host, x_bytes, stream)) return s;
+    if (sbl_status s = linear_impl(x_dev, nullptr, 0.0f, T, K, packed, row_scale, O, n, m, y_dev, y_dtype, nullptr,
+                                   workspace, workspace_bytes, SBL_PATH_AUTO, stream))
+        return s;
+    return sbl_copy_to_host(y_host, y_dev, y_bytes, stream);
 }
 
 sbl_status sbl_linear(const uint16_t* x_bf16, int64_t T, int64_t K, const uint8_t* packed, const float* row_scale,

@@ -233,3 +233,30 @@ def test_prepare_grouped_rejects_on_host():
     assert P(G, (C.c_int64 * G)(0, 0)) == 0                    # nothing to do
     bad = (C.c_void_p * G)(p + 4, p)                           # unaligned latent weights
     assert lib.sbl_prepare_weights_grouped(G, bad, ok_rows, 64, 2, 4, ptrs, ptrs, None, None) == 1
+
+
+def test_host_copies_reject_on_host():
+    from sparse_linear_layers_b200._lib import lib
+    p = 4096  # a fake address: validation fails (or the size is 0) before it could be read
+    assert lib.sbl_copy_to_device(None, None, 0, None) == 0
+    assert lib.sbl_copy_to_host(None, None, 0, None) == 0
+    assert lib.sbl_copy_to_device(None, p, 16, None) == 1
+    assert lib.sbl_copy_to_device(p, None, 16, None) == 1
+    assert lib.sbl_copy_to_host(None, p, 16, None) == 1
+    assert lib.sbl_copy_to_host(p, None, 16, None) == 1
+
+
+def test_linear_hostio_rejects_on_host():
+    from sparse_linear_layers_b200._lib import lib
+    H = lib.sbl_linear_hostio
+    p = 4096
+    # empty problems enqueue nothing
+    assert H(None, 0, 64, None, None, None, 16, 2, 4, None, None, 0, None, 0, None) == 0
+    assert H(None, 4, 64, None, None, None, 0, 2, 4, None, None, 0, None, 0, None) == 0
+    # sbl_linear's checks run first: output dtype, alignment, workspace
+    assert H(p, 4, 64, p, p, p, 16, 2, 4, p, p, 7, p, 1 << 20, None) == 1
+    assert H(p, 4, 64, p + 4, p, p, 16, 2, 4, p, p, 0, p, 1 << 20, None) == 1
+    assert H(p, 4, 64, p, p, p, 16, 2, 4, p, p, 0, p, 16, None) == 6
+    # then the host buffers
+    assert H(None, 4, 64, p, p, p, 16, 2, 4, p, p, 0, p, 1 << 20, None) == 1
+    assert H(p, 4, 64, p, p, p, 16, 2, 4, p, None, 0, p, 1 << 20, None) == 1
