@@ -46,6 +46,20 @@
 
 namespace sbl {
 
+#ifdef SBL_TRACE
+// Debug builds only: clock64 stamps of pipeline events in CTA 0 (the even CTA
+// of the first pair): event e, iteration i -> g_trace_pair[e * 256 + i].
+__device__ unsigned long long* g_trace_pair;
+#define SBLP_TR(e, i)                                                            \
+    do {                                                                         \
+        if (trace_buf && (i) < 256) trace_buf[(e) * 256 + (i)] = clock64();     \
+    } while (0)
+#else
+#define SBLP_TR(e, i) \
+    do {              \
+    } while (0)
+#endif
+
 namespace pp {
 constexpr int BM = 128;                     // tokens per CTA (pair: 256)
 constexpr int BN = 256;                     // outputs per pair tile
@@ -93,6 +107,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
     volatile int* abort_flag = &sm->abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#ifdef SBL_TRACE
+    unsigned long long* const trace_buf = blockIdx.x == 0 ? g_trace_pair : nullptr;
+#endif
+    if (threadIdx.x == 0) SBLP_TR(8, 0);  // entry
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
@@ -137,6 +155,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = sm->tmem_base;
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (threadIdx.x == 0) SBLP_TR(9, 0);  // inputs visible
 
     auto give_up = [&]() {
         if (!*abort_flag) {
@@ -188,6 +207,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
                 }
                 __syncwarp();
                 if (!warp_wait(&sm->tmem_full[b], aph, abort_flag)) { give_up(); break; }
+                if (lane == 0 && warp == 0) SBLP_TR(5, tc);
+                if (lane == 0 && warp == 4) SBLP_TR(7, tc);
                 tc_fence_after();
                 const int trow0 = mt * 2 * pp::BM + static_cast<int>(rank) * pp::BM;
                 const int t = trow0 + row;
@@ -205,6 +226,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) arrive_leader(&sm->tmem_empty[b]);
+                        if (lane == 0 && warp == 0) SBLP_TR(6, tc);
                     }
                     const float* sc = wsc + 32 * k;
                     const int o0 = nt * pp::BN + col0 + 32 * (k - H);  // first output of the round
@@ -306,6 +328,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
                 // the codes have landed; the producer loaded them only after the
                 // pair's MMAs released this stage, so b[s] is free as well
                 if (!mbar_wait(&sm->full_c[s], ph, abort_flag)) { give_up(); ok = false; break; }
+                if (r == 0) SBLP_TR(1, it);
                 // code rows are 32 bytes, 32B-swizzled by TMA: 16-byte half q of
                 // row r sits at half q ^ ((r >> 2) & 1)
                 const uint8_t* src = sm->p[s] + r * 32;
@@ -327,6 +350,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
                 if ((r & 31) == 0) arrive_leader(&sm->full_dec[s]);
+                if (r == 0) SBLP_TR(2, it);
             }
         }
     } else if (warp == pp::WARP_TMA) {
@@ -343,6 +367,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
                     const int s = it % pp::STAGES;
                     const uint32_t ph = (it / pp::STAGES) & 1;
                     if (!mbar_wait(&sm->empty[s], ph ^ 1, abort_flag)) { give_up(); ok = false; break; }
+                    SBLP_TR(0, it);
                     // the even CTA expects the activation bytes of both CTAs
                     if (leader) mbar_arrive_expect_tx(&sm->full_a[s], 2 * pp::A_BYTES);
                     mbar_arrive_expect_tx(&sm->full_c[s], pp::P_BYTES);
@@ -374,6 +399,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
                     const int b = tc & 1;
                     const uint32_t aph = (tc >> 1) & 1;
                     if (!mbar_wait(&sm->tmem_empty[b], aph ^ 1, abort_flag)) { give_up(); break; }
+                    SBLP_TR(4, tc);
                     tc_fence_after();
                     const uint32_t d = tmem_base + b * pp::BN;
                     for (int kb = 0; kb < KB; ++kb, ++it) {
@@ -383,6 +409,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pp::THREADS, 1)
                             !mbar_wait(&sm->full_dec[s], ph, abort_flag)) {
                             give_up(); ok = false; break;
                         }
+                        SBLP_TR(3, it);
                         tc_fence_after();
                         const uint32_t a0 = smem_u32(sm->a[s]), b0 = smem_u32(sm->b[s]);
 #pragma unroll
@@ -529,5 +556,12 @@ cudaError_t launch_prefill_pair(const int8_t* xperm, const float* s_tok, long lo
     int32_t* aa[1] = {acc_out};
     return launch_prefill_pair_group(xperm, s_tok, T, K, 1, &packed, &row_scale, &O, yy, y_bf16, aa, status, stream);
 }
+
+#ifdef SBL_TRACE
+cudaError_t set_pair_trace(void* buf) {
+    unsigned long long* p = static_cast<unsigned long long*>(buf);
+    return cudaMemcpyToSymbol(g_trace_pair, &p, sizeof(p));
+}
+#endif
 
 }  // namespace sbl

@@ -65,6 +65,7 @@ cudaError_t launch_prefill_sp(const int8_t* xq, const float* s_tok, long long T,
                               uint8_t* scratch, unsigned* status, int num_sms, cudaStream_t stream);
 #ifdef SBL_TRACE
 cudaError_t set_prefill_trace(void* buf);
+cudaError_t set_pair_trace(void* buf);
 #endif
 
 // Status word: one per device, read and cleared by sbl_device_status().
@@ -621,8 +622,12 @@ const char* sbl_status_string(sbl_status s) {
 const char* sbl_version(void) { return "sbl 0.1.0 (sm_100a)"; }
 
 #ifdef SBL_TRACE
-// Debug builds only: device buffer of 16 x 256 uint64 for prefill event stamps (NULL disables).
-sbl_status sbl_debug_set_trace(void* buf) { return from_cuda(sbl::set_prefill_trace(buf)); }
+// Debug builds only: device buffer of 16 x 256 uint64 for prefill event stamps, shared by the
+// one-CTA and the CTA-pair kernels (NULL disables).
+sbl_status sbl_debug_set_trace(void* buf) {
+    const cudaError_t e = sbl::set_prefill_trace(buf);
+    return from_cuda(e != cudaSuccess ? e : sbl::set_pair_trace(buf));
+}
 #endif
 
 }  // extern "C"
