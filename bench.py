@@ -276,30 +276,47 @@ class E2E:
     timed region, every copy through the library's C ABI (sbl_copy_to_device,
     sbl_copy_to_host) like every kernel.  Three streams: host-to-device
     copies, the kernels, and device-to-host copies, so both directions of the
-    host link and the kernels overlap across groups and steps.  Events keep every buffer safe:
-    a group's inputs are not overwritten before the previous step's kernels
-    have read them, and its outputs not before they have been copied back."""
+    host link and the kernels overlap across groups and steps.  Two sets of
+    device buffers (inputs and outputs) alternate between steps, as a serving
+    loop double-buffers: a step's inputs land while the previous step
+    computes, and its outputs are written while the previous step's are still
+    being copied back.  Events keep every buffer safe: a set's inputs are not
+    overwritten before the kernels of two steps ago have read them, nor its
+    outputs before they have been copied back."""
+
+    NSETS = 2
 
     def __init__(self, groups):
         self.main = torch.cuda.Stream()
         self.h2d = torch.cuda.Stream()
         self.back = torch.cuda.Stream()
-        self.consumed = {g.name: None for g in groups}
-        self.done = {g.name: None for g in groups}
-        # per group, the (destination, source, bytes) of every copy, checked once
-        # here so the timed loop only makes the C ABI calls
+        self.k = 0
+        self.consumed = {(g.name, s): None for g in groups for s in range(self.NSETS)}
+        self.done = {(g.name, s): None for g in groups for s in range(self.NSETS)}
+        # per group and set: the device buffers, and the (destination, source,
+        # bytes) of every copy, checked once here so the timed loop only makes
+        # the C ABI calls; set 0 is the step's own buffers
         from sparse_linear_layers_b200 import api
         pair = api._need_host_pair
-        self.ins, self.outs = {}, {}
+        self.bufs, self.ins, self.outs = {}, {}, {}
         for g in groups:
-            ins = [(g.x.data_ptr(), g.x_host.data_ptr(), pair(g.x_host, g.x, "x_host", "x")),
-                   (g.x1.data_ptr(), g.x1_host.data_ptr(), pair(g.x1_host, g.x1, "x1_host", "x1"))]
-            ins += [(L.W.data_ptr(), L.W_host.data_ptr(), pair(L.W_host, L.W, "W_host", "W")) for L in g.members]
-            outs = []
-            for L in g.members:
-                outs.append((L.y_host.data_ptr(), L.y.data_ptr(), pair(L.y_host, L.y, "y_host", "y")))
-                outs.append((L.y1_host.data_ptr(), L.y1.data_ptr(), pair(L.y1_host, L.y1, "y1_host", "y1")))
-            self.ins[g.name], self.outs[g.name] = ins, outs
+            for st in range(self.NSETS):
+                if st == 0:
+                    b = dict(x=g.x, x1=g.x1, W=[L.W for L in g.members], y=[L.y for L in g.members],
+                             y1=[L.y1 for L in g.members])
+                else:
+                    b = dict(x=torch.empty_like(g.x), x1=torch.empty_like(g.x1),
+                             W=[torch.empty_like(L.W) for L in g.members], y=[torch.empty_like(L.y) for L in g.members],
+                             y1=[torch.empty_like(L.y1) for L in g.members])
+                ins = [(b["x"].data_ptr(), g.x_host.data_ptr(), pair(g.x_host, b["x"], "x_host", "x")),
+                       (b["x1"].data_ptr(), g.x1_host.data_ptr(), pair(g.x1_host, b["x1"], "x1_host", "x1"))]
+                ins += [(W.data_ptr(), L.W_host.data_ptr(), pair(L.W_host, W, "W_host", "W"))
+                        for L, W in zip(g.members, b["W"])]
+                outs = []
+                for L, y, y1 in zip(g.members, b["y"], b["y1"]):
+                    outs.append((L.y_host.data_ptr(), y.data_ptr(), pair(L.y_host, y, "y_host", "y")))
+                    outs.append((L.y1_host.data_ptr(), y1.data_ptr(), pair(L.y1_host, y1, "y1_host", "y1")))
+                self.bufs[(g.name, st)], self.ins[(g.name, st)], self.outs[(g.name, st)] = b, ins, outs
 
     def begin(self):
         """Order the copy streams after everything already on the main stream."""
@@ -308,37 +325,48 @@ class E2E:
         self.h2d.wait_event(ev)
         self.back.wait_event(ev)
 
+    @staticmethod
+    def _contract(sbl, g, x, ys):
+        if len(g.members) == 1:
+            sbl.sbl_linear(x, g.members[0].w, y=ys[0], workspace=g.ws)
+        else:
+            sbl.sbl_linear_grouped(x, [L.w for L in g.members], ys=ys, workspace=g.ws)
+
     def step(self, sbl, groups):
         from sparse_linear_layers_b200._lib import check, lib
         h2d = d2h = 0
         s_in, s_out = self.h2d.cuda_stream, self.back.cuda_stream
+        st = self.k % self.NSETS
+        self.k += 1
         for g in groups:
+            key = (g.name, st)
+            b = self.bufs[key]
             with torch.cuda.stream(self.h2d):
-                if self.consumed[g.name] is not None:
-                    self.h2d.wait_event(self.consumed[g.name])  # the previous step's kernels read these inputs
-                for dst, src, nb in self.ins[g.name]:
+                if self.consumed[key] is not None:
+                    self.h2d.wait_event(self.consumed[key])  # the kernels that last read this set are done
+                for dst, src, nb in self.ins[key]:
                     check(lib.sbl_copy_to_device(dst, src, nb, s_in), "sbl_copy_to_device")
                     h2d += nb
                 copied = torch.cuda.Event()
                 copied.record(self.h2d)
             with torch.cuda.stream(self.main):
                 self.main.wait_event(copied)
-                if self.done[g.name] is not None:
-                    self.main.wait_event(self.done[g.name])  # the previous step's y copied back
-                sbl.sbl_prepare_weights_grouped([L.W for L in g.members], N, M, outs=[L.w for L in g.members])
-                g.run(sbl)
-                g.run(sbl, decode=True)
+                if self.done[key] is not None:
+                    self.main.wait_event(self.done[key])  # this set's outputs have been copied back
+                sbl.sbl_prepare_weights_grouped(b["W"], N, M, outs=[L.w for L in g.members])
+                self._contract(sbl, g, b["x"], b["y"])
+                self._contract(sbl, g, b["x1"], b["y1"])
                 computed = torch.cuda.Event()
                 computed.record(self.main)
-                self.consumed[g.name] = computed
+                self.consumed[key] = computed
             self.back.wait_event(computed)
             with torch.cuda.stream(self.back):
-                for dst, src, nb in self.outs[g.name]:
+                for dst, src, nb in self.outs[key]:
                     check(lib.sbl_copy_to_host(dst, src, nb, s_out), "sbl_copy_to_host")
                     d2h += nb
                 ev = torch.cuda.Event()
                 ev.record(self.back)
-                self.done[g.name] = ev
+                self.done[key] = ev
         return h2d, d2h
 
     def join(self):
