@@ -305,10 +305,9 @@ __global__ void __launch_bounds__((8 / WPR) * WPR * 32) prep_kernel_rr(const Pre
             for (int g = 0; g < 4; ++g) {
                 uint32_t a[4], d[4];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    a[q] = kr[j][4 * g + q] & 0x7FFFFFFFu;
-                    mx = max(mx, a[q]);
-                }
+                for (int q = 0; q < 4; ++q) a[q] = kr[j][4 * g + q] & 0x7FFFFFFFu;
+                mx = __vimax3_u32(mx, a[0], a[1]);
+                mx = __vimax3_u32(mx, a[2], a[3]);
                 drop4<N>(a, d);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
@@ -319,10 +318,9 @@ __global__ void __launch_bounds__((8 / WPR) * WPR * 32) prep_kernel_rr(const Pre
         } else {
             uint32_t a[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                a[i] = kr[j][i] & 0x7FFFFFFFu;
-                mx = max(mx, a[i]);
-            }
+            for (int i = 0; i < 16; ++i) a[i] = kr[j][i] & 0x7FFFFFFFu;
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) mx = __vimax3_u32(mx, a[i], a[i + 1]);
             const uint32_t keep = group_keep_bits<8>(a, N) | (group_keep_bits<8>(a + 8, N) << 8);
 #pragma unroll
             for (int i = 0; i < 16; ++i) kr[j][i] = ((keep >> i) & 1u) ? kr[j][i] : 0u;
@@ -330,7 +328,7 @@ __global__ void __launch_bounds__((8 / WPR) * WPR * 32) prep_kernel_rr(const Pre
         }
         // 2|w| - 1 over the kept weights: zeros wrap to the largest value
 #pragma unroll
-        for (int i = 0; i < 16; ++i) mn2 = min(mn2, (kr[j][i] << 1) - 1u);
+        for (int i = 0; i < 16; i += 2) mn2 = __vimin3_u32(mn2, (kr[j][i] << 1) - 1u, (kr[j][i + 1] << 1) - 1u);
     }
     mx = __reduce_max_sync(0xFFFFFFFFu, mx);
     mn2 = __reduce_min_sync(0xFFFFFFFFu, mn2);
@@ -432,7 +430,11 @@ __global__ void __launch_bounds__((8 / WPR) * WPR * 32) prep_kernel_rr(const Pre
 
     // pass 3: ternarise and pack.  round(w / scale) != 0 exactly when
     // |w| > scale / 2, an exact compare (scale >= 1e-5 is normal, so halving
-    // it is exact); the code is 01 for +1 and 10 for -1.
+    // it is exact); the code is 01 for +1 and 10 for -1.  With s the sign bit
+    // and a = |w| (both below 2^31), bit 31 of half - (s * 2^31 + a) is
+    // (a > half) XOR s.  Two funnel shifts per weight stack s at bit 2i + 1
+    // and that bit at bit 2i (weights 15 down to 0); then +1 = x AND NOT s
+    // and -1 = s AND NOT x.  A dropped weight is 0 here, so x = s = 0.
     const uint32_t half_bits = __float_as_uint(0.5f * sc);
     uint32_t* prow = reinterpret_cast<uint32_t*>(packed + row * (K >> 2));
     uint16_t* mrow = (WITH_MASK && mask_bits) ? reinterpret_cast<uint16_t*>(mask_bits + row * (K >> 3)) : nullptr;
@@ -440,14 +442,13 @@ __global__ void __launch_bounds__((8 / WPR) * WPR * 32) prep_kernel_rr(const Pre
     for (int j = 0; j < CPT; ++j) {
         const int c = tr + TPR * j;
         if (c >= nchunks) continue;
-        uint32_t nzw = 0, sgw = 0;  // nonzero flags at bits 2i, signs at bits 2i + 1
+        uint32_t acc = 0;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const uint32_t t = half_bits - (kr[j][i] & 0x7FFFFFFFu);  // bit 31: |w| > scale / 2
-            nzw |= (t >> (31 - 2 * i)) & (1u << (2 * i));
-            sgw |= (kr[j][i] >> (30 - 2 * i)) & (2u << (2 * i));
+        for (int i = 15; i >= 0; --i) {
+            acc = __funnelshift_l(kr[j][i], acc, 1);                   // s
+            acc = __funnelshift_l(half_bits - kr[j][i], acc, 1);  // (|w| > scale / 2) XOR s
         }
-        prow[c] = (nzw & ~(sgw >> 1)) | ((nzw << 1) & sgw);
+        prow[c] = (acc & ~(acc >> 1) & 0x55555555u) | (acc & ~(acc << 1) & 0xAAAAAAAAu);
         if constexpr (WITH_MASK)
             if (mrow) mrow[c] = static_cast<uint16_t>(kbits >> (16 * j));
     }
