@@ -49,7 +49,7 @@ WORKLOAD = "qwen2.5-0.5b layer projections (q,k,v,o,gate,up,down), 3:4, prep + T
 # launch ends are not counted).
 # Only valid for the kernel sources the counters were taken on; reported as null
 # once those change.
-PREFILL_TRAFFIC = {"sources_sha256": "7cb7760b82b9a491c8870f3eadc527cf5fe6ee26bab22a2512c73232c2691582", "bytes_per_call": 16878848}
+PREFILL_TRAFFIC = {"sources_sha256": "475680e8ebc388db0be773f273cb4307d186640a9dc5a0486c0853f79df3123a", "bytes_per_call": 16770752}
 
 
 def _kernel_sources_digest():
