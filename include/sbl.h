@@ -382,6 +382,32 @@ sbl_status sbl_linear_rmsnorm(const uint16_t* x_bf16, const float* g, float eps,
                               void* workspace, size_t workspace_bytes, int path, void* stream);
 
 /*
+ * sbl_linear_q — sbl_linear on activations that are already quantised.
+ *
+ * Sparse-BitNet Guide, "Mathematical Formulation of Sparse-BitLinear": the
+ * integer product of the int8 activations with the ternary weights, rescaled
+ * by row_scale[o] / s_tok[t].  Here the activation step (the x̃ equation) is
+ * the caller's: x_q (int8 [T, K], column order, 16-byte aligned) and s_tok
+ * (fp32 [T], 16-byte aligned) exactly as sbl_quant_act writes them.  A
+ * training forward keeps them for the backward; a layer split along K
+ * across GPUs quantises the whole row once and contracts its slice.
+ * packed, row_scale, O, n, m, y, y_dtype and acc_out are as for sbl_linear;
+ * y and acc_out equal sbl_linear's on the x that x_q came from.
+ *   - Needs K % 64 == 0, else SBL_ERR_UNSUPPORTED.  T <= 16 (with K <= 24576)
+ *     runs on the warp-MMA decode kernel, larger sizes on the tensor cores.
+ *   - The workspace is sized by sbl_linear_workspace_bytes().  The dense
+ *     tensor-core GEMMs and the decode kernel read x_q in the weight codes'
+ *     pairing order, written into the workspace by one permutation kernel
+ *     (T * K bytes read and written); the 2:4 sparse GEMM reads x_q in place.
+ *   - x_q and s_tok are read only; the library keeps no reference to them.
+ * Errors as sbl_linear; asynchronous on `stream`.
+ */
+sbl_status sbl_linear_q(const int8_t* x_q, const float* s_tok, int64_t T, int64_t K,
+                        const uint8_t* packed, const float* row_scale, int64_t O, int n, int m,
+                        void* y, int y_dtype, int32_t* acc_out,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * sbl_linear_noalloc — sbl_linear for callers that cannot allocate device memory.
  *
  * The pages have no counterpart for this entry point; it serves callers that

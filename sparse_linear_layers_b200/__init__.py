@@ -13,7 +13,7 @@ GPU library.
 """
 __version__ = "0.1.0"
 
-_API = ("PreparedWeights", "copy_to_device", "copy_to_host", "sbl_decode_max_tokens", "sbl_device_status", "sbl_linear", "sbl_linear_backward", "sbl_linear_backward_workspace_bytes", "sbl_linear_grouped", "sbl_linear_hostio", "sbl_linear_plan",
+_API = ("PreparedWeights", "copy_to_device", "copy_to_host", "sbl_decode_max_tokens", "sbl_device_status", "sbl_linear", "sbl_linear_backward", "sbl_linear_backward_workspace_bytes", "sbl_linear_grouped", "sbl_linear_hostio", "sbl_linear_plan", "sbl_linear_q",
         "sbl_linear_rmsnorm", "sbl_linear_workspace_bytes", "sbl_mask_monitor", "sbl_prepare_weights", "sbl_prepare_weights_grouped", "sbl_quant_act",
         "sbl_rmsnorm_quant_act", "sbl_selftest_bounded_wait", "workspace_for", "RMSNORM_EPS_F32", "SblError")
 

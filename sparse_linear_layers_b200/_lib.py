@@ -51,6 +51,7 @@ SIGNATURES = {
     "sbl_linear_path": (_int, [_vp, _i64, _i64, _vp, _vp, _i64, _int, _int, _vp, _int, _vp, _vp, _sz, _int, _vp]),
     "sbl_linear_rmsnorm": (_int, [_vp, _vp, _f32, _i64, _i64, _vp, _vp, _i64, _int, _int, _vp, _int, _vp, _vp, _sz,
                                   _int, _vp]),
+    "sbl_linear_q": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _i64, _int, _int, _vp, _int, _vp, _vp, _sz, _vp]),
     "sbl_linear_grouped_workspace_bytes": (_sz, [_i64, _i64]),
     "sbl_linear_grouped": (_int, [_vp, _i64, _i64, _int, _vp, _vp, _vp, _int, _int, _vp, _int, _vp, _vp, _sz, _vp]),
     "sbl_linear_noalloc": (_int, [_vp, _i64, _i64, _vp, _vp, _i64, _int, _int, _vp, _int, _vp, _vp]),

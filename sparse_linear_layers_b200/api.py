@@ -201,6 +201,36 @@ def sbl_linear(x: torch.Tensor, w: PreparedWeights, out_dtype: torch.dtype = tor
     return y
 
 
+def sbl_linear_q(x_q: torch.Tensor, s_tok: torch.Tensor, w: PreparedWeights, out_dtype: torch.dtype = torch.float32,
+                 y: Optional[torch.Tensor] = None, acc_out: Optional[torch.Tensor] = None,
+                 workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """sbl_linear on activations quantised already: x_q (int8 [T,K]) and s_tok
+    (fp32 [T]) as sbl_quant_act returns them.  Needs K % 64 == 0."""
+    T, K = _need_2d(x_q, "x_q")
+    _need_cuda(x_q, "x_q", torch.int8)
+    _need_cuda(s_tok, "s_tok", torch.float32, (T,), x_q.device)
+    if K != w.K:
+        raise ValueError(f"x_q has K={K}, weights were prepared with K={w.K}")
+    _need_weights(w, x_q.device)
+    O = w.O
+    if y is None:
+        y = torch.empty((T, O), dtype=out_dtype, device=x_q.device)
+    if y.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("y must be float32 or bfloat16")
+    _need_cuda(y, "y", y.dtype, (T, O), x_q.device)
+    ydt = _lib.SBL_F32 if y.dtype == torch.float32 else _lib.SBL_BF16
+    if acc_out is not None:
+        _need_cuda(acc_out, "acc_out", torch.int32, (T, O), x_q.device)
+    if workspace is None:
+        workspace = workspace_for(T, K, O, w.n, w.m, x_q.device)
+    _need_workspace(workspace, x_q.device)
+    check(lib.sbl_linear_q(x_q.data_ptr(), s_tok.data_ptr(), T, K, w.packed.data_ptr(), w.row_scale.data_ptr(), O,
+                           w.n, w.m, y.data_ptr(), ydt, acc_out.data_ptr() if acc_out is not None else None,
+                           workspace.data_ptr(), workspace.numel(), _stream(stream)),
+          "sbl_linear_q")
+    return y
+
+
 def _need_host_pair(host: torch.Tensor, dev: torch.Tensor, hname: str, dname: str) -> int:
     """Byte count of a host <-> device copy between two contiguous tensors of
     equal size in bytes, the host one in CPU memory, the other on a GPU."""

@@ -18,7 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libsbl.so")
-SOURCES = ("sbl_api.cu", "prep.cu", "quant.cu", "decode.cu", "decode_mma.cu", "prefill.cu", "prefill_pair.cu", "prefill_sp.cu", "mask_monitor.cu", "backward.cu", "backward_tc.cu", "noalloc.cu")
+SOURCES = ("sbl_api.cu", "prep.cu", "quant.cu", "decode.cu", "decode_mma.cu", "prefill.cu", "prefill_pair.cu", "prefill_sp.cu", "mask_monitor.cu", "backward.cu", "backward_tc.cu", "noalloc.cu", "xq_layout.cu")
 ARCH = ("-gencode", "arch=compute_100a,code=sm_100a")
 
 

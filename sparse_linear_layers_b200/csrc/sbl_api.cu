@@ -60,6 +60,8 @@ int prefill_ksplit(long long T, long long K, long long O, int num_sms);
 size_t prefill_split_part_bytes(long long T, long long O, int ksplit);
 int choose_dense_prefill(long long T, long long O, int num_sms, cudaStream_t stream);
 size_t sp_scratch_bytes(long long O, long long K);
+cudaError_t launch_xq_to_pairs(const int8_t* xq, long long T, long long K, int8_t* out, int num_sms,
+                               cudaStream_t stream);
 cudaError_t launch_prefill_sp(const int8_t* xq, const float* s_tok, long long T, long long K, const uint8_t* packed,
                               const float* row_scale, long long O, void* y, int y_bf16, int32_t* acc_out,
                               uint8_t* scratch, unsigned* status, int num_sms, cudaStream_t stream);
@@ -442,6 +444,50 @@ sbl_status sbl_linear_rmsnorm(const uint16_t* x_bf16, const float* g, float eps,
     if (!g) return SBL_ERR_INVALID_ARG;
     return linear_impl(x_bf16, g, eps, T, K, packed, row_scale, O, n, m, y, y_dtype, acc_out, workspace,
                        workspace_bytes, path, stream);
+}
+
+// The contraction on activations the caller quantised already (x_q in column
+// order and s_tok, as sbl_quant_act writes them).  The sparse GEMM reads that
+// order as it is; the dense GEMMs and the warp-MMA decode read the pairing
+// order, which xq_to_pairs_kernel writes into the workspace.
+sbl_status sbl_linear_q(const int8_t* x_q, const float* s_tok, int64_t T, int64_t K, const uint8_t* packed,
+                        const float* row_scale, int64_t O, int n, int m, void* y, int y_dtype, int32_t* acc_out,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+    if (T < 0 || O < 0) return SBL_ERR_INVALID_ARG;
+    if (sbl_status s = check_k(K)) return s;
+    if (!nm_ok(n, m)) return SBL_ERR_UNSUPPORTED;
+    if (y_dtype != SBL_F32 && y_dtype != SBL_BF16) return SBL_ERR_INVALID_ARG;
+    if (K % 64 != 0) return SBL_ERR_UNSUPPORTED;
+    if (T == 0 || O == 0) return SBL_OK;
+    if (!x_q || !s_tok || !packed || !row_scale || !y) return SBL_ERR_INVALID_ARG;
+    if (!aligned(x_q, 16) || !aligned(s_tok, 16) || !aligned(packed, 16) || !aligned(row_scale, 16) ||
+        !aligned(y, 16))
+        return SBL_ERR_INVALID_ARG;
+    if (acc_out && !aligned(acc_out, 16)) return SBL_ERR_INVALID_ARG;
+    if (T > (1ll << 31) - 1 || O > (1ll << 31) - 1) return SBL_ERR_UNSUPPORTED;
+    const bool prefill = T > kDecodeMaxTokens || K > kDecodeMaxK;
+    if (!prefill && !sbl::decode_mma_supported(K)) return SBL_ERR_UNSUPPORTED;
+    const size_t need = base_workspace_bytes(T, K);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return SBL_ERR_WORKSPACE;
+
+    DeviceInfo* d;
+    if (sbl_status s = device_info(&d)) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int ybf = y_dtype == SBL_BF16 ? 1 : 0;
+    const size_t sparse_need = sparse_eligible(K, n, m) ? need + sbl::sp_scratch_bytes(O, K) : 0;
+    if (prefill && sparse_need != 0 && workspace_bytes >= sparse_need && sparse_preferred(T, K, O, d->num_sms))
+        return from_cuda(sbl::launch_prefill_sp(x_q, s_tok, T, K, packed, row_scale, O, y, ybf, acc_out,
+                                                static_cast<uint8_t*>(workspace) + need, d->status, d->num_sms, st));
+    int8_t* xp = static_cast<int8_t*>(workspace);
+    cudaError_t e = sbl::launch_xq_to_pairs(x_q, T, K, xp, d->num_sms, st);
+    if (e != cudaSuccess) return SBL_ERR_CUDA;
+    if (prefill)
+        e = sbl::launch_prefill(xp, s_tok, T, K, packed, row_scale, O, y, ybf, acc_out, d->status, d->num_sms,
+                                sbl::kPrefillAuto, 1, nullptr, st);
+    else
+        e = sbl::launch_decode_mma(packed, row_scale, O, K, nullptr, T, y, ybf, acc_out, d->status, d->num_sms, st, xp,
+                                   s_tok);
+    return from_cuda(e);
 }
 
 sbl_status sbl_copy_to_device(void* device_dst, const void* host_src, size_t bytes, void* stream) {

@@ -8,7 +8,8 @@ Estimator").  Here every step of that runs in the library's kernels:
 
     forward   sbl_prepare_weights (mask, scale, ternarise, pack; every call,
               so the mask follows the latent weights), sbl_quant_act (the
-              int8 activations kept for the backward) and sbl_linear;
+              int8 activations kept for the backward) and sbl_linear_q on
+              those (sbl_linear, which quantises x itself, when K % 64 != 0);
     backward  sbl_linear_backward (dX = dY . (scale * W_t) to the activations,
               dW = dY^T . (x_q / s_t) to every latent weight).
 
@@ -34,7 +35,9 @@ class SparseBitLinearFunction(torch.autograd.Function):
     def forward(ctx, x, weight, n, m, dw_ternary, check_finite=True):
         w = api.sbl_prepare_weights(weight.detach(), n, m)
         xq, s = api.sbl_quant_act(x)
-        y = api.sbl_linear(x, w)
+        # contract the x_q kept for the backward (x is quantised once); the
+        # contraction on quantised activations needs K % 64 == 0
+        y = api.sbl_linear_q(xq, s, w) if weight.shape[1] % 64 == 0 else api.sbl_linear(x, w)
         if check_finite:
             # The kernels do not pass NaN or Inf through: a non-finite latent
             # weight or activation only sets the device status word while the

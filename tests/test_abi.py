@@ -260,3 +260,28 @@ def test_linear_hostio_rejects_on_host():
     # then the host buffers
     assert H(None, 4, 64, p, p, p, 16, 2, 4, p, p, 0, p, 1 << 20, None) == 1
     assert H(p, 4, 64, p, p, p, 16, 2, 4, p, None, 0, p, 1 << 20, None) == 1
+
+
+def test_linear_q_rejects_on_host():
+    from sparse_linear_layers_b200._lib import lib
+    Q = lib.sbl_linear_q
+    p = 4096
+    # empty problems enqueue nothing
+    assert Q(None, None, 0, 64, None, None, 16, 2, 4, None, 0, None, None, 0, None) == 0
+    assert Q(None, None, 4, 64, None, None, 0, 2, 4, None, 0, None, None, 0, None) == 0
+    # K % 64 != 0, an unsupported pattern, a bad output dtype
+    assert Q(p, p, 4, 48, p, p, 16, 2, 4, p, 0, None, p, 1 << 20, None) == 2
+    assert Q(p, p, 4, 64, p, p, 16, 1, 4, p, 0, None, p, 1 << 20, None) == 2
+    assert Q(p, p, 4, 64, p, p, 16, 2, 4, p, 7, None, p, 1 << 20, None) == 1
+    # missing or unaligned activations and scales
+    assert Q(None, p, 4, 64, p, p, 16, 2, 4, p, 0, None, p, 1 << 20, None) == 1
+    assert Q(p, None, 4, 64, p, p, 16, 2, 4, p, 0, None, p, 1 << 20, None) == 1
+    assert Q(p + 8, p, 4, 64, p, p, 16, 2, 4, p, 0, None, p, 1 << 20, None) == 1
+    assert Q(p, p + 4, 4, 64, p, p, 16, 2, 4, p, 0, None, p, 1 << 20, None) == 1
+    assert Q(p, p, 4, 64, p, p, 16, 2, 4, p, 0, p + 4, p, 1 << 20, None) == 1
+    # workspace missing, too small or unaligned
+    assert Q(p, p, 4, 64, p, p, 16, 2, 4, p, 0, None, None, 1 << 20, None) == 6
+    assert Q(p, p, 4, 64, p, p, 16, 2, 4, p, 0, None, p, 16, None) == 6
+    assert Q(p, p, 4, 64, p, p, 16, 2, 4, p, 0, None, p + 16, 1 << 20, None) == 6
+    # negative sizes
+    assert Q(p, p, -1, 64, p, p, 16, 2, 4, p, 0, None, p, 1 << 20, None) == 1
