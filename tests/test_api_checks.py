@@ -133,3 +133,38 @@ def test_prepare_and_quant_checks(rec):
     with pytest.raises(ValueError):
         api.sbl_quant_act(torch.zeros(K, dtype=torch.bfloat16))
     assert rec.calls == []
+
+
+def test_linear_q_checks(rec):
+    w = _w()
+    xq, s = torch.zeros((T, K), dtype=torch.int8), torch.ones(T)
+    api.sbl_linear_q(xq, s, w, y=torch.empty((T, O)), acc_out=torch.empty((T, O), dtype=torch.int32),
+                     workspace=_ws())
+    assert rec.calls == ["sbl_linear_q"]
+    rec.calls.clear()
+    bad_inputs = [(xq.to(torch.uint8), s), (xq, torch.ones(T + 1)), (xq, s.double()), (xq, s.to("meta")),
+                  (xq.to("meta"), s), (torch.zeros((T, K + 64), dtype=torch.int8), s),
+                  (torch.zeros((K, T), dtype=torch.int8).t(), s)]
+    for a, b in bad_inputs:
+        with pytest.raises(ValueError):
+            api.sbl_linear_q(a, b, w, y=torch.empty((T, O)), workspace=_ws())
+    for kw in (dict(y=torch.empty((T, O + 1))), dict(acc_out=torch.empty((T, O), dtype=torch.int64)),
+               dict(workspace=torch.zeros(64, dtype=torch.uint8, device="meta"))):
+        args = dict(y=torch.empty((T, O)), workspace=_ws())
+        args.update(kw)
+        with pytest.raises(ValueError):
+            api.sbl_linear_q(xq, s, w, **args)
+    assert rec.calls == []
+
+
+@pytest.mark.parametrize("k,contraction,other", [(64, "sbl_linear_q", "sbl_linear_path"),
+                                                   (48, "sbl_linear_path", "sbl_linear_q")])
+def test_training_forward_quantises_once(rec, k, contraction, other):
+    """The training layer's forward contracts the x_q it keeps for the backward
+    (sbl_linear_q) when K % 64 == 0, else lets sbl_linear quantise x."""
+    from sparse_linear_layers_b200 import train
+    x = torch.zeros((T, k), dtype=torch.bfloat16)
+    train.SparseBitLinearFunction.apply(x, torch.zeros((O, k)), 2, 4, False, True)
+    assert rec.calls.count("sbl_quant_act") == 1
+    assert contraction in rec.calls and other not in rec.calls
+    assert rec.calls[-1] == "sbl_device_status"
